@@ -1,0 +1,216 @@
+"""Forward and backward of one pre-LayerNorm GPT layer with Megatron tensor
+parallelism, computed shard by shard in float64.  Test infrastructure only.
+
+Layout of the parameters (shard-major, t shards):
+  ln1_g, ln1_b, ln2_g, ln2_b  [h]             replicated
+  w_qkv  [t, 3h/t, h]   b_qkv [t, 3h/t]       column split: shard i owns the
+                                              Q, K, V rows of heads
+                                              i*a/t .. (i+1)*a/t - 1
+  w_o    [t, h, h/t]    b_o   [h]             row split (input columns)
+  w_1    [t, f/t, h]    b_1   [t, f/t]        column split
+  w_2    [t, h, f/t]    b_2   [h]             row split
+Activations are [T, h] with token row r = j*s + p (batch j, position p).
+
+Column split: each shard computes its own output columns from the full
+input; row split: each shard multiplies its slice of the input and the
+partial products are summed ("Megatron-LM 3D parallelism", §1; "Megatron-LM
+overview", §2.2).  Here the sum is an explicit float64 loop over shards.
+"""
+from __future__ import annotations
+
+import math
+import numpy as np
+
+# Plainest readings where the pages are silent:
+#   LayerNorm: affine, biased variance over h, eps passed in (1e-5 by default).
+#   GeLU: the tanh form used by GPT-2 / Megatron's fused bias-GeLU.
+#   Softmax: scores scaled by 1/sqrt(d) before the causal mask; masked
+#            entries are excluded, so their probability is exactly 0.
+GELU_C = math.sqrt(2.0 / math.pi)
+GELU_A = 0.044715
+
+
+def layer_norm_fwd(x: np.ndarray, g: np.ndarray, b: np.ndarray, eps: float):
+    """Row-wise LayerNorm. Returns (y, mu, rstd, xhat)."""
+    mu = x.mean(axis=1)
+    xc = x - mu[:, None]
+    var = (xc * xc).mean(axis=1)
+    rstd = 1.0 / np.sqrt(var + eps)
+    xhat = xc * rstd[:, None]
+    return xhat * g[None, :] + b[None, :], mu, rstd, xhat
+
+
+def layer_norm_bwd(gy: np.ndarray, xhat: np.ndarray, rstd: np.ndarray, g: np.ndarray):
+    """Backward of y = g*xhat + b.  Returns (dx, dg, db)."""
+    dg = (gy * xhat).sum(axis=0)
+    db = gy.sum(axis=0)
+    gh = gy * g[None, :]
+    dx = rstd[:, None] * (gh - gh.mean(axis=1, keepdims=True)
+                          - xhat * (gh * xhat).mean(axis=1, keepdims=True))
+    return dx, dg, db
+
+
+def gelu(z: np.ndarray) -> np.ndarray:
+    u = GELU_C * (z + GELU_A * z ** 3)
+    return 0.5 * z * (1.0 + np.tanh(u))
+
+
+def gelu_prime(z: np.ndarray) -> np.ndarray:
+    u = GELU_C * (z + GELU_A * z ** 3)
+    th = np.tanh(u)
+    return 0.5 * (1.0 + th) + 0.5 * z * (1.0 - th * th) * GELU_C * (1.0 + 3.0 * GELU_A * z * z)
+
+
+def causal_softmax(z: np.ndarray) -> np.ndarray:
+    """Row softmax over q <= p of an [s, s] score block (already scaled);
+    entries with q > p get probability exactly 0."""
+    s = z.shape[0]
+    p = np.zeros_like(z)
+    for r in range(s):
+        row = z[r, : r + 1]
+        e = np.exp(row - row.max())
+        p[r, : r + 1] = e / e.sum()
+    return p
+
+
+def attention_head_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray):
+    """One (batch, head) block of causal self-attention: returns (P, O)."""
+    d = q.shape[1]
+    z = (q @ k.T) / math.sqrt(d)
+    p = causal_softmax(z)
+    return p, p @ v
+
+
+def _check(dims, params):
+    b, s, h, a, f, t = (dims[k] for k in "bshaft")
+    assert h % a == 0 and a % t == 0 and f % t == 0
+    assert params["w_qkv"].shape == (t, 3 * h // t, h)
+    assert params["w_o"].shape == (t, h, h // t)
+    assert params["w_1"].shape == (t, f // t, h)
+    assert params["w_2"].shape == (t, h, f // t)
+    return b, s, h, a, f, t
+
+
+def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5):
+    """Forward pass.  x: [T, h] float64.  Returns (out, cache)."""
+    b, s, h, a, f, t = _check(dims, params)
+    d = h // a
+    hs, a_s = h // t, a // t            # hidden columns and heads per shard
+    T = b * s
+    assert x.shape == (T, h)
+
+    # 1. LN1
+    l1, mu1, rstd1, xhat1 = layer_norm_fwd(x, params["ln1_g"], params["ln1_b"], eps)
+
+    # 2. QKV column-split GEMM: C_i = L1 W_qkv,i^T + b_qkv,i  -> [Q_i | K_i | V_i]
+    c = np.stack([l1 @ params["w_qkv"][i].T + params["b_qkv"][i][None, :] for i in range(t)])
+
+    # 3. causal attention, head by head; head eta of shard i is global head i*a/t+eta
+    probs = np.zeros((t, b, a_s, s, s))
+    o = np.zeros((t, T, hs))
+    for i in range(t):
+        for j in range(b):
+            rows = slice(j * s, (j + 1) * s)
+            for eta in range(a_s):
+                cols = slice(eta * d, (eta + 1) * d)
+                qh = c[i, rows, 0 * hs:1 * hs][:, cols]
+                kh = c[i, rows, 1 * hs:2 * hs][:, cols]
+                vh = c[i, rows, 2 * hs:3 * hs][:, cols]
+                pr, oh = attention_head_fwd(qh, kh, vh)
+                probs[i, j, eta] = pr
+                o[i, rows, cols] = oh
+
+    # 4. out-projection, row split: partial products summed over shards, bias
+    #    added once after the sum, then the residual
+    y_attn = np.zeros((T, h))
+    for i in range(t):
+        y_attn += o[i] @ params["w_o"][i].T
+    hid = x + y_attn + params["b_o"][None, :]
+
+    # 5. LN2
+    l2, mu2, rstd2, xhat2 = layer_norm_fwd(hid, params["ln2_g"], params["ln2_b"], eps)
+
+    # 6. FFN1 column split with fused bias + GeLU
+    z = np.stack([l2 @ params["w_1"][i].T + params["b_1"][i][None, :] for i in range(t)])
+    act = gelu(z)
+
+    # 7. FFN2 row split: shard sum, bias, residual
+    y_mlp = np.zeros((T, h))
+    for i in range(t):
+        y_mlp += act[i] @ params["w_2"][i].T
+    out = hid + y_mlp + params["b_2"][None, :]
+
+    cache = dict(x=x, l1=l1, mu1=mu1, rstd1=rstd1, xhat1=xhat1, c=c, probs=probs, o=o,
+                 hid=hid, l2=l2, mu2=mu2, rstd2=rstd2, xhat2=xhat2, z=z, act=act)
+    return out, cache
+
+
+def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
+    """Backward pass given dOut (already multiplied by the loss scale).
+    Returns (dx, grads) with grads in the same shard-major layout as params."""
+    b, s, h, a, f, t = _check(dims, params)
+    d = h // a
+    hs, a_s = h // t, a // t
+    T = b * s
+    inv_sqrt_d = 1.0 / math.sqrt(d)
+    gr = {}
+
+    # FFN2 (row split): each shard's weight gradient and input gradient
+    gr["b_2"] = dout.sum(axis=0)
+    gr["w_2"] = np.stack([dout.T @ cache["act"][i] for i in range(t)])
+    d_act = np.stack([dout @ params["w_2"][i] for i in range(t)])
+
+    # GeLU backward and FFN1 (column split); the input gradient is the sum
+    # of the shards' partial products
+    dz = d_act * gelu_prime(cache["z"])
+    gr["b_1"] = dz.sum(axis=1)
+    gr["w_1"] = np.stack([dz[i].T @ cache["l2"] for i in range(t)])
+    dl2 = np.zeros((T, h))
+    for i in range(t):
+        dl2 += dz[i] @ params["w_1"][i]
+
+    # LN2 backward plus the residual path
+    dln, gr["ln2_g"], gr["ln2_b"] = layer_norm_bwd(dl2, cache["xhat2"], cache["rstd2"],
+                                                   params["ln2_g"])
+    dhid = dout + dln
+
+    # out-projection (row split)
+    gr["b_o"] = dhid.sum(axis=0)
+    gr["w_o"] = np.stack([dhid.T @ cache["o"][i] for i in range(t)])
+    do = np.stack([dhid @ params["w_o"][i] for i in range(t)])
+
+    # attention backward, head by head
+    c = cache["c"]
+    dc = np.zeros_like(c)
+    for i in range(t):
+        for j in range(b):
+            rows = slice(j * s, (j + 1) * s)
+            for eta in range(a_s):
+                cols = slice(eta * d, (eta + 1) * d)
+                qh = c[i, rows, 0 * hs:1 * hs][:, cols]
+                kh = c[i, rows, 1 * hs:2 * hs][:, cols]
+                vh = c[i, rows, 2 * hs:3 * hs][:, cols]
+                pr = cache["probs"][i, j, eta]
+                doh = do[i, rows, cols]
+                dp = doh @ vh.T
+                dv = pr.T @ doh
+                dzs = pr * (dp - (pr * dp).sum(axis=1, keepdims=True))
+                dsc = dzs * inv_sqrt_d
+                dq = dsc @ kh
+                dk = dsc.T @ qh
+                dc[i, rows, 0 * hs:1 * hs][:, cols] = dq
+                dc[i, rows, 1 * hs:2 * hs][:, cols] = dk
+                dc[i, rows, 2 * hs:3 * hs][:, cols] = dv
+
+    # QKV (column split): per-shard weight and bias grads, shard-summed dL1
+    gr["b_qkv"] = dc.sum(axis=1)
+    gr["w_qkv"] = np.stack([dc[i].T @ cache["l1"] for i in range(t)])
+    dl1 = np.zeros((T, h))
+    for i in range(t):
+        dl1 += dc[i] @ params["w_qkv"][i]
+
+    # LN1 backward plus the residual path
+    dln1, gr["ln1_g"], gr["ln1_b"] = layer_norm_bwd(dl1, cache["xhat1"], cache["rstd1"],
+                                                    params["ln1_g"])
+    dx = dhid + dln1
+    return dx, gr
