@@ -1,0 +1,181 @@
+/*
+ * gptlayer.h — C ABI of the B200 (sm_100a) library for one GPT transformer
+ * layer's training step with Megatron-style tensor parallelism on one GPU.
+ *
+ * What the step computes (sources are the Megatron-LM pages):
+ *   - the GPT layer (pre-LayerNorm; QKV column split; causal attention with
+ *     fused scale-mask-softmax; row-split output projection; column-split
+ *     h->4h GEMM with fused bias+GeLU; row-split 4h->h GEMM):
+ *     "Training GPT-2 with Megatron-LM" §4.1 (layer shapes) and §6.2
+ *     (fused_softmax, fused_bias_gelu); "Megatron-LM 3D parallelism" §1
+ *     (column split owns output columns, row split sums partial products);
+ *     "Megatron-LM overview" §2.2 (FFN column split, QKV split by device);
+ *   - mixed precision with FP32 master weights and dynamic loss scaling:
+ *     "Megatron-LM overview" §3.1; Adam with lr 6e-5: same page, §4.2.
+ *
+ * The tp_size shards all live on the calling GPU.  The partial sums that a
+ * multi-GPU run would all-reduce after each row-split GEMM (forward) and each
+ * column-split input-gradient GEMM (backward) are summed inside the GEMM's
+ * K loop here, so no collective exists on this path.
+ *
+ * Conventions shared by every entry point:
+ *   - All device pointers are caller-owned CUDA device memory; the library
+ *     allocates no device memory.  Every pointer must be 16-byte aligned.
+ *   - All work is enqueued asynchronously on `stream`; no call synchronises
+ *     the host with the device, except gptl_read_device_error().
+ *   - Return value: 0 on success, a negative GPTL_E_* code otherwise.  Input
+ *     validation happens before any launch: on error nothing is enqueued.
+ *   - Kernels never trap.  A device-side failure (a bounded wait that timed
+ *     out, an internal consistency check) sets a library-wide device error
+ *     word, read with gptl_read_device_error().
+ *   - Activations are row-major [T, h] with token row r = j*seq + p (batch j,
+ *     position p), T = batch*seq.  Weights are [out][in] row-major, stored
+ *     shard-major (layouts below).
+ */
+#ifndef GPTLAYER_H
+#define GPTLAYER_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *gptl_stream_t;   /* same type as cudaStream_t */
+
+enum {
+  GPTL_OK = 0,
+  GPTL_E_NULL = -1,    /* a required pointer is NULL                         */
+  GPTL_E_SHAPE = -2,   /* unsupported or inconsistent sizes                  */
+  GPTL_E_ALIGN = -3,   /* a pointer is not 16-byte aligned                   */
+  GPTL_E_DTYPE = -4,   /* dtype is neither GPTL_FP16 nor GPTL_BF16           */
+  GPTL_E_ARCH = -5,    /* the current device is not compute capability 10.x  */
+  GPTL_E_CUDA = -6,    /* a CUDA runtime/driver call or a launch failed      */
+  GPTL_E_DEVICE = -7,  /* the device error word is set (see below)           */
+  GPTL_E_ARG = -8      /* an invalid scalar argument (hyper-parameter)       */
+};
+
+typedef enum { GPTL_FP16 = 0, GPTL_BF16 = 1 } gptl_dtype;
+
+/* Sizes of one layer.  Requirements (GPTL_E_SHAPE otherwise): every field
+ * > 0; heads | hidden; tp | heads; tp | ffn; head_dim = hidden/heads is a
+ * multiple of 16 and at most 256; hidden % 64 == 0; (ffn/tp) % 64 == 0;
+ * seq % 16 == 0; batch*seq < 2^31.  ln_eps > 0 (the pages do not state it;
+ * 1e-5 is the usual GPT-2 value). */
+typedef struct {
+  int batch, seq, hidden, heads, ffn, tp;
+  gptl_dtype dtype;
+  float ln_eps;
+} gptl_shape;
+
+/* Layer parameters in the compute dtype (fp16 or bf16), read-only here.
+ * Column-split tensors: shard i owns output rows; row-split tensors: shard
+ * i owns input columns ("Megatron-LM 3D parallelism" §1).
+ *   ln1_g, ln1_b, ln2_g, ln2_b : [h]
+ *   w_qkv : [t][3h/t][h]  rows of shard i = [Q_i; K_i; V_i], Q_i the rows of
+ *           heads i*a/t .. (i+1)*a/t-1, head-major, head_dim rows each
+ *   b_qkv : [t][3h/t]
+ *   w_o   : [t][h][h/t]   b_o : [h]   (added once, after the shard sum)
+ *   w_1   : [t][f/t][h]   b_1 : [t][f/t]
+ *   w_2   : [t][h][f/t]   b_2 : [h]   (added once, after the shard sum)   */
+typedef struct {
+  const void *ln1_g, *ln1_b;
+  const void *w_qkv, *b_qkv;
+  const void *w_o, *b_o;
+  const void *ln2_g, *ln2_b;
+  const void *w_1, *b_1;
+  const void *w_2, *b_2;
+} gptl_weights;
+
+/* FP32 gradients, same layouts as gptl_weights, multiplied by the loss scale
+ * (they are the gradients of the scaled loss).  gpt_layer_bwd OVERWRITES
+ * them.  Normally these point into the flat gradient arena that
+ * adam_step_fp32_master consumes (see gpt_layer_param_layout). */
+typedef struct {
+  float *ln1_g, *ln1_b, *w_qkv, *b_qkv, *w_o, *b_o,
+        *ln2_g, *ln2_b, *w_1, *b_1, *w_2, *b_2;
+} gptl_grads;
+
+/* Dynamic loss-scale state, in DEVICE memory, caller-initialised to
+ * {scale = initial scale (65536), growth_tracker = 0, found_inf = 0,
+ *  step = 0, error = 0}. */
+typedef struct {
+  float scale;          /* current loss scale S                              */
+  int growth_tracker;   /* clean steps since the last scale change           */
+  int found_inf;        /* written by adam_step_fp32_master                  */
+  int step;             /* Adam steps taken (skipped steps not counted)      */
+  int error;            /* reserved; 0                                       */
+} gptl_scaler_state;
+
+/* Bytes of device workspace the caller provides.
+ *  saved   : activations written by gpt_layer_fwd and read by gpt_layer_bwd;
+ *            must stay untouched between the two calls.
+ *  scratch : temporaries of gpt_layer_bwd (gpt_layer_fwd uses none); may be
+ *            reused freely between calls on the same stream.
+ * Returns GPTL_E_NULL / GPTL_E_SHAPE / GPTL_E_DTYPE on bad arguments. */
+int gpt_layer_workspace_bytes(const gptl_shape *shape, size_t *saved_bytes,
+                              size_t *scratch_bytes);
+
+/* Offsets (in elements) of the 12 parameter tensors inside one flat arena, in
+ * the order ln1_g, ln1_b, w_qkv, b_qkv, w_o, b_o, ln2_g, ln2_b, w_1, b_1, w_2,
+ * b_2, each 64-element aligned, and the arena length n_params (a multiple of
+ * 64).  The same offsets index the fp32 master / m / v / grad arenas and the
+ * 16-bit weight arena.  Padding elements must be zero in the grad arena (the
+ * overflow check scans the whole arena). */
+int gpt_layer_param_layout(const gptl_shape *shape, size_t offsets[12], size_t *n_params);
+
+/* Forward pass.  x: [T,h] input; y: [T,h] output (cdt).  saved: workspace of
+ * saved_bytes; scratch: may be NULL.  x, y and saved must not overlap. */
+int gpt_layer_fwd(const gptl_shape *shape, const gptl_weights *w, const void *x, void *y,
+                  void *saved, void *scratch, gptl_stream_t stream);
+
+/* Backward pass.  dy: [T,h] gradient of the scaled loss w.r.t. y (cdt);
+ * dx: [T,h] output (cdt); g: fp32 gradients, overwritten; saved: as written
+ * by the matching gpt_layer_fwd; scratch: scratch_bytes of workspace. */
+int gpt_layer_bwd(const gptl_shape *shape, const gptl_weights *w, const void *x,
+                  const void *saved, const void *dy, void *dx, const gptl_grads *g,
+                  void *scratch, gptl_stream_t stream);
+
+/* Overflow check + fused unscale/Adam/cast over flat arenas of n_params
+ * elements ("Megatron-LM overview" §3.1 and §4.2).
+ *   1. st->found_inf <- 1 if any grad element is inf or NaN, else 0;
+ *   2. if !found_inf, per element with t = st->step + 1 and S = st->scale:
+ *        g = grad/S; m = b1*m + (1-b1)*g; v = b2*v + (1-b2)*g*g;
+ *        p -= lr*( (m/(1-b1^t)) / (sqrt(v/(1-b2^t)) + eps) + wd*p );
+ *        w16 = round-to-nearest-even(p) in dtype;
+ *      if found_inf, master, m, v and w16 are left bit-unchanged.
+ * master/m/v: [n] fp32 in/out; grad: [n] fp32 in; w16: [n] fp16/bf16 out.
+ * Decisions are made on the device; st is read and written there.
+ * GPTL_E_ARG if lr < 0, beta not in [0,1), eps < 0 or n_params % 4 != 0. */
+int adam_step_fp32_master(size_t n_params, float *master, float *m, float *v,
+                          const float *grad, void *w16, gptl_dtype dtype, float lr,
+                          float beta1, float beta2, float eps, float weight_decay,
+                          gptl_scaler_state *st, gptl_stream_t stream);
+
+/* Dynamic loss-scale update (one device thread), after adam_step_fp32_master:
+ *   found_inf: scale = max(scale*backoff_factor, min_scale); tracker = 0;
+ *   else: tracker += 1; if tracker == growth_interval: scale *= growth_factor,
+ *         tracker = 0; step += 1.
+ * GPTL_E_ARG if growth_interval < 1, growth_factor < 1, backoff_factor not in
+ * (0,1] or min_scale <= 0. */
+int loss_scale_update(gptl_scaler_state *st, int growth_interval, float growth_factor,
+                      float backoff_factor, float min_scale, gptl_stream_t stream);
+
+/* Standalone overflow check (step 1 of adam_step_fp32_master). */
+int gptl_check_overflow(size_t n, const float *grad, gptl_scaler_state *st,
+                        gptl_stream_t stream);
+
+/* Human-readable text of a GPTL_E_* code (static storage). */
+const char *gptl_strerror(int code);
+
+/* Synchronises the current device, then reads (and with clear != 0 resets)
+ * the library's device error word: 0 = no device-side error; otherwise a
+ * bit mask (1 = a pipeline wait timed out in a GEMM, 2 = an internal index
+ * check failed).  Test helper; returns GPTL_E_CUDA if the copy fails. */
+int gptl_read_device_error(int *word, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPTLAYER_H */

@@ -1,0 +1,112 @@
+/*
+ * gptlayer_parts.h — the building blocks of the layer step, exported one by
+ * one so that each kernel can be checked on its own.  Same conventions as
+ * gptlayer.h: caller-owned 16-byte-aligned device pointers, asynchronous on
+ * `stream`, 0 or a negative GPTL_E_* code, validation before any launch.
+ */
+#ifndef GPTLAYER_PARTS_H
+#define GPTLAYER_PARTS_H
+
+#include "gptlayer.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* One operand of gptl_gemm, seen through a 3-D view of a 16-bit tensor:
+ * element (x, row, g) lives at ptr + g*g_pitch + row*row_pitch + x
+ * (pitches in elements, multiples of 8).
+ *   mn_major = 0: `row` indexes M (operand A) or N (operand B) and `x` the
+ *                 reduction index k  ("K-major");
+ *   mn_major = 1: `row` is k and `x` is the M/N index ("MN-major": the
+ *                 tensor core reads it transposed, no copy is made).
+ * For group G and k-shard ks the operand's x offset is
+ *   (G % x_mod) * x_mul + x_off   and its g coordinate is
+ *   G / g_div + (k_shard ? ks : 0).
+ * Reads outside the view's extents return zeros. */
+typedef struct {
+  const void *ptr;
+  long long x_ext, rows_ext, g_ext;
+  long long row_pitch, g_pitch;
+  int mn_major;
+  int x_mod, x_mul, x_off;
+  int g_div;
+  int k_shard;
+} gptl_operand;
+
+enum { GPTL_ACT_NONE = 0, GPTL_ACT_GELU = 1, GPTL_ACT_DGELU = 2 };
+enum {
+  GPTL_CAUSAL_NONE = 0,
+  GPTL_CAUSAL_SKIP_UPPER = 1, /* skip 128 x BN tiles with n0 > m0 + 127    */
+  GPTL_CAUSAL_K_BELOW = 2,    /* reduce only over k < m0 + 128             */
+  GPTL_CAUSAL_K_FROM = 3      /* reduce only over k >= m0                  */
+};
+
+/* out[G](m, n) = epilogue( sum over ks < k_shards, k < K of A(m,k) * B(n,k) )
+ * for m < M, n < N, G < groups, with fp32 accumulation in tensor memory.
+ * Output element (m, n) of group G is at
+ *   out + (G % o_mod)*o_str_mod + (G / o_mod)*o_str_div + m*ldo + n.
+ * Epilogue, in order: + bias[G*bias_g_stride + n] (if bias), + resid[m*ld_resid
+ * + n] (if resid), then act: GELU writes the value to out and GeLU(value) to
+ * out2; DGELU multiplies by GeLU'(aux at the output's index).  out_f32 = 1
+ * stores the raw fp32 sum (no bias/resid/act).  Requirements: K % 16 == 0,
+ * N % 16 == 0, all offsets/pitches multiples of 8 elements. */
+typedef struct {
+  int M, N, K, groups, k_shards, causal;
+  gptl_operand a, b;
+  void *out;
+  int out_f32;
+  long long ldo;
+  int o_mod;
+  long long o_str_mod, o_str_div;
+  const void *bias;
+  long long bias_g_stride;
+  const void *resid;
+  long long ld_resid;
+  const void *aux;
+  void *out2;
+  int act;
+} gptl_gemm_desc;
+
+int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream);
+
+/* LayerNorm forward over `rows` rows of width h: y = g*(x-mu)*rstd + b with the
+ * biased variance; mu and rstd ([rows] fp32) are saved for the backward.
+ * h must split as h/8 = TPR*VPT with TPR a power of two in [16, 256], VPT <= 8. */
+int gptl_layernorm_fwd(int rows, int h, gptl_dtype dtype, const void *x, const void *g,
+                       const void *b, float eps, void *y, float *mu, float *rstd,
+                       gptl_stream_t stream);
+
+/* Scratch bytes gptl_layernorm_bwd needs. */
+size_t gptl_layernorm_bwd_scratch_bytes(int rows, int h);
+
+/* LayerNorm backward: dx = resid + LNbwd(gy); dg = sum_rows gy*xhat,
+ * db = sum_rows gy (fp32, overwritten); dx_sum (optional, may be NULL) =
+ * sum_rows dx.  resid may alias nothing that is written. */
+int gptl_layernorm_bwd(int rows, int h, gptl_dtype dtype, const void *gy, const void *x,
+                       const float *mu, const float *rstd, const void *g, const void *resid,
+                       void *dx, float *dg, float *db, float *dx_sum, void *scratch,
+                       gptl_stream_t stream);
+
+/* Causal softmax in place on `blocks` score blocks [s][s]: row p becomes
+ * softmax over q <= p of scale*S; entries p < q < min(s, 128*(p/128+1)) are
+ * set to 0; the rest of the row is not touched.  s % 16 == 0, s <= 2048. */
+int gptl_softmax_fwd(long long blocks, int s, gptl_dtype dtype, float scale, void *scores,
+                     gptl_stream_t stream);
+
+/* Softmax backward in place: dP -> scale * P * (dP - rowsum(P*dP)) on q <= p,
+ * 0 for p < q < min(s, 128*(p/128+1)). */
+int gptl_softmax_bwd(long long blocks, int s, gptl_dtype dtype, float scale, const void *prob,
+                     void *dprob, gptl_stream_t stream);
+
+/* Scratch bytes gptl_colsum needs. */
+size_t gptl_colsum_scratch_bytes(int n, int groups);
+
+/* out[G*n + c] = sum over r < rows of a[G*gstride + r*ld + c] (fp32). */
+int gptl_colsum(int rows, int n, int groups, long long ld, long long gstride, gptl_dtype dtype,
+                const void *a, float *out, void *scratch, gptl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPTLAYER_PARTS_H */

@@ -1,0 +1,74 @@
+"""The C-ABI library loads without a GPU, exports every function that
+include/*.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+
+import pytest
+
+from transformer_layer_step_b200 import gptlayer as G
+from transformer_layer_step_b200 import synth
+
+
+def test_exports_every_declared_function():
+    lib = G.lib()
+    declared = G.header_functions()
+    assert "gpt_layer_fwd" in declared and "adam_step_fp32_master" in declared
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_strerror_codes():
+    for code in (0, G.E_NULL, G.E_SHAPE, G.E_ALIGN, G.E_DTYPE, G.E_ARCH, G.E_CUDA, G.E_DEVICE, G.E_ARG):
+        assert G.strerror(code) and G.strerror(code) != "unknown error"
+
+
+@pytest.mark.parametrize("name", list(synth.CONFIGS))
+def test_workspace_and_layout(name):
+    c = synth.CONFIGS[name]
+    sh = G.make_shape(c.batch, c.seq, c.hidden, c.heads, c.ffn, c.tp, c.dtype)
+    saved, scratch = G.workspace_bytes(sh)
+    T, h, f = c.tokens, c.hidden, c.ffn
+    assert saved >= 2 * (T * h * 6 + 2 * T * f + c.batch * c.heads * c.seq * c.seq)
+    assert scratch >= 2 * (T * f + 7 * T * h + c.batch * c.heads * c.seq * c.seq)
+    offs, n = G.param_layout(sh)
+    sizes = [h, h, 3 * h * h, 3 * h, h * h, h, h, h, f * h, f, h * f, h]
+    assert n % 64 == 0 and all(o % 64 == 0 for o in offs)
+    for i in range(11):
+        assert offs[i] + sizes[i] <= offs[i + 1]
+    assert offs[11] + sizes[11] <= n
+    assert n - sum(sizes) < 64 * 12
+    assert sum(sizes) == 12 * h * h + 13 * h
+
+
+@pytest.mark.parametrize("bad", [
+    dict(heads=5),                 # heads does not divide hidden
+    dict(tp=3),                    # tp does not divide heads
+    dict(hidden=96, heads=2),      # hidden not a multiple of 64
+    dict(seq=72),                  # seq not a multiple of 16
+    dict(heads=16),                # head_dim 8, not a multiple of 16
+    dict(batch=0),
+    dict(seq=4096),                # beyond the supported sequence length
+])
+def test_shape_validation(bad):
+    args = dict(batch=2, seq=64, hidden=128, heads=4, ffn=512, tp=2, dtype="fp16")
+    args.update(bad)
+    sh = G.make_shape(**args)
+    with pytest.raises(G.GptlError) as e:
+        G.workspace_bytes(sh)
+    assert e.value.code == G.E_SHAPE
+
+
+def test_dtype_and_null_rejected_without_launch():
+    sh = G.make_shape(2, 64, 128, 4, 512, 2, 7)
+    with pytest.raises(G.GptlError) as e:
+        G.workspace_bytes(sh)
+    assert e.value.code == G.E_DTYPE
+    sh = G.make_shape(2, 64, 128, 4, 512, 2, "fp16")
+    w = G.Weights()
+    rc = G.lib().gpt_layer_fwd(ctypes.byref(sh), ctypes.byref(w), 16, 16, 16, None, None)
+    assert rc == G.E_NULL
+    rc = G.lib().adam_step_fp32_master(64, 16, 16, 16, 16, 16, 0, -1.0, 0.9, 0.95, 1e-8, 0.0, 16, None)
+    assert rc == G.E_ARG
+    rc = G.lib().adam_step_fp32_master(64, 17, 16, 16, 16, 16, 0, 1e-3, 0.9, 0.95, 1e-8, 0.0, 16, None)
+    assert rc == G.E_ALIGN
+    rc = G.lib().loss_scale_update(16, 0, 2.0, 0.5, 1.0, None)
+    assert rc == G.E_ARG

@@ -1,0 +1,240 @@
+"""GPU parity of the tcgen05 GEMM (gptl_gemm) in every operand arrangement
+the layer step uses, against the float64 contraction of the same 16-bit
+inputs.  The expected value applies the descriptor's documented view rules
+(include/gptlayer_parts.h) with numpy; shapes span several tiles and ragged
+M/N/K tails."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from transformer_layer_step_b200 import gptlayer as G
+from gpu_util import need_gpu, dev_tensor, host_values, rounded, stream, check_device_error
+
+pytestmark = pytest.mark.gpu
+
+
+def _operand_matrix(buf, op, G_idx, ks, rows_needed, k_len):
+    """[rows_needed, k_len] float64 matrix the operand contributes for group
+    G_idx and k-shard ks; zeros outside the view."""
+    x0 = (G_idx % op["x_mod"]) * op["x_mul"] + op["x_off"]
+    gdiv = op["g_div"]
+    gc = G_idx // gdiv + (ks if op["k_shard"] else 0)
+    out = np.zeros((rows_needed, k_len))
+    xe, re_, ge = op["x_ext"], op["rows_ext"], op["g_ext"]
+    if gc >= ge:
+        return out
+    plane = buf[gc]                                # [rows_ext, x_ext]
+    for r in range(rows_needed):
+        for_k = np.arange(k_len)
+        if not op["mn_major"]:
+            row, xs = r, x0 + for_k
+            if row < re_:
+                ok = xs < xe
+                out[r, ok] = plane[row, xs[ok]]
+        else:
+            xs, rows = x0 + r, for_k
+            if xs < xe:
+                ok = rows < re_
+                out[r, ok] = plane[rows[ok], xs]
+    return out
+
+
+def _expected(desc, abuf, bbuf):
+    M, N, K = desc["M"], desc["N"], desc["K"]
+    res = []
+    for g in range(desc["groups"]):
+        acc = np.zeros((M, N))
+        for ks in range(desc["k_shards"]):
+            A = _operand_matrix(abuf, desc["a"], g, ks, M, K)
+            B = _operand_matrix(bbuf, desc["b"], g, ks, N, K)
+            if desc["causal"] == G.CAUSAL_K_BELOW:
+                m0 = (np.arange(M) // 128) * 128
+                A = A * (np.arange(K)[None, :] < (m0[:, None] + 128))
+            if desc["causal"] == G.CAUSAL_K_FROM:
+                m0 = (np.arange(M) // 128) * 128
+                A = A * (np.arange(K)[None, :] >= m0[:, None])
+            acc += A @ B.T
+        res.append(acc)
+    return np.stack(res)
+
+
+def _op(buf_t, x_ext, rows_ext, g_ext, row_pitch, g_pitch, mn, x_mod=1, x_mul=0, x_off=0,
+        g_div=None, k_shard=0):
+    if g_div is None:
+        g_div = 1 if g_ext > 1 else (1 << 30)
+    d = dict(x_ext=x_ext, rows_ext=rows_ext, g_ext=g_ext, mn_major=mn, x_mod=x_mod, x_mul=x_mul,
+             x_off=x_off, g_div=g_div, k_shard=k_shard)
+    c = G.operand(buf_t, x_ext, rows_ext, g_ext, row_pitch, g_pitch, mn, x_mod, x_mul, x_off,
+                  g_div, k_shard)
+    return d, c
+
+
+def _run(dtype, M, N, K, groups, k_shards, causal, a_spec, b_spec, out_f32=False, bias=False,
+         resid=False, act=G.ACT_NONE, seed=0, std_a=1.0, std_b=0.1):
+    """a_spec/b_spec: (shape of the 3-D buffer [g, rows, x], view kwargs)."""
+    need_gpu()
+    rng = np.random.default_rng(seed)
+    abuf = rounded(rng.standard_normal(a_spec[0]) * std_a, dtype)
+    bbuf = rounded(rng.standard_normal(b_spec[0]) * std_b, dtype)
+    at, bt = dev_tensor(abuf, dtype), dev_tensor(bbuf, dtype)
+    ad, ac = _op(at, a_spec[0][2], a_spec[0][1], a_spec[0][0], a_spec[0][2],
+                 a_spec[0][1] * a_spec[0][2], **a_spec[1])
+    bd, bc = _op(bt, b_spec[0][2], b_spec[0][1], b_spec[0][0], b_spec[0][2],
+                 b_spec[0][1] * b_spec[0][2], **b_spec[1])
+    desc_py = dict(M=M, N=N, K=K, groups=groups, k_shards=k_shards, causal=causal, a=ad, b=bd)
+    exp = _expected(desc_py, abuf, bbuf)
+    if out_f32:
+        out = torch.full((groups, M, N), float("nan"), dtype=torch.float32, device="cuda")
+    else:
+        out = torch.zeros((groups, M, N), dtype=torch.float16 if dtype == "fp16" else torch.bfloat16,
+                          device="cuda")
+    d = G.GemmDesc()
+    d.M, d.N, d.K, d.groups, d.k_shards, d.causal = M, N, K, groups, k_shards, causal
+    d.a, d.b = ac, bc
+    d.out, d.out_f32, d.ldo, d.o_mod, d.o_str_mod, d.o_str_div = out.data_ptr(), int(out_f32), N, 1, 0, M * N
+    bias_v = resid_v = aux_v = None
+    keep = []
+    if bias:
+        bias_v = rounded(rng.standard_normal((groups, N)) * 0.5, dtype)
+        bt_ = dev_tensor(bias_v, dtype)
+        keep.append(bt_)
+        d.bias, d.bias_g_stride = bt_.data_ptr(), N
+    if resid:
+        resid_v = rounded(rng.standard_normal((M, N)), dtype)
+        rt_ = dev_tensor(resid_v, dtype)
+        keep.append(rt_)
+        d.resid, d.ld_resid = rt_.data_ptr(), N
+    out2 = None
+    if act == G.ACT_GELU:
+        out2 = torch.zeros_like(out)
+        d.out2 = out2.data_ptr()
+    if act == G.ACT_DGELU:
+        aux_v = rounded(rng.standard_normal((groups, M, N)), dtype)
+        xt_ = dev_tensor(aux_v, dtype)
+        keep.append(xt_)
+        d.aux = xt_.data_ptr()
+    d.act = act
+    G.gemm(d, dtype, stream())
+    check_device_error()
+    if out_f32:
+        return exp, out.cpu().numpy(), None
+    if bias:
+        exp = exp + bias_v[:, None, :]
+    if resid:
+        exp = exp + resid_v[None]
+    got = host_values(out, dtype)
+    got2 = None
+    if act == G.ACT_GELU:
+        z = rounded(exp, dtype)
+        u = math.sqrt(2 / math.pi) * (z + 0.044715 * z ** 3)
+        exp2 = 0.5 * z * (1 + np.tanh(u))
+        got2 = (host_values(out2, dtype), exp2)
+    if act == G.ACT_DGELU:
+        z = aux_v
+        u = math.sqrt(2 / math.pi) * (z + 0.044715 * z ** 3)
+        th = np.tanh(u)
+        gp = 0.5 * (1 + th) + 0.5 * z * (1 - th * th) * math.sqrt(2 / math.pi) * (1 + 3 * 0.044715 * z * z)
+        exp = exp * gp
+    return exp, got, got2
+
+
+def _close(got, exp, tol, mask=None):
+    if mask is not None:
+        got, exp = got[mask], exp[mask]
+    scale = max(float(np.abs(exp).max()), 1e-6)
+    err = float(np.abs(got - exp).max()) / scale
+    assert err <= tol, err
+
+
+DT = ["bf16", "fp16"]
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_fprop_kmajor_bias_grouped(dtype):
+    # column-split style: A shared, B and out grouped; ragged M and K tail
+    exp, got, _ = _run(dtype, M=300, N=192, K=160, groups=2, k_shards=1, causal=0,
+                       a_spec=((1, 300, 160), dict(mn=0)), b_spec=((2, 192, 160), dict(mn=0)),
+                       bias=True)
+    _close(got, exp, 8e-3)
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_fprop_wide_n_resid(dtype):
+    exp, got, _ = _run(dtype, M=256, N=640, K=128, groups=1, k_shards=1, causal=0,
+                       a_spec=((1, 256, 128), dict(mn=0)), b_spec=((1, 640, 128), dict(mn=0)),
+                       bias=True, resid=True)
+    _close(got, exp, 8e-3)
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_bias_gelu_epilogue(dtype):
+    exp, got, (got2, exp2) = _run(dtype, M=200, N=256, K=192, groups=2, k_shards=1, causal=0,
+                                  a_spec=((1, 200, 192), dict(mn=0)),
+                                  b_spec=((2, 256, 192), dict(mn=0)), bias=True, act=G.ACT_GELU)
+    _close(got, exp, 8e-3)
+    _close(got2, exp2, 1.5e-2)
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_dgelu_epilogue_mn_major_b(dtype):
+    # input-gradient style: B is [g][k][n] (MN-major)
+    exp, got, _ = _run(dtype, M=260, N=128, K=256, groups=2, k_shards=1, causal=0,
+                       a_spec=((1, 260, 256), dict(mn=0)), b_spec=((2, 256, 128), dict(mn=1)),
+                       act=G.ACT_DGELU)
+    _close(got, exp, 1e-2)
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_wgrad_both_mn_major_fp32(dtype):
+    exp, got, _ = _run(dtype, M=192, N=320, K=384, groups=2, k_shards=1, causal=0,
+                       a_spec=((1, 384, 192), dict(mn=1)), b_spec=((2, 384, 320), dict(mn=1)),
+                       out_f32=True)
+    _close(got, exp, 1e-5)
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_k_shard_reduction(dtype):
+    # row-split style: both operands walk 3 shards along the group axis
+    exp, got, _ = _run(dtype, M=384, N=256, K=128, groups=1, k_shards=3, causal=0,
+                       a_spec=((3, 384, 128), dict(mn=0, g_div=1 << 30, k_shard=1)),
+                       b_spec=((3, 256, 128), dict(mn=0, g_div=1 << 30, k_shard=1)),
+                       bias=True, resid=True)
+    _close(got, exp, 8e-3)
+    # column-split input gradient: B MN-major per shard
+    exp, got, _ = _run(dtype, M=256, N=192, K=128, groups=1, k_shards=2, causal=0,
+                       a_spec=((2, 256, 128), dict(mn=0, g_div=1 << 30, k_shard=1)),
+                       b_spec=((2, 128, 192), dict(mn=1, g_div=1 << 30, k_shard=1)))
+    _close(got, exp, 8e-3)
+
+
+@pytest.mark.parametrize("dtype,s,d", [("bf16", 320, 64), ("fp16", 256, 80), ("fp16", 64, 32),
+                                       ("bf16", 256, 128)])
+def test_attention_arrangements(dtype, s, d):
+    """Per-head views into a packed [ij][s][3*heads*d] buffer: scores with
+    upper tiles skipped, P V with the K range limited below the diagonal
+    tile, P^T dO with the K range from the diagonal tile."""
+    heads, ij = 2, 3
+    width = 3 * heads * d
+    grp = ij * heads
+    # scores: Q K^T
+    exp, got, _ = _run(dtype, M=s, N=s, K=d, groups=grp, k_shards=1, causal=G.CAUSAL_SKIP_UPPER,
+                       a_spec=((ij, s, width), dict(mn=0, x_mod=heads, x_mul=d, g_div=heads)),
+                       b_spec=((ij, s, width), dict(mn=0, x_mod=heads, x_mul=d, x_off=heads * d,
+                                                    g_div=heads)), std_b=0.3)
+    low = np.tril(np.ones((s, s), dtype=bool))
+    _close(got, exp, 8e-3, mask=np.broadcast_to(low, got.shape))
+    # P V with lower-triangular P (K range limited)
+    rng = np.random.default_rng(5)
+    exp, got, _ = _run(dtype, M=s, N=d, K=s, groups=grp, k_shards=1, causal=G.CAUSAL_K_BELOW,
+                       a_spec=((grp, s, s), dict(mn=0)),
+                       b_spec=((ij, s, width), dict(mn=1, x_mod=heads, x_mul=d, x_off=2 * heads * d,
+                                                    g_div=heads)), std_a=0.2)
+    _close(got, exp, 8e-3)
+    # P^T dO (A MN-major, K from the diagonal tile)
+    exp, got, _ = _run(dtype, M=s, N=d, K=s, groups=grp, k_shards=1, causal=G.CAUSAL_K_FROM,
+                       a_spec=((grp, s, s), dict(mn=1)),
+                       b_spec=((ij, s, heads * d), dict(mn=1, x_mod=heads, x_mul=d, g_div=heads)),
+                       std_a=0.2)
+    _close(got, exp, 8e-3)

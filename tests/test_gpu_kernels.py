@@ -1,0 +1,167 @@
+"""GPU parity of the bandwidth kernels against the CPU oracle: LayerNorm
+forward/backward, causal softmax forward/backward, column sums, overflow
+check, fused Adam, loss-scale update."""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from transformer_layer_step_b200 import gptlayer as G
+from transformer_layer_step_b200 import synth
+from transformer_layer_step_b200.harness import LayerStep
+from gpu_util import (need_gpu, dev_tensor, host_values, rounded, stream, check_device_error,
+                      rel_max_err)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype,rows,h", [("bf16", 333, 768), ("fp16", 130, 128),
+                                          ("fp16", 97, 1024), ("bf16", 70, 2560),
+                                          ("bf16", 9, 10240)])
+def test_layernorm_fwd_bwd(dtype, rows, h):
+    need_gpu()
+    rng = np.random.default_rng(rows + h)
+    x = rounded(rng.standard_normal((rows, h)) * 2 + 0.5, dtype)
+    g = rounded(1 + 0.1 * rng.standard_normal(h), dtype)
+    b = rounded(0.1 * rng.standard_normal(h), dtype)
+    gy = rounded(rng.standard_normal((rows, h)), dtype)
+    res = rounded(rng.standard_normal((rows, h)), dtype)
+    xt, gt, bt, gyt, rt = (dev_tensor(a, dtype) for a in (x, g, b, gy, res))
+    y = torch.empty_like(xt)
+    mu = torch.empty(rows, dtype=torch.float32, device="cuda")
+    rstd = torch.empty_like(mu)
+    G.layernorm_fwd(rows, h, dtype, xt, gt, bt, 1e-5, y, mu, rstd, stream())
+    ye, mue, rse, xhat = oracle.layer_norm_fwd(x, g, b, 1e-5)
+    torch.cuda.synchronize()
+    assert rel_max_err(host_values(y, dtype), ye) < 2e-2
+    np.testing.assert_allclose(mu.cpu().numpy(), mue, rtol=0, atol=1e-5)
+    np.testing.assert_allclose(rstd.cpu().numpy(), rse, rtol=1e-5)
+
+    dx = torch.empty_like(xt)
+    dg = torch.empty(h, dtype=torch.float32, device="cuda")
+    db = torch.empty_like(dg)
+    dsum = torch.empty_like(dg)
+    scratch = torch.empty(G.layernorm_bwd_scratch_bytes(rows, h), dtype=torch.uint8, device="cuda")
+    G.layernorm_bwd(rows, h, dtype, gyt, xt, mu, rstd, gt, rt, dx, dg, db, dsum, scratch, stream())
+    check_device_error()
+    dxe, dge, dbe = oracle.layer_norm_bwd(gy, xhat, rse, g)
+    dxe = dxe + res
+    assert rel_max_err(host_values(dx, dtype), dxe) < 2e-2
+    assert rel_max_err(dg.cpu().numpy(), dge) < 2e-3
+    assert rel_max_err(db.cpu().numpy(), dbe) < 1e-4
+    assert rel_max_err(dsum.cpu().numpy(), host_values(dx, dtype).sum(axis=0)) < 1e-4
+
+
+@pytest.mark.parametrize("dtype,s,blocks", [("bf16", 1024, 3), ("fp16", 64, 5), ("fp16", 272, 2),
+                                            ("bf16", 2048, 1)])
+def test_causal_softmax_fwd_bwd(dtype, s, blocks):
+    need_gpu()
+    rng = np.random.default_rng(s)
+    d = 64
+    scale = 1.0 / math.sqrt(d)
+    sc = rounded(rng.standard_normal((blocks, s, s)) * 6, dtype)
+    dpv = rounded(rng.standard_normal((blocks, s, s)), dtype)
+    st = dev_tensor(sc, dtype)
+    G.softmax_fwd(blocks, s, dtype, scale, st, stream())
+    dpt = dev_tensor(dpv, dtype)
+    torch.cuda.synchronize()
+    p_gpu = host_values(st, dtype)
+    G.softmax_bwd(blocks, s, dtype, scale, st, dpt, stream())
+    check_device_error()
+    ds_gpu = host_values(dpt, dtype)
+    for blk in range(blocks):
+        pe = oracle.causal_softmax(sc[blk] * scale)
+        low = np.tril(np.ones((s, s), dtype=bool))
+        np.testing.assert_allclose(p_gpu[blk][low], pe[low], rtol=2e-2, atol=1e-3)
+        # zeros above the diagonal inside the diagonal tile
+        for p in range(0, s, 37):
+            end = min(s, (p // 128 + 1) * 128)
+            assert np.all(p_gpu[blk, p, p + 1:end] == 0)
+        # backward: the oracle's formula applied to the GPU's own P
+        pg = p_gpu[blk] * low
+        dse = scale * pg * (dpv[blk] - (pg * dpv[blk]).sum(axis=1, keepdims=True))
+        err = np.abs(ds_gpu[blk][low] - dse[low]).max() / np.abs(dse[low]).max()
+        assert err < 2e-2
+        for p in range(0, s, 41):
+            end = min(s, (p // 128 + 1) * 128)
+            assert np.all(ds_gpu[blk, p, p + 1:end] == 0)
+
+
+@pytest.mark.parametrize("dtype,rows,n,groups", [("bf16", 8192, 768, 1), ("fp16", 130, 256, 2),
+                                                 ("fp16", 1000, 1920, 4)])
+def test_colsum(dtype, rows, n, groups):
+    need_gpu()
+    rng = np.random.default_rng(n)
+    a = rounded(rng.standard_normal((groups, rows, n)), dtype)
+    at = dev_tensor(a, dtype)
+    out = torch.empty(groups * n, dtype=torch.float32, device="cuda")
+    scratch = torch.empty(G.colsum_scratch_bytes(n, groups), dtype=torch.uint8, device="cuda")
+    G.colsum(rows, n, groups, n, rows * n, dtype, at, out, scratch, stream())
+    check_device_error()
+    np.testing.assert_allclose(out.cpu().numpy(), a.sum(axis=1).reshape(-1), rtol=0, atol=1e-3)
+
+
+def test_overflow_and_scaler_decisions():
+    need_gpu()
+    n = 1 << 20
+    g = torch.from_numpy(synth.random_fp32(n, 1)).cuda()
+    state = torch.zeros(8, dtype=torch.int32, device="cuda")
+    for pos, bad in [(None, None), (0, math.inf), (n - 1, -math.inf), (123457, math.nan),
+                     (n // 2, math.inf)]:
+        gg = g.clone()
+        if pos is not None:
+            gg[pos] = bad
+        state[2] = 7
+        G.check_overflow(n, gg, state, stream())
+        torch.cuda.synchronize()
+        assert int(state[2]) == oracle.found_inf(gg.cpu().numpy())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_adam_matches_oracle(dtype):
+    need_gpu()
+    cfg = dataclasses.replace(synth.CONFIGS["tiny"], dtype=dtype)
+    ls = LayerStep(cfg, synth.make_inputs(cfg))
+    n = ls.n_params
+    rng = np.random.default_rng(3)
+    hp = ls.hyper
+    master = ls.master.cpu().numpy().astype(np.float64)
+    m = np.zeros(n)
+    v = np.zeros(n)
+    state = dict(scale=hp["init_scale"], growth_tracker=0, step=0)
+    for step in range(4):
+        grad = (rng.standard_normal(n) * 1e-3 * state["scale"]).astype(np.float32)
+        if step == 2:
+            grad[n // 3] = np.inf                       # this step must be skipped
+        ls.grad.copy_(torch.from_numpy(grad))
+        m_in, v_in, p_in = ls.m.cpu().numpy(), ls.v.cpu().numpy(), ls.master.cpu().numpy()
+        w_in = ls.w16.clone()
+        ls.adam()
+        ls.scale_update()
+        torch.cuda.synchronize()
+        f = oracle.found_inf(grad)
+        f32 = lambda x: float(np.float32(x))
+        pe, me, ve, we = oracle.adam_step(p_in, m_in, v_in, grad, state["scale"], state["step"],
+                                          f32(hp["lr"]), f32(hp["beta1"]), f32(hp["beta2"]),
+                                          f32(hp["eps"]), f32(hp["weight_decay"]), dtype, f)
+        state = oracle.loss_scale_update(state, f, hp["growth_interval"], hp["growth_factor"],
+                                         hp["backoff_factor"], hp["min_scale"])
+        sc = ls.scaler()
+        assert sc["found_inf"] == f
+        assert (sc["scale"], sc["growth_tracker"], sc["step"]) == \
+            (state["scale"], state["growth_tracker"], state["step"])
+        pg, mg, vg = ls.master.cpu().numpy(), ls.m.cpu().numpy(), ls.v.cpu().numpy()
+        if f:
+            assert np.array_equal(pg, p_in) and np.array_equal(mg, m_in) and np.array_equal(vg, v_in)
+            assert torch.equal(ls.w16, w_in)
+            continue
+        lr = f32(hp["lr"])
+        assert np.all(np.abs(pg - pe) <= 1e-6 * np.maximum(np.abs(pe), lr))
+        assert np.all(np.abs(vg - ve) <= 1e-6 * np.abs(ve) + 1e-45)
+        assert np.all(np.abs(mg - me) <= 1e-6 * np.maximum(np.abs(me), np.sqrt(np.mean(me ** 2))))
+        # the 16-bit copy is the RNE cast of the GPU's own fp32 master
+        wg = ls.w16.view(torch.int16).cpu().numpy().view(np.uint16)
+        np.testing.assert_array_equal(wg, oracle.cast_to_16(pg.astype(np.float64), dtype))

@@ -1,0 +1,83 @@
+"""GPU parity of the whole layer step (gpt_layer_fwd, gpt_layer_bwd through
+the C ABI) against the float64 oracle on the same seeded inputs.
+
+Bar: for Out, dX and each of the 12 gradients,
+max|gpu - oracle| <= 2e-2 * RMS(oracle).  The gradients are those of the
+scaled loss (the criterion is scale-invariant)."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from transformer_layer_step_b200 import gptlayer as G
+from transformer_layer_step_b200 import synth
+from transformer_layer_step_b200.harness import LayerStep
+from gpu_util import need_gpu, host_values, check_device_error, rel_max_err
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+SMALL = {
+    # several tiles in every GEMM, ragged tails, t = 2 and t = 4
+    "small-bf16-t2": synth.LayerConfig("small-bf16-t2", 2, 256, 256, 4, 1024, 2, synth.BF16),
+    "small-fp16-t4-d80": synth.LayerConfig("small-fp16-t4-d80", 1, 384, 640, 8, 2560, 4, synth.FP16),
+    "small-bf16-d128": synth.LayerConfig("small-bf16-d128", 3, 128, 512, 4, 2048, 1, synth.BF16),
+}
+
+
+def _run_and_compare(cfg, variant, with_r, seed=0):
+    need_gpu()
+    inp = synth.make_inputs(cfg, seed=seed, variant=variant, with_r=with_r)
+    ls = LayerStep(cfg, inp)
+    scale = ls.hyper["init_scale"]
+    dy_bits = synth.loss_grad_bits(cfg, scale, inp["r"] if with_r else None)
+    ls.set_dy_bits(dy_bits)
+    ls.fwd()
+    ls.bwd()
+    check_device_error()
+    out_gpu = host_values(ls.y, cfg.dtype)
+    dx_gpu = host_values(ls.dx, cfg.dtype)
+    grads_gpu = ls.grads_host()
+
+    x = synth.from_bits(inp["x"], cfg.dtype).reshape(cfg.tokens, cfg.hidden)
+    p = {k: synth.from_bits(v, cfg.dtype).reshape(v.shape) for k, v in inp["params"].items()}
+    dout = synth.from_bits(dy_bits, cfg.dtype).reshape(cfg.tokens, cfg.hidden)
+    out_o, cache = oracle.layer_fwd(x, p, cfg.dims(), ls.hyper["ln_eps"])
+    dx_o, gr_o = oracle.layer_bwd(cache, p, cfg.dims(), dout)
+    errs = {"out": rel_max_err(out_gpu, out_o), "dx": rel_max_err(dx_gpu, dx_o)}
+    for k in gr_o:
+        errs[k] = rel_max_err(grads_gpu[k].reshape(gr_o[k].shape), gr_o[k])
+    bad = {k: v for k, v in errs.items() if not v <= TOL}
+    assert not bad, (bad, errs)
+    return errs
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("variant,with_r", [("biased", True), ("plain", False)])
+def test_small_layers(name, variant, with_r):
+    _run_and_compare(SMALL[name], variant, with_r)
+
+
+@pytest.mark.parametrize("variant,with_r", [("plain", False), ("biased", True)])
+def test_tiny_config(variant, with_r):
+    _run_and_compare(synth.CONFIGS["tiny"], variant, with_r)
+
+
+@pytest.mark.parametrize("name", ["gpt2-117m", "gpt2-345m"])
+def test_full_size_configs(name):
+    _run_and_compare(synth.CONFIGS[name], "biased", True)
+
+
+def test_repeat_is_bitwise_deterministic():
+    need_gpu()
+    cfg = SMALL["small-bf16-t2"]
+    inp = synth.make_inputs(cfg, variant="biased", with_r=True)
+    ls = LayerStep(cfg, inp)
+    ls.set_dy_bits(synth.loss_grad_bits(cfg, 1024.0, inp["r"]))
+    ls.fwd(); ls.bwd()
+    y1, dx1, g1 = ls.y.clone(), ls.dx.clone(), ls.grad.clone()
+    ls.fwd(); ls.bwd()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, ls.y) and torch.equal(dx1, ls.dx) and torch.equal(g1, ls.grad)

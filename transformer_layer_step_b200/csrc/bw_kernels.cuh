@@ -1,0 +1,409 @@
+// bw_kernels.cuh — HBM-bandwidth kernels of the layer step (sm_100a).
+//
+// LayerNorm forward/backward, the fused causal scale-mask-softmax
+// forward/backward ("Training GPT-2 with Megatron-LM" §6.2 fused_softmax),
+// column sums for bias gradients, and the optimizer side of mixed precision
+// ("Megatron-LM overview" §3.1, §4.2): overflow check, fused unscale + Adam +
+// 16-bit cast on FP32 masters, dynamic loss-scale update.
+//
+// All loads and stores are 16-byte vectors on contiguous rows; reductions use
+// warp shuffles and shared memory; statistics and accumulations are fp32.
+#pragma once
+#include "common.cuh"
+
+namespace gptl {
+
+// ------------------------------------------------------------ team reduce
+// A "team" of TPR consecutive threads owns one row.  TPR is a power of two;
+// teams wider than a warp combine their warps through shared memory.
+template <int TPR>
+__device__ __forceinline__ float team_sum(float v, float *red) {
+#pragma unroll
+  for (int o = (TPR < 32 ? TPR : 32) / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if constexpr (TPR > 32) {
+    constexpr int W = TPR / 32;
+    const int lane = threadIdx.x & 31;
+    const int wit = (threadIdx.x / 32) % W;             // warp index within the team
+    const int team = threadIdx.x / TPR;
+    __syncthreads();
+    if (lane == 0) red[team * W + wit] = v;
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < W; ++i) s += red[team * W + i];
+    v = s;
+  }
+  return v;
+}
+
+// ------------------------------------------------------------ LayerNorm fwd
+// y = gamma * (x - mu) * rstd + beta, biased variance, fp32 statistics saved.
+// Each thread holds VPT 16-byte vectors of its row in registers.
+template <typename T, int TPR, int VPT>
+__global__ void __launch_bounds__(256) ln_fwd_kernel(const T *__restrict__ x,
+                                                     const T *__restrict__ gamma,
+                                                     const T *__restrict__ beta, T *__restrict__ y,
+                                                     float *__restrict__ mu_out,
+                                                     float *__restrict__ rstd_out, int rows, int h,
+                                                     float eps) {
+  __shared__ float red[256 / 32 + 8];
+  constexpr int RPB = 256 / TPR;
+  const int team = threadIdx.x / TPR, tl = threadIdx.x % TPR;
+  const int row = blockIdx.x * RPB + team;
+  const bool active = row < rows;
+  const int r = active ? row : rows - 1;
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x + (long long)r * h);
+  float v[VPT][8];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    unpack8<T>(xr[tl + i * TPR], v[i]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s += v[i][e];
+  }
+  const float mu = team_sum<TPR>(s, red) / (float)h;
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float d = v[i][e] - mu;
+      ss += d * d;
+    }
+  const float var = team_sum<TPR>(ss, red) / (float)h;
+  const float rstd = 1.0f / sqrtf(var + eps);
+  if (!active) return;
+  const uint4 *g4 = reinterpret_cast<const uint4 *>(gamma);
+  const uint4 *b4 = reinterpret_cast<const uint4 *>(beta);
+  uint4 *yr = reinterpret_cast<uint4 *>(y + (long long)r * h);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    float g[8], b[8], o[8];
+    unpack8<T>(__ldg(g4 + tl + i * TPR), g);
+    unpack8<T>(__ldg(b4 + tl + i * TPR), b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = (v[i][e] - mu) * rstd * g[e] + b[e];
+    yr[tl + i * TPR] = pack8<T>(o);
+  }
+  if (tl == 0) {
+    mu_out[r] = mu;
+    rstd_out[r] = rstd;
+  }
+}
+
+// ------------------------------------------------------------ LayerNorm bwd
+// dx = resid + rstd * (gh - mean(gh) - xhat * mean(gh * xhat)), gh = gy * gamma.
+// Per-block partial column sums of gy*xhat (dgamma), gy (dbeta) and, when
+// requested, of dx itself (the next bias gradient) go to `part`
+// ([nparts][gridDim.x][h]); reduce_parts_kernel finishes them.
+template <typename T, int TPR, int VPT>
+__global__ void __launch_bounds__(256) ln_bwd_kernel(
+    const T *__restrict__ gy, const T *__restrict__ x, const float *__restrict__ mu_in,
+    const float *__restrict__ rstd_in, const T *__restrict__ gamma, const T *__restrict__ resid,
+    T *__restrict__ dx, float *__restrict__ part, int rows, int h, int want_dx_sum) {
+  extern __shared__ float sm[];          // [RPB][h] staging for the column partials
+  __shared__ float red[256 / 32 + 8];
+  constexpr int RPB = 256 / TPR;
+  const int team = threadIdx.x / TPR, tl = threadIdx.x % TPR;
+  float pg[VPT][8], pb[VPT][8], pd[VPT][8];
+  float gm[VPT][8];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(gamma) + tl + i * TPR), gm[i]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pg[i][e] = pb[i][e] = pd[i][e] = 0.f;
+  }
+  const int row_step = gridDim.x * RPB;
+  // every team runs the same number of iterations (the team reductions
+  // synchronise the whole block when TPR > 32)
+  const int iters = (rows + row_step - 1) / row_step;
+  for (int it = 0; it < iters; ++it) {
+    const int row = it * row_step + blockIdx.x * RPB + team;
+    const bool active = row < rows;
+    const int r = active ? row : rows - 1;
+    const uint4 *gr = reinterpret_cast<const uint4 *>(gy + (long long)r * h);
+    const uint4 *xr = reinterpret_cast<const uint4 *>(x + (long long)r * h);
+    const float mu = mu_in[r], rstd = rstd_in[r];
+    float xh[VPT][8], gh[VPT][8], g[VPT][8];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      float xv[8];
+      unpack8<T>(gr[tl + i * TPR], g[i]);
+      unpack8<T>(xr[tl + i * TPR], xv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        xh[i][e] = (xv[e] - mu) * rstd;
+        gh[i][e] = g[i][e] * gm[i][e];
+        s1 += gh[i][e];
+        s2 += gh[i][e] * xh[i][e];
+      }
+    }
+    const float m1 = team_sum<TPR>(s1, red) / (float)h;
+    const float m2 = team_sum<TPR>(s2, red) / (float)h;
+    if (active) {
+      const uint4 *rr = reinterpret_cast<const uint4 *>(resid + (long long)r * h);
+      uint4 *dr = reinterpret_cast<uint4 *>(dx + (long long)r * h);
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        float rv[8], o[8];
+        unpack8<T>(rr[tl + i * TPR], rv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = rv[e] + rstd * (gh[i][e] - m1 - xh[i][e] * m2);
+        const uint4 q = pack8<T>(o);
+        dr[tl + i * TPR] = q;
+        float oq[8];
+        unpack8<T>(q, oq);                 // sum what was stored
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          pg[i][e] += g[i][e] * xh[i][e];
+          pb[i][e] += g[i][e];
+          pd[i][e] += oq[e];
+        }
+      }
+    }
+  }
+  // combine the RPB teams of this block, one partial array at a time
+  const int nparts = want_dx_sum ? 3 : 2;
+  for (int k = 0; k < nparts; ++k) {
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < VPT; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        sm[team * h + (tl + i * TPR) * 8 + e] = (k == 0 ? pg[i][e] : (k == 1 ? pb[i][e] : pd[i][e]));
+    __syncthreads();
+    float *dst = part + ((long long)k * gridDim.x + blockIdx.x) * h;
+    for (int c = threadIdx.x; c < h; c += blockDim.x) {
+      float s = 0.f;
+      for (int t = 0; t < RPB; ++t) s += sm[t * h + c];
+      dst[c] = s;
+    }
+  }
+}
+
+// out[k][c] = sum_b part[k][b][c], for k < nk arrays of width n.
+__global__ void reduce_parts_kernel(const float *__restrict__ part, int nblocks, int n,
+                                    float *out0, float *out1, float *out2) {
+  const int k = blockIdx.y;
+  float *out = k == 0 ? out0 : (k == 1 ? out1 : out2);
+  const float *src = part + (long long)k * nblocks * n;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < n; c += gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int b = 0; b < nblocks; ++b) s += src[(long long)b * n + c];
+    out[c] = s;
+  }
+}
+
+// ---------------------------------------------------------- column sums
+// Column sums of G matrices [rows][n] (row pitch ld, matrix pitch gstride):
+// block (32 x 8) covers 256 columns of one matrix and every 8*gridDim.y-th
+// row; partials part[blockIdx.y][g][n].
+template <typename T>
+__global__ void __launch_bounds__(256) colsum_kernel(const T *__restrict__ a, int rows, int n,
+                                                     long long ld, long long gstride,
+                                                     float *__restrict__ part, int groups) {
+  __shared__ float sm[8][256 + 8];
+  const int g = blockIdx.z;
+  const int cv = blockIdx.x * 32 + threadIdx.x;    // 8-column vector index
+  const bool col_ok = cv * 8 < n;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const T *base = a + (long long)g * gstride;
+  if (col_ok)
+    for (int r = blockIdx.y * 8 + threadIdx.y; r < rows; r += gridDim.y * 8) {
+      float f[8];
+      unpack8<T>(*reinterpret_cast<const uint4 *>(base + (long long)r * ld + cv * 8), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += f[e];
+    }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) sm[threadIdx.y][threadIdx.x * 8 + e] = acc[e];
+  __syncthreads();
+  const int c = threadIdx.y * 32 + threadIdx.x;     // 0..255 column within the block
+  const int col = blockIdx.x * 256 + c;
+  if (col < n) {
+    float s = 0.f;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) s += sm[t][c];
+    part[((long long)blockIdx.y * groups + g) * n + col] = s;
+  }
+}
+
+// --------------------------------------------------------- causal softmax
+// In place on [rows = G*s][s] score blocks.  Row p of a block: entries q <= p
+// get softmax(scale * S), entries p < q < end of the 128-wide diagonal tile
+// get 0 (the attention GEMMs read those tiles).  One warp per row; each lane
+// holds NV 8-element vectors.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) softmax_fwd_kernel(T *__restrict__ s_io, long long nrows,
+                                                          int s, float scale) {
+  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= nrows) return;
+  const int p = (int)(row % s);
+  const int valid = p + 1;
+  const int wend = min(s, (p / 128 + 1) * 128);
+  uint4 *rp = reinterpret_cast<uint4 *>(s_io + row * (long long)s);
+  const float l2e = 1.4426950408889634f * scale;
+  float v[NV][8];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c0 = (lane + 32 * i) * 8;
+    if (c0 < valid) {
+      unpack8<T>(rp[lane + 32 * i], v[i]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        v[i][e] = (c0 + e < valid) ? v[i][e] * l2e : -INFINITY;
+        mx = fmaxf(mx, v[i][e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c0 = (lane + 32 * i) * 8;
+    if (c0 < valid) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        v[i][e] = (c0 + e < valid) ? exp2f(v[i][e] - mx) : 0.f;
+        sum += v[i][e];
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = 1.0f / sum;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c0 = (lane + 32 * i) * 8;
+    if (c0 < wend) {
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = (c0 < valid) ? v[i][e] * inv : 0.f;
+      rp[lane + 32 * i] = pack8<T>(o);
+    }
+  }
+}
+
+// dS = scale * P * (dP - sum_q P*dP), in place over dP; zeros above the
+// diagonal inside the diagonal tile.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) softmax_bwd_kernel(const T *__restrict__ prob,
+                                                          T *__restrict__ d_io, long long nrows,
+                                                          int s, float scale) {
+  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= nrows) return;
+  const int p = (int)(row % s);
+  const int valid = p + 1;
+  const int wend = min(s, (p / 128 + 1) * 128);
+  const uint4 *pp = reinterpret_cast<const uint4 *>(prob + row * (long long)s);
+  uint4 *dp = reinterpret_cast<uint4 *>(d_io + row * (long long)s);
+  float pv[NV][8], dv[NV][8];
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c0 = (lane + 32 * i) * 8;
+    if (c0 < valid) {
+      unpack8<T>(pp[lane + 32 * i], pv[i]);
+      unpack8<T>(dp[lane + 32 * i], dv[i]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (c0 + e >= valid) pv[i][e] = 0.f;
+        dot += pv[i][e] * dv[i][e];
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c0 = (lane + 32 * i) * 8;
+    if (c0 < wend) {
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = (c0 < valid) ? scale * pv[i][e] * (dv[i][e] - dot) : 0.f;
+      dp[lane + 32 * i] = pack8<T>(o);
+    }
+  }
+}
+
+// ------------------------------------------------------------- optimizer
+// found_inf |= any exponent field all ones in grad[0, n)  (n % 4 == 0)
+__global__ void __launch_bounds__(256) overflow_kernel(const float4 *__restrict__ g, long long n4,
+                                                       int *__restrict__ found) {
+  bool bad = false;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float4 v = __ldcs(g + i);
+    const uint32_t e = 0x7F800000u;
+    bad |= ((__float_as_uint(v.x) & e) == e) | ((__float_as_uint(v.y) & e) == e) |
+           ((__float_as_uint(v.z) & e) == e) | ((__float_as_uint(v.w) & e) == e);
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(found, 1);
+}
+
+struct AdamArgs {
+  float lr, beta1, beta2, eps, wd;
+};
+
+// Fused unscale + Adam + 16-bit cast; skipped entirely when found_inf.
+template <typename T>
+__global__ void __launch_bounds__(256) adam_kernel(float4 *__restrict__ master,
+                                                   float4 *__restrict__ m, float4 *__restrict__ v,
+                                                   const float4 *__restrict__ grad,
+                                                   T *__restrict__ w16, long long n4, AdamArgs a,
+                                                   const gptl_scaler_state *st) {
+  if (st->found_inf) return;
+  const float scale = st->scale;
+  const int t = st->step + 1;
+  const float bc1 = (float)(1.0 - pow((double)a.beta1, (double)t));
+  const float bc2 = (float)(1.0 - pow((double)a.beta2, (double)t));
+  const float omb1 = 1.0f - a.beta1, omb2 = 1.0f - a.beta2;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float4 g4 = __ldcs(grad + i);
+    float4 p4 = master[i], m4 = m[i], v4 = v[i];
+    float gg[4] = {g4.x, g4.y, g4.z, g4.w};
+    float pp[4] = {p4.x, p4.y, p4.z, p4.w};
+    float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+    float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float g = gg[k] / scale;
+      mm[k] = a.beta1 * mm[k] + omb1 * g;
+      vv[k] = a.beta2 * vv[k] + omb2 * (g * g);
+      const float mh = mm[k] / bc1;
+      const float vh = vv[k] / bc2;
+      pp[k] = pp[k] - a.lr * (mh / (sqrtf(vh) + a.eps) + a.wd * pp[k]);
+    }
+    master[i] = make_float4(pp[0], pp[1], pp[2], pp[3]);
+    m[i] = make_float4(mm[0], mm[1], mm[2], mm[3]);
+    v[i] = make_float4(vv[0], vv[1], vv[2], vv[3]);
+    uint2 w;
+    w.x = Cvt<T>::pack2(pp[0], pp[1]);
+    w.y = Cvt<T>::pack2(pp[2], pp[3]);
+    reinterpret_cast<uint2 *>(w16)[i] = w;
+  }
+}
+
+__global__ void scale_update_kernel(gptl_scaler_state *st, int interval, float growth,
+                                    float backoff, float min_scale) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  if (st->found_inf) {
+    st->scale = fmaxf(st->scale * backoff, min_scale);
+    st->growth_tracker = 0;
+  } else {
+    st->growth_tracker += 1;
+    if (st->growth_tracker == interval) {
+      st->scale = st->scale * growth;
+      st->growth_tracker = 0;
+    }
+    st->step += 1;
+  }
+}
+
+}  // namespace gptl

@@ -1,0 +1,359 @@
+// gemm_tc.cuh — persistent tcgen05/TMEM GEMM for sm_100a, fed by TMA.
+//
+// One kernel serves every dense contraction of the layer step: the four
+// linear layers (forward, input gradient, weight gradient) and the six
+// attention products.  D[M,N] = sum_k A[M,k] * B[N,k] per group, with
+//   * operands read through 3-D TMA views (x = contiguous column, row, group)
+//     and staged in 128-row/BN-row x 64-deep shared-memory tiles;
+//   * either operand K-major (rows = M/N index, x = K) or MN-major
+//     (rows = K index, x = M/N), using the hardware transpose of the MMA
+//     instead of any transposing copy;
+//   * an optional walk of the K loop over tensor-parallel shards (the row
+//     split's partial sums and the column split's input-gradient sums are
+//     accumulated in one TMEM accumulator: "Megatron-LM 3D parallelism" §1
+//     describes the all-reduce this replaces);
+//   * causal rules for attention: skip score tiles above the diagonal, or
+//     limit the K range to the lower triangle;
+//   * fused epilogues: bias, residual, bias+GeLU (writes Z and GeLU(Z): the
+//     fused_bias_gelu of "Training GPT-2 with Megatron-LM" §6.2), GeLU'
+//     scaling of an input gradient, fp32 weight-gradient store.
+//
+// Warp roles (192 threads, one CTA per SM): warp 0 issues TMA loads into a
+// multi-stage mbarrier ring, warp 1 allocates TMEM and one thread issues
+// tcgen05.mma (M=128, N=BN, K=16 each), warps 2..5 drain the double-buffered
+// accumulator with tcgen05.ld while the next tile's MMAs run.
+#pragma once
+#include "common.cuh"
+
+namespace gptl {
+
+constexpr int kBM = 128;          // tile rows (UMMA M)
+constexpr int kBK = 64;           // tile depth per pipeline stage
+constexpr int kGemmThreads = 192;
+
+enum : int { kActNone = 0, kActGelu = 1, kActDGelu = 2 };
+enum : int { kCausalNone = 0, kCausalSkipUpper = 1, kCausalKBelow = 2, kCausalKFrom = 3 };
+
+struct OperandRule {
+  int mn_major;                // 0: K-major, 1: MN-major
+  int w;                       // MN-major chunk width in elements (64, 32 or 16)
+  int x_mod, x_mul, x_off;     // column offset of group G: (G % x_mod) * x_mul + x_off
+  int g_div;                   // group coordinate G / g_div ...
+  int k_shard;                 // ... plus the k-shard index when set
+};
+
+struct alignas(64) GemmParams {
+  CUtensorMap map_a;
+  CUtensorMap map_b;
+  OperandRule ra, rb;
+  int M, N, K, groups, k_shards, causal;
+  int bn, bn_alloc, stages, tmem_cols;
+  uint32_t idesc;
+  int m_tiles, n_tiles;
+  long long total_tiles;
+  // epilogue
+  void *out;
+  long long ldo;
+  int o_mod;
+  long long o_str_mod, o_str_div;
+  int out_f32;
+  const void *bias;
+  long long bias_g_stride;
+  const void *resid;
+  long long ld_resid;
+  const void *aux;
+  void *out2;
+  int act;
+};
+
+struct TileInfo {
+  int g, m0, n0, kb_begin, kb_end;
+  bool skip;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const GemmParams &p, long long idx) {
+  TileInfo t;
+  const long long tpg = (long long)p.m_tiles * p.n_tiles;
+  t.g = (int)(idx / tpg);
+  const int rem = (int)(idx - (long long)t.g * tpg);
+  const int mt = rem / p.n_tiles, nt = rem - (rem / p.n_tiles) * p.n_tiles;
+  t.m0 = mt * kBM;
+  t.n0 = nt * p.bn;
+  t.skip = (p.causal == kCausalSkipUpper) && (t.n0 > t.m0 + kBM - 1);
+  t.kb_begin = 0;
+  t.kb_end = (p.K + kBK - 1) / kBK;
+  if (p.causal == kCausalKBelow) t.kb_end = (min(p.K, t.m0 + kBM) + kBK - 1) / kBK;
+  if (p.causal == kCausalKFrom) t.kb_begin = t.m0 / kBK;
+  return t;
+}
+
+__device__ __forceinline__ uint32_t swizzle_layout(int w) {
+  return w == 64 ? 2u : (w == 32 ? 4u : 6u);
+}
+
+// Issue the TMA loads of one operand tile for k-block starting at k0.
+__device__ __forceinline__ void load_operand(const CUtensorMap *map, const OperandRule &r,
+                                             uint32_t dst, int rows, int g, int ks, int mn0,
+                                             int k0, uint32_t bar) {
+  const int x0 = (g % r.x_mod) * r.x_mul + r.x_off;
+  const int gc = g / r.g_div + (r.k_shard ? ks : 0);
+  if (!r.mn_major) {
+    tma_load_3d(dst, map, x0 + k0, mn0, gc, bar);
+  } else {
+    const int chunks = rows / r.w;
+    for (int c = 0; c < chunks; ++c)
+      tma_load_3d(dst + (uint32_t)(c * kBK * r.w * 2), map, x0 + mn0 + c * r.w, k0, gc, bar);
+  }
+}
+
+// Shared-memory descriptor of the 16-deep slice `step` of an operand tile.
+//   K-major tile  [rows][64] (128B rows, 128B swizzle): SBO = 8 rows = 1024 B,
+//                 the slice starts 32 B further per step.
+//   MN-major tile [rows/w chunks][64 k-rows][w]: rows of 2w bytes, SBO = 8
+//                 k-rows = 16w B, LBO = chunk stride = 64 * 2w B; the slice
+//                 starts 16 k-rows further per step.
+__device__ __forceinline__ uint64_t operand_desc(const OperandRule &r, uint32_t base, int step) {
+  if (!r.mn_major) return make_smem_desc(base + (uint32_t)step * 32u, 16u, 1024u, 2u);
+  const uint32_t row_b = (uint32_t)r.w * 2u;
+  return make_smem_desc(base + (uint32_t)step * 16u * row_b, (uint32_t)kBK * row_b, 8u * row_b,
+                        swizzle_layout(r.w));
+}
+
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > kWaitTimeoutNs) return false;
+  return true;
+}
+
+template <typename T>
+__device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int row, int n,
+                                               const uint32_t (&r)[16]) {
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  const long long off = (long long)(g % p.o_mod) * p.o_str_mod +
+                        (long long)(g / p.o_mod) * p.o_str_div + (long long)row * p.ldo + n;
+  if (p.out_f32) {
+    float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    return;
+  }
+  if (p.bias) {
+    const uint4 *b = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.bias) +
+                                                     (long long)g * p.bias_g_stride + n);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float f[8];
+      unpack8<T>(__ldg(b + h), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[8 * h + i] += f[i];
+    }
+  }
+  if (p.resid) {
+    const uint4 *rr = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.resid) +
+                                                      (long long)row * p.ld_resid + n);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float f[8];
+      unpack8<T>(rr[h], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[8 * h + i] += f[i];
+    }
+  }
+  uint4 *o = reinterpret_cast<uint4 *>(static_cast<T *>(p.out) + off);
+  if (p.act == kActGelu) {
+    uint4 *o2 = reinterpret_cast<uint4 *>(static_cast<T *>(p.out2) + off);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float z[8], a[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) z[i] = v[8 * h + i];
+      uint4 zq = pack8<T>(z);
+      float zr[8];
+      unpack8<T>(zq, zr);                 // GeLU of the stored (rounded) Z
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = gelu_f(zr[i]);
+      o[h] = zq;
+      o2[h] = pack8<T>(a);
+    }
+    return;
+  }
+  if (p.act == kActDGelu) {
+    const uint4 *zp = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.aux) + off);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float z[8];
+      unpack8<T>(zp[h], z);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[8 * h + i] *= gelu_prime_f(z[i]);
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = v[8 * h + i];
+    o[h] = pack8<T>(f);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const int a_bytes = kBM * kBK * 2;
+  const int b_bytes = p.bn * kBK * 2;
+  const int stage_bytes = a_bytes + b_bytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.stages * stage_bytes);
+  // bars: full[0,S) empty[S,2S) tfull[2S,2S+2) tempty[2S+2,2S+4) drain[2S+4]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * p.stages + 5);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const uint32_t tiles_s = smem_u32(smem);
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[p.stages + s]); };
+  auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * p.stages + a]); };
+  auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * p.stages + 2 + a]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * p.stages + 4]);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&p.map_a);
+    prefetch_tensormap(&p.map_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, parity = 0;
+      for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
+        const TileInfo ti = tile_info(p, idx);
+        if (ti.skip) continue;
+        for (int ks = 0; ks < p.k_shards; ++ks)
+          for (int kb = ti.kb_begin; kb < ti.kb_end; ++kb) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag)) goto producer_abort;
+            const uint32_t fb = full_bar(stage);
+            mbar_arrive_expect_tx(fb, (uint32_t)stage_bytes);
+            const uint32_t sa = tiles_s + (uint32_t)(stage * stage_bytes);
+            load_operand(&p.map_a, p.ra, sa, kBM, ti.g, ks, ti.m0, kb * kBK, fb);
+            load_operand(&p.map_b, p.rb, sa + a_bytes, p.bn, ti.g, ks, ti.n0, kb * kBK, fb);
+            issued |= 1u << stage;
+            parity = (parity & ~(1u << stage)) | (phase << stage);
+            if (++stage == p.stages) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+      }
+      goto producer_done;
+    producer_abort:
+      // let our own copies land before the CTA exits
+      for (int s = 0; s < p.stages; ++s)
+        if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (parity >> s) & 1u);
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
+        const TileInfo ti = tile_info(p, idx);
+        if (ti.skip) continue;
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1, abort_flag)) goto mma_abort;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.bn_alloc);
+        int it = 0;
+        for (int ks = 0; ks < p.k_shards; ++ks)
+          for (int kb = ti.kb_begin; kb < ti.kb_end; ++kb) {
+            if (!mbar_wait(full_bar(stage), phase, abort_flag)) goto mma_abort;
+            tc_fence_after();
+            const uint32_t sa = tiles_s + (uint32_t)(stage * stage_bytes);
+            const uint32_t sb = sa + (uint32_t)a_bytes;
+            const int nsteps = min(kBK, p.K - kb * kBK) / 16;
+            for (int s = 0; s < nsteps; ++s)
+              tc_mma_f16(d_tmem, operand_desc(p.ra, sa, s), operand_desc(p.rb, sb, s), p.idesc,
+                         (it > 0 || s > 0) ? 1u : 0u);
+            tc_commit(empty_bar(stage));
+            ++it;
+            if (++stage == p.stages) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        tc_commit(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      goto mma_done;
+    mma_abort:
+      // wait for the MMAs already issued before TMEM is released
+      tc_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+    mma_done:;
+    }
+  } else {
+    // -------------------------------------------------- epilogue warps
+    const int q = warp & 3;   // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
+      const TileInfo ti = tile_info(p, idx);
+      if (ti.skip) continue;
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const int row = ti.m0 + q * 32 + lane;
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.bn_alloc);
+      for (int c = 0; c < p.bn / 16; ++c) {
+        const int n = ti.n0 + c * 16;
+        if (n >= p.N) break;
+        uint32_t r[16];
+        tmem_ld16(t_row + (uint32_t)(c * 16), r);
+        tmem_wait_ld();
+        if (row < p.M) epilogue_store<T>(p, ti.g, row, n, r);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
+  }
+}
+
+}  // namespace gptl

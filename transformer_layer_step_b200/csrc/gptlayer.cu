@@ -1,0 +1,970 @@
+// gptlayer.cu — the C ABI of the layer-step library: argument validation,
+// workspace layout, TMA descriptor encoding, kernel launches.
+//
+// One GPT layer training step as the Megatron-LM pages describe it
+// ("Training GPT-2 with Megatron-LM" §4.1 and §6.2; "Megatron-LM 3D
+// parallelism" §1; "Megatron-LM overview" §2.2, §3.1, §4.2), with all
+// tensor-parallel shards on one B200.  Every step of the path runs in this
+// library's kernels; nothing falls back to the host.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "bw_kernels.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gptlayer_parts.h"
+
+using namespace gptl;
+
+namespace {
+
+#define GPTL_CK(x)                                 \
+  do {                                             \
+    if ((x) != cudaSuccess) {                      \
+      (void)cudaGetLastError();                    \
+      return GPTL_E_CUDA;                          \
+    }                                              \
+  } while (0)
+#define GPTL_TRY(x)                                \
+  do {                                             \
+    const int rc_ = (x);                           \
+    if (rc_ != GPTL_OK) return rc_;                \
+  } while (0)
+
+constexpr int kMaxDevices = 64;
+constexpr int kSmemLimit = 232448;   // 227 KB opt-in dynamic shared memory per block
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  int checked = 0, ok = 0, sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+int device_check(int *sms_out = nullptr) {
+  int dev = 0;
+  GPTL_CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return GPTL_E_ARCH;
+  DeviceInfo &d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, sms = 0;
+    GPTL_CK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    GPTL_CK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    d.ok = (major == 10);
+    d.sms = sms;
+    d.checked = 1;
+  }
+  if (!d.ok) return GPTL_E_ARCH;
+  if (sms_out) *sms_out = d.sms;
+  return GPTL_OK;
+}
+
+// ------------------------------------------------------------ TMA encoding
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+int mn_chunk_width(long long rows_tile) {
+  return rows_tile % 64 == 0 ? 64 : (rows_tile % 32 == 0 ? 32 : 16);
+}
+
+int encode_operand(CUtensorMap *map, const gptl_operand &o, gptl_dtype dt, int rows_tile, int w) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return GPTL_E_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)o.x_ext, (cuuint64_t)o.rows_ext, (cuuint64_t)o.g_ext};
+  cuuint64_t strides[2] = {(cuuint64_t)o.row_pitch * 2,
+                           (cuuint64_t)(o.g_ext > 1 ? o.g_pitch : o.rows_ext * o.row_pitch) * 2};
+  cuuint32_t box[3], es[3] = {1, 1, 1};
+  CUtensorMapSwizzle swz;
+  if (!o.mn_major) {
+    box[0] = 64;
+    box[1] = (cuuint32_t)rows_tile;
+    box[2] = 1;
+    swz = CU_TENSOR_MAP_SWIZZLE_128B;
+  } else {
+    box[0] = (cuuint32_t)w;
+    box[1] = (cuuint32_t)kBK;
+    box[2] = 1;
+    swz = w == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : (w == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  }
+  const CUresult r =
+      fn(map, dt == GPTL_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+         const_cast<void *>(o.ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GPTL_OK : GPTL_E_CUDA;
+}
+
+int check_operand(const gptl_operand &o) {
+  if (!o.ptr) return GPTL_E_NULL;
+  if (!aligned16(o.ptr)) return GPTL_E_ALIGN;
+  if (o.x_ext <= 0 || o.rows_ext <= 0 || o.g_ext <= 0 || o.row_pitch <= 0) return GPTL_E_SHAPE;
+  if (o.row_pitch % 8 || (o.g_ext > 1 && (o.g_pitch <= 0 || o.g_pitch % 8))) return GPTL_E_SHAPE;
+  if (o.x_mod < 1 || o.g_div < 1 || o.x_mul % 8 || o.x_off % 8 || o.x_mul < 0 || o.x_off < 0)
+    return GPTL_E_SHAPE;
+  if (o.x_ext >= (1ll << 32) || o.rows_ext >= (1ll << 32) || o.g_ext >= (1ll << 32))
+    return GPTL_E_SHAPE;
+  return GPTL_OK;
+}
+
+int pick_bn(const gptl_gemm_desc &d, int sms) {
+  if (d.causal == GPTL_CAUSAL_SKIP_UPPER) return d.N >= 128 ? 128 : d.N;
+  if (d.N <= 256) return d.N;
+  const long long m_tiles = (d.M + kBM - 1) / kBM;
+  long long best_cost = -1;
+  int best = 256;
+  for (int bn : {256, 128}) {
+    const long long tiles = m_tiles * ((d.N + bn - 1) / bn) * d.groups;
+    const long long waves = (tiles + sms - 1) / sms;
+    const long long cost = waves * (bn + 64);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+template <typename T>
+int launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  GPTL_CK(cudaGetDevice(&dev));
+  if (!attr_set[dev]) {
+    GPTL_CK(cudaFuncSetAttribute(gemm_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemLimit));
+    attr_set[dev] = true;
+  }
+  gemm_tc_kernel<T><<<grid, kGemmThreads, smem, stream>>>(p);
+  GPTL_CK(cudaGetLastError());
+  return GPTL_OK;
+}
+
+int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
+  int sms = 0;
+  GPTL_TRY(device_check(&sms));
+  if (dt != GPTL_FP16 && dt != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!d.out) return GPTL_E_NULL;
+  if (!aligned16(d.out)) return GPTL_E_ALIGN;
+  if (d.M <= 0 || d.N <= 0 || d.K <= 0 || d.groups <= 0 || d.k_shards <= 0) return GPTL_E_SHAPE;
+  if (d.K % 16 || d.N % 16 || d.causal < 0 || d.causal > 3 || d.o_mod < 1) return GPTL_E_SHAPE;
+  const int oal = d.out_f32 ? 4 : 8;
+  if (d.ldo % oal || d.o_str_mod % oal || d.o_str_div % oal || d.ldo < d.N) return GPTL_E_SHAPE;
+  if (d.bias && (!aligned16(d.bias) || d.bias_g_stride % 8)) return GPTL_E_ALIGN;
+  if (d.resid && (!aligned16(d.resid) || d.ld_resid % 8)) return GPTL_E_ALIGN;
+  if (d.act == GPTL_ACT_GELU && !d.out2) return GPTL_E_NULL;
+  if (d.act == GPTL_ACT_DGELU && !d.aux) return GPTL_E_NULL;
+  if ((d.out2 && !aligned16(d.out2)) || (d.aux && !aligned16(d.aux))) return GPTL_E_ALIGN;
+  if (d.act < 0 || d.act > 2) return GPTL_E_SHAPE;
+  GPTL_TRY(check_operand(d.a));
+  GPTL_TRY(check_operand(d.b));
+
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  const int bn = pick_bn(d, sms);
+  const int wa = d.a.mn_major ? mn_chunk_width(kBM) : 64;
+  const int wb = d.b.mn_major ? mn_chunk_width(bn) : 64;
+  GPTL_TRY(encode_operand(&p.map_a, d.a, dt, kBM, wa));
+  GPTL_TRY(encode_operand(&p.map_b, d.b, dt, bn, wb));
+  auto rule = [](const gptl_operand &o, int w) {
+    OperandRule r;
+    r.mn_major = o.mn_major;
+    r.w = w;
+    r.x_mod = o.x_mod;
+    r.x_mul = o.x_mul;
+    r.x_off = o.x_off;
+    r.g_div = o.g_div;
+    r.k_shard = o.k_shard;
+    return r;
+  };
+  p.ra = rule(d.a, wa);
+  p.rb = rule(d.b, wb);
+  p.M = d.M;
+  p.N = d.N;
+  p.K = d.K;
+  p.groups = d.groups;
+  p.k_shards = d.k_shards;
+  p.causal = d.causal;
+  p.bn = bn;
+  int bn_alloc = 32;
+  while (bn_alloc < bn) bn_alloc *= 2;
+  p.bn_alloc = bn_alloc;
+  p.tmem_cols = 2 * bn_alloc;
+  const int stage_bytes = (kBM + bn) * kBK * 2;
+  p.stages = (kSmemLimit - 2048) / stage_bytes;
+  if (p.stages > 8) p.stages = 8;
+  if (p.stages < 2) return GPTL_E_SHAPE;
+  const int smem = 1024 + p.stages * stage_bytes + 256;
+  const uint32_t fmt = dt == GPTL_BF16 ? 1u : 0u;
+  p.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)d.a.mn_major << 15) |
+            ((uint32_t)d.b.mn_major << 16) | ((uint32_t)(bn >> 3) << 17) |
+            ((uint32_t)(kBM >> 4) << 24);
+  p.m_tiles = (d.M + kBM - 1) / kBM;
+  p.n_tiles = (d.N + bn - 1) / bn;
+  p.total_tiles = (long long)p.m_tiles * p.n_tiles * d.groups;
+  p.out = d.out;
+  p.ldo = d.ldo;
+  p.o_mod = d.o_mod;
+  p.o_str_mod = d.o_str_mod;
+  p.o_str_div = d.o_str_div;
+  p.out_f32 = d.out_f32;
+  p.bias = d.out_f32 ? nullptr : d.bias;
+  p.bias_g_stride = d.bias_g_stride;
+  p.resid = d.out_f32 ? nullptr : d.resid;
+  p.ld_resid = d.ld_resid;
+  p.aux = d.aux;
+  p.out2 = d.out2;
+  p.act = d.out_f32 ? 0 : d.act;
+  const int grid = (int)(p.total_tiles < sms ? p.total_tiles : sms);
+  if (dt == GPTL_FP16) return launch_gemm_t<__half>(p, grid, smem, stream);
+  return launch_gemm_t<__nv_bfloat16>(p, grid, smem, stream);
+}
+
+// ------------------------------------------------------------- LayerNorm
+bool ln_split(int h, int *tpr, int *vpt) {
+  if (h <= 0 || h % 8) return false;
+  const int v = h / 8;
+  for (int limit : {5, 8})
+    for (int t : {16, 32, 64, 128, 256})
+      if (v % t == 0 && v / t >= 1 && v / t <= limit) {
+        *tpr = t;
+        *vpt = v / t;
+        return true;
+      }
+  return false;
+}
+
+template <typename T, int TPR, int VPT>
+void ln_fwd_launch(int rows, int h, const void *x, const void *g, const void *b, float eps,
+                   void *y, float *mu, float *rstd, cudaStream_t st) {
+  constexpr int RPB = 256 / TPR;
+  ln_fwd_kernel<T, TPR, VPT><<<(rows + RPB - 1) / RPB, 256, 0, st>>>(
+      (const T *)x, (const T *)g, (const T *)b, (T *)y, mu, rstd, rows, h, eps);
+}
+
+template <typename T, int TPR, int VPT>
+int ln_bwd_launch(int rows, int h, const void *gy, const void *x, const float *mu,
+                  const float *rstd, const void *g, const void *resid, void *dx, float *part,
+                  int nblocks, int want_sum, cudaStream_t st) {
+  constexpr int RPB = 256 / TPR;
+  const int smem = RPB * h * (int)sizeof(float);
+  if (smem > 48 * 1024)
+    GPTL_CK(cudaFuncSetAttribute(ln_bwd_kernel<T, TPR, VPT>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  ln_bwd_kernel<T, TPR, VPT><<<nblocks, 256, smem, st>>>((const T *)gy, (const T *)x, mu, rstd,
+                                                         (const T *)g, (const T *)resid, (T *)dx,
+                                                         part, rows, h, want_sum);
+  return GPTL_OK;
+}
+
+// Calls f.template operator()<TPR, VPT>() for the runtime split.
+template <typename F>
+bool ln_dispatch(int tpr, int vpt, F &&f) {
+#define GPTL_LN_CASE(TP, VP)                 \
+  if (tpr == TP && vpt == VP) {              \
+    f.template operator()<TP, VP>();         \
+    return true;                             \
+  }
+#define GPTL_LN_ROW(TP) \
+  GPTL_LN_CASE(TP, 1) GPTL_LN_CASE(TP, 2) GPTL_LN_CASE(TP, 3) GPTL_LN_CASE(TP, 4) \
+  GPTL_LN_CASE(TP, 5) GPTL_LN_CASE(TP, 6) GPTL_LN_CASE(TP, 7) GPTL_LN_CASE(TP, 8)
+  GPTL_LN_ROW(16) GPTL_LN_ROW(32) GPTL_LN_ROW(64) GPTL_LN_ROW(128) GPTL_LN_ROW(256)
+#undef GPTL_LN_ROW
+#undef GPTL_LN_CASE
+  return false;
+}
+
+int ln_bwd_blocks(int rows, int h, int sms) {
+  int tpr = 0, vpt = 0;
+  if (!ln_split(h, &tpr, &vpt)) return 0;
+  const int rpb = 256 / tpr;
+  int nb = (rows + rpb - 1) / rpb;
+  if (nb > 2 * sms) nb = 2 * sms;
+  if (nb > 512) nb = 512;
+  return nb;
+}
+
+int run_ln_fwd(int rows, int h, gptl_dtype dt, const void *x, const void *g, const void *b,
+               float eps, void *y, float *mu, float *rstd, cudaStream_t st) {
+  int tpr = 0, vpt = 0;
+  if (!ln_split(h, &tpr, &vpt) || rows <= 0) return GPTL_E_SHAPE;
+  const bool ok = ln_dispatch(tpr, vpt, [&]<int TP, int VP>() {
+    if (dt == GPTL_FP16)
+      ln_fwd_launch<__half, TP, VP>(rows, h, x, g, b, eps, y, mu, rstd, st);
+    else
+      ln_fwd_launch<__nv_bfloat16, TP, VP>(rows, h, x, g, b, eps, y, mu, rstd, st);
+  });
+  if (!ok) return GPTL_E_SHAPE;
+  GPTL_CK(cudaGetLastError());
+  return GPTL_OK;
+}
+
+int run_ln_bwd(int rows, int h, gptl_dtype dt, const void *gy, const void *x, const float *mu,
+               const float *rstd, const void *g, const void *resid, void *dx, float *dg, float *db,
+               float *dx_sum, float *part, cudaStream_t st) {
+  int sms = 0;
+  GPTL_TRY(device_check(&sms));
+  int tpr = 0, vpt = 0;
+  if (!ln_split(h, &tpr, &vpt) || rows <= 0) return GPTL_E_SHAPE;
+  const int nb = ln_bwd_blocks(rows, h, sms);
+  const int want = dx_sum ? 1 : 0;
+  int rc = GPTL_OK;
+  const bool ok = ln_dispatch(tpr, vpt, [&]<int TP, int VP>() {
+    if (dt == GPTL_FP16)
+      rc = ln_bwd_launch<__half, TP, VP>(rows, h, gy, x, mu, rstd, g, resid, dx, part, nb, want, st);
+    else
+      rc = ln_bwd_launch<__nv_bfloat16, TP, VP>(rows, h, gy, x, mu, rstd, g, resid, dx, part, nb,
+                                                want, st);
+  });
+  if (!ok) return GPTL_E_SHAPE;
+  GPTL_TRY(rc);
+  GPTL_CK(cudaGetLastError());
+  dim3 rg((h + 255) / 256, 2 + want);
+  reduce_parts_kernel<<<rg, 256, 0, st>>>(part, nb, h, dg, db, dx_sum);
+  GPTL_CK(cudaGetLastError());
+  return GPTL_OK;
+}
+
+// ------------------------------------------------------------- softmax
+int softmax_nv(int s) {
+  const int nv = (s + 255) / 256;
+  return nv <= 1 ? 1 : (nv <= 2 ? 2 : (nv <= 4 ? 4 : 8));
+}
+
+int run_softmax_fwd(long long blocks, int s, gptl_dtype dt, float scale, void *sc,
+                    cudaStream_t st) {
+  if (blocks <= 0 || s <= 0 || s % 16 || s > 2048) return GPTL_E_SHAPE;
+  const long long rows = blocks * s;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  const int nv = softmax_nv(s);
+#define GPTL_SMF(T, NV)                                                                   \
+  if (nv == NV) softmax_fwd_kernel<T, NV><<<grid, 256, 0, st>>>((T *)sc, rows, s, scale);
+  if (dt == GPTL_FP16) {
+    GPTL_SMF(__half, 1) GPTL_SMF(__half, 2) GPTL_SMF(__half, 4) GPTL_SMF(__half, 8)
+  } else {
+    GPTL_SMF(__nv_bfloat16, 1) GPTL_SMF(__nv_bfloat16, 2) GPTL_SMF(__nv_bfloat16, 4)
+    GPTL_SMF(__nv_bfloat16, 8)
+  }
+#undef GPTL_SMF
+  GPTL_CK(cudaGetLastError());
+  return GPTL_OK;
+}
+
+int run_softmax_bwd(long long blocks, int s, gptl_dtype dt, float scale, const void *pr, void *dp,
+                    cudaStream_t st) {
+  if (blocks <= 0 || s <= 0 || s % 16 || s > 2048) return GPTL_E_SHAPE;
+  const long long rows = blocks * s;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  const int nv = softmax_nv(s);
+#define GPTL_SMB(T, NV)                                                                        \
+  if (nv == NV)                                                                                \
+    softmax_bwd_kernel<T, NV><<<grid, 256, 0, st>>>((const T *)pr, (T *)dp, rows, s, scale);
+  if (dt == GPTL_FP16) {
+    GPTL_SMB(__half, 1) GPTL_SMB(__half, 2) GPTL_SMB(__half, 4) GPTL_SMB(__half, 8)
+  } else {
+    GPTL_SMB(__nv_bfloat16, 1) GPTL_SMB(__nv_bfloat16, 2) GPTL_SMB(__nv_bfloat16, 4)
+    GPTL_SMB(__nv_bfloat16, 8)
+  }
+#undef GPTL_SMB
+  GPTL_CK(cudaGetLastError());
+  return GPTL_OK;
+}
+
+// ------------------------------------------------------------- col sums
+constexpr int kColsumMaxSplit = 64;
+
+int run_colsum(int rows, int n, int groups, long long ld, long long gstride, gptl_dtype dt,
+               const void *a, float *out, float *part, cudaStream_t st) {
+  int sms = 0;
+  GPTL_TRY(device_check(&sms));
+  if (rows <= 0 || n <= 0 || groups <= 0 || n % 8 || ld % 8 || (groups > 1 && gstride % 8))
+    return GPTL_E_SHAPE;
+  const int strips = (n + 255) / 256;
+  int split = (2 * sms + strips * groups - 1) / (strips * groups);
+  if (split < 1) split = 1;
+  if (split > kColsumMaxSplit) split = kColsumMaxSplit;
+  if (split > (rows + 7) / 8) split = (rows + 7) / 8;
+  dim3 grid(strips, split, groups), block(32, 8);
+  if (dt == GPTL_FP16)
+    colsum_kernel<__half><<<grid, block, 0, st>>>((const __half *)a, rows, n, ld, gstride, part,
+                                                  groups);
+  else
+    colsum_kernel<__nv_bfloat16><<<grid, block, 0, st>>>((const __nv_bfloat16 *)a, rows, n, ld,
+                                                         gstride, part, groups);
+  GPTL_CK(cudaGetLastError());
+  const int width = n * groups;
+  reduce_parts_kernel<<<dim3((width + 255) / 256, 1), 256, 0, st>>>(part, split, width, out,
+                                                                    nullptr, nullptr);
+  GPTL_CK(cudaGetLastError());
+  return GPTL_OK;
+}
+
+// ------------------------------------------------------------- the layer
+struct Dims {
+  int b, s, h, a, f, t, d, hs, as, fs;
+  long long T;
+  gptl_dtype dt;
+  float eps;
+};
+
+int check_shape(const gptl_shape *sh, Dims *D) {
+  if (!sh) return GPTL_E_NULL;
+  if (sh->dtype != GPTL_FP16 && sh->dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  const int b = sh->batch, s = sh->seq, h = sh->hidden, a = sh->heads, f = sh->ffn, t = sh->tp;
+  if (b <= 0 || s <= 0 || h <= 0 || a <= 0 || f <= 0 || t <= 0) return GPTL_E_SHAPE;
+  if (h % a || a % t || f % t) return GPTL_E_SHAPE;
+  const int d = h / a;
+  if (d % 16 || d > 256 || h % 64 || (f / t) % 64 || s % 16 || s > 2048) return GPTL_E_SHAPE;
+  if ((long long)b * s >= (1ll << 31)) return GPTL_E_SHAPE;
+  if (!(sh->ln_eps > 0.f)) return GPTL_E_SHAPE;
+  int tpr, vpt;
+  if (!ln_split(h, &tpr, &vpt)) return GPTL_E_SHAPE;
+  D->b = b; D->s = s; D->h = h; D->a = a; D->f = f; D->t = t; D->d = d;
+  D->hs = h / t; D->as = a / t; D->fs = f / t;
+  D->T = (long long)b * s;
+  D->dt = sh->dtype;
+  D->eps = sh->ln_eps;
+  return GPTL_OK;
+}
+
+struct Ws {
+  // saved (fwd -> bwd)
+  size_t mu1, rstd1, mu2, rstd2, l1, c, p, o, hid, l2, z, act, saved;
+  // scratch (bwd)
+  size_t dz, dl2, dhid, dO, dp, dc, dl1, part, scratch;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Ws ws_layout(const Dims &D) {
+  Ws w;
+  const size_t e = 2, T = (size_t)D.T, h = D.h, f = D.f;
+  const size_t pe = (size_t)D.b * D.a * D.s * D.s;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += up256(bytes);
+    return o;
+  };
+  w.mu1 = take(T * 4); w.rstd1 = take(T * 4); w.mu2 = take(T * 4); w.rstd2 = take(T * 4);
+  w.l1 = take(T * h * e); w.c = take(3 * T * h * e); w.p = take(pe * e); w.o = take(T * h * e);
+  w.hid = take(T * h * e); w.l2 = take(T * h * e); w.z = take(T * f * e); w.act = take(T * f * e);
+  w.saved = off;
+  off = 0;
+  w.dz = take(T * f * e); w.dl2 = take(T * h * e); w.dhid = take(T * h * e); w.dO = take(T * h * e);
+  w.dp = take(pe * e); w.dc = take(3 * T * h * e); w.dl1 = take(T * h * e);
+  size_t part = 3 * 512 * h;
+  const size_t widest = f > 3 * h ? f : 3 * h;
+  if (kColsumMaxSplit * widest > part) part = kColsumMaxSplit * widest;
+  w.part = take(part * 4);
+  w.scratch = off;
+  return w;
+}
+
+template <typename P> P *at(void *base, size_t off) {
+  return reinterpret_cast<P *>(static_cast<char *>(base) + off);
+}
+template <typename P> const P *at(const void *base, size_t off) {
+  return reinterpret_cast<const P *>(static_cast<const char *>(base) + off);
+}
+
+constexpr int kNoGroup = 1 << 30;
+
+gptl_operand view(const void *ptr, long long x_ext, long long rows, long long g_ext,
+                  long long row_pitch, long long g_pitch, int mn) {
+  gptl_operand o;
+  o.ptr = ptr;
+  o.x_ext = x_ext;
+  o.rows_ext = rows;
+  o.g_ext = g_ext;
+  o.row_pitch = row_pitch;
+  o.g_pitch = g_pitch;
+  o.mn_major = mn;
+  o.x_mod = 1;
+  o.x_mul = 0;
+  o.x_off = 0;
+  o.g_div = g_ext > 1 ? 1 : kNoGroup;
+  o.k_shard = 0;
+  return o;
+}
+
+gptl_gemm_desc gemm(int M, int N, int K, int groups, const gptl_operand &a, const gptl_operand &b,
+                    void *out, long long ldo, long long o_str_div) {
+  gptl_gemm_desc d;
+  memset(&d, 0, sizeof(d));
+  d.M = M; d.N = N; d.K = K; d.groups = groups; d.k_shards = 1;
+  d.a = a; d.b = b;
+  d.out = out; d.ldo = ldo; d.o_mod = 1; d.o_str_div = o_str_div;
+  return d;
+}
+
+int validate_weights(const gptl_weights *w) {
+  if (!w) return GPTL_E_NULL;
+  const void *ps[12] = {w->ln1_g, w->ln1_b, w->w_qkv, w->b_qkv, w->w_o, w->b_o,
+                        w->ln2_g, w->ln2_b, w->w_1, w->b_1, w->w_2, w->b_2};
+  for (const void *p : ps) {
+    if (!p) return GPTL_E_NULL;
+    if (!aligned16(p)) return GPTL_E_ALIGN;
+  }
+  return GPTL_OK;
+}
+
+int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void *saved,
+              cudaStream_t st) {
+  const Ws w = ws_layout(D);
+  const gptl_dtype dt = D.dt;
+  const int T = (int)D.T, h = D.h, t = D.t, s = D.s, d = D.d, hs = D.hs, as = D.as, fs = D.fs;
+  const int G = D.b * D.a;                      // attention groups: (shard, batch, head)
+  void *l1 = at<void>(saved, w.l1), *c = at<void>(saved, w.c), *pb = at<void>(saved, w.p);
+  void *o = at<void>(saved, w.o), *hid = at<void>(saved, w.hid), *l2 = at<void>(saved, w.l2);
+  void *z = at<void>(saved, w.z), *act = at<void>(saved, w.act);
+  float *mu1 = at<float>(saved, w.mu1), *rs1 = at<float>(saved, w.rstd1);
+  float *mu2 = at<float>(saved, w.mu2), *rs2 = at<float>(saved, w.rstd2);
+  const float attn_scale = 1.0f / sqrtf((float)d);
+
+  // LN1
+  GPTL_TRY(run_ln_fwd(T, h, dt, x, W->ln1_g, W->ln1_b, D.eps, l1, mu1, rs1, st));
+  // QKV column split: C_i = L1 W_qkv,i^T + b_qkv,i
+  {
+    gptl_gemm_desc g = gemm(T, 3 * hs, h, t, view(l1, h, T, 1, h, 0, 0),
+                            view(W->w_qkv, h, 3 * hs, t, h, (long long)3 * hs * h, 0), c, 3 * hs,
+                            (long long)T * 3 * hs);
+    g.bias = W->b_qkv;
+    g.bias_g_stride = 3 * hs;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // scores S = Q K^T per (shard, batch, head), lower-triangle tiles only
+  {
+    gptl_operand q = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 0);
+    q.x_mod = as; q.x_mul = d; q.g_div = as;
+    gptl_operand k = q;
+    k.x_off = hs;
+    gptl_gemm_desc g = gemm(s, s, d, G, q, k, pb, s, (long long)s * s);
+    g.causal = GPTL_CAUSAL_SKIP_UPPER;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // fused scale-mask-softmax, in place
+  GPTL_TRY(run_softmax_fwd(G, s, dt, attn_scale, pb, st));
+  // O = P V (K range limited to the lower triangle)
+  {
+    gptl_operand pa = view(pb, s, s, G, s, (long long)s * s, 0);
+    gptl_operand v = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 1);
+    v.x_mod = as; v.x_mul = d; v.x_off = 2 * hs; v.g_div = as;
+    gptl_gemm_desc g = gemm(s, d, s, G, pa, v, o, hs, (long long)s * hs);
+    g.o_mod = as;
+    g.o_str_mod = d;
+    g.causal = GPTL_CAUSAL_K_BELOW;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // out-projection, row split: H = X + sum_i O_i W_o,i^T + b_o
+  {
+    gptl_operand a = view(o, hs, T, t, hs, (long long)T * hs, 0);
+    a.g_div = kNoGroup; a.k_shard = 1;
+    gptl_operand b = view(W->w_o, hs, h, t, hs, (long long)h * hs, 0);
+    b.g_div = kNoGroup; b.k_shard = 1;
+    gptl_gemm_desc g = gemm(T, h, hs, 1, a, b, hid, h, 0);
+    g.k_shards = t;
+    g.bias = W->b_o;
+    g.resid = x;
+    g.ld_resid = h;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // LN2
+  GPTL_TRY(run_ln_fwd(T, h, dt, hid, W->ln2_g, W->ln2_b, D.eps, l2, mu2, rs2, st));
+  // FFN1 column split with fused bias + GeLU: Z_i, A_i = gelu(Z_i)
+  {
+    gptl_gemm_desc g = gemm(T, fs, h, t, view(l2, h, T, 1, h, 0, 0),
+                            view(W->w_1, h, fs, t, h, (long long)fs * h, 0), z, fs,
+                            (long long)T * fs);
+    g.bias = W->b_1;
+    g.bias_g_stride = fs;
+    g.act = GPTL_ACT_GELU;
+    g.out2 = act;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // FFN2 row split: Out = H + sum_i A_i W_2,i^T + b_2
+  {
+    gptl_operand a = view(act, fs, T, t, fs, (long long)T * fs, 0);
+    a.g_div = kNoGroup; a.k_shard = 1;
+    gptl_operand b = view(W->w_2, fs, h, t, fs, (long long)h * fs, 0);
+    b.g_div = kNoGroup; b.k_shard = 1;
+    gptl_gemm_desc g = gemm(T, h, fs, 1, a, b, y, h, 0);
+    g.k_shards = t;
+    g.bias = W->b_2;
+    g.resid = hid;
+    g.ld_resid = h;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  return GPTL_OK;
+}
+
+int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *saved,
+              const void *dy, void *dx, const gptl_grads *gr, void *scratch, cudaStream_t st) {
+  const Ws w = ws_layout(D);
+  const gptl_dtype dt = D.dt;
+  const int T = (int)D.T, h = D.h, t = D.t, s = D.s, d = D.d, hs = D.hs, as = D.as, fs = D.fs;
+  const int G = D.b * D.a;
+  const void *l1 = at<void>(saved, w.l1), *c = at<void>(saved, w.c), *pb = at<void>(saved, w.p);
+  const void *o = at<void>(saved, w.o), *hid = at<void>(saved, w.hid);
+  const void *l2 = at<void>(saved, w.l2), *z = at<void>(saved, w.z), *act = at<void>(saved, w.act);
+  const float *mu1 = at<float>(saved, w.mu1), *rs1 = at<float>(saved, w.rstd1);
+  const float *mu2 = at<float>(saved, w.mu2), *rs2 = at<float>(saved, w.rstd2);
+  void *dz = at<void>(scratch, w.dz), *dl2 = at<void>(scratch, w.dl2);
+  void *dhid = at<void>(scratch, w.dhid), *dO = at<void>(scratch, w.dO);
+  void *dp = at<void>(scratch, w.dp), *dc = at<void>(scratch, w.dc), *dl1 = at<void>(scratch, w.dl1);
+  float *part = at<float>(scratch, w.part);
+  const float attn_scale = 1.0f / sqrtf((float)d);
+
+  // ---- FFN2 (row split)
+  GPTL_TRY(run_colsum(T, h, 1, h, 0, dt, dy, gr->b_2, part, st));
+  {  // dW2_i = dOut^T A_i   [t][h][f/t] fp32
+    gptl_gemm_desc g = gemm(h, fs, T, t, view(dy, h, T, 1, h, 0, 1),
+                            view(act, fs, T, t, fs, (long long)T * fs, 1), gr->w_2, fs,
+                            (long long)h * fs);
+    g.out_f32 = 1;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  {  // dZ_i = (dOut W2_i) * gelu'(Z_i)
+    gptl_gemm_desc g = gemm(T, fs, h, t, view(dy, h, T, 1, h, 0, 0),
+                            view(W->w_2, fs, h, t, fs, (long long)h * fs, 1), dz, fs,
+                            (long long)T * fs);
+    g.act = GPTL_ACT_DGELU;
+    g.aux = z;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // ---- FFN1 (column split)
+  GPTL_TRY(run_colsum(T, fs, t, fs, (long long)T * fs, dt, dz, gr->b_1, part, st));
+  {  // dW1_i = dZ_i^T L2   [t][f/t][h]
+    gptl_gemm_desc g = gemm(fs, h, T, t, view(dz, fs, T, t, fs, (long long)T * fs, 1),
+                            view(l2, h, T, 1, h, 0, 1), gr->w_1, h, (long long)fs * h);
+    g.out_f32 = 1;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  {  // dL2 = sum_i dZ_i W1_i  (shard sum in the K loop)
+    gptl_operand a = view(dz, fs, T, t, fs, (long long)T * fs, 0);
+    a.g_div = kNoGroup; a.k_shard = 1;
+    gptl_operand b = view(W->w_1, h, fs, t, h, (long long)fs * h, 1);
+    b.g_div = kNoGroup; b.k_shard = 1;
+    gptl_gemm_desc g = gemm(T, h, fs, 1, a, b, dl2, h, 0);
+    g.k_shards = t;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // ---- LN2 backward + residual: dH = dOut + LNbwd(dL2); also db_o = sum dH
+  GPTL_TRY(run_ln_bwd(T, h, dt, dl2, hid, mu2, rs2, W->ln2_g, dy, dhid, gr->ln2_g, gr->ln2_b,
+                      gr->b_o, part, st));
+  // ---- out-projection (row split)
+  {  // dWo_i = dH^T O_i   [t][h][h/t]
+    gptl_gemm_desc g = gemm(h, hs, T, t, view(dhid, h, T, 1, h, 0, 1),
+                            view(o, hs, T, t, hs, (long long)T * hs, 1), gr->w_o, hs,
+                            (long long)h * hs);
+    g.out_f32 = 1;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  {  // dO_i = dH Wo_i   [t][T][h/t]
+    gptl_gemm_desc g = gemm(T, hs, h, t, view(dhid, h, T, 1, h, 0, 0),
+                            view(W->w_o, hs, h, t, hs, (long long)h * hs, 1), dO, hs,
+                            (long long)T * hs);
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // ---- attention backward
+  gptl_operand dOv = view(dO, hs, s, (long long)t * D.b, hs, (long long)s * hs, 0);
+  dOv.x_mod = as; dOv.x_mul = d; dOv.g_div = as;
+  gptl_operand cv = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 0);
+  cv.x_mod = as; cv.x_mul = d; cv.g_div = as;
+  {  // dP = dO V^T (lower-triangle tiles)
+    gptl_operand v = cv;
+    v.x_off = 2 * hs;
+    gptl_gemm_desc g = gemm(s, s, d, G, dOv, v, dp, s, (long long)s * s);
+    g.causal = GPTL_CAUSAL_SKIP_UPPER;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  {  // dV = P^T dO  -> V columns of dC
+    gptl_operand a = view(pb, s, s, G, s, (long long)s * s, 1);
+    gptl_operand b = dOv;
+    b.mn_major = 1;
+    gptl_gemm_desc g = gemm(s, d, s, G, a, b, at<void>(dc, (size_t)2 * hs * 2), 3 * hs,
+                            (long long)s * 3 * hs);
+    g.o_mod = as;
+    g.o_str_mod = d;
+    g.causal = GPTL_CAUSAL_K_FROM;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // dS = P (dP - rowsum(P dP)) / sqrt(d), in place over dP
+  GPTL_TRY(run_softmax_bwd(G, s, dt, attn_scale, pb, dp, st));
+  {  // dQ = dS K  -> Q columns of dC
+    gptl_operand a = view(dp, s, s, G, s, (long long)s * s, 0);
+    gptl_operand b = cv;
+    b.mn_major = 1;
+    b.x_off = hs;
+    gptl_gemm_desc g = gemm(s, d, s, G, a, b, dc, 3 * hs, (long long)s * 3 * hs);
+    g.o_mod = as;
+    g.o_str_mod = d;
+    g.causal = GPTL_CAUSAL_K_BELOW;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  {  // dK = dS^T Q  -> K columns of dC
+    gptl_operand a = view(dp, s, s, G, s, (long long)s * s, 1);
+    gptl_operand b = cv;
+    b.mn_major = 1;
+    gptl_gemm_desc g = gemm(s, d, s, G, a, b, at<void>(dc, (size_t)hs * 2), 3 * hs,
+                            (long long)s * 3 * hs);
+    g.o_mod = as;
+    g.o_str_mod = d;
+    g.causal = GPTL_CAUSAL_K_FROM;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // ---- QKV (column split)
+  GPTL_TRY(run_colsum(T, 3 * hs, t, 3 * hs, (long long)T * 3 * hs, dt, dc, gr->b_qkv, part, st));
+  {  // dWqkv_i = dC_i^T L1   [t][3h/t][h]
+    gptl_gemm_desc g = gemm(3 * hs, h, T, t, view(dc, 3 * hs, T, t, 3 * hs, (long long)T * 3 * hs, 1),
+                            view(l1, h, T, 1, h, 0, 1), gr->w_qkv, h, (long long)3 * hs * h);
+    g.out_f32 = 1;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  {  // dL1 = sum_i dC_i Wqkv_i
+    gptl_operand a = view(dc, 3 * hs, T, t, 3 * hs, (long long)T * 3 * hs, 0);
+    a.g_div = kNoGroup; a.k_shard = 1;
+    gptl_operand b = view(W->w_qkv, h, 3 * hs, t, h, (long long)3 * hs * h, 1);
+    b.g_div = kNoGroup; b.k_shard = 1;
+    gptl_gemm_desc g = gemm(T, h, 3 * hs, 1, a, b, dl1, h, 0);
+    g.k_shards = t;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  // ---- LN1 backward + residual: dX = dH + LNbwd(dL1)
+  GPTL_TRY(run_ln_bwd(T, h, dt, dl1, x, mu1, rs1, W->ln1_g, dhid, dx, gr->ln1_g, gr->ln1_b,
+                      nullptr, part, st));
+  return GPTL_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char *gptl_strerror(int code) {
+  switch (code) {
+    case GPTL_OK: return "ok";
+    case GPTL_E_NULL: return "a required pointer is NULL";
+    case GPTL_E_SHAPE: return "unsupported or inconsistent sizes";
+    case GPTL_E_ALIGN: return "a pointer or pitch is not 16-byte aligned";
+    case GPTL_E_DTYPE: return "dtype must be GPTL_FP16 or GPTL_BF16";
+    case GPTL_E_ARCH: return "the current device is not compute capability 10.x (sm_100a)";
+    case GPTL_E_CUDA: return "a CUDA call or kernel launch failed";
+    case GPTL_E_DEVICE: return "the device error word is set";
+    case GPTL_E_ARG: return "invalid scalar argument";
+    default: return "unknown error";
+  }
+}
+
+int gptl_read_device_error(int *word, int clear) {
+  if (!word) return GPTL_E_NULL;
+  GPTL_CK(cudaDeviceSynchronize());
+  GPTL_CK(cudaMemcpyFromSymbol(word, g_device_error, sizeof(int)));
+  if (clear) {
+    const int zero = 0;
+    GPTL_CK(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)));
+  }
+  return GPTL_OK;
+}
+
+int gpt_layer_workspace_bytes(const gptl_shape *shape, size_t *saved_bytes, size_t *scratch_bytes) {
+  Dims D;
+  GPTL_TRY(check_shape(shape, &D));
+  if (!saved_bytes || !scratch_bytes) return GPTL_E_NULL;
+  const Ws w = ws_layout(D);
+  *saved_bytes = w.saved;
+  *scratch_bytes = w.scratch;
+  return GPTL_OK;
+}
+
+int gpt_layer_param_layout(const gptl_shape *shape, size_t offsets[12], size_t *n_params) {
+  Dims D;
+  GPTL_TRY(check_shape(shape, &D));
+  if (!offsets || !n_params) return GPTL_E_NULL;
+  const size_t h = D.h, f = D.f;
+  const size_t sizes[12] = {h, h, 3 * h * h, 3 * h, h * h, h, h, h, f * h, f, h * f, h};
+  size_t off = 0;
+  for (int i = 0; i < 12; ++i) {
+    offsets[i] = off;
+    off += (sizes[i] + 63) / 64 * 64;
+  }
+  *n_params = off;
+  return GPTL_OK;
+}
+
+int gpt_layer_fwd(const gptl_shape *shape, const gptl_weights *w, const void *x, void *y,
+                  void *saved, void *scratch, gptl_stream_t stream) {
+  (void)scratch;
+  Dims D;
+  GPTL_TRY(check_shape(shape, &D));
+  GPTL_TRY(validate_weights(w));
+  if (!x || !y || !saved) return GPTL_E_NULL;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(saved)) return GPTL_E_ALIGN;
+  GPTL_TRY(device_check());
+  return layer_fwd(D, w, x, y, saved, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gpt_layer_bwd(const gptl_shape *shape, const gptl_weights *w, const void *x, const void *saved,
+                  const void *dy, void *dx, const gptl_grads *g, void *scratch,
+                  gptl_stream_t stream) {
+  Dims D;
+  GPTL_TRY(check_shape(shape, &D));
+  GPTL_TRY(validate_weights(w));
+  if (!x || !saved || !dy || !dx || !g || !scratch) return GPTL_E_NULL;
+  if (!aligned16(x) || !aligned16(saved) || !aligned16(dy) || !aligned16(dx) || !aligned16(scratch))
+    return GPTL_E_ALIGN;
+  const float *gp[12] = {g->ln1_g, g->ln1_b, g->w_qkv, g->b_qkv, g->w_o, g->b_o,
+                         g->ln2_g, g->ln2_b, g->w_1, g->b_1, g->w_2, g->b_2};
+  for (const float *p : gp) {
+    if (!p) return GPTL_E_NULL;
+    if (!aligned16(p)) return GPTL_E_ALIGN;
+  }
+  GPTL_TRY(device_check());
+  return layer_bwd(D, w, x, saved, dy, dx, g, scratch, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gptl_check_overflow(size_t n, const float *grad, gptl_scaler_state *st, gptl_stream_t stream) {
+  int sms = 0;
+  if (!grad || !st) return GPTL_E_NULL;
+  if (!aligned16(grad) || (reinterpret_cast<uintptr_t>(st) & 3u)) return GPTL_E_ALIGN;
+  if (n == 0 || n % 4) return GPTL_E_ARG;
+  GPTL_TRY(device_check(&sms));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  GPTL_CK(cudaMemsetAsync(&st->found_inf, 0, sizeof(int), s));
+  const long long n4 = (long long)(n / 4);
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > 4 * sms) blocks = 4 * sms;
+  overflow_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4 *>(grad), n4,
+                                                   &st->found_inf);
+  GPTL_CK(cudaGetLastError());
+  return GPTL_OK;
+}
+
+int adam_step_fp32_master(size_t n_params, float *master, float *m, float *v, const float *grad,
+                          void *w16, gptl_dtype dtype, float lr, float beta1, float beta2, float eps,
+                          float weight_decay, gptl_scaler_state *st, gptl_stream_t stream) {
+  if (!master || !m || !v || !grad || !w16 || !st) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(grad) || !aligned16(w16))
+    return GPTL_E_ALIGN;
+  if (n_params == 0 || n_params % 4 || !(lr >= 0.f) || !(beta1 >= 0.f && beta1 < 1.f) ||
+      !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f) || !(weight_decay >= 0.f))
+    return GPTL_E_ARG;
+  int sms = 0;
+  GPTL_TRY(device_check(&sms));
+  GPTL_TRY(gptl_check_overflow(n_params, grad, st, stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long n4 = (long long)(n_params / 4);
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > 8 * sms) blocks = 8 * sms;
+  AdamArgs a{lr, beta1, beta2, eps, weight_decay};
+  if (dtype == GPTL_FP16)
+    adam_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(
+        reinterpret_cast<float4 *>(master), reinterpret_cast<float4 *>(m),
+        reinterpret_cast<float4 *>(v), reinterpret_cast<const float4 *>(grad),
+        static_cast<__half *>(w16), n4, a, st);
+  else
+    adam_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+        reinterpret_cast<float4 *>(master), reinterpret_cast<float4 *>(m),
+        reinterpret_cast<float4 *>(v), reinterpret_cast<const float4 *>(grad),
+        static_cast<__nv_bfloat16 *>(w16), n4, a, st);
+  GPTL_CK(cudaGetLastError());
+  return GPTL_OK;
+}
+
+int loss_scale_update(gptl_scaler_state *st, int growth_interval, float growth_factor,
+                      float backoff_factor, float min_scale, gptl_stream_t stream) {
+  if (!st) return GPTL_E_NULL;
+  if (growth_interval < 1 || !(growth_factor >= 1.f) || !(backoff_factor > 0.f && backoff_factor <= 1.f) ||
+      !(min_scale > 0.f))
+    return GPTL_E_ARG;
+  GPTL_TRY(device_check());
+  scale_update_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      st, growth_interval, growth_factor, backoff_factor, min_scale);
+  GPTL_CK(cudaGetLastError());
+  return GPTL_OK;
+}
+
+// ---------------------------------------------------------------- parts
+int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream) {
+  if (!d) return GPTL_E_NULL;
+  return run_gemm(*d, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gptl_layernorm_fwd(int rows, int h, gptl_dtype dtype, const void *x, const void *g,
+                       const void *b, float eps, void *y, float *mu, float *rstd,
+                       gptl_stream_t stream) {
+  if (!x || !g || !b || !y || !mu || !rstd) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(x) || !aligned16(g) || !aligned16(b) || !aligned16(y)) return GPTL_E_ALIGN;
+  if (!(eps > 0.f)) return GPTL_E_ARG;
+  GPTL_TRY(device_check());
+  return run_ln_fwd(rows, h, dtype, x, g, b, eps, y, mu, rstd, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t gptl_layernorm_bwd_scratch_bytes(int rows, int h) {
+  (void)rows;
+  return (size_t)3 * 512 * (size_t)(h > 0 ? h : 0) * sizeof(float);
+}
+
+int gptl_layernorm_bwd(int rows, int h, gptl_dtype dtype, const void *gy, const void *x,
+                       const float *mu, const float *rstd, const void *g, const void *resid,
+                       void *dx, float *dg, float *db, float *dx_sum, void *scratch,
+                       gptl_stream_t stream) {
+  if (!gy || !x || !mu || !rstd || !g || !resid || !dx || !dg || !db || !scratch) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(gy) || !aligned16(x) || !aligned16(g) || !aligned16(resid) || !aligned16(dx) ||
+      !aligned16(scratch))
+    return GPTL_E_ALIGN;
+  return run_ln_bwd(rows, h, dtype, gy, x, mu, rstd, g, resid, dx, dg, db, dx_sum,
+                    static_cast<float *>(scratch), reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gptl_softmax_fwd(long long blocks, int s, gptl_dtype dtype, float scale, void *scores,
+                     gptl_stream_t stream) {
+  if (!scores) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(scores)) return GPTL_E_ALIGN;
+  GPTL_TRY(device_check());
+  return run_softmax_fwd(blocks, s, dtype, scale, scores, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gptl_softmax_bwd(long long blocks, int s, gptl_dtype dtype, float scale, const void *prob,
+                     void *dprob, gptl_stream_t stream) {
+  if (!prob || !dprob) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(prob) || !aligned16(dprob)) return GPTL_E_ALIGN;
+  GPTL_TRY(device_check());
+  return run_softmax_bwd(blocks, s, dtype, scale, prob, dprob, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t gptl_colsum_scratch_bytes(int n, int groups) {
+  if (n <= 0 || groups <= 0) return 0;
+  return (size_t)kColsumMaxSplit * (size_t)n * (size_t)groups * sizeof(float);
+}
+
+int gptl_colsum(int rows, int n, int groups, long long ld, long long gstride, gptl_dtype dtype,
+                const void *a, float *out, void *scratch, gptl_stream_t stream) {
+  if (!a || !out || !scratch) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(a) || !aligned16(scratch)) return GPTL_E_ALIGN;
+  return run_colsum(rows, n, groups, ld, gstride, dtype, a, out, static_cast<float *>(scratch),
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

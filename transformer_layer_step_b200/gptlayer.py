@@ -1,0 +1,252 @@
+"""ctypes binding of libgptlayer.so (declared in include/gptlayer.h and
+include/gptlayer_parts.h).
+
+Argument marshalling only: every computation happens in the library's CUDA
+kernels.  Pointers are passed as integers (or objects with .data_ptr(), such
+as torch tensors); streams as the integer handle of a cudaStream_t.  A
+non-zero return code raises GptlError.  If the library has not been built the
+first call raises at once: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libgptlayer.so")
+INCLUDE = os.path.join(os.path.dirname(PKG), "include")
+
+FP16, BF16 = 0, 1
+ACT_NONE, ACT_GELU, ACT_DGELU = 0, 1, 2
+CAUSAL_NONE, CAUSAL_SKIP_UPPER, CAUSAL_K_BELOW, CAUSAL_K_FROM = 0, 1, 2, 3
+E_NULL, E_SHAPE, E_ALIGN, E_DTYPE, E_ARCH, E_CUDA, E_DEVICE, E_ARG = -1, -2, -3, -4, -5, -6, -7, -8
+DTYPES = {"fp16": FP16, "bf16": BF16}
+PARAM_NAMES = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
+               "ln2_g", "ln2_b", "w_1", "b_1", "w_2", "b_2")
+
+
+class GptlError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} ({code})")
+
+
+class Shape(C.Structure):
+    _fields_ = [("batch", C.c_int), ("seq", C.c_int), ("hidden", C.c_int), ("heads", C.c_int),
+                ("ffn", C.c_int), ("tp", C.c_int), ("dtype", C.c_int), ("ln_eps", C.c_float)]
+
+
+class Weights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in PARAM_NAMES]
+
+
+class Grads(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in PARAM_NAMES]
+
+
+class ScalerState(C.Structure):
+    _fields_ = [("scale", C.c_float), ("growth_tracker", C.c_int), ("found_inf", C.c_int),
+                ("step", C.c_int), ("error", C.c_int)]
+
+
+class Operand(C.Structure):
+    _fields_ = [("ptr", C.c_void_p), ("x_ext", C.c_longlong), ("rows_ext", C.c_longlong),
+                ("g_ext", C.c_longlong), ("row_pitch", C.c_longlong), ("g_pitch", C.c_longlong),
+                ("mn_major", C.c_int), ("x_mod", C.c_int), ("x_mul", C.c_int), ("x_off", C.c_int),
+                ("g_div", C.c_int), ("k_shard", C.c_int)]
+
+
+class GemmDesc(C.Structure):
+    _fields_ = [("M", C.c_int), ("N", C.c_int), ("K", C.c_int), ("groups", C.c_int),
+                ("k_shards", C.c_int), ("causal", C.c_int), ("a", Operand), ("b", Operand),
+                ("out", C.c_void_p), ("out_f32", C.c_int), ("ldo", C.c_longlong),
+                ("o_mod", C.c_int), ("o_str_mod", C.c_longlong), ("o_str_div", C.c_longlong),
+                ("bias", C.c_void_p), ("bias_g_stride", C.c_longlong), ("resid", C.c_void_p),
+                ("ld_resid", C.c_longlong), ("aux", C.c_void_p), ("out2", C.c_void_p),
+                ("act", C.c_int)]
+
+
+_lib = None
+
+_SIGS = {
+    "gptl_strerror": (C.c_char_p, [C.c_int]),
+    "gptl_read_device_error": (C.c_int, [C.POINTER(C.c_int), C.c_int]),
+    "gpt_layer_workspace_bytes": (C.c_int, [C.POINTER(Shape), C.POINTER(C.c_size_t),
+                                            C.POINTER(C.c_size_t)]),
+    "gpt_layer_param_layout": (C.c_int, [C.POINTER(Shape), C.POINTER(C.c_size_t),
+                                         C.POINTER(C.c_size_t)]),
+    "gpt_layer_fwd": (C.c_int, [C.POINTER(Shape), C.POINTER(Weights), C.c_void_p, C.c_void_p,
+                                C.c_void_p, C.c_void_p, C.c_void_p]),
+    "gpt_layer_bwd": (C.c_int, [C.POINTER(Shape), C.POINTER(Weights), C.c_void_p, C.c_void_p,
+                                C.c_void_p, C.c_void_p, C.POINTER(Grads), C.c_void_p, C.c_void_p]),
+    "adam_step_fp32_master": (C.c_int, [C.c_size_t, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                        C.c_void_p, C.c_int, C.c_float, C.c_float, C.c_float,
+                                        C.c_float, C.c_float, C.c_void_p, C.c_void_p]),
+    "loss_scale_update": (C.c_int, [C.c_void_p, C.c_int, C.c_float, C.c_float, C.c_float,
+                                    C.c_void_p]),
+    "gptl_check_overflow": (C.c_int, [C.c_size_t, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "gptl_gemm": (C.c_int, [C.POINTER(GemmDesc), C.c_int, C.c_void_p]),
+    "gptl_layernorm_fwd": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
+                                     C.c_void_p, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_void_p]),
+    "gptl_layernorm_bwd_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
+    "gptl_layernorm_bwd": (C.c_int, [C.c_int, C.c_int, C.c_int] + [C.c_void_p] * 11 + [C.c_void_p]),
+    "gptl_softmax_fwd": (C.c_int, [C.c_longlong, C.c_int, C.c_int, C.c_float, C.c_void_p,
+                                   C.c_void_p]),
+    "gptl_softmax_bwd": (C.c_int, [C.c_longlong, C.c_int, C.c_int, C.c_float, C.c_void_p,
+                                   C.c_void_p, C.c_void_p]),
+    "gptl_colsum_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
+    "gptl_colsum": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_longlong, C.c_longlong, C.c_int,
+                              C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+}
+
+
+def lib():
+    """The loaded library (loaded on first use; raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m transformer_layer_step_b200.build`"
+                               " (there is no fallback implementation)")
+        handle = C.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of every function declared in include/*.h."""
+    names = []
+    for fname in sorted(os.listdir(INCLUDE)):
+        if not fname.endswith(".h"):
+            continue
+        text = open(os.path.join(INCLUDE, fname)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z_0-9]*\s*\*?\s*([a-z_][a-z_0-9]*)\s*\(",
+                            text, flags=re.M)
+    return sorted(set(names))
+
+
+def strerror(code: int) -> str:
+    return lib().gptl_strerror(code).decode()
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise GptlError(rc, where)
+
+
+def make_shape(batch, seq, hidden, heads, ffn, tp, dtype, ln_eps=1e-5) -> Shape:
+    return Shape(batch, seq, hidden, heads, ffn, tp, DTYPES.get(dtype, dtype), ln_eps)
+
+
+def workspace_bytes(shape: Shape):
+    a, b = C.c_size_t(), C.c_size_t()
+    _check(lib().gpt_layer_workspace_bytes(C.byref(shape), C.byref(a), C.byref(b)),
+           "gpt_layer_workspace_bytes")
+    return a.value, b.value
+
+
+def param_layout(shape: Shape):
+    offs = (C.c_size_t * 12)()
+    n = C.c_size_t()
+    _check(lib().gpt_layer_param_layout(C.byref(shape), offs, C.byref(n)), "gpt_layer_param_layout")
+    return [int(o) for o in offs], n.value
+
+
+def make_weights(ptrs: dict) -> Weights:
+    return Weights(*[_ptr(ptrs[n]) for n in PARAM_NAMES])
+
+
+def make_grads(ptrs: dict) -> Grads:
+    return Grads(*[_ptr(ptrs[n]) for n in PARAM_NAMES])
+
+
+def layer_fwd(shape, weights: Weights, x, y, saved, scratch=None, stream=0):
+    _check(lib().gpt_layer_fwd(C.byref(shape), C.byref(weights), _ptr(x), _ptr(y), _ptr(saved),
+                               _ptr(scratch), stream), "gpt_layer_fwd")
+
+
+def layer_bwd(shape, weights: Weights, x, saved, dy, dx, grads: Grads, scratch, stream=0):
+    _check(lib().gpt_layer_bwd(C.byref(shape), C.byref(weights), _ptr(x), _ptr(saved), _ptr(dy),
+                               _ptr(dx), C.byref(grads), _ptr(scratch), stream), "gpt_layer_bwd")
+
+
+def adam_step(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps, weight_decay,
+              state, stream=0):
+    _check(lib().adam_step_fp32_master(n_params, _ptr(master), _ptr(m), _ptr(v), _ptr(grad),
+                                       _ptr(w16), DTYPES.get(dtype, dtype), lr, beta1, beta2, eps,
+                                       weight_decay, _ptr(state), stream), "adam_step_fp32_master")
+
+
+def scale_update(state, growth_interval, growth_factor, backoff_factor, min_scale, stream=0):
+    _check(lib().loss_scale_update(_ptr(state), growth_interval, growth_factor, backoff_factor,
+                                   min_scale, stream), "loss_scale_update")
+
+
+def check_overflow(n, grad, state, stream=0):
+    _check(lib().gptl_check_overflow(n, _ptr(grad), _ptr(state), stream), "gptl_check_overflow")
+
+
+def operand(t, x_ext, rows_ext, g_ext, row_pitch, g_pitch=0, mn_major=0, x_mod=1, x_mul=0,
+            x_off=0, g_div=None, k_shard=0) -> Operand:
+    if g_div is None:
+        g_div = 1 if g_ext > 1 else (1 << 30)
+    return Operand(_ptr(t), x_ext, rows_ext, g_ext, row_pitch, g_pitch, mn_major, x_mod, x_mul,
+                   x_off, g_div, k_shard)
+
+
+def gemm(desc: GemmDesc, dtype, stream=0):
+    _check(lib().gptl_gemm(C.byref(desc), DTYPES.get(dtype, dtype), stream), "gptl_gemm")
+
+
+def layernorm_fwd(rows, h, dtype, x, g, b, eps, y, mu, rstd, stream=0):
+    _check(lib().gptl_layernorm_fwd(rows, h, DTYPES.get(dtype, dtype), _ptr(x), _ptr(g), _ptr(b),
+                                    eps, _ptr(y), _ptr(mu), _ptr(rstd), stream), "gptl_layernorm_fwd")
+
+
+def layernorm_bwd_scratch_bytes(rows, h) -> int:
+    return lib().gptl_layernorm_bwd_scratch_bytes(rows, h)
+
+
+def layernorm_bwd(rows, h, dtype, gy, x, mu, rstd, g, resid, dx, dg, db, dx_sum, scratch, stream=0):
+    _check(lib().gptl_layernorm_bwd(rows, h, DTYPES.get(dtype, dtype), _ptr(gy), _ptr(x), _ptr(mu),
+                                    _ptr(rstd), _ptr(g), _ptr(resid), _ptr(dx), _ptr(dg), _ptr(db),
+                                    _ptr(dx_sum), _ptr(scratch), stream), "gptl_layernorm_bwd")
+
+
+def softmax_fwd(blocks, s, dtype, scale, scores, stream=0):
+    _check(lib().gptl_softmax_fwd(blocks, s, DTYPES.get(dtype, dtype), scale, _ptr(scores), stream),
+           "gptl_softmax_fwd")
+
+
+def softmax_bwd(blocks, s, dtype, scale, prob, dprob, stream=0):
+    _check(lib().gptl_softmax_bwd(blocks, s, DTYPES.get(dtype, dtype), scale, _ptr(prob),
+                                  _ptr(dprob), stream), "gptl_softmax_bwd")
+
+
+def colsum_scratch_bytes(n, groups) -> int:
+    return lib().gptl_colsum_scratch_bytes(n, groups)
+
+
+def colsum(rows, n, groups, ld, gstride, dtype, a, out, scratch, stream=0):
+    _check(lib().gptl_colsum(rows, n, groups, ld, gstride, DTYPES.get(dtype, dtype), _ptr(a),
+                             _ptr(out), _ptr(scratch), stream), "gptl_colsum")
+
+
+def read_device_error(clear: bool = True) -> int:
+    w = C.c_int()
+    _check(lib().gptl_read_device_error(C.byref(w), 1 if clear else 0), "gptl_read_device_error")
+    return w.value

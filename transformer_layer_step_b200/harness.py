@@ -1,0 +1,127 @@
+"""Device memory for one layer's training step, held in torch tensors, and the
+four C-ABI calls that make a step.
+
+torch only allocates memory and provides the stream; the fwd, bwd, Adam and
+scaler steps all run in libgptlayer.so.  Layout: one flat arena per kind
+(16-bit weights, fp32 master / m / v / grad), the 12 parameter tensors at the
+offsets the library reports, plus the activation workspace.
+"""
+from __future__ import annotations
+
+import struct
+
+import numpy as np
+import torch
+
+from . import gptlayer as G
+from . import synth
+
+TORCH_DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
+
+
+def bits_to_tensor(bits: np.ndarray, dtype: str, device) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(TORCH_DT[dtype]).to(device)
+
+
+def tensor_to_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+class LayerStep:
+    """Everything one layer step needs on `device`, filled from synth inputs."""
+
+    def __init__(self, cfg: synth.LayerConfig, inputs: dict, device="cuda", hyper=None):
+        self.cfg = cfg
+        self.hyper = dict(synth.HYPER, **(hyper or {}))
+        self.device = torch.device(device)
+        self.shape = G.make_shape(cfg.batch, cfg.seq, cfg.hidden, cfg.heads, cfg.ffn, cfg.tp,
+                                  cfg.dtype, self.hyper["ln_eps"])
+        self.offsets, self.n_params = G.param_layout(self.shape)
+        saved_b, scratch_b = G.workspace_bytes(self.shape)
+        dt = TORCH_DT[cfg.dtype]
+        dev = self.device
+        T, h = cfg.tokens, cfg.hidden
+
+        # flat parameter arenas
+        flat_bits = np.zeros(self.n_params, dtype=np.uint16)
+        self.param_shapes = {}
+        for name, off in zip(G.PARAM_NAMES, self.offsets):
+            arr = inputs["params"][name]
+            self.param_shapes[name] = arr.shape
+            flat_bits[off:off + arr.size] = arr.reshape(-1)
+        self.w16 = bits_to_tensor(flat_bits, cfg.dtype, dev)
+        master = synth.from_bits(flat_bits, cfg.dtype).astype(np.float32)
+        self.master = torch.from_numpy(master).to(dev)
+        self.m = torch.zeros(self.n_params, dtype=torch.float32, device=dev)
+        self.v = torch.zeros(self.n_params, dtype=torch.float32, device=dev)
+        self.grad = torch.zeros(self.n_params, dtype=torch.float32, device=dev)
+
+        self.x = bits_to_tensor(inputs["x"], cfg.dtype, dev).view(T, h)
+        self.y = torch.empty((T, h), dtype=dt, device=dev)
+        self.dx = torch.empty((T, h), dtype=dt, device=dev)
+        self.dy = torch.zeros((T, h), dtype=dt, device=dev)
+        self.saved = torch.empty(max(saved_b, 256), dtype=torch.uint8, device=dev)
+        self.scratch = torch.empty(max(scratch_b, 256), dtype=torch.uint8, device=dev)
+        self.state = torch.zeros(8, dtype=torch.int32, device=dev)
+        self.reset_scaler(self.hyper["init_scale"])
+
+        wp, gp = {}, {}
+        for name, off in zip(G.PARAM_NAMES, self.offsets):
+            wp[name] = self.w16.data_ptr() + 2 * off
+            gp[name] = self.grad.data_ptr() + 4 * off
+        self.weights = G.make_weights(wp)
+        self.grads = G.make_grads(gp)
+
+    # ---------------------------------------------------------------- state
+    def reset_scaler(self, scale: float, tracker: int = 0, step: int = 0):
+        words = struct.unpack("<i", struct.pack("<f", scale))[0]
+        self.state.copy_(torch.tensor([words, tracker, 0, step, 0, 0, 0, 0], dtype=torch.int32))
+
+    def scaler(self) -> dict:
+        s = self.state.cpu().numpy()
+        return dict(scale=float(s[:1].view(np.float32)[0]), growth_tracker=int(s[1]),
+                    found_inf=int(s[2]), step=int(s[3]))
+
+    def set_dy_bits(self, bits: np.ndarray):
+        self.dy.copy_(bits_to_tensor(bits, self.cfg.dtype, self.device).view_as(self.dy))
+
+    # ---------------------------------------------------------------- calls
+    def stream(self) -> int:
+        return torch.cuda.current_stream(self.device).cuda_stream
+
+    def fwd(self):
+        G.layer_fwd(self.shape, self.weights, self.x, self.y, self.saved, None, self.stream())
+
+    def bwd(self):
+        G.layer_bwd(self.shape, self.weights, self.x, self.saved, self.dy, self.dx, self.grads,
+                    self.scratch, self.stream())
+
+    def adam(self):
+        hp = self.hyper
+        G.adam_step(self.n_params, self.master, self.m, self.v, self.grad, self.w16, self.cfg.dtype,
+                    hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], self.state,
+                    self.stream())
+
+    def scale_update(self):
+        hp = self.hyper
+        G.scale_update(self.state, hp["growth_interval"], hp["growth_factor"],
+                       hp["backoff_factor"], hp["min_scale"], self.stream())
+
+    def step(self):
+        self.fwd()
+        self.bwd()
+        self.adam()
+        self.scale_update()
+
+    # ------------------------------------------------------------ readback
+    def param_tensor(self, arena: torch.Tensor, name: str) -> torch.Tensor:
+        off = self.offsets[G.PARAM_NAMES.index(name)]
+        shp = self.param_shapes[name]
+        return arena[off:off + int(np.prod(shp))].view(shp)
+
+    def grads_host(self) -> dict:
+        return {n: self.param_tensor(self.grad, n).cpu().numpy() for n in G.PARAM_NAMES}
+
+    def params_host_bits(self) -> dict:
+        return {n: tensor_to_bits(self.param_tensor(self.w16, n)) for n in G.PARAM_NAMES}
