@@ -15,11 +15,26 @@ Column split: each shard computes its own output columns from the full
 input; row split: each shard multiplies its slice of the input and the
 partial products are summed ("Megatron-LM 3D parallelism", §1; "Megatron-LM
 overview", §2.2).  Here the sum is an explicit float64 loop over shards.
+
+Precision.  With precision=None every value is exact float64.  With
+precision="fp16" or "bf16" the layer is computed the way the pages' mixed
+precision defines it ("Megatron-LM overview", §3.1: FP16 matrix math; the
+layer computes in fp16/bf16): every activation tensor that one step of the
+path hands to the next is held in the 16-bit type (round to nearest, ties to
+even), while the arithmetic inside a step stays exact.  The stored tensors
+are, forward: L1, C = [Q|K|V], the raw scores S = Q K^T, P, O, H, L2, Z,
+A = gelu(Z); backward: dZ (the GeLU backward is applied to dOut W2 before
+the store, as the fused bias-GeLU's backward), dL2, dH, dO, dP, dV, dS, dQ,
+dK, dL1.  The layer outputs Out and dX are returned unrounded (their own
+store is the caller's last rounding) and the weight and bias gradients are
+fp32 quantities, returned exactly.
 """
 from __future__ import annotations
 
 import math
 import numpy as np
+
+from .optim import round_to_16
 
 # Plainest readings where the pages are silent:
 #   LayerNorm: affine, biased variance over h, eps passed in (1e-5 by default).
@@ -73,12 +88,18 @@ def causal_softmax(z: np.ndarray) -> np.ndarray:
     return p
 
 
-def attention_head_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray):
-    """One (batch, head) block of causal self-attention: returns (P, O)."""
+def attention_head_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, precision=None):
+    """One (batch, head) block of causal self-attention: returns (P, O).
+    With a 16-bit precision the raw scores Q K^T and P are stored values."""
     d = q.shape[1]
-    z = (q @ k.T) / math.sqrt(d)
-    p = causal_softmax(z)
+    z = _store(q @ k.T, precision) / math.sqrt(d)
+    p = _store(causal_softmax(z), precision)
     return p, p @ v
+
+
+def _store(a: np.ndarray, precision):
+    """An activation tensor as the next step reads it (see the module doc)."""
+    return a if precision is None else round_to_16(a, precision)
 
 
 def _check(dims, params):
@@ -91,8 +112,10 @@ def _check(dims, params):
     return b, s, h, a, f, t
 
 
-def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5):
-    """Forward pass.  x: [T, h] float64.  Returns (out, cache)."""
+def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precision=None):
+    """Forward pass.  x: [T, h] float64.  precision: None (exact) or the
+    16-bit type the activations are stored in.  Returns (out, cache)."""
+    st = lambda a: _store(a, precision)
     b, s, h, a, f, t = _check(dims, params)
     d = h // a
     hs, a_s = h // t, a // t            # hidden columns and heads per shard
@@ -101,9 +124,10 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5):
 
     # 1. LN1
     l1, mu1, rstd1, xhat1 = layer_norm_fwd(x, params["ln1_g"], params["ln1_b"], eps)
+    l1 = st(l1)
 
     # 2. QKV column-split GEMM: C_i = L1 W_qkv,i^T + b_qkv,i  -> [Q_i | K_i | V_i]
-    c = np.stack([l1 @ params["w_qkv"][i].T + params["b_qkv"][i][None, :] for i in range(t)])
+    c = st(np.stack([l1 @ params["w_qkv"][i].T + params["b_qkv"][i][None, :] for i in range(t)]))
 
     # 3. causal attention, head by head; head eta of shard i is global head i*a/t+eta
     probs = np.zeros((t, b, a_s, s, s))
@@ -116,23 +140,24 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5):
                 qh = c[i, rows, 0 * hs:1 * hs][:, cols]
                 kh = c[i, rows, 1 * hs:2 * hs][:, cols]
                 vh = c[i, rows, 2 * hs:3 * hs][:, cols]
-                pr, oh = attention_head_fwd(qh, kh, vh)
+                pr, oh = attention_head_fwd(qh, kh, vh, precision)
                 probs[i, j, eta] = pr
-                o[i, rows, cols] = oh
+                o[i, rows, cols] = st(oh)
 
     # 4. out-projection, row split: partial products summed over shards, bias
     #    added once after the sum, then the residual
     y_attn = np.zeros((T, h))
     for i in range(t):
         y_attn += o[i] @ params["w_o"][i].T
-    hid = x + y_attn + params["b_o"][None, :]
+    hid = st(x + y_attn + params["b_o"][None, :])
 
     # 5. LN2
     l2, mu2, rstd2, xhat2 = layer_norm_fwd(hid, params["ln2_g"], params["ln2_b"], eps)
+    l2 = st(l2)
 
     # 6. FFN1 column split with fused bias + GeLU
-    z = np.stack([l2 @ params["w_1"][i].T + params["b_1"][i][None, :] for i in range(t)])
-    act = gelu(z)
+    z = st(np.stack([l2 @ params["w_1"][i].T + params["b_1"][i][None, :] for i in range(t)]))
+    act = st(gelu(z))
 
     # 7. FFN2 row split: shard sum, bias, residual
     y_mlp = np.zeros((T, h))
@@ -141,7 +166,8 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5):
     out = hid + y_mlp + params["b_2"][None, :]
 
     cache = dict(x=x, l1=l1, mu1=mu1, rstd1=rstd1, xhat1=xhat1, c=c, probs=probs, o=o,
-                 hid=hid, l2=l2, mu2=mu2, rstd2=rstd2, xhat2=xhat2, z=z, act=act)
+                 hid=hid, l2=l2, mu2=mu2, rstd2=rstd2, xhat2=xhat2, z=z, act=act,
+                 precision=precision)
     return out, cache
 
 
@@ -153,6 +179,7 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
     hs, a_s = h // t, a // t
     T = b * s
     inv_sqrt_d = 1.0 / math.sqrt(d)
+    st = lambda a: _store(a, cache.get("precision"))
     gr = {}
 
     # FFN2 (row split): each shard's weight gradient and input gradient
@@ -162,22 +189,23 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
 
     # GeLU backward and FFN1 (column split); the input gradient is the sum
     # of the shards' partial products
-    dz = d_act * gelu_prime(cache["z"])
+    dz = st(d_act * gelu_prime(cache["z"]))
     gr["b_1"] = dz.sum(axis=1)
     gr["w_1"] = np.stack([dz[i].T @ cache["l2"] for i in range(t)])
     dl2 = np.zeros((T, h))
     for i in range(t):
         dl2 += dz[i] @ params["w_1"][i]
+    dl2 = st(dl2)
 
     # LN2 backward plus the residual path
     dln, gr["ln2_g"], gr["ln2_b"] = layer_norm_bwd(dl2, cache["xhat2"], cache["rstd2"],
                                                    params["ln2_g"])
-    dhid = dout + dln
+    dhid = st(dout + dln)
 
     # out-projection (row split)
     gr["b_o"] = dhid.sum(axis=0)
     gr["w_o"] = np.stack([dhid.T @ cache["o"][i] for i in range(t)])
-    do = np.stack([dhid @ params["w_o"][i] for i in range(t)])
+    do = st(np.stack([dhid @ params["w_o"][i] for i in range(t)]))
 
     # attention backward, head by head
     c = cache["c"]
@@ -192,12 +220,12 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
                 vh = c[i, rows, 2 * hs:3 * hs][:, cols]
                 pr = cache["probs"][i, j, eta]
                 doh = do[i, rows, cols]
-                dp = doh @ vh.T
-                dv = pr.T @ doh
+                dp = st(doh @ vh.T)
+                dv = st(pr.T @ doh)
                 dzs = pr * (dp - (pr * dp).sum(axis=1, keepdims=True))
-                dsc = dzs * inv_sqrt_d
-                dq = dsc @ kh
-                dk = dsc.T @ qh
+                dsc = st(dzs * inv_sqrt_d)
+                dq = st(dsc @ kh)
+                dk = st(dsc.T @ qh)
                 dc[i, rows, 0 * hs:1 * hs][:, cols] = dq
                 dc[i, rows, 1 * hs:2 * hs][:, cols] = dk
                 dc[i, rows, 2 * hs:3 * hs][:, cols] = dv
@@ -208,6 +236,7 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
     dl1 = np.zeros((T, h))
     for i in range(t):
         dl1 += dc[i] @ params["w_qkv"][i]
+    dl1 = st(dl1)
 
     # LN1 backward plus the residual path
     dln1, gr["ln1_g"], gr["ln1_b"] = layer_norm_bwd(dl1, cache["xhat1"], cache["rstd1"],

@@ -66,6 +66,15 @@ def cast_to_16(p: np.ndarray, dtype: str) -> np.ndarray:
     raise ValueError(dtype)
 
 
+def round_to_16(x: np.ndarray, dtype: str) -> np.ndarray:
+    """float64 value of the fp16/bf16 number nearest to x (ties to even):
+    the value a 16-bit activation tensor holds once stored."""
+    bits = cast_to_16(x, dtype)
+    if dtype == "fp16":
+        return bits.view(np.float16).astype(np.float64)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
 def adam_step(master: np.ndarray, m: np.ndarray, v: np.ndarray, grad: np.ndarray,
               scale: float, step: int, lr: float, beta1: float, beta2: float,
               eps: float, weight_decay: float, dtype: str, inf_flag: int):

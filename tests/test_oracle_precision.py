@@ -1,0 +1,104 @@
+"""Pins: the oracle's mixed-precision mode ("Megatron-LM overview", §3.1:
+FP16 matrix math; the layer computes in fp16/bf16).
+
+* round_to_16 is the correctly rounded (ties-to-even) conversion: equal to
+  torch's on float32 inputs, and free of a double rounding on float64 ones.
+* precision=None is the exact float64 layer (itself pinned by finite
+  differences, the sharded == unsharded invariant and the HF GPT-2 block).
+* Every activation the mode stores sits on the 16-bit grid and equals the
+  rounding of that step recomputed exactly from the stored inputs, so the
+  mode is the exact layer with a rounding at each step boundary and nowhere
+  else.
+* fp16 keeps 11 significant bits: the mode stays within a few 2^-11
+  relative steps of the exact layer on the layer outputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.optim import round_to_16
+from transformer_layer_step_b200 import synth
+
+
+def test_round_to_16_matches_torch():
+    rng = np.random.default_rng(5)
+    # float32 inputs: torch converts from float32 in one correctly rounded step
+    x = (rng.standard_normal(50_000) * 10.0 ** rng.integers(-6, 4, 50_000)).astype(np.float32)
+    for dt, tdt in (("fp16", torch.float16), ("bf16", torch.bfloat16)):
+        ref = torch.from_numpy(x).to(tdt).to(torch.float64).numpy()
+        np.testing.assert_array_equal(round_to_16(x.astype(np.float64), dt), ref)
+    # a float64 value just above a bf16 midpoint rounds up (no detour through
+    # float32, which would land on the midpoint and round to even)
+    assert round_to_16(np.array([1 + 2.0 ** -8 + 2.0 ** -40]), "bf16")[0] == 1 + 2.0 ** -7
+    # ties go to the even neighbour
+    assert round_to_16(np.array([1 + 2.0 ** -11]), "fp16")[0] == 1.0
+    assert round_to_16(np.array([1 + 3 * 2.0 ** -11]), "fp16")[0] == 1 + 2.0 ** -9
+    assert round_to_16(np.array([1 + 2.0 ** -8]), "bf16")[0] == 1.0
+
+
+def _inputs(dtype, t=2):
+    cfg = synth.LayerConfig("p", 2, 32, 64, 4, 256, t, dtype)
+    inp = synth.make_inputs(cfg, seed=3, variant="biased", with_r=True)
+    x = synth.from_bits(inp["x"], dtype).reshape(cfg.tokens, cfg.hidden)
+    p = {k: synth.from_bits(v, dtype).reshape(v.shape) for k, v in inp["params"].items()}
+    dout = synth.from_bits(synth.loss_grad_bits(cfg, 1024.0, inp["r"]), dtype).reshape(x.shape)
+    return cfg, x, p, dout
+
+
+def test_none_is_the_exact_layer():
+    cfg, x, p, dout = _inputs("bf16")
+    o1, c1 = oracle.layer_fwd(x, p, cfg.dims())
+    o2, c2 = oracle.layer_fwd(x, p, cfg.dims(), precision=None)
+    np.testing.assert_array_equal(o1, o2)
+    d1, g1 = oracle.layer_bwd(c1, p, cfg.dims(), dout)
+    d2, g2 = oracle.layer_bwd(c2, p, cfg.dims(), dout)
+    np.testing.assert_array_equal(d1, d2)
+    for k in g1:
+        np.testing.assert_array_equal(g1[k], g2[k])
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_stored_tensors_are_rounded_step_outputs(dtype):
+    cfg, x, p, dout = _inputs(dtype)
+    b, s, h, a, f, t = (cfg.dims()[k] for k in "bshaft")
+    d, hs = h // a, h // t
+    out, c = oracle.layer_fwd(x, p, cfg.dims(), precision=dtype)
+    rnd = lambda v: round_to_16(v, dtype)
+    for k in ("l1", "c", "probs", "o", "hid", "l2", "z", "act"):
+        np.testing.assert_array_equal(rnd(c[k]), c[k], err_msg=k)
+    # each stored tensor is its step recomputed exactly from stored inputs, rounded once
+    l1 = (x - x.mean(1, keepdims=True)) / np.sqrt(x.var(1, keepdims=True) + 1e-5)
+    np.testing.assert_array_equal(c["l1"], rnd(l1 * p["ln1_g"] + p["ln1_b"]))
+    for i in range(t):
+        np.testing.assert_array_equal(c["c"][i], rnd(c["l1"] @ p["w_qkv"][i].T + p["b_qkv"][i]))
+        np.testing.assert_array_equal(c["z"][i], rnd(c["l2"] @ p["w_1"][i].T + p["b_1"][i]))
+    np.testing.assert_array_equal(c["act"], rnd(oracle.gelu(c["z"])))
+    q = c["c"][1, s:2 * s, d:2 * d]                 # shard 1, batch 1, head 1
+    k = c["c"][1, s:2 * s, hs + d:hs + 2 * d]
+    v = c["c"][1, s:2 * s, 2 * hs + d:2 * hs + 2 * d]
+    sc = rnd(q @ k.T) / math.sqrt(d)
+    pr = rnd(oracle.causal_softmax(sc))
+    np.testing.assert_array_equal(c["probs"][1, 1, 1], pr)
+    np.testing.assert_array_equal(c["o"][1, s:2 * s, d:2 * d], rnd(pr @ v))
+    hid = x + sum(c["o"][i] @ p["w_o"][i].T for i in range(t)) + p["b_o"]
+    np.testing.assert_allclose(c["hid"], rnd(hid), rtol=0, atol=0)
+    # the layer output itself is returned unrounded
+    y = c["hid"] + sum(c["act"][i] @ p["w_2"][i].T for i in range(t)) + p["b_2"]
+    np.testing.assert_allclose(out, y, rtol=1e-14, atol=1e-14)
+    assert np.any(rnd(out) != out)
+
+
+def test_fp16_mode_is_close_to_exact():
+    cfg, x, p, dout = _inputs("fp16")
+    oe, ce = oracle.layer_fwd(x, p, cfg.dims())
+    om, cm = oracle.layer_fwd(x, p, cfg.dims(), precision="fp16")
+    rms = lambda v: float(np.sqrt(np.mean(v * v)))
+    assert np.abs(om - oe).max() <= 8 * 2.0 ** -11 * np.abs(oe).max()
+    de, ge = oracle.layer_bwd(ce, p, cfg.dims(), dout)
+    dm, gm = oracle.layer_bwd(cm, p, cfg.dims(), dout)
+    assert np.abs(dm - de).max() <= 2e-2 * rms(de)
+    for k in ge:
+        assert np.abs(gm[k] - ge[k]).max() <= 2e-2 * rms(ge[k]), k
