@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Throughput of one GPT transformer layer's training step on B200.
+
+One step = gpt_layer_fwd + gpt_layer_bwd + adam_step_fp32_master +
+loss_scale_update through the C ABI of libgptlayer.so, on one CUDA stream,
+for the GPT-2 117M layer shape (hidden 768, 12 heads, ffn 3072, seq 1024,
+micro-batch 8, tp 1, bf16 compute with fp32 master weights, initial loss
+scale 2^16) on synthetic seeded inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is tokens/s over all ranks with the
+inputs resident in HBM: per-step device time from CUDA events on the
+launching stream, the L2 flushed (256 MiB write) between steps outside the
+per-step events, max over ranks.  Several GPUs run independent replicas
+(the step has no cross-GPU exchange), so scaling is weak.
+
+Also reported: `e2e` (the same step with the inputs copied from pinned host
+memory and the output read back inside the timed region), the roofline of
+the dominant kernel (the tcgen05 GEMM: algorithmic FLOPs over its launches'
+summed device time, from per-launch events recorded by the library in a
+second timed pass), a per-kernel breakdown, SM clocks sampled during the
+timed region, and `cpu_baseline`, the float64 CPU oracle timed on a bounded
+sample of the same workload on this host's cores.
+
+`--impl reference` times that oracle alone, as the comparison arm.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from transformer_layer_step_b200 import synth  # noqa: E402
+
+METRIC = "GPT layer fwd+bwd+Adam tokens/sec at 1 B200"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "gpt2-117m"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = ("transformer_layer_step_b200/csrc/gemm_tc.cuh",
+                  "transformer_layer_step_b200/csrc/common.cuh",
+                  "transformer_layer_step_b200/csrc/bw_kernels.cuh",
+                  "transformer_layer_step_b200/csrc/gptlayer.cu")
+
+
+# ----------------------------------------------------------------- workload
+def step_flops(cfg) -> dict:
+    """Algorithmic FLOPs of one step.  Causal: the attention products count
+    only the lower triangle q <= p that the method computes; dense: the
+    usual full-square convention."""
+    b, s, h, f = cfg.batch, cfg.seq, cfg.hidden, cfg.ffn
+    T = b * s
+    linear = 2 * T * (4 * h * h + 2 * h * f)            # QKV, out-proj, FFN1, FFN2
+    attn_causal = 2 * 2 * b * h * (s * (s + 1) // 2)     # QK^T and PV over the triangle
+    attn_dense = 2 * 2 * b * h * s * s
+    return {"causal": 3 * (linear + attn_causal), "dense": 3 * (linear + attn_dense),
+            "linear": 3 * linear}
+
+
+def kernel_bytes(cfg, n_params: int) -> dict:
+    """Algorithmic HBM bytes per launch of each bandwidth kernel of the step
+    (2-byte activations, 4-byte fp32 state)."""
+    b, s, h, a, f = cfg.batch, cfg.seq, cfg.hidden, cfg.heads, cfg.ffn
+    T = b * s
+    tri = b * a * (s * (s + 1) // 2)
+    return {
+        "F1 ln1": 4 * T * h, "F7 ln2": 4 * T * h,             # read x, write y
+        "B6 ln2 bwd": 8 * T * h, "B12 ln1 bwd": 8 * T * h,    # read gy, x, resid; write dx
+        "F4 softmax": 4 * tri, "B9 softmax bwd": 6 * tri,    # lower triangle only
+        "B2 db2": 2 * T * h, "B3 db1": 2 * T * f, "B11 dbqkv": 2 * T * 3 * h,
+        "O1 overflow": 4 * n_params, "O2 adam": 30 * n_params,
+    }
+
+
+def load_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return json.load(fh), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per GEMM launch-set from the committed ncu summary, or None
+    when the summary is absent or the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(workload)
+    if not ent or ent.get("kernel_sources") != kernel_source_hash():
+        return None
+    return ent.get("gemm_dram_bytes_per_step")
+
+
+# ------------------------------------------------------------ clock sampler
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = max((num(r[2]) for r in rows if num(r[2]) is not None), default=None)
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        loaded = [v for v, p in zip(sm, power) if p is not None and p > 250] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+# --------------------------------------------------------------- CPU oracle
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(cfg, n_seq: int, seq_prefix: int | None = None, repeats: int = 1) -> dict:
+    """Times the oracle (test infrastructure, float64 numpy) on a bounded
+    sample of the workload: fwd + bwd of `n_seq` of the step's sequences
+    (optionally only their first `seq_prefix` positions, a causal problem of
+    its own) at the method's precision, plus the Adam step and overflow check
+    over the same fraction of the parameter arena.  Returns tokens/s."""
+    import oracle
+    s = seq_prefix or cfg.seq
+    sub = dataclasses.replace(cfg, batch=n_seq, seq=s)
+    inp = synth.make_inputs(sub, seed=0, variant="biased", with_r=True)
+    x = synth.from_bits(inp["x"], cfg.dtype).reshape(sub.tokens, cfg.hidden)
+    p = {k: synth.from_bits(v, cfg.dtype).reshape(v.shape) for k, v in inp["params"].items()}
+    dout = synth.from_bits(synth.loss_grad_bits(sub, 65536.0, inp["r"]),
+                           cfg.dtype).reshape(x.shape)
+    n_params = sum(int(v.size) for v in inp["params"].values())
+    frac = sub.tokens / cfg.tokens
+    n_adam = max(1024, int(n_params * frac))
+    rng = np.random.default_rng(1)
+    master = rng.standard_normal(n_adam).astype(np.float32) * 0.02
+    m = np.zeros(n_adam, np.float32)
+    v = np.zeros(n_adam, np.float32)
+    g = rng.standard_normal(n_adam).astype(np.float32)
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        _, cache = oracle.layer_fwd(x, p, sub.dims(), precision=cfg.dtype)
+        oracle.layer_bwd(cache, p, sub.dims(), dout)
+        del cache
+        inf = oracle.found_inf(g)
+        oracle.adam_step(master, m, v, g, 65536.0, 0, 6e-5, 0.9, 0.95, 1e-8, 0.0, cfg.dtype, inf)
+        times.append(time.perf_counter() - t0)
+    desc = (f"{n_seq} of {cfg.batch} sequences" +
+            (f" (first {s} of {cfg.seq} positions)" if seq_prefix else "") +
+            f" fwd+bwd at {cfg.dtype} storage precision, plus overflow check and Adam over "
+            f"{n_adam} of {n_params} parameters; float64 numpy oracle")
+    return {"tokens": sub.tokens, "seconds": times, "sample": desc,
+            "value": sub.tokens * len(times) / sum(times)}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from transformer_layer_step_b200 import gptlayer as G
+    from transformer_layer_step_b200.harness import LayerStep
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inp = synth.make_inputs(cfg, seed=rank, variant="biased", with_r=True)
+    ls = LayerStep(cfg, inp, device=dev)
+    dy_bits = synth.loss_grad_bits(cfg, ls.hyper["init_scale"], inp["r"])
+    ls.set_dy_bits(dy_bits)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    K, W = args.steps, args.warmup
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed_steps(n, body):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        for i in range(n):
+            ev[i][0].record(stream)
+            body()
+            ev[i][1].record(stream)
+            flush.zero_()
+        return ev
+
+    for _ in range(W):
+        ls.step()
+        flush.zero_()
+    torch.cuda.synchronize()
+    if G.read_device_error(clear=True):
+        raise RuntimeError("device error word set during warm-up")
+
+    # ---- value: inputs resident in HBM
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = G.launch_count()
+    ev = timed_steps(K, ls.step)
+    torch.cuda.synchronize()
+    barrier()
+    launches = G.launch_count() - launches0
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(step_ms))
+    ms_per_step = total_ms / K
+
+    # ---- per-launch device times (second pass, library events between launches)
+    per_step = launches // K
+    G.profile_begin(per_step * K + 16)
+    timed_steps(K, ls.step)
+    recs, dropped = G.profile_end(per_step * K + 16)
+    if dropped:
+        raise RuntimeError(f"{dropped} launches were not timed")
+
+    # ---- e2e: pinned host inputs in, output and scaler state out, every step
+    import torch as _t
+    x_host = _t.empty(ls.x.shape, dtype=ls.x.dtype).pin_memory()
+    dy_host = _t.empty(ls.dy.shape, dtype=ls.dy.dtype).pin_memory()
+    y_host = _t.empty(ls.y.shape, dtype=ls.y.dtype).pin_memory()
+    st_host = _t.empty(ls.state.shape, dtype=ls.state.dtype).pin_memory()
+    x_host.copy_(ls.x.cpu())
+    dy_host.copy_(ls.dy.cpu())
+
+    def e2e_step():
+        ls.x.copy_(x_host, non_blocking=True)
+        ls.dy.copy_(dy_host, non_blocking=True)
+        ls.step()
+        y_host.copy_(ls.y, non_blocking=True)
+        st_host.copy_(ls.state, non_blocking=True)
+
+    barrier()
+    torch.cuda.synchronize()
+    ev2 = timed_steps(K, e2e_step)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2)) / K
+    if G.read_device_error(clear=True):
+        raise RuntimeError("device error word set during the timed steps")
+    sc = ls.scaler()
+    h2d = x_host.numel() * x_host.element_size() + dy_host.numel() * dy_host.element_size()
+    d2h = y_host.numel() * y_host.element_size() + st_host.numel() * st_host.element_size()
+    return dict(ms_per_step=ms_per_step, step_ms=step_ms, launches=launches, recs=recs,
+                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks, n_params=ls.n_params,
+                scaler=sc)
+
+
+def summarize_kernels(recs, K, cfg, n_params, peaks, flops):
+    """Per-kernel device time per step, share, and achieved rate."""
+    by_tag, by_kind = {}, {}
+    for kind, tag, ms in recs:
+        e = by_tag.setdefault(tag, {"kind": kind, "launches": 0, "ms": 0.0})
+        e["launches"] += 1
+        e["ms"] += ms
+        k = by_kind.setdefault(kind, {"launches": 0, "ms": 0.0})
+        k["launches"] += 1
+        k["ms"] += ms
+    total = sum(e["ms"] for e in by_kind.values())
+    nbytes = kernel_bytes(cfg, n_params)
+    rows = []
+    for tag, e in by_tag.items():
+        ms = e["ms"] / K
+        row = {"step": tag, "kind": e["kind"], "launches_per_step": e["launches"] // K,
+               "ms_per_step": round(ms, 5), "share": round(e["ms"] / total, 4)}
+        if tag in nbytes and ms > 0:
+            row["GB/s"] = round(nbytes[tag] / (ms * 1e-3) / 1e9, 1)
+            row["frac_hbm"] = round(row["GB/s"] / peaks["hbm_gbs"], 3)
+        rows.append(row)
+    kinds = {k: {"launches_per_step": v["launches"] // K, "ms_per_step": round(v["ms"] / K, 5),
+                 "share": round(v["ms"] / total, 4)} for k, v in by_kind.items()}
+    return rows, kinds, total / K
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the CPU oracle timing (it runs on rank 0 at N=1 only)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    cfg = synth.CONFIGS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    config = {"workload": cfg.name, "batch": cfg.batch, "seq_len": cfg.seq,
+              "hidden": cfg.hidden, "heads": cfg.heads, "ffn": cfg.ffn, "tp": cfg.tp,
+              "tokens_per_step": cfg.tokens, "parallelism": f"replicas{world}",
+              "l2": "flushed between steps (256 MiB write, outside the per-step events)"}
+    flops = step_flops(cfg)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        n = args.steps + args.warmup
+        prefix = None if n <= 30 else max(64, (cfg.seq * 30 // n) // 64 * 64)
+        oracle_sample(cfg, 1, prefix, repeats=args.warmup)
+        r = oracle_sample(cfg, 1, prefix, repeats=args.steps)
+        cores = blas_threads()
+        line = {"impl": "reference", "metric": METRIC, "value": round(r["value"], 3),
+                "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(1e3 * sum(r["seconds"]) / len(r["seconds"]), 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": round(r["value"], 3), "unit": UNIT, "cores": cores,
+                                 "kind": "oracle", "sample": "per step: " + r["sample"]},
+                "e2e": {"value": round(r["value"], 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    import torch
+    res = run_ours(args, cfg, rank, world, local_rank)
+    peaks, peak_src = load_peaks()
+    rows, kinds, prof_ms = summarize_kernels(res["recs"], args.steps, cfg, res["n_params"],
+                                             peaks, flops)
+    gemm_ms = kinds.get("gemm", {}).get("ms_per_step", 0.0)
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    achieved_tf = flops["causal"] / (gemm_ms * 1e-3) / 1e12 if gemm_ms else None
+    traffic = recorded_traffic(cfg.name)
+    ms = res["ms_per_step"]
+    value = world * cfg.tokens / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": cfg.dtype, "data": "synthetic", "config": config,
+        "tflops_causal": round(flops["causal"] / (ms * 1e-3) / 1e12, 1),
+        "tflops_dense_convention": round(flops["dense"] / (ms * 1e-3) / 1e12, 1),
+        "frac_of_bf16_peak": round(flops["causal"] / (ms * 1e-3) / 1e12 / peak_tf, 4),
+        "roofline": {"kernel": "gemm_tc_kernel (all tcgen05 GEMM launches of a step)",
+                     "bound": "tensor",
+                     "achieved": round(achieved_tf, 1) if achieved_tf else None,
+                     "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(achieved_tf / peak_tf, 4) if achieved_tf else None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "work": "causal algorithmic FLOPs of the step's contractions",
+                     "traffic": traffic},
+        "kernels": kinds,
+        "steps_detail": sorted(rows, key=lambda r: -r["ms_per_step"]),
+        "profiled_ms_per_step": round(prof_ms, 4),
+        "e2e": {"value": round(world * cfg.tokens / (res["e2e_ms"] * 1e-3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+        "scaler_after": res["scaler"],
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        r = oracle_sample(cfg, 2)
+        line["cpu_baseline"] = {"value": round(r["value"], 3), "unit": UNIT,
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": r["sample"], "seconds": round(sum(r["seconds"]), 2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libgptlayer.so")
 SOURCES = [os.path.join(PKG, "csrc", "gptlayer.cu")]
 DEPS = SOURCES + [os.path.join(PKG, "csrc", f) for f in ("common.cuh", "gemm_tc.cuh", "bw_kernels.cuh")] + \
-    [os.path.join(ROOT, "include", f) for f in ("gptlayer.h", "gptlayer_parts.h")]
+    [os.path.join(ROOT, "include", f) for f in ("gptlayer.h", "gptlayer_parts.h", "gptlayer_profile.h")]
 
 
 def nvcc_path() -> str:

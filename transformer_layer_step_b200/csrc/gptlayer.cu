@@ -8,12 +8,14 @@
 // library's kernels; nothing falls back to the host.
 #include <math.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "bw_kernels.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gptlayer_parts.h"
+#include "gptlayer_profile.h"
 
 using namespace gptl;
 
@@ -36,6 +38,65 @@ constexpr int kMaxDevices = 64;
 constexpr int kSmemLimit = 232448;   // 227 KB opt-in dynamic shared memory per block
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------- launch recorder
+// Every kernel launch of the library increments g_launches.  While a
+// profiling window is open (gptl_profile_begin .. gptl_profile_end) an event
+// is also recorded on the launch stream at the start of each entry point and
+// after each launch, so that consecutive events bracket one kernel.  The
+// tag names the step of the layer the launch belongs to.
+struct ProfRec {
+  int kind, tag;
+  cudaEvent_t a, b;
+};
+struct Profiler {
+  bool on = false;
+  cudaEvent_t *pool = nullptr;
+  int pool_n = 0, pool_next = 0;
+  ProfRec *recs = nullptr;
+  int cap = 0, n = 0;
+  long long dropped = 0;
+  cudaEvent_t prev = nullptr;
+};
+Profiler g_prof;
+int g_tag = GPTL_TAG_NONE;
+unsigned long long g_launches = 0;
+
+cudaEvent_t prof_event(cudaStream_t st) {
+  if (g_prof.pool_next >= g_prof.pool_n) return nullptr;
+  cudaEvent_t e = g_prof.pool[g_prof.pool_next];
+  if (cudaEventRecord(e, st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  ++g_prof.pool_next;
+  return e;
+}
+
+// Marks the start of an entry point's launches on `st`.
+void prof_start(cudaStream_t st) {
+  if (g_prof.on) g_prof.prev = prof_event(st);
+}
+
+// Called after every successful launch on `st`.
+void prof_launched(cudaStream_t st, int kind) {
+  ++g_launches;
+  if (!g_prof.on) return;
+  cudaEvent_t e = (g_prof.prev && g_prof.n < g_prof.cap) ? prof_event(st) : nullptr;
+  if (!e) {
+    ++g_prof.dropped;
+    g_prof.prev = nullptr;
+    return;
+  }
+  g_prof.recs[g_prof.n++] = ProfRec{kind, g_tag, g_prof.prev, e};
+  g_prof.prev = e;
+}
+
+struct TagScope {
+  int saved;
+  explicit TagScope(int t) : saved(g_tag) { g_tag = t; }
+  ~TagScope() { g_tag = saved; }
+};
 
 struct DeviceInfo {
   int checked = 0, ok = 0, sms = 0;
@@ -152,6 +213,7 @@ int launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) 
   }
   gemm_tc_kernel<T><<<grid, kGemmThreads, smem, stream>>>(p);
   GPTL_CK(cudaGetLastError());
+  prof_launched(stream, GPTL_KIND_GEMM);
   return GPTL_OK;
 }
 
@@ -311,6 +373,7 @@ int run_ln_fwd(int rows, int h, gptl_dtype dt, const void *x, const void *g, con
   });
   if (!ok) return GPTL_E_SHAPE;
   GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_LN_FWD);
   return GPTL_OK;
 }
 
@@ -334,9 +397,11 @@ int run_ln_bwd(int rows, int h, gptl_dtype dt, const void *gy, const void *x, co
   if (!ok) return GPTL_E_SHAPE;
   GPTL_TRY(rc);
   GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_LN_BWD);
   dim3 rg((h + 255) / 256, 2 + want);
   reduce_parts_kernel<<<rg, 256, 0, st>>>(part, nb, h, dg, db, dx_sum);
   GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_REDUCE);
   return GPTL_OK;
 }
 
@@ -362,6 +427,7 @@ int run_softmax_fwd(long long blocks, int s, gptl_dtype dt, float scale, void *s
   }
 #undef GPTL_SMF
   GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_SOFTMAX_FWD);
   return GPTL_OK;
 }
 
@@ -382,6 +448,7 @@ int run_softmax_bwd(long long blocks, int s, gptl_dtype dt, float scale, const v
   }
 #undef GPTL_SMB
   GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_SOFTMAX_BWD);
   return GPTL_OK;
 }
 
@@ -407,10 +474,12 @@ int run_colsum(int rows, int n, int groups, long long ld, long long gstride, gpt
     colsum_kernel<__nv_bfloat16><<<grid, block, 0, st>>>((const __nv_bfloat16 *)a, rows, n, ld,
                                                          gstride, part, groups);
   GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_COLSUM);
   const int width = n * groups;
   reduce_parts_kernel<<<dim3((width + 255) / 256, 1), 256, 0, st>>>(part, split, width, out,
                                                                     nullptr, nullptr);
   GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_REDUCE);
   return GPTL_OK;
 }
 
@@ -536,10 +605,14 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
   float *mu1 = at<float>(saved, w.mu1), *rs1 = at<float>(saved, w.rstd1);
   float *mu2 = at<float>(saved, w.mu2), *rs2 = at<float>(saved, w.rstd2);
   const float attn_scale = 1.0f / sqrtf((float)d);
+  TagScope tag_scope(GPTL_TAG_NONE);
+  prof_start(st);
 
   // LN1
+  g_tag = GPTL_TAG_F1_LN1;
   GPTL_TRY(run_ln_fwd(T, h, dt, x, W->ln1_g, W->ln1_b, D.eps, l1, mu1, rs1, st));
   // QKV column split: C_i = L1 W_qkv,i^T + b_qkv,i
+  g_tag = GPTL_TAG_F2_QKV;
   {
     gptl_gemm_desc g = gemm(T, 3 * hs, h, t, view(l1, h, T, 1, h, 0, 0),
                             view(W->w_qkv, h, 3 * hs, t, h, (long long)3 * hs * h, 0), c, 3 * hs,
@@ -549,6 +622,7 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // scores S = Q K^T per (shard, batch, head), lower-triangle tiles only
+  g_tag = GPTL_TAG_F3_SCORES;
   {
     gptl_operand q = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 0);
     q.x_mod = as; q.x_mul = d; q.g_div = as;
@@ -559,8 +633,10 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // fused scale-mask-softmax, in place
+  g_tag = GPTL_TAG_F4_SOFTMAX;
   GPTL_TRY(run_softmax_fwd(G, s, dt, attn_scale, pb, st));
   // O = P V (K range limited to the lower triangle)
+  g_tag = GPTL_TAG_F5_PV;
   {
     gptl_operand pa = view(pb, s, s, G, s, (long long)s * s, 0);
     gptl_operand v = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 1);
@@ -572,6 +648,7 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // out-projection, row split: H = X + sum_i O_i W_o,i^T + b_o
+  g_tag = GPTL_TAG_F6_OUTPROJ;
   {
     gptl_operand a = view(o, hs, T, t, hs, (long long)T * hs, 0);
     a.g_div = kNoGroup; a.k_shard = 1;
@@ -585,8 +662,10 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // LN2
+  g_tag = GPTL_TAG_F7_LN2;
   GPTL_TRY(run_ln_fwd(T, h, dt, hid, W->ln2_g, W->ln2_b, D.eps, l2, mu2, rs2, st));
   // FFN1 column split with fused bias + GeLU: Z_i, A_i = gelu(Z_i)
+  g_tag = GPTL_TAG_F8_FFN1_GELU;
   {
     gptl_gemm_desc g = gemm(T, fs, h, t, view(l2, h, T, 1, h, 0, 0),
                             view(W->w_1, h, fs, t, h, (long long)fs * h, 0), z, fs,
@@ -598,6 +677,7 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // FFN2 row split: Out = H + sum_i A_i W_2,i^T + b_2
+  g_tag = GPTL_TAG_F10_FFN2;
   {
     gptl_operand a = view(act, fs, T, t, fs, (long long)T * fs, 0);
     a.g_div = kNoGroup; a.k_shard = 1;
@@ -629,9 +709,13 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   void *dp = at<void>(scratch, w.dp), *dc = at<void>(scratch, w.dc), *dl1 = at<void>(scratch, w.dl1);
   float *part = at<float>(scratch, w.part);
   const float attn_scale = 1.0f / sqrtf((float)d);
+  TagScope tag_scope(GPTL_TAG_NONE);
+  prof_start(st);
 
   // ---- FFN2 (row split)
+  g_tag = GPTL_TAG_B2_DB2;
   GPTL_TRY(run_colsum(T, h, 1, h, 0, dt, dy, gr->b_2, part, st));
+  g_tag = GPTL_TAG_B2_DW2;
   {  // dW2_i = dOut^T A_i   [t][h][f/t] fp32
     gptl_gemm_desc g = gemm(h, fs, T, t, view(dy, h, T, 1, h, 0, 1),
                             view(act, fs, T, t, fs, (long long)T * fs, 1), gr->w_2, fs,
@@ -639,6 +723,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     g.out_f32 = 1;
     GPTL_TRY(run_gemm(g, dt, st));
   }
+  g_tag = GPTL_TAG_B1_B3_DZ;
   {  // dZ_i = (dOut W2_i) * gelu'(Z_i)
     gptl_gemm_desc g = gemm(T, fs, h, t, view(dy, h, T, 1, h, 0, 0),
                             view(W->w_2, fs, h, t, fs, (long long)h * fs, 1), dz, fs,
@@ -648,13 +733,16 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // ---- FFN1 (column split)
+  g_tag = GPTL_TAG_B3_DB1;
   GPTL_TRY(run_colsum(T, fs, t, fs, (long long)T * fs, dt, dz, gr->b_1, part, st));
+  g_tag = GPTL_TAG_B5_DW1;
   {  // dW1_i = dZ_i^T L2   [t][f/t][h]
     gptl_gemm_desc g = gemm(fs, h, T, t, view(dz, fs, T, t, fs, (long long)T * fs, 1),
                             view(l2, h, T, 1, h, 0, 1), gr->w_1, h, (long long)fs * h);
     g.out_f32 = 1;
     GPTL_TRY(run_gemm(g, dt, st));
   }
+  g_tag = GPTL_TAG_B4_DL2;
   {  // dL2 = sum_i dZ_i W1_i  (shard sum in the K loop)
     gptl_operand a = view(dz, fs, T, t, fs, (long long)T * fs, 0);
     a.g_div = kNoGroup; a.k_shard = 1;
@@ -665,9 +753,11 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // ---- LN2 backward + residual: dH = dOut + LNbwd(dL2); also db_o = sum dH
+  g_tag = GPTL_TAG_B6_LN2;
   GPTL_TRY(run_ln_bwd(T, h, dt, dl2, hid, mu2, rs2, W->ln2_g, dy, dhid, gr->ln2_g, gr->ln2_b,
                       gr->b_o, part, st));
   // ---- out-projection (row split)
+  g_tag = GPTL_TAG_B7_DWO;
   {  // dWo_i = dH^T O_i   [t][h][h/t]
     gptl_gemm_desc g = gemm(h, hs, T, t, view(dhid, h, T, 1, h, 0, 1),
                             view(o, hs, T, t, hs, (long long)T * hs, 1), gr->w_o, hs,
@@ -675,6 +765,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     g.out_f32 = 1;
     GPTL_TRY(run_gemm(g, dt, st));
   }
+  g_tag = GPTL_TAG_B7_DO;
   {  // dO_i = dH Wo_i   [t][T][h/t]
     gptl_gemm_desc g = gemm(T, hs, h, t, view(dhid, h, T, 1, h, 0, 0),
                             view(W->w_o, hs, h, t, hs, (long long)h * hs, 1), dO, hs,
@@ -686,6 +777,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   dOv.x_mod = as; dOv.x_mul = d; dOv.g_div = as;
   gptl_operand cv = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 0);
   cv.x_mod = as; cv.x_mul = d; cv.g_div = as;
+  g_tag = GPTL_TAG_B8_DP;
   {  // dP = dO V^T (lower-triangle tiles)
     gptl_operand v = cv;
     v.x_off = 2 * hs;
@@ -693,6 +785,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     g.causal = GPTL_CAUSAL_SKIP_UPPER;
     GPTL_TRY(run_gemm(g, dt, st));
   }
+  g_tag = GPTL_TAG_B8_DV;
   {  // dV = P^T dO  -> V columns of dC
     gptl_operand a = view(pb, s, s, G, s, (long long)s * s, 1);
     gptl_operand b = dOv;
@@ -705,7 +798,9 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // dS = P (dP - rowsum(P dP)) / sqrt(d), in place over dP
+  g_tag = GPTL_TAG_B9_SOFTMAX;
   GPTL_TRY(run_softmax_bwd(G, s, dt, attn_scale, pb, dp, st));
+  g_tag = GPTL_TAG_B10_DQ;
   {  // dQ = dS K  -> Q columns of dC
     gptl_operand a = view(dp, s, s, G, s, (long long)s * s, 0);
     gptl_operand b = cv;
@@ -717,6 +812,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     g.causal = GPTL_CAUSAL_K_BELOW;
     GPTL_TRY(run_gemm(g, dt, st));
   }
+  g_tag = GPTL_TAG_B10_DK;
   {  // dK = dS^T Q  -> K columns of dC
     gptl_operand a = view(dp, s, s, G, s, (long long)s * s, 1);
     gptl_operand b = cv;
@@ -729,13 +825,16 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // ---- QKV (column split)
+  g_tag = GPTL_TAG_B11_DBQKV;
   GPTL_TRY(run_colsum(T, 3 * hs, t, 3 * hs, (long long)T * 3 * hs, dt, dc, gr->b_qkv, part, st));
+  g_tag = GPTL_TAG_B11_DWQKV;
   {  // dWqkv_i = dC_i^T L1   [t][3h/t][h]
     gptl_gemm_desc g = gemm(3 * hs, h, T, t, view(dc, 3 * hs, T, t, 3 * hs, (long long)T * 3 * hs, 1),
                             view(l1, h, T, 1, h, 0, 1), gr->w_qkv, h, (long long)3 * hs * h);
     g.out_f32 = 1;
     GPTL_TRY(run_gemm(g, dt, st));
   }
+  g_tag = GPTL_TAG_B11_DL1;
   {  // dL1 = sum_i dC_i Wqkv_i
     gptl_operand a = view(dc, 3 * hs, T, t, 3 * hs, (long long)T * 3 * hs, 0);
     a.g_div = kNoGroup; a.k_shard = 1;
@@ -746,6 +845,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // ---- LN1 backward + residual: dX = dH + LNbwd(dL1)
+  g_tag = GPTL_TAG_B12_LN1;
   GPTL_TRY(run_ln_bwd(T, h, dt, dl1, x, mu1, rs1, W->ln1_g, dhid, dx, gr->ln1_g, gr->ln1_b,
                       nullptr, part, st));
   return GPTL_OK;
@@ -849,9 +949,11 @@ int gptl_check_overflow(size_t n, const float *grad, gptl_scaler_state *st, gptl
   const long long n4 = (long long)(n / 4);
   long long blocks = (n4 + 255) / 256;
   if (blocks > 4 * sms) blocks = 4 * sms;
+  prof_start(s);
   overflow_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4 *>(grad), n4,
                                                    &st->found_inf);
   GPTL_CK(cudaGetLastError());
+  prof_launched(s, GPTL_KIND_OVERFLOW);
   return GPTL_OK;
 }
 
@@ -867,7 +969,9 @@ int adam_step_fp32_master(size_t n_params, float *master, float *m, float *v, co
     return GPTL_E_ARG;
   int sms = 0;
   GPTL_TRY(device_check(&sms));
+  TagScope tag_scope(GPTL_TAG_O1_OVERFLOW);
   GPTL_TRY(gptl_check_overflow(n_params, grad, st, stream));
+  g_tag = GPTL_TAG_O2_ADAM;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const long long n4 = (long long)(n_params / 4);
   long long blocks = (n4 + 255) / 256;
@@ -884,6 +988,7 @@ int adam_step_fp32_master(size_t n_params, float *master, float *m, float *v, co
         reinterpret_cast<float4 *>(v), reinterpret_cast<const float4 *>(grad),
         static_cast<__nv_bfloat16 *>(w16), n4, a, st);
   GPTL_CK(cudaGetLastError());
+  prof_launched(s, GPTL_KIND_ADAM);
   return GPTL_OK;
 }
 
@@ -894,15 +999,20 @@ int loss_scale_update(gptl_scaler_state *st, int growth_interval, float growth_f
       !(min_scale > 0.f))
     return GPTL_E_ARG;
   GPTL_TRY(device_check());
-  scale_update_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      st, growth_interval, growth_factor, backoff_factor, min_scale);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  TagScope tag_scope(GPTL_TAG_O3_SCALE);
+  prof_start(s);
+  scale_update_kernel<<<1, 32, 0, s>>>(st, growth_interval, growth_factor, backoff_factor,
+                                       min_scale);
   GPTL_CK(cudaGetLastError());
+  prof_launched(s, GPTL_KIND_SCALE);
   return GPTL_OK;
 }
 
 // ---------------------------------------------------------------- parts
 int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream) {
   if (!d) return GPTL_E_NULL;
+  prof_start(reinterpret_cast<cudaStream_t>(stream));
   return run_gemm(*d, dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -914,6 +1024,7 @@ int gptl_layernorm_fwd(int rows, int h, gptl_dtype dtype, const void *x, const v
   if (!aligned16(x) || !aligned16(g) || !aligned16(b) || !aligned16(y)) return GPTL_E_ALIGN;
   if (!(eps > 0.f)) return GPTL_E_ARG;
   GPTL_TRY(device_check());
+  prof_start(reinterpret_cast<cudaStream_t>(stream));
   return run_ln_fwd(rows, h, dtype, x, g, b, eps, y, mu, rstd, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -931,6 +1042,7 @@ int gptl_layernorm_bwd(int rows, int h, gptl_dtype dtype, const void *gy, const 
   if (!aligned16(gy) || !aligned16(x) || !aligned16(g) || !aligned16(resid) || !aligned16(dx) ||
       !aligned16(scratch))
     return GPTL_E_ALIGN;
+  prof_start(reinterpret_cast<cudaStream_t>(stream));
   return run_ln_bwd(rows, h, dtype, gy, x, mu, rstd, g, resid, dx, dg, db, dx_sum,
                     static_cast<float *>(scratch), reinterpret_cast<cudaStream_t>(stream));
 }
@@ -941,6 +1053,7 @@ int gptl_softmax_fwd(long long blocks, int s, gptl_dtype dtype, float scale, voi
   if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
   if (!aligned16(scores)) return GPTL_E_ALIGN;
   GPTL_TRY(device_check());
+  prof_start(reinterpret_cast<cudaStream_t>(stream));
   return run_softmax_fwd(blocks, s, dtype, scale, scores, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -950,6 +1063,7 @@ int gptl_softmax_bwd(long long blocks, int s, gptl_dtype dtype, float scale, con
   if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
   if (!aligned16(prob) || !aligned16(dprob)) return GPTL_E_ALIGN;
   GPTL_TRY(device_check());
+  prof_start(reinterpret_cast<cudaStream_t>(stream));
   return run_softmax_bwd(blocks, s, dtype, scale, prob, dprob, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -963,8 +1077,108 @@ int gptl_colsum(int rows, int n, int groups, long long ld, long long gstride, gp
   if (!a || !out || !scratch) return GPTL_E_NULL;
   if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
   if (!aligned16(a) || !aligned16(scratch)) return GPTL_E_ALIGN;
+  prof_start(reinterpret_cast<cudaStream_t>(stream));
   return run_colsum(rows, n, groups, ld, gstride, dtype, a, out, static_cast<float *>(scratch),
                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------- profiling
+unsigned long long gptl_launch_count(void) { return g_launches; }
+
+int gptl_profile_begin(int capacity) {
+  if (capacity <= 0) return GPTL_E_ARG;
+  if (g_prof.on) return GPTL_E_ARG;
+  g_prof = Profiler();
+  const int pool_n = 2 * capacity + 64;
+  g_prof.pool = static_cast<cudaEvent_t *>(calloc((size_t)pool_n, sizeof(cudaEvent_t)));
+  g_prof.recs = static_cast<ProfRec *>(calloc((size_t)capacity, sizeof(ProfRec)));
+  if (!g_prof.pool || !g_prof.recs) {
+    free(g_prof.pool);
+    free(g_prof.recs);
+    g_prof = Profiler();
+    return GPTL_E_ARG;
+  }
+  for (int i = 0; i < pool_n; ++i) {
+    if (cudaEventCreate(&g_prof.pool[i]) != cudaSuccess) {
+      (void)cudaGetLastError();
+      for (int j = 0; j < i; ++j) cudaEventDestroy(g_prof.pool[j]);
+      free(g_prof.pool);
+      free(g_prof.recs);
+      g_prof = Profiler();
+      return GPTL_E_CUDA;
+    }
+  }
+  g_prof.pool_n = pool_n;
+  g_prof.cap = capacity;
+  g_prof.on = true;
+  return GPTL_OK;
+}
+
+int gptl_profile_end(gptl_launch_record *out, int capacity, int *n_out, long long *dropped) {
+  if (!g_prof.on) return GPTL_E_ARG;
+  int rc = GPTL_OK;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    (void)cudaGetLastError();
+    rc = GPTL_E_CUDA;
+  }
+  int n = 0;
+  for (int i = 0; i < g_prof.n && rc == GPTL_OK; ++i) {
+    if (!out || n >= capacity) break;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, g_prof.recs[i].a, g_prof.recs[i].b) != cudaSuccess) {
+      (void)cudaGetLastError();
+      rc = GPTL_E_CUDA;
+      break;
+    }
+    out[n].kind = g_prof.recs[i].kind;
+    out[n].tag = g_prof.recs[i].tag;
+    out[n].ms = ms;
+    ++n;
+  }
+  if (n_out) *n_out = n;
+  if (dropped) *dropped = g_prof.dropped + (g_prof.n - n);
+  for (int i = 0; i < g_prof.pool_n; ++i) cudaEventDestroy(g_prof.pool[i]);
+  free(g_prof.pool);
+  free(g_prof.recs);
+  g_prof = Profiler();
+  return rc;
+}
+
+const char *gptl_tag_name(int tag) {
+  switch (tag) {
+    case GPTL_TAG_NONE: return "-";
+    case GPTL_TAG_F1_LN1: return "F1 ln1";
+    case GPTL_TAG_F2_QKV: return "F2 qkv";
+    case GPTL_TAG_F3_SCORES: return "F3 scores";
+    case GPTL_TAG_F4_SOFTMAX: return "F4 softmax";
+    case GPTL_TAG_F5_PV: return "F5 pv";
+    case GPTL_TAG_F6_OUTPROJ: return "F6 outproj";
+    case GPTL_TAG_F7_LN2: return "F7 ln2";
+    case GPTL_TAG_F8_FFN1_GELU: return "F8/F9 ffn1+gelu";
+    case GPTL_TAG_F10_FFN2: return "F10 ffn2";
+    case GPTL_TAG_B1_B3_DZ: return "B1/B3 dz";
+    case GPTL_TAG_B2_DW2: return "B2 dw2";
+    case GPTL_TAG_B2_DB2: return "B2 db2";
+    case GPTL_TAG_B3_DB1: return "B3 db1";
+    case GPTL_TAG_B4_DL2: return "B4 dl2";
+    case GPTL_TAG_B5_DW1: return "B5 dw1";
+    case GPTL_TAG_B6_LN2: return "B6 ln2 bwd";
+    case GPTL_TAG_B7_DWO: return "B7 dwo";
+    case GPTL_TAG_B7_DO: return "B7 do";
+    case GPTL_TAG_B8_DP: return "B8 dp";
+    case GPTL_TAG_B8_DV: return "B8 dv";
+    case GPTL_TAG_B9_SOFTMAX: return "B9 softmax bwd";
+    case GPTL_TAG_B10_DQ: return "B10 dq";
+    case GPTL_TAG_B10_DK: return "B10 dk";
+    case GPTL_TAG_B11_DBQKV: return "B11 dbqkv";
+    case GPTL_TAG_B11_DWQKV: return "B11 dwqkv";
+    case GPTL_TAG_B11_DL1: return "B11 dl1";
+    case GPTL_TAG_B12_LN1: return "B12 ln1 bwd";
+    case GPTL_TAG_O1_OVERFLOW: return "O1 overflow";
+    case GPTL_TAG_O2_ADAM: return "O2 adam";
+    case GPTL_TAG_O3_SCALE: return "O3 scale";
+    default: return "?";
+  }
 }
 
 }  // extern "C"

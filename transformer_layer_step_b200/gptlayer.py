@@ -1,5 +1,5 @@
-"""ctypes binding of libgptlayer.so (declared in include/gptlayer.h and
-include/gptlayer_parts.h).
+"""ctypes binding of libgptlayer.so (declared in include/gptlayer.h,
+include/gptlayer_parts.h and include/gptlayer_profile.h).
 
 Argument marshalling only: every computation happens in the library's CUDA
 kernels.  Pointers are passed as integers (or objects with .data_ptr(), such
@@ -67,6 +67,13 @@ class GemmDesc(C.Structure):
                 ("act", C.c_int)]
 
 
+class LaunchRecord(C.Structure):
+    _fields_ = [("kind", C.c_int), ("tag", C.c_int), ("ms", C.c_float)]
+
+
+KIND_NAMES = ("gemm", "ln_fwd", "ln_bwd", "softmax_fwd", "softmax_bwd", "colsum", "reduce",
+              "overflow", "adam", "scale")
+
 _lib = None
 
 _SIGS = {
@@ -99,6 +106,11 @@ _SIGS = {
     "gptl_colsum_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "gptl_colsum": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_longlong, C.c_longlong, C.c_int,
                               C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "gptl_launch_count": (C.c_ulonglong, []),
+    "gptl_profile_begin": (C.c_int, [C.c_int]),
+    "gptl_profile_end": (C.c_int, [C.POINTER(LaunchRecord), C.c_int, C.POINTER(C.c_int),
+                                   C.POINTER(C.c_longlong)]),
+    "gptl_tag_name": (C.c_char_p, [C.c_int]),
 }
 
 
@@ -250,3 +262,23 @@ def read_device_error(clear: bool = True) -> int:
     w = C.c_int()
     _check(lib().gptl_read_device_error(C.byref(w), 1 if clear else 0), "gptl_read_device_error")
     return w.value
+
+
+def launch_count() -> int:
+    """Kernels launched through the library by this process so far."""
+    return int(lib().gptl_launch_count())
+
+
+def profile_begin(capacity: int):
+    _check(lib().gptl_profile_begin(capacity), "gptl_profile_begin")
+
+
+def profile_end(capacity: int):
+    """Closes the profiling window; returns ([(kind_name, tag_name, ms)], dropped)."""
+    recs = (LaunchRecord * capacity)()
+    n, dropped = C.c_int(), C.c_longlong()
+    _check(lib().gptl_profile_end(recs, capacity, C.byref(n), C.byref(dropped)),
+           "gptl_profile_end")
+    out = [(KIND_NAMES[r.kind], lib().gptl_tag_name(r.tag).decode(), float(r.ms))
+           for r in recs[:n.value]]
+    return out, int(dropped.value)
