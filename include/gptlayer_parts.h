@@ -46,11 +46,13 @@ enum {
  * for m < M, n < N, G < groups, with fp32 accumulation in tensor memory.
  * Output element (m, n) of group G is at
  *   out + (G % o_mod)*o_str_mod + (G / o_mod)*o_str_div + m*ldo + n.
- * Epilogue, in order: + bias[G*bias_g_stride + n] (if bias), + resid[m*ld_resid
- * + n] (if resid), then act: GELU writes the value to out and GeLU(value) to
- * out2; DGELU multiplies by GeLU'(aux at the output's index).  out_f32 = 1
- * stores the raw fp32 sum (no bias/resid/act).  Requirements: K % 16 == 0,
- * N % 16 == 0, all offsets/pitches multiples of 8 elements. */
+ * Epilogue, in order: + bias[G*bias_g_stride + n] (if bias, 16-bit),
+ * + resid[m*ld_resid + n] (if resid; fp32 when resid_f32, else 16-bit), then
+ * act: GELU writes the value to out and GeLU(value) to out2; DGELU multiplies
+ * by GeLU'(aux at the output's index).  out_f32 = 1 stores the fp32 value
+ * (act must be GPTL_ACT_NONE); otherwise out is 16-bit, rounded to nearest
+ * even.  Requirements: K % 16 == 0, N % 16 == 0, all offsets/pitches
+ * multiples of 8 elements. */
 typedef struct {
   int M, N, K, groups, k_shards, causal;
   gptl_operand a, b;
@@ -66,6 +68,7 @@ typedef struct {
   const void *aux;
   void *out2;
   int act;
+  int resid_f32;
 } gptl_gemm_desc;
 
 int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream);

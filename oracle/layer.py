@@ -22,12 +22,15 @@ precision defines it ("Megatron-LM overview", §3.1: FP16 matrix math; the
 layer computes in fp16/bf16): every activation tensor that one step of the
 path hands to the next is held in the 16-bit type (round to nearest, ties to
 even), while the arithmetic inside a step stays exact.  The stored tensors
-are, forward: L1, C = [Q|K|V], the raw scores S = Q K^T, P, O, H, L2, Z,
+are, forward: L1, C = [Q|K|V], the raw scores S = Q K^T, P, O, L2, Z,
 A = gelu(Z); backward: dZ (the GeLU backward is applied to dOut W2 before
-the store, as the fused bias-GeLU's backward), dL2, dH, dO, dP, dV, dS, dQ,
-dK, dL1.  The layer outputs Out and dX are returned unrounded (their own
-store is the caller's last rounding) and the weight and bias gradients are
-fp32 quantities, returned exactly.
+the store, as the fused bias-GeLU's backward), dL2, dO, dP, dV, dS, dQ, dK,
+dL1, and the 16-bit copy of dH that the out-projection's backward GEMMs
+read.  The residual stream H = X + attention and its gradient dH are the
+FP32 side of mixed precision (like the master weights, they are never
+matrix operands): they stay exact here.  The layer outputs Out and dX are
+returned unrounded (their own store is the caller's last rounding) and the
+weight and bias gradients are fp32 quantities, returned exactly.
 """
 from __future__ import annotations
 
@@ -88,18 +91,27 @@ def causal_softmax(z: np.ndarray) -> np.ndarray:
     return p
 
 
-def attention_head_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, precision=None):
+def attention_head_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, precision=None, noise=None):
     """One (batch, head) block of causal self-attention: returns (P, O).
     With a 16-bit precision the raw scores Q K^T and P are stored values."""
     d = q.shape[1]
-    z = _store(q @ k.T, precision) / math.sqrt(d)
-    p = _store(causal_softmax(z), precision)
+    z = _store(q @ k.T, precision, noise) / math.sqrt(d)
+    p = _store(causal_softmax(z), precision, noise)
     return p, p @ v
 
 
-def _store(a: np.ndarray, precision):
-    """An activation tensor as the next step reads it (see the module doc)."""
-    return a if precision is None else round_to_16(a, precision)
+def _store(a: np.ndarray, precision, noise=None):
+    """An activation tensor as the next step reads it (see the module doc).
+    `noise`, when given, is applied to the value just before it is rounded:
+    a callable that returns the value times (1 + a small relative error),
+    standing for the rounding of a fp32-accumulating implementation, so that
+    a test can measure how far two correct implementations of the 16-bit
+    method drift apart."""
+    if precision is None:
+        return a
+    if noise is not None:
+        a = noise(a)
+    return round_to_16(a, precision)
 
 
 def _check(dims, params):
@@ -112,10 +124,12 @@ def _check(dims, params):
     return b, s, h, a, f, t
 
 
-def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precision=None):
+def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precision=None,
+              noise=None):
     """Forward pass.  x: [T, h] float64.  precision: None (exact) or the
-    16-bit type the activations are stored in.  Returns (out, cache)."""
-    st = lambda a: _store(a, precision)
+    16-bit type the activations are stored in; noise: see _store.
+    Returns (out, cache)."""
+    st = lambda a: _store(a, precision, noise)
     b, s, h, a, f, t = _check(dims, params)
     d = h // a
     hs, a_s = h // t, a // t            # hidden columns and heads per shard
@@ -140,7 +154,7 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precis
                 qh = c[i, rows, 0 * hs:1 * hs][:, cols]
                 kh = c[i, rows, 1 * hs:2 * hs][:, cols]
                 vh = c[i, rows, 2 * hs:3 * hs][:, cols]
-                pr, oh = attention_head_fwd(qh, kh, vh, precision)
+                pr, oh = attention_head_fwd(qh, kh, vh, precision, noise)
                 probs[i, j, eta] = pr
                 o[i, rows, cols] = st(oh)
 
@@ -149,7 +163,7 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precis
     y_attn = np.zeros((T, h))
     for i in range(t):
         y_attn += o[i] @ params["w_o"][i].T
-    hid = st(x + y_attn + params["b_o"][None, :])
+    hid = x + y_attn + params["b_o"][None, :]
 
     # 5. LN2
     l2, mu2, rstd2, xhat2 = layer_norm_fwd(hid, params["ln2_g"], params["ln2_b"], eps)
@@ -167,7 +181,7 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precis
 
     cache = dict(x=x, l1=l1, mu1=mu1, rstd1=rstd1, xhat1=xhat1, c=c, probs=probs, o=o,
                  hid=hid, l2=l2, mu2=mu2, rstd2=rstd2, xhat2=xhat2, z=z, act=act,
-                 precision=precision)
+                 precision=precision, noise=noise)
     return out, cache
 
 
@@ -179,7 +193,7 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
     hs, a_s = h // t, a // t
     T = b * s
     inv_sqrt_d = 1.0 / math.sqrt(d)
-    st = lambda a: _store(a, cache.get("precision"))
+    st = lambda a: _store(a, cache.get("precision"), cache.get("noise"))
     gr = {}
 
     # FFN2 (row split): each shard's weight gradient and input gradient
@@ -200,12 +214,13 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
     # LN2 backward plus the residual path
     dln, gr["ln2_g"], gr["ln2_b"] = layer_norm_bwd(dl2, cache["xhat2"], cache["rstd2"],
                                                    params["ln2_g"])
-    dhid = st(dout + dln)
+    dhid = dout + dln
+    dhid16 = st(dhid)                   # the matrix operand copy of dH
 
     # out-projection (row split)
     gr["b_o"] = dhid.sum(axis=0)
-    gr["w_o"] = np.stack([dhid.T @ cache["o"][i] for i in range(t)])
-    do = st(np.stack([dhid @ params["w_o"][i] for i in range(t)]))
+    gr["w_o"] = np.stack([dhid16.T @ cache["o"][i] for i in range(t)])
+    do = st(np.stack([dhid16 @ params["w_o"][i] for i in range(t)]))
 
     # attention backward, head by head
     c = cache["c"]

@@ -14,54 +14,74 @@
 namespace gptl {
 
 // ------------------------------------------------------------ team reduce
-// A "team" of TPR consecutive threads owns one row.  TPR is a power of two;
-// teams wider than a warp combine their warps through shared memory.
-template <int TPR>
-__device__ __forceinline__ float team_sum(float v, float *red) {
-#pragma unroll
-  for (int o = (TPR < 32 ? TPR : 32) / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if constexpr (TPR > 32) {
-    constexpr int W = TPR / 32;
+// A "team" of tpr consecutive threads owns one row (tpr a power of two, at
+// most the block size).  Teams wider than a warp combine their warps through
+// shared memory; then every thread of the block must call this together.
+__device__ __forceinline__ float team_sum(float v, float *red, int tpr) {
+  const int w = tpr < 32 ? tpr : 32;
+  for (int o = w / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (tpr > 32) {
+    const int nw = tpr / 32;
     const int lane = threadIdx.x & 31;
-    const int wit = (threadIdx.x / 32) % W;             // warp index within the team
-    const int team = threadIdx.x / TPR;
+    const int wit = (threadIdx.x / 32) % nw;             // warp index within the team
+    const int team = threadIdx.x / tpr;
     __syncthreads();
-    if (lane == 0) red[team * W + wit] = v;
+    if (lane == 0) red[team * nw + wit] = v;
     __syncthreads();
     float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < W; ++i) s += red[team * W + i];
+    for (int i = 0; i < nw; ++i) s += red[team * nw + i];
     v = s;
   }
   return v;
 }
 
+// ------------------------------------------------------------ row vectors
+// 8 consecutive elements of a row, from a 16-bit tensor (one 16-byte load) or
+// from an fp32 tensor (two 16-byte loads); `v` indexes 8-element vectors.
+template <typename S, typename T>
+__device__ __forceinline__ void load_vec8(const S *base, long long v, float (&f)[8]) {
+  if constexpr (sizeof(S) == 4) {
+    const float4 a = reinterpret_cast<const float4 *>(base)[2 * v];
+    const float4 b = reinterpret_cast<const float4 *>(base)[2 * v + 1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  } else {
+    unpack8<T>(reinterpret_cast<const uint4 *>(base)[v], f);
+  }
+}
+
+__device__ __forceinline__ void store_vec8_f32(float *base, long long v, const float (&f)[8]) {
+  reinterpret_cast<float4 *>(base)[2 * v] = make_float4(f[0], f[1], f[2], f[3]);
+  reinterpret_cast<float4 *>(base)[2 * v + 1] = make_float4(f[4], f[5], f[6], f[7]);
+}
+
 // ------------------------------------------------------------ LayerNorm fwd
 // y = gamma * (x - mu) * rstd + beta, biased variance, fp32 statistics saved.
-// Each thread holds VPT 16-byte vectors of its row in registers.
-template <typename T, int TPR, int VPT>
-__global__ void __launch_bounds__(256) ln_fwd_kernel(const T *__restrict__ x,
+// x is 16-bit (TX = T) or fp32 (TX = float, the residual stream); y is T.
+// Each thread holds VPT 8-element vectors of its row in registers.
+template <typename T, typename TX, int VPT>
+__global__ void __launch_bounds__(256) ln_fwd_kernel(const TX *__restrict__ x,
                                                      const T *__restrict__ gamma,
                                                      const T *__restrict__ beta, T *__restrict__ y,
                                                      float *__restrict__ mu_out,
                                                      float *__restrict__ rstd_out, int rows, int h,
-                                                     float eps) {
+                                                     float eps, int tpr) {
   __shared__ float red[256 / 32 + 8];
-  constexpr int RPB = 256 / TPR;
+  const int RPB = blockDim.x / tpr;
+  const int TPR = tpr;
   const int team = threadIdx.x / TPR, tl = threadIdx.x % TPR;
   const int row = blockIdx.x * RPB + team;
   const bool active = row < rows;
   const int r = active ? row : rows - 1;
-  const uint4 *xr = reinterpret_cast<const uint4 *>(x + (long long)r * h);
+  const TX *xr = x + (long long)r * h;
   float v[VPT][8];
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
-    unpack8<T>(xr[tl + i * TPR], v[i]);
+    load_vec8<TX, T>(xr, tl + i * TPR, v[i]);
 #pragma unroll
     for (int e = 0; e < 8; ++e) s += v[i][e];
   }
-  const float mu = team_sum<TPR>(s, red) / (float)h;
+  const float mu = team_sum(s, red, TPR) / (float)h;
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < VPT; ++i)
@@ -70,7 +90,7 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const T *__restrict__ x,
       const float d = v[i][e] - mu;
       ss += d * d;
     }
-  const float var = team_sum<TPR>(ss, red) / (float)h;
+  const float var = team_sum(ss, red, TPR) / (float)h;
   const float rstd = 1.0f / sqrtf(var + eps);
   if (!active) return;
   const uint4 *g4 = reinterpret_cast<const uint4 *>(gamma);
@@ -93,26 +113,39 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const T *__restrict__ x,
 
 // ------------------------------------------------------------ LayerNorm bwd
 // dx = resid + rstd * (gh - mean(gh) - xhat * mean(gh * xhat)), gh = gy * gamma.
-// Per-block partial column sums of gy*xhat (dgamma), gy (dbeta) and, when
-// requested, of dx itself (the next bias gradient) go to `part`
-// ([nparts][gridDim.x][h]); reduce_parts_kernel finishes them.
-template <typename T, int TPR, int VPT>
+// x is 16-bit or fp32 (TX), resid 16-bit or fp32 (TR); dx is written as T
+// and, with D32, also in fp32 to dx32 (the residual stream).  Per-block
+// partial column sums go to `part` ([nparts][gridDim.x][h]) in this order:
+// gy*xhat (dgamma), gy (dbeta), then dx if SUM_DX (the fp32 value with D32,
+// else the stored 16-bit value), then resid if SUM_RESID.
+// reduce_parts_kernel finishes them.
+template <typename T, typename TX, typename TR, bool D32, bool SUM_DX, bool SUM_RESID, int VPT>
 __global__ void __launch_bounds__(256) ln_bwd_kernel(
-    const T *__restrict__ gy, const T *__restrict__ x, const float *__restrict__ mu_in,
-    const float *__restrict__ rstd_in, const T *__restrict__ gamma, const T *__restrict__ resid,
-    T *__restrict__ dx, float *__restrict__ part, int rows, int h, int want_dx_sum) {
+    const T *__restrict__ gy, const TX *__restrict__ x, const float *__restrict__ mu_in,
+    const float *__restrict__ rstd_in, const T *__restrict__ gamma, const TR *__restrict__ resid,
+    T *__restrict__ dx, float *__restrict__ dx32, float *__restrict__ part, int rows, int h,
+    int tpr) {
   extern __shared__ float sm[];          // [RPB][h] staging for the column partials
   __shared__ float red[256 / 32 + 8];
-  constexpr int RPB = 256 / TPR;
+  const int TPR = tpr;
+  const int RPB = blockDim.x / tpr;
   const int team = threadIdx.x / TPR, tl = threadIdx.x % TPR;
-  float pg[VPT][8], pb[VPT][8], pd[VPT][8];
+  float pg[VPT][8], pb[VPT][8], pd[SUM_DX ? VPT : 1][8], pr[SUM_RESID ? VPT : 1][8];
   float gm[VPT][8];
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(gamma) + tl + i * TPR), gm[i]);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) pg[i][e] = pb[i][e] = pd[i][e] = 0.f;
+    for (int e = 0; e < 8; ++e) pg[i][e] = pb[i][e] = 0.f;
   }
+#pragma unroll
+  for (int i = 0; i < (SUM_DX ? VPT : 1); ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pd[i][e] = 0.f;
+#pragma unroll
+  for (int i = 0; i < (SUM_RESID ? VPT : 1); ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pr[i][e] = 0.f;
   const int row_step = gridDim.x * RPB;
   // every team runs the same number of iterations (the team reductions
   // synchronise the whole block when TPR > 32)
@@ -122,7 +155,7 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(
     const bool active = row < rows;
     const int r = active ? row : rows - 1;
     const uint4 *gr = reinterpret_cast<const uint4 *>(gy + (long long)r * h);
-    const uint4 *xr = reinterpret_cast<const uint4 *>(x + (long long)r * h);
+    const TX *xr = x + (long long)r * h;
     const float mu = mu_in[r], rstd = rstd_in[r];
     float xh[VPT][8], gh[VPT][8], g[VPT][8];
     float s1 = 0.f, s2 = 0.f;
@@ -130,7 +163,7 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(
     for (int i = 0; i < VPT; ++i) {
       float xv[8];
       unpack8<T>(gr[tl + i * TPR], g[i]);
-      unpack8<T>(xr[tl + i * TPR], xv);
+      load_vec8<TX, T>(xr, tl + i * TPR, xv);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         xh[i][e] = (xv[e] - mu) * rstd;
@@ -139,39 +172,60 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(
         s2 += gh[i][e] * xh[i][e];
       }
     }
-    const float m1 = team_sum<TPR>(s1, red) / (float)h;
-    const float m2 = team_sum<TPR>(s2, red) / (float)h;
+    const float m1 = team_sum(s1, red, TPR) / (float)h;
+    const float m2 = team_sum(s2, red, TPR) / (float)h;
     if (active) {
-      const uint4 *rr = reinterpret_cast<const uint4 *>(resid + (long long)r * h);
+      const TR *rr = resid + (long long)r * h;
       uint4 *dr = reinterpret_cast<uint4 *>(dx + (long long)r * h);
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
         float rv[8], o[8];
-        unpack8<T>(rr[tl + i * TPR], rv);
+        load_vec8<TR, T>(rr, tl + i * TPR, rv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) o[e] = rv[e] + rstd * (gh[i][e] - m1 - xh[i][e] * m2);
         const uint4 q = pack8<T>(o);
         dr[tl + i * TPR] = q;
-        float oq[8];
-        unpack8<T>(q, oq);                 // sum what was stored
+        if constexpr (D32) store_vec8_f32(dx32 + (long long)r * h, tl + i * TPR, o);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           pg[i][e] += g[i][e] * xh[i][e];
           pb[i][e] += g[i][e];
-          pd[i][e] += oq[e];
+        }
+        if constexpr (SUM_DX) {
+          float oq[8];
+          if constexpr (D32) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) oq[e] = o[e];
+          } else {
+            unpack8<T>(q, oq);             // sum what was stored
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pd[i][e] += oq[e];
+        }
+        if constexpr (SUM_RESID) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pr[i][e] += rv[e];
         }
       }
     }
   }
   // combine the RPB teams of this block, one partial array at a time
-  const int nparts = want_dx_sum ? 3 : 2;
+  constexpr int nparts = 2 + (SUM_DX ? 1 : 0) + (SUM_RESID ? 1 : 0);
+#pragma unroll
   for (int k = 0; k < nparts; ++k) {
+    const int which = k < 2 ? k : (k == 2 && SUM_DX ? 2 : 3);
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < VPT; ++i)
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        sm[team * h + (tl + i * TPR) * 8 + e] = (k == 0 ? pg[i][e] : (k == 1 ? pb[i][e] : pd[i][e]));
+      for (int e = 0; e < 8; ++e) {
+        float val;
+        if (which == 0) val = pg[i][e];
+        else if (which == 1) val = pb[i][e];
+        else if (which == 2) val = pd[SUM_DX ? i : 0][e];
+        else val = pr[SUM_RESID ? i : 0][e];
+        sm[team * h + (tl + i * TPR) * 8 + e] = val;
+      }
     __syncthreads();
     float *dst = part + ((long long)k * gridDim.x + blockIdx.x) * h;
     for (int c = threadIdx.x; c < h; c += blockDim.x) {
@@ -182,16 +236,29 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(
   }
 }
 
-// out[k][c] = sum_b part[k][b][c], for k < nk arrays of width n.
-__global__ void reduce_parts_kernel(const float *__restrict__ part, int nblocks, int n,
-                                    float *out0, float *out1, float *out2) {
+// out_k[c] = sum_b part[k][b][c] for the nk = gridDim.y arrays of width n.
+// Block: 32 columns x 16 row groups; fixed summation order (deterministic).
+struct PartOuts {
+  float *o[4];
+};
+__global__ void __launch_bounds__(512) reduce_parts_kernel(const float *__restrict__ part,
+                                                           int nblocks, int n, PartOuts outs) {
+  __shared__ float sm[16][33];
   const int k = blockIdx.y;
-  float *out = k == 0 ? out0 : (k == 1 ? out1 : out2);
+  const int c = blockIdx.x * 32 + threadIdx.x;
   const float *src = part + (long long)k * nblocks * n;
-  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < n; c += gridDim.x * blockDim.x) {
-    float s = 0.f;
-    for (int b = 0; b < nblocks; ++b) s += src[(long long)b * n + c];
-    out[c] = s;
+  float s = 0.f;
+  if (c < n) {
+#pragma unroll 4
+    for (int b = threadIdx.y; b < nblocks; b += 16) s += src[(long long)b * n + c];
+  }
+  sm[threadIdx.y][threadIdx.x] = s;
+  __syncthreads();
+  if (threadIdx.y == 0 && c < n) {
+    float t = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) t += sm[i][threadIdx.x];
+    outs.o[k][c] = t;
   }
 }
 

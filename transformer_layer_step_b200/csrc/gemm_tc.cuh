@@ -61,6 +61,7 @@ struct alignas(64) GemmParams {
   long long bias_g_stride;
   const void *resid;
   long long ld_resid;
+  int resid_f32;
   const void *aux;
   void *out2;
   int act;
@@ -134,12 +135,6 @@ __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int r
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
   const long long off = (long long)(g % p.o_mod) * p.o_str_mod +
                         (long long)(g / p.o_mod) * p.o_str_div + (long long)row * p.ldo + n;
-  if (p.out_f32) {
-    float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    return;
-  }
   if (p.bias) {
     const uint4 *b = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.bias) +
                                                      (long long)g * p.bias_g_stride + n);
@@ -152,15 +147,31 @@ __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int r
     }
   }
   if (p.resid) {
-    const uint4 *rr = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.resid) +
-                                                      (long long)row * p.ld_resid + n);
+    if (p.resid_f32) {
+      const float4 *rr = reinterpret_cast<const float4 *>(static_cast<const float *>(p.resid) +
+                                                          (long long)row * p.ld_resid + n);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float f[8];
-      unpack8<T>(rr[h], f);
+      for (int q = 0; q < 4; ++q) {
+        const float4 f = rr[q];
+        v[4 * q] += f.x; v[4 * q + 1] += f.y; v[4 * q + 2] += f.z; v[4 * q + 3] += f.w;
+      }
+    } else {
+      const uint4 *rr = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.resid) +
+                                                        (long long)row * p.ld_resid + n);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[8 * h + i] += f[i];
+      for (int h = 0; h < 2; ++h) {
+        float f[8];
+        unpack8<T>(rr[h], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[8 * h + i] += f[i];
+      }
     }
+  }
+  if (p.out_f32) {
+    float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    return;
   }
   uint4 *o = reinterpret_cast<uint4 *>(static_cast<T *>(p.out) + off);
   if (p.act == kActGelu) {

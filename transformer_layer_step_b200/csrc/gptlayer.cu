@@ -232,7 +232,7 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   if (d.act == GPTL_ACT_GELU && !d.out2) return GPTL_E_NULL;
   if (d.act == GPTL_ACT_DGELU && !d.aux) return GPTL_E_NULL;
   if ((d.out2 && !aligned16(d.out2)) || (d.aux && !aligned16(d.aux))) return GPTL_E_ALIGN;
-  if (d.act < 0 || d.act > 2) return GPTL_E_SHAPE;
+  if (d.act < 0 || d.act > 2 || (d.out_f32 && d.act != GPTL_ACT_NONE)) return GPTL_E_SHAPE;
   GPTL_TRY(check_operand(d.a));
   GPTL_TRY(check_operand(d.b));
 
@@ -285,13 +285,14 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.o_str_mod = d.o_str_mod;
   p.o_str_div = d.o_str_div;
   p.out_f32 = d.out_f32;
-  p.bias = d.out_f32 ? nullptr : d.bias;
+  p.bias = d.bias;
   p.bias_g_stride = d.bias_g_stride;
-  p.resid = d.out_f32 ? nullptr : d.resid;
+  p.resid = d.resid;
+  p.resid_f32 = d.resid_f32 ? 1 : 0;
   p.ld_resid = d.ld_resid;
   p.aux = d.aux;
   p.out2 = d.out2;
-  p.act = d.out_f32 ? 0 : d.act;
+  p.act = d.act;
   const int grid = (int)(p.total_tiles < sms ? p.total_tiles : sms);
   if (dt == GPTL_FP16) return launch_gemm_t<__half>(p, grid, smem, stream);
   return launch_gemm_t<__nv_bfloat16>(p, grid, smem, stream);
@@ -311,44 +312,20 @@ bool ln_split(int h, int *tpr, int *vpt) {
   return false;
 }
 
-template <typename T, int TPR, int VPT>
-void ln_fwd_launch(int rows, int h, const void *x, const void *g, const void *b, float eps,
-                   void *y, float *mu, float *rstd, cudaStream_t st) {
-  constexpr int RPB = 256 / TPR;
-  ln_fwd_kernel<T, TPR, VPT><<<(rows + RPB - 1) / RPB, 256, 0, st>>>(
-      (const T *)x, (const T *)g, (const T *)b, (T *)y, mu, rstd, rows, h, eps);
-}
-
-template <typename T, int TPR, int VPT>
-int ln_bwd_launch(int rows, int h, const void *gy, const void *x, const float *mu,
-                  const float *rstd, const void *g, const void *resid, void *dx, float *part,
-                  int nblocks, int want_sum, cudaStream_t st) {
-  constexpr int RPB = 256 / TPR;
-  const int smem = RPB * h * (int)sizeof(float);
-  if (smem > 48 * 1024)
-    GPTL_CK(cudaFuncSetAttribute(ln_bwd_kernel<T, TPR, VPT>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  ln_bwd_kernel<T, TPR, VPT><<<nblocks, 256, smem, st>>>((const T *)gy, (const T *)x, mu, rstd,
-                                                         (const T *)g, (const T *)resid, (T *)dx,
-                                                         part, rows, h, want_sum);
-  return GPTL_OK;
-}
-
-// Calls f.template operator()<TPR, VPT>() for the runtime split.
+// Calls f.template operator()<VPT>() for the runtime vectors-per-thread.
 template <typename F>
-bool ln_dispatch(int tpr, int vpt, F &&f) {
-#define GPTL_LN_CASE(TP, VP)                 \
-  if (tpr == TP && vpt == VP) {              \
-    f.template operator()<TP, VP>();         \
-    return true;                             \
+bool ln_dispatch(int vpt, F &&f) {
+  switch (vpt) {
+    case 1: f.template operator()<1>(); return true;
+    case 2: f.template operator()<2>(); return true;
+    case 3: f.template operator()<3>(); return true;
+    case 4: f.template operator()<4>(); return true;
+    case 5: f.template operator()<5>(); return true;
+    case 6: f.template operator()<6>(); return true;
+    case 7: f.template operator()<7>(); return true;
+    case 8: f.template operator()<8>(); return true;
+    default: return false;
   }
-#define GPTL_LN_ROW(TP) \
-  GPTL_LN_CASE(TP, 1) GPTL_LN_CASE(TP, 2) GPTL_LN_CASE(TP, 3) GPTL_LN_CASE(TP, 4) \
-  GPTL_LN_CASE(TP, 5) GPTL_LN_CASE(TP, 6) GPTL_LN_CASE(TP, 7) GPTL_LN_CASE(TP, 8)
-  GPTL_LN_ROW(16) GPTL_LN_ROW(32) GPTL_LN_ROW(64) GPTL_LN_ROW(128) GPTL_LN_ROW(256)
-#undef GPTL_LN_ROW
-#undef GPTL_LN_CASE
-  return false;
 }
 
 int ln_bwd_blocks(int rows, int h, int sms) {
@@ -361,15 +338,25 @@ int ln_bwd_blocks(int rows, int h, int sms) {
   return nb;
 }
 
-int run_ln_fwd(int rows, int h, gptl_dtype dt, const void *x, const void *g, const void *b,
-               float eps, void *y, float *mu, float *rstd, cudaStream_t st) {
+// LayerNorm forward; x is 16-bit, or fp32 when x_f32.
+int run_ln_fwd(int rows, int h, gptl_dtype dt, const void *x, int x_f32, const void *g,
+               const void *b, float eps, void *y, float *mu, float *rstd, cudaStream_t st) {
   int tpr = 0, vpt = 0;
   if (!ln_split(h, &tpr, &vpt) || rows <= 0) return GPTL_E_SHAPE;
-  const bool ok = ln_dispatch(tpr, vpt, [&]<int TP, int VP>() {
-    if (dt == GPTL_FP16)
-      ln_fwd_launch<__half, TP, VP>(rows, h, x, g, b, eps, y, mu, rstd, st);
-    else
-      ln_fwd_launch<__nv_bfloat16, TP, VP>(rows, h, x, g, b, eps, y, mu, rstd, st);
+  const int rpb = 256 / tpr;
+  const unsigned grid = (unsigned)((rows + rpb - 1) / rpb);
+  const bool ok = ln_dispatch(vpt, [&]<int VP>() {
+    auto go = [&]<typename T>() {
+      if (x_f32)
+        ln_fwd_kernel<T, float, VP><<<grid, 256, 0, st>>>((const float *)x, (const T *)g,
+                                                          (const T *)b, (T *)y, mu, rstd, rows,
+                                                          h, eps, tpr);
+      else
+        ln_fwd_kernel<T, T, VP><<<grid, 256, 0, st>>>((const T *)x, (const T *)g, (const T *)b,
+                                                      (T *)y, mu, rstd, rows, h, eps, tpr);
+    };
+    if (dt == GPTL_FP16) go.template operator()<__half>();
+    else go.template operator()<__nv_bfloat16>();
   });
   if (!ok) return GPTL_E_SHAPE;
   GPTL_CK(cudaGetLastError());
@@ -377,32 +364,62 @@ int run_ln_fwd(int rows, int h, gptl_dtype dt, const void *x, const void *g, con
   return GPTL_OK;
 }
 
-int run_ln_bwd(int rows, int h, gptl_dtype dt, const void *gy, const void *x, const float *mu,
-               const float *rstd, const void *g, const void *resid, void *dx, float *dg, float *db,
-               float *dx_sum, float *part, cudaStream_t st) {
+int launch_reduce_parts(const float *part, int nblocks, int n, int nk, float *o0, float *o1,
+                        float *o2, float *o3, cudaStream_t st) {
+  PartOuts outs{{o0, o1, o2, o3}};
+  reduce_parts_kernel<<<dim3((n + 31) / 32, nk), dim3(32, 16), 0, st>>>(part, nblocks, n, outs);
+  GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_REDUCE);
+  return GPTL_OK;
+}
+
+// LayerNorm backward in the three arrangements the library uses:
+//   LNB_PARTS : x, resid 16-bit; dx 16-bit; sums dg, db [, dx];
+//   LNB_H     : x fp32 (the residual stream H), resid 16-bit (dOut); dx written
+//               16-bit and fp32; sums dg, db, dx (fp32 value), resid;
+//   LNB_X     : x 16-bit (the layer input), resid fp32 (dH); dx 16-bit; sums dg, db.
+enum { LNB_PARTS = 0, LNB_H = 1, LNB_X = 2 };
+
+int run_ln_bwd(int variant, int rows, int h, gptl_dtype dt, const void *gy, const void *x,
+               const float *mu, const float *rstd, const void *g, const void *resid, void *dx,
+               float *dx32, float *dg, float *db, float *dx_sum, float *resid_sum, float *part,
+               cudaStream_t st) {
   int sms = 0;
   GPTL_TRY(device_check(&sms));
   int tpr = 0, vpt = 0;
   if (!ln_split(h, &tpr, &vpt) || rows <= 0) return GPTL_E_SHAPE;
   const int nb = ln_bwd_blocks(rows, h, sms);
-  const int want = dx_sum ? 1 : 0;
+  const int smem = (256 / tpr) * h * (int)sizeof(float);
   int rc = GPTL_OK;
-  const bool ok = ln_dispatch(tpr, vpt, [&]<int TP, int VP>() {
-    if (dt == GPTL_FP16)
-      rc = ln_bwd_launch<__half, TP, VP>(rows, h, gy, x, mu, rstd, g, resid, dx, part, nb, want, st);
-    else
-      rc = ln_bwd_launch<__nv_bfloat16, TP, VP>(rows, h, gy, x, mu, rstd, g, resid, dx, part, nb,
-                                                want, st);
+  const bool ok = ln_dispatch(vpt, [&]<int VP>() {
+    auto go = [&]<typename T, typename TX, typename TR, bool D32, bool SDX, bool SRS>() {
+      auto kern = ln_bwd_kernel<T, TX, TR, D32, SDX, SRS, VP>;
+      if (smem > 48 * 1024 &&
+          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+              cudaSuccess) {
+        (void)cudaGetLastError();
+        rc = GPTL_E_CUDA;
+        return;
+      }
+      kern<<<nb, 256, smem, st>>>((const T *)gy, (const TX *)x, mu, rstd, (const T *)g,
+                                  (const TR *)resid, (T *)dx, dx32, part, rows, h, tpr);
+    };
+    auto by_variant = [&]<typename T>() {
+      if (variant == LNB_H) go.template operator()<T, float, T, true, true, true>();
+      else if (variant == LNB_X) go.template operator()<T, T, float, false, false, false>();
+      else if (dx_sum) go.template operator()<T, T, T, false, true, false>();
+      else go.template operator()<T, T, T, false, false, false>();
+    };
+    if (dt == GPTL_FP16) by_variant.template operator()<__half>();
+    else by_variant.template operator()<__nv_bfloat16>();
   });
   if (!ok) return GPTL_E_SHAPE;
   GPTL_TRY(rc);
   GPTL_CK(cudaGetLastError());
   prof_launched(st, GPTL_KIND_LN_BWD);
-  dim3 rg((h + 255) / 256, 2 + want);
-  reduce_parts_kernel<<<rg, 256, 0, st>>>(part, nb, h, dg, db, dx_sum);
-  GPTL_CK(cudaGetLastError());
-  prof_launched(st, GPTL_KIND_REDUCE);
-  return GPTL_OK;
+  if (variant == LNB_H) return launch_reduce_parts(part, nb, h, 4, dg, db, dx_sum, resid_sum, st);
+  if (variant == LNB_X) return launch_reduce_parts(part, nb, h, 2, dg, db, nullptr, nullptr, st);
+  return launch_reduce_parts(part, nb, h, dx_sum ? 3 : 2, dg, db, dx_sum, nullptr, st);
 }
 
 // ------------------------------------------------------------- softmax
@@ -476,11 +493,7 @@ int run_colsum(int rows, int n, int groups, long long ld, long long gstride, gpt
   GPTL_CK(cudaGetLastError());
   prof_launched(st, GPTL_KIND_COLSUM);
   const int width = n * groups;
-  reduce_parts_kernel<<<dim3((width + 255) / 256, 1), 256, 0, st>>>(part, split, width, out,
-                                                                    nullptr, nullptr);
-  GPTL_CK(cudaGetLastError());
-  prof_launched(st, GPTL_KIND_REDUCE);
-  return GPTL_OK;
+  return launch_reduce_parts(part, split, width, 1, out, nullptr, nullptr, nullptr, st);
 }
 
 // ------------------------------------------------------------- the layer
@@ -515,7 +528,7 @@ struct Ws {
   // saved (fwd -> bwd)
   size_t mu1, rstd1, mu2, rstd2, l1, c, p, o, hid, l2, z, act, saved;
   // scratch (bwd)
-  size_t dz, dl2, dhid, dO, dp, dc, dl1, part, scratch;
+  size_t dz, dl2, dhid, dhid32, dO, dp, dc, dl1, part, scratch;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -532,12 +545,15 @@ Ws ws_layout(const Dims &D) {
   };
   w.mu1 = take(T * 4); w.rstd1 = take(T * 4); w.mu2 = take(T * 4); w.rstd2 = take(T * 4);
   w.l1 = take(T * h * e); w.c = take(3 * T * h * e); w.p = take(pe * e); w.o = take(T * h * e);
-  w.hid = take(T * h * e); w.l2 = take(T * h * e); w.z = take(T * f * e); w.act = take(T * f * e);
+  w.hid = take(T * h * 4);             // residual stream H, fp32
+  w.l2 = take(T * h * e); w.z = take(T * f * e); w.act = take(T * f * e);
   w.saved = off;
   off = 0;
-  w.dz = take(T * f * e); w.dl2 = take(T * h * e); w.dhid = take(T * h * e); w.dO = take(T * h * e);
+  w.dz = take(T * f * e); w.dl2 = take(T * h * e); w.dhid = take(T * h * e);
+  w.dhid32 = take(T * h * 4);          // residual-stream gradient dH, fp32
+  w.dO = take(T * h * e);
   w.dp = take(pe * e); w.dc = take(3 * T * h * e); w.dl1 = take(T * h * e);
-  size_t part = 3 * 512 * h;
+  size_t part = 4 * 512 * h;
   const size_t widest = f > 3 * h ? f : 3 * h;
   if (kColsumMaxSplit * widest > part) part = kColsumMaxSplit * widest;
   w.part = take(part * 4);
@@ -610,7 +626,7 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
 
   // LN1
   g_tag = GPTL_TAG_F1_LN1;
-  GPTL_TRY(run_ln_fwd(T, h, dt, x, W->ln1_g, W->ln1_b, D.eps, l1, mu1, rs1, st));
+  GPTL_TRY(run_ln_fwd(T, h, dt, x, 0, W->ln1_g, W->ln1_b, D.eps, l1, mu1, rs1, st));
   // QKV column split: C_i = L1 W_qkv,i^T + b_qkv,i
   g_tag = GPTL_TAG_F2_QKV;
   {
@@ -656,6 +672,7 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
     b.g_div = kNoGroup; b.k_shard = 1;
     gptl_gemm_desc g = gemm(T, h, hs, 1, a, b, hid, h, 0);
     g.k_shards = t;
+    g.out_f32 = 1;                       // H stays fp32 (the residual stream)
     g.bias = W->b_o;
     g.resid = x;
     g.ld_resid = h;
@@ -663,7 +680,7 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
   }
   // LN2
   g_tag = GPTL_TAG_F7_LN2;
-  GPTL_TRY(run_ln_fwd(T, h, dt, hid, W->ln2_g, W->ln2_b, D.eps, l2, mu2, rs2, st));
+  GPTL_TRY(run_ln_fwd(T, h, dt, hid, 1, W->ln2_g, W->ln2_b, D.eps, l2, mu2, rs2, st));
   // FFN1 column split with fused bias + GeLU: Z_i, A_i = gelu(Z_i)
   g_tag = GPTL_TAG_F8_FFN1_GELU;
   {
@@ -687,6 +704,7 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
     g.k_shards = t;
     g.bias = W->b_2;
     g.resid = hid;
+    g.resid_f32 = 1;
     g.ld_resid = h;
     GPTL_TRY(run_gemm(g, dt, st));
   }
@@ -705,6 +723,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   const float *mu1 = at<float>(saved, w.mu1), *rs1 = at<float>(saved, w.rstd1);
   const float *mu2 = at<float>(saved, w.mu2), *rs2 = at<float>(saved, w.rstd2);
   void *dz = at<void>(scratch, w.dz), *dl2 = at<void>(scratch, w.dl2);
+  float *dhid32 = at<float>(scratch, w.dhid32);
   void *dhid = at<void>(scratch, w.dhid), *dO = at<void>(scratch, w.dO);
   void *dp = at<void>(scratch, w.dp), *dc = at<void>(scratch, w.dc), *dl1 = at<void>(scratch, w.dl1);
   float *part = at<float>(scratch, w.part);
@@ -713,8 +732,6 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   prof_start(st);
 
   // ---- FFN2 (row split)
-  g_tag = GPTL_TAG_B2_DB2;
-  GPTL_TRY(run_colsum(T, h, 1, h, 0, dt, dy, gr->b_2, part, st));
   g_tag = GPTL_TAG_B2_DW2;
   {  // dW2_i = dOut^T A_i   [t][h][f/t] fp32
     gptl_gemm_desc g = gemm(h, fs, T, t, view(dy, h, T, 1, h, 0, 1),
@@ -754,8 +771,9 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   }
   // ---- LN2 backward + residual: dH = dOut + LNbwd(dL2); also db_o = sum dH
   g_tag = GPTL_TAG_B6_LN2;
-  GPTL_TRY(run_ln_bwd(T, h, dt, dl2, hid, mu2, rs2, W->ln2_g, dy, dhid, gr->ln2_g, gr->ln2_b,
-                      gr->b_o, part, st));
+  //      (the same pass sums dH into db_o and dOut into db_2)
+  GPTL_TRY(run_ln_bwd(LNB_H, T, h, dt, dl2, hid, mu2, rs2, W->ln2_g, dy, dhid, dhid32, gr->ln2_g,
+                      gr->ln2_b, gr->b_o, gr->b_2, part, st));
   // ---- out-projection (row split)
   g_tag = GPTL_TAG_B7_DWO;
   {  // dWo_i = dH^T O_i   [t][h][h/t]
@@ -846,8 +864,8 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   }
   // ---- LN1 backward + residual: dX = dH + LNbwd(dL1)
   g_tag = GPTL_TAG_B12_LN1;
-  GPTL_TRY(run_ln_bwd(T, h, dt, dl1, x, mu1, rs1, W->ln1_g, dhid, dx, gr->ln1_g, gr->ln1_b,
-                      nullptr, part, st));
+  GPTL_TRY(run_ln_bwd(LNB_X, T, h, dt, dl1, x, mu1, rs1, W->ln1_g, dhid32, dx, nullptr,
+                      gr->ln1_g, gr->ln1_b, nullptr, nullptr, part, st));
   return GPTL_OK;
 }
 
@@ -1025,7 +1043,8 @@ int gptl_layernorm_fwd(int rows, int h, gptl_dtype dtype, const void *x, const v
   if (!(eps > 0.f)) return GPTL_E_ARG;
   GPTL_TRY(device_check());
   prof_start(reinterpret_cast<cudaStream_t>(stream));
-  return run_ln_fwd(rows, h, dtype, x, g, b, eps, y, mu, rstd, reinterpret_cast<cudaStream_t>(stream));
+  return run_ln_fwd(rows, h, dtype, x, 0, g, b, eps, y, mu, rstd,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t gptl_layernorm_bwd_scratch_bytes(int rows, int h) {
@@ -1043,7 +1062,8 @@ int gptl_layernorm_bwd(int rows, int h, gptl_dtype dtype, const void *gy, const 
       !aligned16(scratch))
     return GPTL_E_ALIGN;
   prof_start(reinterpret_cast<cudaStream_t>(stream));
-  return run_ln_bwd(rows, h, dtype, gy, x, mu, rstd, g, resid, dx, dg, db, dx_sum,
+  return run_ln_bwd(LNB_PARTS, rows, h, dtype, gy, x, mu, rstd, g, resid, dx, nullptr, dg, db,
+                    dx_sum, nullptr,
                     static_cast<float *>(scratch), reinterpret_cast<cudaStream_t>(stream));
 }
 

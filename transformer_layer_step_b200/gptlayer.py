@@ -64,7 +64,7 @@ class GemmDesc(C.Structure):
                 ("o_mod", C.c_int), ("o_str_mod", C.c_longlong), ("o_str_div", C.c_longlong),
                 ("bias", C.c_void_p), ("bias_g_stride", C.c_longlong), ("resid", C.c_void_p),
                 ("ld_resid", C.c_longlong), ("aux", C.c_void_p), ("out2", C.c_void_p),
-                ("act", C.c_int)]
+                ("act", C.c_int), ("resid_f32", C.c_int)]
 
 
 class LaunchRecord(C.Structure):
