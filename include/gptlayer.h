@@ -53,7 +53,8 @@ enum {
   GPTL_E_ARCH = -5,    /* the current device is not compute capability 10.x  */
   GPTL_E_CUDA = -6,    /* a CUDA runtime/driver call or a launch failed      */
   GPTL_E_DEVICE = -7,  /* the device error word is set (see below)           */
-  GPTL_E_ARG = -8      /* an invalid scalar argument (hyper-parameter)       */
+  GPTL_E_ARG = -8,     /* an invalid scalar argument (hyper-parameter)       */
+  GPTL_E_TOO_LARGE = -9 /* the sizes exceed a fixed internal capacity         */
 };
 
 typedef enum { GPTL_FP16 = 0, GPTL_BF16 = 1 } gptl_dtype;

@@ -109,6 +109,28 @@ size_t gptl_colsum_scratch_bytes(int n, int groups);
 int gptl_colsum(int rows, int n, int groups, long long ld, long long gstride, gptl_dtype dtype,
                 const void *a, float *out, void *scratch, gptl_stream_t stream);
 
+/* The same column sums as gptl_colsum, for callers that cannot hand the
+ * library any temporary device memory.  A plug-in or custom operator inside a
+ * host framework that owns and pre-plans every device allocation may not call
+ * cudaMalloc (nor ask the framework for memory) in the middle of its work, and
+ * some deployments forbid device allocation after start-up altogether.  This
+ * entry point allocates nothing: its partial sums live in one fixed array of
+ * 64 * 16384 floats (4 MiB) in the library's device memory, which every GPU
+ * that loads the library holds until the process exits.  (The Megatron-LM
+ * pages have no counterpart to this; it is a property of this library.)
+ *   - n * groups must be at most 16384, else GPTL_E_TOO_LARGE and nothing is
+ *     launched; the other arguments and results are those of gptl_colsum,
+ *     summed in the same order.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array: calls whose kernels may overlap on the
+ *     GPU (different streams, or different host threads, on one device) race
+ *     and give wrong sums.  Calls in order on one stream are safe.  The array
+ *     keeps the last call's partial sums; each call writes every partial it
+ *     reads before reading it, so nothing needs clearing in between. */
+int gptl_colsum_noalloc(int rows, int n, int groups, long long ld, long long gstride,
+                        gptl_dtype dtype, const void *a, float *out, gptl_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

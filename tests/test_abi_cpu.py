@@ -17,7 +17,8 @@ def test_exports_every_declared_function():
 
 
 def test_strerror_codes():
-    for code in (0, G.E_NULL, G.E_SHAPE, G.E_ALIGN, G.E_DTYPE, G.E_ARCH, G.E_CUDA, G.E_DEVICE, G.E_ARG):
+    for code in (0, G.E_NULL, G.E_SHAPE, G.E_ALIGN, G.E_DTYPE, G.E_ARCH, G.E_CUDA, G.E_DEVICE, G.E_ARG,
+                 G.E_TOO_LARGE):
         assert G.strerror(code) and G.strerror(code) != "unknown error"
 
 

@@ -496,6 +496,31 @@ int run_colsum(int rows, int n, int groups, long long ld, long long gstride, gpt
   return launch_reduce_parts(part, split, width, 1, out, nullptr, nullptr, nullptr, st);
 }
 
+// Fixed partial-sum storage of gptl_colsum_noalloc: kColsumMaxSplit partial
+// rows of at most kNoAllocMaxWidth columns.  Host code may not use the
+// array's name as a device address; noalloc_scratch() looks the address up
+// once per device, with that device current.
+constexpr int kNoAllocMaxWidth = 16384;
+static __device__ __align__(256) float g_colsum_scratch[(size_t)kColsumMaxSplit * kNoAllocMaxWidth];
+float *g_colsum_scratch_addr[kMaxDevices];
+
+int noalloc_scratch(float **out) {
+  int dev = 0;
+  GPTL_CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return GPTL_E_ARCH;
+  GPTL_TRY(device_check());
+  if (!g_colsum_scratch_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_colsum_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();
+      return GPTL_E_CUDA;
+    }
+    g_colsum_scratch_addr[dev] = static_cast<float *>(p);
+  }
+  *out = g_colsum_scratch_addr[dev];
+  return GPTL_OK;
+}
+
 // ------------------------------------------------------------- the layer
 struct Dims {
   int b, s, h, a, f, t, d, hs, as, fs;
@@ -885,6 +910,7 @@ const char *gptl_strerror(int code) {
     case GPTL_E_CUDA: return "a CUDA call or kernel launch failed";
     case GPTL_E_DEVICE: return "the device error word is set";
     case GPTL_E_ARG: return "invalid scalar argument";
+    case GPTL_E_TOO_LARGE: return "the sizes exceed a fixed internal capacity";
     default: return "unknown error";
   }
 }
@@ -1099,6 +1125,22 @@ int gptl_colsum(int rows, int n, int groups, long long ld, long long gstride, gp
   if (!aligned16(a) || !aligned16(scratch)) return GPTL_E_ALIGN;
   prof_start(reinterpret_cast<cudaStream_t>(stream));
   return run_colsum(rows, n, groups, ld, gstride, dtype, a, out, static_cast<float *>(scratch),
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Column sums with their partials in a fixed device array instead of
+// caller memory (see gptl_colsum_noalloc in gptlayer_parts.h).
+int gptl_colsum_noalloc(int rows, int n, int groups, long long ld, long long gstride,
+                        gptl_dtype dtype, const void *a, float *out, gptl_stream_t stream) {
+  if (!a || !out) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(a)) return GPTL_E_ALIGN;
+  if (rows <= 0 || n <= 0 || groups <= 0) return GPTL_E_SHAPE;
+  if ((long long)n * groups > kNoAllocMaxWidth) return GPTL_E_TOO_LARGE;
+  float *part = nullptr;
+  GPTL_TRY(noalloc_scratch(&part));
+  prof_start(reinterpret_cast<cudaStream_t>(stream));
+  return run_colsum(rows, n, groups, ld, gstride, dtype, a, out, part,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -21,6 +21,7 @@ FP16, BF16 = 0, 1
 ACT_NONE, ACT_GELU, ACT_DGELU = 0, 1, 2
 CAUSAL_NONE, CAUSAL_SKIP_UPPER, CAUSAL_K_BELOW, CAUSAL_K_FROM = 0, 1, 2, 3
 E_NULL, E_SHAPE, E_ALIGN, E_DTYPE, E_ARCH, E_CUDA, E_DEVICE, E_ARG = -1, -2, -3, -4, -5, -6, -7, -8
+E_TOO_LARGE = -9
 DTYPES = {"fp16": FP16, "bf16": BF16}
 PARAM_NAMES = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
                "ln2_g", "ln2_b", "w_1", "b_1", "w_2", "b_2")
@@ -106,6 +107,8 @@ _SIGS = {
     "gptl_colsum_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "gptl_colsum": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_longlong, C.c_longlong, C.c_int,
                               C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "gptl_colsum_noalloc": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_longlong, C.c_longlong,
+                                      C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gptl_launch_count": (C.c_ulonglong, []),
     "gptl_profile_begin": (C.c_int, [C.c_int]),
     "gptl_profile_end": (C.c_int, [C.POINTER(LaunchRecord), C.c_int, C.POINTER(C.c_int),
@@ -256,6 +259,12 @@ def colsum_scratch_bytes(n, groups) -> int:
 def colsum(rows, n, groups, ld, gstride, dtype, a, out, scratch, stream=0):
     _check(lib().gptl_colsum(rows, n, groups, ld, gstride, DTYPES.get(dtype, dtype), _ptr(a),
                              _ptr(out), _ptr(scratch), stream), "gptl_colsum")
+
+
+def colsum_noalloc(rows, n, groups, ld, gstride, dtype, a, out, stream=0):
+    """gptl_colsum without caller scratch (fixed library array; see the header)."""
+    _check(lib().gptl_colsum_noalloc(rows, n, groups, ld, gstride, DTYPES.get(dtype, dtype),
+                                     _ptr(a), _ptr(out), stream), "gptl_colsum_noalloc")
 
 
 def read_device_error(clear: bool = True) -> int:
