@@ -34,7 +34,16 @@ typedef struct {
   int k_shard;
 } gptl_operand;
 
-enum { GPTL_ACT_NONE = 0, GPTL_ACT_GELU = 1, GPTL_ACT_DGELU = 2 };
+enum {
+  GPTL_ACT_NONE = 0,
+  GPTL_ACT_GELU = 1,     /* out = value, out2 = GeLU(value)                   */
+  GPTL_ACT_DGELU = 2,    /* out = value * GeLU'(aux)                          */
+  GPTL_ACT_EXP_LSE = 3,  /* out = exp2(value * ep_scale - row_vec[G][m]);
+                            0 where n > m (attention probabilities from the
+                            scores and each row's base-2 log-sum-exp)         */
+  GPTL_ACT_DSOFTMAX = 4  /* out = ep_scale * aux * (value - row_vec[G][m]);
+                            0 where n > m (softmax backward from dP)          */
+};
 enum {
   GPTL_CAUSAL_NONE = 0,
   GPTL_CAUSAL_SKIP_UPPER = 1, /* skip 128 x BN tiles with n0 > m0 + 127    */
@@ -52,7 +61,14 @@ enum {
  * by GeLU'(aux at the output's index).  out_f32 = 1 stores the fp32 value
  * (act must be GPTL_ACT_NONE); otherwise out is 16-bit, rounded to nearest
  * even.  Requirements: K % 16 == 0, N % 16 == 0, all offsets/pitches
- * multiples of 8 elements. */
+ * multiples of 8 elements.
+ * Split-K: when out_f32 is set with no bias, resid or act, and ws (16-byte
+ * aligned device memory of ws_bytes) is given, the library may cut the K
+ * loop of each output tile into slices computed by different SMs; each slice
+ * writes fp32 partial sums to ws and a second kernel adds them in slice
+ * order (the result is deterministic).  It does so only when the output has
+ * too few tiles to fill the GPU and the partials fit in ws_bytes.  ws may be
+ * NULL (no split). */
 typedef struct {
   int M, N, K, groups, k_shards, causal;
   gptl_operand a, b;
@@ -69,9 +85,25 @@ typedef struct {
   void *out2;
   int act;
   int resid_f32;
+  void *ws;
+  long long ws_bytes;
+  float ep_scale;
+  const float *row_vec;
+  long long row_vec_gstride;
 } gptl_gemm_desc;
 
 int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream);
+
+/* Fused causal attention forward ("Training GPT-2 with Megatron-LM" §6.2
+ * fused softmax; scores never leave the chip).  qkv: [tp][batch*seq][3h/tp],
+ * shard i's columns [Q_i | K_i | V_i], each head_dim = hidden/heads columns
+ * per head.  For every shard, batch element and head:
+ *   O = softmax_{q <= p}(Q K^T / sqrt(head_dim)) V   -> o [tp][batch*seq][h/tp]
+ *   lse[g][p] = log2 sum_{q <= p} exp2(Q_p.K_q log2(e)/sqrt(head_dim))
+ * with g = (shard*batch + batch index)*(heads/tp) + head, lse [g][seq] fp32.
+ * head_dim % 16 == 0 and <= 128, seq % 16 == 0. */
+int gptl_attention_fwd(int batch, int seq, int hidden, int heads, int tp, gptl_dtype dtype,
+                       const void *qkv, void *o, float *lse, gptl_stream_t stream);
 
 /* LayerNorm forward over `rows` rows of width h: y = g*(x-mu)*rstd + b with the
  * biased variance; mu and rstd ([rows] fp32) are saved for the backward.

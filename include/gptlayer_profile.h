@@ -35,17 +35,21 @@ enum {
   GPTL_KIND_OVERFLOW = 7,    /* inf/NaN check over the gradient arena         */
   GPTL_KIND_ADAM = 8,        /* fused unscale + Adam + 16-bit cast            */
   GPTL_KIND_SCALE = 9,       /* loss-scale update                             */
-  GPTL_KIND_COUNT = 10
+  GPTL_KIND_SPLITK = 10,     /* sum of a split-K GEMM's partial tiles         */
+  GPTL_KIND_ATTN_FWD = 11,   /* fused causal attention forward                */
+  GPTL_KIND_ROWDOT = 12,     /* softmax-backward row term dO . O              */
+  GPTL_KIND_COUNT = 13
 };
 
 /* step tags */
 enum {
   GPTL_TAG_NONE = 0,         /* a building-block call made on its own         */
-  GPTL_TAG_F1_LN1, GPTL_TAG_F2_QKV, GPTL_TAG_F3_SCORES, GPTL_TAG_F4_SOFTMAX, GPTL_TAG_F5_PV,
+  GPTL_TAG_F1_LN1, GPTL_TAG_F2_QKV, GPTL_TAG_F3_F5_ATTN,
   GPTL_TAG_F6_OUTPROJ, GPTL_TAG_F7_LN2, GPTL_TAG_F8_FFN1_GELU, GPTL_TAG_F10_FFN2,
   GPTL_TAG_B1_B3_DZ, GPTL_TAG_B2_DW2, GPTL_TAG_B2_DB2, GPTL_TAG_B3_DB1, GPTL_TAG_B4_DL2,
-  GPTL_TAG_B5_DW1, GPTL_TAG_B6_LN2, GPTL_TAG_B7_DWO, GPTL_TAG_B7_DO, GPTL_TAG_B8_DP,
-  GPTL_TAG_B8_DV, GPTL_TAG_B9_SOFTMAX, GPTL_TAG_B10_DQ, GPTL_TAG_B10_DK, GPTL_TAG_B11_DBQKV,
+  GPTL_TAG_B5_DW1, GPTL_TAG_B6_LN2, GPTL_TAG_B7_DWO, GPTL_TAG_B7_DO, GPTL_TAG_B8_P,
+  GPTL_TAG_B9_ROWDOT, GPTL_TAG_B8_B9_DS, GPTL_TAG_B8_DV, GPTL_TAG_B10_DQ, GPTL_TAG_B10_DK,
+  GPTL_TAG_B11_DBQKV,
   GPTL_TAG_B11_DWQKV, GPTL_TAG_B11_DL1, GPTL_TAG_B12_LN1,
   GPTL_TAG_O1_OVERFLOW, GPTL_TAG_O2_ADAM, GPTL_TAG_O3_SCALE,
   GPTL_TAG_COUNT

@@ -22,11 +22,14 @@ precision defines it ("Megatron-LM overview", §3.1: FP16 matrix math; the
 layer computes in fp16/bf16): every activation tensor that one step of the
 path hands to the next is held in the 16-bit type (round to nearest, ties to
 even), while the arithmetic inside a step stays exact.  The stored tensors
-are, forward: L1, C = [Q|K|V], the raw scores S = Q K^T, P, O, L2, Z,
+are, forward: L1, C = [Q|K|V], P (the fused attention keeps the scores on
+chip; its probabilities are 16-bit as a matrix operand), O, L2, Z,
 A = gelu(Z); backward: dZ (the GeLU backward is applied to dOut W2 before
-the store, as the fused bias-GeLU's backward), dL2, dO, dP, dV, dS, dQ, dK,
-dL1, and the 16-bit copy of dH that the out-projection's backward GEMMs
-read.  The residual stream H = X + attention and its gradient dH are the
+the store, as the fused bias-GeLU's backward), dL2, dO, dV, dS, dQ, dK, dL1,
+and the 16-bit copy of dH that the out-projection's backward GEMMs read.
+The softmax backward's row term sum_q P_pq dP_pq is formed as dO_p . O_p
+(equal in exact arithmetic, since O = P V) from the stored dO and O; the
+exact mode uses the plain sum.  The residual stream H = X + attention and its gradient dH are the
 FP32 side of mixed precision (like the master weights, they are never
 matrix operands): they stay exact here.  The layer outputs Out and dX are
 returned unrounded (their own store is the caller's last rounding) and the
@@ -93,9 +96,9 @@ def causal_softmax(z: np.ndarray) -> np.ndarray:
 
 def attention_head_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, precision=None, noise=None):
     """One (batch, head) block of causal self-attention: returns (P, O).
-    With a 16-bit precision the raw scores Q K^T and P are stored values."""
+    With a 16-bit precision P is a stored (rounded) value."""
     d = q.shape[1]
-    z = _store(q @ k.T, precision, noise) / math.sqrt(d)
+    z = (q @ k.T) / math.sqrt(d)
     p = _store(causal_softmax(z), precision, noise)
     return p, p @ v
 
@@ -235,9 +238,13 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
                 vh = c[i, rows, 2 * hs:3 * hs][:, cols]
                 pr = cache["probs"][i, j, eta]
                 doh = do[i, rows, cols]
-                dp = st(doh @ vh.T)
+                dp = doh @ vh.T
                 dv = st(pr.T @ doh)
-                dzs = pr * (dp - (pr * dp).sum(axis=1, keepdims=True))
+                if cache.get("precision") is None:
+                    rowterm = (pr * dp).sum(axis=1, keepdims=True)
+                else:
+                    rowterm = (doh * cache["o"][i, rows, cols]).sum(axis=1, keepdims=True)
+                dzs = pr * (dp - rowterm)
                 dsc = st(dzs * inv_sqrt_d)
                 dq = st(dsc @ kh)
                 dk = st(dsc.T @ qh)

@@ -72,7 +72,8 @@ def _op(buf_t, x_ext, rows_ext, g_ext, row_pitch, g_pitch, mn, x_mod=1, x_mul=0,
 
 
 def _run(dtype, M, N, K, groups, k_shards, causal, a_spec, b_spec, out_f32=False, bias=False,
-         resid=False, act=G.ACT_NONE, seed=0, std_a=1.0, std_b=0.1):
+         resid=False, act=G.ACT_NONE, seed=0, std_a=1.0, std_b=0.1, ws_bytes=0, resid_f32=False,
+         launches=None):
     """a_spec/b_spec: (shape of the 3-D buffer [g, rows, x], view kwargs)."""
     need_gpu()
     rng = np.random.default_rng(seed)
@@ -102,10 +103,19 @@ def _run(dtype, M, N, K, groups, k_shards, causal, a_spec, b_spec, out_f32=False
         keep.append(bt_)
         d.bias, d.bias_g_stride = bt_.data_ptr(), N
     if resid:
-        resid_v = rounded(rng.standard_normal((M, N)), dtype)
-        rt_ = dev_tensor(resid_v, dtype)
+        if resid_f32:
+            resid_v = rng.standard_normal((M, N)).astype(np.float32).astype(np.float64)
+            rt_ = torch.from_numpy(resid_v.astype(np.float32)).cuda()
+            d.resid_f32 = 1
+        else:
+            resid_v = rounded(rng.standard_normal((M, N)), dtype)
+            rt_ = dev_tensor(resid_v, dtype)
         keep.append(rt_)
         d.resid, d.ld_resid = rt_.data_ptr(), N
+    if ws_bytes:
+        ws = torch.full((ws_bytes // 4,), float("nan"), dtype=torch.float32, device="cuda")
+        keep.append(ws)
+        d.ws, d.ws_bytes = ws.data_ptr(), ws_bytes
     out2 = None
     if act == G.ACT_GELU:
         out2 = torch.zeros_like(out)
@@ -116,14 +126,17 @@ def _run(dtype, M, N, K, groups, k_shards, causal, a_spec, b_spec, out_f32=False
         keep.append(xt_)
         d.aux = xt_.data_ptr()
     d.act = act
+    n0 = G.launch_count()
     G.gemm(d, dtype, stream())
     check_device_error()
-    if out_f32:
-        return exp, out.cpu().numpy(), None
+    if launches is not None:
+        launches.append(G.launch_count() - n0)
     if bias:
         exp = exp + bias_v[:, None, :]
     if resid:
         exp = exp + resid_v[None]
+    if out_f32:
+        return exp, out.cpu().numpy(), None
     got = host_values(out, dtype)
     got2 = None
     if act == G.ACT_GELU:
@@ -238,3 +251,36 @@ def test_attention_arrangements(dtype, s, d):
                        b_spec=((ij, s, heads * d), dict(mn=1, x_mod=heads, x_mul=d, g_div=heads)),
                        std_a=0.2)
     _close(got, exp, 8e-3)
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_wgrad_split_k(dtype):
+    """Few output tiles and a long K: the K loop is split across SMs, the fp32
+    partials summed by a second kernel (two launches); deterministic."""
+    kw = dict(M=256, N=128, K=8192, groups=1, k_shards=1, causal=0,
+              a_spec=((1, 8192, 256), dict(mn=1)), b_spec=((1, 8192, 128), dict(mn=1)),
+              out_f32=True, ws_bytes=8 * 256 * 128 * 4)
+    nl = []
+    exp, got, _ = _run(dtype, launches=nl, **kw)
+    _close(got, exp, 5e-5)          # fp32 sums of 8192 products
+    assert nl == [2]
+    _, got2, _ = _run(dtype, **kw)
+    np.testing.assert_array_equal(got, got2)
+    # no workspace: one launch, same values up to the summation order
+    nl = []
+    kw["ws_bytes"] = 0
+    _, got3, _ = _run(dtype, launches=nl, **kw)
+    assert nl == [1]
+    _close(got3, exp, 5e-5)
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_fp32_out_with_bias_and_fp32_residual(dtype):
+    """The residual-stream epilogue: fp32 output of acc + bias (16-bit) +
+    residual (16-bit), and a 16-bit output of acc + bias + fp32 residual."""
+    kw = dict(M=300, N=256, K=192, groups=1, k_shards=1, causal=0,
+              a_spec=((1, 300, 192), dict(mn=0)), b_spec=((1, 256, 192), dict(mn=0)))
+    exp, got, _ = _run(dtype, out_f32=True, bias=True, resid=True, **kw)
+    _close(got, exp, 1e-5)
+    exp, got, _ = _run(dtype, bias=True, resid=True, resid_f32=True, **kw)
+    _close(got, exp, 1e-2)

@@ -79,7 +79,7 @@ def test_stored_tensors_are_rounded_step_outputs(dtype):
     q = c["c"][1, s:2 * s, d:2 * d]                 # shard 1, batch 1, head 1
     k = c["c"][1, s:2 * s, hs + d:hs + 2 * d]
     v = c["c"][1, s:2 * s, 2 * hs + d:2 * hs + 2 * d]
-    sc = rnd(q @ k.T) / math.sqrt(d)
+    sc = (q @ k.T) / math.sqrt(d)
     pr = rnd(oracle.causal_softmax(sc))
     np.testing.assert_array_equal(c["probs"][1, 1, 1], pr)
     np.testing.assert_array_equal(c["o"][1, s:2 * s, d:2 * d], rnd(pr @ v))
@@ -104,3 +104,15 @@ def test_fp16_mode_is_close_to_exact():
     assert np.abs(dm - de).max() <= 2e-2 * rms(de)
     for k in ge:
         assert np.abs(gm[k] - ge[k]).max() <= 2e-2 * rms(ge[k]), k
+
+
+def test_softmax_backward_row_term_identity():
+    """In exact arithmetic sum_q P_pq dP_pq = dO_p . O_p (O = P V), the row
+    term the mixed-precision mode forms from the stored dO and O."""
+    rng = np.random.default_rng(9)
+    s, d = 37, 16
+    q, k, v = (rng.standard_normal((s, d)) for _ in range(3))
+    do = rng.standard_normal((s, d))
+    p, o = oracle.attention_head_fwd(q, k, v)
+    dp = do @ v.T
+    np.testing.assert_allclose((p * dp).sum(axis=1), (do * o).sum(axis=1), rtol=1e-12, atol=1e-12)

@@ -1,0 +1,328 @@
+// attn_tc.cuh — fused causal attention forward on tcgen05 (sm_100a).
+//
+// For every (shard, batch, head) and every 128-row block of queries, the
+// kernel walks the 128-key blocks at or below the diagonal: S = Q K^T goes
+// to tensor memory, an online softmax turns it into P in shared memory (the
+// A operand of the next MMA), and O += P V accumulates in tensor memory.  S
+// and P never reach HBM.  This is the fused scale-mask-softmax of "Training
+// GPT-2 with Megatron-LM" §6.2 carried one step further: the score matrix is
+// consumed where it is produced.  The kernel writes O and the base-2
+// log-sum-exp of each row's scaled scores, from which the backward
+// recomputes P.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over work items):
+//   warp 0     TMA: Q once per item, then K and V of each key block into a
+//              2-stage ring;
+//   warp 1     one thread issues the MMAs: S_j = Q K_j^T into one of two S
+//              buffers, and O += P_{j-1} V_{j-1} once P_{j-1} is ready;
+//   warps 2-5  one query row per thread: read S_j from tensor memory, update
+//              the running max m and sum l, rescale O by exp2(m_old - m_new)
+//              in tensor memory, write P_j (16-bit) to shared memory; at the
+//              end normalise O by 1/l and store it.
+// Tensor memory: S buffers at columns 0 and 128, O at column 256.
+// Shared memory: P [128 x 128] (two 128B-swizzled 64-column atoms), Q as
+// head_dim/16 chunks of [128 rows x 16] (32B swizzle), and per stage K the
+// same way and V as MN-major chunks of [64 keys x vw].
+#pragma once
+#include "common.cuh"
+
+namespace gptl {
+
+constexpr int kAttnThreads = 192;
+constexpr int kAttnTile = 128;          // query rows per item, keys per block
+
+struct AttnParams {
+  CUtensorMap map_qk;   // C as [t*b][s][3h/t]; box {16, 128, 1}, 32B swizzle
+  CUtensorMap map_v;    // same tensor; box {vw, 64, 1}
+  int s, d, hs, as;     // sequence, head_dim, hidden per shard, heads per shard
+  int groups;           // t * b * heads per shard
+  int q_tiles;          // ceil(s / 128)
+  int vw;               // V chunk width in elements (64, 32 or 16)
+  float scale_log2;     // log2(e) / sqrt(head_dim)
+  uint32_t idesc_s, idesc_pv;
+  void *o;              // [t*b*s][h/t]
+  float *lse;           // [groups][s]
+  long long items;      // groups * q_tiles
+  int q_off, k_off, v_off;   // column offsets of Q, K, V inside a shard's 3h/t columns
+};
+
+// K-major operand chunk of 16 columns, 32B swizzle: rows of 32 B, 8-row
+// groups 256 B apart.
+__device__ __forceinline__ uint64_t attn_desc_k16(uint32_t addr) {
+  return make_smem_desc(addr, 16u, 256u, 6u);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const int d = p.d;
+  const uint32_t chunk_bytes = 128u * 32u;                   // one 16-column chunk, 128 rows
+  const uint32_t q_bytes = (uint32_t)(d / 16) * chunk_bytes;  // = 128 * d * 2
+  const uint32_t kv_bytes = 2u * q_bytes;                     // K and V of one stage
+  const uint32_t p_s = smem_u32(smem);                        // P: 32 KB
+  const uint32_t q_s = p_s + 32768u;
+  const uint32_t kv_s = q_s + q_bytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 32768u + q_bytes + 2u * kv_bytes);
+  // bars: q_full q_empty kv_full[2] kv_empty[2] s_full[2] s_empty[2] p_full o_done drain
+  const uint32_t q_full = smem_u32(&bars[0]), q_empty = smem_u32(&bars[1]);
+  auto kv_full = [&](int i) { return smem_u32(&bars[2 + i]); };
+  auto kv_empty = [&](int i) { return smem_u32(&bars[4 + i]); };
+  auto s_full = [&](int i) { return smem_u32(&bars[6 + i]); };
+  auto s_empty = [&](int i) { return smem_u32(&bars[8 + i]); };
+  const uint32_t p_full = smem_u32(&bars[10]), o_done = smem_u32(&bars[11]);
+  const uint32_t drain_bar = smem_u32(&bars[12]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(kv_full(i), 1);
+      mbar_init(kv_empty(i), 1);
+      mbar_init(s_full(i), 1);
+      mbar_init(s_empty(i), 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(o_done, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&p.map_qk);
+    prefetch_tensormap(&p.map_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512u);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_o = tmem_base + 256u;
+
+  // work item -> (group, query block): the longest rows (last query blocks) first
+  auto decode = [&](long long item, int &g, int &qt) {
+    qt = p.q_tiles - 1 - (int)(item / p.groups);
+    g = (int)(item % p.groups);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA
+      uint32_t kv_it = 0, item_n = 0;
+      uint32_t issued = 0, parity_bits = 0;   // stages with loads in flight, for a clean abort
+      int q_parity = -1;                      // parity of the last Q load issued
+      for (long long item = blockIdx.x; item < p.items; item += gridDim.x, ++item_n) {
+        int g, qt;
+        decode(item, g, qt);
+        const int head = g % p.as, zb = g / p.as;
+        if (!mbar_wait(q_empty, (item_n & 1u) ^ 1u, abort_flag)) goto tma_abort;
+        mbar_arrive_expect_tx(q_full, q_bytes);
+        q_parity = (int)(item_n & 1u);
+        for (int c = 0; c < d / 16; ++c)
+          tma_load_3d(q_s + (uint32_t)c * chunk_bytes, &p.map_qk, p.q_off + head * d + c * 16,
+                      qt * kAttnTile, zb, q_full);
+        for (int j = 0; j <= qt; ++j, ++kv_it) {
+          const int st = (int)(kv_it & 1u);
+          const uint32_t ph = (kv_it >> 1) & 1u;
+          if (!mbar_wait(kv_empty(st), ph ^ 1u, abort_flag)) goto tma_abort;
+          mbar_arrive_expect_tx(kv_full(st), kv_bytes);
+          const uint32_t k_s = kv_s + (uint32_t)st * kv_bytes, v_s = k_s + q_bytes;
+          for (int c = 0; c < d / 16; ++c)
+            tma_load_3d(k_s + (uint32_t)c * chunk_bytes, &p.map_qk, p.k_off + head * d + c * 16,
+                        j * kAttnTile, zb, kv_full(st));
+          const int nvc = d / p.vw;
+          for (int kb = 0; kb < 2; ++kb)
+            for (int c = 0; c < nvc; ++c)
+              tma_load_3d(v_s + (uint32_t)((kb * nvc + c) * 64 * p.vw * 2), &p.map_v,
+                          p.v_off + head * d + c * p.vw, j * kAttnTile + kb * 64, zb, kv_full(st));
+          issued |= 1u << st;
+          parity_bits = (parity_bits & ~(1u << st)) | (ph << st);
+        }
+      }
+      goto tma_done;
+    tma_abort:
+      for (int s2 = 0; s2 < 2; ++s2)
+        if (issued & (1u << s2)) mbar_wait_drain(kv_full(s2), (parity_bits >> s2) & 1u);
+      if (q_parity >= 0) mbar_wait_drain(q_full, (uint32_t)q_parity);
+    tma_done:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA
+      uint32_t kv_it = 0, s_it = 0, p_it = 0, item_n = 0;
+      for (long long item = blockIdx.x; item < p.items; item += gridDim.x, ++item_n) {
+        int g, qt;
+        decode(item, g, qt);
+        const int n = qt + 1;
+        if (!mbar_wait(q_full, item_n & 1u, abort_flag)) goto mma_abort;
+        tc_fence_after();
+        for (int j = 0; j <= n; ++j) {
+          if (j < n) {
+            const uint32_t kj = kv_it + (uint32_t)j;
+            if (!mbar_wait(kv_full(kj & 1u), (kj >> 1) & 1u, abort_flag)) goto mma_abort;
+            const int sb = (int)(s_it & 1u);
+            if (!mbar_wait(s_empty(sb), ((s_it >> 1) & 1u) ^ 1u, abort_flag)) goto mma_abort;
+            tc_fence_after();
+            const uint32_t k_s = kv_s + (kj & 1u) * kv_bytes;
+            for (int c = 0; c < d / 16; ++c)
+              tc_mma_f16(tmem_base + (uint32_t)(sb * 128), attn_desc_k16(q_s + (uint32_t)c * chunk_bytes),
+                         attn_desc_k16(k_s + (uint32_t)c * chunk_bytes), p.idesc_s, c > 0 ? 1u : 0u);
+            tc_commit(s_full(sb));
+            ++s_it;
+          }
+          if (j >= 1) {
+            if (!mbar_wait(p_full, p_it & 1u, abort_flag)) goto mma_abort;
+            ++p_it;
+            tc_fence_after();
+            const uint32_t pj = kv_it + (uint32_t)(j - 1);
+            const uint32_t v_s = kv_s + (pj & 1u) * kv_bytes + q_bytes;
+            const uint32_t row_b = (uint32_t)p.vw * 2u;
+            const uint32_t kb_bytes = (uint32_t)(d / p.vw) * 64u * row_b;
+            const uint32_t vsw = p.vw == 64 ? 2u : (p.vw == 32 ? 4u : 6u);
+            for (int st = 0; st < 8; ++st) {
+              const uint64_t adesc =
+                  make_smem_desc(p_s + (uint32_t)(st >> 2) * 16384u + (uint32_t)(st & 3) * 32u, 16u, 1024u, 2u);
+              const uint64_t bdesc = make_smem_desc(v_s + (uint32_t)(st >> 2) * kb_bytes +
+                                                        (uint32_t)(st & 3) * 16u * row_b,
+                                                    64u * row_b, 8u * row_b, vsw);
+              tc_mma_f16(tmem_o, adesc, bdesc, p.idesc_pv, (j > 1 || st > 0) ? 1u : 0u);
+            }
+            tc_commit(o_done);
+            tc_commit(kv_empty(pj & 1u));
+          }
+        }
+        tc_commit(q_empty);
+        kv_it += (uint32_t)n;
+      }
+      goto mma_done;
+    mma_abort:
+      tc_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+    mma_done:;
+    }
+  } else {
+    // -------------------------------------------------- softmax and epilogue
+    const int q4 = warp & 3;                 // TMEM lane quarter of this warp
+    const int row = q4 * 32 + lane;          // query row within the block
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    uint32_t s_it = 0, o_it = 0;
+    for (long long item = blockIdx.x; item < p.items; item += gridDim.x) {
+      int g, qt;
+      decode(item, g, qt);
+      const int n = qt + 1;
+      const int qrow = qt * kAttnTile + row;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) {
+        const int sb = (int)(s_it & 1u);
+        if (!mbar_wait(s_full(sb), (s_it >> 1) & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r[8][16];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) tmem_ld16(tmem_base + lane_off + (uint32_t)(sb * 128 + c * 16), r[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_empty(sb));
+        ++s_it;
+        // scale, mask (only the diagonal block and keys past the sequence), max
+        const bool diag = (j == qt);
+        const int key0 = j * kAttnTile;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int key = key0 + c * 16 + e;
+            float x = __uint_as_float(r[c][e]) * p.scale_log2;
+            if (diag && (key > qrow || key >= p.s)) x = -INFINITY;
+            r[c][e] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+        const float m_new = fmaxf(m, mx);
+        const float alpha = exp2f(m - m_new);
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float pv = exp2f(__uint_as_float(r[c][e]) - m_new);
+            r[c][e] = __float_as_uint(pv);
+            sum += pv;
+          }
+        l = l * alpha + sum;
+        m = m_new;
+        if (j >= 1) {
+          // P_{j-1} V_{j-1} done: O is complete and the P buffer is free
+          if (!mbar_wait(o_done, o_it & 1u, abort_flag)) { ok = false; break; }
+          ++o_it;
+          tc_fence_after();
+          for (int c = 0; c < d / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tmem_o + lane_off + (uint32_t)(c * 16), o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(tmem_o + lane_off + (uint32_t)(c * 16), o);
+          }
+          tmem_wait_st();
+        }
+        // P (16-bit) into the 128B-swizzled K-major A tile: row `row`,
+        // 16-byte chunk c16 of the row goes to atom c16/8, slot (c16%8)^(row%8)
+#pragma unroll
+        for (int c16 = 0; c16 < 16; ++c16) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[c16 >> 1][(c16 & 1) * 8 + e]);
+          const uint32_t addr = p_s + (uint32_t)(c16 >> 3) * 16384u + (uint32_t)row * 128u +
+                                (uint32_t)(((c16 & 7) ^ (row & 7)) * 16);
+          st_shared_v4(addr, pack8<T>(f));
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      // epilogue: wait for the last P V, normalise, store O and the log-sum-exp
+      if (!mbar_wait(o_done, o_it & 1u, abort_flag)) break;
+      ++o_it;
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const int head = g % p.as, zb = g / p.as;
+      T *orow = static_cast<T *>(p.o) + ((long long)zb * p.s + qrow) * p.hs + head * d;
+      for (int c = 0; c < d / 16; ++c) {
+        uint32_t o[16];
+        tmem_ld16(tmem_o + lane_off + (uint32_t)(c * 16), o);
+        tmem_wait_ld();
+        if (qrow < p.s) {
+          float f[8];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[h2 * 8 + e]) * inv_l;
+            reinterpret_cast<uint4 *>(orow + c * 16)[h2] = pack8<T>(f);
+          }
+        }
+      }
+      if (qrow < p.s) p.lse[(long long)g * p.s + qrow] = m + log2f(l);
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512u);
+  }
+}
+
+}  // namespace gptl

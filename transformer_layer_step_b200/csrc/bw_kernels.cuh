@@ -276,13 +276,30 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T *__restrict__ a, in
   const bool col_ok = cv * 8 < n;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   const T *base = a + (long long)g * gstride;
-  if (col_ok)
-    for (int r = blockIdx.y * 8 + threadIdx.y; r < rows; r += gridDim.y * 8) {
+  if (col_ok) {
+    // four independent row loads in flight per thread
+    const int step = gridDim.y * 8;
+    int r = blockIdx.y * 8 + threadIdx.y;
+    for (; r + 3 * step < rows; r += 4 * step) {
+      uint4 q[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        q[u] = __ldcs(reinterpret_cast<const uint4 *>(base + (long long)(r + u * step) * ld + cv * 8));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float f[8];
+        unpack8<T>(q[u], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += f[e];
+      }
+    }
+    for (; r < rows; r += step) {
       float f[8];
       unpack8<T>(*reinterpret_cast<const uint4 *>(base + (long long)r * ld + cv * 8), f);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] += f[e];
     }
+  }
 #pragma unroll
   for (int e = 0; e < 8; ++e) sm[threadIdx.y][threadIdx.x * 8 + e] = acc[e];
   __syncthreads();

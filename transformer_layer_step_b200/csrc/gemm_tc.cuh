@@ -18,10 +18,12 @@
 //     fused_bias_gelu of "Training GPT-2 with Megatron-LM" §6.2), GeLU'
 //     scaling of an input gradient, fp32 weight-gradient store.
 //
-// Warp roles (192 threads, one CTA per SM): warp 0 issues TMA loads into a
+// Warp roles (320 threads, one CTA per SM): warp 0 issues TMA loads into a
 // multi-stage mbarrier ring, warp 1 allocates TMEM and one thread issues
-// tcgen05.mma (M=128, N=BN, K=16 each), warps 2..5 drain the double-buffered
-// accumulator with tcgen05.ld while the next tile's MMAs run.
+// tcgen05.mma (M=128, N=BN, K=16 each), warps 2..9 drain the double-buffered
+// accumulator with tcgen05.ld while the next tile's MMAs run.  A warp may
+// only read the TMEM lane quarter (warp % 4), so two epilogue warps share
+// each quarter and split its columns in half.
 #pragma once
 #include "common.cuh"
 
@@ -29,9 +31,10 @@ namespace gptl {
 
 constexpr int kBM = 128;          // tile rows (UMMA M)
 constexpr int kBK = 64;           // tile depth per pipeline stage
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
+constexpr int kEpiWarps = 8;
 
-enum : int { kActNone = 0, kActGelu = 1, kActDGelu = 2 };
+enum : int { kActNone = 0, kActGelu = 1, kActDGelu = 2, kActExpLse = 3, kActDSoftmax = 4 };
 enum : int { kCausalNone = 0, kCausalSkipUpper = 1, kCausalKBelow = 2, kCausalKFrom = 3 };
 
 struct OperandRule {
@@ -47,6 +50,9 @@ struct alignas(64) GemmParams {
   CUtensorMap map_b;
   OperandRule ra, rb;
   int M, N, K, groups, k_shards, causal;
+  int split;                   // K slices per tile (split-K); 1 = none
+  float *ws;                   // split-K partials [split][groups][M][N] fp32
+  long long ws_slice;          // groups * M * N
   int bn, bn_alloc, stages, tmem_cols;
   uint32_t idesc;
   int m_tiles, n_tiles;
@@ -65,18 +71,23 @@ struct alignas(64) GemmParams {
   const void *aux;
   void *out2;
   int act;
+  float ep_scale;              // EXP_LSE / DSOFTMAX scale
+  const float *row_vec;        // per-row vector of the group: [G][row_vec_gstride]
+  long long row_vec_gstride;
 };
 
 struct TileInfo {
-  int g, m0, n0, kb_begin, kb_end;
+  int g, m0, n0, kb_begin, kb_end, slice;
   bool skip;
 };
 
 __device__ __forceinline__ TileInfo tile_info(const GemmParams &p, long long idx) {
   TileInfo t;
+  const long long tile = idx / p.split;
+  t.slice = (int)(idx - tile * p.split);
   const long long tpg = (long long)p.m_tiles * p.n_tiles;
-  t.g = (int)(idx / tpg);
-  const int rem = (int)(idx - (long long)t.g * tpg);
+  t.g = (int)(tile / tpg);
+  const int rem = (int)(tile - (long long)t.g * tpg);
   const int mt = rem / p.n_tiles, nt = rem - (rem / p.n_tiles) * p.n_tiles;
   t.m0 = mt * kBM;
   t.n0 = nt * p.bn;
@@ -85,6 +96,11 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams &p, long long idx
   t.kb_end = (p.K + kBK - 1) / kBK;
   if (p.causal == kCausalKBelow) t.kb_end = (min(p.K, t.m0 + kBM) + kBK - 1) / kBK;
   if (p.causal == kCausalKFrom) t.kb_begin = t.m0 / kBK;
+  if (p.split > 1) {           // balanced slices, none empty while split <= k-blocks
+    const int nkb = t.kb_end - t.kb_begin, b = t.kb_begin;
+    t.kb_begin = b + (int)((long long)t.slice * nkb / p.split);
+    t.kb_end = b + (int)((long long)(t.slice + 1) * nkb / p.split);
+  }
   return t;
 }
 
@@ -120,19 +136,19 @@ __device__ __forceinline__ uint64_t operand_desc(const OperandRule &r, uint32_t 
                         swizzle_layout(r.w));
 }
 
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
-  const unsigned long long t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity))
-    if (globaltimer() - t0 > kWaitTimeoutNs) return false;
-  return true;
-}
-
 template <typename T>
 __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int row, int n,
-                                               const uint32_t (&r)[16]) {
+                                               int slice, const uint32_t (&r)[16]) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  if (p.split > 1) {           // split-K partial: dense fp32, finished by splitk_reduce_kernel
+    float4 *o = reinterpret_cast<float4 *>(p.ws + (long long)slice * p.ws_slice +
+                                           ((long long)g * p.M + row) * p.N + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    return;
+  }
   const long long off = (long long)(g % p.o_mod) * p.o_str_mod +
                         (long long)(g / p.o_mod) * p.o_str_div + (long long)row * p.ldo + n;
   if (p.bias) {
@@ -191,6 +207,29 @@ __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int r
     }
     return;
   }
+  if (p.act == kActExpLse || p.act == kActDSoftmax) {
+    // attention probabilities recomputed from the scores and the row's
+    // base-2 log-sum-exp, or the softmax backward; both zero above the
+    // diagonal (column n > row)
+    const float rv = p.row_vec[(long long)g * p.row_vec_gstride + row];
+    float pr[16];
+    if (p.act == kActDSoftmax) {
+      const uint4 *pp = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.aux) + off);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float f[8];
+        unpack8<T>(pp[h], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pr[8 * h + i] = f[i];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float val = p.act == kActExpLse ? exp2f(v[i] * p.ep_scale - rv)
+                                            : p.ep_scale * pr[i] * (v[i] - rv);
+      v[i] = (n + i > row) ? 0.f : val;
+    }
+  }
   if (p.act == kActDGelu) {
     const uint4 *zp = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.aux) + off);
 #pragma unroll
@@ -237,7 +276,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4);
+      mbar_init(tempty_bar(a), kEpiWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -331,7 +370,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     }
   } else {
     // -------------------------------------------------- epilogue warps
-    const int q = warp & 3;   // TMEM lane quarter this warp may access
+    const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;        // which half of the tile's columns
     int acc = 0;
     uint32_t acc_phase = 0;
     for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
@@ -341,13 +381,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       tc_fence_after();
       const int row = ti.m0 + q * 32 + lane;
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.bn_alloc);
-      for (int c = 0; c < p.bn / 16; ++c) {
-        const int n = ti.n0 + c * 16;
-        if (n >= p.N) break;
-        uint32_t r[16];
-        tmem_ld16(t_row + (uint32_t)(c * 16), r);
+      // this warp's 16-column chunks: [c0, c1)
+      const int nchunk = p.bn / 16;
+      const int c0 = half ? (nchunk + 1) / 2 : 0;
+      int c1 = half ? nchunk : (nchunk + 1) / 2;
+      const int valid = (p.N - ti.n0 + 15) / 16;   // chunks inside N
+      if (c1 > valid) c1 = valid;
+      // software pipeline: the load of chunk c+1 is in flight while chunk c
+      // is processed (tcgen05.wait::ld waits for every earlier load)
+      uint32_t ra[16], rb[16];
+      if (c0 < c1) {
+        tmem_ld16(t_row + (uint32_t)(c0 * 16), ra);
         tmem_wait_ld();
-        if (row < p.M) epilogue_store<T>(p, ti.g, row, n, r);
+      }
+      for (int c = c0; c < c1; c += 2) {
+        const bool has_b = c + 1 < c1;
+        if (has_b) tmem_ld16(t_row + (uint32_t)((c + 1) * 16), rb);
+        if (row < p.M) epilogue_store<T>(p, ti.g, row, ti.n0 + c * 16, ti.slice, ra);
+        tmem_wait_ld();
+        if (!has_b) break;
+        const bool has_a = c + 2 < c1;
+        if (has_a) tmem_ld16(t_row + (uint32_t)((c + 2) * 16), ra);
+        if (row < p.M) epilogue_store<T>(p, ti.g, row, ti.n0 + (c + 1) * 16, ti.slice, rb);
+        tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
@@ -365,6 +421,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
   }
+}
+
+// out[G](m, n) = sum over s < split of ws[s][G][m][n], in slice order, into
+// the strided fp32 output of the GEMM; 4 columns per thread.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restrict__ ws,
+                                                           long long ws_slice, int split, int M,
+                                                           int N, int groups, float *out,
+                                                           long long ldo, int o_mod,
+                                                           long long o_str_mod,
+                                                           long long o_str_div) {
+  const long long n4 = ws_slice / 4;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long e = i * 4;
+    const int g = (int)(e / ((long long)M * N));
+    const long long rem = e - (long long)g * M * N;
+    const int m = (int)(rem / N), n = (int)(rem - (long long)(rem / N) * N);
+    float4 acc = reinterpret_cast<const float4 *>(ws)[i];
+    for (int s = 1; s < split; ++s) {
+      const float4 v = reinterpret_cast<const float4 *>(ws + (long long)s * ws_slice)[i];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    const long long off = (long long)(g % o_mod) * o_str_mod + (long long)(g / o_mod) * o_str_div +
+                          (long long)m * ldo + n;
+    *reinterpret_cast<float4 *>(out + off) = acc;
+  }
+}
+
+// Row term of the softmax backward: D[g][p] = sum_c dO[p][c] * O[p][c] over
+// the head's d columns (equal to sum_q P[p][q] dP[p][q], since O = P V).
+// One thread per (row, head) of the [t*b*s][h/t] matrices.
+template <typename T>
+__global__ void __launch_bounds__(256) attn_rowdot_kernel(const T *__restrict__ dout,
+                                                          const T *__restrict__ o, float *__restrict__ dvec,
+                                                          long long rows, int s, int hs, int as,
+                                                          int d) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * as) return;
+  const long long r = idx / as;
+  const int head = (int)(idx - r * as);
+  const uint4 *a = reinterpret_cast<const uint4 *>(dout + r * hs + (long long)head * d);
+  const uint4 *b = reinterpret_cast<const uint4 *>(o + r * hs + (long long)head * d);
+  float acc = 0.f;
+  for (int v = 0; v < d / 8; ++v) {
+    float fa[8], fb[8];
+    unpack8<T>(a[v], fa);
+    unpack8<T>(b[v], fb);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc += fa[e] * fb[e];
+  }
+  const long long zb = r / s, pos = r - zb * s;
+  dvec[(zb * as + head) * s + pos] = acc;
 }
 
 }  // namespace gptl

@@ -13,6 +13,7 @@
 
 #include "bw_kernels.cuh"
 #include "common.cuh"
+#include "attn_tc.cuh"
 #include "gemm_tc.cuh"
 #include "gptlayer_parts.h"
 #include "gptlayer_profile.h"
@@ -201,6 +202,31 @@ int pick_bn(const gptl_gemm_desc &d, int sms) {
   return best;
 }
 
+// Split-K slices for an fp32-output GEMM: the count (1..8) that minimises the
+// estimated time of the tile waves plus the reduction of the partials, with
+// the partials fitting in ws_bytes.  Times in microseconds: one 128 x bn x 64
+// k-block at ~8 kFLOP/clock/SM and 1.8 GHz; the reduction streams
+// (2 * split + 1) partial arrays at ~4 TB/s plus a launch.
+int pick_split(long long tiles, int kb_per_shard, int k_shards, int bn, long long out_elems,
+               long long ws_bytes, int sms) {
+  const long long nkb = (long long)kb_per_shard;
+  const double kb_us = 128.0 * bn * 64 * 2 / (8192.0 * 1800.0);
+  double best = (double)((tiles + sms - 1) / sms) * nkb * k_shards * kb_us;
+  int best_s = 1;
+  for (int sp = 2; sp <= 8; ++sp) {
+    if (sp > nkb) break;
+    if ((long long)sp * out_elems * 4 > ws_bytes) break;
+    const long long items = tiles * sp;
+    const double t = (double)((items + sms - 1) / sms) * ((nkb + sp - 1) / sp) * k_shards * kb_us +
+                     (2.0 * sp + 1.0) * out_elems * 4 / 4.0e6 + 3.0;
+    if (t < best) {
+      best = t;
+      best_s = sp;
+    }
+  }
+  return best_s;
+}
+
 template <typename T>
 int launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) {
   static bool attr_set[kMaxDevices] = {};
@@ -232,7 +258,9 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   if (d.act == GPTL_ACT_GELU && !d.out2) return GPTL_E_NULL;
   if (d.act == GPTL_ACT_DGELU && !d.aux) return GPTL_E_NULL;
   if ((d.out2 && !aligned16(d.out2)) || (d.aux && !aligned16(d.aux))) return GPTL_E_ALIGN;
-  if (d.act < 0 || d.act > 2 || (d.out_f32 && d.act != GPTL_ACT_NONE)) return GPTL_E_SHAPE;
+  if (d.act < 0 || d.act > 4 || (d.out_f32 && d.act != GPTL_ACT_NONE)) return GPTL_E_SHAPE;
+  if ((d.act == GPTL_ACT_EXP_LSE || d.act == GPTL_ACT_DSOFTMAX) && !d.row_vec) return GPTL_E_NULL;
+  if (d.act == GPTL_ACT_DSOFTMAX && !d.aux) return GPTL_E_NULL;
   GPTL_TRY(check_operand(d.a));
   GPTL_TRY(check_operand(d.b));
 
@@ -278,7 +306,15 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
             ((uint32_t)(kBM >> 4) << 24);
   p.m_tiles = (d.M + kBM - 1) / kBM;
   p.n_tiles = (d.N + bn - 1) / bn;
-  p.total_tiles = (long long)p.m_tiles * p.n_tiles * d.groups;
+  const long long tiles = (long long)p.m_tiles * p.n_tiles * d.groups;
+  p.split = 1;
+  if (d.out_f32 && !d.bias && !d.resid && d.act == GPTL_ACT_NONE && d.causal == GPTL_CAUSAL_NONE &&
+      d.ws && aligned16(d.ws))
+    p.split = pick_split(tiles, (d.K + kBK - 1) / kBK, d.k_shards, bn,
+                         (long long)d.groups * d.M * d.N, d.ws_bytes, sms);
+  p.ws = static_cast<float *>(d.ws);
+  p.ws_slice = (long long)d.groups * d.M * d.N;
+  p.total_tiles = tiles * p.split;
   p.out = d.out;
   p.ldo = d.ldo;
   p.o_mod = d.o_mod;
@@ -293,9 +329,110 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.aux = d.aux;
   p.out2 = d.out2;
   p.act = d.act;
+  p.ep_scale = d.ep_scale;
+  p.row_vec = d.row_vec;
+  p.row_vec_gstride = d.row_vec_gstride;
   const int grid = (int)(p.total_tiles < sms ? p.total_tiles : sms);
-  if (dt == GPTL_FP16) return launch_gemm_t<__half>(p, grid, smem, stream);
-  return launch_gemm_t<__nv_bfloat16>(p, grid, smem, stream);
+  if (dt == GPTL_FP16) GPTL_TRY(launch_gemm_t<__half>(p, grid, smem, stream));
+  else GPTL_TRY(launch_gemm_t<__nv_bfloat16>(p, grid, smem, stream));
+  if (p.split > 1) {
+    const long long n4 = p.ws_slice / 4;
+    long long blocks = (n4 + 255) / 256;
+    if (blocks > 8 * sms) blocks = 8 * sms;
+    splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        p.ws, p.ws_slice, p.split, d.M, d.N, d.groups, static_cast<float *>(d.out), d.ldo,
+        d.o_mod, d.o_str_mod, d.o_str_div);
+    GPTL_CK(cudaGetLastError());
+    prof_launched(stream, GPTL_KIND_SPLITK);
+  }
+  return GPTL_OK;
+}
+
+// ------------------------------------------------------------- attention
+// Fused causal attention forward over the QKV buffer C [t][T][3h/t] (shard
+// columns [Q_i | K_i | V_i], head-major): O [t][T][h/t] and the base-2
+// log-sum-exp of every row's scaled scores, lse [t*b*(a/t)][s].
+int run_attn_fwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, const void *c, void *o,
+                 float *lse, cudaStream_t st) {
+  int sms = 0;
+  GPTL_TRY(device_check(&sms));
+  if (d % 16 || d > 128 || hs % 8 || s <= 0 || s % 16 || as <= 0 || b <= 0 || t <= 0)
+    return GPTL_E_SHAPE;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return GPTL_E_CUDA;
+  AttnParams p;
+  memset(&p, 0, sizeof(p));
+  const CUtensorMapDataType ty =
+      dt == GPTL_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t dims[3] = {(cuuint64_t)(3 * hs), (cuuint64_t)s, (cuuint64_t)t * b};
+  cuuint64_t strides[2] = {(cuuint64_t)3 * hs * 2, (cuuint64_t)s * 3 * hs * 2};
+  cuuint32_t es[3] = {1, 1, 1};
+  cuuint32_t box_qk[3] = {16, 128, 1};
+  if (fn(&p.map_qk, ty, 3, const_cast<void *>(c), dims, strides, box_qk, es,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return GPTL_E_CUDA;
+  const int vw = d % 64 == 0 ? 64 : (d % 32 == 0 ? 32 : 16);
+  cuuint32_t box_v[3] = {(cuuint32_t)vw, 64, 1};
+  const CUtensorMapSwizzle vsw = vw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                          : (vw == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  if (fn(&p.map_v, ty, 3, const_cast<void *>(c), dims, strides, box_v, es,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, vsw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return GPTL_E_CUDA;
+  p.s = s; p.d = d; p.hs = hs; p.as = as;
+  p.groups = t * b * as;
+  p.q_tiles = (s + kAttnTile - 1) / kAttnTile;
+  p.vw = vw;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+  const uint32_t fmt = dt == GPTL_BF16 ? 1u : 0u;
+  p.idesc_s = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kAttnTile >> 3) << 17) |
+              ((uint32_t)(kAttnTile >> 4) << 24);
+  p.idesc_pv = (1u << 4) | (fmt << 7) | (fmt << 10) | (1u << 16) | ((uint32_t)(d >> 3) << 17) |
+               ((uint32_t)(kAttnTile >> 4) << 24);
+  p.o = o;
+  p.lse = lse;
+  p.items = (long long)p.groups * p.q_tiles;
+  p.q_off = 0; p.k_off = hs; p.v_off = 2 * hs;
+  // P 32 KB + Q + 2 stages of K and V, barriers; at least 120 KB so that one
+  // CTA (and its 512 tensor-memory columns) owns each SM
+  int smem = 1024 + 32768 + 128 * d * 2 * 5 + 256;
+  if (smem < 120 * 1024) smem = 120 * 1024;
+  const int grid = (int)(p.items < sms ? p.items : sms);
+  // the shared-memory opt-in is recorded per device and per dtype (both
+  // instantiations have the same function-pointer type)
+  static bool attr_set[kMaxDevices][2] = {};
+  int dev = 0;
+  GPTL_CK(cudaGetDevice(&dev));
+  auto launch = [&](auto kern) -> int {
+    if (!attr_set[dev][dt]) {
+      GPTL_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
+      attr_set[dev][dt] = true;
+    }
+    kern<<<grid, kAttnThreads, smem, st>>>(p);
+    GPTL_CK(cudaGetLastError());
+    return GPTL_OK;
+  };
+  if (dt == GPTL_FP16) GPTL_TRY(launch(attn_fwd_kernel<__half>));
+  else GPTL_TRY(launch(attn_fwd_kernel<__nv_bfloat16>));
+  prof_launched(st, GPTL_KIND_ATTN_FWD);
+  return GPTL_OK;
+}
+
+// D[g][p] = dO_p . O_p over each head's columns (the softmax backward's row term).
+int run_attn_rowdot(long long rows, int s, int hs, int as, int d, gptl_dtype dt, const void *dout,
+                    const void *o, float *dvec, cudaStream_t st) {
+  const long long n = rows * as;
+  const unsigned grid = (unsigned)((n + 255) / 256);
+  if (dt == GPTL_FP16)
+    attn_rowdot_kernel<__half><<<grid, 256, 0, st>>>((const __half *)dout, (const __half *)o, dvec,
+                                                     rows, s, hs, as, d);
+  else
+    attn_rowdot_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        (const __nv_bfloat16 *)dout, (const __nv_bfloat16 *)o, dvec, rows, s, hs, as, d);
+  GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_ROWDOT);
+  return GPTL_OK;
 }
 
 // ------------------------------------------------------------- LayerNorm
@@ -536,7 +673,7 @@ int check_shape(const gptl_shape *sh, Dims *D) {
   if (b <= 0 || s <= 0 || h <= 0 || a <= 0 || f <= 0 || t <= 0) return GPTL_E_SHAPE;
   if (h % a || a % t || f % t) return GPTL_E_SHAPE;
   const int d = h / a;
-  if (d % 16 || d > 256 || h % 64 || (f / t) % 64 || s % 16 || s > 2048) return GPTL_E_SHAPE;
+  if (d % 16 || d > 128 || h % 64 || (f / t) % 64 || s % 16 || s > 2048) return GPTL_E_SHAPE;
   if ((long long)b * s >= (1ll << 31)) return GPTL_E_SHAPE;
   if (!(sh->ln_eps > 0.f)) return GPTL_E_SHAPE;
   int tpr, vpt;
@@ -551,9 +688,9 @@ int check_shape(const gptl_shape *sh, Dims *D) {
 
 struct Ws {
   // saved (fwd -> bwd)
-  size_t mu1, rstd1, mu2, rstd2, l1, c, p, o, hid, l2, z, act, saved;
+  size_t mu1, rstd1, mu2, rstd2, l1, c, lse, o, hid, l2, z, act, saved;
   // scratch (bwd)
-  size_t dz, dl2, dhid, dhid32, dO, dp, dc, dl1, part, scratch;
+  size_t dz, dl2, dhid, dhid32, dO, p, dp, dvec, dc, dl1, part, splitk, splitk_bytes, scratch;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -569,7 +706,9 @@ Ws ws_layout(const Dims &D) {
     return o;
   };
   w.mu1 = take(T * 4); w.rstd1 = take(T * 4); w.mu2 = take(T * 4); w.rstd2 = take(T * 4);
-  w.l1 = take(T * h * e); w.c = take(3 * T * h * e); w.p = take(pe * e); w.o = take(T * h * e);
+  w.l1 = take(T * h * e); w.c = take(3 * T * h * e);
+  w.lse = take((size_t)D.b * D.a * D.s * 4);   // attention row log-sum-exp, fp32
+  w.o = take(T * h * e);
   w.hid = take(T * h * 4);             // residual stream H, fp32
   w.l2 = take(T * h * e); w.z = take(T * f * e); w.act = take(T * f * e);
   w.saved = off;
@@ -577,11 +716,20 @@ Ws ws_layout(const Dims &D) {
   w.dz = take(T * f * e); w.dl2 = take(T * h * e); w.dhid = take(T * h * e);
   w.dhid32 = take(T * h * 4);          // residual-stream gradient dH, fp32
   w.dO = take(T * h * e);
-  w.dp = take(pe * e); w.dc = take(3 * T * h * e); w.dl1 = take(T * h * e);
+  w.p = take(pe * e);                   // P recomputed for the backward
+  w.dp = take(pe * e);                  // dS
+  w.dvec = take((size_t)D.b * D.a * D.s * 4);
+  w.dc = take(3 * T * h * e); w.dl1 = take(T * h * e);
   size_t part = 4 * 512 * h;
   const size_t widest = f > 3 * h ? f : 3 * h;
   if (kColsumMaxSplit * widest > part) part = kColsumMaxSplit * widest;
   w.part = take(part * 4);
+  // split-K partials of the weight-gradient GEMMs: up to 8 slices of the
+  // largest gradient, at most 64 MiB (large layers have tiles enough)
+  size_t sk = (size_t)8 * h * (f > 3 * h ? f : 3 * h) * 4;
+  if (sk > ((size_t)64 << 20)) sk = (size_t)64 << 20;
+  w.splitk_bytes = sk;
+  w.splitk = take(sk);
   w.scratch = off;
   return w;
 }
@@ -639,13 +787,12 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
   const Ws w = ws_layout(D);
   const gptl_dtype dt = D.dt;
   const int T = (int)D.T, h = D.h, t = D.t, s = D.s, d = D.d, hs = D.hs, as = D.as, fs = D.fs;
-  const int G = D.b * D.a;                      // attention groups: (shard, batch, head)
-  void *l1 = at<void>(saved, w.l1), *c = at<void>(saved, w.c), *pb = at<void>(saved, w.p);
+  void *l1 = at<void>(saved, w.l1), *c = at<void>(saved, w.c);
+  float *lse = at<float>(saved, w.lse);
   void *o = at<void>(saved, w.o), *hid = at<void>(saved, w.hid), *l2 = at<void>(saved, w.l2);
   void *z = at<void>(saved, w.z), *act = at<void>(saved, w.act);
   float *mu1 = at<float>(saved, w.mu1), *rs1 = at<float>(saved, w.rstd1);
   float *mu2 = at<float>(saved, w.mu2), *rs2 = at<float>(saved, w.rstd2);
-  const float attn_scale = 1.0f / sqrtf((float)d);
   TagScope tag_scope(GPTL_TAG_NONE);
   prof_start(st);
 
@@ -662,32 +809,10 @@ int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void
     g.bias_g_stride = 3 * hs;
     GPTL_TRY(run_gemm(g, dt, st));
   }
-  // scores S = Q K^T per (shard, batch, head), lower-triangle tiles only
-  g_tag = GPTL_TAG_F3_SCORES;
-  {
-    gptl_operand q = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 0);
-    q.x_mod = as; q.x_mul = d; q.g_div = as;
-    gptl_operand k = q;
-    k.x_off = hs;
-    gptl_gemm_desc g = gemm(s, s, d, G, q, k, pb, s, (long long)s * s);
-    g.causal = GPTL_CAUSAL_SKIP_UPPER;
-    GPTL_TRY(run_gemm(g, dt, st));
-  }
-  // fused scale-mask-softmax, in place
-  g_tag = GPTL_TAG_F4_SOFTMAX;
-  GPTL_TRY(run_softmax_fwd(G, s, dt, attn_scale, pb, st));
-  // O = P V (K range limited to the lower triangle)
-  g_tag = GPTL_TAG_F5_PV;
-  {
-    gptl_operand pa = view(pb, s, s, G, s, (long long)s * s, 0);
-    gptl_operand v = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 1);
-    v.x_mod = as; v.x_mul = d; v.x_off = 2 * hs; v.g_div = as;
-    gptl_gemm_desc g = gemm(s, d, s, G, pa, v, o, hs, (long long)s * hs);
-    g.o_mod = as;
-    g.o_str_mod = d;
-    g.causal = GPTL_CAUSAL_K_BELOW;
-    GPTL_TRY(run_gemm(g, dt, st));
-  }
+  // causal attention, fused: S, softmax and P stay on chip; O and the
+  // row log-sum-exp go to memory
+  g_tag = GPTL_TAG_F3_F5_ATTN;
+  GPTL_TRY(run_attn_fwd(D.b, s, hs, as, t, d, dt, c, o, lse, st));
   // out-projection, row split: H = X + sum_i O_i W_o,i^T + b_o
   g_tag = GPTL_TAG_F6_OUTPROJ;
   {
@@ -742,7 +867,8 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   const gptl_dtype dt = D.dt;
   const int T = (int)D.T, h = D.h, t = D.t, s = D.s, d = D.d, hs = D.hs, as = D.as, fs = D.fs;
   const int G = D.b * D.a;
-  const void *l1 = at<void>(saved, w.l1), *c = at<void>(saved, w.c), *pb = at<void>(saved, w.p);
+  const void *l1 = at<void>(saved, w.l1), *c = at<void>(saved, w.c);
+  const float *lse = at<float>(saved, w.lse);
   const void *o = at<void>(saved, w.o), *hid = at<void>(saved, w.hid);
   const void *l2 = at<void>(saved, w.l2), *z = at<void>(saved, w.z), *act = at<void>(saved, w.act);
   const float *mu1 = at<float>(saved, w.mu1), *rs1 = at<float>(saved, w.rstd1);
@@ -751,7 +877,11 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   float *dhid32 = at<float>(scratch, w.dhid32);
   void *dhid = at<void>(scratch, w.dhid), *dO = at<void>(scratch, w.dO);
   void *dp = at<void>(scratch, w.dp), *dc = at<void>(scratch, w.dc), *dl1 = at<void>(scratch, w.dl1);
+  void *pb = at<void>(scratch, w.p);
+  float *dvec = at<float>(scratch, w.dvec);
   float *part = at<float>(scratch, w.part);
+  void *splitk = at<void>(scratch, w.splitk);
+  const long long splitk_bytes = (long long)w.splitk_bytes;
   const float attn_scale = 1.0f / sqrtf((float)d);
   TagScope tag_scope(GPTL_TAG_NONE);
   prof_start(st);
@@ -763,6 +893,8 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
                             view(act, fs, T, t, fs, (long long)T * fs, 1), gr->w_2, fs,
                             (long long)h * fs);
     g.out_f32 = 1;
+    g.ws = splitk;
+    g.ws_bytes = splitk_bytes;
     GPTL_TRY(run_gemm(g, dt, st));
   }
   g_tag = GPTL_TAG_B1_B3_DZ;
@@ -782,6 +914,8 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     gptl_gemm_desc g = gemm(fs, h, T, t, view(dz, fs, T, t, fs, (long long)T * fs, 1),
                             view(l2, h, T, 1, h, 0, 1), gr->w_1, h, (long long)fs * h);
     g.out_f32 = 1;
+    g.ws = splitk;
+    g.ws_bytes = splitk_bytes;
     GPTL_TRY(run_gemm(g, dt, st));
   }
   g_tag = GPTL_TAG_B4_DL2;
@@ -806,6 +940,8 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
                             view(o, hs, T, t, hs, (long long)T * hs, 1), gr->w_o, hs,
                             (long long)h * hs);
     g.out_f32 = 1;
+    g.ws = splitk;
+    g.ws_bytes = splitk_bytes;
     GPTL_TRY(run_gemm(g, dt, st));
   }
   g_tag = GPTL_TAG_B7_DO;
@@ -820,12 +956,31 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   dOv.x_mod = as; dOv.x_mul = d; dOv.g_div = as;
   gptl_operand cv = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 0);
   cv.x_mod = as; cv.x_mul = d; cv.g_div = as;
-  g_tag = GPTL_TAG_B8_DP;
-  {  // dP = dO V^T (lower-triangle tiles)
+  g_tag = GPTL_TAG_B8_P;
+  {  // P = exp2(Q K^T * log2(e)/sqrt(d) - lse), recomputed for the lower-triangle tiles
+    gptl_operand k = cv;
+    k.x_off = hs;
+    gptl_gemm_desc g = gemm(s, s, d, G, cv, k, pb, s, (long long)s * s);
+    g.causal = GPTL_CAUSAL_SKIP_UPPER;
+    g.act = GPTL_ACT_EXP_LSE;
+    g.ep_scale = 1.4426950408889634f * attn_scale;
+    g.row_vec = lse;
+    g.row_vec_gstride = s;
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
+  g_tag = GPTL_TAG_B9_ROWDOT;   // D = rowsum(dO * O), the softmax backward's row term
+  GPTL_TRY(run_attn_rowdot((long long)t * T, s, hs, as, d, dt, dO, o, dvec, st));
+  g_tag = GPTL_TAG_B8_B9_DS;
+  {  // dS = P (dO V^T - D) / sqrt(d) in the epilogue of the dP GEMM (lower-triangle tiles)
     gptl_operand v = cv;
     v.x_off = 2 * hs;
     gptl_gemm_desc g = gemm(s, s, d, G, dOv, v, dp, s, (long long)s * s);
     g.causal = GPTL_CAUSAL_SKIP_UPPER;
+    g.act = GPTL_ACT_DSOFTMAX;
+    g.ep_scale = attn_scale;
+    g.aux = pb;
+    g.row_vec = dvec;
+    g.row_vec_gstride = s;
     GPTL_TRY(run_gemm(g, dt, st));
   }
   g_tag = GPTL_TAG_B8_DV;
@@ -840,9 +995,6 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     g.causal = GPTL_CAUSAL_K_FROM;
     GPTL_TRY(run_gemm(g, dt, st));
   }
-  // dS = P (dP - rowsum(P dP)) / sqrt(d), in place over dP
-  g_tag = GPTL_TAG_B9_SOFTMAX;
-  GPTL_TRY(run_softmax_bwd(G, s, dt, attn_scale, pb, dp, st));
   g_tag = GPTL_TAG_B10_DQ;
   {  // dQ = dS K  -> Q columns of dC
     gptl_operand a = view(dp, s, s, G, s, (long long)s * s, 0);
@@ -875,6 +1027,8 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     gptl_gemm_desc g = gemm(3 * hs, h, T, t, view(dc, 3 * hs, T, t, 3 * hs, (long long)T * 3 * hs, 1),
                             view(l1, h, T, 1, h, 0, 1), gr->w_qkv, h, (long long)3 * hs * h);
     g.out_f32 = 1;
+    g.ws = splitk;
+    g.ws_bytes = splitk_bytes;
     GPTL_TRY(run_gemm(g, dt, st));
   }
   g_tag = GPTL_TAG_B11_DL1;
@@ -1128,6 +1282,19 @@ int gptl_colsum(int rows, int n, int groups, long long ld, long long gstride, gp
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
+int gptl_attention_fwd(int batch, int seq, int hidden, int heads, int tp, gptl_dtype dtype,
+                       const void *qkv, void *o, float *lse, gptl_stream_t stream) {
+  if (!qkv || !o || !lse) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(qkv) || !aligned16(o) || !aligned16(lse)) return GPTL_E_ALIGN;
+  if (batch <= 0 || seq <= 0 || hidden <= 0 || heads <= 0 || tp <= 0) return GPTL_E_SHAPE;
+  if (hidden % heads || heads % tp) return GPTL_E_SHAPE;
+  GPTL_TRY(device_check());
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  prof_start(st);
+  return run_attn_fwd(batch, seq, hidden / tp, heads / tp, tp, hidden / heads, dtype, qkv, o, lse, st);
+}
+
 // Column sums with their partials in a fixed device array instead of
 // caller memory (see gptl_colsum_noalloc in gptlayer_parts.h).
 int gptl_colsum_noalloc(int rows, int n, int groups, long long ld, long long gstride,
@@ -1211,9 +1378,7 @@ const char *gptl_tag_name(int tag) {
     case GPTL_TAG_NONE: return "-";
     case GPTL_TAG_F1_LN1: return "F1 ln1";
     case GPTL_TAG_F2_QKV: return "F2 qkv";
-    case GPTL_TAG_F3_SCORES: return "F3 scores";
-    case GPTL_TAG_F4_SOFTMAX: return "F4 softmax";
-    case GPTL_TAG_F5_PV: return "F5 pv";
+    case GPTL_TAG_F3_F5_ATTN: return "F3-F5 attention";
     case GPTL_TAG_F6_OUTPROJ: return "F6 outproj";
     case GPTL_TAG_F7_LN2: return "F7 ln2";
     case GPTL_TAG_F8_FFN1_GELU: return "F8/F9 ffn1+gelu";
@@ -1227,9 +1392,10 @@ const char *gptl_tag_name(int tag) {
     case GPTL_TAG_B6_LN2: return "B6 ln2 bwd";
     case GPTL_TAG_B7_DWO: return "B7 dwo";
     case GPTL_TAG_B7_DO: return "B7 do";
-    case GPTL_TAG_B8_DP: return "B8 dp";
+    case GPTL_TAG_B8_P: return "B8 P recompute";
     case GPTL_TAG_B8_DV: return "B8 dv";
-    case GPTL_TAG_B9_SOFTMAX: return "B9 softmax bwd";
+    case GPTL_TAG_B9_ROWDOT: return "B9 rowdot";
+    case GPTL_TAG_B8_B9_DS: return "B8/B9 dS";
     case GPTL_TAG_B10_DQ: return "B10 dq";
     case GPTL_TAG_B10_DK: return "B10 dk";
     case GPTL_TAG_B11_DBQKV: return "B11 dbqkv";

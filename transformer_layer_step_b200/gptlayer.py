@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG, "libgptlayer.so")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 
 FP16, BF16 = 0, 1
-ACT_NONE, ACT_GELU, ACT_DGELU = 0, 1, 2
+ACT_NONE, ACT_GELU, ACT_DGELU, ACT_EXP_LSE, ACT_DSOFTMAX = 0, 1, 2, 3, 4
 CAUSAL_NONE, CAUSAL_SKIP_UPPER, CAUSAL_K_BELOW, CAUSAL_K_FROM = 0, 1, 2, 3
 E_NULL, E_SHAPE, E_ALIGN, E_DTYPE, E_ARCH, E_CUDA, E_DEVICE, E_ARG = -1, -2, -3, -4, -5, -6, -7, -8
 E_TOO_LARGE = -9
@@ -65,7 +65,9 @@ class GemmDesc(C.Structure):
                 ("o_mod", C.c_int), ("o_str_mod", C.c_longlong), ("o_str_div", C.c_longlong),
                 ("bias", C.c_void_p), ("bias_g_stride", C.c_longlong), ("resid", C.c_void_p),
                 ("ld_resid", C.c_longlong), ("aux", C.c_void_p), ("out2", C.c_void_p),
-                ("act", C.c_int), ("resid_f32", C.c_int)]
+                ("act", C.c_int), ("resid_f32", C.c_int), ("ws", C.c_void_p),
+                ("ws_bytes", C.c_longlong), ("ep_scale", C.c_float), ("row_vec", C.c_void_p),
+                ("row_vec_gstride", C.c_longlong)]
 
 
 class LaunchRecord(C.Structure):
@@ -73,7 +75,7 @@ class LaunchRecord(C.Structure):
 
 
 KIND_NAMES = ("gemm", "ln_fwd", "ln_bwd", "softmax_fwd", "softmax_bwd", "colsum", "reduce",
-              "overflow", "adam", "scale")
+              "overflow", "adam", "scale", "splitk", "attn_fwd", "rowdot")
 
 _lib = None
 
@@ -107,6 +109,8 @@ _SIGS = {
     "gptl_colsum_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "gptl_colsum": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_longlong, C.c_longlong, C.c_int,
                               C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "gptl_attention_fwd": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gptl_colsum_noalloc": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_longlong, C.c_longlong,
                                       C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gptl_launch_count": (C.c_ulonglong, []),
@@ -259,6 +263,11 @@ def colsum_scratch_bytes(n, groups) -> int:
 def colsum(rows, n, groups, ld, gstride, dtype, a, out, scratch, stream=0):
     _check(lib().gptl_colsum(rows, n, groups, ld, gstride, DTYPES.get(dtype, dtype), _ptr(a),
                              _ptr(out), _ptr(scratch), stream), "gptl_colsum")
+
+
+def attention_fwd(batch, seq, hidden, heads, tp, dtype, qkv, o, lse, stream=0):
+    _check(lib().gptl_attention_fwd(batch, seq, hidden, heads, tp, DTYPES.get(dtype, dtype), _ptr(qkv),
+                                    _ptr(o), _ptr(lse), stream), "gptl_attention_fwd")
 
 
 def colsum_noalloc(rows, n, groups, ld, gstride, dtype, a, out, stream=0):

@@ -90,12 +90,13 @@ class LayerStep:
     def stream(self) -> int:
         return torch.cuda.current_stream(self.device).cuda_stream
 
-    def fwd(self):
-        G.layer_fwd(self.shape, self.weights, self.x, self.y, self.saved, None, self.stream())
+    def fwd(self, x=None, y=None):
+        G.layer_fwd(self.shape, self.weights, self.x if x is None else x,
+                    self.y if y is None else y, self.saved, None, self.stream())
 
-    def bwd(self):
-        G.layer_bwd(self.shape, self.weights, self.x, self.saved, self.dy, self.dx, self.grads,
-                    self.scratch, self.stream())
+    def bwd(self, x=None, dy=None):
+        G.layer_bwd(self.shape, self.weights, self.x if x is None else x, self.saved,
+                    self.dy if dy is None else dy, self.dx, self.grads, self.scratch, self.stream())
 
     def adam(self):
         hp = self.hyper
@@ -108,9 +109,11 @@ class LayerStep:
         G.scale_update(self.state, hp["growth_interval"], hp["growth_factor"],
                        hp["backoff_factor"], hp["min_scale"], self.stream())
 
-    def step(self):
-        self.fwd()
-        self.bwd()
+    def step(self, x=None, dy=None, y=None):
+        """fwd + bwd + Adam + scale update; x, dy and y default to this object's
+        buffers (other device buffers of the same shape may be passed)."""
+        self.fwd(x, y)
+        self.bwd(x, dy)
         self.adam()
         self.scale_update()
 
