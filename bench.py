@@ -83,6 +83,8 @@ def kernel_bytes(cfg, n_params: int) -> dict:
         "B6 ln2 bwd": 14 * T * h,   # read dL2, H (fp32), dOut; write dH (16-bit and fp32)
         "B12 ln1 bwd": 10 * T * h,  # read dL1, X, dH (fp32); write dX
         "B9 rowdot": 4 * T * h,                               # read dO and O
+        "B2 dOut^T": 4 * T * h, "B5 L2^T": 4 * T * h,         # transposes: read + write
+        "B7 dH^T": 4 * T * h, "B11 L1^T": 4 * T * h,
         "B3 db1": 2 * T * f, "B11 dbqkv": 2 * T * 3 * h,
         "O1 overflow": 4 * n_params, "O2 adam": 30 * n_params,
     }
@@ -439,8 +441,9 @@ def main():
                                              peaks, flops)
     # the tensor-core kernels: every GEMM launch (with its split-K sums) and
     # the fused attention forward; the work is the step's algorithmic FLOPs
-    # (the backward's recomputation of P is not counted)
-    gemm_ms = sum(kinds.get(k, {}).get("ms_per_step", 0.0) for k in ("gemm", "splitk", "attn_fwd"))
+    # (the backward's recomputation of S and dP is not counted)
+    gemm_ms = sum(kinds.get(k, {}).get("ms_per_step", 0.0)
+                  for k in ("gemm", "splitk", "attn_fwd", "attn_bwd"))
     peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     achieved_tf = flops["causal"] / (gemm_ms * 1e-3) / 1e12 if gemm_ms else None
     traffic = recorded_traffic(cfg.name)
@@ -454,8 +457,8 @@ def main():
         "tflops_causal": round(flops["causal"] / (ms * 1e-3) / 1e12, 1),
         "tflops_dense_convention": round(flops["dense"] / (ms * 1e-3) / 1e12, 1),
         "frac_of_bf16_peak": round(flops["causal"] / (ms * 1e-3) / 1e12 / peak_tf, 4),
-        "roofline": {"kernel": "tcgen05 kernels of a step: gemm_tc_kernel (with split-K sums) "
-                               "and attn_fwd_kernel",
+        "roofline": {"kernel": "tcgen05 kernels of a step: gemm_tc_kernel (with split-K sums), "
+                               "attn_fwd_kernel, attn_bwd_dq_kernel, attn_bwd_kv_kernel",
                      "bound": "tensor",
                      "achieved": round(achieved_tf, 1) if achieved_tf else None,
                      "peak": peak_tf, "unit": "TFLOP/s",

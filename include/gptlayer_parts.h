@@ -105,6 +105,17 @@ int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream);
 int gptl_attention_fwd(int batch, int seq, int hidden, int heads, int tp, gptl_dtype dtype,
                        const void *qkv, void *o, float *lse, gptl_stream_t stream);
 
+/* Fused causal attention backward, the counterpart of gptl_attention_fwd.
+ * Given qkv, o and lse of the forward and dout ([tp][batch*seq][h/tp], the
+ * gradient with respect to o), writes dQ, dK and dV into the Q, K and V
+ * columns of dqkv (same layout as qkv); dvec ([g][seq] fp32, caller scratch)
+ * receives D = dO . O per row.  With P = softmax(Q K^T / sqrt(d)) (causal):
+ *   dV = P^T dO,  dS = P (dO V^T - D) / sqrt(d),  dQ = dS K,  dK = dS^T Q,
+ * P taken in the 16-bit type.  Same size limits as gptl_attention_fwd. */
+int gptl_attention_bwd(int batch, int seq, int hidden, int heads, int tp, gptl_dtype dtype,
+                       const void *qkv, const void *o, const void *dout, const float *lse,
+                       float *dvec, void *dqkv, gptl_stream_t stream);
+
 /* LayerNorm forward over `rows` rows of width h: y = g*(x-mu)*rstd + b with the
  * biased variance; mu and rstd ([rows] fp32) are saved for the backward.
  * h must split as h/8 = TPR*VPT with TPR a power of two in [16, 256], VPT <= 8. */

@@ -38,7 +38,9 @@ enum {
   GPTL_KIND_SPLITK = 10,     /* sum of a split-K GEMM's partial tiles         */
   GPTL_KIND_ATTN_FWD = 11,   /* fused causal attention forward                */
   GPTL_KIND_ROWDOT = 12,     /* softmax-backward row term dO . O              */
-  GPTL_KIND_COUNT = 13
+  GPTL_KIND_TRANSPOSE = 13,  /* token-contiguous copy of a gradient operand   */
+  GPTL_KIND_ATTN_BWD = 14,   /* fused causal attention backward (dQ; dK, dV)  */
+  GPTL_KIND_COUNT = 15
 };
 
 /* step tags */
@@ -47,11 +49,11 @@ enum {
   GPTL_TAG_F1_LN1, GPTL_TAG_F2_QKV, GPTL_TAG_F3_F5_ATTN,
   GPTL_TAG_F6_OUTPROJ, GPTL_TAG_F7_LN2, GPTL_TAG_F8_FFN1_GELU, GPTL_TAG_F10_FFN2,
   GPTL_TAG_B1_B3_DZ, GPTL_TAG_B2_DW2, GPTL_TAG_B2_DB2, GPTL_TAG_B3_DB1, GPTL_TAG_B4_DL2,
-  GPTL_TAG_B5_DW1, GPTL_TAG_B6_LN2, GPTL_TAG_B7_DWO, GPTL_TAG_B7_DO, GPTL_TAG_B8_P,
-  GPTL_TAG_B9_ROWDOT, GPTL_TAG_B8_B9_DS, GPTL_TAG_B8_DV, GPTL_TAG_B10_DQ, GPTL_TAG_B10_DK,
-  GPTL_TAG_B11_DBQKV,
+  GPTL_TAG_B5_DW1, GPTL_TAG_B6_LN2, GPTL_TAG_B7_DWO, GPTL_TAG_B7_DO, GPTL_TAG_B9_ROWDOT,
+  GPTL_TAG_B8_B10_ATTN, GPTL_TAG_B11_DBQKV,
   GPTL_TAG_B11_DWQKV, GPTL_TAG_B11_DL1, GPTL_TAG_B12_LN1,
   GPTL_TAG_O1_OVERFLOW, GPTL_TAG_O2_ADAM, GPTL_TAG_O3_SCALE,
+  GPTL_TAG_B2_DOUT_T, GPTL_TAG_B5_L2_T, GPTL_TAG_B7_DH_T, GPTL_TAG_B11_L1_T, GPTL_TAG_B0_WT,
   GPTL_TAG_COUNT
 };
 

@@ -313,6 +313,43 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T *__restrict__ a, in
   }
 }
 
+// -------------------------------------------------------------- transpose
+// out[c][r] = in[r][c] for a rows x cols 16-bit matrix (row pitches in
+// elements; rows, cols, pitches multiples of 8).  64 x 64 tiles through
+// shared memory: 16-byte coalesced loads, and each thread stores 32
+// contiguous bytes of an output row.
+// blockIdx.z indexes a batch of matrices (pitches bs_in, bs_out elements).
+__global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t *__restrict__ in,
+                                                          uint16_t *__restrict__ out, int rows,
+                                                          int cols, long long ld_in,
+                                                          long long ld_out, long long bs_in,
+                                                          long long bs_out) {
+  __shared__ __align__(16) uint16_t tile[64][64 + 8];
+  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+  in += (long long)blockIdx.z * bs_in;
+  out += (long long)blockIdx.z * bs_out;
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int i = threadIdx.x + it * 256;
+    const int r = i >> 3, v = i & 7;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (r0 + r < rows && c0 + v * 8 < cols)
+      val = __ldcs(reinterpret_cast<const uint4 *>(in + (long long)(r0 + r) * ld_in + c0 + v * 8));
+    *reinterpret_cast<uint4 *>(&tile[r][v * 8]) = val;
+  }
+  __syncthreads();
+  const int c = threadIdx.x & 63, vp = threadIdx.x >> 6;   // output row c0+c, elements 16vp..16vp+15
+  if (c0 + c < cols) {
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      w[k] = (uint32_t)tile[vp * 16 + 2 * k][c] | ((uint32_t)tile[vp * 16 + 2 * k + 1][c] << 16);
+    uint16_t *dst = out + (long long)(c0 + c) * ld_out + r0 + vp * 16;
+    if (r0 + vp * 16 < rows) *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (r0 + vp * 16 + 8 < rows) *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
 // --------------------------------------------------------- causal softmax
 // In place on [rows = G*s][s] score blocks.  Row p of a block: entries q <= p
 // get softmax(scale * S), entries p < q < end of the 128-wide diagonal tile

@@ -136,9 +136,51 @@ __device__ __forceinline__ uint64_t operand_desc(const OperandRule &r, uint32_t 
                         swizzle_layout(r.w));
 }
 
+// Global inputs of one 16-column epilogue chunk, loaded one chunk ahead so
+// that their latency overlaps the previous chunk's arithmetic.
+struct EpiIn {
+  uint4 bias[2];     // 16-bit bias
+  uint4 aux[2];      // 16-bit aux (GeLU' argument or P)
+  uint4 r16[2];      // 16-bit residual
+  float4 r32[4];     // fp32 residual
+};
+
+template <typename T>
+__device__ __forceinline__ void epilogue_load(const GemmParams &p, int g, int row, int n, EpiIn &in) {
+  if (p.split > 1 || row >= p.M) return;
+  if (p.bias) {
+    const uint4 *b = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.bias) +
+                                                     (long long)g * p.bias_g_stride + n);
+    in.bias[0] = __ldg(b);
+    in.bias[1] = __ldg(b + 1);
+  }
+  if (p.resid) {
+    if (p.resid_f32) {
+      const float4 *rr = reinterpret_cast<const float4 *>(static_cast<const float *>(p.resid) +
+                                                          (long long)row * p.ld_resid + n);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) in.r32[q] = rr[q];
+    } else {
+      const uint4 *rr = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.resid) +
+                                                        (long long)row * p.ld_resid + n);
+      in.r16[0] = rr[0];
+      in.r16[1] = rr[1];
+    }
+  }
+  if (p.act == kActDGelu || p.act == kActDSoftmax) {
+    const long long off = (long long)(g % p.o_mod) * p.o_str_mod +
+                          (long long)(g / p.o_mod) * p.o_str_div + (long long)row * p.ldo + n;
+    const uint4 *xp = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.aux) + off);
+    in.aux[0] = xp[0];
+    in.aux[1] = xp[1];
+  }
+}
+
+// rv: the row's entry of row_vec (EXP_LSE / DSOFTMAX), loaded once per tile.
 template <typename T>
 __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int row, int n,
-                                               int slice, const uint32_t (&r)[16]) {
+                                               int slice, const uint32_t (&r)[16], const EpiIn &in,
+                                               float rv) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
@@ -152,32 +194,26 @@ __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int r
   const long long off = (long long)(g % p.o_mod) * p.o_str_mod +
                         (long long)(g / p.o_mod) * p.o_str_div + (long long)row * p.ldo + n;
   if (p.bias) {
-    const uint4 *b = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.bias) +
-                                                     (long long)g * p.bias_g_stride + n);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float f[8];
-      unpack8<T>(__ldg(b + h), f);
+      unpack8<T>(in.bias[h], f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[8 * h + i] += f[i];
     }
   }
   if (p.resid) {
     if (p.resid_f32) {
-      const float4 *rr = reinterpret_cast<const float4 *>(static_cast<const float *>(p.resid) +
-                                                          (long long)row * p.ld_resid + n);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float4 f = rr[q];
-        v[4 * q] += f.x; v[4 * q + 1] += f.y; v[4 * q + 2] += f.z; v[4 * q + 3] += f.w;
+        v[4 * q] += in.r32[q].x; v[4 * q + 1] += in.r32[q].y;
+        v[4 * q + 2] += in.r32[q].z; v[4 * q + 3] += in.r32[q].w;
       }
     } else {
-      const uint4 *rr = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.resid) +
-                                                        (long long)row * p.ld_resid + n);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float f[8];
-        unpack8<T>(rr[h], f);
+        unpack8<T>(in.r16[h], f);
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[8 * h + i] += f[i];
       }
@@ -211,31 +247,24 @@ __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int r
     // attention probabilities recomputed from the scores and the row's
     // base-2 log-sum-exp, or the softmax backward; both zero above the
     // diagonal (column n > row)
-    const float rv = p.row_vec[(long long)g * p.row_vec_gstride + row];
-    float pr[16];
-    if (p.act == kActDSoftmax) {
-      const uint4 *pp = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.aux) + off);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float f[8];
-        unpack8<T>(pp[h], f);
+    for (int h = 0; h < 2; ++h) {
+      float pr[8];
+      if (p.act == kActDSoftmax) unpack8<T>(in.aux[h], pr);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) pr[8 * h + i] = f[i];
+      for (int i = 0; i < 8; ++i) {
+        const float x = v[8 * h + i];
+        const float val = p.act == kActExpLse ? exp2f(x * p.ep_scale - rv)
+                                              : p.ep_scale * pr[i] * (x - rv);
+        v[8 * h + i] = (n + 8 * h + i > row) ? 0.f : val;
       }
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float val = p.act == kActExpLse ? exp2f(v[i] * p.ep_scale - rv)
-                                            : p.ep_scale * pr[i] * (v[i] - rv);
-      v[i] = (n + i > row) ? 0.f : val;
     }
   }
   if (p.act == kActDGelu) {
-    const uint4 *zp = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.aux) + off);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float z[8];
-      unpack8<T>(zp[h], z);
+      unpack8<T>(in.aux[h], z);
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[8 * h + i] *= gelu_prime_f(z[i]);
     }
@@ -390,19 +419,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       // software pipeline: the load of chunk c+1 is in flight while chunk c
       // is processed (tcgen05.wait::ld waits for every earlier load)
       uint32_t ra[16], rb[16];
+      EpiIn ia, ib;
+      float rv = 0.f;
+      if ((p.act == kActExpLse || p.act == kActDSoftmax) && row < p.M)
+        rv = p.row_vec[(long long)ti.g * p.row_vec_gstride + row];
       if (c0 < c1) {
         tmem_ld16(t_row + (uint32_t)(c0 * 16), ra);
+        epilogue_load<T>(p, ti.g, row, ti.n0 + c0 * 16, ia);
         tmem_wait_ld();
       }
       for (int c = c0; c < c1; c += 2) {
         const bool has_b = c + 1 < c1;
-        if (has_b) tmem_ld16(t_row + (uint32_t)((c + 1) * 16), rb);
-        if (row < p.M) epilogue_store<T>(p, ti.g, row, ti.n0 + c * 16, ti.slice, ra);
+        if (has_b) {
+          tmem_ld16(t_row + (uint32_t)((c + 1) * 16), rb);
+          epilogue_load<T>(p, ti.g, row, ti.n0 + (c + 1) * 16, ib);
+        }
+        if (row < p.M) epilogue_store<T>(p, ti.g, row, ti.n0 + c * 16, ti.slice, ra, ia, rv);
         tmem_wait_ld();
         if (!has_b) break;
         const bool has_a = c + 2 < c1;
-        if (has_a) tmem_ld16(t_row + (uint32_t)((c + 2) * 16), ra);
-        if (row < p.M) epilogue_store<T>(p, ti.g, row, ti.n0 + (c + 1) * 16, ti.slice, rb);
+        if (has_a) {
+          tmem_ld16(t_row + (uint32_t)((c + 2) * 16), ra);
+          epilogue_load<T>(p, ti.g, row, ti.n0 + (c + 2) * 16, ia);
+        }
+        if (row < p.M) epilogue_store<T>(p, ti.g, row, ti.n0 + (c + 1) * 16, ti.slice, rb, ib, rv);
         tmem_wait_ld();
       }
       tc_fence_before();

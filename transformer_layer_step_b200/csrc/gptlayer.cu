@@ -13,6 +13,7 @@
 
 #include "bw_kernels.cuh"
 #include "common.cuh"
+#include "attn_bwd_tc.cuh"
 #include "attn_tc.cuh"
 #include "gemm_tc.cuh"
 #include "gptlayer_parts.h"
@@ -419,6 +420,102 @@ int run_attn_fwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
   return GPTL_OK;
 }
 
+// Fused causal attention backward: dQ, dK, dV into the Q, K, V columns of
+// dC [t][T][3h/t] from C, dO [t][T][h/t], the forward's row log-sum-exp and
+// D = dO . O.  Two kernels (per query block: dQ; per key block: dK, dV).
+int run_attn_bwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, const void *c,
+                 const void *dout, const float *lse, const float *dvec, void *dc, cudaStream_t st) {
+  int sms = 0;
+  GPTL_TRY(device_check(&sms));
+  if (d % 16 || d > 128 || hs % 8 || s <= 0 || s % 16 || as <= 0 || b <= 0 || t <= 0)
+    return GPTL_E_SHAPE;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return GPTL_E_CUDA;
+  AttnBwdParams p;
+  memset(&p, 0, sizeof(p));
+  const CUtensorMapDataType ty =
+      dt == GPTL_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint32_t es[3] = {1, 1, 1}, box[3] = {16, 128, 1};
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)(3 * hs), (cuuint64_t)s, (cuuint64_t)t * b};
+    cuuint64_t strides[2] = {(cuuint64_t)3 * hs * 2, (cuuint64_t)s * 3 * hs * 2};
+    if (fn(&p.map_c, ty, 3, const_cast<void *>(c), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GPTL_E_CUDA;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)hs, (cuuint64_t)s, (cuuint64_t)t * b};
+    cuuint64_t strides[2] = {(cuuint64_t)hs * 2, (cuuint64_t)s * hs * 2};
+    if (fn(&p.map_do, ty, 3, const_cast<void *>(dout), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GPTL_E_CUDA;
+  }
+  p.s = s; p.d = d; p.hs = hs; p.as = as;
+  p.groups = t * b * as;
+  p.tiles = (s + 127) / 128;
+  p.scale = 1.0f / sqrtf((float)d);
+  p.scale_log2 = 1.4426950408889634f * p.scale;
+  const uint32_t fmt = dt == GPTL_BF16 ? 1u : 0u;
+  p.idesc_s = (1u << 4) | (fmt << 7) | (fmt << 10) | (16u << 17) | (8u << 24);
+  p.idesc_acc = (1u << 4) | (fmt << 7) | (fmt << 10) | (1u << 16) | ((uint32_t)(d >> 3) << 17) | (8u << 24);
+  p.lse = lse;
+  p.dvec = dvec;
+  p.dc = dc;
+  p.items = (long long)p.groups * p.tiles;
+  p.q_off = 0; p.k_off = hs; p.v_off = 2 * hs;
+  const int tb = 256 * d;
+  int smem_dq = 1024 + 32768 + 6 * tb + 256;
+  int nst = 2;
+  int smem_kv = 1024 + 65536 + 2 * tb + nst * 2 * tb + 2048 + 256;
+  if (smem_kv > kSmemLimit) {
+    nst = 1;
+    smem_kv = 1024 + 65536 + 2 * tb + nst * 2 * tb + 2048 + 256;
+  }
+  p.qdo_stages = nst;
+  // at least 120 KB: one CTA (and its 512 tensor-memory columns) per SM
+  if (smem_dq < 120 * 1024) smem_dq = 120 * 1024;
+  if (smem_kv < 120 * 1024) smem_kv = 120 * 1024;
+  if (smem_dq > kSmemLimit || smem_kv > kSmemLimit) return GPTL_E_SHAPE;
+  const int grid = (int)(p.items < sms ? p.items : sms);
+  static bool attr_set[kMaxDevices][2] = {};
+  int dev = 0;
+  GPTL_CK(cudaGetDevice(&dev));
+  auto launch = [&](auto kq, auto kkv) -> int {
+    if (!attr_set[dev][dt]) {
+      GPTL_CK(cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
+      GPTL_CK(cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
+      attr_set[dev][dt] = true;
+    }
+    kq<<<grid, kAttnBwdThreads, smem_dq, st>>>(p);
+    GPTL_CK(cudaGetLastError());
+    prof_launched(st, GPTL_KIND_ATTN_BWD);
+    kkv<<<grid, kAttnBwdThreads, smem_kv, st>>>(p);
+    GPTL_CK(cudaGetLastError());
+    prof_launched(st, GPTL_KIND_ATTN_BWD);
+    return GPTL_OK;
+  };
+  if (dt == GPTL_FP16) return launch(attn_bwd_dq_kernel<__half>, attn_bwd_kv_kernel<__half>);
+  return launch(attn_bwd_dq_kernel<__nv_bfloat16>, attn_bwd_kv_kernel<__nv_bfloat16>);
+}
+
+// out [cols][rows] = in [rows][cols]^T (16-bit), for `batch` matrices
+// `bs_in` / `bs_out` elements apart.
+int run_transpose(int rows, int cols, const void *in, long long ld_in, void *out, long long ld_out,
+                  cudaStream_t st, int batch = 1, long long bs_in = 0, long long bs_out = 0) {
+  if (rows <= 0 || cols <= 0 || rows % 8 || cols % 8 || ld_in % 8 || ld_out % 8 || batch < 1 ||
+      bs_in % 8 || bs_out % 8)
+    return GPTL_E_SHAPE;
+  dim3 grid((cols + 63) / 64, (rows + 63) / 64, batch);
+  transpose16_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(in),
+                                           static_cast<uint16_t *>(out), rows, cols, ld_in, ld_out,
+                                           bs_in, bs_out);
+  GPTL_CK(cudaGetLastError());
+  prof_launched(st, GPTL_KIND_TRANSPOSE);
+  return GPTL_OK;
+}
+
 // D[g][p] = dO_p . O_p over each head's columns (the softmax backward's row term).
 int run_attn_rowdot(long long rows, int s, int hs, int as, int d, gptl_dtype dt, const void *dout,
                     const void *o, float *dvec, cudaStream_t st) {
@@ -690,7 +787,8 @@ struct Ws {
   // saved (fwd -> bwd)
   size_t mu1, rstd1, mu2, rstd2, l1, c, lse, o, hid, l2, z, act, saved;
   // scratch (bwd)
-  size_t dz, dl2, dhid, dhid32, dO, p, dp, dvec, dc, dl1, part, splitk, splitk_bytes, scratch;
+  size_t dz, dl2, dhid, dhid32, dO, dvec, dc, dl1, xt, w2t, w1t, wot, wqkvt, part, splitk,
+      splitk_bytes, scratch;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -716,10 +814,12 @@ Ws ws_layout(const Dims &D) {
   w.dz = take(T * f * e); w.dl2 = take(T * h * e); w.dhid = take(T * h * e);
   w.dhid32 = take(T * h * 4);          // residual-stream gradient dH, fp32
   w.dO = take(T * h * e);
-  w.p = take(pe * e);                   // P recomputed for the backward
-  w.dp = take(pe * e);                  // dS
   w.dvec = take((size_t)D.b * D.a * D.s * 4);
   w.dc = take(3 * T * h * e); w.dl1 = take(T * h * e);
+  w.xt = take(T * h * e);               // [h][T] transposed operand of a weight gradient
+  // transposed 16-bit weights ([in][out] per shard) for the input-gradient GEMMs
+  w.w2t = take(h * f * e); w.w1t = take(f * h * e); w.wot = take(h * h * e);
+  w.wqkvt = take(3 * h * h * e);
   size_t part = 4 * 512 * h;
   const size_t widest = f > 3 * h ? f : 3 * h;
   if (kColsumMaxSplit * widest > part) part = kColsumMaxSplit * widest;
@@ -876,9 +976,11 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   void *dz = at<void>(scratch, w.dz), *dl2 = at<void>(scratch, w.dl2);
   float *dhid32 = at<float>(scratch, w.dhid32);
   void *dhid = at<void>(scratch, w.dhid), *dO = at<void>(scratch, w.dO);
-  void *dp = at<void>(scratch, w.dp), *dc = at<void>(scratch, w.dc), *dl1 = at<void>(scratch, w.dl1);
-  void *pb = at<void>(scratch, w.p);
+  void *dc = at<void>(scratch, w.dc), *dl1 = at<void>(scratch, w.dl1);
   float *dvec = at<float>(scratch, w.dvec);
+  void *xt = at<void>(scratch, w.xt);   // [h][T]: one token-contiguous copy at a time
+  void *w2t = at<void>(scratch, w.w2t), *w1t = at<void>(scratch, w.w1t);
+  void *wot = at<void>(scratch, w.wot), *wqkvt = at<void>(scratch, w.wqkvt);
   float *part = at<float>(scratch, w.part);
   void *splitk = at<void>(scratch, w.splitk);
   const long long splitk_bytes = (long long)w.splitk_bytes;
@@ -886,10 +988,25 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   TagScope tag_scope(GPTL_TAG_NONE);
   prof_start(st);
 
+  // The input-gradient GEMMs read the weights with the reduction index
+  // contiguous: transposed copies, shard by shard.
+  g_tag = GPTL_TAG_B0_WT;
+  GPTL_TRY(run_transpose(h, fs, W->w_2, fs, w2t, h, st, t, (long long)h * fs, (long long)fs * h));
+  GPTL_TRY(run_transpose(fs, h, W->w_1, h, w1t, fs, st, t, (long long)fs * h, (long long)h * fs));
+  GPTL_TRY(run_transpose(h, hs, W->w_o, hs, wot, h, st, t, (long long)h * hs, (long long)hs * h));
+  GPTL_TRY(run_transpose(3 * hs, h, W->w_qkv, h, wqkvt, 3 * hs, st, t, (long long)3 * hs * h,
+                         (long long)h * 3 * hs));
+
   // ---- FFN2 (row split)
   g_tag = GPTL_TAG_B2_DW2;
+  // Weight gradients reduce over the tokens, the row index of both
+  // activations; the tensor core runs markedly faster when one operand is
+  // token-contiguous, so the smaller operand is transposed first.
+  g_tag = GPTL_TAG_B2_DOUT_T;
+  GPTL_TRY(run_transpose(T, h, dy, h, xt, T, st));
+  g_tag = GPTL_TAG_B2_DW2;
   {  // dW2_i = dOut^T A_i   [t][h][f/t] fp32
-    gptl_gemm_desc g = gemm(h, fs, T, t, view(dy, h, T, 1, h, 0, 1),
+    gptl_gemm_desc g = gemm(h, fs, T, t, view(xt, T, h, 1, T, 0, 0),
                             view(act, fs, T, t, fs, (long long)T * fs, 1), gr->w_2, fs,
                             (long long)h * fs);
     g.out_f32 = 1;
@@ -900,7 +1017,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   g_tag = GPTL_TAG_B1_B3_DZ;
   {  // dZ_i = (dOut W2_i) * gelu'(Z_i)
     gptl_gemm_desc g = gemm(T, fs, h, t, view(dy, h, T, 1, h, 0, 0),
-                            view(W->w_2, fs, h, t, fs, (long long)h * fs, 1), dz, fs,
+                            view(w2t, h, fs, t, h, (long long)fs * h, 0), dz, fs,
                             (long long)T * fs);
     g.act = GPTL_ACT_DGELU;
     g.aux = z;
@@ -909,10 +1026,12 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   // ---- FFN1 (column split)
   g_tag = GPTL_TAG_B3_DB1;
   GPTL_TRY(run_colsum(T, fs, t, fs, (long long)T * fs, dt, dz, gr->b_1, part, st));
+  g_tag = GPTL_TAG_B5_L2_T;
+  GPTL_TRY(run_transpose(T, h, l2, h, xt, T, st));
   g_tag = GPTL_TAG_B5_DW1;
   {  // dW1_i = dZ_i^T L2   [t][f/t][h]
     gptl_gemm_desc g = gemm(fs, h, T, t, view(dz, fs, T, t, fs, (long long)T * fs, 1),
-                            view(l2, h, T, 1, h, 0, 1), gr->w_1, h, (long long)fs * h);
+                            view(xt, T, h, 1, T, 0, 0), gr->w_1, h, (long long)fs * h);
     g.out_f32 = 1;
     g.ws = splitk;
     g.ws_bytes = splitk_bytes;
@@ -922,7 +1041,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   {  // dL2 = sum_i dZ_i W1_i  (shard sum in the K loop)
     gptl_operand a = view(dz, fs, T, t, fs, (long long)T * fs, 0);
     a.g_div = kNoGroup; a.k_shard = 1;
-    gptl_operand b = view(W->w_1, h, fs, t, h, (long long)fs * h, 1);
+    gptl_operand b = view(w1t, fs, h, t, fs, (long long)h * fs, 0);
     b.g_div = kNoGroup; b.k_shard = 1;
     gptl_gemm_desc g = gemm(T, h, fs, 1, a, b, dl2, h, 0);
     g.k_shards = t;
@@ -934,9 +1053,11 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   GPTL_TRY(run_ln_bwd(LNB_H, T, h, dt, dl2, hid, mu2, rs2, W->ln2_g, dy, dhid, dhid32, gr->ln2_g,
                       gr->ln2_b, gr->b_o, gr->b_2, part, st));
   // ---- out-projection (row split)
+  g_tag = GPTL_TAG_B7_DH_T;
+  GPTL_TRY(run_transpose(T, h, dhid, h, xt, T, st));
   g_tag = GPTL_TAG_B7_DWO;
   {  // dWo_i = dH^T O_i   [t][h][h/t]
-    gptl_gemm_desc g = gemm(h, hs, T, t, view(dhid, h, T, 1, h, 0, 1),
+    gptl_gemm_desc g = gemm(h, hs, T, t, view(xt, T, h, 1, T, 0, 0),
                             view(o, hs, T, t, hs, (long long)T * hs, 1), gr->w_o, hs,
                             (long long)h * hs);
     g.out_f32 = 1;
@@ -947,85 +1068,25 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   g_tag = GPTL_TAG_B7_DO;
   {  // dO_i = dH Wo_i   [t][T][h/t]
     gptl_gemm_desc g = gemm(T, hs, h, t, view(dhid, h, T, 1, h, 0, 0),
-                            view(W->w_o, hs, h, t, hs, (long long)h * hs, 1), dO, hs,
+                            view(wot, h, hs, t, h, (long long)hs * h, 0), dO, hs,
                             (long long)T * hs);
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // ---- attention backward
-  gptl_operand dOv = view(dO, hs, s, (long long)t * D.b, hs, (long long)s * hs, 0);
-  dOv.x_mod = as; dOv.x_mul = d; dOv.g_div = as;
-  gptl_operand cv = view(c, 3 * hs, s, (long long)t * D.b, 3 * hs, (long long)s * 3 * hs, 0);
-  cv.x_mod = as; cv.x_mul = d; cv.g_div = as;
-  g_tag = GPTL_TAG_B8_P;
-  {  // P = exp2(Q K^T * log2(e)/sqrt(d) - lse), recomputed for the lower-triangle tiles
-    gptl_operand k = cv;
-    k.x_off = hs;
-    gptl_gemm_desc g = gemm(s, s, d, G, cv, k, pb, s, (long long)s * s);
-    g.causal = GPTL_CAUSAL_SKIP_UPPER;
-    g.act = GPTL_ACT_EXP_LSE;
-    g.ep_scale = 1.4426950408889634f * attn_scale;
-    g.row_vec = lse;
-    g.row_vec_gstride = s;
-    GPTL_TRY(run_gemm(g, dt, st));
-  }
   g_tag = GPTL_TAG_B9_ROWDOT;   // D = rowsum(dO * O), the softmax backward's row term
   GPTL_TRY(run_attn_rowdot((long long)t * T, s, hs, as, d, dt, dO, o, dvec, st));
-  g_tag = GPTL_TAG_B8_B9_DS;
-  {  // dS = P (dO V^T - D) / sqrt(d) in the epilogue of the dP GEMM (lower-triangle tiles)
-    gptl_operand v = cv;
-    v.x_off = 2 * hs;
-    gptl_gemm_desc g = gemm(s, s, d, G, dOv, v, dp, s, (long long)s * s);
-    g.causal = GPTL_CAUSAL_SKIP_UPPER;
-    g.act = GPTL_ACT_DSOFTMAX;
-    g.ep_scale = attn_scale;
-    g.aux = pb;
-    g.row_vec = dvec;
-    g.row_vec_gstride = s;
-    GPTL_TRY(run_gemm(g, dt, st));
-  }
-  g_tag = GPTL_TAG_B8_DV;
-  {  // dV = P^T dO  -> V columns of dC
-    gptl_operand a = view(pb, s, s, G, s, (long long)s * s, 1);
-    gptl_operand b = dOv;
-    b.mn_major = 1;
-    gptl_gemm_desc g = gemm(s, d, s, G, a, b, at<void>(dc, (size_t)2 * hs * 2), 3 * hs,
-                            (long long)s * 3 * hs);
-    g.o_mod = as;
-    g.o_str_mod = d;
-    g.causal = GPTL_CAUSAL_K_FROM;
-    GPTL_TRY(run_gemm(g, dt, st));
-  }
-  g_tag = GPTL_TAG_B10_DQ;
-  {  // dQ = dS K  -> Q columns of dC
-    gptl_operand a = view(dp, s, s, G, s, (long long)s * s, 0);
-    gptl_operand b = cv;
-    b.mn_major = 1;
-    b.x_off = hs;
-    gptl_gemm_desc g = gemm(s, d, s, G, a, b, dc, 3 * hs, (long long)s * 3 * hs);
-    g.o_mod = as;
-    g.o_str_mod = d;
-    g.causal = GPTL_CAUSAL_K_BELOW;
-    GPTL_TRY(run_gemm(g, dt, st));
-  }
-  g_tag = GPTL_TAG_B10_DK;
-  {  // dK = dS^T Q  -> K columns of dC
-    gptl_operand a = view(dp, s, s, G, s, (long long)s * s, 1);
-    gptl_operand b = cv;
-    b.mn_major = 1;
-    gptl_gemm_desc g = gemm(s, d, s, G, a, b, at<void>(dc, (size_t)hs * 2), 3 * hs,
-                            (long long)s * 3 * hs);
-    g.o_mod = as;
-    g.o_str_mod = d;
-    g.causal = GPTL_CAUSAL_K_FROM;
-    GPTL_TRY(run_gemm(g, dt, st));
-  }
+  // fused attention backward: dQ, dK, dV into dC (P and dS stay on chip)
+  g_tag = GPTL_TAG_B8_B10_ATTN;
+  GPTL_TRY(run_attn_bwd(D.b, s, hs, as, t, d, dt, c, dO, lse, dvec, dc, st));
   // ---- QKV (column split)
   g_tag = GPTL_TAG_B11_DBQKV;
   GPTL_TRY(run_colsum(T, 3 * hs, t, 3 * hs, (long long)T * 3 * hs, dt, dc, gr->b_qkv, part, st));
+  g_tag = GPTL_TAG_B11_L1_T;
+  GPTL_TRY(run_transpose(T, h, l1, h, xt, T, st));
   g_tag = GPTL_TAG_B11_DWQKV;
   {  // dWqkv_i = dC_i^T L1   [t][3h/t][h]
     gptl_gemm_desc g = gemm(3 * hs, h, T, t, view(dc, 3 * hs, T, t, 3 * hs, (long long)T * 3 * hs, 1),
-                            view(l1, h, T, 1, h, 0, 1), gr->w_qkv, h, (long long)3 * hs * h);
+                            view(xt, T, h, 1, T, 0, 0), gr->w_qkv, h, (long long)3 * hs * h);
     g.out_f32 = 1;
     g.ws = splitk;
     g.ws_bytes = splitk_bytes;
@@ -1035,7 +1096,7 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   {  // dL1 = sum_i dC_i Wqkv_i
     gptl_operand a = view(dc, 3 * hs, T, t, 3 * hs, (long long)T * 3 * hs, 0);
     a.g_div = kNoGroup; a.k_shard = 1;
-    gptl_operand b = view(W->w_qkv, h, 3 * hs, t, h, (long long)3 * hs * h, 1);
+    gptl_operand b = view(wqkvt, 3 * hs, h, t, 3 * hs, (long long)h * 3 * hs, 0);
     b.g_div = kNoGroup; b.k_shard = 1;
     gptl_gemm_desc g = gemm(T, h, 3 * hs, 1, a, b, dl1, h, 0);
     g.k_shards = t;
@@ -1295,6 +1356,25 @@ int gptl_attention_fwd(int batch, int seq, int hidden, int heads, int tp, gptl_d
   return run_attn_fwd(batch, seq, hidden / tp, heads / tp, tp, hidden / heads, dtype, qkv, o, lse, st);
 }
 
+int gptl_attention_bwd(int batch, int seq, int hidden, int heads, int tp, gptl_dtype dtype,
+                       const void *qkv, const void *o, const void *dout, const float *lse,
+                       float *dvec, void *dqkv, gptl_stream_t stream) {
+  if (!qkv || !o || !dout || !lse || !dvec || !dqkv) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(qkv) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) || !aligned16(dvec) ||
+      !aligned16(dqkv))
+    return GPTL_E_ALIGN;
+  if (batch <= 0 || seq <= 0 || hidden <= 0 || heads <= 0 || tp <= 0) return GPTL_E_SHAPE;
+  if (hidden % heads || heads % tp) return GPTL_E_SHAPE;
+  GPTL_TRY(device_check());
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int hs = hidden / tp, as = heads / tp, d = hidden / heads;
+  if (d % 16 || d > 128 || seq % 16) return GPTL_E_SHAPE;
+  prof_start(st);
+  GPTL_TRY(run_attn_rowdot((long long)tp * batch * seq, seq, hs, as, d, dtype, dout, o, dvec, st));
+  return run_attn_bwd(batch, seq, hs, as, tp, d, dtype, qkv, dout, lse, dvec, dqkv, st);
+}
+
 // Column sums with their partials in a fixed device array instead of
 // caller memory (see gptl_colsum_noalloc in gptlayer_parts.h).
 int gptl_colsum_noalloc(int rows, int n, int groups, long long ld, long long gstride,
@@ -1392,16 +1472,17 @@ const char *gptl_tag_name(int tag) {
     case GPTL_TAG_B6_LN2: return "B6 ln2 bwd";
     case GPTL_TAG_B7_DWO: return "B7 dwo";
     case GPTL_TAG_B7_DO: return "B7 do";
-    case GPTL_TAG_B8_P: return "B8 P recompute";
-    case GPTL_TAG_B8_DV: return "B8 dv";
+    case GPTL_TAG_B8_B10_ATTN: return "B8-B10 attention bwd";
     case GPTL_TAG_B9_ROWDOT: return "B9 rowdot";
-    case GPTL_TAG_B8_B9_DS: return "B8/B9 dS";
-    case GPTL_TAG_B10_DQ: return "B10 dq";
-    case GPTL_TAG_B10_DK: return "B10 dk";
     case GPTL_TAG_B11_DBQKV: return "B11 dbqkv";
     case GPTL_TAG_B11_DWQKV: return "B11 dwqkv";
     case GPTL_TAG_B11_DL1: return "B11 dl1";
     case GPTL_TAG_B12_LN1: return "B12 ln1 bwd";
+    case GPTL_TAG_B0_WT: return "B0 weights^T";
+    case GPTL_TAG_B2_DOUT_T: return "B2 dOut^T";
+    case GPTL_TAG_B5_L2_T: return "B5 L2^T";
+    case GPTL_TAG_B7_DH_T: return "B7 dH^T";
+    case GPTL_TAG_B11_L1_T: return "B11 L1^T";
     case GPTL_TAG_O1_OVERFLOW: return "O1 overflow";
     case GPTL_TAG_O2_ADAM: return "O2 adam";
     case GPTL_TAG_O3_SCALE: return "O3 scale";

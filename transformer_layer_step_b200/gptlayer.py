@@ -75,7 +75,7 @@ class LaunchRecord(C.Structure):
 
 
 KIND_NAMES = ("gemm", "ln_fwd", "ln_bwd", "softmax_fwd", "softmax_bwd", "colsum", "reduce",
-              "overflow", "adam", "scale", "splitk", "attn_fwd", "rowdot")
+              "overflow", "adam", "scale", "splitk", "attn_fwd", "rowdot", "transpose", "attn_bwd")
 
 _lib = None
 
@@ -111,6 +111,7 @@ _SIGS = {
                               C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gptl_attention_fwd": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "gptl_attention_bwd": (C.c_int, [C.c_int] * 6 + [C.c_void_p] * 7),
     "gptl_colsum_noalloc": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_longlong, C.c_longlong,
                                       C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gptl_launch_count": (C.c_ulonglong, []),
@@ -268,6 +269,12 @@ def colsum(rows, n, groups, ld, gstride, dtype, a, out, scratch, stream=0):
 def attention_fwd(batch, seq, hidden, heads, tp, dtype, qkv, o, lse, stream=0):
     _check(lib().gptl_attention_fwd(batch, seq, hidden, heads, tp, DTYPES.get(dtype, dtype), _ptr(qkv),
                                     _ptr(o), _ptr(lse), stream), "gptl_attention_fwd")
+
+
+def attention_bwd(batch, seq, hidden, heads, tp, dtype, qkv, o, dout, lse, dvec, dqkv, stream=0):
+    _check(lib().gptl_attention_bwd(batch, seq, hidden, heads, tp, DTYPES.get(dtype, dtype), _ptr(qkv),
+                                    _ptr(o), _ptr(dout), _ptr(lse), _ptr(dvec), _ptr(dqkv), stream),
+           "gptl_attention_bwd")
 
 
 def colsum_noalloc(rows, n, groups, ld, gstride, dtype, a, out, stream=0):
