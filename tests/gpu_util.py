@@ -32,7 +32,8 @@ def stream() -> int:
 
 def check_device_error():
     torch.cuda.synchronize()
-    assert G.read_device_error(clear=True) == 0
+    word = G.read_device_error(clear=True)
+    assert word == 0, f"device error word {word:#x}"
 
 
 def rel_max_err(got: np.ndarray, ref: np.ndarray) -> float:

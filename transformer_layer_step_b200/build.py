@@ -17,8 +17,15 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libgptlayer.so")
 SOURCES = [os.path.join(PKG, "csrc", "gptlayer.cu")]
-DEPS = SOURCES + [os.path.join(PKG, "csrc", f) for f in ("common.cuh", "gemm_tc.cuh", "bw_kernels.cuh")] + \
-    [os.path.join(ROOT, "include", f) for f in ("gptlayer.h", "gptlayer_parts.h", "gptlayer_profile.h")]
+
+
+def deps() -> list:
+    """Every source and header the library is built from (rebuild if any is newer)."""
+    out = []
+    for d, exts in ((os.path.join(PKG, "csrc"), (".cu", ".cuh", ".h")),
+                    (os.path.join(ROOT, "include"), (".h",))):
+        out += [os.path.join(d, f) for f in sorted(os.listdir(d)) if f.endswith(exts)]
+    return out + [os.path.abspath(__file__)]
 
 
 def nvcc_path() -> str:
@@ -39,7 +46,7 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(d) <= t for d in DEPS)
+    return all(os.path.getmtime(d) <= t for d in deps())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

@@ -51,8 +51,7 @@ class LayerStep:
             self.param_shapes[name] = arr.shape
             flat_bits[off:off + arr.size] = arr.reshape(-1)
         self.w16 = bits_to_tensor(flat_bits, cfg.dtype, dev)
-        master = synth.from_bits(flat_bits, cfg.dtype).astype(np.float32)
-        self.master = torch.from_numpy(master).to(dev)
+        self.master = self.w16.to(torch.float32)       # exact: fp16/bf16 embed in fp32
         self.m = torch.zeros(self.n_params, dtype=torch.float32, device=dev)
         self.v = torch.zeros(self.n_params, dtype=torch.float32, device=dev)
         self.grad = torch.zeros(self.n_params, dtype=torch.float32, device=dev)
