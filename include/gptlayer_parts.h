@@ -37,12 +37,7 @@ typedef struct {
 enum {
   GPTL_ACT_NONE = 0,
   GPTL_ACT_GELU = 1,     /* out = value, out2 = GeLU(value)                   */
-  GPTL_ACT_DGELU = 2,    /* out = value * GeLU'(aux)                          */
-  GPTL_ACT_EXP_LSE = 3,  /* out = exp2(value * ep_scale - row_vec[G][m]);
-                            0 where n > m (attention probabilities from the
-                            scores and each row's base-2 log-sum-exp)         */
-  GPTL_ACT_DSOFTMAX = 4  /* out = ep_scale * aux * (value - row_vec[G][m]);
-                            0 where n > m (softmax backward from dP)          */
+  GPTL_ACT_DGELU = 2     /* out = value * GeLU'(aux)                          */
 };
 enum {
   GPTL_CAUSAL_NONE = 0,
@@ -61,7 +56,10 @@ enum {
  * by GeLU'(aux at the output's index).  out_f32 = 1 stores the fp32 value
  * (act must be GPTL_ACT_NONE); otherwise out is 16-bit, rounded to nearest
  * even.  Requirements: K % 16 == 0, N % 16 == 0, all offsets/pitches
- * multiples of 8 elements.
+ * multiples of 8 elements, out (and out2, ws) 16-byte aligned.  The outputs
+ * are written by tensor stores of whole 32-row boxes clipped to M x N:
+ * nothing outside the M x N window of each group is written, but the groups'
+ * windows must not overlap.
  * Split-K: when out_f32 is set with no bias, resid or act, and ws (16-byte
  * aligned device memory of ws_bytes) is given, the library may cut the K
  * loop of each output tile into slices computed by different SMs; each slice
@@ -87,9 +85,6 @@ typedef struct {
   int resid_f32;
   void *ws;
   long long ws_bytes;
-  float ep_scale;
-  const float *row_vec;
-  long long row_vec_gstride;
 } gptl_gemm_desc;
 
 int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream);

@@ -16,7 +16,11 @@
 //     limit the K range to the lower triangle;
 //   * fused epilogues: bias, residual, bias+GeLU (writes Z and GeLU(Z): the
 //     fused_bias_gelu of "Training GPT-2 with Megatron-LM" §6.2), GeLU'
-//     scaling of an input gradient, fp32 weight-gradient store.
+//     scaling of an input gradient, fp32 weight-gradient store;
+//   * outputs leave through shared memory with TMA tensor stores: each
+//     epilogue warp stages 32-row x 64-byte boxes (64B swizzle) and one lane
+//     stores them, so global writes are whole 32-byte sectors and the ragged
+//     M/N edges are clipped by the tensor map.
 //
 // Warp roles (320 threads, one CTA per SM): warp 0 issues TMA loads into a
 // multi-stage mbarrier ring, warp 1 allocates TMEM and one thread issues
@@ -34,7 +38,10 @@ constexpr int kBK = 64;           // tile depth per pipeline stage
 constexpr int kGemmThreads = 320;
 constexpr int kEpiWarps = 8;
 
-enum : int { kActNone = 0, kActGelu = 1, kActDGelu = 2, kActExpLse = 3, kActDSoftmax = 4 };
+enum : int { kActNone = 0, kActGelu = 1, kActDGelu = 2 };
+
+constexpr int kStageBoxBytes = 2048;                 // one 32-row x 64-byte store box
+constexpr int kStagingBytes = 8 * 2 * kStageBoxBytes;  // two boxes per epilogue warp
 enum : int { kCausalNone = 0, kCausalSkipUpper = 1, kCausalKBelow = 2, kCausalKFrom = 3 };
 
 struct OperandRule {
@@ -48,6 +55,8 @@ struct OperandRule {
 struct alignas(64) GemmParams {
   CUtensorMap map_a;
   CUtensorMap map_b;
+  CUtensorMap map_o;           // output, or the split-K partials; box {64 B / elem, 32, 1, 1}
+  CUtensorMap map_o2;          // GeLU(Z) when act == GELU
   OperandRule ra, rb;
   int M, N, K, groups, k_shards, causal;
   int split;                   // K slices per tile (split-K); 1 = none
@@ -58,22 +67,18 @@ struct alignas(64) GemmParams {
   int m_tiles, n_tiles;
   long long total_tiles;
   // epilogue
-  void *out;
-  long long ldo;
-  int o_mod;
-  long long o_str_mod, o_str_div;
+  int o_mod;                   // output group G at map coordinates (G % o_mod, G / o_mod), or
+  int o_flat;                  // (G, 0) when o_flat is set
   int out_f32;
   const void *bias;
   long long bias_g_stride;
   const void *resid;
   long long ld_resid;
   int resid_f32;
-  const void *aux;
-  void *out2;
+  const void *aux;             // GeLU' argument, same layout as the output
+  long long ldo;
+  long long o_str_mod, o_str_div;
   int act;
-  float ep_scale;              // EXP_LSE / DSOFTMAX scale
-  const float *row_vec;        // per-row vector of the group: [G][row_vec_gstride]
-  long long row_vec_gstride;
 };
 
 struct TileInfo {
@@ -140,60 +145,77 @@ __device__ __forceinline__ uint64_t operand_desc(const OperandRule &r, uint32_t 
 // that their latency overlaps the previous chunk's arithmetic.
 struct EpiIn {
   uint4 bias[2];     // 16-bit bias
-  uint4 aux[2];      // 16-bit aux (GeLU' argument or P)
+  uint4 aux[2];      // 16-bit GeLU' argument
   uint4 r16[2];      // 16-bit residual
   float4 r32[4];     // fp32 residual
 };
 
+// Per-thread row pointers of the epilogue inputs for one tile (null when
+// unused or when the row is past M).
+struct EpiRow {
+  const uint8_t *bias;
+  const uint8_t *resid;
+  const uint8_t *aux;
+};
+
 template <typename T>
-__device__ __forceinline__ void epilogue_load(const GemmParams &p, int g, int row, int n, EpiIn &in) {
-  if (p.split > 1 || row >= p.M) return;
-  if (p.bias) {
-    const uint4 *b = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.bias) +
-                                                     (long long)g * p.bias_g_stride + n);
+__device__ __forceinline__ EpiRow epilogue_row(const GemmParams &p, int g, int row) {
+  EpiRow e{nullptr, nullptr, nullptr};
+  if (p.split > 1 || row >= p.M) return e;
+  if (p.bias) e.bias = reinterpret_cast<const uint8_t *>(static_cast<const T *>(p.bias) +
+                                                        (long long)g * p.bias_g_stride);
+  if (p.resid)
+    e.resid = static_cast<const uint8_t *>(p.resid) +
+              (long long)row * p.ld_resid * (p.resid_f32 ? 4 : (int)sizeof(T));
+  if (p.act == kActDGelu)
+    e.aux = reinterpret_cast<const uint8_t *>(
+        static_cast<const T *>(p.aux) + (long long)(g % p.o_mod) * p.o_str_mod +
+        (long long)(g / p.o_mod) * p.o_str_div + (long long)row * p.ldo);
+  return e;
+}
+
+template <typename T>
+__device__ __forceinline__ void epilogue_load(const GemmParams &p, const EpiRow &e, int n, EpiIn &in) {
+  if (e.bias) {
+    const uint4 *b = reinterpret_cast<const uint4 *>(e.bias) + n / 8;
     in.bias[0] = __ldg(b);
     in.bias[1] = __ldg(b + 1);
   }
-  if (p.resid) {
+  if (e.resid) {
     if (p.resid_f32) {
-      const float4 *rr = reinterpret_cast<const float4 *>(static_cast<const float *>(p.resid) +
-                                                          (long long)row * p.ld_resid + n);
+      const float4 *rr = reinterpret_cast<const float4 *>(e.resid) + n / 4;
 #pragma unroll
       for (int q = 0; q < 4; ++q) in.r32[q] = rr[q];
     } else {
-      const uint4 *rr = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.resid) +
-                                                        (long long)row * p.ld_resid + n);
+      const uint4 *rr = reinterpret_cast<const uint4 *>(e.resid) + n / 8;
       in.r16[0] = rr[0];
       in.r16[1] = rr[1];
     }
   }
-  if (p.act == kActDGelu || p.act == kActDSoftmax) {
-    const long long off = (long long)(g % p.o_mod) * p.o_str_mod +
-                          (long long)(g / p.o_mod) * p.o_str_div + (long long)row * p.ldo + n;
-    const uint4 *xp = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.aux) + off);
+  if (e.aux) {
+    const uint4 *xp = reinterpret_cast<const uint4 *>(e.aux) + n / 8;
     in.aux[0] = xp[0];
     in.aux[1] = xp[1];
   }
 }
 
-// rv: the row's entry of row_vec (EXP_LSE / DSOFTMAX), loaded once per tile.
+// Shared address of 16-byte piece j (0..3) of row r in a 32-row x 64-byte
+// staging box laid out with the 64B swizzle of the store's tensor map.
+__device__ __forceinline__ uint32_t box_piece(uint32_t box, int r, int j) {
+  return box + (uint32_t)(r * 64) + (uint32_t)((j ^ ((r >> 1) & 3)) << 4);
+}
+
+// Finish one 16-column chunk (fp32 accumulator values r) and write it into
+// the staging box(es): 16-bit outputs fill half a box (pieces 2*slot,
+// 2*slot+1), fp32 outputs a whole box.
 template <typename T>
-__device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int row, int n,
-                                               int slice, const uint32_t (&r)[16], const EpiIn &in,
-                                               float rv) {
+__device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow &e,
+                                               const uint32_t (&r)[16], const EpiIn &in,
+                                               uint32_t box, uint32_t box2, int lane, int slot) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-  if (p.split > 1) {           // split-K partial: dense fp32, finished by splitk_reduce_kernel
-    float4 *o = reinterpret_cast<float4 *>(p.ws + (long long)slice * p.ws_slice +
-                                           ((long long)g * p.M + row) * p.N + n);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    return;
-  }
-  const long long off = (long long)(g % p.o_mod) * p.o_str_mod +
-                        (long long)(g / p.o_mod) * p.o_str_div + (long long)row * p.ldo + n;
-  if (p.bias) {
+  if (e.bias) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float f[8];
@@ -202,7 +224,7 @@ __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int r
       for (int i = 0; i < 8; ++i) v[8 * h + i] += f[i];
     }
   }
-  if (p.resid) {
+  if (e.resid) {
     if (p.resid_f32) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -219,48 +241,31 @@ __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int r
       }
     }
   }
-  if (p.out_f32) {
-    float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
+  if (p.out_f32 || p.split > 1) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    for (int j = 0; j < 4; ++j)
+      st_shared_v4(box_piece(box, lane, j),
+                   make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                              __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3])));
     return;
   }
-  uint4 *o = reinterpret_cast<uint4 *>(static_cast<T *>(p.out) + off);
   if (p.act == kActGelu) {
-    uint4 *o2 = reinterpret_cast<uint4 *>(static_cast<T *>(p.out2) + off);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float z[8], a[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) z[i] = v[8 * h + i];
-      uint4 zq = pack8<T>(z);
+      const uint4 zq = pack8<T>(z);
       float zr[8];
       unpack8<T>(zq, zr);                 // GeLU of the stored (rounded) Z
 #pragma unroll
       for (int i = 0; i < 8; ++i) a[i] = gelu_f(zr[i]);
-      o[h] = zq;
-      o2[h] = pack8<T>(a);
+      st_shared_v4(box_piece(box, lane, 2 * slot + h), zq);
+      st_shared_v4(box_piece(box2, lane, 2 * slot + h), pack8<T>(a));
     }
     return;
   }
-  if (p.act == kActExpLse || p.act == kActDSoftmax) {
-    // attention probabilities recomputed from the scores and the row's
-    // base-2 log-sum-exp, or the softmax backward; both zero above the
-    // diagonal (column n > row)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float pr[8];
-      if (p.act == kActDSoftmax) unpack8<T>(in.aux[h], pr);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float x = v[8 * h + i];
-        const float val = p.act == kActExpLse ? exp2f(x * p.ep_scale - rv)
-                                              : p.ep_scale * pr[i] * (x - rv);
-        v[8 * h + i] = (n + 8 * h + i > row) ? 0.f : val;
-      }
-    }
-  }
-  if (p.act == kActDGelu) {
+  if (e.aux) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float z[8];
@@ -274,7 +279,7 @@ __device__ __forceinline__ void epilogue_store(const GemmParams &p, int g, int r
     float f[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) f[i] = v[8 * h + i];
-    o[h] = pack8<T>(f);
+    st_shared_v4(box_piece(box, lane, 2 * slot + h), pack8<T>(f));
   }
 }
 
@@ -286,7 +291,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
   const int a_bytes = kBM * kBK * 2;
   const int b_bytes = p.bn * kBK * 2;
   const int stage_bytes = a_bytes + b_bytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.stages * stage_bytes);
+  const uint32_t staging_s = smem_u32(smem + p.stages * stage_bytes);   // 1024-aligned
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.stages * stage_bytes + kStagingBytes);
   // bars: full[0,S) empty[S,2S) tfull[2S,2S+2) tempty[2S+2,2S+4) drain[2S+4]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * p.stages + 5);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -314,6 +320,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&p.map_a);
     prefetch_tensormap(&p.map_b);
+    prefetch_tensormap(&p.map_o);
+    if (p.act == kActGelu) prefetch_tensormap(&p.map_o2);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
@@ -401,6 +409,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     // -------------------------------------------------- epilogue warps
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;        // which half of the tile's columns
+    const bool wide = p.out_f32 || p.split > 1;     // fp32: one chunk per box
+    const bool gelu = !wide && p.act == kActGelu;   // Z and GeLU(Z): both boxes per chunk pair
+    const uint32_t my_boxes = staging_s + (uint32_t)((warp - 2) * 2 * kStageBoxBytes);
+    int box_i = 0;                           // boxes issued by this warp (selects the buffer)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
@@ -408,41 +420,70 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       if (ti.skip) continue;
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) break;
       tc_fence_after();
-      const int row = ti.m0 + q * 32 + lane;
+      const int row0 = ti.m0 + q * 32;
+      const EpiRow er = epilogue_row<T>(p, ti.g, row0 + lane);
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.bn_alloc);
-      // this warp's 16-column chunks: [c0, c1)
+      // output map coordinates of this tile's group
+      int oz, ow;
+      if (p.split > 1) { oz = ti.slice * p.groups + ti.g; ow = 0; }
+      else if (p.o_flat) { oz = ti.g; ow = 0; }
+      else { oz = ti.g % p.o_mod; ow = ti.g / p.o_mod; }
+      // this warp's 16-column chunks [c0, c1); the halves split at an even
+      // chunk so that a 16-bit box (two chunks) never straddles them
       const int nchunk = p.bn / 16;
-      const int c0 = half ? (nchunk + 1) / 2 : 0;
-      int c1 = half ? nchunk : (nchunk + 1) / 2;
+      const int csplit = 2 * ((nchunk + 3) / 4);
+      const int c0 = half ? csplit : 0;
+      int c1 = half ? nchunk : csplit;
       const int valid = (p.N - ti.n0 + 15) / 16;   // chunks inside N
       if (c1 > valid) c1 = valid;
       // software pipeline: the load of chunk c+1 is in flight while chunk c
       // is processed (tcgen05.wait::ld waits for every earlier load)
       uint32_t ra[16], rb[16];
       EpiIn ia, ib;
-      float rv = 0.f;
-      if ((p.act == kActExpLse || p.act == kActDSoftmax) && row < p.M)
-        rv = p.row_vec[(long long)ti.g * p.row_vec_gstride + row];
+      auto process = [&](int c, const uint32_t (&r)[16], const EpiIn &in) {
+        const int slot = wide ? 0 : ((c - c0) & 1);
+        const bool first = slot == 0, last = wide || slot == 1 || c + 1 == c1;
+        const uint32_t buf = my_boxes + (uint32_t)((gelu ? 0 : (box_i & 1)) * kStageBoxBytes);
+        if (first) {                         // the box buffer(s) must be free again
+          if (lane == 0) {
+            if (gelu) bulk_wait_read<0>();
+            else bulk_wait_read<1>();
+          }
+          __syncwarp();
+        }
+        epilogue_chunk<T>(p, er, r, in, buf, my_boxes + kStageBoxBytes, lane, slot);
+        if (last) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int x = ti.n0 + (c - slot) * 16;
+            tma_store_4d(&p.map_o, buf, x, row0, oz, ow);
+            if (gelu) tma_store_4d(&p.map_o2, my_boxes + kStageBoxBytes, x, row0, oz, ow);
+            bulk_commit();
+          }
+          ++box_i;
+        }
+      };
       if (c0 < c1) {
         tmem_ld16(t_row + (uint32_t)(c0 * 16), ra);
-        epilogue_load<T>(p, ti.g, row, ti.n0 + c0 * 16, ia);
+        epilogue_load<T>(p, er, ti.n0 + c0 * 16, ia);
         tmem_wait_ld();
       }
       for (int c = c0; c < c1; c += 2) {
         const bool has_b = c + 1 < c1;
         if (has_b) {
           tmem_ld16(t_row + (uint32_t)((c + 1) * 16), rb);
-          epilogue_load<T>(p, ti.g, row, ti.n0 + (c + 1) * 16, ib);
+          epilogue_load<T>(p, er, ti.n0 + (c + 1) * 16, ib);
         }
-        if (row < p.M) epilogue_store<T>(p, ti.g, row, ti.n0 + c * 16, ti.slice, ra, ia, rv);
+        process(c, ra, ia);
         tmem_wait_ld();
         if (!has_b) break;
         const bool has_a = c + 2 < c1;
         if (has_a) {
           tmem_ld16(t_row + (uint32_t)((c + 2) * 16), ra);
-          epilogue_load<T>(p, ti.g, row, ti.n0 + (c + 2) * 16, ia);
+          epilogue_load<T>(p, er, ti.n0 + (c + 2) * 16, ia);
         }
-        if (row < p.M) epilogue_store<T>(p, ti.g, row, ti.n0 + (c + 1) * 16, ti.slice, rb, ib, rv);
+        process(c + 1, rb, ib);
         tmem_wait_ld();
       }
       tc_fence_before();
@@ -453,6 +494,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         acc_phase ^= 1;
       }
     }
+    // the staged boxes must be read, and the stores done, before the CTA exits
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -173,6 +173,48 @@ int encode_operand(CUtensorMap *map, const gptl_operand &o, gptl_dtype dt, int r
   return r == CUDA_SUCCESS ? GPTL_OK : GPTL_E_CUDA;
 }
 
+// Tensor map of a GEMM output for the epilogue's 32-row x 64-byte store
+// boxes (64B swizzle).  Group G of the output sits at
+// (G % o_mod) * str_mod + (G / o_mod) * str_div elements; flat = 1 maps it as
+// one coordinate z = G (str_div apart), else as (z, w) = (G % o_mod, G / o_mod).
+int encode_output(CUtensorMap *map, void *ptr, int f32, gptl_dtype dt, long long N, long long M,
+                  long long ld, int groups, int o_mod, long long str_mod, long long str_div,
+                  int *flat) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return GPTL_E_CUDA;
+  const long long es = f32 ? 4 : 2;
+  cuuint64_t dims[4], strides[3];
+  dims[0] = (cuuint64_t)N;
+  dims[1] = (cuuint64_t)M;
+  strides[0] = (cuuint64_t)(ld * es);
+  const long long plane = ld * M * es;   // a valid stride for an extent-1 dimension
+  if (o_mod == 1 || groups == 1) {
+    *flat = 1;
+    dims[2] = (cuuint64_t)groups;
+    dims[3] = 1;
+    const long long s2 = (o_mod == 1 ? str_div : str_mod) * es;
+    strides[1] = (cuuint64_t)(groups > 1 ? s2 : plane);
+    strides[2] = (cuuint64_t)(groups > 1 ? s2 * groups : plane);
+  } else {
+    *flat = 0;
+    const long long nd = (groups + o_mod - 1) / o_mod;
+    dims[2] = (cuuint64_t)o_mod;
+    dims[3] = (cuuint64_t)nd;
+    strides[1] = (cuuint64_t)(str_mod * es);
+    strides[2] = (cuuint64_t)(nd > 1 ? str_div * es : str_mod * es * o_mod);
+  }
+  for (int i = 0; i < 3; ++i)
+    if (strides[i] == 0 || strides[i] % 16 || strides[i] >= (1ull << 40)) return GPTL_E_SHAPE;
+  cuuint32_t box[4] = {(cuuint32_t)(64 / es), 32, 1, 1}, ones[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType ty = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                     : (dt == GPTL_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                        : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  const CUresult r = fn(map, ty, 4, ptr, dims, strides, box, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GPTL_OK : GPTL_E_CUDA;
+}
+
 int check_operand(const gptl_operand &o) {
   if (!o.ptr) return GPTL_E_NULL;
   if (!aligned16(o.ptr)) return GPTL_E_ALIGN;
@@ -259,9 +301,7 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   if (d.act == GPTL_ACT_GELU && !d.out2) return GPTL_E_NULL;
   if (d.act == GPTL_ACT_DGELU && !d.aux) return GPTL_E_NULL;
   if ((d.out2 && !aligned16(d.out2)) || (d.aux && !aligned16(d.aux))) return GPTL_E_ALIGN;
-  if (d.act < 0 || d.act > 4 || (d.out_f32 && d.act != GPTL_ACT_NONE)) return GPTL_E_SHAPE;
-  if ((d.act == GPTL_ACT_EXP_LSE || d.act == GPTL_ACT_DSOFTMAX) && !d.row_vec) return GPTL_E_NULL;
-  if (d.act == GPTL_ACT_DSOFTMAX && !d.aux) return GPTL_E_NULL;
+  if (d.act < 0 || d.act > 2 || (d.out_f32 && d.act != GPTL_ACT_NONE)) return GPTL_E_SHAPE;
   GPTL_TRY(check_operand(d.a));
   GPTL_TRY(check_operand(d.b));
 
@@ -297,10 +337,10 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.bn_alloc = bn_alloc;
   p.tmem_cols = 2 * bn_alloc;
   const int stage_bytes = (kBM + bn) * kBK * 2;
-  p.stages = (kSmemLimit - 2048) / stage_bytes;
+  p.stages = (kSmemLimit - 2048 - kStagingBytes) / stage_bytes;
   if (p.stages > 8) p.stages = 8;
   if (p.stages < 2) return GPTL_E_SHAPE;
-  const int smem = 1024 + p.stages * stage_bytes + 256;
+  const int smem = 1024 + p.stages * stage_bytes + kStagingBytes + 256;
   const uint32_t fmt = dt == GPTL_BF16 ? 1u : 0u;
   p.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)d.a.mn_major << 15) |
             ((uint32_t)d.b.mn_major << 16) | ((uint32_t)(bn >> 3) << 17) |
@@ -316,7 +356,20 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.ws = static_cast<float *>(d.ws);
   p.ws_slice = (long long)d.groups * d.M * d.N;
   p.total_tiles = tiles * p.split;
-  p.out = d.out;
+  if (p.split > 1) {            // partials [split * groups][M][N], dense fp32
+    int flat = 1;
+    GPTL_TRY(encode_output(&p.map_o, d.ws, 1, dt, d.N, d.M, d.N, p.split * d.groups, 1, 0,
+                           (long long)d.M * d.N, &flat));
+    p.o_flat = 1;
+  } else {
+    GPTL_TRY(encode_output(&p.map_o, d.out, d.out_f32, dt, d.N, d.M, d.ldo, d.groups, d.o_mod,
+                           d.o_str_mod, d.o_str_div, &p.o_flat));
+    if (d.act == GPTL_ACT_GELU) {
+      int flat2 = 0;
+      GPTL_TRY(encode_output(&p.map_o2, d.out2, 0, dt, d.N, d.M, d.ldo, d.groups, d.o_mod,
+                             d.o_str_mod, d.o_str_div, &flat2));
+    }
+  }
   p.ldo = d.ldo;
   p.o_mod = d.o_mod;
   p.o_str_mod = d.o_str_mod;
@@ -328,11 +381,7 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.resid_f32 = d.resid_f32 ? 1 : 0;
   p.ld_resid = d.ld_resid;
   p.aux = d.aux;
-  p.out2 = d.out2;
   p.act = d.act;
-  p.ep_scale = d.ep_scale;
-  p.row_vec = d.row_vec;
-  p.row_vec_gstride = d.row_vec_gstride;
   const int grid = (int)(p.total_tiles < sms ? p.total_tiles : sms);
   if (dt == GPTL_FP16) GPTL_TRY(launch_gemm_t<__half>(p, grid, smem, stream));
   else GPTL_TRY(launch_gemm_t<__nv_bfloat16>(p, grid, smem, stream));

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG, "libgptlayer.so")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 
 FP16, BF16 = 0, 1
-ACT_NONE, ACT_GELU, ACT_DGELU, ACT_EXP_LSE, ACT_DSOFTMAX = 0, 1, 2, 3, 4
+ACT_NONE, ACT_GELU, ACT_DGELU = 0, 1, 2
 CAUSAL_NONE, CAUSAL_SKIP_UPPER, CAUSAL_K_BELOW, CAUSAL_K_FROM = 0, 1, 2, 3
 E_NULL, E_SHAPE, E_ALIGN, E_DTYPE, E_ARCH, E_CUDA, E_DEVICE, E_ARG = -1, -2, -3, -4, -5, -6, -7, -8
 E_TOO_LARGE = -9
@@ -66,8 +66,7 @@ class GemmDesc(C.Structure):
                 ("bias", C.c_void_p), ("bias_g_stride", C.c_longlong), ("resid", C.c_void_p),
                 ("ld_resid", C.c_longlong), ("aux", C.c_void_p), ("out2", C.c_void_p),
                 ("act", C.c_int), ("resid_f32", C.c_int), ("ws", C.c_void_p),
-                ("ws_bytes", C.c_longlong), ("ep_scale", C.c_float), ("row_vec", C.c_void_p),
-                ("row_vec_gstride", C.c_longlong)]
+                ("ws_bytes", C.c_longlong)]
 
 
 class LaunchRecord(C.Structure):
