@@ -284,3 +284,36 @@ def test_fp32_out_with_bias_and_fp32_residual(dtype):
     _close(got, exp, 1e-5)
     exp, got, _ = _run(dtype, bias=True, resid=True, resid_f32=True, **kw)
     _close(got, exp, 1e-2)
+
+
+@pytest.mark.parametrize("dtype,out_f32", [("bf16", False), ("fp16", True)])
+def test_interleaved_group_output_and_padding(dtype, out_f32):
+    """Groups written side by side into a padded buffer (o_mod = 2):
+    out + (G % 2) * N + (G / 2) * M * ldo + m * ldo + n, ldo = 2N + 16.  The
+    tensor stores are clipped to each group's M x N window, so the 16 padding
+    columns of every row keep their sentinel."""
+    need_gpu()
+    M, N, K, groups = 200, 96, 64, 4
+    ldo = 2 * N + 16
+    rng = np.random.default_rng(11)
+    abuf = rounded(rng.standard_normal((1, M, K)), dtype)
+    bbuf = rounded(rng.standard_normal((groups, N, K)) * 0.1, dtype)
+    at, bt = dev_tensor(abuf, dtype), dev_tensor(bbuf, dtype)
+    _, ac = _op(at, K, M, 1, K, M * K, 0)
+    _, bc = _op(bt, K, N, groups, K, N * K, 0)
+    tdt = torch.float32 if out_f32 else (torch.float16 if dtype == "fp16" else torch.bfloat16)
+    out = torch.full((groups // 2, M, ldo), float("nan"), dtype=tdt, device="cuda")
+    d = G.GemmDesc()
+    d.M, d.N, d.K, d.groups, d.k_shards, d.causal = M, N, K, groups, 1, 0
+    d.a, d.b = ac, bc
+    d.out, d.out_f32, d.ldo = out.data_ptr(), int(out_f32), ldo
+    d.o_mod, d.o_str_mod, d.o_str_div = 2, N, M * ldo
+    G.gemm(d, dtype, stream())
+    check_device_error()
+    got = out.float().cpu().numpy()
+    for g in range(groups):
+        exp = abuf[0] @ bbuf[g].T
+        part = got[g // 2, :, (g % 2) * N:(g % 2 + 1) * N]
+        tol = 1e-5 if out_f32 else 8e-3
+        assert float(np.abs(part - exp).max()) <= tol * float(np.abs(exp).max())
+    assert np.isnan(got[:, :, 2 * N:]).all()

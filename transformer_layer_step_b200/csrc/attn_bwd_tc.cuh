@@ -27,6 +27,8 @@
 // MMA (one thread), warps 2-9 elementwise work: thread = (row, half of the
 // 128 columns); warp w reads TMEM lane quarter w % 4.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace gptl {
@@ -71,10 +73,6 @@ __device__ __forceinline__ uint32_t abwd_a_addr(uint32_t base, int row, int c16)
          (uint32_t)(((c16 & 7) ^ (row & 7)) * 16);
 }
 
-template <typename T>
-__device__ __forceinline__ float round16(float x) {
-  return Cvt<T>::to_f(Cvt<T>::from_f(x));
-}
 
 // ============================================================ dQ kernel
 template <typename T>
@@ -233,48 +231,64 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
       const int n = qb + 1;
       const int qrow = qb * 128 + row;
       const bool valid_row = qrow < p.s;
-      const float lse2 = valid_row ? p.lse[(long long)g * p.s + qrow] : 0.f;
-      const float dv = valid_row ? p.dvec[(long long)g * p.s + qrow] : 0.f;
+      // P = exp2(S log2(e)/sqrt(d) - lse); dS = P16 (dP - D) / sqrt(d) as
+      // P16 * (dP / sqrt(d) - D / sqrt(d))
+      const float nl = valid_row ? -p.lse[(long long)g * p.s + qrow] : 0.f;
+      const float nsdv = valid_row ? -p.scale * p.dvec[(long long)g * p.s + qrow] : 0.f;
       bool ok = true;
       for (int j = 0; j < n; ++j) {
         if (!mbar_wait(sd_full, sd_it & 1u, abort_flag)) { ok = false; break; }
         ++sd_it;
         tc_fence_after();
-        uint32_t rs[4][16], rd[4][16];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld16(t_s + lane_off + col0 + (uint32_t)(c * 16), rs[c]);
-          tmem_ld16(t_dp + lane_off + col0 + (uint32_t)(c * 16), rd[c]);
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sd_empty);
         const int key0 = j * 128 + (int)col0;
-        const bool diag = (j == qb);
-        uint32_t pk[32];                     // dS, packed pairs of 16-bit values
+        // masking only where a key can be past the row or past the sequence
+        const bool edge = (j == qb) || (j * 128 + 128 > p.s);
+        // two passes over 32 of this thread's 64 columns each (bounded registers)
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t rs[2][16], rd[2][16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float out2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int key = key0 + c * 16 + e + u;
-              const bool live = !diag || (key <= qrow && key < p.s);
-              const float pv = live ? round16<T>(exp2f(__uint_as_float(rs[c][e + u]) * p.scale_log2 - lse2)) : 0.f;
-              out2[u] = p.scale * pv * (__uint_as_float(rd[c][e + u]) - dv);
-            }
-            pk[c * 8 + e / 2] = Cvt<T>::pack2(out2[0], out2[1]);
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld16(t_s + lane_off + col0 + (uint32_t)((2 * hh + c) * 16), rs[c]);
+            tmem_ld16(t_dp + lane_off + col0 + (uint32_t)((2 * hh + c) * 16), rd[c]);
           }
-        if (j >= 1) {   // dQ += dS_{j-1} K_{j-1} done: the dS buffer is free
-          if (!mbar_wait(dq_done, dq_it & 1u, abort_flag)) { ok = false; break; }
-          ++dq_it;
-        }
+          tmem_wait_ld();
+          if (hh == 1) {               // S / dP fully read: the MMAs may overwrite them
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sd_empty);
+          }
+          uint32_t pk[16];                     // dS, packed pairs of 16-bit values
+          auto block = [&](auto masked) {
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16)
-          st_shared_v4(abwd_a_addr(ds_s, row, half * 8 + c16),
-                       make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]));
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+              for (int e = 0; e < 16; e += 2) {
+                float t0 = fmaf(__uint_as_float(rs[c][e]), p.scale_log2, nl);
+                float t1 = fmaf(__uint_as_float(rs[c][e + 1]), p.scale_log2, nl);
+                if (masked) {
+                  const int key = key0 + (2 * hh + c) * 16 + e;
+                  if (key > qrow || key >= p.s) t0 = -INFINITY;
+                  if (key + 1 > qrow || key + 1 >= p.s) t1 = -INFINITY;
+                }
+                // P16: P rounded to the 16-bit operand type (exp2(-inf) = 0)
+                const float2 pr = Cvt<T>::unpack2(Cvt<T>::pack2(ex2_approx(t0), ex2_approx(t1)));
+                const float ds0 = pr.x * fmaf(__uint_as_float(rd[c][e]), p.scale, nsdv);
+                const float ds1 = pr.y * fmaf(__uint_as_float(rd[c][e + 1]), p.scale, nsdv);
+                pk[c * 8 + e / 2] = Cvt<T>::pack2(ds0, ds1);
+              }
+          };
+          if (edge) block(std::true_type{});
+          else block(std::false_type{});
+          if (hh == 0 && j >= 1) {   // dQ += dS_{j-1} K_{j-1} done: the dS buffer is free
+            if (!mbar_wait(dq_done, dq_it & 1u, abort_flag)) { ok = false; break; }
+            ++dq_it;
+          }
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16)
+            st_shared_v4(abwd_a_addr(ds_s, row, half * 8 + hh * 4 + c16),
+                         make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]));
+        }
+        if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
@@ -494,56 +508,82 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
         // used two blocks ago: a thread passes block blk+1's barrier only
         // after all threads have finished block blk.
         float *vb = vecs + (blk & 1u) * 256u;
-        if (tid < 128) {
+        if (tid < 128) {   // -lse and -D/sqrt(d) of the block's queries
           const int q = j * 128 + tid;
-          vb[tid] = q < p.s ? p.lse[(long long)g * p.s + q] : 0.f;
-          vb[128 + tid] = q < p.s ? p.dvec[(long long)g * p.s + q] : 0.f;
+          vb[tid] = q < p.s ? -p.lse[(long long)g * p.s + q] : 0.f;
+          vb[128 + tid] = q < p.s ? -p.scale * p.dvec[(long long)g * p.s + q] : 0.f;
         }
         mbar_arrive(vec_bar((int)(blk & 1u)));
         if (!mbar_wait(vec_bar((int)(blk & 1u)), (blk >> 1) & 1u, abort_flag)) { ok = false; break; }
         if (!mbar_wait(sd_full, sd_it & 1u, abort_flag)) { ok = false; break; }
         ++sd_it;
         tc_fence_after();
-        uint32_t rs[4][16], rd[4][16];
+        // masking only where a query can be before the key or past the sequence
+        const bool edge = (j == kb) || (j * 128 + 128 > p.s);
+        const float4 *vb4 = reinterpret_cast<const float4 *>(vb);
+        // two passes over 32 of this thread's 64 columns each, to bound the
+        // registers held: load S^T and dP^T, form P16 and dS, store both
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t rs[2][16], rd[2][16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld16(t_s + lane_off + col0 + (uint32_t)(c * 16), rs[c]);
-          tmem_ld16(t_dp + lane_off + col0 + (uint32_t)(c * 16), rd[c]);
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sd_empty);
-        const bool diag = (j == kb);
-        uint32_t pp[32], pd[32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float pv2[2], ds2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int ql = (int)col0 + c * 16 + e + u;      // query within the block
-              const int q = j * 128 + ql;
-              const bool live = q < p.s && (!diag || q >= key);
-              const float pv = live ? round16<T>(exp2f(__uint_as_float(rs[c][e + u]) * p.scale_log2 - vb[ql])) : 0.f;
-              pv2[u] = pv;
-              ds2[u] = p.scale * pv * (__uint_as_float(rd[c][e + u]) - vb[128 + ql]);
-            }
-            pp[c * 8 + e / 2] = Cvt<T>::pack2(pv2[0], pv2[1]);
-            pd[c * 8 + e / 2] = Cvt<T>::pack2(ds2[0], ds2[1]);
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld16(t_s + lane_off + col0 + (uint32_t)((2 * hh + c) * 16), rs[c]);
+            tmem_ld16(t_dp + lane_off + col0 + (uint32_t)((2 * hh + c) * 16), rd[c]);
           }
-        if (jj >= 1) {   // dV, dK of the previous block done: P^T and dS^T tiles free
-          if (!mbar_wait(pds_free, pds_it & 1u, abort_flag)) { ok = false; break; }
-          ++pds_it;
-        }
+          tmem_wait_ld();
+          if (hh == 1) {               // S^T / dP^T fully read: the MMAs may overwrite them
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sd_empty);
+          }
+          uint32_t pp[16], pd[16];
+          auto block = [&](auto masked) {
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          st_shared_v4(abwd_a_addr(pt_s, row, half * 8 + c16),
-                       make_uint4(pp[4 * c16], pp[4 * c16 + 1], pp[4 * c16 + 2], pp[4 * c16 + 3]));
-          st_shared_v4(abwd_a_addr(dst_s, row, half * 8 + c16),
-                       make_uint4(pd[4 * c16], pd[4 * c16 + 1], pd[4 * c16 + 2], pd[4 * c16 + 3]));
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+              for (int e = 0; e < 16; e += 4) {
+                const int ql = (int)col0 + (2 * hh + c) * 16 + e;   // query within the block
+                const float4 nl = vb4[ql / 4], nsdv = vb4[32 + ql / 4];
+                float t[4] = {fmaf(__uint_as_float(rs[c][e]), p.scale_log2, nl.x),
+                              fmaf(__uint_as_float(rs[c][e + 1]), p.scale_log2, nl.y),
+                              fmaf(__uint_as_float(rs[c][e + 2]), p.scale_log2, nl.z),
+                              fmaf(__uint_as_float(rs[c][e + 3]), p.scale_log2, nl.w)};
+                if (masked) {
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    const int q = j * 128 + ql + u;
+                    if (q >= p.s || q < key) t[u] = -INFINITY;
+                  }
+                }
+                // P16: P rounded to the 16-bit operand type (exp2(-inf) = 0)
+                const uint32_t p01 = Cvt<T>::pack2(ex2_approx(t[0]), ex2_approx(t[1]));
+                const uint32_t p23 = Cvt<T>::pack2(ex2_approx(t[2]), ex2_approx(t[3]));
+                const float2 a = Cvt<T>::unpack2(p01), b = Cvt<T>::unpack2(p23);
+                pp[c * 8 + e / 2] = p01;
+                pp[c * 8 + e / 2 + 1] = p23;
+                pd[c * 8 + e / 2] = Cvt<T>::pack2(a.x * fmaf(__uint_as_float(rd[c][e]), p.scale, nsdv.x),
+                                                  a.y * fmaf(__uint_as_float(rd[c][e + 1]), p.scale, nsdv.y));
+                pd[c * 8 + e / 2 + 1] =
+                    Cvt<T>::pack2(b.x * fmaf(__uint_as_float(rd[c][e + 2]), p.scale, nsdv.z),
+                                  b.y * fmaf(__uint_as_float(rd[c][e + 3]), p.scale, nsdv.w));
+              }
+          };
+          if (edge) block(std::true_type{});
+          else block(std::false_type{});
+          if (hh == 0 && jj >= 1) {   // dV, dK of the previous block done: P^T and dS^T tiles free
+            if (!mbar_wait(pds_free, pds_it & 1u, abort_flag)) { ok = false; break; }
+            ++pds_it;
+          }
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            const int col16 = half * 8 + hh * 4 + c16;
+            st_shared_v4(abwd_a_addr(pt_s, row, col16),
+                         make_uint4(pp[4 * c16], pp[4 * c16 + 1], pp[4 * c16 + 2], pp[4 * c16 + 3]));
+            st_shared_v4(abwd_a_addr(dst_s, row, col16),
+                         make_uint4(pd[4 * c16], pd[4 * c16 + 1], pd[4 * c16 + 2], pd[4 * c16 + 3]));
+          }
         }
+        if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();

@@ -232,47 +232,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         __syncwarp();
         if (lane == 0) mbar_arrive(s_empty(sb));
         ++s_it;
-        // scale, mask (only the diagonal block and keys past the sequence), max
-        const bool diag = (j == qt);
+        // mask (only where a key can be past the row or past the sequence),
+        // then the row max of the raw scores (the scale is positive)
         const int key0 = j * kAttnTile;
-        float mx = -INFINITY;
+        if (j == qt || key0 + kAttnTile > p.s) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int key = key0 + c * 16 + e;
+              if (key > qrow || key >= p.s) r[c][e] = __float_as_uint(-INFINITY);
+            }
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int key = key0 + c * 16 + e;
-            float x = __uint_as_float(r[c][e]) * p.scale_log2;
-            if (diag && (key > qrow || key >= p.s)) x = -INFINITY;
-            r[c][e] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
+          for (int e = 0; e < 16; e += 2) {
+            mx0 = fmaxf(mx0, __uint_as_float(r[c][e]));
+            mx1 = fmaxf(mx1, __uint_as_float(r[c][e + 1]));
           }
-        const float m_new = fmaxf(m, mx);
-        const float alpha = exp2f(m - m_new);
-        float sum = 0.f;
+        // Running max m in log2 units of the scaled scores.  It is raised
+        // only when a score exceeds it by more than 2^8, so that O and l are
+        // rescaled rarely; meanwhile P <= 2^8, exact in fp32 and in the
+        // 16-bit operand (whose rounding is relative).  O / l is unchanged.
+        const float mx = fmaxf(mx0, mx1) * p.scale_log2;
+        const float m_new = (mx > m + 8.0f) ? mx : m;
+        const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);   // 0 when m = -inf
+        const float nm = -m_new;
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float pv = exp2f(__uint_as_float(r[c][e]) - m_new);
-            r[c][e] = __float_as_uint(pv);
-            sum += pv;
+          for (int e = 0; e < 16; e += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][e]), p.scale_log2, nm));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][e + 1]), p.scale_log2, nm));
+            r[c][e] = __float_as_uint(p0);
+            r[c][e + 1] = __float_as_uint(p1);
+            s0 += p0;
+            s1 += p1;
           }
-        l = l * alpha + sum;
+        l = l * alpha + (s0 + s1);
         m = m_new;
         if (j >= 1) {
           // P_{j-1} V_{j-1} done: O is complete and the P buffer is free
           if (!mbar_wait(o_done, o_it & 1u, abort_flag)) { ok = false; break; }
           ++o_it;
           tc_fence_after();
-          for (int c = 0; c < d / 16; ++c) {
-            uint32_t o[16];
-            tmem_ld16(tmem_o + lane_off + (uint32_t)(c * 16), o);
-            tmem_wait_ld();
+          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+            for (int c = 0; c < d / 16; ++c) {
+              uint32_t o[16];
+              tmem_ld16(tmem_o + lane_off + (uint32_t)(c * 16), o);
+              tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st16(tmem_o + lane_off + (uint32_t)(c * 16), o);
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st16(tmem_o + lane_off + (uint32_t)(c * 16), o);
+            }
+            tmem_wait_st();
           }
-          tmem_wait_st();
         }
         // P (16-bit) into the 128B-swizzled K-major A tile: row `row`,
         // 16-byte chunk c16 of the row goes to atom c16/8, slot (c16%8)^(row%8)
