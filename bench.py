@@ -229,6 +229,26 @@ def oracle_sample(cfg, n_seq: int, seq_prefix: int | None = None, repeats: int =
             "value": sub.tokens * len(times) / sum(times)}
 
 
+# ------------------------------------------------------- replica bookkeeping
+def reduce_max_over_ranks(v: float, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes its own device-timed
+    value and all ranks get the maximum (the job ends when the last replica
+    does).  One collective, taken by every rank in the same order."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, tokens_per_replica_step: int, ms_per_step: float) -> float:
+    """Weak scaling: every replica processes its own batch each step, so the
+    job's throughput is all replicas' tokens over the slowest rank's step time."""
+    return world * tokens_per_replica_step / (ms_per_step * 1e-3)
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_ours(args, cfg, rank, world, local_rank):
     import torch
@@ -251,11 +271,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max_over_ranks(v, world, dev)
 
     def timed_steps(n, body):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -448,7 +464,7 @@ def main():
     achieved_tf = flops["causal"] / (gemm_ms * 1e-3) / 1e12 if gemm_ms else None
     traffic = recorded_traffic(cfg.name)
     ms = res["ms_per_step"]
-    value = world * cfg.tokens / (ms * 1e-3)
+    value = whole_job_tokens_per_s(world, cfg.tokens, ms)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),

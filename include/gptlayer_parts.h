@@ -55,9 +55,10 @@ enum {
  * act: GELU writes the value to out and GeLU(value) to out2; DGELU multiplies
  * by GeLU'(aux at the output's index).  out_f32 = 1 stores the fp32 value
  * (act must be GPTL_ACT_NONE); otherwise out is 16-bit, rounded to nearest
- * even.  Requirements: K % 16 == 0, N % 16 == 0, all offsets/pitches
- * multiples of 8 elements, out (and out2, ws) 16-byte aligned.  The outputs
- * are written by tensor stores of whole 32-row boxes clipped to M x N:
+ * even.  resid and DGELU do not combine.  Requirements: K % 16 == 0,
+ * N % 16 == 0, all offsets/pitches multiples of 8 elements, out (and out2,
+ * ws) 16-byte aligned.  The outputs are written by tensor stores of whole
+ * 32-row boxes clipped to M x N:
  * nothing outside the M x N window of each group is written, but the groups'
  * windows must not overlap.
  * Split-K: when out_f32 is set with no bias, resid or act, and ws (16-byte

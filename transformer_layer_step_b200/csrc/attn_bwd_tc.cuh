@@ -23,9 +23,11 @@
 // K-major operand (reduction over head_dim) and, described differently, as
 // an MN-major operand (reduction over the 128 rows).
 //
-// Warp roles (320 threads, one CTA per SM, persistent): warp 0 TMA, warp 1
-// MMA (one thread), warps 2-9 elementwise work: thread = (row, half of the
-// 128 columns); warp w reads TMEM lane quarter w % 4.
+// Warp roles (352 threads, one CTA per SM, persistent): warp 0 TMA; warp 1
+// issues the S / dP MMAs and warp 10 the accumulating MMAs (dQ, or dV and
+// dK), one thread each, so the two MMA streams run concurrently; warps 2-9
+// elementwise work: thread = (row, half of the 128 columns); warp w reads
+// TMEM lane quarter w % 4.
 #pragma once
 #include <type_traits>
 
@@ -33,7 +35,7 @@
 
 namespace gptl {
 
-constexpr int kAttnBwdThreads = 320;
+constexpr int kAttnBwdThreads = 352;   // 11 warps
 
 struct AttnBwdParams {
   CUtensorMap map_c;     // C as [t*b][s][3h/t]; box {16, 128, 1}, 32B swizzle
@@ -49,7 +51,8 @@ struct AttnBwdParams {
   void *dc;              // [t*b*s][3h/t]: dQ, dK, dV written into their columns
   long long items;       // groups * tiles
   int q_off, k_off, v_off;
-  int qdo_stages;        // dK/dV kernel: Q/dO ring depth (1 or 2)
+  int qdo_stages;        // dK/dV kernel: Q/dO ring depth (1..4)
+  int kv_stages;         // dQ kernel: K/V ring depth (2..4)
 };
 
 // A-operand tile [128 rows][128 cols] (16-bit), K-major, 128B swizzle: two
@@ -86,22 +89,23 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
   const uint32_t tb = (uint32_t)(d / 16) * chunk;             // one [128][d] tile
   const uint32_t ds_s = smem_u32(smem);                       // dS [128 q][128 keys]
   const uint32_t q_s = ds_s + 32768u, do_s = q_s + tb;
-  const uint32_t kv_s = do_s + tb;                            // 2 stages of K, V
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 32768u + 2u * tb + 4u * tb);
+  const uint32_t kv_s = do_s + tb;                            // ring of K, V stages
+  const uint32_t nkv = (uint32_t)p.kv_stages;                // K / V ring depth
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 32768u + 2u * tb + nkv * 2u * tb);
   const uint32_t qdo_full = smem_u32(&bars[0]), qdo_empty = smem_u32(&bars[1]);
   auto kv_full = [&](int i) { return smem_u32(&bars[2 + i]); };
-  auto kv_empty = [&](int i) { return smem_u32(&bars[4 + i]); };
-  const uint32_t sd_full = smem_u32(&bars[6]), sd_empty = smem_u32(&bars[7]);
-  const uint32_t ds_full = smem_u32(&bars[8]), dq_done = smem_u32(&bars[9]);
-  const uint32_t drain_bar = smem_u32(&bars[10]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
+  auto kv_empty = [&](int i) { return smem_u32(&bars[6 + i]); };
+  const uint32_t sd_full = smem_u32(&bars[10]), sd_empty = smem_u32(&bars[11]);
+  const uint32_t ds_full = smem_u32(&bars[12]), dq_done = smem_u32(&bars[13]);
+  const uint32_t drain_bar = smem_u32(&bars[14]), drain_dq = smem_u32(&bars[15]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
     mbar_init(qdo_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(kv_full(i), 1);
       mbar_init(kv_empty(i), 1);
     }
@@ -110,6 +114,7 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
     mbar_init(ds_full, 8);
     mbar_init(dq_done, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(drain_dq, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -149,8 +154,8 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
           tma_load_3d(do_s + (uint32_t)c * chunk, &p.map_do, head * d + c * 16, qb * 128, zb, qdo_full);
         }
         for (int j = 0; j <= qb; ++j, ++kv_it) {
-          const int st = (int)(kv_it & 1u);
-          const uint32_t ph = (kv_it >> 1) & 1u;
+          const int st = (int)(kv_it % nkv);
+          const uint32_t ph = (kv_it / nkv) & 1u;
           if (!mbar_wait(kv_empty(st), ph ^ 1u, abort_flag)) goto tma_abort;
           mbar_arrive_expect_tx(kv_full(st), 2u * tb);
           const uint32_t k_s = kv_s + (uint32_t)st * 2u * tb, v_s = k_s + tb;
@@ -164,28 +169,28 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
       }
       goto tma_done;
     tma_abort:
-      for (int s2 = 0; s2 < 2; ++s2)
+      for (int s2 = 0; s2 < (int)nkv; ++s2)
         if (issued & (1u << s2)) mbar_wait_drain(kv_full(s2), (parity_bits >> s2) & 1u);
       if (q_parity >= 0) mbar_wait_drain(qdo_full, (uint32_t)q_parity);
     tma_done:;
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      uint32_t kv_it = 0, sd_it = 0, ds_it = 0, item_n = 0;
+      // ------------------------------------ MMA: S_j = Q K_j^T, dP_j = dO V_j^T
+      uint32_t kv_it = 0, sd_it = 0, item_n = 0;
       for (long long item = blockIdx.x; item < p.items; item += gridDim.x, ++item_n) {
         int g, qb;
         decode(item, g, qb);
         const int n = qb + 1;
         if (!mbar_wait(qdo_full, item_n & 1u, abort_flag)) goto mma_abort;
         tc_fence_after();
-        // S_j = Q K_j^T and dP_j = dO V_j^T into the single S / dP buffers
-        auto issue_sdp = [&](int j) -> bool {
+        for (int j = 0; j < n; ++j) {
           const uint32_t kj = kv_it + (uint32_t)j;
-          if (!mbar_wait(kv_full(kj & 1u), (kj >> 1) & 1u, abort_flag)) return false;
-          if (!mbar_wait(sd_empty, (sd_it & 1u) ^ 1u, abort_flag)) return false;
+          if (!mbar_wait(kv_full((int)(kj % nkv)), (kj / nkv) & 1u, abort_flag)) goto mma_abort;
+          if (!mbar_wait(sd_empty, (sd_it & 1u) ^ 1u, abort_flag)) goto mma_abort;
           ++sd_it;
           tc_fence_after();
-          const uint32_t k_s = kv_s + (kj & 1u) * 2u * tb, v_s = k_s + tb;
+          const uint32_t k_s = kv_s + (kj % nkv) * 2u * tb, v_s = k_s + tb;
           for (int c = 0; c < d / 16; ++c)
             tc_mma_f16(t_s, abwd_desc_k16(q_s + (uint32_t)c * chunk), abwd_desc_k16(k_s + (uint32_t)c * chunk),
                        p.idesc_s, c > 0 ? 1u : 0u);
@@ -193,23 +198,8 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
             tc_mma_f16(t_dp, abwd_desc_k16(do_s + (uint32_t)c * chunk), abwd_desc_k16(v_s + (uint32_t)c * chunk),
                        p.idesc_s, c > 0 ? 1u : 0u);
           tc_commit(sd_full);
-          return true;
-        };
-        if (!issue_sdp(0)) goto mma_abort;
-        for (int j = 0; j < n; ++j) {
-          if (j + 1 < n && !issue_sdp(j + 1)) goto mma_abort;
-          if (!mbar_wait(ds_full, ds_it & 1u, abort_flag)) goto mma_abort;
-          ++ds_it;
-          tc_fence_after();
-          const uint32_t kj = kv_it + (uint32_t)j;
-          const uint32_t k_s = kv_s + (kj & 1u) * 2u * tb;
-          for (int st = 0; st < 8; ++st)   // dQ += dS K over the 128 keys
-            tc_mma_f16(t_dq, abwd_desc_a(ds_s, st), abwd_desc_mn(k_s, st), p.idesc_acc,
-                       (j > 0 || st > 0) ? 1u : 0u);
-          tc_commit(dq_done);
-          tc_commit(kv_empty(kj & 1u));
         }
-        tc_commit(qdo_empty);
+        tc_commit(qdo_empty);                // Q and dO are read by these MMAs only
         kv_it += (uint32_t)n;
       }
       goto mma_done;
@@ -217,6 +207,37 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
       tc_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0);
     mma_done:;
+    }
+  } else if (warp == 10) {
+    if (lane == 0) {
+      // ---------------------------------------------- MMA: dQ += dS_j K_j
+      // A second issuing thread, alongside the S / dP MMAs.  dS_j exists only
+      // after S_j and dP_j were read, so the K / V stage is free once this
+      // block's dQ MMAs complete.
+      uint32_t kv_it = 0, ds_it = 0;
+      for (long long item = blockIdx.x; item < p.items; item += gridDim.x) {
+        int g, qb;
+        decode(item, g, qb);
+        const int n = qb + 1;
+        for (int j = 0; j < n; ++j) {
+          if (!mbar_wait(ds_full, ds_it & 1u, abort_flag)) goto dq_abort;
+          ++ds_it;
+          tc_fence_after();
+          const uint32_t kj = kv_it + (uint32_t)j;
+          const uint32_t k_s = kv_s + (kj % nkv) * 2u * tb;
+          for (int st = 0; st < 8; ++st)   // dQ += dS K over the 128 keys
+            tc_mma_f16(t_dq, abwd_desc_a(ds_s, st), abwd_desc_mn(k_s, st), p.idesc_acc,
+                       (j > 0 || st > 0) ? 1u : 0u);
+          tc_commit(dq_done);
+          tc_commit(kv_empty((int)(kj % nkv)));
+        }
+        kv_it += (uint32_t)n;
+      }
+      goto dq_mma_done;
+    dq_abort:
+      tc_commit(drain_dq);
+      mbar_wait_drain(drain_dq, 0);
+    dq_mma_done:;
     }
   } else {
     // ------------------------------------------- elementwise: one (row, half)
@@ -348,12 +369,12 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(vecs + 512);
   const uint32_t kv_full = smem_u32(&bars[0]), kv_empty = smem_u32(&bars[1]);
   auto qdo_full = [&](int i) { return smem_u32(&bars[2 + i]); };
-  auto qdo_empty = [&](int i) { return smem_u32(&bars[4 + i]); };
-  const uint32_t sd_full = smem_u32(&bars[6]), sd_empty = smem_u32(&bars[7]);
-  const uint32_t pds_full = smem_u32(&bars[8]), pds_free = smem_u32(&bars[9]);
-  const uint32_t drain_bar = smem_u32(&bars[10]);
-  auto vec_bar = [&](int i) { return smem_u32(&bars[11 + i]); };   // lse/D staged (256 arrivals)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+  auto qdo_empty = [&](int i) { return smem_u32(&bars[6 + i]); };
+  const uint32_t sd_full = smem_u32(&bars[10]), sd_empty = smem_u32(&bars[11]);
+  const uint32_t pds_full = smem_u32(&bars[12]), pds_free = smem_u32(&bars[13]);
+  const uint32_t drain_bar = smem_u32(&bars[14]), drain_acc = smem_u32(&bars[17]);
+  auto vec_bar = [&](int i) { return smem_u32(&bars[15 + i]); };   // lse/D staged (256 arrivals)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -362,7 +383,7 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
     mbar_init(vec_bar(1), 256);
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(qdo_full(i), 1);
       mbar_init(qdo_empty(i), 1);
     }
@@ -371,6 +392,7 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
     mbar_init(pds_full, 8);
     mbar_init(pds_free, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(drain_acc, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -433,18 +455,19 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      uint32_t q_it = 0, sd_it = 0, pds_it = 0, item_n = 0;
+      // ------------------------------- MMA: S^T = K Q_j^T, dP^T = V dO_j^T
+      uint32_t q_it = 0, sd_it = 0, item_n = 0;
       for (long long item = blockIdx.x; item < p.items; item += gridDim.x, ++item_n) {
         int g, kb;
         decode(item, g, kb);
         const int n = p.tiles - kb;
         if (!mbar_wait(kv_full, item_n & 1u, abort_flag)) goto mma_abort;
         tc_fence_after();
-        auto issue_sdp = [&](int jj) -> bool {
+        for (int jj = 0; jj < n; ++jj) {
           const uint32_t qj = q_it + (uint32_t)jj;
           const int st = (int)(qj % (uint32_t)nst);
-          if (!mbar_wait(qdo_full(st), (qj / (uint32_t)nst) & 1u, abort_flag)) return false;
-          if (!mbar_wait(sd_empty, (sd_it & 1u) ^ 1u, abort_flag)) return false;
+          if (!mbar_wait(qdo_full(st), (qj / (uint32_t)nst) & 1u, abort_flag)) goto mma_abort;
+          if (!mbar_wait(sd_empty, (sd_it & 1u) ^ 1u, abort_flag)) goto mma_abort;
           ++sd_it;
           tc_fence_after();
           const uint32_t q_s = qdo_s + (uint32_t)st * 2u * tb, do_s = q_s + tb;
@@ -455,30 +478,8 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
             tc_mma_f16(t_dp, abwd_desc_k16(v_s + (uint32_t)c * chunk), abwd_desc_k16(do_s + (uint32_t)c * chunk),
                        p.idesc_s, c > 0 ? 1u : 0u);
           tc_commit(sd_full);
-          return true;
-        };
-        if (!issue_sdp(0)) goto mma_abort;
-        for (int jj = 0; jj < n; ++jj) {
-          // with two Q/dO stages the next block's S^T, dP^T overlap this
-          // block's elementwise work; with one stage they must wait until
-          // dV, dK of this block have released it
-          if (nst >= 2 && jj + 1 < n && !issue_sdp(jj + 1)) goto mma_abort;
-          if (!mbar_wait(pds_full, pds_it & 1u, abort_flag)) goto mma_abort;
-          ++pds_it;
-          tc_fence_after();
-          const uint32_t qj = q_it + (uint32_t)jj;
-          const int st = (int)(qj % (uint32_t)nst);
-          const uint32_t q_s = qdo_s + (uint32_t)st * 2u * tb, do_s = q_s + tb;
-          for (int k2 = 0; k2 < 8; ++k2) {   // dV += P^T dO, dK += dS^T Q over the 128 queries
-            const uint32_t acc = (jj > 0 || k2 > 0) ? 1u : 0u;
-            tc_mma_f16(t_dv, abwd_desc_a(pt_s, k2), abwd_desc_mn(do_s, k2), p.idesc_acc, acc);
-            tc_mma_f16(t_dk, abwd_desc_a(dst_s, k2), abwd_desc_mn(q_s, k2), p.idesc_acc, acc);
-          }
-          tc_commit(pds_free);
-          tc_commit(qdo_empty(st));
-          if (nst == 1 && jj + 1 < n && !issue_sdp(jj + 1)) goto mma_abort;
         }
-        tc_commit(kv_empty);
+        tc_commit(kv_empty);                 // K and V are read by these MMAs only
         q_it += (uint32_t)n;
       }
       goto mma_done;
@@ -486,6 +487,40 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
       tc_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0);
     mma_done:;
+    }
+  } else if (warp == 10) {
+    if (lane == 0) {
+      // ---------------------- MMA: dV += P_j^T dO_j, dK += dS_j^T Q_j
+      // A second issuing thread, alongside the S^T / dP^T MMAs.  P^T and dS^T
+      // of block j exist only after its S^T / dP^T MMAs completed, so the
+      // Q / dO stage is free once these MMAs complete.
+      uint32_t q_it = 0, pds_it = 0;
+      for (long long item = blockIdx.x; item < p.items; item += gridDim.x) {
+        int g, kb;
+        decode(item, g, kb);
+        const int n = p.tiles - kb;
+        for (int jj = 0; jj < n; ++jj) {
+          if (!mbar_wait(pds_full, pds_it & 1u, abort_flag)) goto acc_abort;
+          ++pds_it;
+          tc_fence_after();
+          const uint32_t qj = q_it + (uint32_t)jj;
+          const int st = (int)(qj % (uint32_t)nst);
+          const uint32_t q_s = qdo_s + (uint32_t)st * 2u * tb, do_s = q_s + tb;
+          for (int k2 = 0; k2 < 8; ++k2) {   // over the 128 queries
+            const uint32_t acc = (jj > 0 || k2 > 0) ? 1u : 0u;
+            tc_mma_f16(t_dv, abwd_desc_a(pt_s, k2), abwd_desc_mn(do_s, k2), p.idesc_acc, acc);
+            tc_mma_f16(t_dk, abwd_desc_a(dst_s, k2), abwd_desc_mn(q_s, k2), p.idesc_acc, acc);
+          }
+          tc_commit(pds_free);
+          tc_commit(qdo_empty(st));
+        }
+        q_it += (uint32_t)n;
+      }
+      goto acc_done;
+    acc_abort:
+      tc_commit(drain_acc);
+      mbar_wait_drain(drain_acc, 0);
+    acc_done:;
     }
   } else {
     // ------------------------------------------- elementwise: one (key row, half)

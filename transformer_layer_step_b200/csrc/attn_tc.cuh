@@ -10,15 +10,16 @@
 // log-sum-exp of each row's scaled scores, from which the backward
 // recomputes P.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work items):
+// Warp roles (224 threads, one CTA per SM, persistent over work items):
 //   warp 0     TMA: Q once per item, then K and V of each key block into a
 //              2-stage ring;
-//   warp 1     one thread issues the MMAs: S_j = Q K_j^T into one of two S
-//              buffers, and O += P_{j-1} V_{j-1} once P_{j-1} is ready;
+//   warp 1     one thread issues S_j = Q K_j^T into one of two S buffers;
+//   warp 6     one thread issues O += P_j V_j once P_j is ready (two issuing
+//              threads, so that the two MMA streams run concurrently);
 //   warps 2-5  one query row per thread: read S_j from tensor memory, update
 //              the running max m and sum l, rescale O by exp2(m_old - m_new)
-//              in tensor memory, write P_j (16-bit) to shared memory; at the
-//              end normalise O by 1/l and store it.
+//              in tensor memory when m moved, write P_j (16-bit) to shared
+//              memory; at the end normalise O by 1/l and store it.
 // Tensor memory: S buffers at columns 0 and 128, O at column 256.
 // Shared memory: P [128 x 128] (two 128B-swizzled 64-column atoms), Q as
 // head_dim/16 chunks of [128 rows x 16] (32B swizzle), and per stage K the
@@ -28,7 +29,7 @@
 
 namespace gptl {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 224;
 constexpr int kAttnTile = 128;          // query rows per item, keys per block
 
 struct AttnParams {
@@ -44,6 +45,7 @@ struct AttnParams {
   float *lse;           // [groups][s]
   long long items;      // groups * q_tiles
   int q_off, k_off, v_off;   // column offsets of Q, K, V inside a shard's 3h/t columns
+  int kv_stages;             // depth of the K / V ring (2..4)
 };
 
 // K-major operand chunk of 16 columns, 32B swizzle: rows of 32 B, 8-row
@@ -64,31 +66,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   const uint32_t p_s = smem_u32(smem);                        // P: 32 KB
   const uint32_t q_s = p_s + 32768u;
   const uint32_t kv_s = q_s + q_bytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 32768u + q_bytes + 2u * kv_bytes);
-  // bars: q_full q_empty kv_full[2] kv_empty[2] s_full[2] s_empty[2] p_full o_done drain
+  const uint32_t nkv = (uint32_t)p.kv_stages;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 32768u + q_bytes + nkv * kv_bytes);
+  // bars: q_full q_empty kv_full[4] kv_empty[4] s_full[2] s_empty[2] p_full o_done drain drain2
   const uint32_t q_full = smem_u32(&bars[0]), q_empty = smem_u32(&bars[1]);
   auto kv_full = [&](int i) { return smem_u32(&bars[2 + i]); };
-  auto kv_empty = [&](int i) { return smem_u32(&bars[4 + i]); };
-  auto s_full = [&](int i) { return smem_u32(&bars[6 + i]); };
-  auto s_empty = [&](int i) { return smem_u32(&bars[8 + i]); };
-  const uint32_t p_full = smem_u32(&bars[10]), o_done = smem_u32(&bars[11]);
-  const uint32_t drain_bar = smem_u32(&bars[12]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+  auto kv_empty = [&](int i) { return smem_u32(&bars[6 + i]); };
+  auto s_full = [&](int i) { return smem_u32(&bars[10 + i]); };
+  auto s_empty = [&](int i) { return smem_u32(&bars[12 + i]); };
+  const uint32_t p_full = smem_u32(&bars[14]), o_done = smem_u32(&bars[15]);
+  const uint32_t drain_bar = smem_u32(&bars[16]), drain_pv = smem_u32(&bars[17]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(kv_full(i), 1);
       mbar_init(kv_empty(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
       mbar_init(s_empty(i), 4);
     }
     mbar_init(p_full, 4);
     mbar_init(o_done, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(drain_pv, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -129,8 +135,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           tma_load_3d(q_s + (uint32_t)c * chunk_bytes, &p.map_qk, p.q_off + head * d + c * 16,
                       qt * kAttnTile, zb, q_full);
         for (int j = 0; j <= qt; ++j, ++kv_it) {
-          const int st = (int)(kv_it & 1u);
-          const uint32_t ph = (kv_it >> 1) & 1u;
+          const int st = (int)(kv_it % nkv);
+          const uint32_t ph = (kv_it / nkv) & 1u;
           if (!mbar_wait(kv_empty(st), ph ^ 1u, abort_flag)) goto tma_abort;
           mbar_arrive_expect_tx(kv_full(st), kv_bytes);
           const uint32_t k_s = kv_s + (uint32_t)st * kv_bytes, v_s = k_s + q_bytes;
@@ -148,57 +154,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       }
       goto tma_done;
     tma_abort:
-      for (int s2 = 0; s2 < 2; ++s2)
+      for (int s2 = 0; s2 < (int)nkv; ++s2)
         if (issued & (1u << s2)) mbar_wait_drain(kv_full(s2), (parity_bits >> s2) & 1u);
       if (q_parity >= 0) mbar_wait_drain(q_full, (uint32_t)q_parity);
     tma_done:;
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ------------------------------------------------------------ MMA
-      uint32_t kv_it = 0, s_it = 0, p_it = 0, item_n = 0;
+      // ------------------------------------------------ MMA: S_j = Q K_j^T
+      uint32_t kv_it = 0, s_it = 0, item_n = 0;
       for (long long item = blockIdx.x; item < p.items; item += gridDim.x, ++item_n) {
         int g, qt;
         decode(item, g, qt);
         const int n = qt + 1;
         if (!mbar_wait(q_full, item_n & 1u, abort_flag)) goto mma_abort;
         tc_fence_after();
-        for (int j = 0; j <= n; ++j) {
-          if (j < n) {
-            const uint32_t kj = kv_it + (uint32_t)j;
-            if (!mbar_wait(kv_full(kj & 1u), (kj >> 1) & 1u, abort_flag)) goto mma_abort;
-            const int sb = (int)(s_it & 1u);
-            if (!mbar_wait(s_empty(sb), ((s_it >> 1) & 1u) ^ 1u, abort_flag)) goto mma_abort;
-            tc_fence_after();
-            const uint32_t k_s = kv_s + (kj & 1u) * kv_bytes;
-            for (int c = 0; c < d / 16; ++c)
-              tc_mma_f16(tmem_base + (uint32_t)(sb * 128), attn_desc_k16(q_s + (uint32_t)c * chunk_bytes),
-                         attn_desc_k16(k_s + (uint32_t)c * chunk_bytes), p.idesc_s, c > 0 ? 1u : 0u);
-            tc_commit(s_full(sb));
-            ++s_it;
-          }
-          if (j >= 1) {
-            if (!mbar_wait(p_full, p_it & 1u, abort_flag)) goto mma_abort;
-            ++p_it;
-            tc_fence_after();
-            const uint32_t pj = kv_it + (uint32_t)(j - 1);
-            const uint32_t v_s = kv_s + (pj & 1u) * kv_bytes + q_bytes;
-            const uint32_t row_b = (uint32_t)p.vw * 2u;
-            const uint32_t kb_bytes = (uint32_t)(d / p.vw) * 64u * row_b;
-            const uint32_t vsw = p.vw == 64 ? 2u : (p.vw == 32 ? 4u : 6u);
-            for (int st = 0; st < 8; ++st) {
-              const uint64_t adesc =
-                  make_smem_desc(p_s + (uint32_t)(st >> 2) * 16384u + (uint32_t)(st & 3) * 32u, 16u, 1024u, 2u);
-              const uint64_t bdesc = make_smem_desc(v_s + (uint32_t)(st >> 2) * kb_bytes +
-                                                        (uint32_t)(st & 3) * 16u * row_b,
-                                                    64u * row_b, 8u * row_b, vsw);
-              tc_mma_f16(tmem_o, adesc, bdesc, p.idesc_pv, (j > 1 || st > 0) ? 1u : 0u);
-            }
-            tc_commit(o_done);
-            tc_commit(kv_empty(pj & 1u));
-          }
+        for (int j = 0; j < n; ++j) {
+          const uint32_t kj = kv_it + (uint32_t)j;
+          if (!mbar_wait(kv_full((int)(kj % nkv)), (kj / nkv) & 1u, abort_flag)) goto mma_abort;
+          const int sb = (int)(s_it & 1u);
+          if (!mbar_wait(s_empty(sb), ((s_it >> 1) & 1u) ^ 1u, abort_flag)) goto mma_abort;
+          tc_fence_after();
+          const uint32_t k_s = kv_s + (kj % nkv) * kv_bytes;
+          for (int c = 0; c < d / 16; ++c)
+            tc_mma_f16(tmem_base + (uint32_t)(sb * 128), attn_desc_k16(q_s + (uint32_t)c * chunk_bytes),
+                       attn_desc_k16(k_s + (uint32_t)c * chunk_bytes), p.idesc_s, c > 0 ? 1u : 0u);
+          tc_commit(s_full(sb));
+          ++s_it;
         }
-        tc_commit(q_empty);
+        tc_commit(q_empty);                  // Q is read by these MMAs only
         kv_it += (uint32_t)n;
       }
       goto mma_done;
@@ -206,6 +190,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       tc_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0);
     mma_done:;
+    }
+  } else if (warp == 6) {
+    if (lane == 0) {
+      // ------------------------------------------- MMA: O += P_j V_j
+      // A second issuing thread: its MMAs run alongside the S MMAs.  P_j
+      // exists only after S_j was read, so K_j is no longer in use when the
+      // stage is released here.
+      uint32_t kv_it = 0, p_it = 0;
+      for (long long item = blockIdx.x; item < p.items; item += gridDim.x) {
+        int g, qt;
+        decode(item, g, qt);
+        const int n = qt + 1;
+        for (int j = 0; j < n; ++j) {
+          if (!mbar_wait(p_full, p_it & 1u, abort_flag)) goto pv_abort;
+          ++p_it;
+          tc_fence_after();
+          const uint32_t pj = kv_it + (uint32_t)j;
+          const uint32_t v_s = kv_s + (pj % nkv) * kv_bytes + q_bytes;
+          const uint32_t row_b = (uint32_t)p.vw * 2u;
+          const uint32_t kb_bytes = (uint32_t)(d / p.vw) * 64u * row_b;
+          const uint32_t vsw = p.vw == 64 ? 2u : (p.vw == 32 ? 4u : 6u);
+          for (int st = 0; st < 8; ++st) {
+            const uint64_t adesc =
+                make_smem_desc(p_s + (uint32_t)(st >> 2) * 16384u + (uint32_t)(st & 3) * 32u, 16u, 1024u, 2u);
+            const uint64_t bdesc = make_smem_desc(v_s + (uint32_t)(st >> 2) * kb_bytes +
+                                                      (uint32_t)(st & 3) * 16u * row_b,
+                                                  64u * row_b, 8u * row_b, vsw);
+            tc_mma_f16(tmem_o, adesc, bdesc, p.idesc_pv, (j > 0 || st > 0) ? 1u : 0u);
+          }
+          tc_commit(o_done);
+          tc_commit(kv_empty((int)(pj % nkv)));
+        }
+        kv_it += (uint32_t)n;
+      }
+      goto pv_done;
+    pv_abort:
+      tc_commit(drain_pv);
+      mbar_wait_drain(drain_pv, 0);
+    pv_done:;
     }
   } else {
     // -------------------------------------------------- softmax and epilogue

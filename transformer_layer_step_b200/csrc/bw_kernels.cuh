@@ -314,39 +314,70 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T *__restrict__ a, in
 }
 
 // -------------------------------------------------------------- transpose
-// out[c][r] = in[r][c] for a rows x cols 16-bit matrix (row pitches in
-// elements; rows, cols, pitches multiples of 8).  64 x 64 tiles through
-// shared memory: 16-byte coalesced loads, and each thread stores 32
-// contiguous bytes of an output row.
-// blockIdx.z indexes a batch of matrices (pitches bs_in, bs_out elements).
-__global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t *__restrict__ in,
-                                                          uint16_t *__restrict__ out, int rows,
-                                                          int cols, long long ld_in,
-                                                          long long ld_out, long long bs_in,
-                                                          long long bs_out) {
-  __shared__ __align__(16) uint16_t tile[64][64 + 8];
-  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
-  in += (long long)blockIdx.z * bs_in;
-  out += (long long)blockIdx.z * bs_out;
+// out[c][r] = in[r][c] for up to kMaxTransposeJobs 16-bit matrices (each a
+// batch of `batch` matrices bs_in / bs_out elements apart; rows, cols and all
+// pitches multiples of 8) in one launch; blockIdx.x runs over the 64 x 64
+// tiles of all jobs.
+//
+// A tile goes through shared memory as 32-bit words holding the pair of
+// elements (r, c), (r+1, c), stored at word [c][r/2 ^ swz(c)] with
+// swz(c) = 4 ((c / 8 + c % 8) % 8): the 8 column groups a warp writes land in
+// distinct banks, and a 16-byte read of four consecutive pairs of one output
+// row stays contiguous and aligned.  Loads and stores are 16-byte vectors,
+// coalesced in 128-byte rows.
+constexpr int kMaxTransposeJobs = 4;
+struct TransposeJob {
+  const uint16_t *in;
+  uint16_t *out;
+  int rows, cols;
+  long long ld_in, ld_out, bs_in, bs_out;
+  int tiles_c, tiles_r;        // 64 x 64 tiles per matrix
+  long long tile0;             // first global tile index of this job
+};
+struct TransposeJobs {
+  TransposeJob job[kMaxTransposeJobs];
+  int n;
+};
+
+__device__ __forceinline__ int transpose_swz(int c) { return 4 * (((c >> 3) + (c & 7)) & 7); }
+
+__global__ void __launch_bounds__(256) transpose16_kernel(const __grid_constant__ TransposeJobs jobs) {
+  __shared__ __align__(16) uint32_t tile[64 * 32];
+  long long t = blockIdx.x;
+  int jn = 0;
+  while (jn + 1 < jobs.n && t >= jobs.job[jn + 1].tile0) ++jn;
+  const TransposeJob &J = jobs.job[jn];
+  t -= J.tile0;
+  const long long per = (long long)J.tiles_c * J.tiles_r;
+  const long long b = t / per;
+  const int rem = (int)(t - b * per);
+  const int r0 = (rem / J.tiles_c) * 64, c0 = (rem % J.tiles_c) * 64;
+  const uint16_t *in = J.in + b * J.bs_in;
+  uint16_t *out = J.out + b * J.bs_out;
+  const int tid = threadIdx.x;
+  {
+    const int cg = tid & 7, rp = tid >> 3;   // columns 8 cg .. 8 cg + 7, rows 2 rp, 2 rp + 1
+    const int r = r0 + 2 * rp, c = c0 + 8 * cg;
+    uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+    if (c < J.cols) {
+      if (r < J.rows) v0 = __ldcs(reinterpret_cast<const uint4 *>(in + (long long)r * J.ld_in + c));
+      if (r + 1 < J.rows) v1 = __ldcs(reinterpret_cast<const uint4 *>(in + (long long)(r + 1) * J.ld_in + c));
+    }
+    const uint32_t a[4] = {v0.x, v0.y, v0.z, v0.w}, bb[4] = {v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-  for (int it = 0; it < 2; ++it) {
-    const int i = threadIdx.x + it * 256;
-    const int r = i >> 3, v = i & 7;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (r0 + r < rows && c0 + v * 8 < cols)
-      val = __ldcs(reinterpret_cast<const uint4 *>(in + (long long)(r0 + r) * ld_in + c0 + v * 8));
-    *reinterpret_cast<uint4 *>(&tile[r][v * 8]) = val;
+    for (int i = 0; i < 4; ++i) {
+      const int ce = 8 * cg + 2 * i;           // even column of the word pair
+      tile[ce * 32 + (rp ^ transpose_swz(ce))] = __byte_perm(a[i], bb[i], 0x5410);
+      tile[(ce + 1) * 32 + (rp ^ transpose_swz(ce + 1))] = __byte_perm(a[i], bb[i], 0x7632);
+    }
   }
   __syncthreads();
-  const int c = threadIdx.x & 63, vp = threadIdx.x >> 6;   // output row c0+c, elements 16vp..16vp+15
-  if (c0 + c < cols) {
-    uint32_t w[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      w[k] = (uint32_t)tile[vp * 16 + 2 * k][c] | ((uint32_t)tile[vp * 16 + 2 * k + 1][c] << 16);
-    uint16_t *dst = out + (long long)(c0 + c) * ld_out + r0 + vp * 16;
-    if (r0 + vp * 16 < rows) *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-    if (r0 + vp * 16 + 8 < rows) *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+  for (int pass = 0; pass < 2; ++pass) {
+    const int c = pass * 32 + (tid >> 3), q = tid & 7;   // output row c, elements 8 q .. 8 q + 7
+    const uint4 w = *reinterpret_cast<const uint4 *>(&tile[c * 32 + ((4 * q) ^ transpose_swz(c))]);
+    if (c0 + c < J.cols && r0 + 8 * q < J.rows)
+      *reinterpret_cast<uint4 *>(out + (long long)(c0 + c) * J.ld_out + r0 + 8 * q) = w;
   }
 }
 

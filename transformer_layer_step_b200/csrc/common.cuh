@@ -118,8 +118,8 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
 }
 
 // --------------------------------------------------------------------- TMA
-// 3-D tiled tensor load into shared memory, completing on an mbarrier.  No
-// multicast: every CTA loads its own operands.
+// 3-D tiled tensor load into shared memory, completing on an mbarrier.
+// Every CTA loads its own operands from this GPU's memory.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             int z, uint32_t bar) {
   asm volatile(

@@ -35,7 +35,7 @@ namespace gptl {
 
 constexpr int kBM = 128;          // tile rows (UMMA M)
 constexpr int kBK = 64;           // tile depth per pipeline stage
-constexpr int kGemmThreads = 320;
+constexpr int kGemmThreads = 384;
 constexpr int kEpiWarps = 8;
 
 enum : int { kActNone = 0, kActGelu = 1, kActDGelu = 2 };
@@ -60,6 +60,7 @@ struct alignas(64) GemmParams {
   OperandRule ra, rb;
   int M, N, K, groups, k_shards, causal;
   int split;                   // K slices per tile (split-K); 1 = none
+  int pipe_k;                  // 1: both pipelines work on every tile, one K half each
   float *ws;                   // split-K partials [split][groups][M][N] fp32
   long long ws_slice;          // groups * M * N
   int bn, bn_alloc, stages, tmem_cols;
@@ -145,9 +146,8 @@ __device__ __forceinline__ uint64_t operand_desc(const OperandRule &r, uint32_t 
 // that their latency overlaps the previous chunk's arithmetic.
 struct EpiIn {
   uint4 bias[2];     // 16-bit bias
-  uint4 aux[2];      // 16-bit GeLU' argument
-  uint4 r16[2];      // 16-bit residual
-  float4 r32[4];     // fp32 residual
+  uint4 v[4];        // fp32 residual (4 vectors), or 16-bit residual / GeLU' argument (2):
+                     // a GEMM has at most one of them
 };
 
 // Per-thread row pointers of the epilogue inputs for one tile (null when
@@ -183,19 +183,18 @@ __device__ __forceinline__ void epilogue_load(const GemmParams &p, const EpiRow 
   }
   if (e.resid) {
     if (p.resid_f32) {
-      const float4 *rr = reinterpret_cast<const float4 *>(e.resid) + n / 4;
+      const uint4 *rr = reinterpret_cast<const uint4 *>(e.resid) + n / 4;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) in.r32[q] = rr[q];
+      for (int q = 0; q < 4; ++q) in.v[q] = rr[q];
     } else {
       const uint4 *rr = reinterpret_cast<const uint4 *>(e.resid) + n / 8;
-      in.r16[0] = rr[0];
-      in.r16[1] = rr[1];
+      in.v[0] = rr[0];
+      in.v[1] = rr[1];
     }
-  }
-  if (e.aux) {
+  } else if (e.aux) {
     const uint4 *xp = reinterpret_cast<const uint4 *>(e.aux) + n / 8;
-    in.aux[0] = xp[0];
-    in.aux[1] = xp[1];
+    in.v[0] = xp[0];
+    in.v[1] = xp[1];
   }
 }
 
@@ -228,14 +227,14 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow
     if (p.resid_f32) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        v[4 * q] += in.r32[q].x; v[4 * q + 1] += in.r32[q].y;
-        v[4 * q + 2] += in.r32[q].z; v[4 * q + 3] += in.r32[q].w;
+        v[4 * q] += __uint_as_float(in.v[q].x); v[4 * q + 1] += __uint_as_float(in.v[q].y);
+        v[4 * q + 2] += __uint_as_float(in.v[q].z); v[4 * q + 3] += __uint_as_float(in.v[q].w);
       }
     } else {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float f[8];
-        unpack8<T>(in.r16[h], f);
+        unpack8<T>(in.v[h], f);
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[8 * h + i] += f[i];
       }
@@ -269,7 +268,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       float z[8];
-      unpack8<T>(in.aux[h], z);
+      unpack8<T>(in.v[h], z);
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[8 * h + i] *= gelu_prime_f(z[i]);
     }
@@ -283,6 +282,32 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow
   }
 }
 
+// Two independent pipelines share the CTA.  Either the CTA's tiles alternate
+// between them (local tile t goes to pipeline t % 2), or, with pipe_k (few,
+// long-K tiles), both work on every tile: pipeline p reduces the p-th half of
+// the tile's k-blocks into its own accumulator and the epilogue adds the two
+// (acc0 + acc1, a fixed order).  Each pipeline has its own
+// producer warp, shared-memory ring (p.stages stages), MMA-issuing warp and
+// TMEM accumulator (columns [pipe * bn_alloc, +bn)).  Measured on B200, one
+// thread's stream of tcgen05.mma instructions runs at a fixed rate per
+// instruction well below the tensor core's, and two issuing warps run
+// concurrently; the two accumulators also give the epilogue of one tile the
+// other pipeline's MMAs to overlap with.
+// Does pipeline pp take local tile t, and which of its k-blocks?
+__device__ __forceinline__ bool pipe_takes(const GemmParams &p, int t, int pp) {
+  return p.pipe_k ? true : ((t & 1) == pp);
+}
+__device__ __forceinline__ void pipe_kb_range(const GemmParams &p, const TileInfo &ti, int pp,
+                                              int &kb0, int &kb1) {
+  kb0 = ti.kb_begin;
+  kb1 = ti.kb_end;
+  if (p.pipe_k) {
+    const int mid = ti.kb_begin + (ti.kb_end - ti.kb_begin) / 2;
+    if (pp == 0) kb1 = mid;
+    else kb0 = mid;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -291,29 +316,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
   const int a_bytes = kBM * kBK * 2;
   const int b_bytes = p.bn * kBK * 2;
   const int stage_bytes = a_bytes + b_bytes;
-  const uint32_t staging_s = smem_u32(smem + p.stages * stage_bytes);   // 1024-aligned
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.stages * stage_bytes + kStagingBytes);
-  // bars: full[0,S) empty[S,2S) tfull[2S,2S+2) tempty[2S+2,2S+4) drain[2S+4]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * p.stages + 5);
+  const int S = p.stages;                                   // stages per pipeline
+  const uint32_t staging_s = smem_u32(smem + 2 * S * stage_bytes);   // 1024-aligned
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * S * stage_bytes + kStagingBytes);
+  // bars: full[pipe][S] empty[pipe][S] tfull[2] tempty[2] drain[2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 6);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const uint32_t tiles_s = smem_u32(smem);
-  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
-  auto empty_bar = [&](int s) { return smem_u32(&bars[p.stages + s]); };
-  auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * p.stages + a]); };
-  auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * p.stages + 2 + a]); };
-  const uint32_t drain_bar = smem_u32(&bars[2 * p.stages + 4]);
+  auto full_bar = [&](int pp, int s) { return smem_u32(&bars[pp * S + s]); };
+  auto empty_bar = [&](int pp, int s) { return smem_u32(&bars[2 * S + pp * S + s]); };
+  auto tfull_bar = [&](int pp) { return smem_u32(&bars[4 * S + pp]); };
+  auto tempty_bar = [&](int pp) { return smem_u32(&bars[4 * S + 2 + pp]); };
+  auto drain_bar = [&](int pp) { return smem_u32(&bars[4 * S + 4 + pp]); };
+  auto stage_addr = [&](int pp, int s) { return tiles_s + (uint32_t)((pp * S + s) * stage_bytes); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < p.stages; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+    for (int pp = 0; pp < 2; ++pp) {
+      for (int s = 0; s < S; ++s) {
+        mbar_init(full_bar(pp, s), 1);
+        mbar_init(empty_bar(pp, s), 1);
+      }
+      mbar_init(tfull_bar(pp), 1);
+      mbar_init(tempty_bar(pp), kEpiWarps);
+      mbar_init(drain_bar(pp), 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), kEpiWarps);
-    }
-    mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -332,25 +359,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < 4) {
+    const int pp = warp >> 1;                 // pipeline of this warp
+    if (lane == 0 && (warp & 1) == 0) {
       // ------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0, issued = 0, parity = 0;
+      int t = 0;                              // local tile counter (non-skipped tiles)
       for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
         const TileInfo ti = tile_info(p, idx);
         if (ti.skip) continue;
+        if (!pipe_takes(p, t++, pp)) continue;
+        int kb0, kb1;
+        pipe_kb_range(p, ti, pp, kb0, kb1);
         for (int ks = 0; ks < p.k_shards; ++ks)
-          for (int kb = ti.kb_begin; kb < ti.kb_end; ++kb) {
-            if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag)) goto producer_abort;
-            const uint32_t fb = full_bar(stage);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(empty_bar(pp, stage), phase ^ 1, abort_flag)) goto producer_abort;
+            const uint32_t fb = full_bar(pp, stage);
             mbar_arrive_expect_tx(fb, (uint32_t)stage_bytes);
-            const uint32_t sa = tiles_s + (uint32_t)(stage * stage_bytes);
+            const uint32_t sa = stage_addr(pp, stage);
             load_operand(&p.map_a, p.ra, sa, kBM, ti.g, ks, ti.m0, kb * kBK, fb);
             load_operand(&p.map_b, p.rb, sa + a_bytes, p.bn, ti.g, ks, ti.n0, kb * kBK, fb);
             issued |= 1u << stage;
             parity = (parity & ~(1u << stage)) | (phase << stage);
-            if (++stage == p.stages) {
+            if (++stage == S) {
               stage = 0;
               phase ^= 1;
             }
@@ -359,70 +391,75 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       goto producer_done;
     producer_abort:
       // let our own copies land before the CTA exits
-      for (int s = 0; s < p.stages; ++s)
-        if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (parity >> s) & 1u);
+      for (int s = 0; s < S; ++s)
+        if (issued & (1u << s)) mbar_wait_drain(full_bar(pp, s), (parity >> s) & 1u);
     producer_done:;
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      int stage = 0, acc = 0;
+      int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
+      int t = 0;
+      const uint32_t d_tmem = tmem_base + (uint32_t)(pp * p.bn_alloc);
       for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
         const TileInfo ti = tile_info(p, idx);
         if (ti.skip) continue;
-        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1, abort_flag)) goto mma_abort;
+        if (!pipe_takes(p, t++, pp)) continue;
+        if (!mbar_wait(tempty_bar(pp), acc_phase ^ 1, abort_flag)) goto mma_abort;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * p.bn_alloc);
+        int kb0, kb1;
+        pipe_kb_range(p, ti, pp, kb0, kb1);
         int it = 0;
         for (int ks = 0; ks < p.k_shards; ++ks)
-          for (int kb = ti.kb_begin; kb < ti.kb_end; ++kb) {
-            if (!mbar_wait(full_bar(stage), phase, abort_flag)) goto mma_abort;
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(full_bar(pp, stage), phase, abort_flag)) goto mma_abort;
             tc_fence_after();
-            const uint32_t sa = tiles_s + (uint32_t)(stage * stage_bytes);
+            const uint32_t sa = stage_addr(pp, stage);
             const uint32_t sb = sa + (uint32_t)a_bytes;
             const int nsteps = min(kBK, p.K - kb * kBK) / 16;
             for (int s = 0; s < nsteps; ++s)
               tc_mma_f16(d_tmem, operand_desc(p.ra, sa, s), operand_desc(p.rb, sb, s), p.idesc,
                          (it > 0 || s > 0) ? 1u : 0u);
-            tc_commit(empty_bar(stage));
+            tc_commit(empty_bar(pp, stage));
             ++it;
-            if (++stage == p.stages) {
+            if (++stage == S) {
               stage = 0;
               phase ^= 1;
             }
           }
-        tc_commit(tfull_bar(acc));
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1;
-        }
+        tc_commit(tfull_bar(pp));
+        acc_phase ^= 1;
       }
       goto mma_done;
     mma_abort:
       // wait for the MMAs already issued before TMEM is released
-      tc_commit(drain_bar);
-      mbar_wait_drain(drain_bar, 0);
+      tc_commit(drain_bar(pp));
+      mbar_wait_drain(drain_bar(pp), 0);
     mma_done:;
     }
   } else {
     // -------------------------------------------------- epilogue warps
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;        // which half of the tile's columns
+    const int half = (warp - 4) >> 2;        // which half of the tile's columns
     const bool wide = p.out_f32 || p.split > 1;     // fp32: one chunk per box
     const bool gelu = !wide && p.act == kActGelu;   // Z and GeLU(Z): both boxes per chunk pair
-    const uint32_t my_boxes = staging_s + (uint32_t)((warp - 2) * 2 * kStageBoxBytes);
+    const uint32_t my_boxes = staging_s + (uint32_t)((warp - 4) * 2 * kStageBoxBytes);
     int box_i = 0;                           // boxes issued by this warp (selects the buffer)
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    uint32_t acc_phase[2] = {0u, 0u};
+    int t = 0;
     for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
       const TileInfo ti = tile_info(p, idx);
       if (ti.skip) continue;
-      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) break;
+      const int pp = p.pipe_k ? 0 : (t & 1);   // accumulator (with pipe_k: the first of two)
+      ++t;
+      bool got = mbar_wait(tfull_bar(pp), acc_phase[pp], abort_flag);
+      if (got && p.pipe_k) got = mbar_wait(tfull_bar(1), acc_phase[1], abort_flag);
+      if (!got) break;
+      acc_phase[pp] ^= 1;
+      if (p.pipe_k) acc_phase[1] ^= 1;
       tc_fence_after();
       const int row0 = ti.m0 + q * 32;
       const EpiRow er = epilogue_row<T>(p, ti.g, row0 + lane);
-      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.bn_alloc);
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(pp * p.bn_alloc);
       // output map coordinates of this tile's group
       int oz, ow;
       if (p.split > 1) { oz = ti.slice * p.groups + ti.g; ow = 0; }
@@ -440,6 +477,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       // is processed (tcgen05.wait::ld waits for every earlier load)
       uint32_t ra[16], rb[16];
       EpiIn ia, ib;
+      const uint32_t t_row2 = t_row + (uint32_t)p.bn_alloc;   // pipe_k: the second K half
+      auto ld = [&](int c, uint32_t (&r)[16]) { tmem_ld16(t_row + (uint32_t)(c * 16), r); };
+      // pipe_k: add the second accumulator's chunk c (loaded here, not ahead)
+      auto sum2 = [&](int c, uint32_t (&r)[16]) {
+        if (p.pipe_k) {
+          uint32_t r2[16];
+          tmem_ld16(t_row2 + (uint32_t)(c * 16), r2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
+        }
+      };
       auto process = [&](int c, const uint32_t (&r)[16], const EpiIn &in) {
         const int slot = wide ? 0 : ((c - c0) & 1);
         const bool first = slot == 0, last = wide || slot == 1 || c + 1 == c1;
@@ -465,33 +514,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         }
       };
       if (c0 < c1) {
-        tmem_ld16(t_row + (uint32_t)(c0 * 16), ra);
+        ld(c0, ra);
         epilogue_load<T>(p, er, ti.n0 + c0 * 16, ia);
         tmem_wait_ld();
+        sum2(c0, ra);
       }
       for (int c = c0; c < c1; c += 2) {
         const bool has_b = c + 1 < c1;
         if (has_b) {
-          tmem_ld16(t_row + (uint32_t)((c + 1) * 16), rb);
+          ld(c + 1, rb);
           epilogue_load<T>(p, er, ti.n0 + (c + 1) * 16, ib);
         }
         process(c, ra, ia);
         tmem_wait_ld();
         if (!has_b) break;
+        sum2(c + 1, rb);
         const bool has_a = c + 2 < c1;
         if (has_a) {
-          tmem_ld16(t_row + (uint32_t)((c + 2) * 16), ra);
+          ld(c + 2, ra);
           epilogue_load<T>(p, er, ti.n0 + (c + 2) * 16, ia);
         }
         process(c + 1, rb, ib);
         tmem_wait_ld();
+        if (has_a) sum2(c + 2, ra);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1;
+      if (lane == 0) {
+        mbar_arrive(tempty_bar(pp));
+        if (p.pipe_k) mbar_arrive(tempty_bar(1));
       }
     }
     // the staged boxes must be read, and the stores done, before the CTA exits
@@ -535,28 +586,43 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restr
 
 // Row term of the softmax backward: D[g][p] = sum_c dO[p][c] * O[p][c] over
 // the head's d columns (equal to sum_q P[p][q] dP[p][q], since O = P V).
-// One thread per (row, head) of the [t*b*s][h/t] matrices.
+// A warp per row of the [t*b*s][h/t] matrices reads the row in coalesced
+// 16-byte vectors and leaves one partial dot per vector in shared memory;
+// then one thread per (row, head) adds the head's d/8 partials in order.
+// Block: 8 rows; hs / 8 <= kRowdotMaxVec vectors per row.
+constexpr int kRowdotMaxVec = 512;
 template <typename T>
 __global__ void __launch_bounds__(256) attn_rowdot_kernel(const T *__restrict__ dout,
                                                           const T *__restrict__ o, float *__restrict__ dvec,
                                                           long long rows, int s, int hs, int as,
                                                           int d) {
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= rows * as) return;
-  const long long r = idx / as;
-  const int head = (int)(idx - r * as);
-  const uint4 *a = reinterpret_cast<const uint4 *>(dout + r * hs + (long long)head * d);
-  const uint4 *b = reinterpret_cast<const uint4 *>(o + r * hs + (long long)head * d);
-  float acc = 0.f;
-  for (int v = 0; v < d / 8; ++v) {
-    float fa[8], fb[8];
-    unpack8<T>(a[v], fa);
-    unpack8<T>(b[v], fb);
+  __shared__ float part[8][kRowdotMaxVec];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long r = (long long)blockIdx.x * 8 + w;
+  const int nv = hs / 8;
+  if (r < rows) {
+    const uint4 *a = reinterpret_cast<const uint4 *>(dout + r * hs);
+    const uint4 *b = reinterpret_cast<const uint4 *>(o + r * hs);
+    for (int v = lane; v < nv; v += 32) {
+      float fa[8], fb[8];
+      unpack8<T>(__ldcs(a + v), fa);
+      unpack8<T>(__ldcs(b + v), fb);
+      float acc = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc += fa[e] * fb[e];
+      for (int e = 0; e < 8; ++e) acc = fmaf(fa[e], fb[e], acc);
+      part[w][v] = acc;
+    }
   }
-  const long long zb = r / s, pos = r - zb * s;
-  dvec[(zb * as + head) * s + pos] = acc;
+  __syncthreads();
+  const int rl = threadIdx.x / as, head = threadIdx.x - rl * as;   // (row in block, head)
+  const long long rr = (long long)blockIdx.x * 8 + rl;
+  if (rl < 8 && rr < rows) {
+    const int vh = d / 8;
+    float acc = 0.f;
+    for (int v = 0; v < vh; ++v) acc += part[rl][head * vh + v];
+    const long long zb = rr / s, pos = rr - zb * s;
+    dvec[(zb * as + head) * s + pos] = acc;
+  }
 }
 
 }  // namespace gptl

@@ -245,29 +245,50 @@ int pick_bn(const gptl_gemm_desc &d, int sms) {
   return best;
 }
 
-// Split-K slices for an fp32-output GEMM: the count (1..8) that minimises the
-// estimated time of the tile waves plus the reduction of the partials, with
-// the partials fitting in ws_bytes.  Times in microseconds: one 128 x bn x 64
-// k-block at ~8 kFLOP/clock/SM and 1.8 GHz; the reduction streams
-// (2 * split + 1) partial arrays at ~4 TB/s plus a launch.
-int pick_split(long long tiles, int kb_per_shard, int k_shards, int bn, long long out_elems,
-               long long ws_bytes, int sms) {
-  const long long nkb = (long long)kb_per_shard;
-  const double kb_us = 128.0 * bn * 64 * 2 / (8192.0 * 1800.0);
-  double best = (double)((tiles + sms - 1) / sms) * nkb * k_shards * kb_us;
-  int best_s = 1;
-  for (int sp = 2; sp <= 8; ++sp) {
-    if (sp > nkb) break;
-    if ((long long)sp * out_elems * 4 > ws_bytes) break;
-    const long long items = tiles * sp;
-    const double t = (double)((items + sms - 1) / sms) * ((nkb + sp - 1) / sp) * k_shards * kb_us +
-                     (2.0 * sp + 1.0) * out_elems * 4 / 4.0e6 + 3.0;
-    if (t < best) {
-      best = t;
-      best_s = sp;
+// Tiling of one GEMM call: BN, split-K slices (fp32 output with a workspace
+// only) and whether the CTA's two pipelines share each tile as K halves.
+// Chosen by a time estimate in microseconds.  A k-block through one pipeline
+// costs about the same for BN = 128 and 256 (the MMA-issuing thread, not the
+// tensor core, sets the pace: measured on B200), ~0.55 us.
+//   tiles alternating between the pipelines: ceil(ceil(items / SMs) / 2) x kb
+//   both pipelines on every tile:            ceil(items / SMs) x ceil(kb / 2)
+// where items = tiles x split and kb = k-blocks of one item; split > 1 adds
+// the partial-sum pass, (2 split + 1) fp32 arrays at ~4 TB/s plus a launch.
+struct GemmTiling {
+  int bn, split, pipe_k;
+};
+GemmTiling choose_tiling(const gptl_gemm_desc &d, int sms, bool can_split) {
+  GemmTiling best{pick_bn(d, sms), 1, 0};
+  if (d.causal != GPTL_CAUSAL_NONE) return best;
+  const double t_kb = 0.55;
+  const long long m_tiles = (d.M + kBM - 1) / kBM;
+  const long long kb_all = (long long)((d.K + kBK - 1) / kBK) * d.k_shards;
+  const double out_bytes = (double)d.groups * d.M * d.N * 4.0;
+  double best_t = -1.0;
+  const int n_bn = d.N <= 256 ? 1 : 2;
+  for (int ib = 0; ib < n_bn; ++ib) {
+    const int bn = d.N <= 256 ? d.N : (ib == 0 ? 256 : 128);
+    const long long tiles = m_tiles * ((d.N + bn - 1) / bn) * d.groups;
+    for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
+      if (sp > (d.K + kBK - 1) / kBK) break;
+      if (sp > 1 && (double)sp * out_bytes > (double)d.ws_bytes) break;
+      const long long items = tiles * sp;
+      const long long kb = (kb_all + sp - 1) / sp;
+      const long long per_cta = (items + sms - 1) / sms;
+      for (int pk = 0; pk < 2; ++pk) {
+        // every slice must give each pipeline at least one k-block
+        if (pk && ((d.K + kBK - 1) / kBK) / sp < 2) continue;
+        double t = pk ? (double)per_cta * ((kb + 1) / 2) * t_kb
+                      : (double)((per_cta + 1) / 2) * kb * t_kb;
+        if (sp > 1) t += (2.0 * sp + 1.0) * out_bytes / 4.0e6 + 3.0;
+        if (best_t < 0 || t < best_t * 0.999) {
+          best_t = t;
+          best = GemmTiling{bn, sp, pk};
+        }
+      }
     }
   }
-  return best_s;
+  return best;
 }
 
 template <typename T>
@@ -302,12 +323,16 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   if (d.act == GPTL_ACT_DGELU && !d.aux) return GPTL_E_NULL;
   if ((d.out2 && !aligned16(d.out2)) || (d.aux && !aligned16(d.aux))) return GPTL_E_ALIGN;
   if (d.act < 0 || d.act > 2 || (d.out_f32 && d.act != GPTL_ACT_NONE)) return GPTL_E_SHAPE;
+  if (d.resid && d.act == GPTL_ACT_DGELU) return GPTL_E_SHAPE;   // one epilogue input per GEMM
   GPTL_TRY(check_operand(d.a));
   GPTL_TRY(check_operand(d.b));
 
   GemmParams p;
   memset(&p, 0, sizeof(p));
-  const int bn = pick_bn(d, sms);
+  const bool can_split = d.out_f32 && !d.bias && !d.resid && d.act == GPTL_ACT_NONE &&
+                         d.causal == GPTL_CAUSAL_NONE && d.ws && aligned16(d.ws);
+  const GemmTiling tl = choose_tiling(d, sms, can_split);
+  const int bn = tl.bn;
   const int wa = d.a.mn_major ? mn_chunk_width(kBM) : 64;
   const int wb = d.b.mn_major ? mn_chunk_width(bn) : 64;
   GPTL_TRY(encode_operand(&p.map_a, d.a, dt, kBM, wa));
@@ -337,10 +362,11 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.bn_alloc = bn_alloc;
   p.tmem_cols = 2 * bn_alloc;
   const int stage_bytes = (kBM + bn) * kBK * 2;
-  p.stages = (kSmemLimit - 2048 - kStagingBytes) / stage_bytes;
-  if (p.stages > 8) p.stages = 8;
+  // stages per pipeline; the kernel runs two pipelines with a ring each
+  p.stages = (kSmemLimit - 2048 - kStagingBytes) / (2 * stage_bytes);
+  if (p.stages > 4) p.stages = 4;
   if (p.stages < 2) return GPTL_E_SHAPE;
-  const int smem = 1024 + p.stages * stage_bytes + kStagingBytes + 256;
+  const int smem = 1024 + 2 * p.stages * stage_bytes + kStagingBytes + 512;
   const uint32_t fmt = dt == GPTL_BF16 ? 1u : 0u;
   p.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)d.a.mn_major << 15) |
             ((uint32_t)d.b.mn_major << 16) | ((uint32_t)(bn >> 3) << 17) |
@@ -348,11 +374,8 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.m_tiles = (d.M + kBM - 1) / kBM;
   p.n_tiles = (d.N + bn - 1) / bn;
   const long long tiles = (long long)p.m_tiles * p.n_tiles * d.groups;
-  p.split = 1;
-  if (d.out_f32 && !d.bias && !d.resid && d.act == GPTL_ACT_NONE && d.causal == GPTL_CAUSAL_NONE &&
-      d.ws && aligned16(d.ws))
-    p.split = pick_split(tiles, (d.K + kBK - 1) / kBK, d.k_shards, bn,
-                         (long long)d.groups * d.M * d.N, d.ws_bytes, sms);
+  p.split = tl.split;
+  p.pipe_k = tl.pipe_k;
   p.ws = static_cast<float *>(d.ws);
   p.ws_slice = (long long)d.groups * d.M * d.N;
   p.total_tiles = tiles * p.split;
@@ -446,7 +469,12 @@ int run_attn_fwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
   p.q_off = 0; p.k_off = hs; p.v_off = 2 * hs;
   // P 32 KB + Q + 2 stages of K and V, barriers; at least 120 KB so that one
   // CTA (and its 512 tensor-memory columns) owns each SM
-  int smem = 1024 + 32768 + 128 * d * 2 * 5 + 256;
+  // P 32 KB, Q, the K / V ring (as deep as fits, 2..4 stages), barriers
+  const int kv_stage = 2 * 128 * d * 2;
+  p.kv_stages = (kSmemLimit - 1024 - 32768 - 128 * d * 2 - 512) / kv_stage;
+  if (p.kv_stages > 4) p.kv_stages = 4;
+  if (p.kv_stages < 2) return GPTL_E_SHAPE;
+  int smem = 1024 + 32768 + 128 * d * 2 + p.kv_stages * kv_stage + 512;
   if (smem < 120 * 1024) smem = 120 * 1024;
   const int grid = (int)(p.items < sms ? p.items : sms);
   // the shared-memory opt-in is recorded per device and per dtype (both
@@ -515,13 +543,18 @@ int run_attn_bwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
   p.items = (long long)p.groups * p.tiles;
   p.q_off = 0; p.k_off = hs; p.v_off = 2 * hs;
   const int tb = 256 * d;
-  int smem_dq = 1024 + 32768 + 6 * tb + 256;
-  int nst = 2;
-  int smem_kv = 1024 + 65536 + 2 * tb + nst * 2 * tb + 2048 + 256;
-  if (smem_kv > kSmemLimit) {
-    nst = 1;
-    smem_kv = 1024 + 65536 + 2 * tb + nst * 2 * tb + 2048 + 256;
-  }
+  // rings as deep as shared memory allows (up to 4 stages): dQ kernel dS
+  // 32 KB + Q, dO + K/V stages; dK/dV kernel P^T, dS^T 64 KB + K, V + Q/dO
+  // stages + the staged lse / D vectors
+  int nkv = (kSmemLimit - 1024 - 32768 - 2 * tb - 512) / (2 * tb);
+  if (nkv > 4) nkv = 4;
+  if (nkv < 2) return GPTL_E_SHAPE;
+  int smem_dq = 1024 + 32768 + 2 * tb + nkv * 2 * tb + 512;
+  int nst = (kSmemLimit - 1024 - 65536 - 2 * tb - 2048 - 512) / (2 * tb);
+  if (nst > 4) nst = 4;
+  if (nst < 1) return GPTL_E_SHAPE;
+  int smem_kv = 1024 + 65536 + 2 * tb + nst * 2 * tb + 2048 + 512;
+  p.kv_stages = nkv;
   p.qdo_stages = nst;
   // at least 120 KB: one CTA (and its 512 tensor-memory columns) per SM
   if (smem_dq < 120 * 1024) smem_dq = 120 * 1024;
@@ -551,25 +584,59 @@ int run_attn_bwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
 
 // out [cols][rows] = in [rows][cols]^T (16-bit), for `batch` matrices
 // `bs_in` / `bs_out` elements apart.
-int run_transpose(int rows, int cols, const void *in, long long ld_in, void *out, long long ld_out,
-                  cudaStream_t st, int batch = 1, long long bs_in = 0, long long bs_out = 0) {
-  if (rows <= 0 || cols <= 0 || rows % 8 || cols % 8 || ld_in % 8 || ld_out % 8 || batch < 1 ||
-      bs_in % 8 || bs_out % 8)
-    return GPTL_E_SHAPE;
-  dim3 grid((cols + 63) / 64, (rows + 63) / 64, batch);
-  transpose16_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(in),
-                                           static_cast<uint16_t *>(out), rows, cols, ld_in, ld_out,
-                                           bs_in, bs_out);
+// One launch for up to kMaxTransposeJobs transposes (see transpose16_kernel).
+struct TransposeSpec {
+  int rows, cols;
+  const void *in;
+  long long ld_in;
+  void *out;
+  long long ld_out;
+  int batch;
+  long long bs_in, bs_out;
+};
+int run_transposes(const TransposeSpec *spec, int n, cudaStream_t st) {
+  if (n < 1 || n > kMaxTransposeJobs) return GPTL_E_ARG;
+  TransposeJobs jobs;
+  memset(&jobs, 0, sizeof(jobs));
+  long long tiles = 0;
+  for (int i = 0; i < n; ++i) {
+    const TransposeSpec &s = spec[i];
+    if (s.rows <= 0 || s.cols <= 0 || s.rows % 8 || s.cols % 8 || s.ld_in % 8 || s.ld_out % 8 ||
+        s.batch < 1 || s.bs_in % 8 || s.bs_out % 8)
+      return GPTL_E_SHAPE;
+    TransposeJob &J = jobs.job[i];
+    J.in = static_cast<const uint16_t *>(s.in);
+    J.out = static_cast<uint16_t *>(s.out);
+    J.rows = s.rows;
+    J.cols = s.cols;
+    J.ld_in = s.ld_in;
+    J.ld_out = s.ld_out;
+    J.bs_in = s.bs_in;
+    J.bs_out = s.bs_out;
+    J.tiles_c = (s.cols + 63) / 64;
+    J.tiles_r = (s.rows + 63) / 64;
+    J.tile0 = tiles;
+    tiles += (long long)J.tiles_c * J.tiles_r * s.batch;
+  }
+  jobs.n = n;
+  if (tiles >= (1ll << 31)) return GPTL_E_SHAPE;
+  transpose16_kernel<<<(unsigned)tiles, 256, 0, st>>>(jobs);
   GPTL_CK(cudaGetLastError());
   prof_launched(st, GPTL_KIND_TRANSPOSE);
   return GPTL_OK;
 }
 
+int run_transpose(int rows, int cols, const void *in, long long ld_in, void *out, long long ld_out,
+                  cudaStream_t st, int batch = 1, long long bs_in = 0, long long bs_out = 0) {
+  const TransposeSpec s{rows, cols, in, ld_in, out, ld_out, batch, bs_in, bs_out};
+  return run_transposes(&s, 1, st);
+}
+
 // D[g][p] = dO_p . O_p over each head's columns (the softmax backward's row term).
 int run_attn_rowdot(long long rows, int s, int hs, int as, int d, gptl_dtype dt, const void *dout,
                     const void *o, float *dvec, cudaStream_t st) {
-  const long long n = rows * as;
-  const unsigned grid = (unsigned)((n + 255) / 256);
+  if (hs % 8 || d % 8 || hs / 8 > kRowdotMaxVec || as > 32) return GPTL_E_SHAPE;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
   if (dt == GPTL_FP16)
     attn_rowdot_kernel<__half><<<grid, 256, 0, st>>>((const __half *)dout, (const __half *)o, dvec,
                                                      rows, s, hs, as, d);
@@ -762,7 +829,8 @@ int run_colsum(int rows, int n, int groups, long long ld, long long gstride, gpt
   if (rows <= 0 || n <= 0 || groups <= 0 || n % 8 || ld % 8 || (groups > 1 && gstride % 8))
     return GPTL_E_SHAPE;
   const int strips = (n + 255) / 256;
-  int split = (2 * sms + strips * groups - 1) / (strips * groups);
+  // enough blocks for ~8 per SM (bytes in flight for HBM bandwidth)
+  int split = (8 * sms + strips * groups - 1) / (strips * groups);
   if (split < 1) split = 1;
   if (split > kColsumMaxSplit) split = kColsumMaxSplit;
   if (split > (rows + 7) / 8) split = (rows + 7) / 8;
@@ -1040,11 +1108,14 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   // The input-gradient GEMMs read the weights with the reduction index
   // contiguous: transposed copies, shard by shard.
   g_tag = GPTL_TAG_B0_WT;
-  GPTL_TRY(run_transpose(h, fs, W->w_2, fs, w2t, h, st, t, (long long)h * fs, (long long)fs * h));
-  GPTL_TRY(run_transpose(fs, h, W->w_1, h, w1t, fs, st, t, (long long)fs * h, (long long)h * fs));
-  GPTL_TRY(run_transpose(h, hs, W->w_o, hs, wot, h, st, t, (long long)h * hs, (long long)hs * h));
-  GPTL_TRY(run_transpose(3 * hs, h, W->w_qkv, h, wqkvt, 3 * hs, st, t, (long long)3 * hs * h,
-                         (long long)h * 3 * hs));
+  {
+    const TransposeSpec wt[4] = {
+        {h, fs, W->w_2, fs, w2t, h, t, (long long)h * fs, (long long)fs * h},
+        {fs, h, W->w_1, h, w1t, fs, t, (long long)fs * h, (long long)h * fs},
+        {h, hs, W->w_o, hs, wot, h, t, (long long)h * hs, (long long)hs * h},
+        {3 * hs, h, W->w_qkv, h, wqkvt, 3 * hs, t, (long long)3 * hs * h, (long long)h * 3 * hs}};
+    GPTL_TRY(run_transposes(wt, 4, st));
+  }
 
   // ---- FFN2 (row split)
   g_tag = GPTL_TAG_B2_DW2;
