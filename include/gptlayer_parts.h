@@ -90,6 +90,18 @@ typedef struct {
 
 int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream);
 
+/* How gptl_gemm would run *d on the current device (no device work, same
+ * argument checks and error codes as gptl_gemm): the tile width bn, the
+ * split-K slice count (1 = none) and the use of each SM's two MMA pipelines:
+ *   GPTL_GEMM_ALTERNATE  128 x bn tiles alternate between the pipelines;
+ *   GPTL_GEMM_K_HALVES   both pipelines on each 128 x bn tile, one half of its
+ *                        K range each, summed in a fixed order;
+ *   GPTL_GEMM_M256       256 x bn tiles, one 128-row half per pipeline.
+ * Results do not depend on the choice beyond fp32 summation order, and are
+ * deterministic for a given choice. */
+enum { GPTL_GEMM_ALTERNATE = 0, GPTL_GEMM_K_HALVES = 1, GPTL_GEMM_M256 = 2 };
+int gptl_gemm_plan(const gptl_gemm_desc *d, gptl_dtype dtype, int *bn, int *split, int *mode);
+
 /* Fused causal attention forward ("Training GPT-2 with Megatron-LM" §6.2
  * fused softmax; scores never leave the chip).  qkv: [tp][batch*seq][3h/tp],
  * shard i's columns [Q_i | K_i | V_i], each head_dim = hidden/heads columns

@@ -317,3 +317,58 @@ def test_interleaved_group_output_and_padding(dtype, out_f32):
         tol = 1e-5 if out_f32 else 8e-3
         assert float(np.abs(part - exp).max()) <= tol * float(np.abs(exp).max())
     assert np.isnan(got[:, :, 2 * N:]).all()
+
+
+def _plan(M, N, K, groups, a_spec, b_spec, out_f32=False, ws_bytes=0, dtype="bf16"):
+    rng = np.random.default_rng(0)
+    at = dev_tensor(rounded(rng.standard_normal(a_spec[0]), dtype), dtype)
+    bt = dev_tensor(rounded(rng.standard_normal(b_spec[0]), dtype), dtype)
+    _, ac = _op(at, a_spec[0][2], a_spec[0][1], a_spec[0][0], a_spec[0][2],
+                a_spec[0][1] * a_spec[0][2], **a_spec[1])
+    _, bc = _op(bt, b_spec[0][2], b_spec[0][1], b_spec[0][0], b_spec[0][2],
+                b_spec[0][1] * b_spec[0][2], **b_spec[1])
+    out = torch.empty((groups, M, N), dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
+    ws = torch.empty((max(ws_bytes, 16) // 4,), dtype=torch.float32, device="cuda")
+    d = G.GemmDesc()
+    d.M, d.N, d.K, d.groups, d.k_shards, d.causal = M, N, K, groups, 1, 0
+    d.a, d.b = ac, bc
+    d.out, d.out_f32, d.ldo, d.o_mod, d.o_str_div = out.data_ptr(), int(out_f32), N, 1, M * N
+    if ws_bytes:
+        d.ws, d.ws_bytes = ws.data_ptr(), ws_bytes
+    return G.gemm_plan(d, dtype)
+
+
+def test_pipeline_modes_with_several_tiles_per_sm():
+    """Each way of using an SM's two MMA pipelines (tiles alternating between
+    them, both on one tile's K halves, 256-row tiles split by M) on shapes
+    with more tiles than SMs, so that every CTA walks several tiles; the
+    library reports which way it chose (gptl_gemm_plan) and the cases must
+    cover all three."""
+    need_gpu()
+    cases = [
+        # 256-row tiles: many rows, moderate N and K
+        dict(dtype="bf16", M=8192, N=1280, K=768, groups=1, k_shards=1, causal=0,
+             a_spec=((1, 8192, 768), dict(mn=0)), b_spec=((1, 1280, 768), dict(mn=0)), bias=True),
+        # one 128-row tile per group, many groups: tiles alternate
+        dict(dtype="fp16", M=128, N=256, K=64, groups=400, k_shards=1, causal=0,
+             a_spec=((1, 128, 64), dict(mn=0)), b_spec=((400, 256, 64), dict(mn=0))),
+        # few tiles, long K, no workspace: K halves
+        dict(dtype="bf16", M=256, N=256, K=4096, groups=1, k_shards=1, causal=0,
+             a_spec=((1, 256, 4096), dict(mn=0)), b_spec=((1, 256, 4096), dict(mn=0)), out_f32=True),
+        # weight-gradient shape with a workspace: split-K slices as well
+        dict(dtype="bf16", M=768, N=1024, K=8192, groups=1, k_shards=1, causal=0,
+             a_spec=((1, 8192, 768), dict(mn=1)), b_spec=((1, 8192, 1024), dict(mn=1)),
+             out_f32=True, ws_bytes=8 * 768 * 1024 * 4),
+    ]
+    modes = set()
+    for kw in cases:
+        bn, split, mode = _plan(kw["M"], kw["N"], kw["K"], kw["groups"], kw["a_spec"], kw["b_spec"],
+                                kw.get("out_f32", False), kw.get("ws_bytes", 0), kw["dtype"])
+        modes.add(mode)
+        exp, got, _ = _run(**kw)
+        tol = 5e-5 if kw.get("out_f32") else 8e-3
+        _close(got, exp, tol)
+        # the same plan twice gives the same bits
+        _, got2, _ = _run(**kw)
+        np.testing.assert_array_equal(got, got2)
+    assert modes == {G.GEMM_ALTERNATE, G.GEMM_K_HALVES, G.GEMM_M256}, modes

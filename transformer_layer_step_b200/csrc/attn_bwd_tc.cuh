@@ -23,9 +23,10 @@
 // K-major operand (reduction over head_dim) and, described differently, as
 // an MN-major operand (reduction over the 128 rows).
 //
-// Warp roles (352 threads, one CTA per SM, persistent): warp 0 TMA; warp 1
-// issues the S / dP MMAs and warp 10 the accumulating MMAs (dQ, or dV and
-// dK), one thread each, so the two MMA streams run concurrently; warps 2-9
+// Warp roles (384 threads, one CTA per SM, persistent): warp 0 TMA; warp 1
+// issues the S / dP MMAs, warp 10 the accumulating MMAs (dQ, or dV) and
+// warp 11 those of dK, one thread each, so that the MMA streams run
+// concurrently (warp 11 is idle in the dQ kernel); warps 2-9
 // elementwise work: thread = (row, half of the 128 columns); warp w reads
 // TMEM lane quarter w % 4.
 #pragma once
@@ -35,7 +36,7 @@
 
 namespace gptl {
 
-constexpr int kAttnBwdThreads = 352;   // 11 warps
+constexpr int kAttnBwdThreads = 384;   // 12 warps
 
 struct AttnBwdParams {
   CUtensorMap map_c;     // C as [t*b][s][3h/t]; box {16, 128, 1}, 32B swizzle
@@ -239,6 +240,8 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
       mbar_wait_drain(drain_dq, 0);
     dq_mma_done:;
     }
+  } else if (warp == 11) {
+    // no role in this kernel (the block size is shared with the dK/dV kernel)
   } else {
     // ------------------------------------------- elementwise: one (row, half)
     const int q4 = warp & 3, half = (warp - 2) >> 2;
@@ -373,8 +376,9 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
   const uint32_t sd_full = smem_u32(&bars[10]), sd_empty = smem_u32(&bars[11]);
   const uint32_t pds_full = smem_u32(&bars[12]), pds_free = smem_u32(&bars[13]);
   const uint32_t drain_bar = smem_u32(&bars[14]), drain_acc = smem_u32(&bars[17]);
+  const uint32_t drain_acc2 = smem_u32(&bars[18]);
   auto vec_bar = [&](int i) { return smem_u32(&bars[15 + i]); };   // lse/D staged (256 arrivals)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 19);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -385,14 +389,15 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
     mbar_init(kv_empty, 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(qdo_full(i), 1);
-      mbar_init(qdo_empty(i), 1);
+      mbar_init(qdo_empty(i), 2);   // the dV and the dK issuer
     }
     mbar_init(sd_full, 1);
     mbar_init(sd_empty, 8);
     mbar_init(pds_full, 8);
-    mbar_init(pds_free, 1);
+    mbar_init(pds_free, 2);          // the dV and the dK issuer
     mbar_init(drain_bar, 1);
     mbar_init(drain_acc, 1);
+    mbar_init(drain_acc2, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -488,12 +493,14 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
       mbar_wait_drain(drain_bar, 0);
     mma_done:;
     }
-  } else if (warp == 10) {
+  } else if (warp == 10 || warp == 11) {
     if (lane == 0) {
-      // ---------------------- MMA: dV += P_j^T dO_j, dK += dS_j^T Q_j
-      // A second issuing thread, alongside the S^T / dP^T MMAs.  P^T and dS^T
-      // of block j exist only after its S^T / dP^T MMAs completed, so the
-      // Q / dO stage is free once these MMAs complete.
+      // -------------- MMA: dV += P_j^T dO_j (warp 10), dK += dS_j^T Q_j (warp 11)
+      // Issuing threads of their own, alongside the S^T / dP^T MMAs.  P^T and
+      // dS^T of block j exist only after its S^T / dP^T MMAs completed, so the
+      // Q / dO stage is free once both of these streams complete block j.
+      const bool is_dv = warp == 10;
+      const uint32_t drain = is_dv ? drain_acc : drain_acc2;
       uint32_t q_it = 0, pds_it = 0;
       for (long long item = blockIdx.x; item < p.items; item += gridDim.x) {
         int g, kb;
@@ -508,8 +515,8 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
           const uint32_t q_s = qdo_s + (uint32_t)st * 2u * tb, do_s = q_s + tb;
           for (int k2 = 0; k2 < 8; ++k2) {   // over the 128 queries
             const uint32_t acc = (jj > 0 || k2 > 0) ? 1u : 0u;
-            tc_mma_f16(t_dv, abwd_desc_a(pt_s, k2), abwd_desc_mn(do_s, k2), p.idesc_acc, acc);
-            tc_mma_f16(t_dk, abwd_desc_a(dst_s, k2), abwd_desc_mn(q_s, k2), p.idesc_acc, acc);
+            if (is_dv) tc_mma_f16(t_dv, abwd_desc_a(pt_s, k2), abwd_desc_mn(do_s, k2), p.idesc_acc, acc);
+            else tc_mma_f16(t_dk, abwd_desc_a(dst_s, k2), abwd_desc_mn(q_s, k2), p.idesc_acc, acc);
           }
           tc_commit(pds_free);
           tc_commit(qdo_empty(st));
@@ -518,8 +525,8 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
       }
       goto acc_done;
     acc_abort:
-      tc_commit(drain_acc);
-      mbar_wait_drain(drain_acc, 0);
+      tc_commit(drain);
+      mbar_wait_drain(drain, 0);
     acc_done:;
     }
   } else {

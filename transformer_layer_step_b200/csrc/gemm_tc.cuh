@@ -61,6 +61,7 @@ struct alignas(64) GemmParams {
   int M, N, K, groups, k_shards, causal;
   int split;                   // K slices per tile (split-K); 1 = none
   int pipe_k;                  // 1: both pipelines work on every tile, one K half each
+  int m2;                      // 1: 256-row tiles, one M half per pipeline, one shared ring
   float *ws;                   // split-K partials [split][groups][M][N] fp32
   long long ws_slice;          // groups * M * N
   int bn, bn_alloc, stages, tmem_cols;
@@ -95,7 +96,7 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams &p, long long idx
   t.g = (int)(tile / tpg);
   const int rem = (int)(tile - (long long)t.g * tpg);
   const int mt = rem / p.n_tiles, nt = rem - (rem / p.n_tiles) * p.n_tiles;
-  t.m0 = mt * kBM;
+  t.m0 = mt * (p.m2 ? 2 * kBM : kBM);
   t.n0 = nt * p.bn;
   t.skip = (p.causal == kCausalSkipUpper) && (t.n0 > t.m0 + kBM - 1);
   t.kb_begin = 0;
@@ -295,7 +296,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow
 // other pipeline's MMAs to overlap with.
 // Does pipeline pp take local tile t, and which of its k-blocks?
 __device__ __forceinline__ bool pipe_takes(const GemmParams &p, int t, int pp) {
-  return p.pipe_k ? true : ((t & 1) == pp);
+  return (p.pipe_k || p.m2) ? true : ((t & 1) == pp);
 }
 __device__ __forceinline__ void pipe_kb_range(const GemmParams &p, const TileInfo &ti, int pp,
                                               int &kb0, int &kb1) {
@@ -313,12 +314,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  const int a_bytes = kBM * kBK * 2;
+  const int a_rows = p.m2 ? 2 * kBM : kBM;
+  const int a_bytes = a_rows * kBK * 2;
   const int b_bytes = p.bn * kBK * 2;
   const int stage_bytes = a_bytes + b_bytes;
-  const int S = p.stages;                                   // stages per pipeline
-  const uint32_t staging_s = smem_u32(smem + 2 * S * stage_bytes);   // 1024-aligned
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * S * stage_bytes + kStagingBytes);
+  const int S = p.stages;                                   // stages per ring
+  const int rings = p.m2 ? 1 : 2;                           // m2: one ring both pipelines read
+  const uint32_t staging_s = smem_u32(smem + rings * S * stage_bytes);   // 1024-aligned
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + rings * S * stage_bytes + kStagingBytes);
   // bars: full[pipe][S] empty[pipe][S] tfull[2] tempty[2] drain[2]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 6);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     for (int pp = 0; pp < 2; ++pp) {
       for (int s = 0; s < S; ++s) {
         mbar_init(full_bar(pp, s), 1);
-        mbar_init(empty_bar(pp, s), 1);
+        mbar_init(empty_bar(pp, s), p.m2 ? 2 : 1);   // m2: both MMA warps release a stage
       }
       mbar_init(tfull_bar(pp), 1);
       mbar_init(tempty_bar(pp), kEpiWarps);
@@ -361,7 +364,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
 
   if (warp < 4) {
     const int pp = warp >> 1;                 // pipeline of this warp
-    if (lane == 0 && (warp & 1) == 0) {
+    const bool producer_warp = (warp & 1) == 0;
+    // m2: the one shared ring is filled by pipeline 0's producer alone
+    if (lane == 0 && producer_warp && !(p.m2 && pp == 1)) {
       // ------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0, issued = 0, parity = 0;
@@ -378,7 +383,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
             const uint32_t fb = full_bar(pp, stage);
             mbar_arrive_expect_tx(fb, (uint32_t)stage_bytes);
             const uint32_t sa = stage_addr(pp, stage);
-            load_operand(&p.map_a, p.ra, sa, kBM, ti.g, ks, ti.m0, kb * kBK, fb);
+            load_operand(&p.map_a, p.ra, sa, a_rows, ti.g, ks, ti.m0, kb * kBK, fb);
             load_operand(&p.map_b, p.rb, sa + a_bytes, p.bn, ti.g, ks, ti.n0, kb * kBK, fb);
             issued |= 1u << stage;
             parity = (parity & ~(1u << stage)) | (phase << stage);
@@ -394,12 +399,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       for (int s = 0; s < S; ++s)
         if (issued & (1u << s)) mbar_wait_drain(full_bar(pp, s), (parity >> s) & 1u);
     producer_done:;
-    } else if (lane == 0) {
+    } else if (lane == 0 && !producer_warp) {
       // ------------------------------------------------ MMA issuer
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       int t = 0;
       const uint32_t d_tmem = tmem_base + (uint32_t)(pp * p.bn_alloc);
+      const int ring = p.m2 ? 0 : pp;
       for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
         const TileInfo ti = tile_info(p, idx);
         if (ti.skip) continue;
@@ -411,15 +417,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         int it = 0;
         for (int ks = 0; ks < p.k_shards; ++ks)
           for (int kb = kb0; kb < kb1; ++kb) {
-            if (!mbar_wait(full_bar(pp, stage), phase, abort_flag)) goto mma_abort;
+            if (!mbar_wait(full_bar(ring, stage), phase, abort_flag)) goto mma_abort;
             tc_fence_after();
-            const uint32_t sa = stage_addr(pp, stage);
-            const uint32_t sb = sa + (uint32_t)a_bytes;
+            // m2: this pipeline's 128 rows of the 256-row A tile (K-major rows,
+            // or MN-major column chunks: 16 KB into the tile either way)
+            const uint32_t sa = stage_addr(ring, stage) + (p.m2 ? (uint32_t)(pp * kBM * kBK * 2) : 0u);
+            const uint32_t sb = stage_addr(ring, stage) + (uint32_t)a_bytes;
             const int nsteps = min(kBK, p.K - kb * kBK) / 16;
             for (int s = 0; s < nsteps; ++s)
               tc_mma_f16(d_tmem, operand_desc(p.ra, sa, s), operand_desc(p.rb, sb, s), p.idesc,
                          (it > 0 || s > 0) ? 1u : 0u);
-            tc_commit(empty_bar(pp, stage));
+            tc_commit(empty_bar(ring, stage));
             ++it;
             if (++stage == S) {
               stage = 0;
@@ -449,17 +457,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
       const TileInfo ti = tile_info(p, idx);
       if (ti.skip) continue;
-      const int pp = p.pipe_k ? 0 : (t & 1);   // accumulator (with pipe_k: the first of two)
+      // accumulator of this tile; with pipe_k or m2 both are (pp = 0 and 1)
+      const bool both = p.pipe_k || p.m2;
+      const int pp = both ? 0 : (t & 1);
       ++t;
       bool got = mbar_wait(tfull_bar(pp), acc_phase[pp], abort_flag);
-      if (got && p.pipe_k) got = mbar_wait(tfull_bar(1), acc_phase[1], abort_flag);
+      if (got && both) got = mbar_wait(tfull_bar(1), acc_phase[1], abort_flag);
       if (!got) break;
       acc_phase[pp] ^= 1;
-      if (p.pipe_k) acc_phase[1] ^= 1;
+      if (both) acc_phase[1] ^= 1;
       tc_fence_after();
-      const int row0 = ti.m0 + q * 32;
+      for (int hf = 0; hf < (p.m2 ? 2 : 1); ++hf) {   // m2: the tile's two 128-row halves
+      const int row0 = ti.m0 + hf * kBM + q * 32;
       const EpiRow er = epilogue_row<T>(p, ti.g, row0 + lane);
-      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(pp * p.bn_alloc);
+      const uint32_t t_row =
+          tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((pp + hf) * p.bn_alloc);
       // output map coordinates of this tile's group
       int oz, ow;
       if (p.split > 1) { oz = ti.slice * p.groups + ti.g; ow = 0; }
@@ -538,11 +550,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         tmem_wait_ld();
         if (has_a) sum2(c + 2, ra);
       }
+      }   // halves
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(tempty_bar(pp));
-        if (p.pipe_k) mbar_arrive(tempty_bar(1));
+        if (both) mbar_arrive(tempty_bar(1));
       }
     }
     // the staged boxes must be read, and the stores done, before the CTA exits

@@ -246,44 +246,59 @@ int pick_bn(const gptl_gemm_desc &d, int sms) {
 }
 
 // Tiling of one GEMM call: BN, split-K slices (fp32 output with a workspace
-// only) and whether the CTA's two pipelines share each tile as K halves.
-// Chosen by a time estimate in microseconds.  A k-block through one pipeline
-// costs about the same for BN = 128 and 256 (the MMA-issuing thread, not the
-// tensor core, sets the pace: measured on B200), ~0.55 us.
-//   tiles alternating between the pipelines: ceil(ceil(items / SMs) / 2) x kb
-//   both pipelines on every tile:            ceil(items / SMs) x ceil(kb / 2)
-// where items = tiles x split and kb = k-blocks of one item; split > 1 adds
-// the partial-sum pass, (2 split + 1) fp32 arrays at ~4 TB/s plus a launch.
+// only) and the use of the CTA's two pipelines, chosen by a time estimate in
+// microseconds.  Per-k-block times measured on B200 (BN = 256; a k-block is
+// 64 deep), with both pipelines of an SM busy unless noted:
+//   alternate   tiles alternate between the pipelines, 128 x BN tiles:
+//               1.17 per k-block of each pipeline (0.9 when one runs alone);
+//               one tile's epilogue overlaps the other pipeline's MMAs
+//   K halves    both pipelines on one 128 x BN tile: 1.17 per k-block of each
+//   m2          256 x BN tiles, one M half per pipeline, one shared ring:
+//               ~1.0 per k-block of the pair (a third less operand traffic
+//               from L2 per FLOP than 128 x BN tiles)
+// The last two cannot overlap a tile's epilogue with the next tile's MMAs
+// (all 512 TMEM columns hold the tile): ~1.3 us per 128 x 256 half tile,
+// ~5 with GeLU / GeLU' (measured: the 256-row mode loses to alternating
+// tiles on the GeLU GEMMs, wins on the others).  Split-K adds the partial-sum
+// pass, (2 split + 1) fp32 arrays at ~4 TB/s plus a launch.
 struct GemmTiling {
-  int bn, split, pipe_k;
+  int bn, split, pipe_k, m2;
 };
 GemmTiling choose_tiling(const gptl_gemm_desc &d, int sms, bool can_split) {
-  GemmTiling best{pick_bn(d, sms), 1, 0};
+  GemmTiling best{pick_bn(d, sms), 1, 0, 0};
   if (d.causal != GPTL_CAUSAL_NONE) return best;
-  const double t_kb = 0.55;
-  const long long m_tiles = (d.M + kBM - 1) / kBM;
   const long long kb_all = (long long)((d.K + kBK - 1) / kBK) * d.k_shards;
   const double out_bytes = (double)d.groups * d.M * d.N * 4.0;
+  const double e_half = (d.act == GPTL_ACT_NONE ? 1.3 : 5.0);
   double best_t = -1.0;
   const int n_bn = d.N <= 256 ? 1 : 2;
   for (int ib = 0; ib < n_bn; ++ib) {
     const int bn = d.N <= 256 ? d.N : (ib == 0 ? 256 : 128);
-    const long long tiles = m_tiles * ((d.N + bn - 1) / bn) * d.groups;
-    for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
-      if (sp > (d.K + kBK - 1) / kBK) break;
-      if (sp > 1 && (double)sp * out_bytes > (double)d.ws_bytes) break;
-      const long long items = tiles * sp;
-      const long long kb = (kb_all + sp - 1) / sp;
-      const long long per_cta = (items + sms - 1) / sms;
-      for (int pk = 0; pk < 2; ++pk) {
-        // every slice must give each pipeline at least one k-block
-        if (pk && ((d.K + kBK - 1) / kBK) / sp < 2) continue;
-        double t = pk ? (double)per_cta * ((kb + 1) / 2) * t_kb
-                      : (double)((per_cta + 1) / 2) * kb * t_kb;
+    const double e_tile = e_half * bn / 256.0;
+    const long long n_tiles = (d.N + bn - 1) / bn;
+    for (int mode = 0; mode < 3; ++mode) {          // alternate, K halves, m2
+      if (mode == 2 && d.M <= kBM) continue;
+      const long long m_tiles = (d.M + (mode == 2 ? 2 * kBM : kBM) - 1) / (mode == 2 ? 2 * kBM : kBM);
+      const long long tiles = m_tiles * n_tiles * d.groups;
+      for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
+        if (sp > (d.K + kBK - 1) / kBK) break;
+        if (sp > 1 && (double)sp * out_bytes > (double)d.ws_bytes) break;
+        // K halves: every slice must give each pipeline at least one k-block
+        if (mode == 1 && ((d.K + kBK - 1) / kBK) / sp < 2) continue;
+        const long long items = tiles * sp;
+        const long long kb = (kb_all + sp - 1) / sp;
+        const long long per_cta = (items + sms - 1) / sms;
+        double t;
+        if (mode == 0)
+          t = per_cta >= 2 ? (double)((per_cta + 1) / 2) * kb * 1.17 + e_tile : kb * 0.9 + e_tile;
+        else if (mode == 1)
+          t = (double)per_cta * ((kb + 1) / 2 * 1.17 + e_tile);
+        else
+          t = (double)per_cta * (kb * 1.0 + 2.0 * e_tile);
         if (sp > 1) t += (2.0 * sp + 1.0) * out_bytes / 4.0e6 + 3.0;
         if (best_t < 0 || t < best_t * 0.999) {
           best_t = t;
-          best = GemmTiling{bn, sp, pk};
+          best = GemmTiling{bn, sp, mode == 1 ? 1 : 0, mode == 2 ? 1 : 0};
         }
       }
     }
@@ -307,9 +322,8 @@ int launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) 
   return GPTL_OK;
 }
 
-int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
-  int sms = 0;
-  GPTL_TRY(device_check(&sms));
+// Argument checks of gptl_gemm (no device work).
+int gemm_validate(const gptl_gemm_desc &d, gptl_dtype dt) {
   if (dt != GPTL_FP16 && dt != GPTL_BF16) return GPTL_E_DTYPE;
   if (!d.out) return GPTL_E_NULL;
   if (!aligned16(d.out)) return GPTL_E_ALIGN;
@@ -326,16 +340,27 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   if (d.resid && d.act == GPTL_ACT_DGELU) return GPTL_E_SHAPE;   // one epilogue input per GEMM
   GPTL_TRY(check_operand(d.a));
   GPTL_TRY(check_operand(d.b));
+  return GPTL_OK;
+}
 
-  GemmParams p;
-  memset(&p, 0, sizeof(p));
+GemmTiling gemm_plan(const gptl_gemm_desc &d, int sms) {
   const bool can_split = d.out_f32 && !d.bias && !d.resid && d.act == GPTL_ACT_NONE &&
                          d.causal == GPTL_CAUSAL_NONE && d.ws && aligned16(d.ws);
-  const GemmTiling tl = choose_tiling(d, sms, can_split);
+  return choose_tiling(d, sms, can_split);
+}
+
+int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
+  int sms = 0;
+  GPTL_TRY(device_check(&sms));
+  GPTL_TRY(gemm_validate(d, dt));
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  const GemmTiling tl = gemm_plan(d, sms);
   const int bn = tl.bn;
   const int wa = d.a.mn_major ? mn_chunk_width(kBM) : 64;
   const int wb = d.b.mn_major ? mn_chunk_width(bn) : 64;
-  GPTL_TRY(encode_operand(&p.map_a, d.a, dt, kBM, wa));
+  const int a_rows = tl.m2 ? 2 * kBM : kBM;   // rows of A per tile
+  GPTL_TRY(encode_operand(&p.map_a, d.a, dt, a_rows, wa));
   GPTL_TRY(encode_operand(&p.map_b, d.b, dt, bn, wb));
   auto rule = [](const gptl_operand &o, int w) {
     OperandRule r;
@@ -361,21 +386,23 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   while (bn_alloc < bn) bn_alloc *= 2;
   p.bn_alloc = bn_alloc;
   p.tmem_cols = 2 * bn_alloc;
-  const int stage_bytes = (kBM + bn) * kBK * 2;
-  // stages per pipeline; the kernel runs two pipelines with a ring each
-  p.stages = (kSmemLimit - 2048 - kStagingBytes) / (2 * stage_bytes);
+  const int stage_bytes = (a_rows + bn) * kBK * 2;
+  // stages per ring: two rings (one per pipeline), or one shared ring in m2
+  const int rings = tl.m2 ? 1 : 2;
+  p.stages = (kSmemLimit - 2048 - kStagingBytes) / (rings * stage_bytes);
   if (p.stages > 4) p.stages = 4;
   if (p.stages < 2) return GPTL_E_SHAPE;
-  const int smem = 1024 + 2 * p.stages * stage_bytes + kStagingBytes + 512;
+  const int smem = 1024 + rings * p.stages * stage_bytes + kStagingBytes + 512;
   const uint32_t fmt = dt == GPTL_BF16 ? 1u : 0u;
   p.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)d.a.mn_major << 15) |
             ((uint32_t)d.b.mn_major << 16) | ((uint32_t)(bn >> 3) << 17) |
             ((uint32_t)(kBM >> 4) << 24);
-  p.m_tiles = (d.M + kBM - 1) / kBM;
+  p.m_tiles = (d.M + a_rows - 1) / a_rows;
   p.n_tiles = (d.N + bn - 1) / bn;
   const long long tiles = (long long)p.m_tiles * p.n_tiles * d.groups;
   p.split = tl.split;
   p.pipe_k = tl.pipe_k;
+  p.m2 = tl.m2;
   p.ws = static_cast<float *>(d.ws);
   p.ws_slice = (long long)d.groups * d.M * d.N;
   p.total_tiles = tiles * p.split;
@@ -1393,6 +1420,18 @@ int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream) {
   if (!d) return GPTL_E_NULL;
   prof_start(reinterpret_cast<cudaStream_t>(stream));
   return run_gemm(*d, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gptl_gemm_plan(const gptl_gemm_desc *d, gptl_dtype dtype, int *bn, int *split, int *mode) {
+  if (!d || !bn || !split || !mode) return GPTL_E_NULL;
+  int sms = 0;
+  GPTL_TRY(device_check(&sms));
+  GPTL_TRY(gemm_validate(*d, dtype));
+  const GemmTiling tl = gemm_plan(*d, sms);
+  *bn = tl.bn;
+  *split = tl.split;
+  *mode = tl.m2 ? GPTL_GEMM_M256 : (tl.pipe_k ? GPTL_GEMM_K_HALVES : GPTL_GEMM_ALTERNATE);
+  return GPTL_OK;
 }
 
 int gptl_layernorm_fwd(int rows, int h, gptl_dtype dtype, const void *x, const void *g,

@@ -96,6 +96,8 @@ _SIGS = {
                                     C.c_void_p]),
     "gptl_check_overflow": (C.c_int, [C.c_size_t, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gptl_gemm": (C.c_int, [C.POINTER(GemmDesc), C.c_int, C.c_void_p]),
+    "gptl_gemm_plan": (C.c_int, [C.POINTER(GemmDesc), C.c_int, C.POINTER(C.c_int),
+                                 C.POINTER(C.c_int), C.POINTER(C.c_int)]),
     "gptl_layernorm_fwd": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
                                      C.c_void_p, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_void_p]),
@@ -229,6 +231,17 @@ def operand(t, x_ext, rows_ext, g_ext, row_pitch, g_pitch=0, mn_major=0, x_mod=1
 
 def gemm(desc: GemmDesc, dtype, stream=0):
     _check(lib().gptl_gemm(C.byref(desc), DTYPES.get(dtype, dtype), stream), "gptl_gemm")
+
+
+GEMM_ALTERNATE, GEMM_K_HALVES, GEMM_M256 = 0, 1, 2
+
+
+def gemm_plan(desc: GemmDesc, dtype) -> tuple:
+    """(bn, split, mode) that gptl_gemm would use for desc on this device."""
+    bn, split, mode = C.c_int(), C.c_int(), C.c_int()
+    _check(lib().gptl_gemm_plan(C.byref(desc), DTYPES.get(dtype, dtype), C.byref(bn),
+                                C.byref(split), C.byref(mode)), "gptl_gemm_plan")
+    return bn.value, split.value, mode.value
 
 
 def layernorm_fwd(rows, h, dtype, x, g, b, eps, y, mu, rstd, stream=0):
