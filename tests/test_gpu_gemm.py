@@ -346,9 +346,9 @@ def test_pipeline_modes_with_several_tiles_per_sm():
     cover all three."""
     need_gpu()
     cases = [
-        # 256-row tiles: many rows, moderate N and K
-        dict(dtype="bf16", M=8192, N=1280, K=768, groups=1, k_shards=1, causal=0,
-             a_spec=((1, 8192, 768), dict(mn=0)), b_spec=((1, 1280, 768), dict(mn=0)), bias=True),
+        # the attention-input projection's shape: 256-row tiles, ~2 per SM
+        dict(dtype="bf16", M=8192, N=2304, K=768, groups=1, k_shards=1, causal=0,
+             a_spec=((1, 8192, 768), dict(mn=0)), b_spec=((1, 2304, 768), dict(mn=0)), bias=True),
         # one 128-row tile per group, many groups: tiles alternate
         dict(dtype="fp16", M=128, N=256, K=64, groups=400, k_shards=1, causal=0,
              a_spec=((1, 128, 64), dict(mn=0)), b_spec=((400, 256, 64), dict(mn=0))),

@@ -119,33 +119,43 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const TX *__restrict__ x,
 // gy*xhat (dgamma), gy (dbeta), then dx if SUM_DX (the fp32 value with D32,
 // else the stored 16-bit value), then resid if SUM_RESID.
 // reduce_parts_kernel finishes them.
+// Each row team keeps its running column sums in its own shared-memory
+// rows ([team][part][h]; a thread only touches its own columns), so the
+// registers stay low enough for two blocks per SM; the teams are added in a
+// fixed order at the end.
 template <typename T, typename TX, typename TR, bool D32, bool SUM_DX, bool SUM_RESID, int VPT>
-__global__ void __launch_bounds__(256) ln_bwd_kernel(
+__global__ void __launch_bounds__(256, VPT <= 3 ? 2 : 1) ln_bwd_kernel(
     const T *__restrict__ gy, const TX *__restrict__ x, const float *__restrict__ mu_in,
     const float *__restrict__ rstd_in, const T *__restrict__ gamma, const TR *__restrict__ resid,
     T *__restrict__ dx, float *__restrict__ dx32, float *__restrict__ part, int rows, int h,
     int tpr) {
-  extern __shared__ float sm[];          // [RPB][h] staging for the column partials
+  constexpr int nparts = 2 + (SUM_DX ? 1 : 0) + (SUM_RESID ? 1 : 0);
+  extern __shared__ float sm[];          // [RPB][nparts][h] running column sums
   __shared__ float red[256 / 32 + 8];
   const int TPR = tpr;
   const int RPB = blockDim.x / tpr;
   const int team = threadIdx.x / TPR, tl = threadIdx.x % TPR;
-  float pg[VPT][8], pb[VPT][8], pd[SUM_DX ? VPT : 1][8], pr[SUM_RESID ? VPT : 1][8];
+  float *acc = sm + (size_t)team * nparts * h;
   float gm[VPT][8];
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(gamma) + tl + i * TPR), gm[i]);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) pg[i][e] = pb[i][e] = 0.f;
+    for (int k = 0; k < nparts; ++k) {
+      float4 *a4 = reinterpret_cast<float4 *>(acc + k * h + (tl + i * TPR) * 8);
+      a4[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      a4[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
-#pragma unroll
-  for (int i = 0; i < (SUM_DX ? VPT : 1); ++i)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) pd[i][e] = 0.f;
-#pragma unroll
-  for (int i = 0; i < (SUM_RESID ? VPT : 1); ++i)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) pr[i][e] = 0.f;
+  // adds v[8] into the running sums of part k, columns (tl + i*TPR)*8 ..
+  auto add8 = [&](int k, int i, const float (&v)[8]) {
+    float4 *a4 = reinterpret_cast<float4 *>(acc + k * h + (tl + i * TPR) * 8);
+    float4 s0 = a4[0], s1 = a4[1];
+    s0.x += v[0]; s0.y += v[1]; s0.z += v[2]; s0.w += v[3];
+    s1.x += v[4]; s1.y += v[5]; s1.z += v[6]; s1.w += v[7];
+    a4[0] = s0;
+    a4[1] = s1;
+  };
   const int row_step = gridDim.x * RPB;
   // every team runs the same number of iterations (the team reductions
   // synchronise the whole block when TPR > 32)
@@ -186,11 +196,11 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(
         const uint4 q = pack8<T>(o);
         dr[tl + i * TPR] = q;
         if constexpr (D32) store_vec8_f32(dx32 + (long long)r * h, tl + i * TPR, o);
+        float gx[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pg[i][e] += g[i][e] * xh[i][e];
-          pb[i][e] += g[i][e];
-        }
+        for (int e = 0; e < 8; ++e) gx[e] = g[i][e] * xh[i][e];
+        add8(0, i, gx);
+        add8(1, i, g[i]);
         if constexpr (SUM_DX) {
           float oq[8];
           if constexpr (D32) {
@@ -199,38 +209,20 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(
           } else {
             unpack8<T>(q, oq);             // sum what was stored
           }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) pd[i][e] += oq[e];
+          add8(2, i, oq);
         }
-        if constexpr (SUM_RESID) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) pr[i][e] += rv[e];
-        }
+        if constexpr (SUM_RESID) add8(SUM_DX ? 3 : 2, i, rv);
       }
     }
   }
-  // combine the RPB teams of this block, one partial array at a time
-  constexpr int nparts = 2 + (SUM_DX ? 1 : 0) + (SUM_RESID ? 1 : 0);
+  // combine the RPB teams of this block in team order, one part at a time
+  __syncthreads();
 #pragma unroll
   for (int k = 0; k < nparts; ++k) {
-    const int which = k < 2 ? k : (k == 2 && SUM_DX ? 2 : 3);
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < VPT; ++i)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float val;
-        if (which == 0) val = pg[i][e];
-        else if (which == 1) val = pb[i][e];
-        else if (which == 2) val = pd[SUM_DX ? i : 0][e];
-        else val = pr[SUM_RESID ? i : 0][e];
-        sm[team * h + (tl + i * TPR) * 8 + e] = val;
-      }
-    __syncthreads();
     float *dst = part + ((long long)k * gridDim.x + blockIdx.x) * h;
     for (int c = threadIdx.x; c < h; c += blockDim.x) {
       float s = 0.f;
-      for (int t = 0; t < RPB; ++t) s += sm[t * h + c];
+      for (int t = 0; t < RPB; ++t) s += sm[((size_t)t * nparts + k) * h + c];
       dst[c] = s;
     }
   }

@@ -766,12 +766,13 @@ int run_ln_bwd(int variant, int rows, int h, gptl_dtype dt, const void *gy, cons
   int tpr = 0, vpt = 0;
   if (!ln_split(h, &tpr, &vpt) || rows <= 0) return GPTL_E_SHAPE;
   const int nb = ln_bwd_blocks(rows, h, sms);
-  const int smem = (256 / tpr) * h * (int)sizeof(float);
+  const int nparts = variant == LNB_H ? 4 : (variant == LNB_X ? 2 : (dx_sum ? 3 : 2));
+  const int smem = (256 / tpr) * nparts * h * (int)sizeof(float);   // per-team running sums
   int rc = GPTL_OK;
   const bool ok = ln_dispatch(vpt, [&]<int VP>() {
     auto go = [&]<typename T, typename TX, typename TR, bool D32, bool SDX, bool SRS>() {
       auto kern = ln_bwd_kernel<T, TX, TR, D32, SDX, SRS, VP>;
-      if (smem > 48 * 1024 &&
+      if (smem > 40 * 1024 &&   // the opt-in also covers the kernel's static shared memory
           cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
               cudaSuccess) {
         (void)cudaGetLastError();
