@@ -52,6 +52,8 @@ DEFAULT_WORKLOAD = "gpt2-117m"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = ("transformer_layer_step_b200/csrc/gemm_tc.cuh",
+                  "transformer_layer_step_b200/csrc/attn_tc.cuh",
+                  "transformer_layer_step_b200/csrc/attn_bwd_tc.cuh",
                   "transformer_layer_step_b200/csrc/common.cuh",
                   "transformer_layer_step_b200/csrc/bw_kernels.cuh",
                   "transformer_layer_step_b200/csrc/gptlayer.cu")
@@ -290,16 +292,34 @@ def run_ours(args, cfg, rank, world, local_rank):
     if G.read_device_error(clear=True):
         raise RuntimeError("device error word set during warm-up")
 
+    # ---- the step as a CUDA graph (captured after the warm-up, which set the
+    # kernels' shared-memory opt-ins): one launch of the graph per step, so no
+    # host launch latency between the step's kernels
+    step_fn = ls.step
+    graph = None
+    graph_launches = 0
+    if not args.no_graph:
+        n0 = G.launch_count()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            ls.step()
+        graph_launches = G.launch_count() - n0
+        for _ in range(2):
+            graph.replay()
+            flush.zero_()
+        torch.cuda.synchronize()
+        step_fn = graph.replay
+
     # ---- value: inputs resident in HBM
     sampler = ClockSampler(local_rank)
     sampler.start()
     barrier()
     torch.cuda.synchronize()
     launches0 = G.launch_count()
-    ev = timed_steps(K, ls.step)
+    ev = timed_steps(K, step_fn)
     torch.cuda.synchronize()
     barrier()
-    launches = G.launch_count() - launches0
+    launches = G.launch_count() - launches0 + graph_launches * K
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = max_over_ranks(sum(step_ms))
@@ -410,6 +430,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.CONFIGS))
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the step's kernels one by one instead of as a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the CPU oracle timing (it runs on rank 0 at N=1 only)")
     args = ap.parse_args()
@@ -422,6 +444,7 @@ def main():
     config = {"workload": cfg.name, "batch": cfg.batch, "seq_len": cfg.seq,
               "hidden": cfg.hidden, "heads": cfg.heads, "ffn": cfg.ffn, "tp": cfg.tp,
               "tokens_per_step": cfg.tokens, "parallelism": f"replicas{world}",
+              "step_launch": "kernel by kernel" if args.no_graph else "one CUDA graph per step",
               "l2": "flushed between steps (256 MiB write, outside the per-step events)"}
     flops = step_flops(cfg)
 
@@ -492,7 +515,7 @@ def main():
         "scaler_after": res["scaler"],
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        r = oracle_sample(cfg, 2)
+        r = oracle_sample(cfg, 4)          # about 10 s of float64 CPU work
         line["cpu_baseline"] = {"value": round(r["value"], 3), "unit": UNIT,
                                 "cores": blas_threads(), "kind": "oracle",
                                 "sample": r["sample"], "seconds": round(sum(r["seconds"]), 2)}

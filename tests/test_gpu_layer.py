@@ -138,3 +138,35 @@ def test_repeat_is_bitwise_deterministic():
     ls.fwd(); ls.bwd()
     torch.cuda.synchronize()
     assert torch.equal(y1, ls.y) and torch.equal(dx1, ls.dx) and torch.equal(g1, ls.grad)
+
+
+def test_cuda_graph_of_the_step_matches_eager_launches():
+    """The whole step (fwd, bwd, overflow check, Adam, scale update) captured
+    as one CUDA graph and replayed gives bit-identical outputs, gradients,
+    weights and scaler state to launching it kernel by kernel (the library
+    makes no host synchronisation or allocation inside a step)."""
+    need_gpu()
+    cfg = synth.CONFIGS["gpt2-117m"]
+    inp = synth.make_inputs(cfg, variant="biased", with_r=True)
+
+    def fresh():
+        ls = LayerStep(cfg, inp)
+        ls.set_dy_bits(synth.loss_grad_bits(cfg, ls.hyper["init_scale"], inp["r"]))
+        return ls
+
+    eager = fresh()
+    for _ in range(2):
+        eager.step()
+    torch.cuda.synchronize()
+
+    graphed = fresh()
+    graphed.step()                          # eager first step: shared-memory opt-ins are set
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        graphed.step()                      # captured, not run
+    g.replay()
+    torch.cuda.synchronize()
+    check_device_error()
+    for name in ("y", "dx", "grad", "master", "m", "v", "w16", "state"):
+        assert torch.equal(getattr(eager, name), getattr(graphed, name)), name
