@@ -543,19 +543,30 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
       const int n = p.tiles - kb;
       const int key = kb * 128 + row;
       bool ok = true;
+      // -lse and -D/sqrt(d) of one query block, for threads tid < 128
+      auto vec_load = [&](int jq, float &a, float &b2) {
+        const int q = jq * 128 + tid;
+        a = q < p.s ? -p.lse[(long long)g * p.s + q] : 0.f;
+        b2 = q < p.s ? -p.scale * p.dvec[(long long)g * p.s + q] : 0.f;
+      };
+      // Block j's vectors are staged in vecs[blk & 1] (double-buffered) and
+      // published by vec_bar[blk & 1]: the first block's at the item start,
+      // every later block's at the end of the block before it, from loads
+      // issued at that block's start (their latency hides behind its work).
+      // A thread passes block blk's barrier only after every thread has
+      // finished block blk - 1, so the buffer rewritten at the end of block
+      // blk (last read in block blk - 1) is free.
+      float nl_next = 0.f, nd_next = 0.f;
+      if (tid < 128) {
+        vec_load(kb, nl_next, nd_next);
+        vecs[(blk & 1u) * 256u + tid] = nl_next;
+        vecs[(blk & 1u) * 256u + 128u + tid] = nd_next;
+      }
+      mbar_arrive(vec_bar((int)(blk & 1u)));
       for (int jj = 0; jj < n; ++jj, ++blk) {
         const int j = kb + jj;
-        // stage this query block's lse and D (double-buffered).  The bounded
-        // barrier on vec_bar also ends every thread's reads of the buffer
-        // used two blocks ago: a thread passes block blk+1's barrier only
-        // after all threads have finished block blk.
         float *vb = vecs + (blk & 1u) * 256u;
-        if (tid < 128) {   // -lse and -D/sqrt(d) of the block's queries
-          const int q = j * 128 + tid;
-          vb[tid] = q < p.s ? -p.lse[(long long)g * p.s + q] : 0.f;
-          vb[128 + tid] = q < p.s ? -p.scale * p.dvec[(long long)g * p.s + q] : 0.f;
-        }
-        mbar_arrive(vec_bar((int)(blk & 1u)));
+        if (tid < 128 && jj + 1 < n) vec_load(j + 1, nl_next, nd_next);
         if (!mbar_wait(vec_bar((int)(blk & 1u)), (blk >> 1) & 1u, abort_flag)) { ok = false; break; }
         if (!mbar_wait(sd_full, sd_it & 1u, abort_flag)) { ok = false; break; }
         ++sd_it;
@@ -630,6 +641,13 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(pds_full);
+        if (jj + 1 < n) {             // publish the next block's vectors
+          if (tid < 128) {
+            vecs[((blk + 1) & 1u) * 256u + tid] = nl_next;
+            vecs[((blk + 1) & 1u) * 256u + 128u + tid] = nd_next;
+          }
+          mbar_arrive(vec_bar((int)((blk + 1) & 1u)));
+        }
       }
       if (!ok) break;
       if (!mbar_wait(pds_free, pds_it & 1u, abort_flag)) break;
