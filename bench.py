@@ -348,21 +348,6 @@ def run_ours(args, cfg, rank, world, local_rank):
     yb = [torch.empty_like(ls.y) for _ in range(2)]
     stb = [torch.empty_like(ls.state) for _ in range(2)]   # per-step snapshot of the scaler
     copy_stream = torch.cuda.Stream(dev)
-    # the step on each buffer set, as a CUDA graph like the value's steps
-    e2e_step = [lambda b=b: ls.step(x=xb[b], dy=dyb[b], y=yb[b]) for b in range(2)]
-    if not args.no_graph:
-        e2e_graphs = []
-        for b in range(2):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                e2e_step[b]()
-            e2e_graphs.append(g)
-        e2e_step = [g.replay for g in e2e_graphs]
-        for b in range(2):                      # first replays upload the graphs
-            xb[b].copy_(ls.x)
-            dyb[b].copy_(ls.dy)
-            e2e_step[b]()
-        torch.cuda.synchronize()
     copied = [torch.cuda.Event() for _ in range(2)]
     computed = [torch.cuda.Event() for _ in range(2)]
     read_back = [torch.cuda.Event() for _ in range(2)]
@@ -387,7 +372,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         stream.wait_event(copied[b])
         if i >= 2:
             stream.wait_event(read_back[b])              # y buffer b read back (step i-2)
-        e2e_step[b]()
+        ls.step(x=xb[b], dy=dyb[b], y=yb[b])
         stb[b].copy_(ls.state, non_blocking=True)
         computed[b].record(stream)
         if i + 1 < K:

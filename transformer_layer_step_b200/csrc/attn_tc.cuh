@@ -18,10 +18,12 @@
 //              threads, so that the two MMA streams run concurrently);
 //   warps 2-5  one query row per thread: read S_j from tensor memory, update
 //              the running max m and sum l, rescale O by exp2(m_old - m_new)
-//              in tensor memory when m moved, write P_j (16-bit) to shared
-//              memory; at the end normalise O by 1/l and store it.
+//              in tensor memory when m moved, write P_j (16-bit) to one of
+//              two shared-memory buffers (so that P_j is formed while
+//              P_{j-1} V_{j-1} runs); at the end normalise O by 1/l and
+//              store it.
 // Tensor memory: S buffers at columns 0 and 128, O at column 256.
-// Shared memory: P [128 x 128] (two 128B-swizzled 64-column atoms), Q as
+// Shared memory: two P buffers [128 x 128] (two 128B-swizzled 64-column atoms each), Q as
 // head_dim/16 chunks of [128 rows x 16] (32B swizzle), and per stage K the
 // same way and V as MN-major chunks of [64 keys x vw].
 #pragma once
@@ -63,20 +65,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   const uint32_t chunk_bytes = 128u * 32u;                   // one 16-column chunk, 128 rows
   const uint32_t q_bytes = (uint32_t)(d / 16) * chunk_bytes;  // = 128 * d * 2
   const uint32_t kv_bytes = 2u * q_bytes;                     // K and V of one stage
-  const uint32_t p_s = smem_u32(smem);                        // P: 32 KB
-  const uint32_t q_s = p_s + 32768u;
+  const uint32_t p_s = smem_u32(smem);                        // P: two 32 KB buffers
+  const uint32_t q_s = p_s + 65536u;
   const uint32_t kv_s = q_s + q_bytes;
   const uint32_t nkv = (uint32_t)p.kv_stages;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 32768u + q_bytes + nkv * kv_bytes);
-  // bars: q_full q_empty kv_full[4] kv_empty[4] s_full[2] s_empty[2] p_full o_done drain drain2
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 65536u + q_bytes + nkv * kv_bytes);
+  // bars: q_full q_empty kv_full[4] kv_empty[4] s_full[2] s_empty[2] p_full[2] pv_done[2] drain drain2
   const uint32_t q_full = smem_u32(&bars[0]), q_empty = smem_u32(&bars[1]);
   auto kv_full = [&](int i) { return smem_u32(&bars[2 + i]); };
   auto kv_empty = [&](int i) { return smem_u32(&bars[6 + i]); };
   auto s_full = [&](int i) { return smem_u32(&bars[10 + i]); };
   auto s_empty = [&](int i) { return smem_u32(&bars[12 + i]); };
-  const uint32_t p_full = smem_u32(&bars[14]), o_done = smem_u32(&bars[15]);
-  const uint32_t drain_bar = smem_u32(&bars[16]), drain_pv = smem_u32(&bars[17]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+  // P_j lives in buffer j % 2 (j counted over all of the CTA's blocks):
+  // p_full[b] publishes it, pv_done[b] reports its P V products complete
+  auto p_full = [&](int b) { return smem_u32(&bars[14 + b]); };
+  auto pv_done = [&](int b) { return smem_u32(&bars[16 + b]); };
+  const uint32_t drain_bar = smem_u32(&bars[18]), drain_pv = smem_u32(&bars[19]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -91,8 +96,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_init(s_full(i), 1);
       mbar_init(s_empty(i), 4);
     }
-    mbar_init(p_full, 4);
-    mbar_init(o_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(p_full(b), 4);
+      mbar_init(pv_done(b), 1);
+    }
     mbar_init(drain_bar, 1);
     mbar_init(drain_pv, 1);
     *abort_flag = 0;
@@ -197,15 +204,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       // A second issuing thread: its MMAs run alongside the S MMAs.  P_j
       // exists only after S_j was read, so K_j is no longer in use when the
       // stage is released here.
-      uint32_t kv_it = 0, p_it = 0;
+      uint32_t kv_it = 0, pb = 0;              // pb: the CTA's block counter (P buffer pb % 2)
       for (long long item = blockIdx.x; item < p.items; item += gridDim.x) {
         int g, qt;
         decode(item, g, qt);
         const int n = qt + 1;
-        for (int j = 0; j < n; ++j) {
-          if (!mbar_wait(p_full, p_it & 1u, abort_flag)) goto pv_abort;
-          ++p_it;
+        for (int j = 0; j < n; ++j, ++pb) {
+          const int buf = (int)(pb & 1u);
+          if (!mbar_wait(p_full(buf), (pb >> 1) & 1u, abort_flag)) goto pv_abort;
           tc_fence_after();
+          const uint32_t pbuf = p_s + (uint32_t)buf * 32768u;
           const uint32_t pj = kv_it + (uint32_t)j;
           const uint32_t v_s = kv_s + (pj % nkv) * kv_bytes + q_bytes;
           const uint32_t row_b = (uint32_t)p.vw * 2u;
@@ -213,13 +221,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           const uint32_t vsw = p.vw == 64 ? 2u : (p.vw == 32 ? 4u : 6u);
           for (int st = 0; st < 8; ++st) {
             const uint64_t adesc =
-                make_smem_desc(p_s + (uint32_t)(st >> 2) * 16384u + (uint32_t)(st & 3) * 32u, 16u, 1024u, 2u);
+                make_smem_desc(pbuf + (uint32_t)(st >> 2) * 16384u + (uint32_t)(st & 3) * 32u, 16u, 1024u, 2u);
             const uint64_t bdesc = make_smem_desc(v_s + (uint32_t)(st >> 2) * kb_bytes +
                                                       (uint32_t)(st & 3) * 16u * row_b,
                                                   64u * row_b, 8u * row_b, vsw);
             tc_mma_f16(tmem_o, adesc, bdesc, p.idesc_pv, (j > 0 || st > 0) ? 1u : 0u);
           }
-          tc_commit(o_done);
+          tc_commit(pv_done(buf));
           tc_commit(kv_empty((int)(pj % nkv)));
         }
         kv_it += (uint32_t)n;
@@ -235,7 +243,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     const int q4 = warp & 3;                 // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;          // query row within the block
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    uint32_t s_it = 0, o_it = 0;
+    uint32_t s_it = 0, pb = 0;                 // pb: the CTA's block counter (P buffer pb % 2)
+    // wait until the P V products of block k (a CTA block counter) are done;
+    // only ever called for the latest block that used P buffer k % 2
+    auto wait_pv = [&](uint32_t k) { return mbar_wait(pv_done((int)(k & 1u)), (k >> 1) & 1u, abort_flag); };
     for (long long item = blockIdx.x; item < p.items; item += gridDim.x) {
       int g, qt;
       decode(item, g, qt);
@@ -243,7 +254,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       const int qrow = qt * kAttnTile + row;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < n && ok; ++j) {
+      for (int j = 0; j < n && ok; ++j, ++pb) {
         const int sb = (int)(s_it & 1u);
         if (!mbar_wait(s_full(sb), (s_it >> 1) & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -297,12 +308,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           }
         l = l * alpha + (s0 + s1);
         m = m_new;
-        if (j >= 1) {
-          // P_{j-1} V_{j-1} done: O is complete and the P buffer is free
-          if (!mbar_wait(o_done, o_it & 1u, abort_flag)) { ok = false; break; }
-          ++o_it;
+        // rescale O (rare): needs every earlier P V product done, i.e. block j-1's
+        if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+          if (!wait_pv(pb - 1)) { ok = false; break; }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+          {
             for (int c = 0; c < d / 16; ++c) {
               uint32_t o[16];
               tmem_ld16(tmem_o + lane_off + (uint32_t)(c * 16), o);
@@ -314,26 +324,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
             tmem_wait_st();
           }
         }
+        // P buffer pb % 2 is free once block pb-2's P V products are done (an
+        // earlier item's blocks are all done: its end waited for its last)
+        if (j >= 2 && !wait_pv(pb - 2)) { ok = false; break; }
         // P (16-bit) into the 128B-swizzled K-major A tile: row `row`,
         // 16-byte chunk c16 of the row goes to atom c16/8, slot (c16%8)^(row%8)
+        const uint32_t pbuf = p_s + (pb & 1u) * 32768u;
 #pragma unroll
         for (int c16 = 0; c16 < 16; ++c16) {
           float f[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[c16 >> 1][(c16 & 1) * 8 + e]);
-          const uint32_t addr = p_s + (uint32_t)(c16 >> 3) * 16384u + (uint32_t)row * 128u +
+          const uint32_t addr = pbuf + (uint32_t)(c16 >> 3) * 16384u + (uint32_t)row * 128u +
                                 (uint32_t)(((c16 & 7) ^ (row & 7)) * 16);
           st_shared_v4(addr, pack8<T>(f));
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(p_full((int)(pb & 1u)));
       }
       if (!ok) break;
       // epilogue: wait for the last P V, normalise, store O and the log-sum-exp
-      if (!mbar_wait(o_done, o_it & 1u, abort_flag)) break;
-      ++o_it;
+      if (!wait_pv(pb - 1)) break;
       tc_fence_after();
       const float inv_l = 1.0f / l;
       const int head = g % p.as, zb = g / p.as;

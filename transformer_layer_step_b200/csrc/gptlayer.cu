@@ -496,12 +496,12 @@ int run_attn_fwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
   p.q_off = 0; p.k_off = hs; p.v_off = 2 * hs;
   // P 32 KB + Q + 2 stages of K and V, barriers; at least 120 KB so that one
   // CTA (and its 512 tensor-memory columns) owns each SM
-  // P 32 KB, Q, the K / V ring (as deep as fits, 2..4 stages), barriers
+  // P 2 x 32 KB, Q, the K / V ring (as deep as fits, 2..4 stages), barriers
   const int kv_stage = 2 * 128 * d * 2;
-  p.kv_stages = (kSmemLimit - 1024 - 32768 - 128 * d * 2 - 512) / kv_stage;
+  p.kv_stages = (kSmemLimit - 1024 - 65536 - 128 * d * 2 - 512) / kv_stage;
   if (p.kv_stages > 4) p.kv_stages = 4;
   if (p.kv_stages < 2) return GPTL_E_SHAPE;
-  int smem = 1024 + 32768 + 128 * d * 2 + p.kv_stages * kv_stage + 512;
+  int smem = 1024 + 65536 + 128 * d * 2 + p.kv_stages * kv_stage + 512;
   if (smem < 120 * 1024) smem = 120 * 1024;
   const int grid = (int)(p.items < sms ? p.items : sms);
   // the shared-memory opt-in is recorded per device and per dtype (both
