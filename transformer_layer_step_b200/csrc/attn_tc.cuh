@@ -14,15 +14,16 @@
 //   warp 0     TMA: Q once per item, then K and V of each key block into a
 //              2-stage ring;
 //   warp 1     one thread issues S_j = Q K_j^T into one of two S buffers;
-//   warp 6     one thread issues O += P_j V_j once P_j is ready (two issuing
-//              threads, so that the two MMA streams run concurrently);
+//   warps 6-7  one thread each issues O += P_j V_j once P_j is ready, warp 6
+//              over keys 0..63 of the block into O, warp 7 over keys 64..127
+//              into O2 (added at the end): the MMA streams run concurrently;
 //   warps 2-5  one query row per thread: read S_j from tensor memory, update
 //              the running max m and sum l, rescale O by exp2(m_old - m_new)
 //              in tensor memory when m moved, write P_j (16-bit) to one of
 //              two shared-memory buffers (so that P_j is formed while
 //              P_{j-1} V_{j-1} runs); at the end normalise O by 1/l and
 //              store it.
-// Tensor memory: S buffers at columns 0 and 128, O at column 256.
+// Tensor memory: S buffers at columns 0 and 128, O at column 256, O2 at 384.
 // Shared memory: two P buffers [128 x 128] (two 128B-swizzled 64-column atoms each), Q as
 // head_dim/16 chunks of [128 rows x 16] (32B swizzle), and per stage K the
 // same way and V as MN-major chunks of [64 keys x vw].
@@ -31,7 +32,7 @@
 
 namespace gptl {
 
-constexpr int kAttnThreads = 224;
+constexpr int kAttnThreads = 256;
 constexpr int kAttnTile = 128;          // query rows per item, keys per block
 
 struct AttnParams {
@@ -81,7 +82,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   auto p_full = [&](int b) { return smem_u32(&bars[14 + b]); };
   auto pv_done = [&](int b) { return smem_u32(&bars[16 + b]); };
   const uint32_t drain_bar = smem_u32(&bars[18]), drain_pv = smem_u32(&bars[19]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
+  const uint32_t drain_pv2 = smem_u32(&bars[20]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 21);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -90,7 +92,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     mbar_init(q_empty, 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(kv_full(i), 1);
-      mbar_init(kv_empty(i), 1);
+      mbar_init(kv_empty(i), 2);   // both P V issuers release a stage
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
@@ -98,10 +100,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(p_full(b), 4);
-      mbar_init(pv_done(b), 1);
+      mbar_init(pv_done(b), 2);    // both halves of P_j V_j
     }
     mbar_init(drain_bar, 1);
     mbar_init(drain_pv, 1);
+    mbar_init(drain_pv2, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -117,7 +120,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tmem_o = tmem_base + 256u;
+  const uint32_t tmem_o = tmem_base + 256u;    // O over keys 0..63 of each block
+  const uint32_t tmem_o2 = tmem_base + 384u;   // O over keys 64..127 (added at the end)
 
   // work item -> (group, query block): the longest rows (last query blocks) first
   auto decode = [&](long long item, int &g, int &qt) {
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_wait_drain(drain_bar, 0);
     mma_done:;
     }
-  } else if (warp == 6) {
+  } else if (warp == 6 || warp == 7) {
     if (lane == 0) {
       // ------------------------------------------- MMA: O += P_j V_j
       // A second issuing thread: its MMAs run alongside the S MMAs.  P_j
@@ -219,13 +223,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           const uint32_t row_b = (uint32_t)p.vw * 2u;
           const uint32_t kb_bytes = (uint32_t)(d / p.vw) * 64u * row_b;
           const uint32_t vsw = p.vw == 64 ? 2u : (p.vw == 32 ? 4u : 6u);
-          for (int st = 0; st < 8; ++st) {
+          // warp 6: keys 0..63 of the block into O, warp 7: keys 64..127 into O2
+          const int st0 = warp == 6 ? 0 : 4;
+          const uint32_t acc_t = warp == 6 ? tmem_o : tmem_o2;
+          for (int st = st0; st < st0 + 4; ++st) {
             const uint64_t adesc =
                 make_smem_desc(pbuf + (uint32_t)(st >> 2) * 16384u + (uint32_t)(st & 3) * 32u, 16u, 1024u, 2u);
             const uint64_t bdesc = make_smem_desc(v_s + (uint32_t)(st >> 2) * kb_bytes +
                                                       (uint32_t)(st & 3) * 16u * row_b,
                                                   64u * row_b, 8u * row_b, vsw);
-            tc_mma_f16(tmem_o, adesc, bdesc, p.idesc_pv, (j > 0 || st > 0) ? 1u : 0u);
+            tc_mma_f16(acc_t, adesc, bdesc, p.idesc_pv, (j > 0 || st > st0) ? 1u : 0u);
           }
           tc_commit(pv_done(buf));
           tc_commit(kv_empty((int)(pj % nkv)));
@@ -234,8 +241,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       }
       goto pv_done;
     pv_abort:
-      tc_commit(drain_pv);
-      mbar_wait_drain(drain_pv, 0);
+      tc_commit(warp == 6 ? drain_pv : drain_pv2);
+      mbar_wait_drain(warp == 6 ? drain_pv : drain_pv2, 0);
     pv_done:;
     }
   } else {
@@ -313,13 +320,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           if (!wait_pv(pb - 1)) { ok = false; break; }
           tc_fence_after();
           {
-            for (int c = 0; c < d / 16; ++c) {
+            for (int c = 0; c < 2 * (d / 16); ++c) {   // O, then O2
+              const uint32_t ta = (c < d / 16 ? tmem_o : tmem_o2 - (uint32_t)d) + lane_off + (uint32_t)(c * 16);
               uint32_t o[16];
-              tmem_ld16(tmem_o + lane_off + (uint32_t)(c * 16), o);
+              tmem_ld16(ta, o);
               tmem_wait_ld();
 #pragma unroll
               for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st16(tmem_o + lane_off + (uint32_t)(c * 16), o);
+              tmem_st16(ta, o);
             }
             tmem_wait_st();
           }
@@ -352,15 +360,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       const int head = g % p.as, zb = g / p.as;
       T *orow = static_cast<T *>(p.o) + ((long long)zb * p.s + qrow) * p.hs + head * d;
       for (int c = 0; c < d / 16; ++c) {
-        uint32_t o[16];
+        uint32_t o[16], o2[16];
         tmem_ld16(tmem_o + lane_off + (uint32_t)(c * 16), o);
+        tmem_ld16(tmem_o2 + lane_off + (uint32_t)(c * 16), o2);
         tmem_wait_ld();
         if (qrow < p.s) {
           float f[8];
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[h2 * 8 + e]) * inv_l;
+            for (int e = 0; e < 8; ++e)
+              f[e] = (__uint_as_float(o[h2 * 8 + e]) + __uint_as_float(o2[h2 * 8 + e])) * inv_l;
             reinterpret_cast<uint4 *>(orow + c * 16)[h2] = pack8<T>(f);
           }
         }
