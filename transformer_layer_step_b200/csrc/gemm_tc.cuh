@@ -1,10 +1,10 @@
 // gemm_tc.cuh — persistent tcgen05/TMEM GEMM for sm_100a, fed by TMA.
 //
-// One kernel serves every dense contraction of the layer step: the four
-// linear layers (forward, input gradient, weight gradient) and the six
-// attention products.  D[M,N] = sum_k A[M,k] * B[N,k] per group, with
+// One kernel serves every dense contraction of the layer step outside
+// attention: the four linear layers (forward, input gradient, weight
+// gradient).  D[M,N] = sum_k A[M,k] * B[N,k] per group, with
 //   * operands read through 3-D TMA views (x = contiguous column, row, group)
-//     and staged in 128-row/BN-row x 64-deep shared-memory tiles;
+//     and staged in 128- or 256-row / BN-row x 64-deep shared-memory tiles;
 //   * either operand K-major (rows = M/N index, x = K) or MN-major
 //     (rows = K index, x = M/N), using the hardware transpose of the MMA
 //     instead of any transposing copy;
@@ -12,8 +12,8 @@
 //     split's partial sums and the column split's input-gradient sums are
 //     accumulated in one TMEM accumulator: "Megatron-LM 3D parallelism" §1
 //     describes the all-reduce this replaces);
-//   * causal rules for attention: skip score tiles above the diagonal, or
-//     limit the K range to the lower triangle;
+//   * causal rules (skip tiles above the diagonal, or limit the K range to
+//     the lower triangle), kept for the unfused attention products;
 //   * fused epilogues: bias, residual, bias+GeLU (writes Z and GeLU(Z): the
 //     fused_bias_gelu of "Training GPT-2 with Megatron-LM" §6.2), GeLU'
 //     scaling of an input gradient, fp32 weight-gradient store;
@@ -22,12 +22,14 @@
 //     stores them, so global writes are whole 32-byte sectors and the ragged
 //     M/N edges are clipped by the tensor map.
 //
-// Warp roles (320 threads, one CTA per SM): warp 0 issues TMA loads into a
-// multi-stage mbarrier ring, warp 1 allocates TMEM and one thread issues
-// tcgen05.mma (M=128, N=BN, K=16 each), warps 2..9 drain the double-buffered
-// accumulator with tcgen05.ld while the next tile's MMAs run.  A warp may
-// only read the TMEM lane quarter (warp % 4), so two epilogue warps share
-// each quarter and split its columns in half.
+// Warp roles (384 threads, one CTA per SM): two pipelines, each a TMA
+// producer warp (0, 2), an MMA warp (1, 3) whose one thread issues
+// tcgen05.mma (M=128, N=BN, K=16 each) and a TMEM accumulator of BN columns;
+// warp 1 allocates the 512 TMEM columns.  Warps 4..11 drain accumulators with
+// tcgen05.ld: a warp may only read the TMEM lane quarter (warp % 4), so two
+// epilogue warps share each quarter and split its columns in half.  How the
+// pipelines share the work (alternating tiles, K halves of each tile, or
+// 256-row tiles split by M) is described at gemm_tc_kernel.
 #pragma once
 #include "common.cuh"
 
