@@ -344,8 +344,10 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     # ---- e2e: every step's inputs (x, dOut) copied in from pinned host memory
     # and its output y plus the scaler state read back, inside the timed
-    # region.  A copy stream overlaps step i+1's input copy and step i's
-    # read-back with the compute of step i (double-buffered device buffers).
+    # region.  Double-buffered device buffers; one copy stream per direction,
+    # so that step i+1's input copy, step i-1's read-back and step i's compute
+    # run at the same time (host-to-device and device-to-host use separate
+    # copy engines and separate PCIe directions).
     x_host = torch.empty(ls.x.shape, dtype=ls.x.dtype).pin_memory()
     dy_host = torch.empty(ls.dy.shape, dtype=ls.dy.dtype).pin_memory()
     y_host = torch.empty(ls.y.shape, dtype=ls.y.dtype).pin_memory()
@@ -356,7 +358,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     dyb = [torch.empty_like(ls.dy) for _ in range(2)]
     yb = [torch.empty_like(ls.y) for _ in range(2)]
     stb = [torch.empty_like(ls.state) for _ in range(2)]   # per-step snapshot of the scaler
-    copy_stream = torch.cuda.Stream(dev)
+    h2d_stream = torch.cuda.Stream(dev)
+    d2h_stream = torch.cuda.Stream(dev)
     copied = [torch.cuda.Event() for _ in range(2)]
     computed = [torch.cuda.Event() for _ in range(2)]
     read_back = [torch.cuda.Event() for _ in range(2)]
@@ -364,33 +367,51 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     def copy_in(i):
         b = i % 2
-        with torch.cuda.stream(copy_stream):
+        with torch.cuda.stream(h2d_stream):
             if i >= 2:
-                copy_stream.wait_event(computed[b])      # step i-2 done with these buffers
+                h2d_stream.wait_event(computed[b])       # step i-2 done with these buffers
             xb[b].copy_(x_host, non_blocking=True)
             dyb[b].copy_(dy_host, non_blocking=True)
-            copied[b].record(copy_stream)
+            copied[b].record(h2d_stream)
+
+    def compute(b):
+        ls.step(x=xb[b], dy=dyb[b], y=yb[b])
+        stb[b].copy_(ls.state, non_blocking=True)
+
+    # one CUDA graph per buffer set replays the step (--e2e-eager: kernel by kernel)
+    e2e_step = [lambda b=b: compute(b) for b in range(2)]
+    e2e_graphs = []
+    if not args.e2e_eager:
+        for b in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                compute(b)
+            e2e_graphs.append(g)
+            e2e_step[b] = g.replay
+        for b in range(2):
+            e2e_step[b]()
+        torch.cuda.synchronize()
 
     barrier()
     torch.cuda.synchronize()
     t0.record(stream)
-    copy_stream.wait_event(t0)
+    h2d_stream.wait_event(t0)
+    d2h_stream.wait_event(t0)
     copy_in(0)
     for i in range(K):
         b = i % 2
         stream.wait_event(copied[b])
         if i >= 2:
             stream.wait_event(read_back[b])              # y buffer b read back (step i-2)
-        ls.step(x=xb[b], dy=dyb[b], y=yb[b])
-        stb[b].copy_(ls.state, non_blocking=True)
+        e2e_step[b]()
         computed[b].record(stream)
         if i + 1 < K:
             copy_in(i + 1)
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(computed[b])
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(computed[b])
             y_host.copy_(yb[b], non_blocking=True)
             st_host.copy_(stb[b], non_blocking=True)
-            read_back[b].record(copy_stream)
+            read_back[b].record(d2h_stream)
     stream.wait_event(read_back[(K - 1) % 2])
     t1.record(stream)
     torch.cuda.synchronize()
@@ -441,6 +462,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.CONFIGS))
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step's kernels one by one instead of as a CUDA graph")
+    ap.add_argument("--e2e-eager", action="store_true",
+                    help="launch the end-to-end steps kernel by kernel instead of as CUDA graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the CPU oracle timing (it runs on rank 0 at N=1 only)")
     args = ap.parse_args()
@@ -454,6 +477,8 @@ def main():
               "hidden": cfg.hidden, "heads": cfg.heads, "ffn": cfg.ffn, "tp": cfg.tp,
               "tokens_per_step": cfg.tokens, "parallelism": f"replicas{world}",
               "step_launch": "kernel by kernel" if args.no_graph else "one CUDA graph per step",
+              "e2e_step_launch": "kernel by kernel" if args.e2e_eager else "one CUDA graph per step",
+              "e2e_copies": "one stream per direction, overlapped with the neighbouring steps",
               "l2": "flushed between steps (256 MiB write, outside the per-step events)"}
     flops = step_flops(cfg)
 
