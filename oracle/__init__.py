@@ -19,7 +19,8 @@ in the function that uses it.
 
 Modules:
   layer   layer_fwd / layer_bwd (shard by shard, as the TP split computes it)
-  optim   found_inf, adam_step, loss_scale_update, cast_to_16
+  optim   found_inf, adam_step, loss_scale_update, cast_to_16, grad_norm,
+          clip_coefficient, accumulate
 
 Parity status: every function is pinned by tests in tests/test_oracle_*.py
 (finite differences, sharded == unsharded, closed forms, hand-computed
@@ -30,8 +31,10 @@ themselves, while the code that implements them is pinned.
 """
 from .layer import (layer_fwd, layer_bwd, layer_norm_fwd, layer_norm_bwd, gelu,
                     gelu_prime, causal_softmax, attention_head_fwd)
-from .optim import found_inf, adam_step, loss_scale_update, cast_to_16
+from .optim import (found_inf, adam_step, loss_scale_update, cast_to_16, grad_norm,
+                    clip_coefficient, accumulate)
 
 __all__ = ["layer_fwd", "layer_bwd", "layer_norm_fwd", "layer_norm_bwd", "gelu",
            "gelu_prime", "causal_softmax", "attention_head_fwd", "found_inf",
-           "adam_step", "loss_scale_update", "cast_to_16"]
+           "adam_step", "loss_scale_update", "cast_to_16", "grad_norm", "clip_coefficient",
+           "accumulate"]

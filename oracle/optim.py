@@ -4,7 +4,11 @@ master weights, dynamic loss-scale update.  Test infrastructure only.
 "Megatron-LM overview" §3.1: matrices are multiplied in FP16, an FP32 master
 copy of the weights receives the update, and the loss is scaled
 dynamically.  §4.2 names Adam with lr 6e-5.  §5.1 advises adjusting the
-initial scale when loss scaling misbehaves.
+initial scale when loss scaling misbehaves, and names gradient clipping
+that is too strong as a cause of non-convergence.  "Training GPT-2 with
+Megatron-LM" §4.3 accumulates gradients over micro-batches
+(--gradient-accumulation-steps) and its troubleshooting list adds
+--clip-grad 1.0 against NaN losses.
 
 Readings where the pages are silent:
   * overflow: any inf or NaN in the (scaled) fp32 gradients;
@@ -13,7 +17,13 @@ Readings where the pages are silent:
   * Adam: bias-corrected, eps outside the square root, decoupled weight
     decay (0 by default);
   * scaler: back off on the first overflow (no hysteresis), floor
-    min_scale, multiply by growth_factor after growth_interval clean steps.
+    min_scale, multiply by growth_factor after growth_interval clean steps;
+  * clipping: by the global L2 norm of the unscaled gradient over the whole
+    parameter arena, coefficient max_norm / (norm + 1e-6) applied when it is
+    below 1 (the usual global-norm clip; the pages give only the threshold);
+  * accumulation: the gradients of the micro-batches are summed in fp32
+    (the gradient of the summed loss); averaging, if wanted, belongs to the
+    loss gradient that the caller feeds to the backward pass.
 """
 from __future__ import annotations
 
@@ -75,11 +85,36 @@ def round_to_16(x: np.ndarray, dtype: str) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+def grad_norm(grad: np.ndarray, scale: float) -> float:
+    """Global L2 norm of the unscaled gradient, sqrt(sum_i (grad_i / S)^2),
+    in float64 from the fp32 (scaled) gradient arena."""
+    g = np.asarray(grad, dtype=np.float64).reshape(-1) / scale
+    return float(np.sqrt(np.dot(g, g)))
+
+
+def clip_coefficient(norm: float, max_norm: float) -> float:
+    """Factor applied to the unscaled gradient by global-norm clipping:
+    max_norm / (norm + 1e-6) when that is below 1, else exactly 1."""
+    c = max_norm / (norm + 1e-6)
+    return c if c < 1.0 else 1.0
+
+
+def accumulate(acc: np.ndarray, grad: np.ndarray) -> np.ndarray:
+    """acc + grad rounded to fp32 (one fp32 addition per element).  The
+    float64 sum of two fp32 numbers rounds to the same fp32 value as the
+    fp32 addition, so this is the exact fp32 result."""
+    return (np.asarray(acc, dtype=np.float32).astype(np.float64) +
+            np.asarray(grad, dtype=np.float32).astype(np.float64)).astype(np.float32)
+
+
 def adam_step(master: np.ndarray, m: np.ndarray, v: np.ndarray, grad: np.ndarray,
               scale: float, step: int, lr: float, beta1: float, beta2: float,
-              eps: float, weight_decay: float, dtype: str, inf_flag: int):
+              eps: float, weight_decay: float, dtype: str, inf_flag: int,
+              clip_coef: float = 1.0):
     """One Adam update on FP32 masters, computed in float64 from the fp32
     inputs.  `step` is the number of steps taken so far (t = step + 1).
+    The unscaled gradient grad / scale is multiplied by clip_coef (from
+    clip_coefficient; 1 without clipping) before it enters the moments.
 
     Returns (master, m, v, w16_bits) as float64/float64/float64/uint16; on
     overflow (inf_flag == 1) returns the inputs unchanged and w16 = None."""
@@ -88,7 +123,7 @@ def adam_step(master: np.ndarray, m: np.ndarray, v: np.ndarray, grad: np.ndarray
     p = np.asarray(master, dtype=np.float64)
     m = np.asarray(m, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
-    g = np.asarray(grad, dtype=np.float64) / scale
+    g = np.asarray(grad, dtype=np.float64) / scale * clip_coef
     t = step + 1
     m_new = beta1 * m + (1.0 - beta1) * g
     v_new = beta2 * v + (1.0 - beta2) * g * g
