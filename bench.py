@@ -420,11 +420,61 @@ def run_ours(args, cfg, rank, world, local_rank):
     if G.read_device_error(clear=True):
         raise RuntimeError("device error word set during the timed steps")
     sc = ls.scaler()
+    ext = measure_extensions(G, ls, cfg, dev, flush, peaks=load_peaks()[0])
     h2d = x_host.numel() * x_host.element_size() + dy_host.numel() * dy_host.element_size()
     d2h = y_host.numel() * y_host.element_size() + st_host.numel() * st_host.element_size()
     return dict(ms_per_step=ms_per_step, step_ms=step_ms, launches=launches, recs=recs,
                 e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks, n_params=ls.n_params,
-                scaler=sc)
+                scaler=sc, ext=ext)
+
+
+def measure_extensions(G, ls, cfg, dev, flush, peaks, reps=5):
+    """Per-launch device times of the optimizer extensions on this workload's
+    parameter arena: the clipped optimizer step (norm + overflow pass, clip
+    coefficient, Adam) with max_norm 1.0, and one gradient accumulation.
+    They run on copies of the optimizer state, after the timed regions, with
+    the L2 flushed before each call.  Algorithmic bytes per parameter: norm
+    pass 4 (read grad), Adam 30, accumulation 12 (read acc and grad, write
+    acc)."""
+    import torch
+    n = ls.n_params
+    hp = ls.hyper
+    st = ls.stream()
+    master, m, v, w16, state = (ls.master.clone(), ls.m.clone(), ls.v.clone(), ls.w16.clone(),
+                                ls.state.clone())
+    acc = ls.grad.clone()
+    ws = torch.zeros(G.CLIP_WORKSPACE_BYTES // 4, dtype=torch.float32, device=dev)
+    cap = 4 * reps + 4
+    G.profile_begin(cap)
+    for _ in range(reps):
+        flush.zero_()
+        G.adam_step_clip(n, master, m, v, ls.grad, w16, cfg.dtype, hp["lr"], hp["beta1"],
+                         hp["beta2"], hp["eps"], hp["weight_decay"], 1.0, ws, state, st)
+        flush.zero_()
+        G.grad_accumulate(n, acc, ls.grad, st)
+    recs, dropped = G.profile_end(cap)
+    if dropped:
+        raise RuntimeError(f"{dropped} extension launches were not timed")
+    ms = {}
+    for kind, _tag, t in recs:
+        ms.setdefault(kind, []).append(t)
+    mean = {k: sum(v) / len(v) for k, v in ms.items()}
+    hbm = peaks["hbm_gbs"]
+
+    def rate(kind, bpp):
+        gbs = bpp * n / (mean[kind] * 1e-3) / 1e9
+        return {"ms": round(mean[kind], 5), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
+
+    return {
+        "params": n,
+        "clip_step_ms": round(mean["overflow"] + mean["clip"] + mean["adam"], 5),
+        "norm_overflow_pass": rate("overflow", 4),
+        "clip_coefficient_ms": round(mean["clip"], 5),
+        "adam": rate("adam", 30),
+        "accumulate": rate("accumulate", 12),
+        "norm_of_unscaled_grad": round(float(ws[0]), 6),
+        "clip_coef": round(float(ws[1]), 6),
+    }
 
 
 def summarize_kernels(recs, K, cfg, n_params, peaks, flops):
@@ -547,6 +597,7 @@ def main():
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
         "scaler_after": res["scaler"],
+        "optimizer_extensions": res["ext"],
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         r = oracle_sample(cfg, 4)          # about 10 s of float64 CPU work

@@ -163,6 +163,47 @@ int adam_step_fp32_master(size_t n_params, float *master, float *m, float *v,
 int loss_scale_update(gptl_scaler_state *st, int growth_interval, float growth_factor,
                       float backoff_factor, float min_scale, gptl_stream_t stream);
 
+/* Bytes of device workspace adam_step_fp32_master_clip takes (clip_ws). */
+#define GPTL_CLIP_WORKSPACE_BYTES 16384
+
+/* adam_step_fp32_master with gradient clipping by global norm ("Training
+ * GPT-2 with Megatron-LM", troubleshooting: --clip-grad 1.0 against NaN
+ * losses; "Megatron-LM overview" §5.1: too strong a clip slows convergence).
+ *   1. one pass over grad: st->found_inf as in adam_step_fp32_master, and
+ *      float64 partial sums of grad^2 (fixed order, so the result is
+ *      bit-reproducible on a given GPU);
+ *   2. with S = st->scale, into clip_ws:
+ *        float at byte 0: norm = sqrt(sum_i (grad_i / S)^2), the L2 norm of
+ *                         the unscaled gradient over the whole arena;
+ *        float at byte 4: coef = max_norm / (norm + 1e-6) if that is < 1,
+ *                         else exactly 1;
+ *   3. if !found_inf: the Adam update of adam_step_fp32_master with the
+ *      unscaled gradient taken as grad / (S / coef), i.e. (grad / S) * coef
+ *      up to one fp32 rounding; with coef == 1 the update is bit-identical
+ *      to adam_step_fp32_master's.
+ * clip_ws: GPTL_CLIP_WORKSPACE_BYTES of DEVICE memory, 16-byte aligned, owned
+ * by the caller; norm and coef stay there after the call (read them after
+ * the stream has reached this point).  On overflow the step is skipped as in
+ * adam_step_fp32_master, and norm / coef are whatever the inf or NaN give.
+ * Other arguments and errors as adam_step_fp32_master; also GPTL_E_NULL if
+ * clip_ws is NULL, GPTL_E_ALIGN if it is not 16-byte aligned, GPTL_E_ARG if
+ * max_norm is not a finite positive number. */
+int adam_step_fp32_master_clip(size_t n_params, float *master, float *m, float *v,
+                               const float *grad, void *w16, gptl_dtype dtype, float lr,
+                               float beta1, float beta2, float eps, float weight_decay,
+                               float max_norm, void *clip_ws, gptl_scaler_state *st,
+                               gptl_stream_t stream);
+
+/* Gradient accumulation over micro-batches ("Training GPT-2 with
+ * Megatron-LM" §4.3, --gradient-accumulation-steps): acc[i] += grad[i] for
+ * i < n, in fp32 with one rounding per element.  Typical use: gpt_layer_bwd
+ * writes each micro-batch's gradients into a second arena, which is added to
+ * the accumulating arena; the sum is the gradient of the summed loss (scale
+ * dOut by 1/micro-batches for the mean).  acc, grad: DEVICE, 16-byte
+ * aligned, not overlapping.  GPTL_E_NULL / GPTL_E_ALIGN; GPTL_E_ARG if n is
+ * 0 or not a multiple of 4, or the ranges overlap. */
+int gptl_grad_accumulate(size_t n, float *acc, const float *grad, gptl_stream_t stream);
+
 /* Standalone overflow check (step 1 of adam_step_fp32_master). */
 int gptl_check_overflow(size_t n, const float *grad, gptl_scaler_state *st,
                         gptl_stream_t stream);

@@ -40,7 +40,9 @@ enum {
   GPTL_KIND_ROWDOT = 12,     /* softmax-backward row term dO . O              */
   GPTL_KIND_TRANSPOSE = 13,  /* token-contiguous copy of a gradient operand   */
   GPTL_KIND_ATTN_BWD = 14,   /* fused causal attention backward (dQ; dK, dV)  */
-  GPTL_KIND_COUNT = 15
+  GPTL_KIND_CLIP = 15,       /* global-norm clip coefficient (one block)      */
+  GPTL_KIND_ACCUMULATE = 16, /* gradient accumulation acc += grad             */
+  GPTL_KIND_COUNT = 17
 };
 
 /* step tags */

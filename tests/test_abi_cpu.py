@@ -78,3 +78,28 @@ def test_dtype_and_null_rejected_without_launch():
     assert rc == G.E_ALIGN
     rc = G.lib().loss_scale_update(16, 0, 2.0, 0.5, 1.0, None)
     assert rc == G.E_ARG
+
+
+def test_clip_and_accumulate_arguments_rejected_without_launch():
+    import re
+    import os
+    hdr = open(os.path.join(G.INCLUDE, "gptlayer.h")).read()
+    assert int(re.search(r"#define GPTL_CLIP_WORKSPACE_BYTES (\d+)", hdr).group(1)) == \
+        G.CLIP_WORKSPACE_BYTES
+    clip = G.lib().adam_step_fp32_master_clip
+    ok = (64, 16, 16, 16, 16, 16, 0, 1e-3, 0.9, 0.95, 1e-8, 0.0, 1.0, 16, 16, None)
+    for i, bad, code in [(13, None, G.E_NULL),                # no workspace
+                         (13, 24, G.E_ALIGN),                 # workspace not 16-byte aligned
+                         (12, 0.0, G.E_ARG),                  # max_norm must be positive
+                         (12, -1.0, G.E_ARG),
+                         (12, float("inf"), G.E_ARG),
+                         (12, float("nan"), G.E_ARG),
+                         (0, 66, G.E_ARG)]:                   # n % 4 != 0
+        args = list(ok)
+        args[i] = bad
+        assert clip(*args) == code, (i, bad)
+    acc = G.lib().gptl_grad_accumulate
+    assert acc(64, None, 16, None) == G.E_NULL
+    assert acc(64, 16, 20, None) == G.E_ALIGN
+    assert acc(66, 16, 1024, None) == G.E_ARG
+    assert acc(64, 1024, 1024 + 128, None) == G.E_ARG       # ranges overlap

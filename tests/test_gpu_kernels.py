@@ -165,3 +165,104 @@ def test_adam_matches_oracle(dtype):
         # the 16-bit copy is the RNE cast of the GPU's own fp32 master
         wg = ls.w16.view(torch.int16).cpu().numpy().view(np.uint16)
         np.testing.assert_array_equal(wg, oracle.cast_to_16(pg.astype(np.float64), dtype))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_clipped_adam_matches_oracle(dtype):
+    """adam_step_fp32_master_clip against the oracle's global-norm clip and
+    Adam: the reported norm and coefficient, the update, the skip on
+    overflow; unclipped steps bit-equal to adam_step_fp32_master; the norm
+    bit-reproducible."""
+    need_gpu()
+    cfg = dataclasses.replace(synth.CONFIGS["tiny"], dtype=dtype)
+    ls = LayerStep(cfg, synth.make_inputs(cfg))
+    n = ls.n_params
+    rng = np.random.default_rng(4)
+    hp = ls.hyper
+    f32 = lambda x: float(np.float32(x))
+    max_norm = 1.0
+    ws = torch.zeros(G.CLIP_WORKSPACE_BYTES // 4, dtype=torch.float32, device="cuda")
+    state = dict(scale=hp["init_scale"], growth_tracker=0, step=0)
+    # target norms of the unscaled gradient: below, far above, overflow, just
+    # below and just above the threshold
+    for step, target in enumerate([0.3, 5.0, None, 0.9999, 1.0001, 40.0]):
+        S = state["scale"]
+        grad = rng.standard_normal(n)
+        grad = (grad / np.sqrt((grad ** 2).sum()) * (target or 1.0) * S).astype(np.float32)
+        if target is None:
+            grad[n // 5] = np.inf
+        ls.grad.copy_(torch.from_numpy(grad))
+        m_in, v_in, p_in = ls.m.cpu().numpy(), ls.v.cpu().numpy(), ls.master.cpu().numpy()
+        w_in = ls.w16.clone()
+        plain = [ls.master.clone(), ls.m.clone(), ls.v.clone(), ls.w16.clone(), ls.state.clone()]
+        G.adam_step_clip(n, ls.master, ls.m, ls.v, ls.grad, ls.w16, dtype, hp["lr"], hp["beta1"],
+                         hp["beta2"], hp["eps"], hp["weight_decay"], max_norm, ws, ls.state,
+                         stream())
+        torch.cuda.synchronize()
+        norm_got, coef_got = float(ws[0]), float(ws[1])
+        if step == 0:            # the same inputs again: bit-identical norm
+            ws2 = torch.zeros_like(ws)
+            again = [t.clone() for t in plain]
+            G.adam_step_clip(n, again[0], again[1], again[2], ls.grad, again[3], dtype, hp["lr"],
+                             hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], max_norm,
+                             ws2, again[4], stream())
+            torch.cuda.synchronize()
+            assert torch.equal(ws2[:2], ws[:2])
+        check_device_error()
+        f = oracle.found_inf(grad)
+        assert ls.scaler()["found_inf"] == f
+        ls.scale_update()
+        torch.cuda.synchronize()
+        pe, me, ve, _ = (p_in, m_in, v_in, None)
+        if not f:
+            norm_ref = oracle.grad_norm(grad, S)
+            coef_ref = oracle.clip_coefficient(norm_ref, max_norm)
+            assert abs(norm_got - norm_ref) <= 1e-6 * norm_ref, (norm_got, norm_ref)
+            assert (coef_got == 1.0) == (coef_ref == 1.0), (coef_got, coef_ref)
+            assert abs(coef_got - coef_ref) <= 1e-6 * coef_ref
+            assert (coef_ref < 1.0) == (target > max_norm)
+            pe, me, ve, _ = oracle.adam_step(p_in, m_in, v_in, grad, S, state["step"], f32(hp["lr"]),
+                                             f32(hp["beta1"]), f32(hp["beta2"]), f32(hp["eps"]),
+                                             f32(hp["weight_decay"]), dtype, f, clip_coef=coef_ref)
+        state = oracle.loss_scale_update(state, f, hp["growth_interval"], hp["growth_factor"],
+                                         hp["backoff_factor"], hp["min_scale"])
+        sc = ls.scaler()
+        assert (sc["scale"], sc["growth_tracker"], sc["step"]) == \
+            (state["scale"], state["growth_tracker"], state["step"])
+        pg, mg, vg = ls.master.cpu().numpy(), ls.m.cpu().numpy(), ls.v.cpu().numpy()
+        if f:
+            assert np.array_equal(pg, p_in) and np.array_equal(mg, m_in) and np.array_equal(vg, v_in)
+            assert torch.equal(ls.w16, w_in)
+            continue
+        lr = f32(hp["lr"])
+        assert np.all(np.abs(pg - pe) <= 1e-6 * np.maximum(np.abs(pe), lr))
+        assert np.all(np.abs(vg - ve) <= 1e-6 * np.abs(ve) + 1e-45)
+        assert np.all(np.abs(mg - me) <= 1e-6 * np.maximum(np.abs(me), np.sqrt(np.mean(me ** 2))))
+        wg = ls.w16.view(torch.int16).cpu().numpy().view(np.uint16)
+        np.testing.assert_array_equal(wg, oracle.cast_to_16(pg.astype(np.float64), dtype))
+        if coef_got == 1.0:      # no clipping: the plain optimizer step, bit for bit
+            G.adam_step(n, plain[0], plain[1], plain[2], ls.grad, plain[3], dtype, hp["lr"],
+                        hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], plain[4], stream())
+            torch.cuda.synchronize()
+            assert torch.equal(plain[0], ls.master) and torch.equal(plain[1], ls.m)
+            assert torch.equal(plain[2], ls.v) and torch.equal(plain[3], ls.w16)
+
+
+def test_grad_accumulate_is_fp32_addition():
+    need_gpu()
+    rng = np.random.default_rng(12)
+    n = (1 << 20) + 4 * 37
+    parts = []
+    for _ in range(3):
+        g = (rng.standard_normal(n) * 10.0 ** rng.integers(-12, 12, n)).astype(np.float32)
+        parts.append(g)
+    parts[1][:100] = -parts[0][:100]                          # exact cancellation
+    parts[1][100:200] = parts[0][100:200] * np.float32(2.0 ** -24)   # addends near half an ulp
+    acc_t = torch.from_numpy(parts[0].copy()).cuda()
+    want = parts[0]
+    for g in parts[1:]:
+        G.grad_accumulate(n, acc_t, torch.from_numpy(g).cuda(), stream())
+        want = oracle.accumulate(want, g)
+    check_device_error()
+    got = acc_t.cpu().numpy()
+    np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32))

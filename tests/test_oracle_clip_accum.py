@@ -85,7 +85,7 @@ def test_accumulate_is_fp32_addition():
     a = (rng.standard_normal(20000) * 10.0 ** rng.integers(-20, 20, 20000)).astype(np.float32)
     b = (rng.standard_normal(20000) * 10.0 ** rng.integers(-20, 20, 20000)).astype(np.float32)
     b[:10] = -a[:10]                                   # exact cancellation
-    b[10:20] = a[10:20] * np.float32(2.0 ** -24)      # halfway cases of the rounding
+    b[10:20] = a[10:20] * np.float32(2.0 ** -24)      # addends near half an ulp
     want = (torch.from_numpy(a) + torch.from_numpy(b)).numpy()
     got = oracle.accumulate(a, b)
     assert got.dtype == np.float32

@@ -16,7 +16,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libgptlayer.so")
-SOURCES = [os.path.join(PKG, "csrc", "gptlayer.cu")]
+SOURCES = [os.path.join(PKG, "csrc", "libgptlayer.cu")]
 
 
 def deps() -> list:

@@ -74,7 +74,8 @@ class LaunchRecord(C.Structure):
 
 
 KIND_NAMES = ("gemm", "ln_fwd", "ln_bwd", "softmax_fwd", "softmax_bwd", "colsum", "reduce",
-              "overflow", "adam", "scale", "splitk", "attn_fwd", "rowdot", "transpose", "attn_bwd")
+              "overflow", "adam", "scale", "splitk", "attn_fwd", "rowdot", "transpose", "attn_bwd",
+              "clip", "accumulate")
 
 _lib = None
 
@@ -95,6 +96,11 @@ _SIGS = {
     "loss_scale_update": (C.c_int, [C.c_void_p, C.c_int, C.c_float, C.c_float, C.c_float,
                                     C.c_void_p]),
     "gptl_check_overflow": (C.c_int, [C.c_size_t, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "adam_step_fp32_master_clip": (C.c_int, [C.c_size_t, C.c_void_p, C.c_void_p, C.c_void_p,
+                                             C.c_void_p, C.c_void_p, C.c_int, C.c_float,
+                                             C.c_float, C.c_float, C.c_float, C.c_float,
+                                             C.c_float, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "gptl_grad_accumulate": (C.c_int, [C.c_size_t, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gptl_gemm": (C.c_int, [C.POINTER(GemmDesc), C.c_int, C.c_void_p]),
     "gptl_gemm_plan": (C.c_int, [C.POINTER(GemmDesc), C.c_int, C.POINTER(C.c_int),
                                  C.POINTER(C.c_int), C.POINTER(C.c_int)]),
@@ -210,6 +216,25 @@ def adam_step(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps, w
     _check(lib().adam_step_fp32_master(n_params, _ptr(master), _ptr(m), _ptr(v), _ptr(grad),
                                        _ptr(w16), DTYPES.get(dtype, dtype), lr, beta1, beta2, eps,
                                        weight_decay, _ptr(state), stream), "adam_step_fp32_master")
+
+
+# bytes of the clip workspace (GPTL_CLIP_WORKSPACE_BYTES in gptlayer.h); the
+# norm of the unscaled gradient is the float at byte 0, the clip coefficient
+# the float at byte 4
+CLIP_WORKSPACE_BYTES = 16384
+
+
+def adam_step_clip(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps, weight_decay,
+                   max_norm, clip_ws, state, stream=0):
+    _check(lib().adam_step_fp32_master_clip(n_params, _ptr(master), _ptr(m), _ptr(v), _ptr(grad),
+                                            _ptr(w16), DTYPES.get(dtype, dtype), lr, beta1, beta2,
+                                            eps, weight_decay, max_norm, _ptr(clip_ws),
+                                            _ptr(state), stream),
+           "adam_step_fp32_master_clip")
+
+
+def grad_accumulate(n, acc, grad, stream=0):
+    _check(lib().gptl_grad_accumulate(n, _ptr(acc), _ptr(grad), stream), "gptl_grad_accumulate")
 
 
 def scale_update(state, growth_interval, growth_factor, backoff_factor, min_scale, stream=0):
