@@ -392,27 +392,32 @@ def run_ours(args, cfg, rank, world, local_rank):
             e2e_step[b]()
         torch.cuda.synchronize()
 
+    def e2e_steps(n):
+        copy_in(0)
+        for i in range(n):
+            b = i % 2
+            stream.wait_event(copied[b])
+            if i >= 2:
+                stream.wait_event(read_back[b])          # y buffer b read back (step i-2)
+            e2e_step[b]()
+            computed[b].record(stream)
+            if i + 1 < n:
+                copy_in(i + 1)
+            with torch.cuda.stream(d2h_stream):
+                d2h_stream.wait_event(computed[b])
+                y_host.copy_(yb[b], non_blocking=True)
+                st_host.copy_(stb[b], non_blocking=True)
+                read_back[b].record(d2h_stream)
+        stream.wait_event(read_back[(n - 1) % 2])
+
+    e2e_steps(W)                                         # untimed: warms the copy path
+    torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     t0.record(stream)
     h2d_stream.wait_event(t0)
     d2h_stream.wait_event(t0)
-    copy_in(0)
-    for i in range(K):
-        b = i % 2
-        stream.wait_event(copied[b])
-        if i >= 2:
-            stream.wait_event(read_back[b])              # y buffer b read back (step i-2)
-        e2e_step[b]()
-        computed[b].record(stream)
-        if i + 1 < K:
-            copy_in(i + 1)
-        with torch.cuda.stream(d2h_stream):
-            d2h_stream.wait_event(computed[b])
-            y_host.copy_(yb[b], non_blocking=True)
-            st_host.copy_(stb[b], non_blocking=True)
-            read_back[b].record(d2h_stream)
-    stream.wait_event(read_back[(K - 1) % 2])
+    e2e_steps(K)
     t1.record(stream)
     torch.cuda.synchronize()
     barrier()
