@@ -182,8 +182,9 @@ int loss_scale_update(gptl_scaler_state *st, int growth_interval, float growth_f
  *      up to one fp32 rounding; with coef == 1 the update is bit-identical
  *      to adam_step_fp32_master's.
  * clip_ws: GPTL_CLIP_WORKSPACE_BYTES of DEVICE memory, 16-byte aligned, owned
- * by the caller; norm and coef stay there after the call (read them after
- * the stream has reached this point).  On overflow the step is skipped as in
+ * by the caller, overlapping none of the arenas or st; norm and coef stay
+ * there after the call (read them after the stream has reached this point).
+ * Calls that share one clip_ws must be ordered on the device.  On overflow the step is skipped as in
  * adam_step_fp32_master, and norm / coef are whatever the inf or NaN give.
  * Other arguments and errors as adam_step_fp32_master; also GPTL_E_NULL if
  * clip_ws is NULL, GPTL_E_ALIGN if it is not 16-byte aligned, GPTL_E_ARG if
