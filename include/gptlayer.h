@@ -92,7 +92,9 @@ typedef struct {
 /* FP32 gradients, same layouts as gptl_weights, multiplied by the loss scale
  * (they are the gradients of the scaled loss).  gpt_layer_bwd OVERWRITES
  * them.  Normally these point into the flat gradient arena that
- * adam_step_fp32_master consumes (see gpt_layer_param_layout). */
+ * adam_step_fp32_master consumes (see gpt_layer_param_layout); to accumulate
+ * over micro-batches, write each into a second arena and add it with
+ * gptl_grad_accumulate. */
 typedef struct {
   float *ln1_g, *ln1_b, *w_qkv, *b_qkv, *w_o, *b_o,
         *ln2_g, *ln2_b, *w_1, *b_1, *w_2, *b_2;
