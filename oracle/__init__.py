@@ -18,7 +18,8 @@ Adam constants, scaler growth rule) the plainest reading is taken and named
 in the function that uses it.
 
 Modules:
-  layer   layer_fwd / layer_bwd (shard by shard, as the TP split computes it)
+  layer   layer_fwd / layer_bwd (shard by shard, as the TP split computes it),
+          stack_fwd / stack_bwd (layers of one shape, chained)
   optim   found_inf, adam_step, loss_scale_update, cast_to_16, grad_norm,
           clip_coefficient, accumulate
 
@@ -30,11 +31,11 @@ choice and cannot be pinned to the pages: parity unpinned for those choices
 themselves, while the code that implements them is pinned.
 """
 from .layer import (layer_fwd, layer_bwd, layer_norm_fwd, layer_norm_bwd, gelu,
-                    gelu_prime, causal_softmax, attention_head_fwd)
+                    gelu_prime, causal_softmax, attention_head_fwd, stack_fwd, stack_bwd)
 from .optim import (found_inf, adam_step, loss_scale_update, cast_to_16, grad_norm,
                     clip_coefficient, accumulate)
 
-__all__ = ["layer_fwd", "layer_bwd", "layer_norm_fwd", "layer_norm_bwd", "gelu",
+__all__ = ["layer_fwd", "layer_bwd", "stack_fwd", "stack_bwd", "layer_norm_fwd", "layer_norm_bwd", "gelu",
            "gelu_prime", "causal_softmax", "attention_head_fwd", "found_inf",
            "adam_step", "loss_scale_update", "cast_to_16", "grad_norm", "clip_coefficient",
            "accumulate"]

@@ -265,3 +265,34 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
                                                     params["ln1_g"])
     dx = dhid + dln1
     return dx, gr
+
+
+def stack_fwd(x: np.ndarray, params_list: list, dims: dict, eps: float = 1e-5, precision=None):
+    """Forward of a stack of layers of one shape ("Training GPT-2 with
+    Megatron-LM" §4.1 runs --num-layers 32 of them): layer l's output is
+    layer l+1's input.  With a precision, the output a layer hands to the
+    next is held in the 16-bit type, the store between the two layers.
+    Returns (out, caches); out is the last layer's output, unrounded."""
+    caches = []
+    h = x
+    for l, p in enumerate(params_list):
+        if l > 0 and precision is not None:
+            h = round_to_16(h, precision)
+        h, c = layer_fwd(h, p, dims, eps, precision)
+        caches.append(c)
+    return h, caches
+
+
+def stack_bwd(caches: list, params_list: list, dims: dict, dout: np.ndarray):
+    """Backward through stack_fwd's layers in reverse order: layer l's dX is
+    layer l-1's dOut, held in the 16-bit type between the two layers under a
+    precision.  Returns (dx, grads) with grads[l] the gradients of layer l."""
+    grads = [None] * len(params_list)
+    d = dout
+    last = len(params_list) - 1
+    for l in range(last, -1, -1):
+        prec = caches[l].get("precision")
+        if l < last and prec is not None:
+            d = round_to_16(d, prec)
+        d, grads[l] = layer_bwd(caches[l], params_list[l], dims, d)
+    return d, grads
