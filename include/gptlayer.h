@@ -165,6 +165,37 @@ int adam_step_fp32_master(size_t n_params, float *master, float *m, float *v,
 int loss_scale_update(gptl_scaler_state *st, int growth_interval, float growth_factor,
                       float backoff_factor, float min_scale, gptl_stream_t stream);
 
+/* Stacks of n_layers layers of one shape ("Training GPT-2 with Megatron-LM"
+ * §4.1: --num-layers 32).  Layer l has its own weights w[l] and gradients
+ * g[l] (normally layer l's block of one arena holding every layer's
+ * parameters back to back, n_params of gpt_layer_param_layout apart, which
+ * one adam_step_fp32_master call over n_layers * n_params then updates).
+ *  saved_bytes  : n_layers per-layer saved workspaces (256-byte multiples);
+ *  scratch_bytes: the layer scratch plus two [T,h] buffers for the input
+ *                 gradients handed between layers.
+ * GPTL_E_ARG if n_layers < 1; otherwise as gpt_layer_workspace_bytes. */
+int gpt_stack_workspace_bytes(const gptl_shape *shape, int n_layers, size_t *saved_bytes,
+                              size_t *scratch_bytes);
+
+/* Forward through layers 0..n_layers-1: layer 0 reads x, layer l > 0 reads
+ * layer l-1's output.  acts: n_layers [T,h] outputs (cdt) back to back,
+ * layer l's at acts + l*T*h elements; the stack's output is the last one.
+ * w: n_layers gptl_weights; saved: gpt_stack_workspace_bytes' saved bytes,
+ * untouched until gpt_stack_bwd.  x, acts and saved must not overlap.
+ * All arguments are checked before the first launch. */
+int gpt_stack_fwd(const gptl_shape *shape, int n_layers, const gptl_weights *w, const void *x,
+                  void *acts, void *saved, gptl_stream_t stream);
+
+/* Backward through layers n_layers-1..0: the last layer reads dy (gradient
+ * of the scaled loss w.r.t. the stack's output), layer l < n_layers-1 reads
+ * layer l+1's input gradient, and layer 0 writes dx.  x, acts and saved as
+ * passed to / written by gpt_stack_fwd; g: n_layers gptl_grads, each
+ * OVERWRITTEN; scratch: gpt_stack_workspace_bytes' scratch bytes.  All
+ * arguments are checked before the first launch. */
+int gpt_stack_bwd(const gptl_shape *shape, int n_layers, const gptl_weights *w, const void *x,
+                  const void *acts, const void *saved, const void *dy, void *dx,
+                  const gptl_grads *g, void *scratch, gptl_stream_t stream);
+
 /* Bytes of device workspace adam_step_fp32_master_clip takes (clip_ws). */
 #define GPTL_CLIP_WORKSPACE_BYTES 16384
 

@@ -103,3 +103,30 @@ def test_clip_and_accumulate_arguments_rejected_without_launch():
     assert acc(64, 16, 20, None) == G.E_ALIGN
     assert acc(66, 16, 1024, None) == G.E_ARG
     assert acc(64, 1024, 1024 + 128, None) == G.E_ARG       # ranges overlap
+
+
+def test_stack_workspace_and_arguments_rejected_without_launch():
+    sh = G.make_shape(2, 64, 128, 4, 512, 2, "fp16")
+    saved1, scratch1 = G.workspace_bytes(sh)
+    for n in (1, 3, 32):
+        saved, scratch = G.stack_workspace_bytes(sh, n)
+        per = (saved1 + 255) // 256 * 256
+        act = (2 * 64 * 128 * 2 + 255) // 256 * 256
+        assert saved == n * per
+        assert scratch == (scratch1 + 255) // 256 * 256 + 2 * act
+    with pytest.raises(G.GptlError) as e:
+        G.stack_workspace_bytes(sh, 0)
+    assert e.value.code == G.E_ARG
+    w = G.make_weights({n: 4096 for n in G.PARAM_NAMES})
+    g = G.make_grads({n: 4096 for n in G.PARAM_NAMES})
+    lib = G.lib()
+    ws = (G.Weights * 2)(w, w)
+    gs = (G.Grads * 2)(g, g)
+    assert lib.gpt_stack_fwd(ctypes.byref(sh), 0, ws, 16, 32, 48, None) == G.E_ARG
+    assert lib.gpt_stack_fwd(ctypes.byref(sh), 2, ws, None, 32, 48, None) == G.E_NULL
+    assert lib.gpt_stack_fwd(ctypes.byref(sh), 2, ws, 16, 40, 48, None) == G.E_ALIGN
+    bad = (G.Weights * 2)(w, G.make_weights({n: (8 if n == "w_o" else 4096) for n in G.PARAM_NAMES}))
+    assert lib.gpt_stack_fwd(ctypes.byref(sh), 2, bad, 16, 32, 48, None) == G.E_ALIGN
+    gbad = (G.Grads * 2)(g, G.make_grads({n: (None if n == "b_2" else 4096) for n in G.PARAM_NAMES}))
+    assert lib.gpt_stack_bwd(ctypes.byref(sh), 2, ws, 16, 32, 48, 64, 80, gbad, 96, None) == G.E_NULL
+    assert lib.gpt_stack_bwd(ctypes.byref(sh), 2, ws, 16, 32, 48, 64, 80, gs, None, None) == G.E_NULL

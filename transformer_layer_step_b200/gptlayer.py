@@ -90,6 +90,13 @@ _SIGS = {
                                 C.c_void_p, C.c_void_p, C.c_void_p]),
     "gpt_layer_bwd": (C.c_int, [C.POINTER(Shape), C.POINTER(Weights), C.c_void_p, C.c_void_p,
                                 C.c_void_p, C.c_void_p, C.POINTER(Grads), C.c_void_p, C.c_void_p]),
+    "gpt_stack_workspace_bytes": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(C.c_size_t),
+                                            C.POINTER(C.c_size_t)]),
+    "gpt_stack_fwd": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(Weights), C.c_void_p,
+                                C.c_void_p, C.c_void_p, C.c_void_p]),
+    "gpt_stack_bwd": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(Weights), C.c_void_p,
+                                C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.POINTER(Grads),
+                                C.c_void_p, C.c_void_p]),
     "adam_step_fp32_master": (C.c_int, [C.c_size_t, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                         C.c_void_p, C.c_int, C.c_float, C.c_float, C.c_float,
                                         C.c_float, C.c_float, C.c_void_p, C.c_void_p]),
@@ -209,6 +216,30 @@ def layer_fwd(shape, weights: Weights, x, y, saved, scratch=None, stream=0):
 def layer_bwd(shape, weights: Weights, x, saved, dy, dx, grads: Grads, scratch, stream=0):
     _check(lib().gpt_layer_bwd(C.byref(shape), C.byref(weights), _ptr(x), _ptr(saved), _ptr(dy),
                                _ptr(dx), C.byref(grads), _ptr(scratch), stream), "gpt_layer_bwd")
+
+
+def stack_workspace_bytes(shape: Shape, n_layers: int):
+    a, b = C.c_size_t(), C.c_size_t()
+    _check(lib().gpt_stack_workspace_bytes(C.byref(shape), n_layers, C.byref(a), C.byref(b)),
+           "gpt_stack_workspace_bytes")
+    return a.value, b.value
+
+
+def stack_fwd(shape, weights, x, acts, saved, stream=0):
+    """weights: a sequence of Weights, one per layer."""
+    arr = (Weights * len(weights))(*weights)
+    _check(lib().gpt_stack_fwd(C.byref(shape), len(weights), arr, _ptr(x), _ptr(acts),
+                               _ptr(saved), stream), "gpt_stack_fwd")
+
+
+def stack_bwd(shape, weights, x, acts, saved, dy, dx, grads, scratch, stream=0):
+    """weights, grads: sequences of Weights / Grads, one per layer."""
+    if len(grads) != len(weights):
+        raise ValueError("one Grads per layer")
+    wa = (Weights * len(weights))(*weights)
+    ga = (Grads * len(grads))(*grads)
+    _check(lib().gpt_stack_bwd(C.byref(shape), len(weights), wa, _ptr(x), _ptr(acts), _ptr(saved),
+                               _ptr(dy), _ptr(dx), ga, _ptr(scratch), stream), "gpt_stack_bwd")
 
 
 def adam_step(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps, weight_decay,

@@ -127,3 +127,83 @@ class LayerStep:
 
     def params_host_bits(self) -> dict:
         return {n: tensor_to_bits(self.param_tensor(self.w16, n)) for n in G.PARAM_NAMES}
+
+
+class LayerStack(LayerStep):
+    """A stack of layers of one shape on `device` ("Training GPT-2 with
+    Megatron-LM" §4.1 trains --num-layers of them): every layer's parameters
+    back to back in one flat arena per kind (layer l's block starts at
+    l * n_layer_params), the layers' saved workspaces, their outputs `acts`
+    ([L, T, h]; the stack's output is acts[-1]), and ONE optimizer step over
+    the whole arena.  fwd / bwd make one gpt_stack_fwd / gpt_stack_bwd call;
+    adam, scale_update and the scaler helpers are LayerStep's, applied to the
+    stack's arenas."""
+
+    def __init__(self, cfg: synth.LayerConfig, layer_params: list, x_bits: np.ndarray,
+                 device="cuda", hyper=None):
+        self.cfg = cfg
+        self.hyper = dict(synth.HYPER, **(hyper or {}))
+        self.device = torch.device(device)
+        self.shape = G.make_shape(cfg.batch, cfg.seq, cfg.hidden, cfg.heads, cfg.ffn, cfg.tp,
+                                  cfg.dtype, self.hyper["ln_eps"])
+        self.n_layers = L = len(layer_params)
+        self.offsets, self.n_layer_params = G.param_layout(self.shape)
+        self.n_params = L * self.n_layer_params
+        saved_b, scratch_b = G.stack_workspace_bytes(self.shape, L)
+        dt = TORCH_DT[cfg.dtype]
+        dev = self.device
+        T, h = cfg.tokens, cfg.hidden
+
+        flat_bits = np.zeros(self.n_params, dtype=np.uint16)
+        self.param_shapes = {}
+        for l, params in enumerate(layer_params):
+            base = l * self.n_layer_params
+            for name, off in zip(G.PARAM_NAMES, self.offsets):
+                arr = params[name]
+                self.param_shapes[name] = arr.shape
+                flat_bits[base + off:base + off + arr.size] = arr.reshape(-1)
+        self.w16 = bits_to_tensor(flat_bits, cfg.dtype, dev)
+        self.master = self.w16.to(torch.float32)
+        self.m = torch.zeros(self.n_params, dtype=torch.float32, device=dev)
+        self.v = torch.zeros(self.n_params, dtype=torch.float32, device=dev)
+        self.grad = torch.zeros(self.n_params, dtype=torch.float32, device=dev)
+
+        self.x = bits_to_tensor(x_bits, cfg.dtype, dev).view(T, h)
+        self.acts = torch.empty((L, T, h), dtype=dt, device=dev)
+        self.y = self.acts[L - 1]
+        self.dx = torch.empty((T, h), dtype=dt, device=dev)
+        self.dy = torch.zeros((T, h), dtype=dt, device=dev)
+        self.saved = torch.empty(max(saved_b, 256), dtype=torch.uint8, device=dev)
+        self.scratch = torch.empty(max(scratch_b, 256), dtype=torch.uint8, device=dev)
+        self.state = torch.zeros(8, dtype=torch.int32, device=dev)
+        self.reset_scaler(self.hyper["init_scale"])
+
+        self.layer_weights, self.layer_grads = [], []
+        for l in range(L):
+            base = l * self.n_layer_params
+            self.layer_weights.append(G.make_weights(
+                {n: self.w16.data_ptr() + 2 * (base + off) for n, off in zip(G.PARAM_NAMES, self.offsets)}))
+            self.layer_grads.append(G.make_grads(
+                {n: self.grad.data_ptr() + 4 * (base + off) for n, off in zip(G.PARAM_NAMES, self.offsets)}))
+
+    def fwd(self, x=None, y=None):
+        if y is not None:
+            raise ValueError("the stack writes its output into acts[-1]")
+        G.stack_fwd(self.shape, self.layer_weights, self.x if x is None else x, self.acts,
+                    self.saved, self.stream())
+
+    def bwd(self, x=None, dy=None):
+        G.stack_bwd(self.shape, self.layer_weights, self.x if x is None else x, self.acts,
+                    self.saved, self.dy if dy is None else dy, self.dx, self.layer_grads,
+                    self.scratch, self.stream())
+
+    def layer_param_tensor(self, arena: torch.Tensor, layer: int, name: str) -> torch.Tensor:
+        off = layer * self.n_layer_params + self.offsets[G.PARAM_NAMES.index(name)]
+        shp = self.param_shapes[name]
+        return arena[off:off + int(np.prod(shp))].view(shp)
+
+    def layer_grads_host(self, layer: int) -> dict:
+        return {n: self.layer_param_tensor(self.grad, layer, n).cpu().numpy() for n in G.PARAM_NAMES}
+
+    def param_tensor(self, arena, name):
+        raise TypeError("a stack has one block per layer: use layer_param_tensor")
