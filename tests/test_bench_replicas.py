@@ -67,3 +67,13 @@ def test_single_rank_needs_no_collective():
     b = _bench()
     assert b.reduce_max_over_ranks(2.5, 1, "cpu") == 2.5
     assert b.whole_job_tokens_per_s(1, 8192, 2.0) == pytest.approx(8192 / 2e-3)
+
+
+def test_kernel_hash_ignores_comments_only():
+    import bench
+    src = "int a; // note\n/* block\n comment */ int b;\n\n  // indented\nint c; /* tail */\n"
+    assert bench.code_without_comments(src) == "int a;\n int b;\nint c;"
+    reworded = src.replace("note", "other words").replace("block", "blk")
+    assert bench.code_without_comments(reworded) == bench.code_without_comments(src)
+    assert bench.code_without_comments(src.replace("int b", "int bb")) != \
+        bench.code_without_comments(src)
