@@ -10,9 +10,9 @@
 // log-sum-exp of each row's scaled scores, from which the backward
 // recomputes P.
 //
-// Warp roles (224 threads, one CTA per SM, persistent over work items):
+// Warp roles (256 threads, one CTA per SM, persistent over work items):
 //   warp 0     TMA: Q once per item, then K and V of each key block into a
-//              2-stage ring;
+//              ring of kv_stages (2..4) stages;
 //   warp 1     one thread issues S_j = Q K_j^T into one of two S buffers;
 //   warps 6-7  one thread each issues O += P_j V_j once P_j is ready, warp 6
 //              over keys 0..63 of the block into O, warp 7 over keys 64..127
