@@ -2,7 +2,9 @@
 //
 // LayerNorm forward/backward, the fused causal scale-mask-softmax
 // forward/backward ("Training GPT-2 with Megatron-LM" §6.2 fused_softmax),
-// column sums for bias gradients, and the optimizer side of mixed precision
+// column sums for bias gradients, batched 16-bit transposes (the
+// token-contiguous copies that weight-gradient GEMMs read as K-major
+// operands), and the optimizer side of mixed precision
 // ("Megatron-LM overview" §3.1, §4.2): overflow check, fused unscale + Adam +
 // 16-bit cast on FP32 masters, dynamic loss-scale update.
 //
