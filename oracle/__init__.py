@@ -19,6 +19,7 @@ in the function that uses it.
 
 Modules:
   layer   layer_fwd / layer_bwd (shard by shard, as the TP split computes it),
+          attention_head_fwd / attention_head_bwd (one causal head),
           stack_fwd / stack_bwd (layers of one shape, chained)
   optim   found_inf, adam_step, loss_scale_update, cast_to_16, grad_norm,
           clip_coefficient, accumulate
@@ -31,11 +32,13 @@ choice and cannot be pinned to the pages: parity unpinned for those choices
 themselves, while the code that implements them is pinned.
 """
 from .layer import (layer_fwd, layer_bwd, layer_norm_fwd, layer_norm_bwd, gelu,
-                    gelu_prime, causal_softmax, attention_head_fwd, stack_fwd, stack_bwd)
+                    gelu_prime, causal_softmax, attention_head_fwd, attention_head_bwd,
+                    stack_fwd, stack_bwd, STORE_POINTS)
 from .optim import (found_inf, adam_step, loss_scale_update, cast_to_16, grad_norm,
                     clip_coefficient, accumulate)
 
 __all__ = ["layer_fwd", "layer_bwd", "stack_fwd", "stack_bwd", "layer_norm_fwd", "layer_norm_bwd", "gelu",
-           "gelu_prime", "causal_softmax", "attention_head_fwd", "found_inf",
+           "gelu_prime", "causal_softmax", "attention_head_fwd", "attention_head_bwd",
+           "STORE_POINTS", "found_inf",
            "adam_step", "loss_scale_update", "cast_to_16", "grad_norm", "clip_coefficient",
            "accumulate"]

@@ -94,25 +94,60 @@ def causal_softmax(z: np.ndarray) -> np.ndarray:
     return p
 
 
-def attention_head_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, precision=None, noise=None):
+def attention_head_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, precision=None, noise=None,
+                       noise_at=None):
     """One (batch, head) block of causal self-attention: returns (P, O).
-    With a 16-bit precision P is a stored (rounded) value."""
+    With a 16-bit precision P is a stored (rounded) value; O is returned
+    unrounded (the layer stores it)."""
     d = q.shape[1]
     z = (q @ k.T) / math.sqrt(d)
-    p = _store(causal_softmax(z), precision, noise)
+    p = _store(causal_softmax(z), precision, noise, "p", noise_at)
     return p, p @ v
 
 
-def _store(a: np.ndarray, precision, noise=None):
+def attention_head_bwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, p: np.ndarray,
+                       do: np.ndarray, o: np.ndarray, precision=None, noise=None, noise_at=None):
+    """Backward of one (batch, head) block of causal self-attention, given
+    its probabilities P (as attention_head_fwd returns them), the output
+    gradient dO and the output O.  Returns (dQ, dK, dV).
+
+    dP = dO V^T; dV = P^T dO; dZ = P (dP - r) with the row term
+    r_p = sum_q P_pq dP_pq; dS = dZ / sqrt(d); dQ = dS K; dK = dS^T Q.  In
+    the mixed-precision mode dV, dS (the operand of both products), dQ and dK
+    are stored, and the row term is formed as dO_p . O_p from the stored dO
+    and O (equal in exact arithmetic, since O = P V); dP stays exact, as the
+    fused kernel keeps it on chip."""
+    st = lambda a, name: _store(a, precision, noise, name, noise_at)
+    d = q.shape[1]
+    dp = do @ v.T
+    dv = st(p.T @ do, "dv")
+    if precision is None:
+        rowterm = (p * dp).sum(axis=1, keepdims=True)
+    else:
+        rowterm = (do * o).sum(axis=1, keepdims=True)
+    dsc = st((p * (dp - rowterm)) * (1.0 / math.sqrt(d)), "ds")
+    return st(dsc @ k, "dq"), st(dsc.T @ q, "dk"), dv
+
+
+# The tensors the mixed-precision mode holds in the 16-bit type, by name, in
+# the order the step produces them (see the module doc).
+FWD_STORE_POINTS = ("l1", "c", "p", "o", "l2", "z", "act")
+BWD_STORE_POINTS = ("dz", "dl2", "dh16", "do", "dv", "ds", "dq", "dk", "dl1")
+STORE_POINTS = FWD_STORE_POINTS + BWD_STORE_POINTS
+
+
+def _store(a: np.ndarray, precision, noise=None, name=None, noise_at=None):
     """An activation tensor as the next step reads it (see the module doc).
     `noise`, when given, is applied to the value just before it is rounded:
     a callable that returns the value times (1 + a small relative error),
     standing for the rounding of a fp32-accumulating implementation, so that
     a test can measure how far two correct implementations of the 16-bit
-    method drift apart."""
+    method drift apart.  `noise_at`, a set of store-point names, limits the
+    noise to those stores (None: every store)."""
+    assert name in STORE_POINTS, name
     if precision is None:
         return a
-    if noise is not None:
+    if noise is not None and (noise_at is None or name in noise_at):
         a = noise(a)
     return round_to_16(a, precision)
 
@@ -128,11 +163,14 @@ def _check(dims, params):
 
 
 def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precision=None,
-              noise=None):
+              noise=None, noise_at=None):
     """Forward pass.  x: [T, h] float64.  precision: None (exact) or the
-    16-bit type the activations are stored in; noise: see _store.
+    16-bit type the activations are stored in; noise, noise_at: see _store
+    (both are kept in the cache for the backward pass).
     Returns (out, cache)."""
-    st = lambda a: _store(a, precision, noise)
+    st = lambda a, name: _store(a, precision, noise, name, noise_at)
+    if noise_at is not None:
+        assert set(noise_at) <= set(STORE_POINTS), noise_at
     b, s, h, a, f, t = _check(dims, params)
     d = h // a
     hs, a_s = h // t, a // t            # hidden columns and heads per shard
@@ -141,10 +179,10 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precis
 
     # 1. LN1
     l1, mu1, rstd1, xhat1 = layer_norm_fwd(x, params["ln1_g"], params["ln1_b"], eps)
-    l1 = st(l1)
+    l1 = st(l1, "l1")
 
     # 2. QKV column-split GEMM: C_i = L1 W_qkv,i^T + b_qkv,i  -> [Q_i | K_i | V_i]
-    c = st(np.stack([l1 @ params["w_qkv"][i].T + params["b_qkv"][i][None, :] for i in range(t)]))
+    c = st(np.stack([l1 @ params["w_qkv"][i].T + params["b_qkv"][i][None, :] for i in range(t)]), "c")
 
     # 3. causal attention, head by head; head eta of shard i is global head i*a/t+eta
     probs = np.zeros((t, b, a_s, s, s))
@@ -157,9 +195,9 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precis
                 qh = c[i, rows, 0 * hs:1 * hs][:, cols]
                 kh = c[i, rows, 1 * hs:2 * hs][:, cols]
                 vh = c[i, rows, 2 * hs:3 * hs][:, cols]
-                pr, oh = attention_head_fwd(qh, kh, vh, precision, noise)
+                pr, oh = attention_head_fwd(qh, kh, vh, precision, noise, noise_at)
                 probs[i, j, eta] = pr
-                o[i, rows, cols] = st(oh)
+                o[i, rows, cols] = st(oh, "o")
 
     # 4. out-projection, row split: partial products summed over shards, bias
     #    added once after the sum, then the residual
@@ -170,11 +208,11 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precis
 
     # 5. LN2
     l2, mu2, rstd2, xhat2 = layer_norm_fwd(hid, params["ln2_g"], params["ln2_b"], eps)
-    l2 = st(l2)
+    l2 = st(l2, "l2")
 
     # 6. FFN1 column split with fused bias + GeLU
-    z = st(np.stack([l2 @ params["w_1"][i].T + params["b_1"][i][None, :] for i in range(t)]))
-    act = st(gelu(z))
+    z = st(np.stack([l2 @ params["w_1"][i].T + params["b_1"][i][None, :] for i in range(t)]), "z")
+    act = st(gelu(z), "act")
 
     # 7. FFN2 row split: shard sum, bias, residual
     y_mlp = np.zeros((T, h))
@@ -184,19 +222,22 @@ def layer_fwd(x: np.ndarray, params: dict, dims: dict, eps: float = 1e-5, precis
 
     cache = dict(x=x, l1=l1, mu1=mu1, rstd1=rstd1, xhat1=xhat1, c=c, probs=probs, o=o,
                  hid=hid, l2=l2, mu2=mu2, rstd2=rstd2, xhat2=xhat2, z=z, act=act,
-                 precision=precision, noise=noise)
+                 precision=precision, noise=noise, noise_at=noise_at)
     return out, cache
 
 
-def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
+def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray, keep: dict = None):
     """Backward pass given dOut (already multiplied by the loss scale).
-    Returns (dx, grads) with grads in the same shard-major layout as params."""
+    Returns (dx, grads) with grads in the same shard-major layout as params.
+    When `keep` is a dict, the backward's intermediate tensors are left in it
+    (dz, dl2, dh, dh16, do, dc, dl1), so that a test can check each stored
+    tensor against its step recomputed from the stored inputs."""
     b, s, h, a, f, t = _check(dims, params)
     d = h // a
     hs, a_s = h // t, a // t
     T = b * s
-    inv_sqrt_d = 1.0 / math.sqrt(d)
-    st = lambda a: _store(a, cache.get("precision"), cache.get("noise"))
+    precision, noise, noise_at = cache.get("precision"), cache.get("noise"), cache.get("noise_at")
+    st = lambda a, name: _store(a, precision, noise, name, noise_at)
     gr = {}
 
     # FFN2 (row split): each shard's weight gradient and input gradient
@@ -206,24 +247,24 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
 
     # GeLU backward and FFN1 (column split); the input gradient is the sum
     # of the shards' partial products
-    dz = st(d_act * gelu_prime(cache["z"]))
+    dz = st(d_act * gelu_prime(cache["z"]), "dz")
     gr["b_1"] = dz.sum(axis=1)
     gr["w_1"] = np.stack([dz[i].T @ cache["l2"] for i in range(t)])
     dl2 = np.zeros((T, h))
     for i in range(t):
         dl2 += dz[i] @ params["w_1"][i]
-    dl2 = st(dl2)
+    dl2 = st(dl2, "dl2")
 
     # LN2 backward plus the residual path
     dln, gr["ln2_g"], gr["ln2_b"] = layer_norm_bwd(dl2, cache["xhat2"], cache["rstd2"],
                                                    params["ln2_g"])
     dhid = dout + dln
-    dhid16 = st(dhid)                   # the matrix operand copy of dH
+    dhid16 = st(dhid, "dh16")           # the matrix operand copy of dH
 
     # out-projection (row split)
     gr["b_o"] = dhid.sum(axis=0)
     gr["w_o"] = np.stack([dhid16.T @ cache["o"][i] for i in range(t)])
-    do = st(np.stack([dhid16 @ params["w_o"][i] for i in range(t)]))
+    do = st(np.stack([dhid16 @ params["w_o"][i] for i in range(t)]), "do")
 
     # attention backward, head by head
     c = cache["c"]
@@ -238,16 +279,8 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
                 vh = c[i, rows, 2 * hs:3 * hs][:, cols]
                 pr = cache["probs"][i, j, eta]
                 doh = do[i, rows, cols]
-                dp = doh @ vh.T
-                dv = st(pr.T @ doh)
-                if cache.get("precision") is None:
-                    rowterm = (pr * dp).sum(axis=1, keepdims=True)
-                else:
-                    rowterm = (doh * cache["o"][i, rows, cols]).sum(axis=1, keepdims=True)
-                dzs = pr * (dp - rowterm)
-                dsc = st(dzs * inv_sqrt_d)
-                dq = st(dsc @ kh)
-                dk = st(dsc.T @ qh)
+                dq, dk, dv = attention_head_bwd(qh, kh, vh, pr, doh, cache["o"][i, rows, cols],
+                                                precision, noise, noise_at)
                 dc[i, rows, 0 * hs:1 * hs][:, cols] = dq
                 dc[i, rows, 1 * hs:2 * hs][:, cols] = dk
                 dc[i, rows, 2 * hs:3 * hs][:, cols] = dv
@@ -258,12 +291,14 @@ def layer_bwd(cache: dict, params: dict, dims: dict, dout: np.ndarray):
     dl1 = np.zeros((T, h))
     for i in range(t):
         dl1 += dc[i] @ params["w_qkv"][i]
-    dl1 = st(dl1)
+    dl1 = st(dl1, "dl1")
 
     # LN1 backward plus the residual path
     dln1, gr["ln1_g"], gr["ln1_b"] = layer_norm_bwd(dl1, cache["xhat1"], cache["rstd1"],
                                                     params["ln1_g"])
     dx = dhid + dln1
+    if keep is not None:
+        keep.update(dz=dz, dl2=dl2, dh=dhid, dh16=dhid16, do=do, dc=dc, dl1=dl1)
     return dx, gr
 
 
