@@ -1,11 +1,17 @@
 #!/usr/bin/env python
 """Throughput of one GPT transformer layer's training step on B200.
 
-One step = gpt_layer_fwd + gpt_layer_bwd + adam_step_fp32_master +
-loss_scale_update through the C ABI of libgptlayer.so, on one CUDA stream,
-for the GPT-2 117M layer shape (hidden 768, 12 heads, ffn 3072, seq 1024,
-micro-batch 8, tp 1, bf16 compute with fp32 master weights, initial loss
-scale 2^16) on synthetic seeded inputs.
+One step = gpt_layer_fwd + gpt_layer_bwd_checked +
+adam_step_fp32_master_prechecked + loss_scale_update through the C ABI of
+libgptlayer.so, on one CUDA stream (the overflow check of the dynamic loss
+scaling made by the kernels that write the gradients; --scan-overflow uses
+gpt_layer_bwd + adam_step_fp32_master, whose check re-reads the arena),
+by default for the hidden-10240 layer of the Megatron-LM 3D-parallelism
+example (hidden 10240, 80 heads of 128, ffn 40960, seq 2048, micro-batch 1,
+tp 4 sharded on one GPU, bf16 compute with fp32 master weights, weights
+N(0, 0.006), initial loss scale 2^16), the largest of the pages' GPT layer
+shapes, on synthetic seeded inputs.  --workload picks another shape (the
+GPT-2 117M / 345M layers, the 2.4B model's layer, the tiny layer).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -17,9 +23,11 @@ per-step events, max over ranks.  Several GPUs run independent replicas
 
 Also reported: `e2e` (the same step with the inputs copied from pinned host
 memory and the output read back inside the timed region), the roofline of
-the dominant kernel (the tcgen05 GEMM: algorithmic FLOPs over its launches'
-summed device time, from per-launch events recorded by the library in a
-second timed pass), a per-kernel breakdown, SM clocks sampled during the
+the dominant kernel (the one with the largest share of the step's device
+time, from per-launch events recorded by the library in a second timed
+pass: the tcgen05 GEMM at the default shape, its algorithmic FLOPs over its
+launches' summed time), the same figures for every kernel family
+(`roofline_by_kernel`), a per-kernel breakdown, SM clocks sampled during the
 timed region, and `cpu_baseline`, the float64 CPU oracle timed on a bounded
 sample of the same workload on this host's cores.
 
@@ -49,7 +57,7 @@ from transformer_layer_step_b200 import synth  # noqa: E402
 
 METRIC = "GPT layer fwd+bwd+Adam tokens/sec at 1 B200"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "gpt2-117m"
+DEFAULT_WORKLOAD = "large-h10240"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = ("transformer_layer_step_b200/csrc/gemm_tc.cuh",
@@ -71,26 +79,70 @@ def step_flops(cfg) -> dict:
     attn_causal = 2 * 2 * b * h * (s * (s + 1) // 2)     # QK^T and PV over the triangle
     attn_dense = 2 * 2 * b * h * s * s
     return {"causal": 3 * (linear + attn_causal), "dense": 3 * (linear + attn_dense),
-            "linear": 3 * linear}
+            "linear": 3 * linear, "attn_fwd": attn_causal, "attn_bwd": 2 * attn_causal}
 
 
-def kernel_bytes(cfg, n_params: int) -> dict:
-    """Algorithmic HBM bytes per launch of each bandwidth kernel of the step
-    (2-byte activations, 4-byte fp32 state)."""
+def kernel_bytes(cfg, n_params: int, layers: int = 1) -> dict:
+    """Algorithmic HBM bytes of each bandwidth kernel of the step, summed over
+    its launches in one step (2-byte activations, 4-byte fp32 state; a stack
+    of `layers` layers launches each per-layer kernel once per layer; the
+    optimizer's n_params covers every layer)."""
     b, s, h, a, f = cfg.batch, cfg.seq, cfg.hidden, cfg.heads, cfg.ffn
     T = b * s
     # the residual stream H and its gradient dH are fp32 (4 B), the rest 2 B
-    return {
+    per_layer = {
         "F1 ln1": 4 * T * h,                                  # read x, write L1
         "F7 ln2": 6 * T * h,                                  # read H (fp32), write L2
         "B6 ln2 bwd": 14 * T * h,   # read dL2, H (fp32), dOut; write dH (16-bit and fp32)
         "B12 ln1 bwd": 10 * T * h,  # read dL1, X, dH (fp32); write dX
         "B9 rowdot": 4 * T * h,                               # read dO and O
+        "B0 weights^T": 4 * (4 * h * h + 2 * h * f),          # the four weight matrices
         "B2 dOut^T": 4 * T * h, "B5 L2^T": 4 * T * h,         # transposes: read + write
         "B7 dH^T": 4 * T * h, "B11 L1^T": 4 * T * h,
         "B3 db1": 2 * T * f, "B11 dbqkv": 2 * T * 3 * h,
-        "O1 overflow": 4 * n_params, "O2 adam": 30 * n_params,
     }
+    out = {k: v * layers for k, v in per_layer.items()}
+    out.update({"O1 overflow": 4 * n_params, "O2 adam": 30 * n_params})
+    return out
+
+
+def kernel_rooflines(kinds: dict, rows: list, cfg, n_params: int, flops: dict, peaks: dict,
+                     peak_src: str, layers: int = 1) -> dict:
+    """Achieved rate against the roofline of every kernel family of the
+    step, per step: the tensor-core families (the GEMM with its split-K sums,
+    the attention forward and backward) as algorithmic FLOPs over their
+    summed launch time against the measured bf16 GEMM rate (sustained: they
+    are timed inside a long step), the bandwidth families as algorithmic
+    bytes (kernel_bytes, summed over the step's launches of the family) over
+    their time against the measured copy bandwidth."""
+    def ms(*names):
+        return sum(kinds.get(k, {}).get("ms_per_step", 0.0) for k in names)
+
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    hbm = peaks["hbm_gbs"]
+    out = {}
+    for fam, names, work in (("gemm", ("gemm", "splitk"), flops["linear"]),
+                             ("attn_fwd", ("attn_fwd",), flops["attn_fwd"]),
+                             ("attn_bwd", ("attn_bwd", "rowdot"), flops["attn_bwd"])):
+        t = ms(*names)
+        if t > 0:
+            a = work / (t * 1e-3) / 1e12
+            out[fam] = {"bound": "tensor", "ms_per_step": round(t, 5), "achieved": round(a, 1),
+                        "peak": peak_tf, "unit": "TFLOP/s", "frac": round(a / peak_tf, 4),
+                        "peak_source": f"{peak_src} bf16_tflops_sustained"}
+    nbytes = kernel_bytes(cfg, n_params, layers)
+    for row in rows:
+        if row["step"] not in nbytes or row["kind"] in ("gemm", "splitk", "attn_fwd", "attn_bwd"):
+            continue
+        fam = out.setdefault(row["kind"], {"bound": "hbm", "ms_per_step": 0.0, "bytes": 0})
+        fam["ms_per_step"] += row["ms_per_step"]
+        fam["bytes"] += nbytes[row["step"]]
+    for fam in out.values():
+        if fam["bound"] == "hbm" and fam["ms_per_step"] > 0:
+            a = fam["bytes"] / (fam["ms_per_step"] * 1e-3) / 1e9
+            fam.update(ms_per_step=round(fam["ms_per_step"], 5), achieved=round(a, 1), peak=hbm,
+                       unit="GB/s", frac=round(a / hbm, 4), peak_source=f"{peak_src} hbm_gbs")
+    return out
 
 
 def load_peaks() -> tuple[dict, str]:
@@ -118,19 +170,29 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per GEMM launch-set from the committed ncu summary, or None
-    when the summary is absent or the kernels changed since it was taken."""
+# the kernels behind each family name of kernel_rooflines
+DOMINANT_KERNELS = {
+    "gemm": "gemm_tc_kernel (the tcgen05 GEMM; its split-K sums included)",
+    "attn_fwd": "attn_fwd_kernel", "attn_bwd": "attn_bwd_dq_kernel + attn_bwd_kv_kernel (+ row term)",
+    "adam": "adam_kernel", "overflow": "overflow_kernel",
+}
+
+
+def recorded_traffic(workload: str, family: str):
+    """DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
+    step's launches of a kernel family, from the committed ncu summary
+    (profiles/traffic.json), or None when it is absent or the kernels
+    changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as fh:
             rec = json.load(fh)
     except (OSError, ValueError):
         return None
-    ent = rec.get(workload)
+    ent = rec.get(workload, {}).get(family)
     if not ent or ent.get("kernel_sources") != kernel_source_hash():
         return None
-    return ent.get("gemm_dram_bytes_per_step")
+    return ent.get("dram_bytes_per_step")
 
 
 # ------------------------------------------------------------ clock sampler
@@ -201,6 +263,24 @@ def blas_threads() -> int:
         return 1
 
 
+def sample_plan(cfg, seconds: float) -> tuple[int, int | None]:
+    """Size of a bounded oracle sample: (sequences, position prefix or None)
+    whose fwd + bwd + Adam takes about `seconds` on a 16-core host, from a
+    rough cost model of the float64 oracle measured on the GPT-2 117M and
+    2.4B shapes: ~2 us per token and hidden unit of element-wise work and
+    16-bit rounding, ~2e11 FLOP/s in the BLAS products, ~20 ns per parameter
+    in the optimizer step over the same fraction of the arena.  At least 64
+    positions of one sequence."""
+    h, f, s = cfg.hidden, cfg.ffn, cfg.seq
+    n_params = 12 * h * h + 13 * h
+    per_token = (2e-6 * h + 3 * 2 * (4 * h * h + 2 * h * f) / 2e11
+                 + n_params / cfg.tokens * 2e-8)
+    tokens = int(seconds / per_token)
+    if tokens >= s:
+        return max(1, min(cfg.batch, tokens // s)), None
+    return 1, max(64, tokens // 64 * 64)
+
+
 def oracle_sample(cfg, n_seq: int, seq_prefix: int | None = None, repeats: int = 1) -> dict:
     """Times the oracle (test infrastructure, float64 numpy) on a bounded
     sample of the workload: fwd + bwd of `n_seq` of the step's sequences
@@ -265,12 +345,18 @@ def run_ours(args, cfg, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from transformer_layer_step_b200 import gptlayer as G
-    from transformer_layer_step_b200.harness import LayerStep
+    from transformer_layer_step_b200.harness import LayerStack, LayerStep
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     inp = synth.make_inputs(cfg, seed=rank, variant="biased", with_r=True)
-    ls = LayerStep(cfg, inp, device=dev)
+    stack = args.layers > 1
+    if stack:
+        # L layers of the shape, each starting from the same seeded weights,
+        # with parameters of their own in one arena, and one Adam over all
+        ls = LayerStack(cfg, [inp["params"]] * args.layers, inp["x"], device=dev)
+    else:
+        ls = LayerStep(cfg, inp, device=dev)
     dy_bits = synth.loss_grad_bits(cfg, ls.hyper["init_scale"], inp["r"])
     ls.set_dy_bits(dy_bits)
     stream = torch.cuda.current_stream(dev)
@@ -294,8 +380,13 @@ def run_ours(args, cfg, rank, world, local_rank):
             flush.zero_()
         return ev
 
+    fused = not args.scan_overflow and not stack
+
+    def step(**kw):
+        ls.step(fused_check=fused, **kw)
+
     for _ in range(W):
-        ls.step()
+        step()
         flush.zero_()
     torch.cuda.synchronize()
     if G.read_device_error(clear=True):
@@ -304,14 +395,14 @@ def run_ours(args, cfg, rank, world, local_rank):
     # ---- the step as a CUDA graph (captured after the warm-up, which set the
     # kernels' shared-memory opt-ins): one launch of the graph per step, so no
     # host launch latency between the step's kernels
-    step_fn = ls.step
+    step_fn = step
     graph = None
     graph_launches = 0
     if not args.no_graph:
         n0 = G.launch_count()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            ls.step()
+            step()
         graph_launches = G.launch_count() - n0
         for _ in range(2):
             graph.replay()
@@ -337,7 +428,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     # ---- per-launch device times (second pass, library events between launches)
     per_step = launches // K
     G.profile_begin(per_step * K + 16)
-    timed_steps(K, ls.step)
+    timed_steps(K, step)
     recs, dropped = G.profile_end(per_step * K + 16)
     if dropped:
         raise RuntimeError(f"{dropped} launches were not timed")
@@ -375,7 +466,11 @@ def run_ours(args, cfg, rank, world, local_rank):
             copied[b].record(h2d_stream)
 
     def compute(b):
-        ls.step(x=xb[b], dy=dyb[b], y=yb[b])
+        if stack:                 # the stack writes its output into its last activation
+            step(x=xb[b], dy=dyb[b])
+            yb[b].copy_(ls.y, non_blocking=True)
+        else:
+            step(x=xb[b], dy=dyb[b], y=yb[b])
         stb[b].copy_(ls.state, non_blocking=True)
 
     # one CUDA graph per buffer set replays the step (--e2e-eager: kernel by kernel)
@@ -425,7 +520,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     if G.read_device_error(clear=True):
         raise RuntimeError("device error word set during the timed steps")
     sc = ls.scaler()
-    ext = measure_extensions(G, ls, cfg, dev, flush, peaks=load_peaks()[0])
+    # (a stack's arena is too large for the extensions' copies of the state)
+    ext = None if stack else measure_extensions(G, ls, cfg, dev, flush, peaks=load_peaks()[0])
     h2d = x_host.numel() * x_host.element_size() + dy_host.numel() * dy_host.element_size()
     d2h = y_host.numel() * y_host.element_size() + st_host.numel() * st_host.element_size()
     return dict(ms_per_step=ms_per_step, step_ms=step_ms, launches=launches, recs=recs,
@@ -482,7 +578,7 @@ def measure_extensions(G, ls, cfg, dev, flush, peaks, reps=5):
     }
 
 
-def summarize_kernels(recs, K, cfg, n_params, peaks, flops):
+def summarize_kernels(recs, K, cfg, n_params, peaks, flops, layers=1):
     """Per-kernel device time per step, share, and achieved rate."""
     by_tag, by_kind = {}, {}
     for kind, tag, ms in recs:
@@ -493,7 +589,7 @@ def summarize_kernels(recs, K, cfg, n_params, peaks, flops):
         k["launches"] += 1
         k["ms"] += ms
     total = sum(e["ms"] for e in by_kind.values())
-    nbytes = kernel_bytes(cfg, n_params)
+    nbytes = kernel_bytes(cfg, n_params, layers)
     rows = []
     for tag, e in by_tag.items():
         ms = e["ms"] / K
@@ -508,10 +604,105 @@ def summarize_kernels(recs, K, cfg, n_params, peaks, flops):
     return rows, kinds, total / K
 
 
+# ------------------------------------------------------- single-kernel cases
+CASES = ("gemm-ffn2", "gemm-dw1", "attention", "layernorm", "adam")
+
+
+def run_case(args, cfg):
+    """One launch (or launch pair) of one kernel family at this workload's
+    shapes, holding at most a few GB on the device, for a profiler capture of
+    that kernel alone: the tcgen05 GEMM as the FFN2 product (row split, shard
+    sum in the K loop, bias + fp32 residual epilogue) or as the FFN1 weight
+    gradient (fp32 output, token reduction), the fused attention forward and
+    backward, the LayerNorm forward and backward, or the optimizer step (the
+    overflow check and Adam) over 64 M parameters.  Runs the case `warmup`
+    times, then once more between CUDA events, and prints the time."""
+    import torch
+    from transformer_layer_step_b200 import gptlayer as G
+    torch.cuda.set_device(0)
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float16
+    T, h, f, t = cfg.tokens, cfg.hidden, cfg.ffn, cfg.tp
+    fs, hs = f // t, h // t
+    st = torch.cuda.current_stream().cuda_stream
+    rnd = lambda *shape, std=1.0: (torch.randn(*shape, device="cuda") * std).to(tdt)
+    if args.case == "gemm-ffn2":          # Out = H + sum_i A_i W2_i^T + b2
+        a, w = rnd(t, T, fs), rnd(t, h, fs, std=0.02)
+        hid = torch.randn(T, h, device="cuda")
+        b2, out = rnd(h), torch.empty(T, h, dtype=tdt, device="cuda")
+        d = G.GemmDesc()
+        d.M, d.N, d.K, d.groups, d.k_shards = T, h, fs, 1, t
+        d.a = G.operand(a, fs, T, t, fs, T * fs, g_div=1 << 30, k_shard=1)
+        d.b = G.operand(w, fs, h, t, fs, h * fs, g_div=1 << 30, k_shard=1)
+        d.out, d.ldo, d.o_mod = out.data_ptr(), h, 1
+        d.bias, d.resid, d.ld_resid, d.resid_f32 = b2.data_ptr(), hid.data_ptr(), h, 1
+        work = lambda: G.gemm(d, cfg.dtype, st)
+        flops = 2.0 * T * h * f
+    elif args.case == "gemm-dw1":         # dW1_i = dZ_i^T L2   [t][f/t][h] fp32
+        dz, l2t = rnd(t, T, fs), rnd(h, T)
+        out = torch.empty(t, fs, h, dtype=torch.float32, device="cuda")
+        ws = torch.empty(64 << 20, dtype=torch.uint8, device="cuda")
+        d = G.GemmDesc()
+        d.M, d.N, d.K, d.groups, d.k_shards = fs, h, T, t, 1
+        d.a = G.operand(dz, fs, T, t, fs, T * fs, mn_major=1)
+        d.b = G.operand(l2t, T, h, 1, T)
+        d.out, d.out_f32, d.ldo, d.o_mod, d.o_str_div = out.data_ptr(), 1, h, 1, fs * h
+        d.ws, d.ws_bytes = ws.data_ptr(), 64 << 20
+        work = lambda: G.gemm(d, cfg.dtype, st)
+        flops = 2.0 * T * h * f
+    elif args.case == "attention":
+        as_ = cfg.heads // t
+        c = rnd(t, T, 3 * hs)
+        o, do = torch.empty(t, T, hs, dtype=tdt, device="cuda"), rnd(t, T, hs)
+        lse = torch.empty(t * cfg.batch * as_, cfg.seq, device="cuda")
+        dvec, dc = torch.empty_like(lse), torch.empty_like(c)
+
+        def work():
+            G.attention_fwd(cfg.batch, cfg.seq, h, cfg.heads, t, cfg.dtype, c, o, lse, st)
+            G.attention_bwd(cfg.batch, cfg.seq, h, cfg.heads, t, cfg.dtype, c, o, do, lse, dvec,
+                            dc, st)
+        flops = 3 * 2 * 2 * cfg.batch * h * (cfg.seq * (cfg.seq + 1) // 2)
+    elif args.case == "layernorm":
+        x, gy, res = rnd(T, h), rnd(T, h), rnd(T, h)
+        g, b = rnd(h), rnd(h)
+        y, dx = torch.empty_like(x), torch.empty_like(x)
+        mu, rs = torch.empty(T, device="cuda"), torch.empty(T, device="cuda")
+        dg, db, dsum = (torch.empty(h, device="cuda") for _ in range(3))
+        scr = torch.empty(G.layernorm_bwd_scratch_bytes(T, h), dtype=torch.uint8, device="cuda")
+
+        def work():
+            G.layernorm_fwd(T, h, cfg.dtype, x, g, b, 1e-5, y, mu, rs, st)
+            G.layernorm_bwd(T, h, cfg.dtype, gy, x, mu, rs, g, res, dx, dg, db, dsum, scr, st)
+        flops = 0.0
+    else:                                 # adam: overflow check + Adam over 64 M parameters
+        n = 64 << 20
+        p32, m, v, g = (torch.randn(n, device="cuda") * 0.02 for _ in range(4))
+        w16 = torch.empty(n, dtype=tdt, device="cuda")
+        state = torch.zeros(8, dtype=torch.int32, device="cuda")
+        state[0] = int(np.array([65536.0], np.float32).view(np.int32)[0])
+        work = lambda: G.adam_step(n, p32, m, v, g, w16, cfg.dtype, 6e-5, 0.9, 0.95, 1e-8, 0.0,
+                                   state, st)
+        flops = 0.0
+    for _ in range(args.warmup):
+        work()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    work()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if G.read_device_error(clear=True):
+        raise RuntimeError("device error word set")
+    line = {"case": args.case, "workload": cfg.name, "ms": round(ms, 4)}
+    if flops:
+        line["TFLOP/s"] = round(flops / (ms * 1e-3) / 1e12, 1)
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.CONFIGS))
@@ -519,8 +710,18 @@ def main():
                     help="launch the step's kernels one by one instead of as a CUDA graph")
     ap.add_argument("--e2e-eager", action="store_true",
                     help="launch the end-to-end steps kernel by kernel instead of as CUDA graphs")
+    ap.add_argument("--scan-overflow", action="store_true",
+                    help="check the gradients for inf/NaN in a separate pass over the arena "
+                         "(gpt_layer_bwd + adam_step_fp32_master) instead of in the kernels "
+                         "that write them (gpt_layer_bwd_checked + adam_step_fp32_master_prechecked)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the CPU oracle timing (it runs on rank 0 at N=1 only)")
+    ap.add_argument("--layers", type=int, default=1,
+                    help="a stack of this many layers of the workload's shape per step "
+                         "(gpt_stack_fwd / gpt_stack_bwd and one Adam over every layer)")
+    ap.add_argument("--case", choices=CASES,
+                    help="run one kernel family once at this workload's shapes (a small "
+                         "device footprint for a profiler capture) instead of the benchmark")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -532,18 +733,30 @@ def main():
               "hidden": cfg.hidden, "heads": cfg.heads, "ffn": cfg.ffn, "tp": cfg.tp,
               "tokens_per_step": cfg.tokens, "parallelism": f"replicas{world}",
               "step_launch": "kernel by kernel" if args.no_graph else "one CUDA graph per step",
+              "overflow_check": ("a separate pass over the gradient arena" if args.scan_overflow
+                                 else "in the kernels that write the gradients"),
               "e2e_step_launch": "kernel by kernel" if args.e2e_eager else "one CUDA graph per step",
               "e2e_copies": "one stream per direction, overlapped with the neighbouring steps",
               "l2": "flushed between steps (256 MiB write, outside the per-step events)"}
-    flops = step_flops(cfg)
+    L = args.layers
+    if L < 1:
+        ap.error("--layers must be at least 1")
+    if L > 1:
+        config.update(layers=L, workload=f"{cfg.name} x{L} layers",
+                      overflow_check="a separate pass over the gradient arena")
+    flops = {k: L * v for k, v in step_flops(cfg).items()}
+
+    if args.case:
+        run_case(args, cfg)
+        return
 
     if args.impl == "reference":
         if rank != 0:
             return
-        n = args.steps + args.warmup
-        prefix = None if n <= 30 else max(64, (cfg.seq * 30 // n) // 64 * 64)
-        oracle_sample(cfg, 1, prefix, repeats=args.warmup)
-        r = oracle_sample(cfg, 1, prefix, repeats=args.steps)
+        # every step a bounded sample: the whole run about two minutes of CPU work
+        n_seq, prefix = sample_plan(cfg, 120.0 / (args.steps + args.warmup))
+        oracle_sample(cfg, n_seq, prefix, repeats=args.warmup)
+        r = oracle_sample(cfg, n_seq, prefix, repeats=args.steps)
         cores = blas_threads()
         line = {"impl": "reference", "metric": METRIC, "value": round(r["value"], 3),
                 "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -566,15 +779,21 @@ def main():
     res = run_ours(args, cfg, rank, world, local_rank)
     peaks, peak_src = load_peaks()
     rows, kinds, prof_ms = summarize_kernels(res["recs"], args.steps, cfg, res["n_params"],
-                                             peaks, flops)
-    # the tensor-core kernels: every GEMM launch (with its split-K sums) and
-    # the fused attention forward; the work is the step's algorithmic FLOPs
-    # (the backward's recomputation of S and dP is not counted)
-    gemm_ms = sum(kinds.get(k, {}).get("ms_per_step", 0.0)
-                  for k in ("gemm", "splitk", "attn_fwd", "attn_bwd"))
+                                             peaks, flops, L)
+    by_kernel = kernel_rooflines(kinds, rows, cfg, res["n_params"], flops, peaks, peak_src, L)
+    dom_name = max(by_kernel, key=lambda k: by_kernel[k]["ms_per_step"])
+    dom = by_kernel[dom_name]
     peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    achieved_tf = flops["causal"] / (gemm_ms * 1e-3) / 1e12 if gemm_ms else None
-    traffic = recorded_traffic(cfg.name)
+    traffic = recorded_traffic(cfg.name, dom_name) if L == 1 else None
+    roofline = {"kernel": DOMINANT_KERNELS.get(dom_name, dom_name), "bound": dom["bound"],
+                "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
+                "frac": dom["frac"], "peak_source": dom["peak_source"],
+                "unit_of_work": "one layer step's launches of the kernel",
+                "work": ("algorithmic FLOPs of the step's twelve linear-layer products (causal "
+                         "attention excluded)" if dom_name == "gemm" else
+                         "algorithmic work of the step's launches of the kernel"),
+                "share_of_step": round(dom["ms_per_step"] / prof_ms, 4) if prof_ms else None,
+                "traffic": traffic}
     ms = res["ms_per_step"]
     value = whole_job_tokens_per_s(world, cfg.tokens, ms)
     line = {
@@ -585,15 +804,8 @@ def main():
         "tflops_causal": round(flops["causal"] / (ms * 1e-3) / 1e12, 1),
         "tflops_dense_convention": round(flops["dense"] / (ms * 1e-3) / 1e12, 1),
         "frac_of_bf16_peak": round(flops["causal"] / (ms * 1e-3) / 1e12 / peak_tf, 4),
-        "roofline": {"kernel": "tcgen05 kernels of a step: gemm_tc_kernel (with split-K sums), "
-                               "attn_fwd_kernel, attn_bwd_dq_kernel, attn_bwd_kv_kernel",
-                     "bound": "tensor",
-                     "achieved": round(achieved_tf, 1) if achieved_tf else None,
-                     "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": round(achieved_tf / peak_tf, 4) if achieved_tf else None,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained",
-                     "work": "causal algorithmic FLOPs of the step's contractions",
-                     "traffic": traffic},
+        "roofline": roofline,
+        "roofline_by_kernel": by_kernel,
         "kernels": kinds,
         "steps_detail": sorted(rows, key=lambda r: -r["ms_per_step"]),
         "profiled_ms_per_step": round(prof_ms, 4),
@@ -605,10 +817,13 @@ def main():
         "optimizer_extensions": res["ext"],
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        r = oracle_sample(cfg, 4)          # about 10 s of float64 CPU work
-        line["cpu_baseline"] = {"value": round(r["value"], 3), "unit": UNIT,
+        r = oracle_sample(cfg, *sample_plan(cfg, 10.0))   # about 10 s of float64 CPU work
+        # a stack runs its layers one after another: one layer's oracle time, L times
+        line["cpu_baseline"] = {"value": round(r["value"] / L, 3), "unit": UNIT,
                                 "cores": blas_threads(), "kind": "oracle",
-                                "sample": r["sample"], "seconds": round(sum(r["seconds"]), 2)}
+                                "sample": r["sample"] + (f"; one layer timed, the stack taken as "
+                                                         f"{L} such layers" if L > 1 else ""),
+                                "seconds": round(sum(r["seconds"]), 2)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -106,7 +106,8 @@ typedef struct {
 typedef struct {
   float scale;          /* current loss scale S                              */
   int growth_tracker;   /* clean steps since the last scale change           */
-  int found_inf;        /* written by adam_step_fp32_master                  */
+  int found_inf;        /* written by adam_step_fp32_master (or by           */
+                        /* gpt_layer_bwd_checked)                            */
   int step;             /* Adam steps taken (skipped steps not counted)      */
   int error;            /* reserved; 0                                       */
 } gptl_scaler_state;
@@ -155,6 +156,31 @@ int adam_step_fp32_master(size_t n_params, float *master, float *m, float *v,
                           const float *grad, void *w16, gptl_dtype dtype, float lr,
                           float beta1, float beta2, float eps, float weight_decay,
                           gptl_scaler_state *st, gptl_stream_t stream);
+
+/* The step's overflow check folded into the backward ("Megatron-LM
+ * overview" §3.1, dynamic loss scaling; the fused kernels of "Training GPT-2
+ * with Megatron-LM" §6.2 taken to the optimizer side).  gpt_layer_bwd_checked
+ * is gpt_layer_bwd that also sets st->found_inf (DEVICE) to 1 if any
+ * gradient value it writes is inf or NaN, else 0: the kernels that write the
+ * 12 gradients (the fp32 weight-gradient GEMMs' epilogues or their split-K
+ * sums, and the column-sum reductions of the biases and LayerNorm
+ * parameters) each test the values they store, so no pass re-reads the
+ * arena.  adam_step_fp32_master_prechecked is adam_step_fp32_master without
+ * step 1: it takes st->found_inf as it stands.  Used as a pair, with the
+ * gradient arena holding exactly what gpt_layer_bwd_checked wrote and zero
+ * padding, they make the same decision, bit for bit, as
+ * gpt_layer_bwd + adam_step_fp32_master, at 4 bytes per parameter less HBM
+ * traffic.  If anything else writes the arena in between (accumulation,
+ * an injected value), use adam_step_fp32_master, which scans it.
+ * Arguments and errors as gpt_layer_bwd / adam_step_fp32_master; also
+ * GPTL_E_NULL if st is NULL and GPTL_E_ALIGN if it is not 4-byte aligned. */
+int gpt_layer_bwd_checked(const gptl_shape *shape, const gptl_weights *w, const void *x,
+                          const void *saved, const void *dy, void *dx, const gptl_grads *g,
+                          void *scratch, gptl_scaler_state *st, gptl_stream_t stream);
+int adam_step_fp32_master_prechecked(size_t n_params, float *master, float *m, float *v,
+                                     const float *grad, void *w16, gptl_dtype dtype, float lr,
+                                     float beta1, float beta2, float eps, float weight_decay,
+                                     gptl_scaler_state *st, gptl_stream_t stream);
 
 /* Dynamic loss-scale update (one device thread), after adam_step_fp32_master:
  *   found_inf: scale = max(scale*backoff_factor, min_scale); tracker = 0;

@@ -39,12 +39,6 @@ enum {
   GPTL_ACT_GELU = 1,     /* out = value, out2 = GeLU(value)                   */
   GPTL_ACT_DGELU = 2     /* out = value * GeLU'(aux)                          */
 };
-enum {
-  GPTL_CAUSAL_NONE = 0,
-  GPTL_CAUSAL_SKIP_UPPER = 1, /* skip 128 x BN tiles with n0 > m0 + 127    */
-  GPTL_CAUSAL_K_BELOW = 2,    /* reduce only over k < m0 + 128             */
-  GPTL_CAUSAL_K_FROM = 3      /* reduce only over k >= m0                  */
-};
 
 /* out[G](m, n) = epilogue( sum over ks < k_shards, k < K of A(m,k) * B(n,k) )
  * for m < M, n < N, G < groups, with fp32 accumulation in tensor memory.
@@ -58,9 +52,9 @@ enum {
  * even.  resid and DGELU do not combine.  Requirements: K % 16 == 0,
  * N % 16 == 0, all offsets/pitches multiples of 8 elements, out (and out2,
  * ws) 16-byte aligned.  The outputs are written by tensor stores of whole
- * 32-row boxes clipped to M x N:
- * nothing outside the M x N window of each group is written, but the groups'
- * windows must not overlap.
+ * 32-row boxes clipped to M x N: nothing outside the M x N window of each
+ * group is written, but the groups' windows must not overlap.  causal is
+ * reserved and must be 0.
  * Split-K: when out_f32 is set with no bias, resid or act, and ws (16-byte
  * aligned device memory of ws_bytes) is given, the library may cut the K
  * loop of each output tile into slices computed by different SMs; each slice
@@ -96,10 +90,15 @@ int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream);
  *   GPTL_GEMM_ALTERNATE  128 x bn tiles alternate between the pipelines;
  *   GPTL_GEMM_K_HALVES   both pipelines on each 128 x bn tile, one half of its
  *                        K range each, summed in a fixed order;
- *   GPTL_GEMM_M256       256 x bn tiles, one 128-row half per pipeline.
+ *   GPTL_GEMM_M256       256 x bn tiles, one 128-row half per pipeline;
+ *   GPTL_GEMM_PAIR       256 x bn tiles on a cluster of two CTAs (two SMs):
+ *                        one MMA stream for both (tcgen05 cta_group::2), each
+ *                        SM staging its 128 rows of A and half of B, and two
+ *                        accumulators per SM so that a tile's epilogue
+ *                        overlaps the next tile's MMAs.
  * Results do not depend on the choice beyond fp32 summation order, and are
  * deterministic for a given choice. */
-enum { GPTL_GEMM_ALTERNATE = 0, GPTL_GEMM_K_HALVES = 1, GPTL_GEMM_M256 = 2 };
+enum { GPTL_GEMM_ALTERNATE = 0, GPTL_GEMM_K_HALVES = 1, GPTL_GEMM_M256 = 2, GPTL_GEMM_PAIR = 3 };
 int gptl_gemm_plan(const gptl_gemm_desc *d, gptl_dtype dtype, int *bn, int *split, int *mode);
 
 /* Fused causal attention forward ("Training GPT-2 with Megatron-LM" §6.2
@@ -142,17 +141,6 @@ int gptl_layernorm_bwd(int rows, int h, gptl_dtype dtype, const void *gy, const 
                        void *dx, float *dg, float *db, float *dx_sum, void *scratch,
                        gptl_stream_t stream);
 
-/* Causal softmax in place on `blocks` score blocks [s][s]: row p becomes
- * softmax over q <= p of scale*S; entries p < q < min(s, 128*(p/128+1)) are
- * set to 0; the rest of the row is not touched.  s % 16 == 0, s <= 2048. */
-int gptl_softmax_fwd(long long blocks, int s, gptl_dtype dtype, float scale, void *scores,
-                     gptl_stream_t stream);
-
-/* Softmax backward in place: dP -> scale * P * (dP - rowsum(P*dP)) on q <= p,
- * 0 for p < q < min(s, 128*(p/128+1)). */
-int gptl_softmax_bwd(long long blocks, int s, gptl_dtype dtype, float scale, const void *prob,
-                     void *dprob, gptl_stream_t stream);
-
 /* Scratch bytes gptl_colsum needs. */
 size_t gptl_colsum_scratch_bytes(int n, int groups);
 
@@ -174,6 +162,9 @@ int gptl_colsum(int rows, int n, int groups, long long ld, long long gstride, gp
  *     summed in the same order.
  *   - The first call on each device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept with the id of the CUDA context it came from: after
+ *     a device reset the next call (again outside any capture) looks it up
+ *     anew.  Host threads may call concurrently; a mutex guards the lookup.
  *   - All calls share the one array: calls whose kernels may overlap on the
  *     GPU (different streams, or different host threads, on one device) race
  *     and give wrong sums.  Calls in order on one stream are safe.  The array

@@ -28,8 +28,8 @@ enum {
   GPTL_KIND_GEMM = 0,        /* tcgen05 tensor-core GEMM (every contraction)  */
   GPTL_KIND_LN_FWD = 1,      /* LayerNorm forward                             */
   GPTL_KIND_LN_BWD = 2,      /* LayerNorm backward (rows pass)                */
-  GPTL_KIND_SOFTMAX_FWD = 3, /* causal scale-mask-softmax forward             */
-  GPTL_KIND_SOFTMAX_BWD = 4, /* softmax backward                              */
+  GPTL_KIND_RESERVED_3 = 3,  /* not launched (the attention kernels fuse the  */
+  GPTL_KIND_RESERVED_4 = 4,  /* scale-mask-softmax)                           */
   GPTL_KIND_COLSUM = 5,      /* column sums (bias gradients), partial pass    */
   GPTL_KIND_REDUCE = 6,      /* final pass of a two-pass column reduction     */
   GPTL_KIND_OVERFLOW = 7,    /* inf/NaN check over the gradient arena         */

@@ -130,3 +130,30 @@ def test_stack_workspace_and_arguments_rejected_without_launch():
     gbad = (G.Grads * 2)(g, G.make_grads({n: (None if n == "b_2" else 4096) for n in G.PARAM_NAMES}))
     assert lib.gpt_stack_bwd(ctypes.byref(sh), 2, ws, 16, 32, 48, 64, 80, gbad, 96, None) == G.E_NULL
     assert lib.gpt_stack_bwd(ctypes.byref(sh), 2, ws, 16, 32, 48, 64, 80, gs, None, None) == G.E_NULL
+
+
+@pytest.mark.parametrize("shape", [
+    dict(batch=1, seq=128, hidden=8192, heads=64, ffn=32768, tp=1, dtype="bf16"),    # h/t = 8192
+    dict(batch=1, seq=128, hidden=8192, heads=128, ffn=32768, tp=2, dtype="bf16"),   # 64 heads/shard
+    dict(batch=1, seq=2048, hidden=10240, heads=80, ffn=40960, tp=1, dtype="bf16"),
+])
+def test_wide_shapes_are_accepted(shape):
+    """Shapes whose row term covers more than 4096 columns or 32 heads per
+    shard are run by the chunked row-dot kernel: sizing accepts them, since
+    every launch-time limit is checked up front."""
+    saved, scratch = G.workspace_bytes(G.make_shape(**shape))
+    assert saved > 0 and scratch > 0
+
+
+def test_layernorm_backward_limit_is_checked_up_front():
+    """hidden 16384 would need 256 KB of running sums per LayerNorm-2
+    backward block, above the 227 KB shared-memory limit: the sizing call
+    refuses the shape, so fwd / bwd never start a step they cannot finish."""
+    sh = G.make_shape(1, 128, 16384, 128, 65536, 1, "bf16")
+    with pytest.raises(G.GptlError) as e:
+        G.workspace_bytes(sh)
+    assert e.value.code == G.E_SHAPE
+    w = G.make_weights({n: 4096 for n in G.PARAM_NAMES})
+    before = G.launch_count()
+    assert G.lib().gpt_layer_fwd(ctypes.byref(sh), ctypes.byref(w), 16, 32, 48, None, None) == G.E_SHAPE
+    assert G.launch_count() == before

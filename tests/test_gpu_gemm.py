@@ -49,12 +49,6 @@ def _expected(desc, abuf, bbuf):
         for ks in range(desc["k_shards"]):
             A = _operand_matrix(abuf, desc["a"], g, ks, M, K)
             B = _operand_matrix(bbuf, desc["b"], g, ks, N, K)
-            if desc["causal"] == G.CAUSAL_K_BELOW:
-                m0 = (np.arange(M) // 128) * 128
-                A = A * (np.arange(K)[None, :] < (m0[:, None] + 128))
-            if desc["causal"] == G.CAUSAL_K_FROM:
-                m0 = (np.arange(M) // 128) * 128
-                A = A * (np.arange(K)[None, :] >= m0[:, None])
             acc += A @ B.T
         res.append(acc)
     return np.stack(res)
@@ -222,37 +216,6 @@ def test_k_shard_reduction(dtype):
     _close(got, exp, 8e-3)
 
 
-@pytest.mark.parametrize("dtype,s,d", [("bf16", 320, 64), ("fp16", 256, 80), ("fp16", 64, 32),
-                                       ("bf16", 256, 128)])
-def test_attention_arrangements(dtype, s, d):
-    """Per-head views into a packed [ij][s][3*heads*d] buffer: scores with
-    upper tiles skipped, P V with the K range limited below the diagonal
-    tile, P^T dO with the K range from the diagonal tile."""
-    heads, ij = 2, 3
-    width = 3 * heads * d
-    grp = ij * heads
-    # scores: Q K^T
-    exp, got, _ = _run(dtype, M=s, N=s, K=d, groups=grp, k_shards=1, causal=G.CAUSAL_SKIP_UPPER,
-                       a_spec=((ij, s, width), dict(mn=0, x_mod=heads, x_mul=d, g_div=heads)),
-                       b_spec=((ij, s, width), dict(mn=0, x_mod=heads, x_mul=d, x_off=heads * d,
-                                                    g_div=heads)), std_b=0.3)
-    low = np.tril(np.ones((s, s), dtype=bool))
-    _close(got, exp, 8e-3, mask=np.broadcast_to(low, got.shape))
-    # P V with lower-triangular P (K range limited)
-    rng = np.random.default_rng(5)
-    exp, got, _ = _run(dtype, M=s, N=d, K=s, groups=grp, k_shards=1, causal=G.CAUSAL_K_BELOW,
-                       a_spec=((grp, s, s), dict(mn=0)),
-                       b_spec=((ij, s, width), dict(mn=1, x_mod=heads, x_mul=d, x_off=2 * heads * d,
-                                                    g_div=heads)), std_a=0.2)
-    _close(got, exp, 8e-3)
-    # P^T dO (A MN-major, K from the diagonal tile)
-    exp, got, _ = _run(dtype, M=s, N=d, K=s, groups=grp, k_shards=1, causal=G.CAUSAL_K_FROM,
-                       a_spec=((grp, s, s), dict(mn=1)),
-                       b_spec=((ij, s, heads * d), dict(mn=1, x_mod=heads, x_mul=d, g_div=heads)),
-                       std_a=0.2)
-    _close(got, exp, 8e-3)
-
-
 @pytest.mark.parametrize("dtype", DT)
 def test_wgrad_split_k(dtype):
     """Few output tiles and a long K: the K loop is split across SMs, the fp32
@@ -339,16 +302,23 @@ def _plan(M, N, K, groups, a_spec, b_spec, out_f32=False, ws_bytes=0, dtype="bf1
 
 
 def test_pipeline_modes_with_several_tiles_per_sm():
-    """Each way of using an SM's two MMA pipelines (tiles alternating between
-    them, both on one tile's K halves, 256-row tiles split by M) on shapes
-    with more tiles than SMs, so that every CTA walks several tiles; the
-    library reports which way it chose (gptl_gemm_plan) and the cases must
-    cover all three."""
+    """Each way of running the GEMM (tiles alternating between an SM's two
+    MMA pipelines, both pipelines on one tile's K halves, 256-row tiles split
+    by M, and 256-row tiles on a cluster of two SMs) on shapes with more
+    tiles than SMs, so that every CTA walks several tiles; the library
+    reports which way it chose (gptl_gemm_plan) and the cases must cover all
+    four."""
     need_gpu()
     cases = [
-        # the attention-input projection's shape: 256-row tiles, ~2 per SM
+        # the attention-input projection's shape: 256-row tiles on CTA pairs
         dict(dtype="bf16", M=8192, N=2304, K=768, groups=1, k_shards=1, causal=0,
              a_spec=((1, 8192, 768), dict(mn=0)), b_spec=((1, 2304, 768), dict(mn=0)), bias=True),
+        # the GPT-2 FFN2 shape: 256-row tiles on one SM
+        dict(dtype="bf16", M=8192, N=768, K=3072, groups=1, k_shards=1, causal=0,
+             a_spec=((1, 8192, 3072), dict(mn=0)), b_spec=((1, 768, 3072), dict(mn=0)), bias=True),
+        # CTA pairs with MN-major operands, fp32 output and a ragged M tail
+        dict(dtype="fp16", M=1000, N=1024, K=2048, groups=3, k_shards=1, causal=0,
+             a_spec=((3, 2048, 1000), dict(mn=1)), b_spec=((1, 2048, 1024), dict(mn=1)), out_f32=True),
         # one 128-row tile per group, many groups: tiles alternate
         dict(dtype="fp16", M=128, N=256, K=64, groups=400, k_shards=1, causal=0,
              a_spec=((1, 128, 64), dict(mn=0)), b_spec=((400, 256, 64), dict(mn=0))),
@@ -371,4 +341,4 @@ def test_pipeline_modes_with_several_tiles_per_sm():
         # the same plan twice gives the same bits
         _, got2, _ = _run(**kw)
         np.testing.assert_array_equal(got, got2)
-    assert modes == {G.GEMM_ALTERNATE, G.GEMM_K_HALVES, G.GEMM_M256}, modes
+    assert modes == {G.GEMM_ALTERNATE, G.GEMM_K_HALVES, G.GEMM_M256, G.GEMM_PAIR}, modes

@@ -1,6 +1,6 @@
 """GPU parity of the bandwidth kernels against the CPU oracle: LayerNorm
-forward/backward, causal softmax forward/backward, column sums, overflow
-check, fused Adam, loss-scale update."""
+forward/backward, column sums, overflow check, fused Adam, loss-scale
+update, clipping and accumulation."""
 import dataclasses
 import math
 
@@ -53,41 +53,6 @@ def test_layernorm_fwd_bwd(dtype, rows, h):
     assert rel_max_err(dg.cpu().numpy(), dge) < 2e-3
     assert rel_max_err(db.cpu().numpy(), dbe) < 1e-4
     assert rel_max_err(dsum.cpu().numpy(), host_values(dx, dtype).sum(axis=0)) < 1e-4
-
-
-@pytest.mark.parametrize("dtype,s,blocks", [("bf16", 1024, 3), ("fp16", 64, 5), ("fp16", 272, 2),
-                                            ("bf16", 2048, 1)])
-def test_causal_softmax_fwd_bwd(dtype, s, blocks):
-    need_gpu()
-    rng = np.random.default_rng(s)
-    d = 64
-    scale = 1.0 / math.sqrt(d)
-    sc = rounded(rng.standard_normal((blocks, s, s)) * 6, dtype)
-    dpv = rounded(rng.standard_normal((blocks, s, s)), dtype)
-    st = dev_tensor(sc, dtype)
-    G.softmax_fwd(blocks, s, dtype, scale, st, stream())
-    dpt = dev_tensor(dpv, dtype)
-    torch.cuda.synchronize()
-    p_gpu = host_values(st, dtype)
-    G.softmax_bwd(blocks, s, dtype, scale, st, dpt, stream())
-    check_device_error()
-    ds_gpu = host_values(dpt, dtype)
-    for blk in range(blocks):
-        pe = oracle.causal_softmax(sc[blk] * scale)
-        low = np.tril(np.ones((s, s), dtype=bool))
-        np.testing.assert_allclose(p_gpu[blk][low], pe[low], rtol=2e-2, atol=1e-3)
-        # zeros above the diagonal inside the diagonal tile
-        for p in range(0, s, 37):
-            end = min(s, (p // 128 + 1) * 128)
-            assert np.all(p_gpu[blk, p, p + 1:end] == 0)
-        # backward: the oracle's formula applied to the GPU's own P
-        pg = p_gpu[blk] * low
-        dse = scale * pg * (dpv[blk] - (pg * dpv[blk]).sum(axis=1, keepdims=True))
-        err = np.abs(ds_gpu[blk][low] - dse[low]).max() / np.abs(dse[low]).max()
-        assert err < 2e-2
-        for p in range(0, s, 41):
-            end = min(s, (p // 128 + 1) * 128)
-            assert np.all(ds_gpu[blk, p, p + 1:end] == 0)
 
 
 @pytest.mark.parametrize("dtype,rows,n,groups", [("bf16", 8192, 768, 1), ("fp16", 130, 256, 2),

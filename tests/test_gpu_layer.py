@@ -5,32 +5,30 @@ Bar: for Out, dX and each of the 12 gradients,
 max|gpu - oracle| <= 2e-2 * RMS(oracle), the oracle run at the method's own
 precision (activations handed between steps held in the 16-bit type; see
 oracle/layer.py).  The gradients are those of the scaled loss (the criterion
-is scale-invariant).
+is scale-invariant).  Every tensor also meets an RMS-error bar of 2e-2, and
+every fp16 tensor meets the 2e-2 max-abs bar against the all-float64 oracle
+(the plain definition) as well.
 
-bf16 keeps 8 significant bits.  Two correct implementations of the bf16
-method that differ only in how their fp32 sums round (the oracle, and the
-oracle with a 2^-22 relative perturbation before each 16-bit store) already
-drift apart by more than 2e-2 * RMS on heavy-tailed weight gradients: each
-one-ulp difference in a stored activation moves every value computed from
-it.  For a bf16 tensor whose own drift (the larger of two perturbation
-seeds) exceeds 1e-2, the bar becomes twice that drift, together with an
-RMS-error bar of 2e-2 * RMS that a real defect would break.  fp16 tensors
-keep the plain bar.  The distance to the all-float64 oracle is reported
-beside it."""
-import dataclasses
-
-import numpy as np
+One measured limit stands, for bf16 only.  bf16 keeps 8 significant bits,
+and two correct implementations of the bf16 method that differ only in how
+their fp32 sums round drift apart by more than 2e-2 * RMS in max-abs on
+heavy-tailed tensors (tests/test_oracle_precision.py,
+test_bf16_drift_floor_exceeds_the_bar_on_w_qkv): the QKV weight gradient,
+whose largest entries are about ten times its RMS, and at the hidden-10240
+shape a few more.  When a bf16 tensor misses the max-abs bar, the test
+measures that drift on the same step (the oracle again with 2^-22 relative
+noise before each 16-bit store) and reports an expected failure with both
+numbers if the GPU stays within twice it and every other bar holds; beyond
+twice the drift it fails.  It is never passed on a wider bar."""
 import pytest
 import torch
 
-import oracle
-from transformer_layer_step_b200 import gptlayer as G
 from transformer_layer_step_b200 import synth
 from transformer_layer_step_b200.harness import LayerStep
-from gpu_util import need_gpu, host_values, check_device_error, rel_max_err
+from gpu_util import need_gpu, check_device_error
+from layer_parity import run_gpu, check_against_oracle
 
 pytestmark = pytest.mark.gpu
-TOL = 2e-2
 
 SMALL = {
     # several tiles in every GEMM, ragged tails, t = 2 and t = 4
@@ -40,75 +38,13 @@ SMALL = {
 }
 
 
-DRIFT = 2.0 ** -22
-
-
-def _errs(out_gpu, dx_gpu, grads_gpu, out_o, dx_o, gr_o, stat=rel_max_err):
-    errs = {"out": stat(out_gpu, out_o), "dx": stat(dx_gpu, dx_o)}
-    for k in gr_o:
-        errs[k] = stat(grads_gpu[k].reshape(gr_o[k].shape), gr_o[k])
-    return errs
-
-
-def rel_rms_err(got, ref):
-    return float(np.sqrt(np.mean((got - ref) ** 2)) / max(np.sqrt(np.mean(ref ** 2)), 1e-30))
-
-
-def drift_floor(x, p, cfg, eps, dout, out_o, dx_o, gr_o):
-    """Largest distance, over two perturbation seeds, between the oracle and
-    the same 16-bit method with fp32-sized rounding differences."""
-    floor = {}
-    for seed in (1, 2):
-        rng = np.random.default_rng(seed)
-        noise = lambda a: a * (1.0 + DRIFT * rng.standard_normal(a.shape))
-        o2, c2 = oracle.layer_fwd(x, p, cfg.dims(), eps, precision=cfg.dtype, noise=noise)
-        d2, g2 = oracle.layer_bwd(c2, p, cfg.dims(), dout)
-        del c2
-        e = _errs(o2, d2, g2, out_o, dx_o, gr_o)
-        floor = {k: max(v, floor.get(k, 0.0)) for k, v in e.items()}
-    return floor
-
-
 def _run_and_compare(cfg, variant, with_r, seed=0):
     need_gpu()
     inp = synth.make_inputs(cfg, seed=seed, variant=variant, with_r=with_r)
-    ls = LayerStep(cfg, inp)
-    scale = ls.hyper["init_scale"]
-    eps = ls.hyper["ln_eps"]
-    dy_bits = synth.loss_grad_bits(cfg, scale, inp["r"] if with_r else None)
-    ls.set_dy_bits(dy_bits)
-    ls.fwd()
-    ls.bwd()
-    check_device_error()
-    out_gpu = host_values(ls.y, cfg.dtype)
-    dx_gpu = host_values(ls.dx, cfg.dtype)
-    grads_gpu = ls.grads_host()
-    del ls
-
-    x = synth.from_bits(inp["x"], cfg.dtype).reshape(cfg.tokens, cfg.hidden)
-    p = {k: synth.from_bits(v, cfg.dtype).reshape(v.shape) for k, v in inp["params"].items()}
-    dout = synth.from_bits(dy_bits, cfg.dtype).reshape(cfg.tokens, cfg.hidden)
-    out_e, cache = oracle.layer_fwd(x, p, cfg.dims(), eps)
-    dx_e, gr_e = oracle.layer_bwd(cache, p, cfg.dims(), dout)
-    del cache
-    exact = _errs(out_gpu, dx_gpu, grads_gpu, out_e, dx_e, gr_e)
-    out_o, cache = oracle.layer_fwd(x, p, cfg.dims(), eps, precision=cfg.dtype)
-    dx_o, gr_o = oracle.layer_bwd(cache, p, cfg.dims(), dout)
-    del cache
-    errs = _errs(out_gpu, dx_gpu, grads_gpu, out_o, dx_o, gr_o)
-    rms_errs = _errs(out_gpu, dx_gpu, grads_gpu, out_o, dx_o, gr_o, stat=rel_rms_err)
-    bars = {k: TOL for k in errs}
-    floor = {}
-    if cfg.dtype == synth.BF16:
-        floor = drift_floor(x, p, cfg, eps, dout, out_o, dx_o, gr_o)
-        bars = {k: max(TOL, 2.0 * floor[k]) if floor[k] > 1e-2 else TOL for k in errs}
-    r5 = lambda d: {k: round(v, 5) for k, v in d.items()}
-    print(cfg.name, variant, {"vs_method": r5(errs), "rms_err": r5(rms_errs),
-                              "drift_floor": r5(floor), "vs_float64": r5(exact)})
-    bad = {k: (v, bars[k]) for k, v in errs.items() if not v <= bars[k]}
-    bad.update({("rms", k): v for k, v in rms_errs.items() if not v <= TOL})
-    assert not bad, (bad, errs)
-    return errs
+    dy_bits = synth.loss_grad_bits(cfg, synth.HYPER["init_scale"], inp["r"] if with_r else None)
+    out_gpu, dx_gpu, grads_gpu = run_gpu(cfg, inp, dy_bits)
+    return check_against_oracle(cfg, inp, dy_bits, out_gpu, dx_gpu, grads_gpu,
+                                eps=synth.HYPER["ln_eps"])
 
 
 @pytest.mark.parametrize("name", list(SMALL))

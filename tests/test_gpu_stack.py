@@ -7,11 +7,7 @@ C ABI, and one optimizer call over every layer's parameters).
   directions.  The kernels are deterministic, so any plumbing mistake (a
   wrong buffer, offset or order) shows as a mismatch.
 * Parity with the oracle's stack (fp16) for the output, dX and every
-  layer's gradients.  Each layer meets the layer test's 2e-2 * RMS bar on
-  its own (tests/test_gpu_layer.py, and the composition above makes the
-  stack's layers those layers); through the residual stream a layer passes
-  the error of its input on with a gain of about one and adds its own, so
-  the bar for the whole stack is the number of layers times 2e-2.
+  layer's gradients, each within the layer test's 2e-2 * RMS bar.
 * The optimizer call covers the whole arena: every layer's block matches
   the oracle's Adam.
 """
@@ -98,7 +94,7 @@ def test_stack_matches_oracle_and_one_adam_covers_every_layer():
         for k in gr_o[l]:
             errs[(l, k)] = rel_max_err(g[k].reshape(gr_o[l][k].shape), gr_o[l][k])
     print({str(k): round(v, 5) for k, v in errs.items()})
-    assert all(v <= N_LAYERS * 2e-2 for v in errs.values()), errs
+    assert all(v <= 2e-2 for v in errs.values()), errs
 
     # one optimizer call over the L * n_layer_params arena
     hp = st.hyper

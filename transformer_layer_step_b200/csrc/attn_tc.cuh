@@ -1,39 +1,49 @@
 // attn_tc.cuh — fused causal attention forward on tcgen05 (sm_100a).
 //
 // For every (shard, batch, head) and every 128-row block of queries, the
-// kernel walks the 128-key blocks at or below the diagonal: S = Q K^T goes
-// to tensor memory, an online softmax turns it into P in shared memory (the
-// A operand of the next MMA), and O += P V accumulates in tensor memory.  S
-// and P never reach HBM.  This is the fused scale-mask-softmax of "Training
-// GPT-2 with Megatron-LM" §6.2 carried one step further: the score matrix is
-// consumed where it is produced.  The kernel writes O and the base-2
-// log-sum-exp of each row's scaled scores, from which the backward
-// recomputes P.
+// kernel makes two passes over the 128-key blocks at or below the diagonal.
+// Pass 1 computes S = Q K^T into tensor memory and reduces each row to its
+// base-2 log-sum-exp lse = log2(sum_q 2^(S_pq log2(e)/sqrt(d))).  Pass 2
+// computes S again, turns it into the normalised probabilities
+// P = 2^(S log2(e)/sqrt(d) - lse), rounds them to the 16-bit type as the A
+// operand of the next MMA (shared memory), and accumulates O += P V in tensor
+// memory.  S and P never reach HBM.  This is the fused scale-mask-softmax of
+// "Training GPT-2 with Megatron-LM" §6.2 (its output, the normalised P in
+// 16 bits, is the operand of P V) carried one step further: the score matrix
+// is consumed where it is produced.  Normalising before the rounding keeps
+// the 16-bit operand exactly the one the unfused method multiplies; a single
+// pass that rounds exp(S - running max) and divides by the row sum at the end
+// would round different values.  The kernel writes O and lse, from which the
+// backward recomputes P.
 //
-// Warp roles (256 threads, one CTA per SM, persistent over work items):
-//   warp 0     TMA: Q once per item, then K and V of each key block into a
-//              ring of kv_stages (2..4) stages;
-//   warp 1     one thread issues S_j = Q K_j^T into one of two S buffers;
-//   warps 6-7  one thread each issues O += P_j V_j once P_j is ready, warp 6
-//              over keys 0..63 of the block into O, warp 7 over keys 64..127
-//              into O2 (added at the end): the MMA streams run concurrently;
-//   warps 2-5  one query row per thread: read S_j from tensor memory, update
-//              the running max m and sum l, rescale O by exp2(m_old - m_new)
-//              in tensor memory when m moved, write P_j (16-bit) to one of
-//              two shared-memory buffers (so that P_j is formed while
-//              P_{j-1} V_{j-1} runs); at the end normalise O by 1/l and
-//              store it.
+// Warp roles (384 threads, one CTA per SM, persistent over work items):
+//   warp 0      TMA: Q once per item, then per key block K (pass 1) or K and
+//               V (pass 2) into a ring of kv_stages (2..4) stages;
+//   warp 1      one thread issues S_j = Q K_j^T into one of two S buffers;
+//   warps 2-3   one thread each issues O += P_j V_j once P_j is ready, warp 2
+//               over keys 0..63 of the block into O, warp 3 over keys 64..127
+//               into O2 (added at the end): the MMA streams run concurrently;
+//   warps 4-11  softmax: warp w reads TMEM lane quarter w % 4 (32 query rows,
+//               one per thread) and half (w - 4) / 4 of the key block's 128
+//               columns.  Pass 1 keeps a running max and sum per half row;
+//               the two halves of a row meet once per item through shared
+//               memory to form lse.  Pass 2 writes its 64 columns of P_j into
+//               one of two shared-memory P buffers (so that P_j is formed
+//               while P_{j-1} V_{j-1} runs).  At the end each warp stores its
+//               share of O's columns.
 // Tensor memory: S buffers at columns 0 and 128, O at column 256, O2 at 384.
-// Shared memory: two P buffers [128 x 128] (two 128B-swizzled 64-column atoms each), Q as
-// head_dim/16 chunks of [128 rows x 16] (32B swizzle), and per stage K the
-// same way and V as MN-major chunks of [64 keys x vw].
+// Shared memory: two P buffers [128 x 128] (two 128B-swizzled 64-column
+// atoms each), Q as head_dim/16 chunks of [128 rows x 16] (32B swizzle), per
+// stage K the same way and V as MN-major chunks of [64 keys x vw], then the
+// barriers and the half-row log-sum-exps.
 #pragma once
 #include "common.cuh"
 
 namespace gptl {
 
-constexpr int kAttnThreads = 256;
+constexpr int kAttnThreads = 384;
 constexpr int kAttnTile = 128;          // query rows per item, keys per block
+constexpr int kAttnTailBytes = 1280;    // barriers (256 B) + half-row lse [2][128] fp32
 
 struct AttnParams {
   CUtensorMap map_qk;   // C as [t*b][s][3h/t]; box {16, 128, 1}, 32B swizzle
@@ -57,6 +67,14 @@ __device__ __forceinline__ uint64_t attn_desc_k16(uint32_t addr) {
   return make_smem_desc(addr, 16u, 256u, 6u);
 }
 
+// log2(2^a + 2^b) for the two halves of a row (either may be -inf); the
+// same value whichever half computes it.
+__device__ __forceinline__ float lse_merge(float a, float b) {
+  const float mx = fmaxf(a, b);
+  if (mx == -INFINITY) return -INFINITY;
+  return mx + log2f(ex2_approx(a - mx) + ex2_approx(b - mx));
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -71,20 +89,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   const uint32_t kv_s = q_s + q_bytes;
   const uint32_t nkv = (uint32_t)p.kv_stages;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 65536u + q_bytes + nkv * kv_bytes);
-  // bars: q_full q_empty kv_full[4] kv_empty[4] s_full[2] s_empty[2] p_full[2] pv_done[2] drain drain2
+  // bars: q_full q_empty kv_full[4] kv_empty[4] s_full[2] s_empty[2] p_full[2] pv_done[2]
+  //       stat_full[4] stat_read[4] drain drain_pv[2]
   const uint32_t q_full = smem_u32(&bars[0]), q_empty = smem_u32(&bars[1]);
   auto kv_full = [&](int i) { return smem_u32(&bars[2 + i]); };
   auto kv_empty = [&](int i) { return smem_u32(&bars[6 + i]); };
   auto s_full = [&](int i) { return smem_u32(&bars[10 + i]); };
   auto s_empty = [&](int i) { return smem_u32(&bars[12 + i]); };
-  // P_j lives in buffer j % 2 (j counted over all of the CTA's blocks):
-  // p_full[b] publishes it, pv_done[b] reports its P V products complete
+  // P_j (pass 2) lives in buffer j % 2 (j counted over all of the CTA's
+  // pass-2 blocks): p_full[b] publishes it, pv_done[b] reports its P V
+  // products complete
   auto p_full = [&](int b) { return smem_u32(&bars[14 + b]); };
   auto pv_done = [&](int b) { return smem_u32(&bars[16 + b]); };
-  const uint32_t drain_bar = smem_u32(&bars[18]), drain_pv = smem_u32(&bars[19]);
-  const uint32_t drain_pv2 = smem_u32(&bars[20]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 21);
+  // the two softmax warps of lane quarter q exchange their half-row lse
+  auto stat_full = [&](int q) { return smem_u32(&bars[18 + q]); };
+  auto stat_read = [&](int q) { return smem_u32(&bars[22 + q]); };
+  const uint32_t drain_bar = smem_u32(&bars[26]);
+  auto drain_pv = [&](int h) { return smem_u32(&bars[27 + h]); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 29);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *half_lse = reinterpret_cast<float *>(bars + 32);     // [2 halves][128 rows]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -92,19 +116,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     mbar_init(q_empty, 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(kv_full(i), 1);
-      mbar_init(kv_empty(i), 2);   // both P V issuers release a stage
+      mbar_init(kv_empty(i), 2);   // pass 2: both P V issuers; pass 1: two commits of the S issuer
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(s_empty(i), 4);
+      mbar_init(s_empty(i), 8);    // the eight softmax warps
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(p_full(b), 4);
+      mbar_init(p_full(b), 8);
       mbar_init(pv_done(b), 2);    // both halves of P_j V_j
     }
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(stat_full(q), 64);  // every thread of the quarter's two warps
+      mbar_init(stat_read(q), 64);
+    }
     mbar_init(drain_bar, 1);
-    mbar_init(drain_pv, 1);
-    mbar_init(drain_pv2, 1);
+    mbar_init(drain_pv(0), 1);
+    mbar_init(drain_pv(1), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -139,26 +167,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         int g, qt;
         decode(item, g, qt);
         const int head = g % p.as, zb = g / p.as;
+        const int n = qt + 1;
         if (!mbar_wait(q_empty, (item_n & 1u) ^ 1u, abort_flag)) goto tma_abort;
         mbar_arrive_expect_tx(q_full, q_bytes);
         q_parity = (int)(item_n & 1u);
         for (int c = 0; c < d / 16; ++c)
           tma_load_3d(q_s + (uint32_t)c * chunk_bytes, &p.map_qk, p.q_off + head * d + c * 16,
                       qt * kAttnTile, zb, q_full);
-        for (int j = 0; j <= qt; ++j, ++kv_it) {
+        for (int it = 0; it < 2 * n; ++it, ++kv_it) {
+          const int j = it < n ? it : it - n;
+          const bool with_v = it >= n;            // pass 2
           const int st = (int)(kv_it % nkv);
           const uint32_t ph = (kv_it / nkv) & 1u;
           if (!mbar_wait(kv_empty(st), ph ^ 1u, abort_flag)) goto tma_abort;
-          mbar_arrive_expect_tx(kv_full(st), kv_bytes);
+          mbar_arrive_expect_tx(kv_full(st), with_v ? kv_bytes : q_bytes);
           const uint32_t k_s = kv_s + (uint32_t)st * kv_bytes, v_s = k_s + q_bytes;
           for (int c = 0; c < d / 16; ++c)
             tma_load_3d(k_s + (uint32_t)c * chunk_bytes, &p.map_qk, p.k_off + head * d + c * 16,
                         j * kAttnTile, zb, kv_full(st));
-          const int nvc = d / p.vw;
-          for (int kb = 0; kb < 2; ++kb)
-            for (int c = 0; c < nvc; ++c)
-              tma_load_3d(v_s + (uint32_t)((kb * nvc + c) * 64 * p.vw * 2), &p.map_v,
-                          p.v_off + head * d + c * p.vw, j * kAttnTile + kb * 64, zb, kv_full(st));
+          if (with_v) {
+            const int nvc = d / p.vw;
+            for (int kb = 0; kb < 2; ++kb)
+              for (int c = 0; c < nvc; ++c)
+                tma_load_3d(v_s + (uint32_t)((kb * nvc + c) * 64 * p.vw * 2), &p.map_v,
+                            p.v_off + head * d + c * p.vw, j * kAttnTile + kb * 64, zb, kv_full(st));
+          }
           issued |= 1u << st;
           parity_bits = (parity_bits & ~(1u << st)) | (ph << st);
         }
@@ -180,8 +213,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         const int n = qt + 1;
         if (!mbar_wait(q_full, item_n & 1u, abort_flag)) goto mma_abort;
         tc_fence_after();
-        for (int j = 0; j < n; ++j) {
-          const uint32_t kj = kv_it + (uint32_t)j;
+        for (int it = 0; it < 2 * n; ++it) {
+          const uint32_t kj = kv_it + (uint32_t)it;
           if (!mbar_wait(kv_full((int)(kj % nkv)), (kj / nkv) & 1u, abort_flag)) goto mma_abort;
           const int sb = (int)(s_it & 1u);
           if (!mbar_wait(s_empty(sb), ((s_it >> 1) & 1u) ^ 1u, abort_flag)) goto mma_abort;
@@ -191,10 +224,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
             tc_mma_f16(tmem_base + (uint32_t)(sb * 128), attn_desc_k16(q_s + (uint32_t)c * chunk_bytes),
                        attn_desc_k16(k_s + (uint32_t)c * chunk_bytes), p.idesc_s, c > 0 ? 1u : 0u);
           tc_commit(s_full(sb));
+          if (it < n) {                      // pass 1: the stage held K only, now read
+            tc_commit(kv_empty((int)(kj % nkv)));
+            tc_commit(kv_empty((int)(kj % nkv)));
+          }
           ++s_it;
         }
         tc_commit(q_empty);                  // Q is read by these MMAs only
-        kv_it += (uint32_t)n;
+        kv_it += (uint32_t)(2 * n);
       }
       goto mma_done;
     mma_abort:
@@ -202,13 +239,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_wait_drain(drain_bar, 0);
     mma_done:;
     }
-  } else if (warp == 6 || warp == 7) {
+  } else if (warp == 2 || warp == 3) {
     if (lane == 0) {
       // ------------------------------------------- MMA: O += P_j V_j
-      // A second issuing thread: its MMAs run alongside the S MMAs.  P_j
-      // exists only after S_j was read, so K_j is no longer in use when the
-      // stage is released here.
-      uint32_t kv_it = 0, pb = 0;              // pb: the CTA's block counter (P buffer pb % 2)
+      // Second and third issuing threads: their MMAs run alongside the S
+      // MMAs.  P_j exists only after S_j was read, so K_j is no longer in use
+      // when the stage is released here.
+      const int h = warp - 2;
+      uint32_t kv_it = 0, pb = 0;              // pb: the CTA's pass-2 block counter (P buffer pb % 2)
       for (long long item = blockIdx.x; item < p.items; item += gridDim.x) {
         int g, qt;
         decode(item, g, qt);
@@ -218,134 +256,129 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           if (!mbar_wait(p_full(buf), (pb >> 1) & 1u, abort_flag)) goto pv_abort;
           tc_fence_after();
           const uint32_t pbuf = p_s + (uint32_t)buf * 32768u;
-          const uint32_t pj = kv_it + (uint32_t)j;
+          const uint32_t pj = kv_it + (uint32_t)(n + j);
           const uint32_t v_s = kv_s + (pj % nkv) * kv_bytes + q_bytes;
           const uint32_t row_b = (uint32_t)p.vw * 2u;
           const uint32_t kb_bytes = (uint32_t)(d / p.vw) * 64u * row_b;
           const uint32_t vsw = p.vw == 64 ? 2u : (p.vw == 32 ? 4u : 6u);
-          // warp 6: keys 0..63 of the block into O, warp 7: keys 64..127 into O2
-          const int st0 = warp == 6 ? 0 : 4;
-          const uint32_t acc_t = warp == 6 ? tmem_o : tmem_o2;
-          for (int st = st0; st < st0 + 4; ++st) {
+          // issuer 0: keys 0..63 of the block into O, issuer 1: keys 64..127 into O2
+          const uint32_t acc_t = h == 0 ? tmem_o : tmem_o2;
+          for (int st = 0; st < 4; ++st) {
             const uint64_t adesc =
-                make_smem_desc(pbuf + (uint32_t)(st >> 2) * 16384u + (uint32_t)(st & 3) * 32u, 16u, 1024u, 2u);
-            const uint64_t bdesc = make_smem_desc(v_s + (uint32_t)(st >> 2) * kb_bytes +
-                                                      (uint32_t)(st & 3) * 16u * row_b,
+                make_smem_desc(pbuf + (uint32_t)h * 16384u + (uint32_t)st * 32u, 16u, 1024u, 2u);
+            const uint64_t bdesc = make_smem_desc(v_s + (uint32_t)h * kb_bytes + (uint32_t)st * 16u * row_b,
                                                   64u * row_b, 8u * row_b, vsw);
-            tc_mma_f16(acc_t, adesc, bdesc, p.idesc_pv, (j > 0 || st > st0) ? 1u : 0u);
+            tc_mma_f16(acc_t, adesc, bdesc, p.idesc_pv, (j > 0 || st > 0) ? 1u : 0u);
           }
           tc_commit(pv_done(buf));
           tc_commit(kv_empty((int)(pj % nkv)));
         }
-        kv_it += (uint32_t)n;
+        kv_it += (uint32_t)(2 * n);
       }
       goto pv_done;
     pv_abort:
-      tc_commit(warp == 6 ? drain_pv : drain_pv2);
-      mbar_wait_drain(warp == 6 ? drain_pv : drain_pv2, 0);
+      tc_commit(drain_pv(h));
+      mbar_wait_drain(drain_pv(h), 0);
     pv_done:;
     }
   } else {
     // -------------------------------------------------- softmax and epilogue
     const int q4 = warp & 3;                 // TMEM lane quarter of this warp
+    const int half = (warp - 4) >> 2;        // which 64 of the block's 128 keys
     const int row = q4 * 32 + lane;          // query row within the block
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    uint32_t s_it = 0, pb = 0;                 // pb: the CTA's block counter (P buffer pb % 2)
-    // wait until the P V products of block k (a CTA block counter) are done;
-    // only ever called for the latest block that used P buffer k % 2
+    uint32_t s_it = 0, pb = 0, item_n = 0;   // pb: the CTA's pass-2 block counter
+    // wait until the P V products of pass-2 block k are done; only ever
+    // called for the latest block that used P buffer k % 2
     auto wait_pv = [&](uint32_t k) { return mbar_wait(pv_done((int)(k & 1u)), (k >> 1) & 1u, abort_flag); };
-    for (long long item = blockIdx.x; item < p.items; item += gridDim.x) {
+    // S_j, columns [half * 64, +64) of S buffer s_it % 2, masked past the
+    // diagonal and the sequence end; releases the S buffer
+    auto read_s = [&](int j, int qrow, uint32_t (&r)[4][16]) -> bool {
+      const int sb = (int)(s_it & 1u);
+      if (!mbar_wait(s_full(sb), (s_it >> 1) & 1u, abort_flag)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld16(tmem_base + lane_off + (uint32_t)(sb * 128 + half * 64 + c * 16), r[c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_empty(sb));
+      ++s_it;
+      const int key0 = j * kAttnTile + half * 64;
+      if (j * kAttnTile + kAttnTile - 1 >= qrow - row || key0 + 64 > p.s) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int key = key0 + c * 16 + e;
+            if (key > qrow || key >= p.s) r[c][e] = __float_as_uint(-INFINITY);
+          }
+      }
+      return true;
+    };
+    for (long long item = blockIdx.x; item < p.items; item += gridDim.x, ++item_n) {
       int g, qt;
       decode(item, g, qt);
       const int n = qt + 1;
       const int qrow = qt * kAttnTile + row;
-      float m = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < n && ok; ++j, ++pb) {
-        const int sb = (int)(s_it & 1u);
-        if (!mbar_wait(s_full(sb), (s_it >> 1) & 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t r[8][16];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) tmem_ld16(tmem_base + lane_off + (uint32_t)(sb * 128 + c * 16), r[c]);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_empty(sb));
-        ++s_it;
-        // mask (only where a key can be past the row or past the sequence),
-        // then the row max of the raw scores (the scale is positive)
-        const int key0 = j * kAttnTile;
-        if (j == qt || key0 + kAttnTile > p.s) {
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int key = key0 + c * 16 + e;
-              if (key > qrow || key >= p.s) r[c][e] = __float_as_uint(-INFINITY);
-            }
-        }
+      // ---- pass 1: running max m and sum l of 2^(S c) over this half row
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        uint32_t r[4][16];
+        if (!read_s(j, qrow, r)) { ok = false; break; }
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
             mx0 = fmaxf(mx0, __uint_as_float(r[c][e]));
             mx1 = fmaxf(mx1, __uint_as_float(r[c][e + 1]));
           }
-        // Running max m in log2 units of the scaled scores.  It is raised
-        // only when a score exceeds it by more than 2^8, so that O and l are
-        // rescaled rarely; meanwhile P <= 2^8, exact in fp32 and in the
-        // 16-bit operand (whose rounding is relative).  O / l is unchanged.
-        const float mx = fmaxf(mx0, mx1) * p.scale_log2;
-        const float m_new = (mx > m + 8.0f) ? mx : m;
-        const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);   // 0 when m = -inf
+        const float m_new = fmaxf(m, fmaxf(mx0, mx1) * p.scale_log2);
+        if (m_new == -INFINITY) continue;      // every key so far masked
         const float nm = -m_new;
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][e]), p.scale_log2, nm));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][e + 1]), p.scale_log2, nm));
-            r[c][e] = __float_as_uint(p0);
-            r[c][e + 1] = __float_as_uint(p1);
-            s0 += p0;
-            s1 += p1;
+            s0 += ex2_approx(fmaf(__uint_as_float(r[c][e]), p.scale_log2, nm));
+            s1 += ex2_approx(fmaf(__uint_as_float(r[c][e + 1]), p.scale_log2, nm));
           }
-        l = l * alpha + (s0 + s1);
+        l = l * (m_new == m ? 1.0f : ex2_approx(m - m_new)) + (s0 + s1);   // 0 while m = -inf
         m = m_new;
-        // rescale O (rare): needs every earlier P V product done, i.e. block j-1's
-        if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-          if (!wait_pv(pb - 1)) { ok = false; break; }
-          tc_fence_after();
-          {
-            for (int c = 0; c < 2 * (d / 16); ++c) {   // O, then O2
-              const uint32_t ta = (c < d / 16 ? tmem_o : tmem_o2 - (uint32_t)d) + lane_off + (uint32_t)(c * 16);
-              uint32_t o[16];
-              tmem_ld16(ta, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st16(ta, o);
-            }
-            tmem_wait_st();
-          }
-        }
+      }
+      if (!ok) break;
+      // ---- the row's lse from its two halves (shared memory, once per item)
+      const float lse_h = l > 0.f ? m + log2f(l) : -INFINITY;
+      if (item_n > 0 && !mbar_wait(stat_read(q4), (item_n - 1) & 1u, abort_flag)) break;
+      half_lse[half * 128 + row] = lse_h;
+      mbar_arrive(stat_full(q4));
+      if (!mbar_wait(stat_full(q4), item_n & 1u, abort_flag)) break;
+      const float lse_o = half_lse[(half ^ 1) * 128 + row];
+      mbar_arrive(stat_read(q4));
+      const float lse = half == 0 ? lse_merge(lse_h, lse_o) : lse_merge(lse_o, lse_h);
+      const float nl = lse == -INFINITY ? 0.f : -lse;
+      // ---- pass 2: P = 2^(S c - lse) in 16 bits, the A operand of P V
+      for (int j = 0; j < n; ++j, ++pb) {
+        uint32_t r[4][16];
+        if (!read_s(j, qrow, r)) { ok = false; break; }
         // P buffer pb % 2 is free once block pb-2's P V products are done (an
         // earlier item's blocks are all done: its end waited for its last)
         if (j >= 2 && !wait_pv(pb - 2)) { ok = false; break; }
-        // P (16-bit) into the 128B-swizzled K-major A tile: row `row`,
-        // 16-byte chunk c16 of the row goes to atom c16/8, slot (c16%8)^(row%8)
-        const uint32_t pbuf = p_s + (pb & 1u) * 32768u;
+        // this half's 64 columns form atom `half` of the 128B-swizzled
+        // K-major A tile: 16-byte chunk c8 of row `row` goes to slot
+        // c8 ^ (row % 8)
+        const uint32_t pbuf = p_s + (pb & 1u) * 32768u + (uint32_t)half * 16384u + (uint32_t)row * 128u;
 #pragma unroll
-        for (int c16 = 0; c16 < 16; ++c16) {
+        for (int c8 = 0; c8 < 8; ++c8) {
           float f[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[c16 >> 1][(c16 & 1) * 8 + e]);
-          const uint32_t addr = pbuf + (uint32_t)(c16 >> 3) * 16384u + (uint32_t)row * 128u +
-                                (uint32_t)(((c16 & 7) ^ (row & 7)) * 16);
-          st_shared_v4(addr, pack8<T>(f));
+          for (int e = 0; e < 8; ++e)
+            f[e] = ex2_approx(fmaf(__uint_as_float(r[c8 >> 1][(c8 & 1) * 8 + e]), p.scale_log2, nl));
+          st_shared_v4(pbuf + (uint32_t)(((c8 & 7) ^ (row & 7)) * 16), pack8<T>(f));
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -353,13 +386,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         if (lane == 0) mbar_arrive(p_full((int)(pb & 1u)));
       }
       if (!ok) break;
-      // epilogue: wait for the last P V, normalise, store O and the log-sum-exp
+      // ---- epilogue: wait for the last P V, store this warp's share of O
+      // (chunks [0, ch) for half 0, [ch, d/16) for half 1) and the lse
       if (!wait_pv(pb - 1)) break;
       tc_fence_after();
-      const float inv_l = 1.0f / l;
       const int head = g % p.as, zb = g / p.as;
       T *orow = static_cast<T *>(p.o) + ((long long)zb * p.s + qrow) * p.hs + head * d;
-      for (int c = 0; c < d / 16; ++c) {
+      const int nc = d / 16, ch = (nc + 1) / 2;
+      for (int c = half ? ch : 0; c < (half ? nc : ch); ++c) {
         uint32_t o[16], o2[16];
         tmem_ld16(tmem_o + lane_off + (uint32_t)(c * 16), o);
         tmem_ld16(tmem_o2 + lane_off + (uint32_t)(c * 16), o2);
@@ -370,12 +404,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              f[e] = (__uint_as_float(o[h2 * 8 + e]) + __uint_as_float(o2[h2 * 8 + e])) * inv_l;
+              f[e] = __uint_as_float(o[h2 * 8 + e]) + __uint_as_float(o2[h2 * 8 + e]);
             reinterpret_cast<uint4 *>(orow + c * 16)[h2] = pack8<T>(f);
           }
         }
       }
-      if (qrow < p.s) p.lse[(long long)g * p.s + qrow] = m + log2f(l);
+      if (half == 0 && qrow < p.s) p.lse[(long long)g * p.s + qrow] = lse;
       tc_fence_before();
     }
   }

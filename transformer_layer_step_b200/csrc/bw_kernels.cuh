@@ -1,8 +1,7 @@
 // bw_kernels.cuh — HBM-bandwidth kernels of the layer step (sm_100a).
 //
-// LayerNorm forward/backward, the fused causal scale-mask-softmax
-// forward/backward ("Training GPT-2 with Megatron-LM" §6.2 fused_softmax),
-// column sums for bias gradients, batched 16-bit transposes (the
+// LayerNorm forward/backward, column sums for bias gradients, batched
+// 16-bit transposes (the
 // token-contiguous copies that weight-gradient GEMMs read as K-major
 // operands), and the optimizer side of mixed precision
 // ("Megatron-LM overview" §3.1, §4.2): overflow check, fused unscale + Adam +
@@ -232,8 +231,10 @@ __global__ void __launch_bounds__(256, VPT <= 3 ? 2 : 1) ln_bwd_kernel(
 
 // out_k[c] = sum_b part[k][b][c] for the nk = gridDim.y arrays of width n.
 // Block: 32 columns x 16 row groups; fixed summation order (deterministic).
+// With `flag`, any inf or NaN sum sets it to 1.
 struct PartOuts {
   float *o[4];
+  int *flag;
 };
 __global__ void __launch_bounds__(512) reduce_parts_kernel(const float *__restrict__ part,
                                                            int nblocks, int n, PartOuts outs) {
@@ -248,11 +249,16 @@ __global__ void __launch_bounds__(512) reduce_parts_kernel(const float *__restri
   }
   sm[threadIdx.y][threadIdx.x] = s;
   __syncthreads();
-  if (threadIdx.y == 0 && c < n) {
-    float t = 0.f;
+  if (threadIdx.y == 0) {                 // one warp
+    bool bad = false;
+    if (c < n) {
+      float t = 0.f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) t += sm[i][threadIdx.x];
-    outs.o[k][c] = t;
+      for (int i = 0; i < 16; ++i) t += sm[i][threadIdx.x];
+      outs.o[k][c] = t;
+      bad = !(fabsf(t) <= 3.402823466e38f);
+    }
+    if (outs.flag && __any_sync(0xffffffffu, bad) && threadIdx.x == 0) atomicOr(outs.flag, 1);
   }
 }
 
@@ -375,108 +381,6 @@ __global__ void __launch_bounds__(256) transpose16_kernel(const __grid_constant_
   }
 }
 
-// --------------------------------------------------------- causal softmax
-// In place on [rows = G*s][s] score blocks.  Row p of a block: entries q <= p
-// get softmax(scale * S), entries p < q < end of the 128-wide diagonal tile
-// get 0 (the attention GEMMs read those tiles).  One warp per row; each lane
-// holds NV 8-element vectors.
-template <typename T, int NV>
-__global__ void __launch_bounds__(256) softmax_fwd_kernel(T *__restrict__ s_io, long long nrows,
-                                                          int s, float scale) {
-  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  if (row >= nrows) return;
-  const int p = (int)(row % s);
-  const int valid = p + 1;
-  const int wend = min(s, (p / 128 + 1) * 128);
-  uint4 *rp = reinterpret_cast<uint4 *>(s_io + row * (long long)s);
-  const float l2e = 1.4426950408889634f * scale;
-  float v[NV][8];
-  float mx = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c0 = (lane + 32 * i) * 8;
-    if (c0 < valid) {
-      unpack8<T>(rp[lane + 32 * i], v[i]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        v[i][e] = (c0 + e < valid) ? v[i][e] * l2e : -INFINITY;
-        mx = fmaxf(mx, v[i][e]);
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float sum = 0.f;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c0 = (lane + 32 * i) * 8;
-    if (c0 < valid) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        v[i][e] = (c0 + e < valid) ? exp2f(v[i][e] - mx) : 0.f;
-        sum += v[i][e];
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  const float inv = 1.0f / sum;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c0 = (lane + 32 * i) * 8;
-    if (c0 < wend) {
-      float o[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = (c0 < valid) ? v[i][e] * inv : 0.f;
-      rp[lane + 32 * i] = pack8<T>(o);
-    }
-  }
-}
-
-// dS = scale * P * (dP - sum_q P*dP), in place over dP; zeros above the
-// diagonal inside the diagonal tile.
-template <typename T, int NV>
-__global__ void __launch_bounds__(256) softmax_bwd_kernel(const T *__restrict__ prob,
-                                                          T *__restrict__ d_io, long long nrows,
-                                                          int s, float scale) {
-  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  if (row >= nrows) return;
-  const int p = (int)(row % s);
-  const int valid = p + 1;
-  const int wend = min(s, (p / 128 + 1) * 128);
-  const uint4 *pp = reinterpret_cast<const uint4 *>(prob + row * (long long)s);
-  uint4 *dp = reinterpret_cast<uint4 *>(d_io + row * (long long)s);
-  float pv[NV][8], dv[NV][8];
-  float dot = 0.f;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c0 = (lane + 32 * i) * 8;
-    if (c0 < valid) {
-      unpack8<T>(pp[lane + 32 * i], pv[i]);
-      unpack8<T>(dp[lane + 32 * i], dv[i]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (c0 + e >= valid) pv[i][e] = 0.f;
-        dot += pv[i][e] * dv[i][e];
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c0 = (lane + 32 * i) * 8;
-    if (c0 < wend) {
-      float o[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = (c0 < valid) ? scale * pv[i][e] * (dv[i][e] - dot) : 0.f;
-      dp[lane + 32 * i] = pack8<T>(o);
-    }
-  }
-}
-
 // ------------------------------------------------------------- optimizer
 // found_inf |= any exponent field all ones in grad[0, n)  (n % 4 == 0)
 __global__ void __launch_bounds__(256) overflow_kernel(const float4 *__restrict__ g, long long n4,
@@ -503,11 +407,20 @@ __global__ void __launch_bounds__(256) adam_kernel(float4 *__restrict__ master,
                                                    const float4 *__restrict__ grad,
                                                    T *__restrict__ w16, long long n4, AdamArgs a,
                                                    const gptl_scaler_state *st) {
-  if (st->found_inf) return;
-  const float scale = st->scale;
-  const int t = st->step + 1;
-  const float bc1 = (float)(1.0 - pow((double)a.beta1, (double)t));
-  const float bc2 = (float)(1.0 - pow((double)a.beta2, (double)t));
+  // the scaler state and the bias corrections 1 - beta^t (in fp64) are read
+  // and formed once per block, not per thread
+  __shared__ float sh[3];
+  __shared__ int skip;
+  if (threadIdx.x == 0) {
+    skip = st->found_inf;
+    const int t = st->step + 1;
+    sh[0] = st->scale;
+    sh[1] = (float)(1.0 - pow((double)a.beta1, (double)t));
+    sh[2] = (float)(1.0 - pow((double)a.beta2, (double)t));
+  }
+  __syncthreads();
+  if (skip) return;
+  const float scale = sh[0], bc1 = sh[1], bc2 = sh[2];
   const float omb1 = 1.0f - a.beta1, omb2 = 1.0f - a.beta2;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (long long)gridDim.x * blockDim.x) {

@@ -12,8 +12,6 @@
 //     split's partial sums and the column split's input-gradient sums are
 //     accumulated in one TMEM accumulator: "Megatron-LM 3D parallelism" §1
 //     describes the all-reduce this replaces);
-//   * causal rules (skip tiles above the diagonal, or limit the K range to
-//     the lower triangle), kept for the unfused attention products;
 //   * fused epilogues: bias, residual, bias+GeLU (writes Z and GeLU(Z): the
 //     fused_bias_gelu of "Training GPT-2 with Megatron-LM" §6.2), GeLU'
 //     scaling of an input gradient, fp32 weight-gradient store;
@@ -44,7 +42,6 @@ enum : int { kActNone = 0, kActGelu = 1, kActDGelu = 2 };
 
 constexpr int kStageBoxBytes = 2048;                 // one 32-row x 64-byte store box
 constexpr int kStagingBytes = 8 * 2 * kStageBoxBytes;  // two boxes per epilogue warp
-enum : int { kCausalNone = 0, kCausalSkipUpper = 1, kCausalKBelow = 2, kCausalKFrom = 3 };
 
 struct OperandRule {
   int mn_major;                // 0: K-major, 1: MN-major
@@ -60,7 +57,7 @@ struct alignas(64) GemmParams {
   CUtensorMap map_o;           // output, or the split-K partials; box {64 B / elem, 32, 1, 1}
   CUtensorMap map_o2;          // GeLU(Z) when act == GELU
   OperandRule ra, rb;
-  int M, N, K, groups, k_shards, causal;
+  int M, N, K, groups, k_shards;
   int split;                   // K slices per tile (split-K); 1 = none
   int pipe_k;                  // 1: both pipelines work on every tile, one K half each
   int m2;                      // 1: 256-row tiles, one M half per pipeline, one shared ring
@@ -83,11 +80,14 @@ struct alignas(64) GemmParams {
   long long ldo;
   long long o_str_mod, o_str_div;
   int act;
+  int *nonfinite;              // fp32 outputs: set to 1 if any value written is inf or NaN
 };
+
+// true when an fp32 value is inf or NaN (all exponent bits set)
+__device__ __forceinline__ bool not_finite(float v) { return !(fabsf(v) <= 3.402823466e38f); }
 
 struct TileInfo {
   int g, m0, n0, kb_begin, kb_end, slice;
-  bool skip;
 };
 
 __device__ __forceinline__ TileInfo tile_info(const GemmParams &p, long long idx) {
@@ -100,11 +100,8 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams &p, long long idx
   const int mt = rem / p.n_tiles, nt = rem - (rem / p.n_tiles) * p.n_tiles;
   t.m0 = mt * (p.m2 ? 2 * kBM : kBM);
   t.n0 = nt * p.bn;
-  t.skip = (p.causal == kCausalSkipUpper) && (t.n0 > t.m0 + kBM - 1);
   t.kb_begin = 0;
   t.kb_end = (p.K + kBK - 1) / kBK;
-  if (p.causal == kCausalKBelow) t.kb_end = (min(p.K, t.m0 + kBM) + kBK - 1) / kBK;
-  if (p.causal == kCausalKFrom) t.kb_begin = t.m0 / kBK;
   if (p.split > 1) {           // balanced slices, none empty while split <= k-blocks
     const int nkb = t.kb_end - t.kb_begin, b = t.kb_begin;
     t.kb_begin = b + (int)((long long)t.slice * nkb / p.split);
@@ -159,11 +156,12 @@ struct EpiRow {
   const uint8_t *bias;
   const uint8_t *resid;
   const uint8_t *aux;
+  bool row_ok;                 // the row is inside M
 };
 
 template <typename T>
 __device__ __forceinline__ EpiRow epilogue_row(const GemmParams &p, int g, int row) {
-  EpiRow e{nullptr, nullptr, nullptr};
+  EpiRow e{nullptr, nullptr, nullptr, row < p.M};
   if (p.split > 1 || row >= p.M) return e;
   if (p.bias) e.bias = reinterpret_cast<const uint8_t *>(static_cast<const T *>(p.bias) +
                                                         (long long)g * p.bias_g_stride);
@@ -213,7 +211,8 @@ __device__ __forceinline__ uint32_t box_piece(uint32_t box, int r, int j) {
 template <typename T>
 __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow &e,
                                                const uint32_t (&r)[16], const EpiIn &in,
-                                               uint32_t box, uint32_t box2, int lane, int slot) {
+                                               uint32_t box, uint32_t box2, int lane, int slot,
+                                               bool &bad) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
@@ -244,6 +243,10 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow
     }
   }
   if (p.out_f32 || p.split > 1) {
+    if (p.nonfinite && p.split == 1 && e.row_ok) {   // split-K: checked on the final sums
+#pragma unroll
+      for (int i = 0; i < 16; ++i) bad |= not_finite(v[i]);
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j)
       st_shared_v4(box_piece(box, lane, j),
@@ -372,10 +375,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       // ------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0, issued = 0, parity = 0;
-      int t = 0;                              // local tile counter (non-skipped tiles)
+      int t = 0;                              // local tile counter
       for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
         const TileInfo ti = tile_info(p, idx);
-        if (ti.skip) continue;
         if (!pipe_takes(p, t++, pp)) continue;
         int kb0, kb1;
         pipe_kb_range(p, ti, pp, kb0, kb1);
@@ -410,7 +412,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       const int ring = p.m2 ? 0 : pp;
       for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
         const TileInfo ti = tile_info(p, idx);
-        if (ti.skip) continue;
         if (!pipe_takes(p, t++, pp)) continue;
         if (!mbar_wait(tempty_bar(pp), acc_phase ^ 1, abort_flag)) goto mma_abort;
         tc_fence_after();
@@ -454,11 +455,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     const bool gelu = !wide && p.act == kActGelu;   // Z and GeLU(Z): both boxes per chunk pair
     const uint32_t my_boxes = staging_s + (uint32_t)((warp - 4) * 2 * kStageBoxBytes);
     int box_i = 0;                           // boxes issued by this warp (selects the buffer)
+    bool bad = false;                        // an fp32 output value was inf or NaN
     uint32_t acc_phase[2] = {0u, 0u};
     int t = 0;
     for (long long idx = blockIdx.x; idx < p.total_tiles; idx += gridDim.x) {
       const TileInfo ti = tile_info(p, idx);
-      if (ti.skip) continue;
       // accumulator of this tile; with pipe_k or m2 both are (pp = 0 and 1)
       const bool both = p.pipe_k || p.m2;
       const int pp = both ? 0 : (t & 1);
@@ -514,7 +515,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
           }
           __syncwarp();
         }
-        epilogue_chunk<T>(p, er, r, in, buf, my_boxes + kStageBoxBytes, lane, slot);
+        epilogue_chunk<T>(p, er, r, in, buf, my_boxes + kStageBoxBytes, lane, slot, bad);
         if (last) {
           fence_proxy_async_smem();
           __syncwarp();
@@ -560,6 +561,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         if (both) mbar_arrive(tempty_bar(1));
       }
     }
+    if (p.nonfinite && __any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.nonfinite, 1);
     // the staged boxes must be read, and the stores done, before the CTA exits
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -574,14 +576,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
 }
 
 // out[G](m, n) = sum over s < split of ws[s][G][m][n], in slice order, into
-// the strided fp32 output of the GEMM; 4 columns per thread.
+// the strided fp32 output of the GEMM; 4 columns per thread.  With
+// `nonfinite`, any inf or NaN sum sets it to 1.
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restrict__ ws,
                                                            long long ws_slice, int split, int M,
                                                            int N, int groups, float *out,
                                                            long long ldo, int o_mod,
                                                            long long o_str_mod,
-                                                           long long o_str_div) {
+                                                           long long o_str_div, int *nonfinite) {
   const long long n4 = ws_slice / 4;
+  bool bad = false;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (long long)gridDim.x * blockDim.x) {
     const long long e = i * 4;
@@ -596,47 +600,58 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restr
     const long long off = (long long)(g % o_mod) * o_str_mod + (long long)(g / o_mod) * o_str_div +
                           (long long)m * ldo + n;
     *reinterpret_cast<float4 *>(out + off) = acc;
+    bad |= not_finite(acc.x) | not_finite(acc.y) | not_finite(acc.z) | not_finite(acc.w);
   }
+  if (nonfinite && __any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(nonfinite, 1);
 }
 
 // Row term of the softmax backward: D[g][p] = sum_c dO[p][c] * O[p][c] over
 // the head's d columns (equal to sum_q P[p][q] dP[p][q], since O = P V).
-// A warp per row of the [t*b*s][h/t] matrices reads the row in coalesced
-// 16-byte vectors and leaves one partial dot per vector in shared memory;
-// then one thread per (row, head) adds the head's d/8 partials in order.
-// Block: 8 rows; hs / 8 <= kRowdotMaxVec vectors per row.
-constexpr int kRowdotMaxVec = 512;
+// A block takes 8 rows of the [t*b*s][h/t] matrices and walks them in chunks
+// of whole heads (at most kRowdotChunkVec 16-byte vectors per row): a warp per
+// row reads the chunk in coalesced vectors and leaves one partial dot per
+// vector in shared memory; then one thread per (row, head of the chunk) adds
+// the head's d/8 partials in order.  Any row width and number of heads.
+constexpr int kRowdotChunkVec = 512;
 template <typename T>
 __global__ void __launch_bounds__(256) attn_rowdot_kernel(const T *__restrict__ dout,
                                                           const T *__restrict__ o, float *__restrict__ dvec,
                                                           long long rows, int s, int hs, int as,
                                                           int d) {
-  __shared__ float part[8][kRowdotMaxVec];
+  __shared__ float part[8][kRowdotChunkVec];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long r = (long long)blockIdx.x * 8 + w;
-  const int nv = hs / 8;
-  if (r < rows) {
-    const uint4 *a = reinterpret_cast<const uint4 *>(dout + r * hs);
-    const uint4 *b = reinterpret_cast<const uint4 *>(o + r * hs);
-    for (int v = lane; v < nv; v += 32) {
-      float fa[8], fb[8];
-      unpack8<T>(__ldcs(a + v), fa);
-      unpack8<T>(__ldcs(b + v), fb);
-      float acc = 0.f;
+  const long long r0 = (long long)blockIdx.x * 8;
+  const long long r = r0 + w;
+  const int vh = d / 8;                        // vectors per head
+  const int hpc = kRowdotChunkVec / vh;        // whole heads per chunk
+  for (int h0 = 0; h0 < as; h0 += hpc) {
+    const int nh = min(hpc, as - h0);
+    const int nv = nh * vh;
+    if (r < rows) {
+      const uint4 *a = reinterpret_cast<const uint4 *>(dout + r * hs) + h0 * vh;
+      const uint4 *b = reinterpret_cast<const uint4 *>(o + r * hs) + h0 * vh;
+      for (int v = lane; v < nv; v += 32) {
+        float fa[8], fb[8];
+        unpack8<T>(__ldcs(a + v), fa);
+        unpack8<T>(__ldcs(b + v), fb);
+        float acc = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc = fmaf(fa[e], fb[e], acc);
-      part[w][v] = acc;
+        for (int e = 0; e < 8; ++e) acc = fmaf(fa[e], fb[e], acc);
+        part[w][v] = acc;
+      }
     }
-  }
-  __syncthreads();
-  const int rl = threadIdx.x / as, head = threadIdx.x - rl * as;   // (row in block, head)
-  const long long rr = (long long)blockIdx.x * 8 + rl;
-  if (rl < 8 && rr < rows) {
-    const int vh = d / 8;
-    float acc = 0.f;
-    for (int v = 0; v < vh; ++v) acc += part[rl][head * vh + v];
-    const long long zb = rr / s, pos = rr - zb * s;
-    dvec[(zb * as + head) * s + pos] = acc;
+    __syncthreads();
+    for (int i = threadIdx.x; i < 8 * nh; i += blockDim.x) {
+      const int rl = i / nh, hc = i - rl * nh;    // (row in block, head in chunk)
+      const long long rr = r0 + rl;
+      if (rr < rows) {
+        float acc = 0.f;
+        for (int v = 0; v < vh; ++v) acc += part[rl][hc * vh + v];
+        const long long zb = rr / s, pos = rr - zb * s;
+        dvec[(zb * as + h0 + hc) * s + pos] = acc;
+      }
+    }
+    __syncthreads();
   }
 }
 

@@ -11,11 +11,15 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
+#include <mutex>
+
 #include "bw_kernels.cuh"
 #include "common.cuh"
 #include "attn_bwd_tc.cuh"
 #include "attn_tc.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_pair.cuh"
 #include "gptlayer_parts.h"
 #include "gptlayer_profile.h"
 
@@ -63,6 +67,15 @@ struct Profiler {
 Profiler g_prof;
 int g_tag = GPTL_TAG_NONE;
 unsigned long long g_launches = 0;
+// While a checked backward runs on this host thread (gpt_layer_bwd_checked),
+// the device word that the kernels writing gradients set on an inf or NaN:
+// the fp32-output GEMMs, their split-K sums and the column-sum reductions.
+thread_local int *g_nonfinite = nullptr;
+struct NonfiniteScope {
+  int *saved;
+  explicit NonfiniteScope(int *f) : saved(g_nonfinite) { g_nonfinite = f; }
+  ~NonfiniteScope() { g_nonfinite = saved; }
+};
 
 cudaEvent_t prof_event(cudaStream_t st) {
   if (g_prof.pool_next >= g_prof.pool_n) return nullptr;
@@ -228,7 +241,6 @@ int check_operand(const gptl_operand &o) {
 }
 
 int pick_bn(const gptl_gemm_desc &d, int sms) {
-  if (d.causal == GPTL_CAUSAL_SKIP_UPPER) return d.N >= 128 ? 128 : d.N;
   if (d.N <= 256) return d.N;
   const long long m_tiles = (d.M + kBM - 1) / kBM;
   long long best_cost = -1;
@@ -252,35 +264,45 @@ int pick_bn(const gptl_gemm_desc &d, int sms) {
 //   alternate   tiles alternate between the pipelines, 128 x BN tiles:
 //               1.17 per k-block of each pipeline (0.9 when one runs alone);
 //               one tile's epilogue overlaps the other pipeline's MMAs
-//   K halves    both pipelines on one 128 x BN tile: 1.17 per k-block of each
+//   K halves    both pipelines on one 128 x BN tile: 1.13 per k-block of each
 //   m2          256 x BN tiles, one M half per pipeline, one shared ring:
-//               ~1.0 per k-block of the pair (a third less operand traffic
+//               0.8 per k-block of the pair (a third less operand traffic
 //               from L2 per FLOP than 128 x BN tiles)
-// The last two cannot overlap a tile's epilogue with the next tile's MMAs
-// (all 512 TMEM columns hold the tile): ~1.3 us per 128 x 256 half tile,
-// ~5 with GeLU / GeLU' (measured: the 256-row mode loses to alternating
-// tiles on the GeLU GEMMs, wins on the others).  Split-K adds the partial-sum
-// pass, (2 split + 1) fp32 arrays at ~4 TB/s plus a launch.
+// Narrower tiles (BN 224, 192, 160, 128) take proportionally less: half of
+// the time scales with the MMA work (BN) and half with the operand bytes
+// (rows of A + BN).  They trade a little of that rate for a tile count that
+// fills the last wave: a 2048 x 10240 output is 320 tiles of 256 x 256 (2.2
+// waves of 148 SMs, so three rounds at 72 % occupancy) but 432 tiles of
+// 256 x 192 (2.9 waves, 97 %).
+// The K-halves and m2 modes cannot overlap a tile's epilogue with the next
+// tile's MMAs (all 512 TMEM columns hold the tile): ~1.3 us per 128 x 256
+// half tile, ~5 with GeLU / GeLU' (measured: the 256-row mode loses to
+// alternating tiles on the GeLU GEMMs, wins on the others).  Split-K adds the
+// partial-sum pass, (2 split + 1) fp32 arrays at ~4 TB/s plus a launch.
 struct GemmTiling {
-  int bn, split, pipe_k, m2;
+  int bn, split, pipe_k, m2, pair;
 };
 GemmTiling choose_tiling(const gptl_gemm_desc &d, int sms, bool can_split) {
-  GemmTiling best{pick_bn(d, sms), 1, 0, 0};
-  if (d.causal != GPTL_CAUSAL_NONE) return best;
+  GemmTiling best{pick_bn(d, sms), 1, 0, 0, 0};
   const long long kb_all = (long long)((d.K + kBK - 1) / kBK) * d.k_shards;
   const double out_bytes = (double)d.groups * d.M * d.N * 4.0;
   const double e_half = (d.act == GPTL_ACT_NONE ? 1.3 : 5.0);
   double best_t = -1.0;
-  const int n_bn = d.N <= 256 ? 1 : 2;
-  for (int ib = 0; ib < n_bn; ++ib) {
-    const int bn = d.N <= 256 ? d.N : (ib == 0 ? 256 : 128);
+  static const int kBnChoices[] = {256, 224, 192, 160, 128};
+  for (int bn_c : kBnChoices) {
+    const int bn = d.N <= 256 ? d.N : bn_c;
+    if (d.N <= 256 && bn_c != 256) break;         // N fits one tile column: BN = N
     const double e_tile = e_half * bn / 256.0;
     const long long n_tiles = (d.N + bn - 1) / bn;
-    for (int mode = 0; mode < 3; ++mode) {          // alternate, K halves, m2
-      if (mode == 2 && d.M <= kBM) continue;
-      const long long m_tiles = (d.M + (mode == 2 ? 2 * kBM : kBM) - 1) / (mode == 2 ? 2 * kBM : kBM);
+    for (int mode = 0; mode < 4; ++mode) {          // alternate, K halves, m2, CTA pairs
+      if (mode >= 2 && d.M <= kBM) continue;
+      if (mode == 3 && (bn % 32 || sms < 2)) continue;   // each CTA of a pair takes BN/2 rows of B
+      const int rows = mode >= 2 ? 2 * kBM : kBM;
+      const long long m_tiles = (d.M + rows - 1) / rows;
       const long long tiles = m_tiles * n_tiles * d.groups;
-      for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
+      // per-k-block time of this BN: half scales with BN, half with A rows + BN
+      const double width = 0.5 * bn / 256.0 + 0.5 * (double)(rows + bn) / (double)(rows + 256);
+      for (int sp = 1; sp <= (can_split && mode != 3 ? 8 : 1); ++sp) {
         if (sp > (d.K + kBK - 1) / kBK) break;
         if (sp > 1 && (double)sp * out_bytes > (double)d.ws_bytes) break;
         // K halves: every slice must give each pipeline at least one k-block
@@ -288,17 +310,22 @@ GemmTiling choose_tiling(const gptl_gemm_desc &d, int sms, bool can_split) {
         const long long items = tiles * sp;
         const long long kb = (kb_all + sp - 1) / sp;
         const long long per_cta = (items + sms - 1) / sms;
+        const long long per_pair = (items + sms / 2 - 1) / (sms / 2);
         double t;
         if (mode == 0)
-          t = per_cta >= 2 ? (double)((per_cta + 1) / 2) * kb * 1.17 + e_tile : kb * 0.9 + e_tile;
+          t = per_cta >= 2 ? (double)((per_cta + 1) / 2) * kb * 1.17 * width + e_tile
+                           : kb * 0.9 * width + e_tile;
         else if (mode == 1)
-          t = (double)per_cta * ((kb + 1) / 2 * 1.17 + e_tile);
-        else
-          t = (double)per_cta * (kb * 1.0 + 2.0 * e_tile);
+          t = (double)per_cta * ((kb + 1) / 2 * 1.13 * width + e_tile);
+        else if (mode == 2)
+          t = (double)per_cta * (kb * 0.8 * width + 2.0 * e_tile);
+        else    // a pair's tile: each SM half the MMA work of m2's per k-block; the
+                // epilogue overlaps the next tile's MMAs, except where it is longer
+          t = (double)per_pair * std::max(kb * 0.42 * width, 2.0 * e_tile) + 2.0 * e_tile;
         if (sp > 1) t += (2.0 * sp + 1.0) * out_bytes / 4.0e6 + 3.0;
         if (best_t < 0 || t < best_t * 0.999) {
           best_t = t;
-          best = GemmTiling{bn, sp, mode == 1 ? 1 : 0, mode == 2 ? 1 : 0};
+          best = GemmTiling{bn, sp, mode == 1 ? 1 : 0, mode >= 2 ? 1 : 0, mode == 3 ? 1 : 0};
         }
       }
     }
@@ -322,13 +349,29 @@ int launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) 
   return GPTL_OK;
 }
 
+template <typename T>
+int launch_gemm_pair_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) {
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  GPTL_CK(cudaGetDevice(&dev));
+  if (!attr_set[dev]) {
+    GPTL_CK(cudaFuncSetAttribute(gemm_pair_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemLimit));
+    attr_set[dev] = true;
+  }
+  gemm_pair_kernel<T><<<grid, kPairThreads, smem, stream>>>(p);   // clusters of 2 (static)
+  GPTL_CK(cudaGetLastError());
+  prof_launched(stream, GPTL_KIND_GEMM);
+  return GPTL_OK;
+}
+
 // Argument checks of gptl_gemm (no device work).
 int gemm_validate(const gptl_gemm_desc &d, gptl_dtype dt) {
   if (dt != GPTL_FP16 && dt != GPTL_BF16) return GPTL_E_DTYPE;
   if (!d.out) return GPTL_E_NULL;
   if (!aligned16(d.out)) return GPTL_E_ALIGN;
   if (d.M <= 0 || d.N <= 0 || d.K <= 0 || d.groups <= 0 || d.k_shards <= 0) return GPTL_E_SHAPE;
-  if (d.K % 16 || d.N % 16 || d.causal < 0 || d.causal > 3 || d.o_mod < 1) return GPTL_E_SHAPE;
+  if (d.K % 16 || d.N % 16 || d.causal != 0 || d.o_mod < 1) return GPTL_E_SHAPE;
   const int oal = d.out_f32 ? 4 : 8;
   if (d.ldo % oal || d.o_str_mod % oal || d.o_str_div % oal || d.ldo < d.N) return GPTL_E_SHAPE;
   if (d.bias && (!aligned16(d.bias) || d.bias_g_stride % 8)) return GPTL_E_ALIGN;
@@ -344,8 +387,8 @@ int gemm_validate(const gptl_gemm_desc &d, gptl_dtype dt) {
 }
 
 GemmTiling gemm_plan(const gptl_gemm_desc &d, int sms) {
-  const bool can_split = d.out_f32 && !d.bias && !d.resid && d.act == GPTL_ACT_NONE &&
-                         d.causal == GPTL_CAUSAL_NONE && d.ws && aligned16(d.ws);
+  const bool can_split = d.out_f32 && !d.bias && !d.resid && d.act == GPTL_ACT_NONE && d.ws &&
+                         aligned16(d.ws);
   return choose_tiling(d, sms, can_split);
 }
 
@@ -357,11 +400,13 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   memset(&p, 0, sizeof(p));
   const GemmTiling tl = gemm_plan(d, sms);
   const int bn = tl.bn;
+  // rows of A and B staged per SM: a pair's CTA takes 128 rows of A and BN/2 of B
+  const int a_rows = tl.m2 && !tl.pair ? 2 * kBM : kBM;
+  const int b_rows = tl.pair ? bn / 2 : bn;
   const int wa = d.a.mn_major ? mn_chunk_width(kBM) : 64;
-  const int wb = d.b.mn_major ? mn_chunk_width(bn) : 64;
-  const int a_rows = tl.m2 ? 2 * kBM : kBM;   // rows of A per tile
+  const int wb = d.b.mn_major ? mn_chunk_width(b_rows) : 64;
   GPTL_TRY(encode_operand(&p.map_a, d.a, dt, a_rows, wa));
-  GPTL_TRY(encode_operand(&p.map_b, d.b, dt, bn, wb));
+  GPTL_TRY(encode_operand(&p.map_b, d.b, dt, b_rows, wb));
   auto rule = [](const gptl_operand &o, int w) {
     OperandRule r;
     r.mn_major = o.mn_major;
@@ -380,24 +425,27 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.K = d.K;
   p.groups = d.groups;
   p.k_shards = d.k_shards;
-  p.causal = d.causal;
   p.bn = bn;
   int bn_alloc = 32;
   while (bn_alloc < bn) bn_alloc *= 2;
   p.bn_alloc = bn_alloc;
   p.tmem_cols = 2 * bn_alloc;
-  const int stage_bytes = (a_rows + bn) * kBK * 2;
+  const int stage_bytes = (a_rows + b_rows) * kBK * 2;
   // stages per ring: two rings (one per pipeline), or one shared ring in m2
+  // and in a pair's CTA
   const int rings = tl.m2 ? 1 : 2;
   p.stages = (kSmemLimit - 2048 - kStagingBytes) / (rings * stage_bytes);
-  if (p.stages > 4) p.stages = 4;
+  const int max_stages = tl.pair ? kPairMaxStages : 4;
+  if (p.stages > max_stages) p.stages = max_stages;
   if (p.stages < 2) return GPTL_E_SHAPE;
   const int smem = 1024 + rings * p.stages * stage_bytes + kStagingBytes + 512;
   const uint32_t fmt = dt == GPTL_BF16 ? 1u : 0u;
+  const int mma_m = tl.pair ? 2 * kBM : kBM;    // a pair's MMA spans both CTAs' rows
   p.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)d.a.mn_major << 15) |
             ((uint32_t)d.b.mn_major << 16) | ((uint32_t)(bn >> 3) << 17) |
-            ((uint32_t)(kBM >> 4) << 24);
-  p.m_tiles = (d.M + a_rows - 1) / a_rows;
+            ((uint32_t)(mma_m >> 4) << 24);
+  const int tile_rows = tl.m2 ? 2 * kBM : kBM;
+  p.m_tiles = (d.M + tile_rows - 1) / tile_rows;
   p.n_tiles = (d.N + bn - 1) / bn;
   const long long tiles = (long long)p.m_tiles * p.n_tiles * d.groups;
   p.split = tl.split;
@@ -432,6 +480,13 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.ld_resid = d.ld_resid;
   p.aux = d.aux;
   p.act = d.act;
+  p.nonfinite = d.out_f32 ? g_nonfinite : nullptr;
+  if (tl.pair) {
+    const long long pairs = p.total_tiles < sms / 2 ? p.total_tiles : sms / 2;
+    if (dt == GPTL_FP16) GPTL_TRY(launch_gemm_pair_t<__half>(p, (int)(2 * pairs), smem, stream));
+    else GPTL_TRY(launch_gemm_pair_t<__nv_bfloat16>(p, (int)(2 * pairs), smem, stream));
+    return GPTL_OK;
+  }
   const int grid = (int)(p.total_tiles < sms ? p.total_tiles : sms);
   if (dt == GPTL_FP16) GPTL_TRY(launch_gemm_t<__half>(p, grid, smem, stream));
   else GPTL_TRY(launch_gemm_t<__nv_bfloat16>(p, grid, smem, stream));
@@ -441,7 +496,7 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
     if (blocks > 8 * sms) blocks = 8 * sms;
     splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
         p.ws, p.ws_slice, p.split, d.M, d.N, d.groups, static_cast<float *>(d.out), d.ldo,
-        d.o_mod, d.o_str_mod, d.o_str_div);
+        d.o_mod, d.o_str_mod, d.o_str_div, p.nonfinite);
     GPTL_CK(cudaGetLastError());
     prof_launched(stream, GPTL_KIND_SPLITK);
   }
@@ -494,14 +549,14 @@ int run_attn_fwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
   p.lse = lse;
   p.items = (long long)p.groups * p.q_tiles;
   p.q_off = 0; p.k_off = hs; p.v_off = 2 * hs;
-  // P 32 KB + Q + 2 stages of K and V, barriers; at least 120 KB so that one
-  // CTA (and its 512 tensor-memory columns) owns each SM
   // P 2 x 32 KB, Q, the K / V ring (as deep as fits, 2..4 stages), barriers
+  // and the half-row lse; at least 120 KB so that one CTA (and its 512
+  // tensor-memory columns) owns each SM
   const int kv_stage = 2 * 128 * d * 2;
-  p.kv_stages = (kSmemLimit - 1024 - 65536 - 128 * d * 2 - 512) / kv_stage;
+  p.kv_stages = (kSmemLimit - 1024 - 65536 - 128 * d * 2 - kAttnTailBytes) / kv_stage;
   if (p.kv_stages > 4) p.kv_stages = 4;
   if (p.kv_stages < 2) return GPTL_E_SHAPE;
-  int smem = 1024 + 65536 + 128 * d * 2 + p.kv_stages * kv_stage + 512;
+  int smem = 1024 + 65536 + 128 * d * 2 + p.kv_stages * kv_stage + kAttnTailBytes;
   if (smem < 120 * 1024) smem = 120 * 1024;
   const int grid = (int)(p.items < sms ? p.items : sms);
   // the shared-memory opt-in is recorded per device and per dtype (both
@@ -662,7 +717,7 @@ int run_transpose(int rows, int cols, const void *in, long long ld_in, void *out
 // D[g][p] = dO_p . O_p over each head's columns (the softmax backward's row term).
 int run_attn_rowdot(long long rows, int s, int hs, int as, int d, gptl_dtype dt, const void *dout,
                     const void *o, float *dvec, cudaStream_t st) {
-  if (hs % 8 || d % 8 || hs / 8 > kRowdotMaxVec || as > 32) return GPTL_E_SHAPE;
+  if (hs % 8 || d % 8 || d <= 0 || d / 8 > kRowdotChunkVec || (long long)as * d != hs) return GPTL_E_SHAPE;
   const unsigned grid = (unsigned)((rows + 7) / 8);
   if (dt == GPTL_FP16)
     attn_rowdot_kernel<__half><<<grid, 256, 0, st>>>((const __half *)dout, (const __half *)o, dvec,
@@ -705,6 +760,16 @@ bool ln_dispatch(int vpt, F &&f) {
   }
 }
 
+// Dynamic shared memory of ln_bwd_kernel with `nparts` running column sums
+// per row team (0 when h has no split).  The kernel's static shared memory is
+// under 1 KB; kLnBwdSmemMax keeps that margin below the opt-in limit.
+constexpr int kLnBwdSmemMax = kSmemLimit - 1024;
+long long ln_bwd_smem(int h, int nparts) {
+  int tpr = 0, vpt = 0;
+  if (!ln_split(h, &tpr, &vpt)) return 0;
+  return (long long)(256 / tpr) * nparts * h * (long long)sizeof(float);
+}
+
 int ln_bwd_blocks(int rows, int h, int sms) {
   int tpr = 0, vpt = 0;
   if (!ln_split(h, &tpr, &vpt)) return 0;
@@ -743,7 +808,7 @@ int run_ln_fwd(int rows, int h, gptl_dtype dt, const void *x, int x_f32, const v
 
 int launch_reduce_parts(const float *part, int nblocks, int n, int nk, float *o0, float *o1,
                         float *o2, float *o3, cudaStream_t st) {
-  PartOuts outs{{o0, o1, o2, o3}};
+  PartOuts outs{{o0, o1, o2, o3}, g_nonfinite};
   reduce_parts_kernel<<<dim3((n + 31) / 32, nk), dim3(32, 16), 0, st>>>(part, nblocks, n, outs);
   GPTL_CK(cudaGetLastError());
   prof_launched(st, GPTL_KIND_REDUCE);
@@ -767,7 +832,9 @@ int run_ln_bwd(int variant, int rows, int h, gptl_dtype dt, const void *gy, cons
   if (!ln_split(h, &tpr, &vpt) || rows <= 0) return GPTL_E_SHAPE;
   const int nb = ln_bwd_blocks(rows, h, sms);
   const int nparts = variant == LNB_H ? 4 : (variant == LNB_X ? 2 : (dx_sum ? 3 : 2));
-  const int smem = (256 / tpr) * nparts * h * (int)sizeof(float);   // per-team running sums
+  const long long smem_ll = ln_bwd_smem(h, nparts);   // per-team running sums
+  if (smem_ll <= 0 || smem_ll > kLnBwdSmemMax) return GPTL_E_SHAPE;
+  const int smem = (int)smem_ll;
   int rc = GPTL_OK;
   const bool ok = ln_dispatch(vpt, [&]<int VP>() {
     auto go = [&]<typename T, typename TX, typename TR, bool D32, bool SDX, bool SRS>() {
@@ -798,53 +865,6 @@ int run_ln_bwd(int variant, int rows, int h, gptl_dtype dt, const void *gy, cons
   if (variant == LNB_H) return launch_reduce_parts(part, nb, h, 4, dg, db, dx_sum, resid_sum, st);
   if (variant == LNB_X) return launch_reduce_parts(part, nb, h, 2, dg, db, nullptr, nullptr, st);
   return launch_reduce_parts(part, nb, h, dx_sum ? 3 : 2, dg, db, dx_sum, nullptr, st);
-}
-
-// ------------------------------------------------------------- softmax
-int softmax_nv(int s) {
-  const int nv = (s + 255) / 256;
-  return nv <= 1 ? 1 : (nv <= 2 ? 2 : (nv <= 4 ? 4 : 8));
-}
-
-int run_softmax_fwd(long long blocks, int s, gptl_dtype dt, float scale, void *sc,
-                    cudaStream_t st) {
-  if (blocks <= 0 || s <= 0 || s % 16 || s > 2048) return GPTL_E_SHAPE;
-  const long long rows = blocks * s;
-  const unsigned grid = (unsigned)((rows + 7) / 8);
-  const int nv = softmax_nv(s);
-#define GPTL_SMF(T, NV)                                                                   \
-  if (nv == NV) softmax_fwd_kernel<T, NV><<<grid, 256, 0, st>>>((T *)sc, rows, s, scale);
-  if (dt == GPTL_FP16) {
-    GPTL_SMF(__half, 1) GPTL_SMF(__half, 2) GPTL_SMF(__half, 4) GPTL_SMF(__half, 8)
-  } else {
-    GPTL_SMF(__nv_bfloat16, 1) GPTL_SMF(__nv_bfloat16, 2) GPTL_SMF(__nv_bfloat16, 4)
-    GPTL_SMF(__nv_bfloat16, 8)
-  }
-#undef GPTL_SMF
-  GPTL_CK(cudaGetLastError());
-  prof_launched(st, GPTL_KIND_SOFTMAX_FWD);
-  return GPTL_OK;
-}
-
-int run_softmax_bwd(long long blocks, int s, gptl_dtype dt, float scale, const void *pr, void *dp,
-                    cudaStream_t st) {
-  if (blocks <= 0 || s <= 0 || s % 16 || s > 2048) return GPTL_E_SHAPE;
-  const long long rows = blocks * s;
-  const unsigned grid = (unsigned)((rows + 7) / 8);
-  const int nv = softmax_nv(s);
-#define GPTL_SMB(T, NV)                                                                        \
-  if (nv == NV)                                                                                \
-    softmax_bwd_kernel<T, NV><<<grid, 256, 0, st>>>((const T *)pr, (T *)dp, rows, s, scale);
-  if (dt == GPTL_FP16) {
-    GPTL_SMB(__half, 1) GPTL_SMB(__half, 2) GPTL_SMB(__half, 4) GPTL_SMB(__half, 8)
-  } else {
-    GPTL_SMB(__nv_bfloat16, 1) GPTL_SMB(__nv_bfloat16, 2) GPTL_SMB(__nv_bfloat16, 4)
-    GPTL_SMB(__nv_bfloat16, 8)
-  }
-#undef GPTL_SMB
-  GPTL_CK(cudaGetLastError());
-  prof_launched(st, GPTL_KIND_SOFTMAX_BWD);
-  return GPTL_OK;
 }
 
 // ------------------------------------------------------------- col sums
@@ -878,25 +898,67 @@ int run_colsum(int rows, int n, int groups, long long ld, long long gstride, gpt
 // Fixed partial-sum storage of gptl_colsum_noalloc: kColsumMaxSplit partial
 // rows of at most kNoAllocMaxWidth columns.  Host code may not use the
 // array's name as a device address; noalloc_scratch() looks the address up
-// once per device, with that device current.
+// with the device current, once per CUDA context: the cached address is kept
+// with the id of the context it came from, so that a device reset (which
+// ends the context and the array's old mapping with it) leads to a fresh
+// lookup instead of a stale pointer.  A mutex guards the table, which host
+// threads share.
 constexpr int kNoAllocMaxWidth = 16384;
 static __device__ __align__(256) float g_colsum_scratch[(size_t)kColsumMaxSplit * kNoAllocMaxWidth];
-float *g_colsum_scratch_addr[kMaxDevices];
+struct NoAllocSlot {
+  unsigned long long ctx_id;
+  float *addr;
+};
+NoAllocSlot g_colsum_scratch_slot[kMaxDevices];
+std::mutex g_colsum_scratch_mu;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Id of the calling thread's current CUDA context, or 0 when there is none
+// (or the driver cannot say).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    (void)cudaGetLastError();
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 int noalloc_scratch(float **out) {
   int dev = 0;
   GPTL_CK(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return GPTL_E_ARCH;
   GPTL_TRY(device_check());
-  if (!g_colsum_scratch_addr[dev]) {
+  std::lock_guard<std::mutex> lock(g_colsum_scratch_mu);
+  NoAllocSlot &slot = g_colsum_scratch_slot[dev];
+  const unsigned long long id = current_context_id();
+  if (!slot.addr || id == 0 || slot.ctx_id != id) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_colsum_scratch) != cudaSuccess || !p) {
       (void)cudaGetLastError();
       return GPTL_E_CUDA;
     }
-    g_colsum_scratch_addr[dev] = static_cast<float *>(p);
+    slot.addr = static_cast<float *>(p);
+    slot.ctx_id = current_context_id();   // the lookup made the context current if it was not
   }
-  *out = g_colsum_scratch_addr[dev];
+  *out = slot.addr;
   return GPTL_OK;
 }
 
@@ -920,6 +982,12 @@ int check_shape(const gptl_shape *sh, Dims *D) {
   if (!(sh->ln_eps > 0.f)) return GPTL_E_SHAPE;
   int tpr, vpt;
   if (!ln_split(h, &tpr, &vpt)) return GPTL_E_SHAPE;
+  // every launch-time limit of the step is checked here, so that no call
+  // fails after its first launch: the LayerNorm backward's running sums (four
+  // per row team in the LayerNorm-2 backward) must fit in shared memory.  The
+  // attention kernels' shared memory fits for every d <= 128, and the GEMM's
+  // stages for every tile it picks.
+  if (ln_bwd_smem(h, 4) > kLnBwdSmemMax) return GPTL_E_SHAPE;
   D->b = b; D->s = s; D->h = h; D->a = a; D->f = f; D->t = t; D->d = d;
   D->hs = h / t; D->as = a / t; D->fs = f / t;
   D->T = (long long)b * s;
@@ -1326,11 +1394,10 @@ int gpt_layer_fwd(const gptl_shape *shape, const gptl_weights *w, const void *x,
   return layer_fwd(D, w, x, y, saved, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int gpt_layer_bwd(const gptl_shape *shape, const gptl_weights *w, const void *x, const void *saved,
-                  const void *dy, void *dx, const gptl_grads *g, void *scratch,
-                  gptl_stream_t stream) {
-  Dims D;
-  GPTL_TRY(check_shape(shape, &D));
+namespace {
+int bwd_validate(const gptl_shape *shape, const gptl_weights *w, const void *x, const void *saved,
+                 const void *dy, void *dx, const gptl_grads *g, void *scratch, Dims *D) {
+  GPTL_TRY(check_shape(shape, D));
   GPTL_TRY(validate_weights(w));
   if (!x || !saved || !dy || !dx || !g || !scratch) return GPTL_E_NULL;
   if (!aligned16(x) || !aligned16(saved) || !aligned16(dy) || !aligned16(dx) || !aligned16(scratch))
@@ -1341,7 +1408,80 @@ int gpt_layer_bwd(const gptl_shape *shape, const gptl_weights *w, const void *x,
     if (!p) return GPTL_E_NULL;
     if (!aligned16(p)) return GPTL_E_ALIGN;
   }
-  GPTL_TRY(device_check());
+  return device_check();
+}
+
+int adam_validate(size_t n_params, float *master, float *m, float *v, const float *grad, void *w16,
+                  gptl_dtype dtype, float lr, float beta1, float beta2, float eps,
+                  float weight_decay, gptl_scaler_state *st) {
+  if (!master || !m || !v || !grad || !w16 || !st) return GPTL_E_NULL;
+  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
+  if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(grad) || !aligned16(w16) ||
+      (reinterpret_cast<uintptr_t>(st) & 3u))
+    return GPTL_E_ALIGN;
+  if (n_params == 0 || n_params % 4 || !(lr >= 0.f) || !(beta1 >= 0.f && beta1 < 1.f) ||
+      !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f) || !(weight_decay >= 0.f))
+    return GPTL_E_ARG;
+  return device_check();
+}
+
+// O2: the fused unscale + Adam + cast kernel; skips itself when st->found_inf.
+int launch_adam(size_t n_params, float *master, float *m, float *v, const float *grad, void *w16,
+                gptl_dtype dtype, float lr, float beta1, float beta2, float eps,
+                float weight_decay, gptl_scaler_state *st, cudaStream_t s) {
+  int sms = 0;
+  GPTL_TRY(device_check(&sms));
+  const long long n4 = (long long)(n_params / 4);
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > 8 * sms) blocks = 8 * sms;
+  AdamArgs a{lr, beta1, beta2, eps, weight_decay};
+  if (dtype == GPTL_FP16)
+    adam_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(
+        reinterpret_cast<float4 *>(master), reinterpret_cast<float4 *>(m),
+        reinterpret_cast<float4 *>(v), reinterpret_cast<const float4 *>(grad),
+        static_cast<__half *>(w16), n4, a, st);
+  else
+    adam_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+        reinterpret_cast<float4 *>(master), reinterpret_cast<float4 *>(m),
+        reinterpret_cast<float4 *>(v), reinterpret_cast<const float4 *>(grad),
+        static_cast<__nv_bfloat16 *>(w16), n4, a, st);
+  GPTL_CK(cudaGetLastError());
+  prof_launched(s, GPTL_KIND_ADAM);
+  return GPTL_OK;
+}
+}  // namespace
+
+int gpt_layer_bwd_checked(const gptl_shape *shape, const gptl_weights *w, const void *x,
+                          const void *saved, const void *dy, void *dx, const gptl_grads *g,
+                          void *scratch, gptl_scaler_state *st, gptl_stream_t stream) {
+  Dims D;
+  if (!st) return GPTL_E_NULL;
+  if (reinterpret_cast<uintptr_t>(st) & 3u) return GPTL_E_ALIGN;
+  GPTL_TRY(bwd_validate(shape, w, x, saved, dy, dx, g, scratch, &D));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  GPTL_CK(cudaMemsetAsync(&st->found_inf, 0, sizeof(int), s));
+  NonfiniteScope scope(&st->found_inf);
+  return layer_bwd(D, w, x, saved, dy, dx, g, scratch, s);
+}
+
+int adam_step_fp32_master_prechecked(size_t n_params, float *master, float *m, float *v,
+                                     const float *grad, void *w16, gptl_dtype dtype, float lr,
+                                     float beta1, float beta2, float eps, float weight_decay,
+                                     gptl_scaler_state *st, gptl_stream_t stream) {
+  GPTL_TRY(adam_validate(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps,
+                         weight_decay, st));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  TagScope tag_scope(GPTL_TAG_O2_ADAM);
+  prof_start(s);
+  return launch_adam(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps, weight_decay,
+                     st, s);
+}
+
+int gpt_layer_bwd(const gptl_shape *shape, const gptl_weights *w, const void *x, const void *saved,
+                  const void *dy, void *dx, const gptl_grads *g, void *scratch,
+                  gptl_stream_t stream) {
+  Dims D;
+  GPTL_TRY(bwd_validate(shape, w, x, saved, dy, dx, g, scratch, &D));
   return layer_bwd(D, w, x, saved, dy, dx, g, scratch, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1367,36 +1507,13 @@ int gptl_check_overflow(size_t n, const float *grad, gptl_scaler_state *st, gptl
 int adam_step_fp32_master(size_t n_params, float *master, float *m, float *v, const float *grad,
                           void *w16, gptl_dtype dtype, float lr, float beta1, float beta2, float eps,
                           float weight_decay, gptl_scaler_state *st, gptl_stream_t stream) {
-  if (!master || !m || !v || !grad || !w16 || !st) return GPTL_E_NULL;
-  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
-  if (!aligned16(master) || !aligned16(m) || !aligned16(v) || !aligned16(grad) || !aligned16(w16))
-    return GPTL_E_ALIGN;
-  if (n_params == 0 || n_params % 4 || !(lr >= 0.f) || !(beta1 >= 0.f && beta1 < 1.f) ||
-      !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f) || !(weight_decay >= 0.f))
-    return GPTL_E_ARG;
-  int sms = 0;
-  GPTL_TRY(device_check(&sms));
+  GPTL_TRY(adam_validate(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps,
+                         weight_decay, st));
   TagScope tag_scope(GPTL_TAG_O1_OVERFLOW);
   GPTL_TRY(gptl_check_overflow(n_params, grad, st, stream));
   g_tag = GPTL_TAG_O2_ADAM;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const long long n4 = (long long)(n_params / 4);
-  long long blocks = (n4 + 255) / 256;
-  if (blocks > 8 * sms) blocks = 8 * sms;
-  AdamArgs a{lr, beta1, beta2, eps, weight_decay};
-  if (dtype == GPTL_FP16)
-    adam_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(
-        reinterpret_cast<float4 *>(master), reinterpret_cast<float4 *>(m),
-        reinterpret_cast<float4 *>(v), reinterpret_cast<const float4 *>(grad),
-        static_cast<__half *>(w16), n4, a, st);
-  else
-    adam_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
-        reinterpret_cast<float4 *>(master), reinterpret_cast<float4 *>(m),
-        reinterpret_cast<float4 *>(v), reinterpret_cast<const float4 *>(grad),
-        static_cast<__nv_bfloat16 *>(w16), n4, a, st);
-  GPTL_CK(cudaGetLastError());
-  prof_launched(s, GPTL_KIND_ADAM);
-  return GPTL_OK;
+  return launch_adam(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps, weight_decay,
+                     st, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int loss_scale_update(gptl_scaler_state *st, int growth_interval, float growth_factor,
@@ -1431,7 +1548,8 @@ int gptl_gemm_plan(const gptl_gemm_desc *d, gptl_dtype dtype, int *bn, int *spli
   const GemmTiling tl = gemm_plan(*d, sms);
   *bn = tl.bn;
   *split = tl.split;
-  *mode = tl.m2 ? GPTL_GEMM_M256 : (tl.pipe_k ? GPTL_GEMM_K_HALVES : GPTL_GEMM_ALTERNATE);
+  *mode = tl.pair ? GPTL_GEMM_PAIR
+                  : (tl.m2 ? GPTL_GEMM_M256 : (tl.pipe_k ? GPTL_GEMM_K_HALVES : GPTL_GEMM_ALTERNATE));
   return GPTL_OK;
 }
 
@@ -1466,26 +1584,6 @@ int gptl_layernorm_bwd(int rows, int h, gptl_dtype dtype, const void *gy, const 
   return run_ln_bwd(LNB_PARTS, rows, h, dtype, gy, x, mu, rstd, g, resid, dx, nullptr, dg, db,
                     dx_sum, nullptr,
                     static_cast<float *>(scratch), reinterpret_cast<cudaStream_t>(stream));
-}
-
-int gptl_softmax_fwd(long long blocks, int s, gptl_dtype dtype, float scale, void *scores,
-                     gptl_stream_t stream) {
-  if (!scores) return GPTL_E_NULL;
-  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
-  if (!aligned16(scores)) return GPTL_E_ALIGN;
-  GPTL_TRY(device_check());
-  prof_start(reinterpret_cast<cudaStream_t>(stream));
-  return run_softmax_fwd(blocks, s, dtype, scale, scores, reinterpret_cast<cudaStream_t>(stream));
-}
-
-int gptl_softmax_bwd(long long blocks, int s, gptl_dtype dtype, float scale, const void *prob,
-                     void *dprob, gptl_stream_t stream) {
-  if (!prob || !dprob) return GPTL_E_NULL;
-  if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
-  if (!aligned16(prob) || !aligned16(dprob)) return GPTL_E_ALIGN;
-  GPTL_TRY(device_check());
-  prof_start(reinterpret_cast<cudaStream_t>(stream));
-  return run_softmax_bwd(blocks, s, dtype, scale, prob, dprob, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t gptl_colsum_scratch_bytes(int n, int groups) {

@@ -19,7 +19,6 @@ INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 
 FP16, BF16 = 0, 1
 ACT_NONE, ACT_GELU, ACT_DGELU = 0, 1, 2
-CAUSAL_NONE, CAUSAL_SKIP_UPPER, CAUSAL_K_BELOW, CAUSAL_K_FROM = 0, 1, 2, 3
 E_NULL, E_SHAPE, E_ALIGN, E_DTYPE, E_ARCH, E_CUDA, E_DEVICE, E_ARG = -1, -2, -3, -4, -5, -6, -7, -8
 E_TOO_LARGE = -9
 DTYPES = {"fp16": FP16, "bf16": BF16}
@@ -73,7 +72,7 @@ class LaunchRecord(C.Structure):
     _fields_ = [("kind", C.c_int), ("tag", C.c_int), ("ms", C.c_float)]
 
 
-KIND_NAMES = ("gemm", "ln_fwd", "ln_bwd", "softmax_fwd", "softmax_bwd", "colsum", "reduce",
+KIND_NAMES = ("gemm", "ln_fwd", "ln_bwd", "reserved3", "reserved4", "colsum", "reduce",
               "overflow", "adam", "scale", "splitk", "attn_fwd", "rowdot", "transpose", "attn_bwd",
               "clip", "accumulate")
 
@@ -90,6 +89,13 @@ _SIGS = {
                                 C.c_void_p, C.c_void_p, C.c_void_p]),
     "gpt_layer_bwd": (C.c_int, [C.POINTER(Shape), C.POINTER(Weights), C.c_void_p, C.c_void_p,
                                 C.c_void_p, C.c_void_p, C.POINTER(Grads), C.c_void_p, C.c_void_p]),
+    "gpt_layer_bwd_checked": (C.c_int, [C.POINTER(Shape), C.POINTER(Weights), C.c_void_p,
+                                        C.c_void_p, C.c_void_p, C.c_void_p, C.POINTER(Grads),
+                                        C.c_void_p, C.c_void_p, C.c_void_p]),
+    "adam_step_fp32_master_prechecked": (C.c_int, [C.c_size_t, C.c_void_p, C.c_void_p,
+                                                   C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                                   C.c_float, C.c_float, C.c_float, C.c_float,
+                                                   C.c_float, C.c_void_p, C.c_void_p]),
     "gpt_stack_workspace_bytes": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(C.c_size_t),
                                             C.POINTER(C.c_size_t)]),
     "gpt_stack_fwd": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(Weights), C.c_void_p,
@@ -116,10 +122,6 @@ _SIGS = {
                                      C.c_void_p]),
     "gptl_layernorm_bwd_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "gptl_layernorm_bwd": (C.c_int, [C.c_int, C.c_int, C.c_int] + [C.c_void_p] * 11 + [C.c_void_p]),
-    "gptl_softmax_fwd": (C.c_int, [C.c_longlong, C.c_int, C.c_int, C.c_float, C.c_void_p,
-                                   C.c_void_p]),
-    "gptl_softmax_bwd": (C.c_int, [C.c_longlong, C.c_int, C.c_int, C.c_float, C.c_void_p,
-                                   C.c_void_p, C.c_void_p]),
     "gptl_colsum_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "gptl_colsum": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_longlong, C.c_longlong, C.c_int,
                               C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
@@ -218,6 +220,14 @@ def layer_bwd(shape, weights: Weights, x, saved, dy, dx, grads: Grads, scratch, 
                                _ptr(dx), C.byref(grads), _ptr(scratch), stream), "gpt_layer_bwd")
 
 
+def layer_bwd_checked(shape, weights: Weights, x, saved, dy, dx, grads: Grads, scratch, state,
+                      stream=0):
+    """gpt_layer_bwd that also sets state.found_inf from the gradients it writes."""
+    _check(lib().gpt_layer_bwd_checked(C.byref(shape), C.byref(weights), _ptr(x), _ptr(saved),
+                                       _ptr(dy), _ptr(dx), C.byref(grads), _ptr(scratch),
+                                       _ptr(state), stream), "gpt_layer_bwd_checked")
+
+
 def stack_workspace_bytes(shape: Shape, n_layers: int):
     a, b = C.c_size_t(), C.c_size_t()
     _check(lib().gpt_stack_workspace_bytes(C.byref(shape), n_layers, C.byref(a), C.byref(b)),
@@ -247,6 +257,15 @@ def adam_step(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps, w
     _check(lib().adam_step_fp32_master(n_params, _ptr(master), _ptr(m), _ptr(v), _ptr(grad),
                                        _ptr(w16), DTYPES.get(dtype, dtype), lr, beta1, beta2, eps,
                                        weight_decay, _ptr(state), stream), "adam_step_fp32_master")
+
+
+def adam_step_prechecked(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps,
+                         weight_decay, state, stream=0):
+    """adam_step_fp32_master taking state.found_inf as gpt_layer_bwd_checked left it."""
+    _check(lib().adam_step_fp32_master_prechecked(n_params, _ptr(master), _ptr(m), _ptr(v),
+                                                  _ptr(grad), _ptr(w16), DTYPES.get(dtype, dtype),
+                                                  lr, beta1, beta2, eps, weight_decay, _ptr(state),
+                                                  stream), "adam_step_fp32_master_prechecked")
 
 
 # bytes of the clip workspace (GPTL_CLIP_WORKSPACE_BYTES in gptlayer.h); the
@@ -289,7 +308,7 @@ def gemm(desc: GemmDesc, dtype, stream=0):
     _check(lib().gptl_gemm(C.byref(desc), DTYPES.get(dtype, dtype), stream), "gptl_gemm")
 
 
-GEMM_ALTERNATE, GEMM_K_HALVES, GEMM_M256 = 0, 1, 2
+GEMM_ALTERNATE, GEMM_K_HALVES, GEMM_M256, GEMM_PAIR = 0, 1, 2, 3
 
 
 def gemm_plan(desc: GemmDesc, dtype) -> tuple:
@@ -313,16 +332,6 @@ def layernorm_bwd(rows, h, dtype, gy, x, mu, rstd, g, resid, dx, dg, db, dx_sum,
     _check(lib().gptl_layernorm_bwd(rows, h, DTYPES.get(dtype, dtype), _ptr(gy), _ptr(x), _ptr(mu),
                                     _ptr(rstd), _ptr(g), _ptr(resid), _ptr(dx), _ptr(dg), _ptr(db),
                                     _ptr(dx_sum), _ptr(scratch), stream), "gptl_layernorm_bwd")
-
-
-def softmax_fwd(blocks, s, dtype, scale, scores, stream=0):
-    _check(lib().gptl_softmax_fwd(blocks, s, DTYPES.get(dtype, dtype), scale, _ptr(scores), stream),
-           "gptl_softmax_fwd")
-
-
-def softmax_bwd(blocks, s, dtype, scale, prob, dprob, stream=0):
-    _check(lib().gptl_softmax_bwd(blocks, s, DTYPES.get(dtype, dtype), scale, _ptr(prob),
-                                  _ptr(dprob), stream), "gptl_softmax_bwd")
 
 
 def colsum_scratch_bytes(n, groups) -> int:

@@ -93,27 +93,41 @@ class LayerStep:
         G.layer_fwd(self.shape, self.weights, self.x if x is None else x,
                     self.y if y is None else y, self.saved, None, self.stream())
 
-    def bwd(self, x=None, dy=None):
-        G.layer_bwd(self.shape, self.weights, self.x if x is None else x, self.saved,
-                    self.dy if dy is None else dy, self.dx, self.grads, self.scratch, self.stream())
+    def bwd(self, x=None, dy=None, checked=False):
+        """gpt_layer_bwd, or with checked=True gpt_layer_bwd_checked (the
+        overflow flag set from the gradients as they are written)."""
+        x = self.x if x is None else x
+        dy = self.dy if dy is None else dy
+        if checked:
+            G.layer_bwd_checked(self.shape, self.weights, x, self.saved, dy, self.dx, self.grads,
+                                self.scratch, self.state, self.stream())
+        else:
+            G.layer_bwd(self.shape, self.weights, x, self.saved, dy, self.dx, self.grads,
+                        self.scratch, self.stream())
 
-    def adam(self):
+    def adam(self, prechecked=False):
+        """adam_step_fp32_master (overflow scan + update), or with
+        prechecked=True the update alone, on the flag a checked backward set."""
         hp = self.hyper
-        G.adam_step(self.n_params, self.master, self.m, self.v, self.grad, self.w16, self.cfg.dtype,
-                    hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], self.state,
-                    self.stream())
+        fn = G.adam_step_prechecked if prechecked else G.adam_step
+        fn(self.n_params, self.master, self.m, self.v, self.grad, self.w16, self.cfg.dtype,
+           hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], self.state,
+           self.stream())
 
     def scale_update(self):
         hp = self.hyper
         G.scale_update(self.state, hp["growth_interval"], hp["growth_factor"],
                        hp["backoff_factor"], hp["min_scale"], self.stream())
 
-    def step(self, x=None, dy=None, y=None):
+    def step(self, x=None, dy=None, y=None, fused_check=False):
         """fwd + bwd + Adam + scale update; x, dy and y default to this object's
-        buffers (other device buffers of the same shape may be passed)."""
+        buffers (other device buffers of the same shape may be passed).  With
+        fused_check the overflow check is folded into the backward
+        (gpt_layer_bwd_checked + adam_step_fp32_master_prechecked): the same
+        decisions and results, without the pass that re-reads the gradients."""
         self.fwd(x, y)
-        self.bwd(x, dy)
-        self.adam()
+        self.bwd(x, dy, checked=fused_check)
+        self.adam(prechecked=fused_check)
         self.scale_update()
 
     # ------------------------------------------------------------ readback
@@ -192,7 +206,9 @@ class LayerStack(LayerStep):
         G.stack_fwd(self.shape, self.layer_weights, self.x if x is None else x, self.acts,
                     self.saved, self.stream())
 
-    def bwd(self, x=None, dy=None):
+    def bwd(self, x=None, dy=None, checked=False):
+        if checked:
+            raise ValueError("the stack's backward has no checked variant: scan the arena in Adam")
         G.stack_bwd(self.shape, self.layer_weights, self.x if x is None else x, self.acts,
                     self.saved, self.dy if dy is None else dy, self.dx, self.layer_grads,
                     self.scratch, self.stream())
