@@ -90,15 +90,10 @@ int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream);
  *   GPTL_GEMM_ALTERNATE  128 x bn tiles alternate between the pipelines;
  *   GPTL_GEMM_K_HALVES   both pipelines on each 128 x bn tile, one half of its
  *                        K range each, summed in a fixed order;
- *   GPTL_GEMM_M256       256 x bn tiles, one 128-row half per pipeline;
- *   GPTL_GEMM_PAIR       256 x bn tiles on a cluster of two CTAs (two SMs):
- *                        one MMA stream for both (tcgen05 cta_group::2), each
- *                        SM staging its 128 rows of A and half of B, and two
- *                        accumulators per SM so that a tile's epilogue
- *                        overlaps the next tile's MMAs.
+ *   GPTL_GEMM_M256       256 x bn tiles, one 128-row half per pipeline.
  * Results do not depend on the choice beyond fp32 summation order, and are
  * deterministic for a given choice. */
-enum { GPTL_GEMM_ALTERNATE = 0, GPTL_GEMM_K_HALVES = 1, GPTL_GEMM_M256 = 2, GPTL_GEMM_PAIR = 3 };
+enum { GPTL_GEMM_ALTERNATE = 0, GPTL_GEMM_K_HALVES = 1, GPTL_GEMM_M256 = 2 };
 int gptl_gemm_plan(const gptl_gemm_desc *d, gptl_dtype dtype, int *bn, int *split, int *mode);
 
 /* Fused causal attention forward ("Training GPT-2 with Megatron-LM" §6.2

@@ -66,6 +66,7 @@ struct alignas(64) GemmParams {
   int bn, bn_alloc, stages, tmem_cols;
   uint32_t idesc;
   int m_tiles, n_tiles;
+  int band;                    // tile order: bands of `band` N tiles, M tiles fastest in a band
   long long total_tiles;
   // epilogue
   int o_mod;                   // output group G at map coordinates (G % o_mod, G / o_mod), or
@@ -97,7 +98,12 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams &p, long long idx
   const long long tpg = (long long)p.m_tiles * p.n_tiles;
   t.g = (int)(tile / tpg);
   const int rem = (int)(tile - (long long)t.g * tpg);
-  const int mt = rem / p.n_tiles, nt = rem - (rem / p.n_tiles) * p.n_tiles;
+  // the tiles of a band of N columns in M order: the CTAs working at the same
+  // time read the same k-slabs of B (the weights, in most products) from L2,
+  // instead of each streaming a B tile that the other M rows need later
+  const int span = p.m_tiles * p.band;
+  const int bnd = rem / span, r2 = rem - bnd * span;
+  const int mt = r2 % p.m_tiles, nt = bnd * p.band + r2 / p.m_tiles;
   t.m0 = mt * (p.m2 ? 2 * kBM : kBM);
   t.n0 = nt * p.bn;
   t.kb_begin = 0;

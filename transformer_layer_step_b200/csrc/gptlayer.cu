@@ -11,7 +11,6 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include <algorithm>
 #include <mutex>
 
 #include "bw_kernels.cuh"
@@ -19,7 +18,6 @@
 #include "attn_bwd_tc.cuh"
 #include "attn_tc.cuh"
 #include "gemm_tc.cuh"
-#include "gemm_pair.cuh"
 #include "gptlayer_parts.h"
 #include "gptlayer_profile.h"
 
@@ -280,10 +278,10 @@ int pick_bn(const gptl_gemm_desc &d, int sms) {
 // alternating tiles on the GeLU GEMMs, wins on the others).  Split-K adds the
 // partial-sum pass, (2 split + 1) fp32 arrays at ~4 TB/s plus a launch.
 struct GemmTiling {
-  int bn, split, pipe_k, m2, pair;
+  int bn, split, pipe_k, m2;
 };
 GemmTiling choose_tiling(const gptl_gemm_desc &d, int sms, bool can_split) {
-  GemmTiling best{pick_bn(d, sms), 1, 0, 0, 0};
+  GemmTiling best{pick_bn(d, sms), 1, 0, 0};
   const long long kb_all = (long long)((d.K + kBK - 1) / kBK) * d.k_shards;
   const double out_bytes = (double)d.groups * d.M * d.N * 4.0;
   const double e_half = (d.act == GPTL_ACT_NONE ? 1.3 : 5.0);
@@ -294,15 +292,14 @@ GemmTiling choose_tiling(const gptl_gemm_desc &d, int sms, bool can_split) {
     if (d.N <= 256 && bn_c != 256) break;         // N fits one tile column: BN = N
     const double e_tile = e_half * bn / 256.0;
     const long long n_tiles = (d.N + bn - 1) / bn;
-    for (int mode = 0; mode < 4; ++mode) {          // alternate, K halves, m2, CTA pairs
-      if (mode >= 2 && d.M <= kBM) continue;
-      if (mode == 3 && (bn % 32 || sms < 2)) continue;   // each CTA of a pair takes BN/2 rows of B
-      const int rows = mode >= 2 ? 2 * kBM : kBM;
+    for (int mode = 0; mode < 3; ++mode) {          // alternate, K halves, m2
+      if (mode == 2 && d.M <= kBM) continue;
+      const int rows = mode == 2 ? 2 * kBM : kBM;
       const long long m_tiles = (d.M + rows - 1) / rows;
       const long long tiles = m_tiles * n_tiles * d.groups;
       // per-k-block time of this BN: half scales with BN, half with A rows + BN
       const double width = 0.5 * bn / 256.0 + 0.5 * (double)(rows + bn) / (double)(rows + 256);
-      for (int sp = 1; sp <= (can_split && mode != 3 ? 8 : 1); ++sp) {
+      for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
         if (sp > (d.K + kBK - 1) / kBK) break;
         if (sp > 1 && (double)sp * out_bytes > (double)d.ws_bytes) break;
         // K halves: every slice must give each pipeline at least one k-block
@@ -310,22 +307,18 @@ GemmTiling choose_tiling(const gptl_gemm_desc &d, int sms, bool can_split) {
         const long long items = tiles * sp;
         const long long kb = (kb_all + sp - 1) / sp;
         const long long per_cta = (items + sms - 1) / sms;
-        const long long per_pair = (items + sms / 2 - 1) / (sms / 2);
         double t;
         if (mode == 0)
           t = per_cta >= 2 ? (double)((per_cta + 1) / 2) * kb * 1.17 * width + e_tile
                            : kb * 0.9 * width + e_tile;
         else if (mode == 1)
           t = (double)per_cta * ((kb + 1) / 2 * 1.13 * width + e_tile);
-        else if (mode == 2)
+        else
           t = (double)per_cta * (kb * 0.8 * width + 2.0 * e_tile);
-        else    // a pair's tile: each SM half the MMA work of m2's per k-block; the
-                // epilogue overlaps the next tile's MMAs, except where it is longer
-          t = (double)per_pair * std::max(kb * 0.42 * width, 2.0 * e_tile) + 2.0 * e_tile;
         if (sp > 1) t += (2.0 * sp + 1.0) * out_bytes / 4.0e6 + 3.0;
         if (best_t < 0 || t < best_t * 0.999) {
           best_t = t;
-          best = GemmTiling{bn, sp, mode == 1 ? 1 : 0, mode >= 2 ? 1 : 0, mode == 3 ? 1 : 0};
+          best = GemmTiling{bn, sp, mode == 1 ? 1 : 0, mode == 2 ? 1 : 0};
         }
       }
     }
@@ -344,22 +337,6 @@ int launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) 
     attr_set[dev] = true;
   }
   gemm_tc_kernel<T><<<grid, kGemmThreads, smem, stream>>>(p);
-  GPTL_CK(cudaGetLastError());
-  prof_launched(stream, GPTL_KIND_GEMM);
-  return GPTL_OK;
-}
-
-template <typename T>
-int launch_gemm_pair_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) {
-  static bool attr_set[kMaxDevices] = {};
-  int dev = 0;
-  GPTL_CK(cudaGetDevice(&dev));
-  if (!attr_set[dev]) {
-    GPTL_CK(cudaFuncSetAttribute(gemm_pair_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemLimit));
-    attr_set[dev] = true;
-  }
-  gemm_pair_kernel<T><<<grid, kPairThreads, smem, stream>>>(p);   // clusters of 2 (static)
   GPTL_CK(cudaGetLastError());
   prof_launched(stream, GPTL_KIND_GEMM);
   return GPTL_OK;
@@ -400,13 +377,11 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   memset(&p, 0, sizeof(p));
   const GemmTiling tl = gemm_plan(d, sms);
   const int bn = tl.bn;
-  // rows of A and B staged per SM: a pair's CTA takes 128 rows of A and BN/2 of B
-  const int a_rows = tl.m2 && !tl.pair ? 2 * kBM : kBM;
-  const int b_rows = tl.pair ? bn / 2 : bn;
   const int wa = d.a.mn_major ? mn_chunk_width(kBM) : 64;
-  const int wb = d.b.mn_major ? mn_chunk_width(b_rows) : 64;
+  const int wb = d.b.mn_major ? mn_chunk_width(bn) : 64;
+  const int a_rows = tl.m2 ? 2 * kBM : kBM;   // rows of A per tile
   GPTL_TRY(encode_operand(&p.map_a, d.a, dt, a_rows, wa));
-  GPTL_TRY(encode_operand(&p.map_b, d.b, dt, b_rows, wb));
+  GPTL_TRY(encode_operand(&p.map_b, d.b, dt, bn, wb));
   auto rule = [](const gptl_operand &o, int w) {
     OperandRule r;
     r.mn_major = o.mn_major;
@@ -430,22 +405,18 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   while (bn_alloc < bn) bn_alloc *= 2;
   p.bn_alloc = bn_alloc;
   p.tmem_cols = 2 * bn_alloc;
-  const int stage_bytes = (a_rows + b_rows) * kBK * 2;
+  const int stage_bytes = (a_rows + bn) * kBK * 2;
   // stages per ring: two rings (one per pipeline), or one shared ring in m2
-  // and in a pair's CTA
   const int rings = tl.m2 ? 1 : 2;
   p.stages = (kSmemLimit - 2048 - kStagingBytes) / (rings * stage_bytes);
-  const int max_stages = tl.pair ? kPairMaxStages : 4;
-  if (p.stages > max_stages) p.stages = max_stages;
+  if (p.stages > 4) p.stages = 4;
   if (p.stages < 2) return GPTL_E_SHAPE;
   const int smem = 1024 + rings * p.stages * stage_bytes + kStagingBytes + 512;
   const uint32_t fmt = dt == GPTL_BF16 ? 1u : 0u;
-  const int mma_m = tl.pair ? 2 * kBM : kBM;    // a pair's MMA spans both CTAs' rows
   p.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)d.a.mn_major << 15) |
             ((uint32_t)d.b.mn_major << 16) | ((uint32_t)(bn >> 3) << 17) |
-            ((uint32_t)(mma_m >> 4) << 24);
-  const int tile_rows = tl.m2 ? 2 * kBM : kBM;
-  p.m_tiles = (d.M + tile_rows - 1) / tile_rows;
+            ((uint32_t)(kBM >> 4) << 24);
+  p.m_tiles = (d.M + a_rows - 1) / a_rows;
   p.n_tiles = (d.N + bn - 1) / bn;
   const long long tiles = (long long)p.m_tiles * p.n_tiles * d.groups;
   p.split = tl.split;
@@ -454,6 +425,12 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.ws = static_cast<float *>(d.ws);
   p.ws_slice = (long long)d.groups * d.M * d.N;
   p.total_tiles = tiles * p.split;
+  {  // a band of N tiles per wave: every M tile of the band runs at once
+    long long band = sms / p.m_tiles;
+    if (band < 1) band = 1;
+    if (band > p.n_tiles) band = p.n_tiles;
+    p.band = (int)band;
+  }
   if (p.split > 1) {            // partials [split * groups][M][N], dense fp32
     int flat = 1;
     GPTL_TRY(encode_output(&p.map_o, d.ws, 1, dt, d.N, d.M, d.N, p.split * d.groups, 1, 0,
@@ -481,12 +458,6 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.aux = d.aux;
   p.act = d.act;
   p.nonfinite = d.out_f32 ? g_nonfinite : nullptr;
-  if (tl.pair) {
-    const long long pairs = p.total_tiles < sms / 2 ? p.total_tiles : sms / 2;
-    if (dt == GPTL_FP16) GPTL_TRY(launch_gemm_pair_t<__half>(p, (int)(2 * pairs), smem, stream));
-    else GPTL_TRY(launch_gemm_pair_t<__nv_bfloat16>(p, (int)(2 * pairs), smem, stream));
-    return GPTL_OK;
-  }
   const int grid = (int)(p.total_tiles < sms ? p.total_tiles : sms);
   if (dt == GPTL_FP16) GPTL_TRY(launch_gemm_t<__half>(p, grid, smem, stream));
   else GPTL_TRY(launch_gemm_t<__nv_bfloat16>(p, grid, smem, stream));
@@ -1548,8 +1519,7 @@ int gptl_gemm_plan(const gptl_gemm_desc *d, gptl_dtype dtype, int *bn, int *spli
   const GemmTiling tl = gemm_plan(*d, sms);
   *bn = tl.bn;
   *split = tl.split;
-  *mode = tl.pair ? GPTL_GEMM_PAIR
-                  : (tl.m2 ? GPTL_GEMM_M256 : (tl.pipe_k ? GPTL_GEMM_K_HALVES : GPTL_GEMM_ALTERNATE));
+  *mode = tl.m2 ? GPTL_GEMM_M256 : (tl.pipe_k ? GPTL_GEMM_K_HALVES : GPTL_GEMM_ALTERNATE);
   return GPTL_OK;
 }
 

@@ -308,7 +308,7 @@ def gemm(desc: GemmDesc, dtype, stream=0):
     _check(lib().gptl_gemm(C.byref(desc), DTYPES.get(dtype, dtype), stream), "gptl_gemm")
 
 
-GEMM_ALTERNATE, GEMM_K_HALVES, GEMM_M256, GEMM_PAIR = 0, 1, 2, 3
+GEMM_ALTERNATE, GEMM_K_HALVES, GEMM_M256 = 0, 1, 2
 
 
 def gemm_plan(desc: GemmDesc, dtype) -> tuple:
