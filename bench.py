@@ -99,7 +99,10 @@ def kernel_bytes(cfg, n_params: int, layers: int = 1) -> dict:
         "B0 weights^T": 4 * (4 * h * h + 2 * h * f),          # the four weight matrices
         "B2 dOut^T": 4 * T * h, "B5 L2^T": 4 * T * h,         # transposes: read + write
         "B7 dH^T": 4 * T * h, "B11 L1^T": 4 * T * h,
-        "B3 db1": 2 * T * f, "B11 dbqkv": 2 * T * 3 * h,
+        # bias gradients: the GEMM / attention kernels that write dZ and dC
+        # sum every 32 rows; this pass reads those partials and writes the sum
+        "B3 db1": 4 * f * ((T + 31) // 32 + 1),
+        "B11 dbqkv": 4 * 3 * h * (b * ((s + 31) // 32) + 1),
     }
     out = {k: v * layers for k, v in per_layer.items()}
     out.update({"O1 overflow": 4 * n_params, "O2 adam": 30 * n_params})
@@ -354,9 +357,10 @@ def run_ours(args, cfg, rank, world, local_rank):
     if stack:
         # L layers of the shape, each starting from the same seeded weights,
         # with parameters of their own in one arena, and one Adam over all
-        ls = LayerStack(cfg, [inp["params"]] * args.layers, inp["x"], device=dev)
+        ls = LayerStack(cfg, [inp["params"]] * args.layers, inp["x"], device=dev,
+                        recompute_gelu=args.recompute_gelu)
     else:
-        ls = LayerStep(cfg, inp, device=dev)
+        ls = LayerStep(cfg, inp, device=dev, recompute_gelu=args.recompute_gelu)
     dy_bits = synth.loss_grad_bits(cfg, ls.hyper["init_scale"], inp["r"])
     ls.set_dy_bits(dy_bits)
     stream = torch.cuda.current_stream(dev)
@@ -655,11 +659,14 @@ def run_case(args, cfg):
         o, do = torch.empty(t, T, hs, dtype=tdt, device="cuda"), rnd(t, T, hs)
         lse = torch.empty(t * cfg.batch * as_, cfg.seq, device="cuda")
         dvec, dc = torch.empty_like(lse), torch.empty_like(c)
+        # the QKV bias gradient, summed by the kernels that write dC
+        dpart = torch.empty(cfg.batch * ((cfg.seq + 31) // 32) * 3 * h, device="cuda")
+        db = torch.empty(3 * h, device="cuda")
 
         def work():
             G.attention_fwd(cfg.batch, cfg.seq, h, cfg.heads, t, cfg.dtype, c, o, lse, st)
             G.attention_bwd(cfg.batch, cfg.seq, h, cfg.heads, t, cfg.dtype, c, o, do, lse, dvec,
-                            dc, st)
+                            dc, dpart, db, stream=st)
         flops = 3 * 2 * 2 * cfg.batch * h * (cfg.seq * (cfg.seq + 1) // 2)
     elif args.case == "layernorm":
         x, gy, res = rnd(T, h), rnd(T, h), rnd(T, h)
@@ -719,6 +726,9 @@ def main():
     ap.add_argument("--layers", type=int, default=1,
                     help="a stack of this many layers of the workload's shape per step "
                          "(gpt_stack_fwd / gpt_stack_bwd and one Adam over every layer)")
+    ap.add_argument("--recompute-gelu", action="store_true",
+                    help="selective recompute: the FFN activation is written again in the "
+                         "backward (by the FFN2 input-gradient GEMM) instead of saved")
     ap.add_argument("--case", choices=CASES,
                     help="run one kernel family once at this workload's shapes (a small "
                          "device footprint for a profiler capture) instead of the benchmark")
@@ -738,6 +748,8 @@ def main():
               "e2e_step_launch": "kernel by kernel" if args.e2e_eager else "one CUDA graph per step",
               "e2e_copies": "one stream per direction, overlapped with the neighbouring steps",
               "l2": "flushed between steps (256 MiB write, outside the per-step events)"}
+    if args.recompute_gelu:
+        config["recompute_gelu"] = True
     L = args.layers
     if L < 1:
         ap.error("--layers must be at least 1")

@@ -63,11 +63,19 @@ typedef enum { GPTL_FP16 = 0, GPTL_BF16 = 1 } gptl_dtype;
  * > 0; heads | hidden; tp | heads; tp | ffn; head_dim = hidden/heads is a
  * multiple of 16 and at most 256; hidden % 64 == 0; (ffn/tp) % 64 == 0;
  * seq % 16 == 0; batch*seq < 2^31.  ln_eps > 0 (the pages do not state it;
- * 1e-5 is the usual GPT-2 value). */
+ * 1e-5 is the usual GPT-2 value).
+ * recompute_gelu (0 or 1): selective recompute of the FFN activation
+ * ("Training GPT-2 with Megatron-LM", troubleshooting: activation
+ * recomputation; "Megatron-LM overview" §3.3).  With 1, A = GeLU(Z) is not
+ * kept in the saved workspace (batch*seq*ffn*2 bytes less): the forward writes
+ * it into scratch for FFN2, and the backward writes it again from the saved Z
+ * in the epilogue of the FFN2 input-gradient GEMM, which reads Z anyway.
+ * The results are bit-identical to recompute_gelu = 0. */
 typedef struct {
   int batch, seq, hidden, heads, ffn, tp;
   gptl_dtype dtype;
   float ln_eps;
+  int recompute_gelu;
 } gptl_shape;
 
 /* Layer parameters in the compute dtype (fp16 or bf16), read-only here.
@@ -115,8 +123,9 @@ typedef struct {
 /* Bytes of device workspace the caller provides.
  *  saved   : activations written by gpt_layer_fwd and read by gpt_layer_bwd;
  *            must stay untouched between the two calls.
- *  scratch : temporaries of gpt_layer_bwd (gpt_layer_fwd uses none); may be
- *            reused freely between calls on the same stream.
+ *  scratch : temporaries of gpt_layer_bwd (and, with recompute_gelu, of
+ *            gpt_layer_fwd); may be reused freely between calls on the same
+ *            stream.
  * Returns GPTL_E_NULL / GPTL_E_SHAPE / GPTL_E_DTYPE on bad arguments. */
 int gpt_layer_workspace_bytes(const gptl_shape *shape, size_t *saved_bytes,
                               size_t *scratch_bytes);
@@ -130,7 +139,8 @@ int gpt_layer_workspace_bytes(const gptl_shape *shape, size_t *saved_bytes,
 int gpt_layer_param_layout(const gptl_shape *shape, size_t offsets[12], size_t *n_params);
 
 /* Forward pass.  x: [T,h] input; y: [T,h] output (cdt).  saved: workspace of
- * saved_bytes; scratch: may be NULL.  x, y and saved must not overlap. */
+ * saved_bytes; scratch: scratch_bytes of workspace with recompute_gelu (else
+ * unused, may be NULL).  x, y, saved and scratch must not overlap. */
 int gpt_layer_fwd(const gptl_shape *shape, const gptl_weights *w, const void *x, void *y,
                   void *saved, void *scratch, gptl_stream_t stream);
 
@@ -207,10 +217,11 @@ int gpt_stack_workspace_bytes(const gptl_shape *shape, int n_layers, size_t *sav
  * layer l-1's output.  acts: n_layers [T,h] outputs (cdt) back to back,
  * layer l's at acts + l*T*h elements; the stack's output is the last one.
  * w: n_layers gptl_weights; saved: gpt_stack_workspace_bytes' saved bytes,
- * untouched until gpt_stack_bwd.  x, acts and saved must not overlap.
- * All arguments are checked before the first launch. */
+ * untouched until gpt_stack_bwd; scratch: its scratch bytes when the shape
+ * has recompute_gelu (else may be NULL).  x, acts, saved and scratch must not
+ * overlap.  All arguments are checked before the first launch. */
 int gpt_stack_fwd(const gptl_shape *shape, int n_layers, const gptl_weights *w, const void *x,
-                  void *acts, void *saved, gptl_stream_t stream);
+                  void *acts, void *saved, void *scratch, gptl_stream_t stream);
 
 /* Backward through layers n_layers-1..0: the last layer reads dy (gradient
  * of the scaled loss w.r.t. the stack's output), layer l < n_layers-1 reads

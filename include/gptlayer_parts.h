@@ -37,7 +37,7 @@ typedef struct {
 enum {
   GPTL_ACT_NONE = 0,
   GPTL_ACT_GELU = 1,     /* out = value, out2 = GeLU(value)                   */
-  GPTL_ACT_DGELU = 2     /* out = value * GeLU'(aux)                          */
+  GPTL_ACT_DGELU = 2     /* out = value * GeLU'(aux); out2 (optional) = GeLU(aux) */
 };
 
 /* out[G](m, n) = epilogue( sum over ks < k_shards, k < K of A(m,k) * B(n,k) )
@@ -47,7 +47,10 @@ enum {
  * Epilogue, in order: + bias[G*bias_g_stride + n] (if bias, 16-bit),
  * + resid[m*ld_resid + n] (if resid; fp32 when resid_f32, else 16-bit), then
  * act: GELU writes the value to out and GeLU(value) to out2; DGELU multiplies
- * by GeLU'(aux at the output's index).  out_f32 = 1 stores the fp32 value
+ * by GeLU'(aux at the output's index) and, if out2 is not NULL, also writes
+ * GeLU(aux) to out2 (the activation recomputed from its stored argument; with
+ * the GELU epilogue's rounding, bit-identical to what GELU wrote for the same
+ * 16-bit argument).  out_f32 = 1 stores the fp32 value
  * (act must be GPTL_ACT_NONE); otherwise out is 16-bit, rounded to nearest
  * even.  resid and DGELU do not combine.  Requirements: K % 16 == 0,
  * N % 16 == 0, all offsets/pitches multiples of 8 elements, out (and out2,
@@ -61,7 +64,15 @@ enum {
  * writes fp32 partial sums to ws and a second kernel adds them in slice
  * order (the result is deterministic).  It does so only when the output has
  * too few tiles to fill the GPU and the partials fit in ws_bytes.  ws may be
- * NULL (no split). */
+ * NULL (no split).
+ * Column sums: when colsum is not NULL (16-byte aligned fp32 device memory of
+ * ceil(M/32) * groups * N floats), the epilogue also writes, for every group
+ * G, column n and r < ceil(M/32),
+ *   colsum[(r*groups + G)*N + n] = sum over m in [32r, min(32r+32, M)) of
+ *                                  out[G](m, n) as stored (16-bit),
+ * each added in a fixed order; the caller adds the ceil(M/32) partial rows
+ * (a bias gradient).  It needs a 16-bit output (out_f32 = 0) and act other
+ * than GELU, and it rules out split-K. */
 typedef struct {
   int M, N, K, groups, k_shards, causal;
   gptl_operand a, b;
@@ -80,6 +91,7 @@ typedef struct {
   int resid_f32;
   void *ws;
   long long ws_bytes;
+  float *colsum;
 } gptl_gemm_desc;
 
 int gptl_gemm(const gptl_gemm_desc *d, gptl_dtype dtype, gptl_stream_t stream);
@@ -113,10 +125,17 @@ int gptl_attention_fwd(int batch, int seq, int hidden, int heads, int tp, gptl_d
  * columns of dqkv (same layout as qkv); dvec ([g][seq] fp32, caller scratch)
  * receives D = dO . O per row.  With P = softmax(Q K^T / sqrt(d)) (causal):
  *   dV = P^T dO,  dS = P (dO V^T - D) / sqrt(d),  dQ = dS K,  dK = dS^T Q,
- * P taken in the 16-bit type.  Same size limits as gptl_attention_fwd. */
+ * P taken in the 16-bit type.  Same size limits as gptl_attention_fwd.
+ * dbias (optional, with dbias_part): the QKV bias gradient, [tp][3h/tp] fp32,
+ * the column sums of each shard's dqkv over its batch*seq rows, of the values
+ * as stored; the kernels that write dQ, dK and dV sum every 32 rows into
+ * dbias_part (caller scratch of batch * ceil(seq/32) * 3 * hidden floats) and
+ * a second pass adds those in a fixed order.  Both NULL: no bias gradient;
+ * only one NULL: GPTL_E_NULL. */
 int gptl_attention_bwd(int batch, int seq, int hidden, int heads, int tp, gptl_dtype dtype,
                        const void *qkv, const void *o, const void *dout, const float *lse,
-                       float *dvec, void *dqkv, gptl_stream_t stream);
+                       float *dvec, void *dqkv, float *dbias_part, float *dbias,
+                       gptl_stream_t stream);
 
 /* LayerNorm forward over `rows` rows of width h: y = g*(x-mu)*rstd + b with the
  * biased variance; mu and rstd ([rows] fp32) are saved for the backward.

@@ -78,6 +78,17 @@ def test_dtype_and_null_rejected_without_launch():
     assert rc == G.E_ALIGN
     rc = G.lib().loss_scale_update(16, 0, 2.0, 0.5, 1.0, None)
     assert rc == G.E_ARG
+    # recompute_gelu: the forward writes A into scratch, so it needs scratch
+    shr = G.make_shape(2, 64, 128, 4, 512, 2, "fp16", recompute_gelu=1)
+    rc = G.lib().gpt_layer_fwd(ctypes.byref(shr), ctypes.byref(w), 16, 16, 16, None, None)
+    assert rc == G.E_NULL
+    # the attention backward's bias gradient needs both its partials and its output
+    rc = G.lib().gptl_attention_bwd(1, 64, 128, 4, 1, 0, 16, 16, 16, 16, 16, 16, None, 16, None)
+    assert rc == G.E_NULL
+    rc = G.lib().gptl_attention_bwd(1, 64, 128, 4, 1, 0, 16, 16, 16, 16, 16, 16, 16, None, None)
+    assert rc == G.E_NULL
+    rc = G.lib().gptl_attention_bwd(1, 64, 128, 4, 1, 0, 16, 16, 16, 16, 16, 16, 20, 16, None)
+    assert rc == G.E_ALIGN
 
 
 def test_clip_and_accumulate_arguments_rejected_without_launch():
@@ -122,11 +133,11 @@ def test_stack_workspace_and_arguments_rejected_without_launch():
     lib = G.lib()
     ws = (G.Weights * 2)(w, w)
     gs = (G.Grads * 2)(g, g)
-    assert lib.gpt_stack_fwd(ctypes.byref(sh), 0, ws, 16, 32, 48, None) == G.E_ARG
-    assert lib.gpt_stack_fwd(ctypes.byref(sh), 2, ws, None, 32, 48, None) == G.E_NULL
-    assert lib.gpt_stack_fwd(ctypes.byref(sh), 2, ws, 16, 40, 48, None) == G.E_ALIGN
+    assert lib.gpt_stack_fwd(ctypes.byref(sh), 0, ws, 16, 32, 48, None, None) == G.E_ARG
+    assert lib.gpt_stack_fwd(ctypes.byref(sh), 2, ws, None, 32, 48, None, None) == G.E_NULL
+    assert lib.gpt_stack_fwd(ctypes.byref(sh), 2, ws, 16, 40, 48, None, None) == G.E_ALIGN
     bad = (G.Weights * 2)(w, G.make_weights({n: (8 if n == "w_o" else 4096) for n in G.PARAM_NAMES}))
-    assert lib.gpt_stack_fwd(ctypes.byref(sh), 2, bad, 16, 32, 48, None) == G.E_ALIGN
+    assert lib.gpt_stack_fwd(ctypes.byref(sh), 2, bad, 16, 32, 48, None, None) == G.E_ALIGN
     gbad = (G.Grads * 2)(g, G.make_grads({n: (None if n == "b_2" else 4096) for n in G.PARAM_NAMES}))
     assert lib.gpt_stack_bwd(ctypes.byref(sh), 2, ws, 16, 32, 48, 64, 80, gbad, 96, None) == G.E_NULL
     assert lib.gpt_stack_bwd(ctypes.byref(sh), 2, ws, 16, 32, 48, 64, 80, gs, None, None) == G.E_NULL
@@ -157,3 +168,19 @@ def test_layernorm_backward_limit_is_checked_up_front():
     before = G.launch_count()
     assert G.lib().gpt_layer_fwd(ctypes.byref(sh), ctypes.byref(w), 16, 32, 48, None, None) == G.E_SHAPE
     assert G.launch_count() == before
+
+
+@pytest.mark.parametrize("name", ["tiny", "gpt2-117m", "large-h10240"])
+def test_gelu_recompute_moves_the_activation_to_scratch(name):
+    """recompute_gelu keeps A = GeLU(Z) (batch*seq*ffn 16-bit values) out of
+    the saved workspace and in scratch; other values of the flag are rejected."""
+    c = synth.CONFIGS[name]
+    args = (c.batch, c.seq, c.hidden, c.heads, c.ffn, c.tp, c.dtype)
+    saved0, scratch0 = G.workspace_bytes(G.make_shape(*args))
+    saved1, scratch1 = G.workspace_bytes(G.make_shape(*args, recompute_gelu=1))
+    a = c.batch * c.seq * c.ffn * 2
+    a256 = (a + 255) // 256 * 256
+    assert saved0 - saved1 == a256 and scratch1 - scratch0 == a256
+    with pytest.raises(G.GptlError) as e:
+        G.workspace_bytes(G.make_shape(*args, recompute_gelu=2))
+    assert e.value.code == G.E_SHAPE

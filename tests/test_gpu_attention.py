@@ -115,9 +115,19 @@ def test_attention_bwd(b, s, h, a, t, dtype):
     G.attention_fwd(b, s, h, a, t, dtype, qkv_t, o, lse, stream())
     dvec = torch.zeros_like(lse)
     dqkv = torch.full((t, b * s, 3 * hs), float("nan"), dtype=tdt, device="cuda")
-    G.attention_bwd(b, s, h, a, t, dtype, qkv_t, o, dout_t, lse, dvec, dqkv, stream())
+    dpart = torch.full((b * ((s + 31) // 32) * 3 * h,), float("nan"), device="cuda")
+    dbias = torch.full((t, 3 * hs), float("nan"), device="cuda")
+    G.attention_bwd(b, s, h, a, t, dtype, qkv_t, o, dout_t, lse, dvec, dqkv, dpart, dbias,
+                    stream=stream())
     check_device_error()
     got = host_values(dqkv, dtype)
+    # the bias gradient that the kernels sum as they store dQ, dK, dV: the
+    # column sums of the stored values, per shard (fp32 sums of 32 rows, then
+    # of the partial rows)
+    want = got.astype(np.float64).sum(axis=1)
+    db = dbias.cpu().numpy().astype(np.float64)
+    bound = 4e-6 * np.abs(got).astype(np.float64).sum(axis=1) + 1e-30
+    assert np.all(np.abs(db - want) <= bound), float(np.max(np.abs(db - want) / bound))
     o_used = host_values(o, dtype)
     u = 2.0 ** -8 if dtype == "bf16" else 2.0 ** -11
     for i in range(t):

@@ -67,8 +67,10 @@ def _op(buf_t, x_ext, rows_ext, g_ext, row_pitch, g_pitch, mn, x_mod=1, x_mul=0,
 
 def _run(dtype, M, N, K, groups, k_shards, causal, a_spec, b_spec, out_f32=False, bias=False,
          resid=False, act=G.ACT_NONE, seed=0, std_a=1.0, std_b=0.1, ws_bytes=0, resid_f32=False,
-         launches=None):
-    """a_spec/b_spec: (shape of the 3-D buffer [g, rows, x], view kwargs)."""
+         launches=None, colsum=False, dgelu_out2=False, extras=None):
+    """a_spec/b_spec: (shape of the 3-D buffer [g, rows, x], view kwargs).  With
+    colsum / dgelu_out2, extras receives the column-sum partials [ceil(M/32)][g][N]
+    and the second (GeLU) output of a DGELU epilogue."""
     need_gpu()
     rng = np.random.default_rng(seed)
     abuf = rounded(rng.standard_normal(a_spec[0]) * std_a, dtype)
@@ -111,9 +113,13 @@ def _run(dtype, M, N, K, groups, k_shards, causal, a_spec, b_spec, out_f32=False
         keep.append(ws)
         d.ws, d.ws_bytes = ws.data_ptr(), ws_bytes
     out2 = None
-    if act == G.ACT_GELU:
+    if act == G.ACT_GELU or dgelu_out2:
         out2 = torch.zeros_like(out)
         d.out2 = out2.data_ptr()
+    cs = None
+    if colsum:
+        cs = torch.full(((M + 31) // 32, groups, N), float("nan"), dtype=torch.float32, device="cuda")
+        d.colsum = cs.data_ptr()
     if act == G.ACT_DGELU:
         aux_v = rounded(rng.standard_normal((groups, M, N)), dtype)
         xt_ = dev_tensor(aux_v, dtype)
@@ -125,6 +131,10 @@ def _run(dtype, M, N, K, groups, k_shards, causal, a_spec, b_spec, out_f32=False
     check_device_error()
     if launches is not None:
         launches.append(G.launch_count() - n0)
+    if extras is not None:
+        extras["colsum"] = None if cs is None else cs.cpu().numpy().astype(np.float64)
+        extras["out2"] = None if out2 is None or act != G.ACT_DGELU else host_values(out2, dtype)
+        extras["aux"] = aux_v
     if bias:
         exp = exp + bias_v[:, None, :]
     if resid:
@@ -191,6 +201,58 @@ def test_dgelu_epilogue_mn_major_b(dtype):
                        a_spec=((1, 260, 256), dict(mn=0)), b_spec=((2, 256, 128), dict(mn=1)),
                        act=G.ACT_DGELU)
     _close(got, exp, 1e-2)
+
+
+@pytest.mark.parametrize("dtype", DT)
+@pytest.mark.parametrize("M,K,groups", [(260, 256, 2), (700, 512, 3)])
+def test_dgelu_colsum_and_recomputed_activation(dtype, M, K, groups):
+    """The FFN2 input-gradient GEMM with its two extra epilogue outputs: the
+    32-row column sums of the stored dZ (the partials of the FFN1 bias
+    gradient; a 32-row group partly past M, and groups wholly past it that
+    must not be written) and GeLU of the stored Z again (the activation
+    recomputed for the FFN2 weight gradient)."""
+    N = 320
+    ex = {}
+    exp, got, _ = _run(dtype, M=M, N=N, K=K, groups=groups, k_shards=1, causal=0,
+                       a_spec=((1, M, K), dict(mn=0)), b_spec=((groups, K, N), dict(mn=1)),
+                       act=G.ACT_DGELU, colsum=True, dgelu_out2=True, extras=ex)
+    _close(got, exp, 1e-2)
+    rows = (M + 31) // 32
+    g64 = got.astype(np.float64)
+    want = np.stack([g64[:, 32 * r:32 * r + 32, :].sum(axis=1) for r in range(rows)])
+    mag = np.stack([np.abs(g64[:, 32 * r:32 * r + 32, :]).sum(axis=1) for r in range(rows)])
+    assert ex["colsum"].shape == want.shape
+    err = np.abs(ex["colsum"] - want)
+    assert np.all(err <= 1e-6 * mag + 1e-30), float(np.max(err / (mag + 1e-30)))
+    # GeLU of the stored argument, as the forward's bias-GeLU epilogue computes it
+    z = ex["aux"]
+    u = math.sqrt(2 / math.pi) * (z + 0.044715 * z ** 3)
+    _close(ex["out2"], 0.5 * z * (1 + np.tanh(u)), 1.5e-2)
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_recomputed_activation_is_bit_identical(dtype):
+    """GeLU recomputed in the DGELU epilogue from a stored Z equals, bit for
+    bit, the GeLU that the bias-GeLU epilogue wrote beside that Z."""
+    need_gpu()
+    M, N, K, groups = 300, 256, 128, 2
+    rng = np.random.default_rng(5)
+    tdt = torch.float16 if dtype == "fp16" else torch.bfloat16
+    at = dev_tensor(rounded(rng.standard_normal((1, M, K)), dtype), dtype)
+    bt = dev_tensor(rounded(rng.standard_normal((groups, N, K)) * 0.2, dtype), dtype)
+    _, ac = _op(at, K, M, 1, K, M * K, mn=0)
+    _, bc = _op(bt, K, N, groups, K, N * K, mn=0)
+    z, act1, dz, act2 = (torch.zeros((groups, M, N), dtype=tdt, device="cuda") for _ in range(4))
+    d = G.GemmDesc()
+    d.M, d.N, d.K, d.groups, d.k_shards, d.causal = M, N, K, groups, 1, 0
+    d.a, d.b = ac, bc
+    d.out, d.out_f32, d.ldo, d.o_mod, d.o_str_mod, d.o_str_div = z.data_ptr(), 0, N, 1, 0, M * N
+    d.out2, d.act = act1.data_ptr(), G.ACT_GELU
+    G.gemm(d, dtype, stream())
+    d.out, d.out2, d.aux, d.act = dz.data_ptr(), act2.data_ptr(), z.data_ptr(), G.ACT_DGELU
+    G.gemm(d, dtype, stream())
+    check_device_error()
+    assert torch.equal(act1.view(torch.int16), act2.view(torch.int16))
 
 
 @pytest.mark.parametrize("dtype", DT)

@@ -106,3 +106,29 @@ def test_cuda_graph_of_the_step_matches_eager_launches():
     check_device_error()
     for name in ("y", "dx", "grad", "master", "m", "v", "w16", "state"):
         assert torch.equal(getattr(eager, name), getattr(graphed, name)), name
+
+
+@pytest.mark.parametrize("name", ["small-bf16-t2", "small-fp16-t4-d80"])
+def test_gelu_recompute_is_bit_identical(name):
+    """Selective recompute of the FFN activation (the shape's recompute_gelu):
+    A = GeLU(Z) is not saved but written again from the saved Z by the FFN2
+    input-gradient GEMM.  Output, input gradient and every gradient equal the
+    saving run's bit for bit, and the saved workspace is smaller by A."""
+    need_gpu()
+    cfg = SMALL[name]
+    inp = synth.make_inputs(cfg, variant="biased", with_r=True)
+    dy = synth.loss_grad_bits(cfg, synth.HYPER["init_scale"], inp["r"])
+    runs = []
+    for recompute in (False, True):
+        ls = LayerStep(cfg, inp, recompute_gelu=recompute)
+        ls.set_dy_bits(dy)
+        ls.fwd()
+        ls.scratch.fill_(0xFF)               # the backward may not rely on scratch contents
+        ls.bwd()
+        torch.cuda.synchronize()
+        check_device_error()
+        runs.append((ls.y.clone(), ls.dx.clone(), ls.grad.clone(), ls.saved.numel()))
+        del ls
+    (y0, dx0, g0, s0), (y1, dx1, g1, s1) = runs
+    assert torch.equal(y0, y1) and torch.equal(dx0, dx1) and torch.equal(g0, g1)
+    assert s0 - s1 >= cfg.tokens * cfg.ffn * 2

@@ -114,3 +114,25 @@ def test_stack_matches_oracle_and_one_adam_covers_every_layer():
     for l in range(N_LAYERS):        # every layer's block moved
         blk = slice(l * n, (l + 1) * n)
         assert np.count_nonzero(pg[blk] != p_in[blk]) > 0.9 * np.count_nonzero(grad[blk])
+
+
+def test_stack_with_gelu_recompute_is_bit_identical():
+    """The stack with recompute_gelu (each layer's A written again in its
+    backward instead of saved) equals the saving stack bit for bit, and its
+    saved workspace is smaller by one A per layer."""
+    need_gpu()
+    params, x_bits, r_bits = _inputs()
+    dy_bits = synth.loss_grad_bits(CFG, synth.HYPER["init_scale"], r_bits)
+    runs = []
+    for recompute in (False, True):
+        st = LayerStack(CFG, params, x_bits, recompute_gelu=recompute)
+        st.set_dy_bits(dy_bits)
+        st.fwd()
+        st.bwd()
+        torch.cuda.synchronize()
+        check_device_error()
+        runs.append((st.acts.clone(), st.dx.clone(), st.grad.clone(), st.saved.numel()))
+        del st
+    (a0, dx0, g0, s0), (a1, dx1, g1, s1) = runs
+    assert torch.equal(a0, a1) and torch.equal(dx0, dx1) and torch.equal(g0, g1)
+    assert s0 - s1 >= N_LAYERS * CFG.tokens * CFG.ffn * 2

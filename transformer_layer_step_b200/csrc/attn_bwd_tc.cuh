@@ -54,7 +54,24 @@ struct AttnBwdParams {
   int q_off, k_off, v_off;
   int qdo_stages;        // dK/dV kernel: Q/dO ring depth (1..4)
   int kv_stages;         // dQ kernel: K/V ring depth (2..4)
+  // bias-gradient partials (null: none): colsum[(bb * cs_rows + r) * cs_width
+  // + i * 3h/t + column] = sum of the stored dQ/dK/dV values of shard i,
+  // batch element bb, rows 32 r .. 32 r + 31 of the sequence
+  float *colsum;
+  int batch, cs_rows, cs_width;   // cs_rows = ceil(s / 32), cs_width = t * 3h/t
 };
+
+// The 32-row column sums of one warp's 16-column chunk (values as stored, 0
+// for rows past the sequence) into the bias-gradient partials; zb = shard *
+// batch + batch element, rgrp = the 32-row group of the sequence, col = the
+// chunk's first column within the shard's 3h/t.
+__device__ __forceinline__ void attn_colsum_chunk(const AttnBwdParams &p, const float (&v)[16],
+                                                  int lane, int zb, int rgrp, int col) {
+  const float sum = warp_colsum16(v, lane);
+  if ((lane & 1) == 0 && rgrp < p.cs_rows)
+    p.colsum[((long long)(zb % p.batch) * p.cs_rows + rgrp) * p.cs_width +
+             (long long)(zb / p.batch) * (3 * p.hs) + col + ((lane >> 1) & 15)] = sum;
+}
 
 // A-operand tile [128 rows][128 cols] (16-bit), K-major, 128B swizzle: two
 // 64-column atoms 16 KB apart.  Descriptor of k-step st (16 columns).
@@ -330,15 +347,19 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
         uint32_t o[16];
         tmem_ld16(t_dq + lane_off + (uint32_t)(c * 16), o);
         tmem_wait_ld();
-        if (valid_row) {
+        float cs[16];                  // the stored values, for the bias gradient
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
           float f[8];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[h2 * 8 + e]);
+          const uint4 pk = pack8<T>(f);
+          if (valid_row) reinterpret_cast<uint4 *>(out + c * 16)[h2] = pk;
+          unpack8<T>(pk, f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[h2 * 8 + e]);
-            reinterpret_cast<uint4 *>(out + c * 16)[h2] = pack8<T>(f);
-          }
+          for (int e = 0; e < 8; ++e) cs[h2 * 8 + e] = valid_row ? f[e] : 0.f;
         }
+        if (p.colsum) attn_colsum_chunk(p, cs, lane, zb, qb * 4 + q4, p.q_off + head * d + c * 16);
       }
       tc_fence_before();
     }
@@ -662,16 +683,21 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1)
         uint32_t o[16];
         tmem_ld16((half ? t_dk : t_dv) + lane_off + (uint32_t)(c * 16), o);
         tmem_wait_ld();
-        if (valid) {
-          T *dst = rowp + (half ? p.k_off : p.v_off) + c * 16;
+        T *dst = rowp + (half ? p.k_off : p.v_off) + c * 16;
+        const int col = (half ? p.k_off : p.v_off) + head * d + c * 16;   // within the shard's 3h/t
+        float cs[16];                  // the stored values, for the bias gradient
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
           float f[8];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[h2 * 8 + e]);
+          const uint4 pk = pack8<T>(f);
+          if (valid) reinterpret_cast<uint4 *>(dst)[h2] = pk;
+          unpack8<T>(pk, f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[h2 * 8 + e]);
-            reinterpret_cast<uint4 *>(dst)[h2] = pack8<T>(f);
-          }
+          for (int e = 0; e < 8; ++e) cs[h2 * 8 + e] = valid ? f[e] : 0.f;
         }
+        if (p.colsum) attn_colsum_chunk(p, cs, lane, zb, kb * 4 + q4, col);
       }
       tc_fence_before();
     }

@@ -331,4 +331,25 @@ __device__ __forceinline__ float gelu_prime_f(float z) {
   return s * fmaf(z * (1.0f - s), fmaf(c6, zc * zc, c2), 1.0f);
 }
 
+// Sum of v[j] over the warp's 32 lanes for each of the 16 columns j, in five
+// exchange steps (16 shuffles): each step hands half of the remaining
+// columns to the partner lane and keeps the other half.  Lane l ends with
+// the sum of column (l >> 1) & 15 (lanes l and l ^ 1 hold the same value);
+// the order of the additions is fixed.
+__device__ __forceinline__ float warp_colsum16(const float (&v)[16], int lane) {
+  float s8[8], s4[4], s2[2];
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    s8[i] = (b4 ? v[i + 8] : v[i]) + __shfl_xor_sync(0xffffffffu, b4 ? v[i] : v[i + 8], 16);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    s4[i] = (b3 ? s8[i + 4] : s8[i]) + __shfl_xor_sync(0xffffffffu, b3 ? s8[i] : s8[i + 4], 8);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    s2[i] = (b2 ? s4[i + 2] : s4[i]) + __shfl_xor_sync(0xffffffffu, b2 ? s4[i] : s4[i + 2], 4);
+  const float s1 = (b1 ? s2[1] : s2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? s2[0] : s2[1], 2);
+  return s1 + __shfl_xor_sync(0xffffffffu, s1, 1);
+}
+
 }  // namespace gptl

@@ -14,7 +14,10 @@
 //     describes the all-reduce this replaces);
 //   * fused epilogues: bias, residual, bias+GeLU (writes Z and GeLU(Z): the
 //     fused_bias_gelu of "Training GPT-2 with Megatron-LM" §6.2), GeLU'
-//     scaling of an input gradient, fp32 weight-gradient store;
+//     scaling of an input gradient (optionally writing GeLU of its stored
+//     argument again: the activation recomputed for the weight gradient),
+//     32-row column sums of a 16-bit output (a bias gradient's partial
+//     sums), fp32 weight-gradient store;
 //   * outputs leave through shared memory with TMA tensor stores: each
 //     epilogue warp stages 32-row x 64-byte boxes (64B swizzle) and one lane
 //     stores them, so global writes are whole 32-byte sectors and the ragged
@@ -81,7 +84,10 @@ struct alignas(64) GemmParams {
   long long ldo;
   long long o_str_mod, o_str_div;
   int act;
+  int write_o2;                // GELU: GeLU(value) to map_o2; DGELU: GeLU(aux) to map_o2
   int *nonfinite;              // fp32 outputs: set to 1 if any value written is inf or NaN
+  float *colsum;               // 16-bit outputs: 32-row column sums [colsum_rows][groups][N]
+  int colsum_rows;             // ceil(M / 32)
 };
 
 // true when an fp32 value is inf or NaN (all exponent bits set)
@@ -213,12 +219,14 @@ __device__ __forceinline__ uint32_t box_piece(uint32_t box, int r, int j) {
 
 // Finish one 16-column chunk (fp32 accumulator values r) and write it into
 // the staging box(es): 16-bit outputs fill half a box (pieces 2*slot,
-// 2*slot+1), fp32 outputs a whole box.
+// 2*slot+1), fp32 outputs a whole box.  With p.colsum, the warp also sums the
+// chunk's 16 columns as stored (rounded; rows past M count 0) over its 32
+// rows and writes the sums to cs_out[0..15] (when cs_out is not null).
 template <typename T>
 __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow &e,
                                                const uint32_t (&r)[16], const EpiIn &in,
                                                uint32_t box, uint32_t box2, int lane, int slot,
-                                               bool &bad) {
+                                               bool &bad, float *cs_out) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
@@ -279,10 +287,15 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow
   if (e.aux) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      float z[8];
+      float z[8], a[8];
       unpack8<T>(in.v[h], z);
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[8 * h + i] *= gelu_prime_f(z[i]);
+      if (p.write_o2) {               // the activation, recomputed from its stored argument
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = gelu_f(z[i]);
+        st_shared_v4(box_piece(box2, lane, 2 * slot + h), pack8<T>(a));
+      }
     }
   }
 #pragma unroll
@@ -290,7 +303,17 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow
     float f[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) f[i] = v[8 * h + i];
-    st_shared_v4(box_piece(box, lane, 2 * slot + h), pack8<T>(f));
+    const uint4 pk = pack8<T>(f);
+    st_shared_v4(box_piece(box, lane, 2 * slot + h), pk);
+    if (p.colsum) {                     // the stored values, for the column sums
+      unpack8<T>(pk, f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[8 * h + i] = e.row_ok ? f[i] : 0.f;
+    }
+  }
+  if (p.colsum) {
+    const float sum = warp_colsum16(v, lane);
+    if (cs_out && (lane & 1) == 0) cs_out[(lane >> 1) & 15] = sum;
   }
 }
 
@@ -362,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     prefetch_tensormap(&p.map_a);
     prefetch_tensormap(&p.map_b);
     prefetch_tensormap(&p.map_o);
-    if (p.act == kActGelu) prefetch_tensormap(&p.map_o2);
+    if (p.write_o2) prefetch_tensormap(&p.map_o2);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
@@ -458,7 +481,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - 4) >> 2;        // which half of the tile's columns
     const bool wide = p.out_f32 || p.split > 1;     // fp32: one chunk per box
-    const bool gelu = !wide && p.act == kActGelu;   // Z and GeLU(Z): both boxes per chunk pair
+    const bool two = !wide && p.write_o2;     // a second output: both boxes per chunk pair
     const uint32_t my_boxes = staging_s + (uint32_t)((warp - 4) * 2 * kStageBoxBytes);
     int box_i = 0;                           // boxes issued by this warp (selects the buffer)
     bool bad = false;                        // an fp32 output value was inf or NaN
@@ -513,22 +536,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       auto process = [&](int c, const uint32_t (&r)[16], const EpiIn &in) {
         const int slot = wide ? 0 : ((c - c0) & 1);
         const bool first = slot == 0, last = wide || slot == 1 || c + 1 == c1;
-        const uint32_t buf = my_boxes + (uint32_t)((gelu ? 0 : (box_i & 1)) * kStageBoxBytes);
+        const uint32_t buf = my_boxes + (uint32_t)((two ? 0 : (box_i & 1)) * kStageBoxBytes);
         if (first) {                         // the box buffer(s) must be free again
           if (lane == 0) {
-            if (gelu) bulk_wait_read<0>();
+            if (two) bulk_wait_read<0>();
             else bulk_wait_read<1>();
           }
           __syncwarp();
         }
-        epilogue_chunk<T>(p, er, r, in, buf, my_boxes + kStageBoxBytes, lane, slot, bad);
+        // this warp's 32 rows form partial row row0 / 32 of the column sums
+        float *cs_out = nullptr;
+        if (p.colsum && (row0 >> 5) < p.colsum_rows)
+          cs_out = p.colsum + ((long long)(row0 >> 5) * p.groups + ti.g) * p.N + ti.n0 + c * 16;
+        epilogue_chunk<T>(p, er, r, in, buf, my_boxes + kStageBoxBytes, lane, slot, bad, cs_out);
         if (last) {
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
             const int x = ti.n0 + (c - slot) * 16;
             tma_store_4d(&p.map_o, buf, x, row0, oz, ow);
-            if (gelu) tma_store_4d(&p.map_o2, my_boxes + kStageBoxBytes, x, row0, oz, ow);
+            if (two) tma_store_4d(&p.map_o2, my_boxes + kStageBoxBytes, x, row0, oz, ow);
             bulk_commit();
           }
           ++box_i;

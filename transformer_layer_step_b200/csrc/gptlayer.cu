@@ -358,6 +358,8 @@ int gemm_validate(const gptl_gemm_desc &d, gptl_dtype dt) {
   if ((d.out2 && !aligned16(d.out2)) || (d.aux && !aligned16(d.aux))) return GPTL_E_ALIGN;
   if (d.act < 0 || d.act > 2 || (d.out_f32 && d.act != GPTL_ACT_NONE)) return GPTL_E_SHAPE;
   if (d.resid && d.act == GPTL_ACT_DGELU) return GPTL_E_SHAPE;   // one epilogue input per GEMM
+  if (d.colsum && !aligned16(d.colsum)) return GPTL_E_ALIGN;
+  if (d.colsum && (d.out_f32 || d.act == GPTL_ACT_GELU)) return GPTL_E_SHAPE;
   GPTL_TRY(check_operand(d.a));
   GPTL_TRY(check_operand(d.b));
   return GPTL_OK;
@@ -365,7 +367,7 @@ int gemm_validate(const gptl_gemm_desc &d, gptl_dtype dt) {
 
 GemmTiling gemm_plan(const gptl_gemm_desc &d, int sms) {
   const bool can_split = d.out_f32 && !d.bias && !d.resid && d.act == GPTL_ACT_NONE && d.ws &&
-                         aligned16(d.ws);
+                         aligned16(d.ws) && !d.colsum;
   return choose_tiling(d, sms, can_split);
 }
 
@@ -439,7 +441,8 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   } else {
     GPTL_TRY(encode_output(&p.map_o, d.out, d.out_f32, dt, d.N, d.M, d.ldo, d.groups, d.o_mod,
                            d.o_str_mod, d.o_str_div, &p.o_flat));
-    if (d.act == GPTL_ACT_GELU) {
+    if (d.act == GPTL_ACT_GELU || (d.act == GPTL_ACT_DGELU && d.out2)) {
+      p.write_o2 = 1;
       int flat2 = 0;
       GPTL_TRY(encode_output(&p.map_o2, d.out2, 0, dt, d.N, d.M, d.ldo, d.groups, d.o_mod,
                              d.o_str_mod, d.o_str_div, &flat2));
@@ -458,6 +461,8 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.aux = d.aux;
   p.act = d.act;
   p.nonfinite = d.out_f32 ? g_nonfinite : nullptr;
+  p.colsum = d.colsum;
+  p.colsum_rows = (d.M + 31) / 32;
   const int grid = (int)(p.total_tiles < sms ? p.total_tiles : sms);
   if (dt == GPTL_FP16) GPTL_TRY(launch_gemm_t<__half>(p, grid, smem, stream));
   else GPTL_TRY(launch_gemm_t<__nv_bfloat16>(p, grid, smem, stream));
@@ -553,8 +558,10 @@ int run_attn_fwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
 // Fused causal attention backward: dQ, dK, dV into the Q, K, V columns of
 // dC [t][T][3h/t] from C, dO [t][T][h/t], the forward's row log-sum-exp and
 // D = dO . O.  Two kernels (per query block: dQ; per key block: dK, dV).
+// part (may be null): the bias-gradient partials of dC, [b * ceil(s/32)][t * 3hs] fp32.
 int run_attn_bwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, const void *c,
-                 const void *dout, const float *lse, const float *dvec, void *dc, cudaStream_t st) {
+                 const void *dout, const float *lse, const float *dvec, void *dc, float *part,
+                 cudaStream_t st) {
   int sms = 0;
   GPTL_TRY(device_check(&sms));
   if (d % 16 || d > 128 || hs % 8 || s <= 0 || s % 16 || as <= 0 || b <= 0 || t <= 0)
@@ -595,6 +602,10 @@ int run_attn_bwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
   p.dc = dc;
   p.items = (long long)p.groups * p.tiles;
   p.q_off = 0; p.k_off = hs; p.v_off = 2 * hs;
+  p.colsum = part;
+  p.batch = b;
+  p.cs_rows = (s + 31) / 32;
+  p.cs_width = t * 3 * hs;
   const int tb = 256 * d;
   // rings as deep as shared memory allows (up to 4 stages): dQ kernel dS
   // 32 KB + Q, dO + K/V stages; dK/dV kernel P^T, dS^T 64 KB + K, V + Q/dO
@@ -939,6 +950,7 @@ struct Dims {
   long long T;
   gptl_dtype dt;
   float eps;
+  int recompute;   // the FFN activation A is recomputed in the backward, not saved
 };
 
 int check_shape(const gptl_shape *sh, Dims *D) {
@@ -951,6 +963,7 @@ int check_shape(const gptl_shape *sh, Dims *D) {
   if (d % 16 || d > 128 || h % 64 || (f / t) % 64 || s % 16 || s > 2048) return GPTL_E_SHAPE;
   if ((long long)b * s >= (1ll << 31)) return GPTL_E_SHAPE;
   if (!(sh->ln_eps > 0.f)) return GPTL_E_SHAPE;
+  if (sh->recompute_gelu != 0 && sh->recompute_gelu != 1) return GPTL_E_SHAPE;
   int tpr, vpt;
   if (!ln_split(h, &tpr, &vpt)) return GPTL_E_SHAPE;
   // every launch-time limit of the step is checked here, so that no call
@@ -964,6 +977,7 @@ int check_shape(const gptl_shape *sh, Dims *D) {
   D->T = (long long)b * s;
   D->dt = sh->dtype;
   D->eps = sh->ln_eps;
+  D->recompute = sh->recompute_gelu;
   return GPTL_OK;
 }
 
@@ -980,7 +994,6 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 Ws ws_layout(const Dims &D) {
   Ws w;
   const size_t e = 2, T = (size_t)D.T, h = D.h, f = D.f;
-  const size_t pe = (size_t)D.b * D.a * D.s * D.s;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -992,9 +1005,13 @@ Ws ws_layout(const Dims &D) {
   w.lse = take((size_t)D.b * D.a * D.s * 4);   // attention row log-sum-exp, fp32
   w.o = take(T * h * e);
   w.hid = take(T * h * 4);             // residual stream H, fp32
-  w.l2 = take(T * h * e); w.z = take(T * f * e); w.act = take(T * f * e);
+  w.l2 = take(T * h * e); w.z = take(T * f * e);
+  if (!D.recompute) w.act = take(T * f * e);
   w.saved = off;
   off = 0;
+  // with recompute, A = GeLU(Z) lives in scratch: the forward writes it for
+  // FFN2, the backward writes it again from the saved Z
+  if (D.recompute) w.act = take(T * f * e);
   w.dz = take(T * f * e); w.dl2 = take(T * h * e); w.dhid = take(T * h * e);
   w.dhid32 = take(T * h * 4);          // residual-stream gradient dH, fp32
   w.dO = take(T * h * e);
@@ -1004,9 +1021,12 @@ Ws ws_layout(const Dims &D) {
   // transposed 16-bit weights ([in][out] per shard) for the input-gradient GEMMs
   w.w2t = take(h * f * e); w.w1t = take(f * h * e); w.wot = take(h * h * e);
   w.wqkvt = take(3 * h * h * e);
+  // partial sums: the LayerNorm backward's, and the 32-row column sums of dZ
+  // and dC (b * ceil(s/32) rows of the wider of f and 3h)
   size_t part = 4 * 512 * h;
   const size_t widest = f > 3 * h ? f : 3 * h;
-  if (kColsumMaxSplit * widest > part) part = kColsumMaxSplit * widest;
+  const size_t cs_rows = (size_t)D.b * ((D.s + 31) / 32);
+  if (cs_rows * widest > part) part = cs_rows * widest;
   w.part = take(part * 4);
   // split-K partials of the weight-gradient GEMMs: up to 8 slices of the
   // largest gradient, at most 64 MiB (large layers have tiles enough)
@@ -1067,14 +1087,15 @@ int validate_weights(const gptl_weights *w) {
 }
 
 int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void *saved,
-              cudaStream_t st) {
+              void *scratch, cudaStream_t st) {
   const Ws w = ws_layout(D);
   const gptl_dtype dt = D.dt;
   const int T = (int)D.T, h = D.h, t = D.t, s = D.s, d = D.d, hs = D.hs, as = D.as, fs = D.fs;
   void *l1 = at<void>(saved, w.l1), *c = at<void>(saved, w.c);
   float *lse = at<float>(saved, w.lse);
   void *o = at<void>(saved, w.o), *hid = at<void>(saved, w.hid), *l2 = at<void>(saved, w.l2);
-  void *z = at<void>(saved, w.z), *act = at<void>(saved, w.act);
+  void *z = at<void>(saved, w.z);
+  void *act = D.recompute ? at<void>(scratch, w.act) : at<void>(saved, w.act);
   float *mu1 = at<float>(saved, w.mu1), *rs1 = at<float>(saved, w.rstd1);
   float *mu2 = at<float>(saved, w.mu2), *rs2 = at<float>(saved, w.rstd2);
   TagScope tag_scope(GPTL_TAG_NONE);
@@ -1150,11 +1171,13 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   const Ws w = ws_layout(D);
   const gptl_dtype dt = D.dt;
   const int T = (int)D.T, h = D.h, t = D.t, s = D.s, d = D.d, hs = D.hs, as = D.as, fs = D.fs;
-  const int G = D.b * D.a;
   const void *l1 = at<void>(saved, w.l1), *c = at<void>(saved, w.c);
   const float *lse = at<float>(saved, w.lse);
   const void *o = at<void>(saved, w.o), *hid = at<void>(saved, w.hid);
-  const void *l2 = at<void>(saved, w.l2), *z = at<void>(saved, w.z), *act = at<void>(saved, w.act);
+  const void *l2 = at<void>(saved, w.l2), *z = at<void>(saved, w.z);
+  // A = GeLU(Z): saved by the forward, or (recompute) written again below
+  void *act_re = D.recompute ? at<void>(scratch, w.act) : nullptr;
+  const void *act = D.recompute ? act_re : at<void>(saved, w.act);
   const float *mu1 = at<float>(saved, w.mu1), *rs1 = at<float>(saved, w.rstd1);
   const float *mu2 = at<float>(saved, w.mu2), *rs2 = at<float>(saved, w.rstd2);
   void *dz = at<void>(scratch, w.dz), *dl2 = at<void>(scratch, w.dl2);
@@ -1185,12 +1208,23 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   }
 
   // ---- FFN2 (row split)
-  g_tag = GPTL_TAG_B2_DW2;
   // Weight gradients reduce over the tokens, the row index of both
   // activations; the tensor core runs markedly faster when one operand is
   // token-contiguous, so the smaller operand is transposed first.
   g_tag = GPTL_TAG_B2_DOUT_T;
   GPTL_TRY(run_transpose(T, h, dy, h, xt, T, st));
+  g_tag = GPTL_TAG_B1_B3_DZ;
+  {  // dZ_i = (dOut W2_i) * gelu'(Z_i); the epilogue also sums dZ_i's columns
+     // over each 32 rows (db_1's partials)
+    gptl_gemm_desc g = gemm(T, fs, h, t, view(dy, h, T, 1, h, 0, 0),
+                            view(w2t, h, fs, t, h, (long long)fs * h, 0), dz, fs,
+                            (long long)T * fs);
+    g.act = GPTL_ACT_DGELU;
+    g.aux = z;
+    g.colsum = part;
+    g.out2 = act_re;                     // recompute: A_i = gelu(Z_i) again, for dW2
+    GPTL_TRY(run_gemm(g, dt, st));
+  }
   g_tag = GPTL_TAG_B2_DW2;
   {  // dW2_i = dOut^T A_i   [t][h][f/t] fp32
     gptl_gemm_desc g = gemm(h, fs, T, t, view(xt, T, h, 1, T, 0, 0),
@@ -1201,18 +1235,9 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     g.ws_bytes = splitk_bytes;
     GPTL_TRY(run_gemm(g, dt, st));
   }
-  g_tag = GPTL_TAG_B1_B3_DZ;
-  {  // dZ_i = (dOut W2_i) * gelu'(Z_i)
-    gptl_gemm_desc g = gemm(T, fs, h, t, view(dy, h, T, 1, h, 0, 0),
-                            view(w2t, h, fs, t, h, (long long)fs * h, 0), dz, fs,
-                            (long long)T * fs);
-    g.act = GPTL_ACT_DGELU;
-    g.aux = z;
-    GPTL_TRY(run_gemm(g, dt, st));
-  }
   // ---- FFN1 (column split)
-  g_tag = GPTL_TAG_B3_DB1;
-  GPTL_TRY(run_colsum(T, fs, t, fs, (long long)T * fs, dt, dz, gr->b_1, part, st));
+  g_tag = GPTL_TAG_B3_DB1;   // db_1 = the partials' sum, in a fixed order
+  GPTL_TRY(launch_reduce_parts(part, (T + 31) / 32, t * fs, 1, gr->b_1, nullptr, nullptr, nullptr, st));
   g_tag = GPTL_TAG_B5_L2_T;
   GPTL_TRY(run_transpose(T, h, l2, h, xt, T, st));
   g_tag = GPTL_TAG_B5_DW1;
@@ -1262,12 +1287,14 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   // ---- attention backward
   g_tag = GPTL_TAG_B9_ROWDOT;   // D = rowsum(dO * O), the softmax backward's row term
   GPTL_TRY(run_attn_rowdot((long long)t * T, s, hs, as, d, dt, dO, o, dvec, st));
-  // fused attention backward: dQ, dK, dV into dC (P and dS stay on chip)
+  // fused attention backward: dQ, dK, dV into dC (P and dS stay on chip),
+  // with the 32-row column sums of dC (db_qkv's partials)
   g_tag = GPTL_TAG_B8_B10_ATTN;
-  GPTL_TRY(run_attn_bwd(D.b, s, hs, as, t, d, dt, c, dO, lse, dvec, dc, st));
+  GPTL_TRY(run_attn_bwd(D.b, s, hs, as, t, d, dt, c, dO, lse, dvec, dc, part, st));
   // ---- QKV (column split)
   g_tag = GPTL_TAG_B11_DBQKV;
-  GPTL_TRY(run_colsum(T, 3 * hs, t, 3 * hs, (long long)T * 3 * hs, dt, dc, gr->b_qkv, part, st));
+  GPTL_TRY(launch_reduce_parts(part, D.b * ((s + 31) / 32), t * 3 * hs, 1, gr->b_qkv, nullptr,
+                               nullptr, nullptr, st));
   g_tag = GPTL_TAG_B11_L1_T;
   GPTL_TRY(run_transpose(T, h, l1, h, xt, T, st));
   g_tag = GPTL_TAG_B11_DWQKV;
@@ -1355,14 +1382,14 @@ int gpt_layer_param_layout(const gptl_shape *shape, size_t offsets[12], size_t *
 
 int gpt_layer_fwd(const gptl_shape *shape, const gptl_weights *w, const void *x, void *y,
                   void *saved, void *scratch, gptl_stream_t stream) {
-  (void)scratch;
   Dims D;
   GPTL_TRY(check_shape(shape, &D));
   GPTL_TRY(validate_weights(w));
-  if (!x || !y || !saved) return GPTL_E_NULL;
-  if (!aligned16(x) || !aligned16(y) || !aligned16(saved)) return GPTL_E_ALIGN;
+  if (!x || !y || !saved || (D.recompute && !scratch)) return GPTL_E_NULL;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(saved) || (scratch && !aligned16(scratch)))
+    return GPTL_E_ALIGN;
   GPTL_TRY(device_check());
-  return layer_fwd(D, w, x, y, saved, reinterpret_cast<cudaStream_t>(stream));
+  return layer_fwd(D, w, x, y, saved, scratch, reinterpret_cast<cudaStream_t>(stream));
 }
 
 namespace {
@@ -1586,8 +1613,11 @@ int gptl_attention_fwd(int batch, int seq, int hidden, int heads, int tp, gptl_d
 
 int gptl_attention_bwd(int batch, int seq, int hidden, int heads, int tp, gptl_dtype dtype,
                        const void *qkv, const void *o, const void *dout, const float *lse,
-                       float *dvec, void *dqkv, gptl_stream_t stream) {
+                       float *dvec, void *dqkv, float *dbias_part, float *dbias,
+                       gptl_stream_t stream) {
   if (!qkv || !o || !dout || !lse || !dvec || !dqkv) return GPTL_E_NULL;
+  if ((dbias_part == nullptr) != (dbias == nullptr)) return GPTL_E_NULL;
+  if (dbias && (!aligned16(dbias_part) || !aligned16(dbias))) return GPTL_E_ALIGN;
   if (dtype != GPTL_FP16 && dtype != GPTL_BF16) return GPTL_E_DTYPE;
   if (!aligned16(qkv) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) || !aligned16(dvec) ||
       !aligned16(dqkv))
@@ -1600,7 +1630,11 @@ int gptl_attention_bwd(int batch, int seq, int hidden, int heads, int tp, gptl_d
   if (d % 16 || d > 128 || seq % 16) return GPTL_E_SHAPE;
   prof_start(st);
   GPTL_TRY(run_attn_rowdot((long long)tp * batch * seq, seq, hs, as, d, dtype, dout, o, dvec, st));
-  return run_attn_bwd(batch, seq, hs, as, tp, d, dtype, qkv, dout, lse, dvec, dqkv, st);
+  GPTL_TRY(run_attn_bwd(batch, seq, hs, as, tp, d, dtype, qkv, dout, lse, dvec, dqkv, dbias_part,
+                        st));
+  if (!dbias) return GPTL_OK;
+  return launch_reduce_parts(dbias_part, batch * ((seq + 31) / 32), tp * 3 * hs, 1, dbias, nullptr,
+                             nullptr, nullptr, st);
 }
 
 // Column sums with their partials in a fixed device array instead of

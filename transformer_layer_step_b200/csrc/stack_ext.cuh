@@ -61,19 +61,21 @@ int gpt_stack_workspace_bytes(const gptl_shape *shape, int n_layers, size_t *sav
 }
 
 int gpt_stack_fwd(const gptl_shape *shape, int n_layers, const gptl_weights *w, const void *x,
-                  void *acts, void *saved, gptl_stream_t stream) {
+                  void *acts, void *saved, void *scratch, gptl_stream_t stream) {
   Dims D;
   StackSizes s;
   GPTL_TRY(stack_sizes(shape, n_layers, &D, &s));
-  if (!w || !x || !acts || !saved) return GPTL_E_NULL;
-  if (!aligned16(x) || !aligned16(acts) || !aligned16(saved)) return GPTL_E_ALIGN;
+  if (!w || !x || !acts || !saved || (D.recompute && !scratch)) return GPTL_E_NULL;
+  if (!aligned16(x) || !aligned16(acts) || !aligned16(saved) || (scratch && !aligned16(scratch)))
+    return GPTL_E_ALIGN;
   for (int l = 0; l < n_layers; ++l) GPTL_TRY(validate_weights(&w[l]));
   GPTL_TRY(device_check());
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const void *in = x;
   for (int l = 0; l < n_layers; ++l) {
     void *out = static_cast<uint8_t *>(acts) + (size_t)l * s.act;
-    GPTL_TRY(layer_fwd(D, &w[l], in, out, static_cast<uint8_t *>(saved) + (size_t)l * s.saved, st));
+    GPTL_TRY(layer_fwd(D, &w[l], in, out, static_cast<uint8_t *>(saved) + (size_t)l * s.saved,
+                       scratch, st));
     in = out;
   }
   return GPTL_OK;

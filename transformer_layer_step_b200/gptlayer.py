@@ -34,7 +34,8 @@ class GptlError(RuntimeError):
 
 class Shape(C.Structure):
     _fields_ = [("batch", C.c_int), ("seq", C.c_int), ("hidden", C.c_int), ("heads", C.c_int),
-                ("ffn", C.c_int), ("tp", C.c_int), ("dtype", C.c_int), ("ln_eps", C.c_float)]
+                ("ffn", C.c_int), ("tp", C.c_int), ("dtype", C.c_int), ("ln_eps", C.c_float),
+                ("recompute_gelu", C.c_int)]
 
 
 class Weights(C.Structure):
@@ -65,7 +66,7 @@ class GemmDesc(C.Structure):
                 ("bias", C.c_void_p), ("bias_g_stride", C.c_longlong), ("resid", C.c_void_p),
                 ("ld_resid", C.c_longlong), ("aux", C.c_void_p), ("out2", C.c_void_p),
                 ("act", C.c_int), ("resid_f32", C.c_int), ("ws", C.c_void_p),
-                ("ws_bytes", C.c_longlong)]
+                ("ws_bytes", C.c_longlong), ("colsum", C.c_void_p)]
 
 
 class LaunchRecord(C.Structure):
@@ -99,7 +100,7 @@ _SIGS = {
     "gpt_stack_workspace_bytes": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(C.c_size_t),
                                             C.POINTER(C.c_size_t)]),
     "gpt_stack_fwd": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(Weights), C.c_void_p,
-                                C.c_void_p, C.c_void_p, C.c_void_p]),
+                                C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gpt_stack_bwd": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(Weights), C.c_void_p,
                                 C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.POINTER(Grads),
                                 C.c_void_p, C.c_void_p]),
@@ -127,7 +128,7 @@ _SIGS = {
                               C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gptl_attention_fwd": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
-    "gptl_attention_bwd": (C.c_int, [C.c_int] * 6 + [C.c_void_p] * 7),
+    "gptl_attention_bwd": (C.c_int, [C.c_int] * 6 + [C.c_void_p] * 9),
     "gptl_colsum_noalloc": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_longlong, C.c_longlong,
                                       C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     "gptl_launch_count": (C.c_ulonglong, []),
@@ -184,8 +185,9 @@ def _check(rc: int, where: str):
         raise GptlError(rc, where)
 
 
-def make_shape(batch, seq, hidden, heads, ffn, tp, dtype, ln_eps=1e-5) -> Shape:
-    return Shape(batch, seq, hidden, heads, ffn, tp, DTYPES.get(dtype, dtype), ln_eps)
+def make_shape(batch, seq, hidden, heads, ffn, tp, dtype, ln_eps=1e-5, recompute_gelu=0) -> Shape:
+    return Shape(batch, seq, hidden, heads, ffn, tp, DTYPES.get(dtype, dtype), ln_eps,
+                 int(recompute_gelu))
 
 
 def workspace_bytes(shape: Shape):
@@ -235,11 +237,12 @@ def stack_workspace_bytes(shape: Shape, n_layers: int):
     return a.value, b.value
 
 
-def stack_fwd(shape, weights, x, acts, saved, stream=0):
-    """weights: a sequence of Weights, one per layer."""
+def stack_fwd(shape, weights, x, acts, saved, scratch=None, stream=0):
+    """weights: a sequence of Weights, one per layer; scratch: needed when the
+    shape has recompute_gelu."""
     arr = (Weights * len(weights))(*weights)
     _check(lib().gpt_stack_fwd(C.byref(shape), len(weights), arr, _ptr(x), _ptr(acts),
-                               _ptr(saved), stream), "gpt_stack_fwd")
+                               _ptr(saved), _ptr(scratch), stream), "gpt_stack_fwd")
 
 
 def stack_bwd(shape, weights, x, acts, saved, dy, dx, grads, scratch, stream=0):
@@ -348,9 +351,11 @@ def attention_fwd(batch, seq, hidden, heads, tp, dtype, qkv, o, lse, stream=0):
                                     _ptr(o), _ptr(lse), stream), "gptl_attention_fwd")
 
 
-def attention_bwd(batch, seq, hidden, heads, tp, dtype, qkv, o, dout, lse, dvec, dqkv, stream=0):
+def attention_bwd(batch, seq, hidden, heads, tp, dtype, qkv, o, dout, lse, dvec, dqkv,
+                  dbias_part=None, dbias=None, stream=0):
     _check(lib().gptl_attention_bwd(batch, seq, hidden, heads, tp, DTYPES.get(dtype, dtype), _ptr(qkv),
-                                    _ptr(o), _ptr(dout), _ptr(lse), _ptr(dvec), _ptr(dqkv), stream),
+                                    _ptr(o), _ptr(dout), _ptr(lse), _ptr(dvec), _ptr(dqkv),
+                                    _ptr(dbias_part), _ptr(dbias), stream),
            "gptl_attention_bwd")
 
 

@@ -31,12 +31,13 @@ def tensor_to_bits(t: torch.Tensor) -> np.ndarray:
 class LayerStep:
     """Everything one layer step needs on `device`, filled from synth inputs."""
 
-    def __init__(self, cfg: synth.LayerConfig, inputs: dict, device="cuda", hyper=None):
+    def __init__(self, cfg: synth.LayerConfig, inputs: dict, device="cuda", hyper=None,
+                 recompute_gelu=False):
         self.cfg = cfg
         self.hyper = dict(synth.HYPER, **(hyper or {}))
         self.device = torch.device(device)
         self.shape = G.make_shape(cfg.batch, cfg.seq, cfg.hidden, cfg.heads, cfg.ffn, cfg.tp,
-                                  cfg.dtype, self.hyper["ln_eps"])
+                                  cfg.dtype, self.hyper["ln_eps"], recompute_gelu)
         self.offsets, self.n_params = G.param_layout(self.shape)
         saved_b, scratch_b = G.workspace_bytes(self.shape)
         dt = TORCH_DT[cfg.dtype]
@@ -91,7 +92,7 @@ class LayerStep:
 
     def fwd(self, x=None, y=None):
         G.layer_fwd(self.shape, self.weights, self.x if x is None else x,
-                    self.y if y is None else y, self.saved, None, self.stream())
+                    self.y if y is None else y, self.saved, self.scratch, self.stream())
 
     def bwd(self, x=None, dy=None, checked=False):
         """gpt_layer_bwd, or with checked=True gpt_layer_bwd_checked (the
@@ -154,12 +155,12 @@ class LayerStack(LayerStep):
     stack's arenas."""
 
     def __init__(self, cfg: synth.LayerConfig, layer_params: list, x_bits: np.ndarray,
-                 device="cuda", hyper=None):
+                 device="cuda", hyper=None, recompute_gelu=False):
         self.cfg = cfg
         self.hyper = dict(synth.HYPER, **(hyper or {}))
         self.device = torch.device(device)
         self.shape = G.make_shape(cfg.batch, cfg.seq, cfg.hidden, cfg.heads, cfg.ffn, cfg.tp,
-                                  cfg.dtype, self.hyper["ln_eps"])
+                                  cfg.dtype, self.hyper["ln_eps"], recompute_gelu)
         self.n_layers = L = len(layer_params)
         self.offsets, self.n_layer_params = G.param_layout(self.shape)
         self.n_params = L * self.n_layer_params
@@ -204,7 +205,7 @@ class LayerStack(LayerStep):
         if y is not None:
             raise ValueError("the stack writes its output into acts[-1]")
         G.stack_fwd(self.shape, self.layer_weights, self.x if x is None else x, self.acts,
-                    self.saved, self.stream())
+                    self.saved, self.scratch, self.stream())
 
     def bwd(self, x=None, dy=None, checked=False):
         if checked:
