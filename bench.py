@@ -82,11 +82,13 @@ def step_flops(cfg) -> dict:
             "linear": 3 * linear, "attn_fwd": attn_causal, "attn_bwd": 2 * attn_causal}
 
 
-def kernel_bytes(cfg, n_params: int, layers: int = 1) -> dict:
+def kernel_bytes(cfg, n_params: int, layers: int = 1, weight_copies: bool = False) -> dict:
     """Algorithmic HBM bytes of each bandwidth kernel of the step, summed over
     its launches in one step (2-byte activations, 4-byte fp32 state; a stack
     of `layers` layers launches each per-layer kernel once per layer; the
-    optimizer's n_params covers every layer)."""
+    optimizer's n_params covers every layer).  With weight_copies the
+    optimizer step also writes the transposed 16-bit weight matrices (2 B per
+    matrix element) and the backward does not transpose them."""
     b, s, h, a, f = cfg.batch, cfg.seq, cfg.hidden, cfg.heads, cfg.ffn
     T = b * s
     # the residual stream H and its gradient dH are fp32 (4 B), the rest 2 B
@@ -105,12 +107,15 @@ def kernel_bytes(cfg, n_params: int, layers: int = 1) -> dict:
         "B11 dbqkv": 4 * 3 * h * (b * ((s + 31) // 32) + 1),
     }
     out = {k: v * layers for k, v in per_layer.items()}
-    out.update({"O1 overflow": 4 * n_params, "O2 adam": 30 * n_params})
+    adam = 30 * n_params
+    if weight_copies:
+        adam += 2 * (4 * h * h + 2 * h * f) * layers
+    out.update({"O1 overflow": 4 * n_params, "O2 adam": adam})
     return out
 
 
 def kernel_rooflines(kinds: dict, rows: list, cfg, n_params: int, flops: dict, peaks: dict,
-                     peak_src: str, layers: int = 1) -> dict:
+                     peak_src: str, layers: int = 1, weight_copies: bool = False) -> dict:
     """Achieved rate against the roofline of every kernel family of the
     step, per step: the tensor-core families (the GEMM with its split-K sums,
     the attention forward and backward) as algorithmic FLOPs over their
@@ -133,7 +138,7 @@ def kernel_rooflines(kinds: dict, rows: list, cfg, n_params: int, flops: dict, p
             out[fam] = {"bound": "tensor", "ms_per_step": round(t, 5), "achieved": round(a, 1),
                         "peak": peak_tf, "unit": "TFLOP/s", "frac": round(a / peak_tf, 4),
                         "peak_source": f"{peak_src} bf16_tflops_sustained"}
-    nbytes = kernel_bytes(cfg, n_params, layers)
+    nbytes = kernel_bytes(cfg, n_params, layers, weight_copies)
     for row in rows:
         if row["step"] not in nbytes or row["kind"] in ("gemm", "splitk", "attn_fwd", "attn_bwd"):
             continue
@@ -358,9 +363,11 @@ def run_ours(args, cfg, rank, world, local_rank):
         # L layers of the shape, each starting from the same seeded weights,
         # with parameters of their own in one arena, and one Adam over all
         ls = LayerStack(cfg, [inp["params"]] * args.layers, inp["x"], device=dev,
-                        recompute_gelu=args.recompute_gelu)
+                        recompute_gelu=args.recompute_gelu,
+                        weight_copies=not args.transpose_in_backward)
     else:
-        ls = LayerStep(cfg, inp, device=dev, recompute_gelu=args.recompute_gelu)
+        ls = LayerStep(cfg, inp, device=dev, recompute_gelu=args.recompute_gelu,
+                       weight_copies=not args.transpose_in_backward)
     dy_bits = synth.loss_grad_bits(cfg, ls.hyper["init_scale"], inp["r"])
     ls.set_dy_bits(dy_bits)
     stream = torch.cuda.current_stream(dev)
@@ -582,7 +589,7 @@ def measure_extensions(G, ls, cfg, dev, flush, peaks, reps=5):
     }
 
 
-def summarize_kernels(recs, K, cfg, n_params, peaks, flops, layers=1):
+def summarize_kernels(recs, K, cfg, n_params, peaks, flops, layers=1, weight_copies=False):
     """Per-kernel device time per step, share, and achieved rate."""
     by_tag, by_kind = {}, {}
     for kind, tag, ms in recs:
@@ -593,7 +600,7 @@ def summarize_kernels(recs, K, cfg, n_params, peaks, flops, layers=1):
         k["launches"] += 1
         k["ms"] += ms
     total = sum(e["ms"] for e in by_kind.values())
-    nbytes = kernel_bytes(cfg, n_params, layers)
+    nbytes = kernel_bytes(cfg, n_params, layers, weight_copies)
     rows = []
     for tag, e in by_tag.items():
         ms = e["ms"] / K
@@ -726,6 +733,10 @@ def main():
     ap.add_argument("--layers", type=int, default=1,
                     help="a stack of this many layers of the workload's shape per step "
                          "(gpt_stack_fwd / gpt_stack_bwd and one Adam over every layer)")
+    ap.add_argument("--transpose-in-backward", action="store_true",
+                    help="the backward transposes the weight matrices itself every step, instead "
+                         "of reading the copies that the optimizer step writes "
+                         "(gpt_layer_adam_step)")
     ap.add_argument("--recompute-gelu", action="store_true",
                     help="selective recompute: the FFN activation is written again in the "
                          "backward (by the FFN2 input-gradient GEMM) instead of saved")
@@ -748,6 +759,8 @@ def main():
               "e2e_step_launch": "kernel by kernel" if args.e2e_eager else "one CUDA graph per step",
               "e2e_copies": "one stream per direction, overlapped with the neighbouring steps",
               "l2": "flushed between steps (256 MiB write, outside the per-step events)"}
+    config["weight_transposes"] = ("in the backward" if args.transpose_in_backward else
+                                   "written by the optimizer step (gpt_layer_adam_step)")
     if args.recompute_gelu:
         config["recompute_gelu"] = True
     L = args.layers
@@ -790,9 +803,10 @@ def main():
     import torch
     res = run_ours(args, cfg, rank, world, local_rank)
     peaks, peak_src = load_peaks()
+    wcp = not args.transpose_in_backward
     rows, kinds, prof_ms = summarize_kernels(res["recs"], args.steps, cfg, res["n_params"],
-                                             peaks, flops, L)
-    by_kernel = kernel_rooflines(kinds, rows, cfg, res["n_params"], flops, peaks, peak_src, L)
+                                             peaks, flops, L, wcp)
+    by_kernel = kernel_rooflines(kinds, rows, cfg, res["n_params"], flops, peaks, peak_src, L, wcp)
     dom_name = max(by_kernel, key=lambda k: by_kernel[k]["ms_per_step"])
     dom = by_kernel[dom_name]
     peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])

@@ -95,6 +95,13 @@ typedef struct {
   const void *ln2_g, *ln2_b;
   const void *w_1, *b_1;
   const void *w_2, *b_2;
+  /* Optional (all four or none): the four weight matrices transposed shard
+   * by shard, as gpt_layer_adam_step and gpt_layer_transpose_weights write
+   * them: w_qkv_t [t][h][3h/t], w_o_t [t][h/t][h], w_1_t [t][h][f/t],
+   * w_2_t [t][f/t][h].  The backward's input-gradient products read these;
+   * when they are NULL the backward transposes the weights itself into its
+   * scratch.  The forward ignores them. */
+  const void *w_qkv_t, *w_o_t, *w_1_t, *w_2_t;
 } gptl_weights;
 
 /* FP32 gradients, same layouts as gptl_weights, multiplied by the loss scale
@@ -232,6 +239,35 @@ int gpt_stack_fwd(const gptl_shape *shape, int n_layers, const gptl_weights *w, 
 int gpt_stack_bwd(const gptl_shape *shape, int n_layers, const gptl_weights *w, const void *x,
                   const void *acts, const void *saved, const void *dy, void *dx,
                   const gptl_grads *g, void *scratch, gptl_stream_t stream);
+
+/* The optimizer step for n_layers layers of one shape whose parameters lie
+ * back to back in one arena (n_layers * n_params elements, n_params and the
+ * offsets of gpt_layer_param_layout), that also writes the transposed 16-bit
+ * copy of every layer's four weight matrices into w16t: for the matrix at
+ * offset o of the layout, shard i ([rows][cols] at o + i*rows*cols) goes
+ * transposed to w16t + o + i*rows*cols as [cols][rows].  Elements of w16t
+ * outside the four matrices are not written.  Point gptl_weights' *_t
+ * fields of layer l at w16t + l*n_params + o, and the next backward reads
+ * these copies instead of transposing the weights (at h = 10240, t = 4 that
+ * is 2.5 GB per step written here instead of 5 GB moved there).
+ *   prechecked = 0: overflow check of grad first, as adam_step_fp32_master;
+ *   prechecked = 1: the flag gpt_layer_bwd_checked left in st->found_inf, as
+ *                   adam_step_fp32_master_prechecked.
+ * master, m, v, w16 and w16t are updated exactly as adam_step_fp32_master
+ * updates master, m, v and w16 (the same arithmetic, bit for bit); on a
+ * skipped step nothing is written.  w16t must not overlap the other arrays.
+ * Errors as gpt_layer_workspace_bytes and adam_step_fp32_master, and
+ * GPTL_E_ARG if n_layers < 1 or prechecked is not 0 or 1. */
+int gpt_layer_adam_step(const gptl_shape *shape, int n_layers, float *master, float *m, float *v,
+                        const float *grad, void *w16, void *w16t, float lr, float beta1,
+                        float beta2, float eps, float weight_decay, int prechecked,
+                        gptl_scaler_state *st, gptl_stream_t stream);
+
+/* The transposed copies alone, from the 16-bit weights w16 (n_layers arenas
+ * as above) into w16t: for the first backward, or after the weights were
+ * changed by anything other than gpt_layer_adam_step. */
+int gpt_layer_transpose_weights(const gptl_shape *shape, int n_layers, const void *w16, void *w16t,
+                                gptl_stream_t stream);
 
 /* Bytes of device workspace adam_step_fp32_master_clip takes (clip_ws). */
 #define GPTL_CLIP_WORKSPACE_BYTES 16384

@@ -184,3 +184,24 @@ def test_gelu_recompute_moves_the_activation_to_scratch(name):
     with pytest.raises(G.GptlError) as e:
         G.workspace_bytes(G.make_shape(*args, recompute_gelu=2))
     assert e.value.code == G.E_SHAPE
+
+
+def test_weight_copy_arguments_rejected_without_launch():
+    """gpt_layer_adam_step / gpt_layer_transpose_weights and the optional
+    transposed-weight fields of gptl_weights are checked before any launch."""
+    lib = G.lib()
+    sh = G.make_shape(2, 64, 128, 4, 512, 2, "fp16")
+    st = 16
+    args = lambda n_layers, w16t, pre: (ctypes.byref(sh), n_layers, 16, 16, 16, 16, 16, w16t,
+                                        1e-3, 0.9, 0.95, 1e-8, 0.0, pre, st, None)
+    assert lib.gpt_layer_adam_step(*args(0, 16, 0)) == G.E_ARG
+    assert lib.gpt_layer_adam_step(*args(1, 16, 2)) == G.E_ARG
+    assert lib.gpt_layer_adam_step(*args(1, None, 0)) == G.E_NULL
+    assert lib.gpt_layer_adam_step(*args(1, 24, 1)) == G.E_ALIGN
+    assert lib.gpt_layer_transpose_weights(ctypes.byref(sh), 1, None, 16, None) == G.E_NULL
+    assert lib.gpt_layer_transpose_weights(ctypes.byref(sh), 0, 16, 16, None) == G.E_ARG
+    # the four copies come all together or not at all
+    w = G.make_weights({n: 16 for n in G.PARAM_NAMES} | {"w_qkv_t": 16, "w_o_t": 16})
+    assert lib.gpt_layer_fwd(ctypes.byref(sh), ctypes.byref(w), 16, 16, 16, None, None) == G.E_NULL
+    w = G.make_weights({n: 16 for n in G.PARAM_NAMES} | {n: 16 for n in G.WT_NAMES[:3]} | {"w_2_t": 24})
+    assert lib.gpt_layer_fwd(ctypes.byref(sh), ctypes.byref(w), 16, 16, 16, None, None) == G.E_ALIGN

@@ -400,15 +400,24 @@ struct AdamArgs {
   float lr, beta1, beta2, eps, wd;
 };
 
-// Fused unscale + Adam + 16-bit cast; skipped entirely when found_inf.
-template <typename T>
-__global__ void __launch_bounds__(256) adam_kernel(float4 *__restrict__ master,
-                                                   float4 *__restrict__ m, float4 *__restrict__ v,
-                                                   const float4 *__restrict__ grad,
-                                                   T *__restrict__ w16, long long n4, AdamArgs a,
-                                                   const gptl_scaler_state *st) {
-  // the scaler state and the bias corrections 1 - beta^t (in fp64) are read
-  // and formed once per block, not per thread
+// One element of the fused unscale + Adam update ("Megatron-LM overview"
+// §3.1, §4.2): g = grad / S; m = b1 m + (1 - b1) g; v = b2 v + (1 - b2) g^2;
+// p -= lr ((m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps) + wd p).  Both
+// optimizer kernels call this one function, so they round alike.
+__device__ __forceinline__ void adam_update(const AdamArgs &a, float scale, float bc1, float bc2,
+                                            float g_scaled, float &p, float &m, float &v) {
+  const float g = g_scaled / scale;
+  m = a.beta1 * m + (1.0f - a.beta1) * g;
+  v = a.beta2 * v + (1.0f - a.beta2) * (g * g);
+  const float mh = m / bc1;
+  const float vh = v / bc2;
+  p = p - a.lr * (mh / (sqrtf(vh) + a.eps) + a.wd * p);
+}
+
+// The scaler state and the bias corrections 1 - beta^t (in fp64), read and
+// formed once per block; false when the step is skipped (found_inf).
+__device__ __forceinline__ bool adam_block_state(const AdamArgs &a, const gptl_scaler_state *st,
+                                                 float &scale, float &bc1, float &bc2) {
   __shared__ float sh[3];
   __shared__ int skip;
   if (threadIdx.x == 0) {
@@ -419,34 +428,164 @@ __global__ void __launch_bounds__(256) adam_kernel(float4 *__restrict__ master,
     sh[2] = (float)(1.0 - pow((double)a.beta2, (double)t));
   }
   __syncthreads();
-  if (skip) return;
-  const float scale = sh[0], bc1 = sh[1], bc2 = sh[2];
-  const float omb1 = 1.0f - a.beta1, omb2 = 1.0f - a.beta2;
+  scale = sh[0];
+  bc1 = sh[1];
+  bc2 = sh[2];
+  return !skip;
+}
+
+// Fused unscale + Adam + 16-bit cast over a flat arena; skipped entirely
+// when found_inf.
+template <typename T>
+__global__ void __launch_bounds__(256) adam_kernel(float4 *__restrict__ master,
+                                                   float4 *__restrict__ m, float4 *__restrict__ v,
+                                                   const float4 *__restrict__ grad,
+                                                   T *__restrict__ w16, long long n4, AdamArgs a,
+                                                   const gptl_scaler_state *st) {
+  float scale, bc1, bc2;
+  if (!adam_block_state(a, st, scale, bc1, bc2)) return;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (long long)gridDim.x * blockDim.x) {
     const float4 g4 = __ldcs(grad + i);
     float4 p4 = master[i], m4 = m[i], v4 = v[i];
-    float gg[4] = {g4.x, g4.y, g4.z, g4.w};
-    float pp[4] = {p4.x, p4.y, p4.z, p4.w};
-    float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-    float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float g = gg[k] / scale;
-      mm[k] = a.beta1 * mm[k] + omb1 * g;
-      vv[k] = a.beta2 * vv[k] + omb2 * (g * g);
-      const float mh = mm[k] / bc1;
-      const float vh = vv[k] / bc2;
-      pp[k] = pp[k] - a.lr * (mh / (sqrtf(vh) + a.eps) + a.wd * pp[k]);
-    }
-    master[i] = make_float4(pp[0], pp[1], pp[2], pp[3]);
-    m[i] = make_float4(mm[0], mm[1], mm[2], mm[3]);
-    v[i] = make_float4(vv[0], vv[1], vv[2], vv[3]);
+    adam_update(a, scale, bc1, bc2, g4.x, p4.x, m4.x, v4.x);
+    adam_update(a, scale, bc1, bc2, g4.y, p4.y, m4.y, v4.y);
+    adam_update(a, scale, bc1, bc2, g4.z, p4.z, m4.z, v4.z);
+    adam_update(a, scale, bc1, bc2, g4.w, p4.w, m4.w, v4.w);
+    master[i] = p4;
+    m[i] = m4;
+    v[i] = v4;
     uint2 w;
-    w.x = Cvt<T>::pack2(pp[0], pp[1]);
-    w.y = Cvt<T>::pack2(pp[2], pp[3]);
+    w.x = Cvt<T>::pack2(p4.x, p4.y);
+    w.y = Cvt<T>::pack2(p4.z, p4.w);
     reinterpret_cast<uint2 *>(w16)[i] = w;
   }
+}
+
+// ------------------------------------- Adam that also writes W^T (16-bit)
+// The optimizer step over n_layers layers' arenas (n_params apart) that also
+// writes each weight matrix's transposed 16-bit copy into w16t, at the same
+// offsets: the input-gradient products of the next backward read those
+// instead of transposing the weights again.  Blocks [0, mat_blocks) each take
+// a 64 x 64 tile of one shard of one weight matrix: the tile's rows are read
+// and written as 16-byte vectors (every array once), and its 16-bit values go
+// through shared memory to be written as rows of the transposed copy.  The
+// remaining blocks take 1024-element chunks of the vectors between the
+// matrices (LayerNorm parameters, biases, padding).
+struct AdamMat {
+  long long off;               // first element of shard 0 within a layer
+  int rows, cols;              // one shard: [rows][cols]
+  int tiles_r, tiles_c;        // 64 x 64 tiles per shard
+  long long tile0;             // first tile of this matrix within a layer
+};
+struct AdamVec {
+  long long off, len;          // a range of elements within a layer
+  long long chunk0;            // its first 1024-element chunk within a layer
+};
+struct AdamWtPlan {
+  AdamMat mat[4];
+  AdamVec vec[5];
+  int nmat, nvec, shards;
+  long long layer_stride;      // n_params
+  long long mat_tiles;         // per layer
+  long long vec_chunks;        // per layer
+  long long mat_blocks;        // n_layers * mat_tiles
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) adam_wt_kernel(float *__restrict__ master, float *__restrict__ m,
+                                                      float *__restrict__ v,
+                                                      const float *__restrict__ grad,
+                                                      T *__restrict__ w16, T *__restrict__ w16t,
+                                                      const __grid_constant__ AdamWtPlan P, AdamArgs a,
+                                                      const gptl_scaler_state *st) {
+  __shared__ uint16_t tile[64][66];    // [column][row] of the tile, 16-bit; padded rows
+  float scale, bc1, bc2;
+  if (!adam_block_state(a, st, scale, bc1, bc2)) return;
+  const int tid = threadIdx.x;
+  long long b = blockIdx.x;
+  if (b < P.mat_blocks) {
+    const long long layer = b / P.mat_tiles;
+    long long t = b - layer * P.mat_tiles;
+    int k = 0;
+    while (k + 1 < P.nmat && t >= P.mat[k + 1].tile0) ++k;
+    const AdamMat &M = P.mat[k];
+    t -= M.tile0;
+    const int per = M.tiles_r * M.tiles_c;
+    const int shard = (int)(t / per);
+    const int rem = (int)(t - (long long)shard * per);
+    const int r0 = (rem / M.tiles_c) * 64, c0 = (rem % M.tiles_c) * 64;
+    const long long base = layer * P.layer_stride + M.off + (long long)shard * M.rows * M.cols;
+    // rows r0 + rr, columns c0 + 4 cq .. + 3: 16 threads per row, 16 rows a pass
+    const int cq = tid & 15;
+    const int c = c0 + 4 * cq;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int rr = pass * 16 + (tid >> 4);
+      const int r = r0 + rr;
+      uint16_t out[4] = {0, 0, 0, 0};
+      if (r < M.rows && c < M.cols) {
+        const long long i = base + (long long)r * M.cols + c;   // multiple of 4
+        const float4 g4 = __ldcs(reinterpret_cast<const float4 *>(grad + i));
+        float4 p4 = *reinterpret_cast<float4 *>(master + i);
+        float4 m4 = *reinterpret_cast<float4 *>(m + i);
+        float4 v4 = *reinterpret_cast<float4 *>(v + i);
+        adam_update(a, scale, bc1, bc2, g4.x, p4.x, m4.x, v4.x);
+        adam_update(a, scale, bc1, bc2, g4.y, p4.y, m4.y, v4.y);
+        adam_update(a, scale, bc1, bc2, g4.z, p4.z, m4.z, v4.z);
+        adam_update(a, scale, bc1, bc2, g4.w, p4.w, m4.w, v4.w);
+        *reinterpret_cast<float4 *>(master + i) = p4;
+        *reinterpret_cast<float4 *>(m + i) = m4;
+        *reinterpret_cast<float4 *>(v + i) = v4;
+        uint2 w;
+        w.x = Cvt<T>::pack2(p4.x, p4.y);
+        w.y = Cvt<T>::pack2(p4.z, p4.w);
+        *reinterpret_cast<uint2 *>(w16 + i) = w;
+        out[0] = (uint16_t)(w.x & 0xffffu); out[1] = (uint16_t)(w.x >> 16);
+        out[2] = (uint16_t)(w.y & 0xffffu); out[3] = (uint16_t)(w.y >> 16);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tile[4 * cq + e][rr] = out[e];
+    }
+    __syncthreads();
+    // transposed rows c0 + cc, elements r0 + 8 q .. + 7 (16 bytes each)
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      const int cc = pass * 32 + (tid >> 3), q = tid & 7;
+      if (c0 + cc < M.cols && r0 + 8 * q < M.rows) {
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(&tile[cc][8 * q]);
+        const uint4 val = make_uint4(src[0], src[1], src[2], src[3]);
+        *reinterpret_cast<uint4 *>(w16t + base + (long long)(c0 + cc) * M.rows + r0 + 8 * q) = val;
+      }
+    }
+    return;
+  }
+  // a 1024-element chunk of one vector range of one layer
+  b -= P.mat_blocks;
+  const long long layer = b / P.vec_chunks;
+  long long ch = b - layer * P.vec_chunks;
+  int k = 0;
+  while (k + 1 < P.nvec && ch >= P.vec[k + 1].chunk0) ++k;
+  const AdamVec &V = P.vec[k];
+  ch -= V.chunk0;
+  const long long e0 = ch * 1024 + 4 * tid;
+  if (e0 >= V.len) return;
+  const long long i = layer * P.layer_stride + V.off + e0;   // multiple of 4
+  const float4 g4 = __ldcs(reinterpret_cast<const float4 *>(grad + i));
+  float4 p4 = *reinterpret_cast<float4 *>(master + i);
+  float4 m4 = *reinterpret_cast<float4 *>(m + i);
+  float4 v4 = *reinterpret_cast<float4 *>(v + i);
+  adam_update(a, scale, bc1, bc2, g4.x, p4.x, m4.x, v4.x);
+  adam_update(a, scale, bc1, bc2, g4.y, p4.y, m4.y, v4.y);
+  adam_update(a, scale, bc1, bc2, g4.z, p4.z, m4.z, v4.z);
+  adam_update(a, scale, bc1, bc2, g4.w, p4.w, m4.w, v4.w);
+  *reinterpret_cast<float4 *>(master + i) = p4;
+  *reinterpret_cast<float4 *>(m + i) = m4;
+  *reinterpret_cast<float4 *>(v + i) = v4;
+  uint2 w;
+  w.x = Cvt<T>::pack2(p4.x, p4.y);
+  w.y = Cvt<T>::pack2(p4.z, p4.w);
+  *reinterpret_cast<uint2 *>(w16 + i) = w;
 }
 
 __global__ void scale_update_kernel(gptl_scaler_state *st, int interval, float growth,

@@ -140,6 +140,22 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, uint32_t sr
       "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
       : "memory");
 }
+// The same store with an L2 eviction-priority hint (a createpolicy value):
+// outputs that nothing reads soon (the weight gradients, read by the
+// optimizer step) leave L2 first and do not push the operands out.
+__device__ __forceinline__ void tma_store_4d_hint(const CUtensorMap *map, uint32_t src, int x, int y,
+                                                  int z, int w, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group.L2::cache_hint"
+      " [%0, {%2, %3, %4, %5}], [%1], %6;" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "r"(z), "r"(w), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -88,6 +88,7 @@ struct alignas(64) GemmParams {
   int *nonfinite;              // fp32 outputs: set to 1 if any value written is inf or NaN
   float *colsum;               // 16-bit outputs: 32-row column sums [colsum_rows][groups][N]
   int colsum_rows;             // ceil(M / 32)
+  int out_evict_first;         // store the output with L2 evict-first priority
 };
 
 // true when an fp32 value is inf or NaN (all exponent bits set)
@@ -554,7 +555,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
           __syncwarp();
           if (lane == 0) {
             const int x = ti.n0 + (c - slot) * 16;
-            tma_store_4d(&p.map_o, buf, x, row0, oz, ow);
+            if (p.out_evict_first) tma_store_4d_hint(&p.map_o, buf, x, row0, oz, ow, l2_policy_evict_first());
+            else tma_store_4d(&p.map_o, buf, x, row0, oz, ow);
             if (two) tma_store_4d(&p.map_o2, my_boxes + kStageBoxBytes, x, row0, oz, ow);
             bulk_commit();
           }

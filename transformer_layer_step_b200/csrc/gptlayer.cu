@@ -463,6 +463,10 @@ int run_gemm(const gptl_gemm_desc &d, gptl_dtype dt, cudaStream_t stream) {
   p.nonfinite = d.out_f32 ? g_nonfinite : nullptr;
   p.colsum = d.colsum;
   p.colsum_rows = (d.M + 31) / 32;
+  // fp32 outputs without a residual are weight gradients, which the next
+  // kernels do not read: their stores leave L2 first instead of evicting
+  // the operands that the other CTAs are still reading
+  p.out_evict_first = d.out_f32 && !d.resid && p.split == 1;
   const int grid = (int)(p.total_tiles < sms ? p.total_tiles : sms);
   if (dt == GPTL_FP16) GPTL_TRY(launch_gemm_t<__half>(p, grid, smem, stream));
   else GPTL_TRY(launch_gemm_t<__nv_bfloat16>(p, grid, smem, stream));
@@ -1083,7 +1087,29 @@ int validate_weights(const gptl_weights *w) {
     if (!p) return GPTL_E_NULL;
     if (!aligned16(p)) return GPTL_E_ALIGN;
   }
+  // the transposed copies: all four or none
+  const void *ts[4] = {w->w_qkv_t, w->w_o_t, w->w_1_t, w->w_2_t};
+  int given = 0;
+  for (const void *p : ts) {
+    if (!p) continue;
+    ++given;
+    if (!aligned16(p)) return GPTL_E_ALIGN;
+  }
+  if (given != 0 && given != 4) return GPTL_E_NULL;
   return GPTL_OK;
+}
+
+// The four weight matrices transposed shard by shard (one launch): the
+// layout gptl_weights' *_t fields describe.
+int run_weight_transposes(const Dims &D, const gptl_weights *W, void *wqkvt, void *wot, void *w1t,
+                          void *w2t, cudaStream_t st) {
+  const int h = D.h, t = D.t, hs = D.hs, fs = D.fs;
+  const TransposeSpec wt[4] = {
+      {h, fs, W->w_2, fs, w2t, h, t, (long long)h * fs, (long long)fs * h},
+      {fs, h, W->w_1, h, w1t, fs, t, (long long)fs * h, (long long)h * fs},
+      {h, hs, W->w_o, hs, wot, h, t, (long long)h * hs, (long long)hs * h},
+      {3 * hs, h, W->w_qkv, h, wqkvt, 3 * hs, t, (long long)3 * hs * h, (long long)h * 3 * hs}};
+  return run_transposes(wt, 4, st);
 }
 
 int layer_fwd(const Dims &D, const gptl_weights *W, const void *x, void *y, void *saved,
@@ -1186,8 +1212,12 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   void *dc = at<void>(scratch, w.dc), *dl1 = at<void>(scratch, w.dl1);
   float *dvec = at<float>(scratch, w.dvec);
   void *xt = at<void>(scratch, w.xt);   // [h][T]: one token-contiguous copy at a time
-  void *w2t = at<void>(scratch, w.w2t), *w1t = at<void>(scratch, w.w1t);
-  void *wot = at<void>(scratch, w.wot), *wqkvt = at<void>(scratch, w.wqkvt);
+  // the transposed weights: the caller's copies, or transposed below
+  const bool own_wt = W->w_qkv_t == nullptr;
+  const void *w2t = own_wt ? at<void>(scratch, w.w2t) : W->w_2_t;
+  const void *w1t = own_wt ? at<void>(scratch, w.w1t) : W->w_1_t;
+  const void *wot = own_wt ? at<void>(scratch, w.wot) : W->w_o_t;
+  const void *wqkvt = own_wt ? at<void>(scratch, w.wqkvt) : W->w_qkv_t;
   float *part = at<float>(scratch, w.part);
   void *splitk = at<void>(scratch, w.splitk);
   const long long splitk_bytes = (long long)w.splitk_bytes;
@@ -1196,16 +1226,11 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   prof_start(st);
 
   // The input-gradient GEMMs read the weights with the reduction index
-  // contiguous: transposed copies, shard by shard.
+  // contiguous: transposed copies, shard by shard (unless the caller's
+  // optimizer step wrote them already).
   g_tag = GPTL_TAG_B0_WT;
-  {
-    const TransposeSpec wt[4] = {
-        {h, fs, W->w_2, fs, w2t, h, t, (long long)h * fs, (long long)fs * h},
-        {fs, h, W->w_1, h, w1t, fs, t, (long long)fs * h, (long long)h * fs},
-        {h, hs, W->w_o, hs, wot, h, t, (long long)h * hs, (long long)hs * h},
-        {3 * hs, h, W->w_qkv, h, wqkvt, 3 * hs, t, (long long)3 * hs * h, (long long)h * 3 * hs}};
-    GPTL_TRY(run_transposes(wt, 4, st));
-  }
+  if (own_wt) GPTL_TRY(run_weight_transposes(D, W, at<void>(scratch, w.wqkvt), at<void>(scratch, w.wot),
+                                             at<void>(scratch, w.w1t), at<void>(scratch, w.w2t), st));
 
   // ---- FFN2 (row split)
   // Weight gradients reduce over the tokens, the row index of both
@@ -1447,7 +1472,131 @@ int launch_adam(size_t n_params, float *master, float *m, float *v, const float 
   prof_launched(s, GPTL_KIND_ADAM);
   return GPTL_OK;
 }
+
+// Element offsets of the 12 parameter tensors in one layer's arena (the
+// layout gpt_layer_param_layout reports) and its length.
+void param_offsets(const Dims &D, size_t off[12], size_t *n_params) {
+  const size_t h = D.h, f = D.f;
+  const size_t sizes[12] = {h, h, 3 * h * h, 3 * h, h * h, h, h, h, f * h, f, h * f, h};
+  size_t o = 0;
+  for (int i = 0; i < 12; ++i) {
+    off[i] = o;
+    o += (sizes[i] + 63) / 64 * 64;
+  }
+  *n_params = o;
+}
+
+// The optimizer step that also writes the transposed weight matrices
+// (adam_wt_kernel): the plan lists each layer's four matrices (shards of
+// [rows][cols]) and the five vector ranges between them.
+int launch_adam_wt(const Dims &D, int n_layers, float *master, float *m, float *v,
+                   const float *grad, void *w16, void *w16t, float lr, float beta1, float beta2,
+                   float eps, float weight_decay, gptl_scaler_state *st, cudaStream_t s) {
+  size_t off[12], n_params = 0;
+  param_offsets(D, off, &n_params);
+  AdamWtPlan P;
+  memset(&P, 0, sizeof(P));
+  const int h = D.h, hs = D.hs, fs = D.fs;
+  // (tensor index, shard rows, shard cols): w_qkv, w_o, w_1, w_2
+  const int mats[4][3] = {{2, 3 * hs, h}, {4, h, hs}, {8, fs, h}, {10, h, fs}};
+  long long tiles = 0;
+  for (int k = 0; k < 4; ++k) {
+    AdamMat &M = P.mat[k];
+    M.off = (long long)off[mats[k][0]];
+    M.rows = mats[k][1];
+    M.cols = mats[k][2];
+    M.tiles_r = (M.rows + 63) / 64;
+    M.tiles_c = (M.cols + 63) / 64;
+    M.tile0 = tiles;
+    tiles += (long long)D.t * M.tiles_r * M.tiles_c;
+  }
+  P.nmat = 4;
+  P.mat_tiles = tiles;
+  // the vectors: [ln1_g, w_qkv), [b_qkv, w_o), [b_o, w_1), [b_1, w_2), [b_2, end)
+  const size_t vr[5][2] = {{off[0], off[2]}, {off[3], off[4]}, {off[5], off[8]}, {off[9], off[10]},
+                           {off[11], n_params}};
+  long long chunks = 0;
+  for (int k = 0; k < 5; ++k) {
+    AdamVec &V = P.vec[k];
+    V.off = (long long)vr[k][0];
+    V.len = (long long)(vr[k][1] - vr[k][0]);
+    V.chunk0 = chunks;
+    chunks += (V.len + 1023) / 1024;
+  }
+  P.nvec = 5;
+  P.vec_chunks = chunks;
+  P.shards = D.t;
+  P.layer_stride = (long long)n_params;
+  P.mat_blocks = (long long)n_layers * P.mat_tiles;
+  const long long blocks = P.mat_blocks + (long long)n_layers * P.vec_chunks;
+  if (blocks >= (1ll << 31)) return GPTL_E_SHAPE;
+  AdamArgs a{lr, beta1, beta2, eps, weight_decay};
+  if (D.dt == GPTL_FP16)
+    adam_wt_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(
+        master, m, v, grad, static_cast<__half *>(w16), static_cast<__half *>(w16t), P, a, st);
+  else
+    adam_wt_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+        master, m, v, grad, static_cast<__nv_bfloat16 *>(w16), static_cast<__nv_bfloat16 *>(w16t),
+        P, a, st);
+  GPTL_CK(cudaGetLastError());
+  prof_launched(s, GPTL_KIND_ADAM);
+  return GPTL_OK;
+}
 }  // namespace
+
+int gpt_layer_adam_step(const gptl_shape *shape, int n_layers, float *master, float *m, float *v,
+                        const float *grad, void *w16, void *w16t, float lr, float beta1,
+                        float beta2, float eps, float weight_decay, int prechecked,
+                        gptl_scaler_state *st, gptl_stream_t stream) {
+  Dims D;
+  GPTL_TRY(check_shape(shape, &D));
+  if (n_layers < 1 || (prechecked != 0 && prechecked != 1)) return GPTL_E_ARG;
+  size_t off[12], n_params = 0;
+  param_offsets(D, off, &n_params);
+  if (!w16t) return GPTL_E_NULL;
+  if (!aligned16(w16t)) return GPTL_E_ALIGN;
+  const size_t n_all = n_params * (size_t)n_layers;
+  GPTL_TRY(adam_validate(n_all, master, m, v, grad, w16, D.dt, lr, beta1, beta2, eps,
+                         weight_decay, st));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  TagScope tag_scope(GPTL_TAG_O1_OVERFLOW);
+  if (!prechecked) {
+    GPTL_TRY(gptl_check_overflow(n_all, grad, st, stream));
+  } else {
+    prof_start(s);
+  }
+  g_tag = GPTL_TAG_O2_ADAM;
+  return launch_adam_wt(D, n_layers, master, m, v, grad, w16, w16t, lr, beta1, beta2, eps,
+                        weight_decay, st, s);
+}
+
+int gpt_layer_transpose_weights(const gptl_shape *shape, int n_layers, const void *w16, void *w16t,
+                                gptl_stream_t stream) {
+  Dims D;
+  GPTL_TRY(check_shape(shape, &D));
+  if (n_layers < 1) return GPTL_E_ARG;
+  if (!w16 || !w16t) return GPTL_E_NULL;
+  if (!aligned16(w16) || !aligned16(w16t)) return GPTL_E_ALIGN;
+  GPTL_TRY(device_check());
+  size_t off[12], n_params = 0;
+  param_offsets(D, off, &n_params);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  TagScope tag_scope(GPTL_TAG_B0_WT);
+  prof_start(s);
+  for (int l = 0; l < n_layers; ++l) {
+    const size_t base = (size_t)l * n_params * 2;   // bytes
+    auto in = [&](int i) { return static_cast<const void *>(static_cast<const char *>(w16) + base + off[i] * 2); };
+    auto out = [&](int i) { return static_cast<void *>(static_cast<char *>(w16t) + base + off[i] * 2); };
+    gptl_weights W;
+    memset(&W, 0, sizeof(W));
+    W.w_qkv = in(2);
+    W.w_o = in(4);
+    W.w_1 = in(8);
+    W.w_2 = in(10);
+    GPTL_TRY(run_weight_transposes(D, &W, out(2), out(4), out(8), out(10), s));
+  }
+  return GPTL_OK;
+}
 
 int gpt_layer_bwd_checked(const gptl_shape *shape, const gptl_weights *w, const void *x,
                           const void *saved, const void *dy, void *dx, const gptl_grads *g,

@@ -24,6 +24,8 @@ E_TOO_LARGE = -9
 DTYPES = {"fp16": FP16, "bf16": BF16}
 PARAM_NAMES = ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
                "ln2_g", "ln2_b", "w_1", "b_1", "w_2", "b_2")
+# optional transposed copies of the four weight matrices (gptl_weights)
+WT_NAMES = ("w_qkv_t", "w_o_t", "w_1_t", "w_2_t")
 
 
 class GptlError(RuntimeError):
@@ -39,7 +41,7 @@ class Shape(C.Structure):
 
 
 class Weights(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in PARAM_NAMES]
+    _fields_ = [(n, C.c_void_p) for n in PARAM_NAMES + WT_NAMES]
 
 
 class Grads(C.Structure):
@@ -97,6 +99,10 @@ _SIGS = {
                                                    C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                                    C.c_float, C.c_float, C.c_float, C.c_float,
                                                    C.c_float, C.c_void_p, C.c_void_p]),
+    "gpt_layer_adam_step": (C.c_int, [C.POINTER(Shape), C.c_int] + [C.c_void_p] * 6 +
+                            [C.c_float] * 5 + [C.c_int, C.c_void_p, C.c_void_p]),
+    "gpt_layer_transpose_weights": (C.c_int, [C.POINTER(Shape), C.c_int, C.c_void_p, C.c_void_p,
+                                              C.c_void_p]),
     "gpt_stack_workspace_bytes": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(C.c_size_t),
                                             C.POINTER(C.c_size_t)]),
     "gpt_stack_fwd": (C.c_int, [C.POINTER(Shape), C.c_int, C.POINTER(Weights), C.c_void_p,
@@ -205,7 +211,8 @@ def param_layout(shape: Shape):
 
 
 def make_weights(ptrs: dict) -> Weights:
-    return Weights(*[_ptr(ptrs[n]) for n in PARAM_NAMES])
+    """ptrs: the 12 parameter pointers, and optionally the 4 WT_NAMES copies."""
+    return Weights(*[_ptr(ptrs[n]) for n in PARAM_NAMES], *[_ptr(ptrs.get(n)) for n in WT_NAMES])
 
 
 def make_grads(ptrs: dict) -> Grads:
@@ -260,6 +267,21 @@ def adam_step(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps, w
     _check(lib().adam_step_fp32_master(n_params, _ptr(master), _ptr(m), _ptr(v), _ptr(grad),
                                        _ptr(w16), DTYPES.get(dtype, dtype), lr, beta1, beta2, eps,
                                        weight_decay, _ptr(state), stream), "adam_step_fp32_master")
+
+
+def layer_adam_step(shape, n_layers, master, m, v, grad, w16, w16t, lr, beta1, beta2, eps,
+                    weight_decay, prechecked, state, stream=0):
+    """gpt_layer_adam_step: the optimizer step that also writes the transposed
+    weight matrices of n_layers layer arenas into w16t."""
+    _check(lib().gpt_layer_adam_step(C.byref(shape), n_layers, _ptr(master), _ptr(m), _ptr(v),
+                                     _ptr(grad), _ptr(w16), _ptr(w16t), lr, beta1, beta2, eps,
+                                     weight_decay, int(prechecked), _ptr(state), stream),
+           "gpt_layer_adam_step")
+
+
+def transpose_weights(shape, n_layers, w16, w16t, stream=0):
+    _check(lib().gpt_layer_transpose_weights(C.byref(shape), n_layers, _ptr(w16), _ptr(w16t), stream),
+           "gpt_layer_transpose_weights")
 
 
 def adam_step_prechecked(n_params, master, m, v, grad, w16, dtype, lr, beta1, beta2, eps,

@@ -32,7 +32,7 @@ class LayerStep:
     """Everything one layer step needs on `device`, filled from synth inputs."""
 
     def __init__(self, cfg: synth.LayerConfig, inputs: dict, device="cuda", hyper=None,
-                 recompute_gelu=False):
+                 recompute_gelu=False, weight_copies=False):
         self.cfg = cfg
         self.hyper = dict(synth.HYPER, **(hyper or {}))
         self.device = torch.device(device)
@@ -66,12 +66,35 @@ class LayerStep:
         self.state = torch.zeros(8, dtype=torch.int32, device=dev)
         self.reset_scaler(self.hyper["init_scale"])
 
+        self.n_layers = 1
+        self.w16t = self._weight_copies(weight_copies)
         wp, gp = {}, {}
         for name, off in zip(G.PARAM_NAMES, self.offsets):
             wp[name] = self.w16.data_ptr() + 2 * off
             gp[name] = self.grad.data_ptr() + 4 * off
+        wp.update(self._copy_ptrs(0))
         self.weights = G.make_weights(wp)
         self.grads = G.make_grads(gp)
+
+    # ---------------------------------------------------------------- W^T
+    def _weight_copies(self, on: bool):
+        """With weight_copies the optimizer step (gpt_layer_adam_step) keeps
+        transposed copies of the weight matrices in w16t (the same offsets as
+        w16), and the backward reads them instead of transposing the weights;
+        the first copies are made here."""
+        if not on:
+            return None
+        w16t = torch.zeros_like(self.w16)
+        G.transpose_weights(self.shape, self.n_layers, self.w16, w16t, self.stream())
+        return w16t
+
+    def _copy_ptrs(self, layer: int) -> dict:
+        if self.w16t is None:
+            return {}
+        base = layer * self.n_layer_params if hasattr(self, "n_layer_params") else 0
+        names = dict(zip(G.PARAM_NAMES, self.offsets))
+        return {wt: self.w16t.data_ptr() + 2 * (base + names[w])
+                for wt, w in zip(G.WT_NAMES, ("w_qkv", "w_o", "w_1", "w_2"))}
 
     # ---------------------------------------------------------------- state
     def reset_scaler(self, scale: float, tracker: int = 0, step: int = 0):
@@ -110,6 +133,11 @@ class LayerStep:
         """adam_step_fp32_master (overflow scan + update), or with
         prechecked=True the update alone, on the flag a checked backward set."""
         hp = self.hyper
+        if self.w16t is not None:          # also writes the transposed weights
+            G.layer_adam_step(self.shape, self.n_layers, self.master, self.m, self.v, self.grad,
+                              self.w16, self.w16t, hp["lr"], hp["beta1"], hp["beta2"], hp["eps"],
+                              hp["weight_decay"], prechecked, self.state, self.stream())
+            return
         fn = G.adam_step_prechecked if prechecked else G.adam_step
         fn(self.n_params, self.master, self.m, self.v, self.grad, self.w16, self.cfg.dtype,
            hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], self.state,
@@ -155,7 +183,7 @@ class LayerStack(LayerStep):
     stack's arenas."""
 
     def __init__(self, cfg: synth.LayerConfig, layer_params: list, x_bits: np.ndarray,
-                 device="cuda", hyper=None, recompute_gelu=False):
+                 device="cuda", hyper=None, recompute_gelu=False, weight_copies=False):
         self.cfg = cfg
         self.hyper = dict(synth.HYPER, **(hyper or {}))
         self.device = torch.device(device)
@@ -193,11 +221,13 @@ class LayerStack(LayerStep):
         self.state = torch.zeros(8, dtype=torch.int32, device=dev)
         self.reset_scaler(self.hyper["init_scale"])
 
+        self.w16t = self._weight_copies(weight_copies)
         self.layer_weights, self.layer_grads = [], []
         for l in range(L):
             base = l * self.n_layer_params
-            self.layer_weights.append(G.make_weights(
-                {n: self.w16.data_ptr() + 2 * (base + off) for n, off in zip(G.PARAM_NAMES, self.offsets)}))
+            wp = {n: self.w16.data_ptr() + 2 * (base + off) for n, off in zip(G.PARAM_NAMES, self.offsets)}
+            wp.update(self._copy_ptrs(l))
+            self.layer_weights.append(G.make_weights(wp))
             self.layer_grads.append(G.make_grads(
                 {n: self.grad.data_ptr() + 4 * (base + off) for n, off in zip(G.PARAM_NAMES, self.offsets)}))
 
