@@ -483,6 +483,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     const int half = (warp - 4) >> 2;        // which half of the tile's columns
     const bool wide = p.out_f32 || p.split > 1;     // fp32: one chunk per box
     const bool two = !wide && p.write_o2;     // a second output: both boxes per chunk pair
+    // no bias, residual, activation or second K half: nothing to load per chunk
+    const bool grouped = !p.bias && !p.resid && p.act == kActNone && !p.pipe_k;
     const uint32_t my_boxes = staging_s + (uint32_t)((warp - 4) * 2 * kStageBoxBytes);
     int box_i = 0;                           // boxes issued by this warp (selects the buffer)
     bool bad = false;                        // an fp32 output value was inf or NaN
@@ -518,8 +520,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       int c1 = half ? nchunk : csplit;
       const int valid = (p.N - ti.n0 + 15) / 16;   // chunks inside N
       if (c1 > valid) c1 = valid;
-      // software pipeline: the load of chunk c+1 is in flight while chunk c
-      // is processed (tcgen05.wait::ld waits for every earlier load)
       uint32_t ra[16], rb[16];
       EpiIn ia, ib;
       const uint32_t t_row2 = t_row + (uint32_t)p.bn_alloc;   // pipe_k: the second K half
@@ -563,6 +563,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
           ++box_i;
         }
       };
+      if (grouped) {
+        // chunks in pairs, both tensor-memory loads in flight before one
+        // wait: the load latency, which bounds this epilogue, is paid once
+        // per 32 columns (measured on the 10240 x 10240 x 2048 weight-
+        // gradient product: 372 -> 353 us)
+        for (int c = c0; c < c1; c += 2) {
+          const bool has_b = c + 1 < c1;
+          ld(c, ra);
+          if (has_b) ld(c + 1, rb);
+          tmem_wait_ld();
+          process(c, ra, ia);
+          if (has_b) process(c + 1, rb, ia);
+        }
+        continue;
+      }
+      // with epilogue inputs: the load of chunk c+1 (and its inputs) is in
+      // flight while chunk c is processed (tcgen05.wait::ld waits for every
+      // earlier load)
       if (c0 < c1) {
         ld(c0, ra);
         epilogue_load<T>(p, er, ti.n0 + c0 * 16, ia);
