@@ -616,7 +616,7 @@ def summarize_kernels(recs, K, cfg, n_params, peaks, flops, layers=1, weight_cop
 
 
 # ------------------------------------------------------- single-kernel cases
-CASES = ("gemm-ffn2", "gemm-dw1", "attention", "layernorm", "adam")
+CASES = ("gemm-ffn2", "gemm-dw1", "attention", "layernorm", "adam", "adam-wt")
 
 
 def run_case(args, cfg):
@@ -686,6 +686,19 @@ def run_case(args, cfg):
         def work():
             G.layernorm_fwd(T, h, cfg.dtype, x, g, b, 1e-5, y, mu, rs, st)
             G.layernorm_bwd(T, h, cfg.dtype, gy, x, mu, rs, g, res, dx, dg, db, dsum, scr, st)
+        flops = 0.0
+    elif args.case == "adam-wt":          # the step's optimizer: Adam + the transposed weights
+        # of one layer of the 2.4B recipe's shape (78.7 M parameters, 1.4 GB of arrays)
+        c2 = synth.CONFIGS["gpt-2.4b"]
+        sh = G.make_shape(c2.batch, c2.seq, c2.hidden, c2.heads, c2.ffn, c2.tp, cfg.dtype)
+        _, n = G.param_layout(sh)
+        p32, m, v, g = (torch.randn(n, device="cuda") * 0.02 for _ in range(4))
+        w16 = torch.empty(n, dtype=tdt, device="cuda")
+        w16t = torch.zeros_like(w16)
+        state = torch.zeros(8, dtype=torch.int32, device="cuda")
+        state[0] = int(np.array([65536.0], np.float32).view(np.int32)[0])
+        work = lambda: G.layer_adam_step(sh, 1, p32, m, v, g, w16, w16t, 6e-5, 0.9, 0.95, 1e-8, 0.0,
+                                         True, state, st)
         flops = 0.0
     else:                                 # adam: overflow check + Adam over 64 M parameters
         n = 64 << 20

@@ -16,34 +16,38 @@
 // would round different values.  The kernel writes O and lse, from which the
 // backward recomputes P.
 //
-// Warp roles (384 threads, one CTA per SM, persistent over work items):
+// Warp roles (640 threads, one CTA per SM, persistent over work items):
 //   warp 0      TMA: Q once per item, then per key block K (pass 1) or K and
 //               V (pass 2) into a ring of kv_stages (2..4) stages;
 //   warp 1      one thread issues S_j = Q K_j^T into one of two S buffers;
 //   warps 2-3   one thread each issues O += P_j V_j once P_j is ready, warp 2
 //               over keys 0..63 of the block into O, warp 3 over keys 64..127
 //               into O2 (added at the end): the MMA streams run concurrently;
-//   warps 4-11  softmax: warp w reads TMEM lane quarter w % 4 (32 query rows,
-//               one per thread) and half (w - 4) / 4 of the key block's 128
-//               columns.  Pass 1 keeps a running max and sum per half row;
-//               the two halves of a row meet once per item through shared
-//               memory to form lse.  Pass 2 writes its 64 columns of P_j into
-//               one of two shared-memory P buffers (so that P_j is formed
-//               while P_{j-1} V_{j-1} runs).  At the end each warp stores its
-//               share of O's columns.
+//   warps 4-19  softmax: warp w reads TMEM lane quarter w % 4 (32 query rows,
+//               one per thread) and quarter (w - 4) / 4 of the key block's
+//               128 columns (32 columns), four warps per SM sub-partition to
+//               hide the latency of their tensor-memory loads and exp2 chains.
+//               Pass 1 keeps a running max and sum per quarter row; the four
+//               quarters of a row meet once per item through shared memory to
+//               form lse.  Pass 2 writes its 32 columns of P_j into one of two
+//               shared-memory P buffers (so that P_j is formed while
+//               P_{j-1} V_{j-1} runs).  At the end each warp stores its share
+//               of O's columns.
 // Tensor memory: S buffers at columns 0 and 128, O at column 256, O2 at 384.
 // Shared memory: two P buffers [128 x 128] (two 128B-swizzled 64-column
 // atoms each), Q as head_dim/16 chunks of [128 rows x 16] (32B swizzle), per
 // stage K the same way and V as MN-major chunks of [64 keys x vw], then the
-// barriers and the half-row log-sum-exps.
+// barriers.  The quarter-row log-sum-exps are exchanged inside P buffer 0,
+// which is idle between an item's passes: lane quarter q uses bytes
+// [4096 q, +512) of its first atom, the rows that only q's warps write.
 #pragma once
 #include "common.cuh"
 
 namespace gptl {
 
-constexpr int kAttnThreads = 384;
+constexpr int kAttnThreads = 640;    // 20 warps: 4 roles + 16 softmax
 constexpr int kAttnTile = 128;          // query rows per item, keys per block
-constexpr int kAttnTailBytes = 1280;    // barriers (256 B) + half-row lse [2][128] fp32
+constexpr int kAttnTailBytes = 256;     // barriers
 
 struct AttnParams {
   CUtensorMap map_qk;   // C as [t*b][s][3h/t]; box {16, 128, 1}, 32B swizzle
@@ -101,14 +105,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   // products complete
   auto p_full = [&](int b) { return smem_u32(&bars[14 + b]); };
   auto pv_done = [&](int b) { return smem_u32(&bars[16 + b]); };
-  // the two softmax warps of lane quarter q exchange their half-row lse
+  // the four softmax warps of lane quarter q exchange their quarter-row lse
   auto stat_full = [&](int q) { return smem_u32(&bars[18 + q]); };
   auto stat_read = [&](int q) { return smem_u32(&bars[22 + q]); };
   const uint32_t drain_bar = smem_u32(&bars[26]);
   auto drain_pv = [&](int h) { return smem_u32(&bars[27 + h]); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 29);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  float *half_lse = reinterpret_cast<float *>(bars + 32);     // [2 halves][128 rows]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -120,15 +123,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(s_empty(i), 8);    // the eight softmax warps
+      mbar_init(s_empty(i), 16);   // the sixteen softmax warps
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(p_full(b), 8);
+      mbar_init(p_full(b), 16);
       mbar_init(pv_done(b), 2);    // both halves of P_j V_j
     }
     for (int q = 0; q < 4; ++q) {
-      mbar_init(stat_full(q), 64);  // every thread of the quarter's two warps
-      mbar_init(stat_read(q), 64);
+      mbar_init(stat_full(q), 128);  // every thread of the quarter's four warps
+      mbar_init(stat_read(q), 128);
     }
     mbar_init(drain_bar, 1);
     mbar_init(drain_pv(0), 1);
@@ -284,31 +287,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   } else {
     // -------------------------------------------------- softmax and epilogue
     const int q4 = warp & 3;                 // TMEM lane quarter of this warp
-    const int half = (warp - 4) >> 2;        // which 64 of the block's 128 keys
+    const int qc = (warp - 4) >> 2;          // which 32 of the block's 128 keys
     const int row = q4 * 32 + lane;          // query row within the block
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    // the quarter-row lse exchange of lane quarter q4 (inside P buffer 0)
+    float *xlse = reinterpret_cast<float *>(smem + q4 * 4096);
     uint32_t s_it = 0, pb = 0, item_n = 0;   // pb: the CTA's pass-2 block counter
     // wait until the P V products of pass-2 block k are done; only ever
     // called for the latest block that used P buffer k % 2
     auto wait_pv = [&](uint32_t k) { return mbar_wait(pv_done((int)(k & 1u)), (k >> 1) & 1u, abort_flag); };
-    // S_j, columns [half * 64, +64) of S buffer s_it % 2, masked past the
+    // S_j, columns [qc * 32, +32) of S buffer s_it % 2, masked past the
     // diagonal and the sequence end; releases the S buffer
-    auto read_s = [&](int j, int qrow, uint32_t (&r)[4][16]) -> bool {
+    auto read_s = [&](int j, int qrow, uint32_t (&r)[2][16]) -> bool {
       const int sb = (int)(s_it & 1u);
       if (!mbar_wait(s_full(sb), (s_it >> 1) & 1u, abort_flag)) return false;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld16(tmem_base + lane_off + (uint32_t)(sb * 128 + half * 64 + c * 16), r[c]);
+      for (int c = 0; c < 2; ++c)
+        tmem_ld16(tmem_base + lane_off + (uint32_t)(sb * 128 + qc * 32 + c * 16), r[c]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_empty(sb));
       ++s_it;
-      const int key0 = j * kAttnTile + half * 64;
-      if (j * kAttnTile + kAttnTile - 1 >= qrow - row || key0 + 64 > p.s) {
+      const int key0 = j * kAttnTile + qc * 32;
+      if (j * kAttnTile + kAttnTile - 1 >= qrow - row || key0 + 32 > p.s) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int key = key0 + c * 16 + e;
@@ -323,62 +328,66 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       const int n = qt + 1;
       const int qrow = qt * kAttnTile + row;
       bool ok = true;
-      // ---- pass 1: running max m and sum l of 2^(S c) over this half row
+      // ---- pass 1: running max m and sum l of 2^(S c) over this quarter row
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
-        uint32_t r[4][16];
+        uint32_t r[2][16];
         if (!read_s(j, qrow, r)) { ok = false; break; }
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            mx0 = fmaxf(mx0, __uint_as_float(r[c][e]));
-            mx1 = fmaxf(mx1, __uint_as_float(r[c][e + 1]));
-          }
-        const float m_new = fmaxf(m, fmaxf(mx0, mx1) * p.scale_log2);
+          for (int e = 0; e < 16; e += 4)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(r[c][e + k]));
+        const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2);
         if (m_new == -INFINITY) continue;      // every key so far masked
         const float nm = -m_new;
-        float s0 = 0.f, s1 = 0.f;
+        float sm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            s0 += ex2_approx(fmaf(__uint_as_float(r[c][e]), p.scale_log2, nm));
-            s1 += ex2_approx(fmaf(__uint_as_float(r[c][e + 1]), p.scale_log2, nm));
-          }
-        l = l * (m_new == m ? 1.0f : ex2_approx(m - m_new)) + (s0 + s1);   // 0 while m = -inf
+          for (int e = 0; e < 16; e += 4)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              sm[k] += ex2_approx(fmaf(__uint_as_float(r[c][e + k]), p.scale_log2, nm));
+        l = l * (m_new == m ? 1.0f : ex2_approx(m - m_new)) + ((sm[0] + sm[1]) + (sm[2] + sm[3]));
         m = m_new;
       }
       if (!ok) break;
-      // ---- the row's lse from its two halves (shared memory, once per item)
-      const float lse_h = l > 0.f ? m + log2f(l) : -INFINITY;
-      if (item_n > 0 && !mbar_wait(stat_read(q4), (item_n - 1) & 1u, abort_flag)) break;
-      half_lse[half * 128 + row] = lse_h;
+      // ---- the row's lse from its four quarters (shared memory, once per
+      // item; P buffer 0 is idle here: the previous item's P V products all
+      // completed before its O was stored)
+      const float lse_q = l > 0.f ? m + log2f(l) : -INFINITY;
+      xlse[qc * 32 + lane] = lse_q;
       mbar_arrive(stat_full(q4));
       if (!mbar_wait(stat_full(q4), item_n & 1u, abort_flag)) break;
-      const float lse_o = half_lse[(half ^ 1) * 128 + row];
+      const float l0 = xlse[lane], l1 = xlse[32 + lane], l2 = xlse[64 + lane], l3 = xlse[96 + lane];
       mbar_arrive(stat_read(q4));
-      const float lse = half == 0 ? lse_merge(lse_h, lse_o) : lse_merge(lse_o, lse_h);
+      // every warp of the quarter forms the same value, in the same order
+      const float lse = lse_merge(lse_merge(l0, l1), lse_merge(l2, l3));
       const float nl = lse == -INFINITY ? 0.f : -lse;
+      // the exchange slots are read by all four warps before P overwrites them
+      if (!mbar_wait(stat_read(q4), item_n & 1u, abort_flag)) break;
       // ---- pass 2: P = 2^(S c - lse) in 16 bits, the A operand of P V
       for (int j = 0; j < n; ++j, ++pb) {
-        uint32_t r[4][16];
+        uint32_t r[2][16];
         if (!read_s(j, qrow, r)) { ok = false; break; }
         // P buffer pb % 2 is free once block pb-2's P V products are done (an
         // earlier item's blocks are all done: its end waited for its last)
         if (j >= 2 && !wait_pv(pb - 2)) { ok = false; break; }
-        // this half's 64 columns form atom `half` of the 128B-swizzled
-        // K-major A tile: 16-byte chunk c8 of row `row` goes to slot
-        // c8 ^ (row % 8)
-        const uint32_t pbuf = p_s + (pb & 1u) * 32768u + (uint32_t)half * 16384u + (uint32_t)row * 128u;
+        // this quarter's 32 columns: 16-byte chunks 4 (qc % 2) .. + 3 of atom
+        // qc / 2 of the 128B-swizzled K-major A tile; chunk c8 of row `row`
+        // goes to slot c8 ^ (row % 8)
+        const uint32_t pbuf = p_s + (pb & 1u) * 32768u + (uint32_t)(qc >> 1) * 16384u + (uint32_t)row * 128u;
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
+        for (int i = 0; i < 4; ++i) {
           float f[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            f[e] = ex2_approx(fmaf(__uint_as_float(r[c8 >> 1][(c8 & 1) * 8 + e]), p.scale_log2, nl));
-          st_shared_v4(pbuf + (uint32_t)(((c8 & 7) ^ (row & 7)) * 16), pack8<T>(f));
+            f[e] = ex2_approx(fmaf(__uint_as_float(r[i >> 1][(i & 1) * 8 + e]), p.scale_log2, nl));
+          const int c8 = (qc & 1) * 4 + i;
+          st_shared_v4(pbuf + (uint32_t)((c8 ^ (row & 7)) * 16), pack8<T>(f));
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -387,13 +396,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       }
       if (!ok) break;
       // ---- epilogue: wait for the last P V, store this warp's share of O
-      // (chunks [0, ch) for half 0, [ch, d/16) for half 1) and the lse
+      // (16-column chunks [qc nc / 4, (qc + 1) nc / 4)) and the lse
       if (!wait_pv(pb - 1)) break;
       tc_fence_after();
       const int head = g % p.as, zb = g / p.as;
       T *orow = static_cast<T *>(p.o) + ((long long)zb * p.s + qrow) * p.hs + head * d;
-      const int nc = d / 16, ch = (nc + 1) / 2;
-      for (int c = half ? ch : 0; c < (half ? nc : ch); ++c) {
+      const int nc = d / 16;
+      for (int c = (qc * nc) / 4; c < ((qc + 1) * nc) / 4; ++c) {
         uint32_t o[16], o2[16];
         tmem_ld16(tmem_o + lane_off + (uint32_t)(c * 16), o);
         tmem_ld16(tmem_o2 + lane_off + (uint32_t)(c * 16), o2);
@@ -409,7 +418,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           }
         }
       }
-      if (half == 0 && qrow < p.s) p.lse[(long long)g * p.s + qrow] = lse;
+      if (qc == 0 && qrow < p.s) p.lse[(long long)g * p.s + qrow] = lse;
       tc_fence_before();
     }
   }
