@@ -101,9 +101,10 @@ def kernel_bytes(cfg, n_params: int, layers: int = 1, weight_copies: bool = Fals
         "B0 weights^T": 4 * (4 * h * h + 2 * h * f),          # the four weight matrices
         "B2 dOut^T": 4 * T * h, "B5 L2^T": 4 * T * h,         # transposes: read + write
         "B7 dH^T": 4 * T * h, "B11 L1^T": 4 * T * h,
-        # bias gradients: the GEMM / attention kernels that write dZ and dC
-        # sum every 32 rows; this pass reads those partials and writes the sum
-        "B3 db1": 4 * f * ((T + 31) // 32 + 1),
+        # bias gradients: db_1 a column-sum pass over dZ; db_qkv summed every
+        # 32 rows by the attention kernels that write dC, then this pass reads
+        # those partials and writes the sum
+        "B3 db1": 2 * T * f,
         "B11 dbqkv": 4 * 3 * h * (b * ((s + 31) // 32) + 1),
     }
     out = {k: v * layers for k, v in per_layer.items()}

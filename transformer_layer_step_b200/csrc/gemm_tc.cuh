@@ -223,7 +223,7 @@ __device__ __forceinline__ uint32_t box_piece(uint32_t box, int r, int j) {
 // 2*slot+1), fp32 outputs a whole box.  With p.colsum, the warp also sums the
 // chunk's 16 columns as stored (rounded; rows past M count 0) over its 32
 // rows and writes the sums to cs_out[0..15] (when cs_out is not null).
-template <typename T>
+template <typename T, bool CS>
 __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow &e,
                                                const uint32_t (&r)[16], const EpiIn &in,
                                                uint32_t box, uint32_t box2, int lane, int slot,
@@ -306,13 +306,13 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams &p, const EpiRow
     for (int i = 0; i < 8; ++i) f[i] = v[8 * h + i];
     const uint4 pk = pack8<T>(f);
     st_shared_v4(box_piece(box, lane, 2 * slot + h), pk);
-    if (p.colsum) {                     // the stored values, for the column sums
+    if constexpr (CS) {                 // the stored values, for the column sums
       unpack8<T>(pk, f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[8 * h + i] = e.row_ok ? f[i] : 0.f;
     }
   }
-  if (p.colsum) {
+  if constexpr (CS) {
     const float sum = warp_colsum16(v, lane);
     if (cs_out && (lane & 1) == 0) cs_out[(lane >> 1) & 15] = sum;
   }
@@ -344,7 +344,10 @@ __device__ __forceinline__ void pipe_kb_range(const GemmParams &p, const TileInf
   }
 }
 
-template <typename T>
+// CS: the instantiation with the epilogue's column sums (p.colsum set); the
+// others carry no code for them (measured: that code alone slowed every
+// short-K product at the GPT-2 117M shape by 3-10 %).
+template <typename T, bool CS>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -547,9 +550,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         }
         // this warp's 32 rows form partial row row0 / 32 of the column sums
         float *cs_out = nullptr;
-        if (p.colsum && (row0 >> 5) < p.colsum_rows)
+        if (CS && (row0 >> 5) < p.colsum_rows)
           cs_out = p.colsum + ((long long)(row0 >> 5) * p.groups + ti.g) * p.N + ti.n0 + c * 16;
-        epilogue_chunk<T>(p, er, r, in, buf, my_boxes + kStageBoxBytes, lane, slot, bad, cs_out);
+        epilogue_chunk<T, CS>(p, er, r, in, buf, my_boxes + kStageBoxBytes, lane, slot, bad, cs_out);
         if (last) {
           fence_proxy_async_smem();
           __syncwarp();

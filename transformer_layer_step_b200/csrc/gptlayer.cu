@@ -328,15 +328,17 @@ GemmTiling choose_tiling(const gptl_gemm_desc &d, int sms, bool can_split) {
 
 template <typename T>
 int launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) {
-  static bool attr_set[kMaxDevices] = {};
+  // opt-ins per device, for the instantiations without and with column sums
+  static bool attr_set[kMaxDevices][2] = {};
   int dev = 0;
   GPTL_CK(cudaGetDevice(&dev));
-  if (!attr_set[dev]) {
-    GPTL_CK(cudaFuncSetAttribute(gemm_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemLimit));
-    attr_set[dev] = true;
+  const int cs = p.colsum ? 1 : 0;
+  auto kern = cs ? gemm_tc_kernel<T, true> : gemm_tc_kernel<T, false>;
+  if (!attr_set[dev][cs]) {
+    GPTL_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
+    attr_set[dev][cs] = true;
   }
-  gemm_tc_kernel<T><<<grid, kGemmThreads, smem, stream>>>(p);
+  kern<<<grid, kGemmThreads, smem, stream>>>(p);
   GPTL_CK(cudaGetLastError());
   prof_launched(stream, GPTL_KIND_GEMM);
   return GPTL_OK;
@@ -1025,12 +1027,13 @@ Ws ws_layout(const Dims &D) {
   // transposed 16-bit weights ([in][out] per shard) for the input-gradient GEMMs
   w.w2t = take(h * f * e); w.w1t = take(f * h * e); w.wot = take(h * h * e);
   w.wqkvt = take(3 * h * h * e);
-  // partial sums: the LayerNorm backward's, and the 32-row column sums of dZ
-  // and dC (b * ceil(s/32) rows of the wider of f and 3h)
+  // partial sums: the LayerNorm backward's, the column-sum pass's (db_1) and
+  // the 32-row column sums of dC (b * ceil(s/32) rows of 3h)
   size_t part = 4 * 512 * h;
   const size_t widest = f > 3 * h ? f : 3 * h;
+  if (kColsumMaxSplit * widest > part) part = kColsumMaxSplit * widest;
   const size_t cs_rows = (size_t)D.b * ((D.s + 31) / 32);
-  if (cs_rows * widest > part) part = cs_rows * widest;
+  if (cs_rows * 3 * h > part) part = cs_rows * 3 * h;
   w.part = take(part * 4);
   // split-K partials of the weight-gradient GEMMs: up to 8 slices of the
   // largest gradient, at most 64 MiB (large layers have tiles enough)
@@ -1239,14 +1242,15 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
   g_tag = GPTL_TAG_B2_DOUT_T;
   GPTL_TRY(run_transpose(T, h, dy, h, xt, T, st));
   g_tag = GPTL_TAG_B1_B3_DZ;
-  {  // dZ_i = (dOut W2_i) * gelu'(Z_i); the epilogue also sums dZ_i's columns
-     // over each 32 rows (db_1's partials)
+  {  // dZ_i = (dOut W2_i) * gelu'(Z_i)
+    // (db_1 is a separate column-sum pass below: summing in this GEMM's
+    // epilogue, which its tensor-memory load latency already bounds, measured
+    // slower at both the GPT-2 117M and the hidden-10240 shapes)
     gptl_gemm_desc g = gemm(T, fs, h, t, view(dy, h, T, 1, h, 0, 0),
                             view(w2t, h, fs, t, h, (long long)fs * h, 0), dz, fs,
                             (long long)T * fs);
     g.act = GPTL_ACT_DGELU;
     g.aux = z;
-    g.colsum = part;
     g.out2 = act_re;                     // recompute: A_i = gelu(Z_i) again, for dW2
     GPTL_TRY(run_gemm(g, dt, st));
   }
@@ -1261,8 +1265,8 @@ int layer_bwd(const Dims &D, const gptl_weights *W, const void *x, const void *s
     GPTL_TRY(run_gemm(g, dt, st));
   }
   // ---- FFN1 (column split)
-  g_tag = GPTL_TAG_B3_DB1;   // db_1 = the partials' sum, in a fixed order
-  GPTL_TRY(launch_reduce_parts(part, (T + 31) / 32, t * fs, 1, gr->b_1, nullptr, nullptr, nullptr, st));
+  g_tag = GPTL_TAG_B3_DB1;
+  GPTL_TRY(run_colsum(T, fs, t, fs, (long long)T * fs, dt, dz, gr->b_1, part, st));
   g_tag = GPTL_TAG_B5_L2_T;
   GPTL_TRY(run_transpose(T, h, l2, h, xt, T, st));
   g_tag = GPTL_TAG_B5_DW1;
