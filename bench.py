@@ -60,12 +60,14 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "large-h10240"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
-KERNEL_SOURCES = ("transformer_layer_step_b200/csrc/gemm_tc.cuh",
-                  "transformer_layer_step_b200/csrc/attn_tc.cuh",
-                  "transformer_layer_step_b200/csrc/attn_bwd_tc.cuh",
-                  "transformer_layer_step_b200/csrc/common.cuh",
-                  "transformer_layer_step_b200/csrc/bw_kernels.cuh",
-                  "transformer_layer_step_b200/csrc/gptlayer.cu")
+# the sources each recorded DRAM traffic depends on: the family's kernels,
+# the shared device helpers, and the host code that picks its launch shape
+# and lays out its operands
+FAMILY_SOURCES = {
+    "gemm": ("transformer_layer_step_b200/csrc/gemm_tc.cuh",
+             "transformer_layer_step_b200/csrc/common.cuh",
+             "transformer_layer_step_b200/csrc/gptlayer.cu"),
+}
 
 
 # ----------------------------------------------------------------- workload
@@ -171,9 +173,9 @@ def code_without_comments(text: str) -> str:
     return "\n".join(ln for ln in lines if ln)
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(family: str = "gemm") -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in FAMILY_SOURCES[family]:
         with open(os.path.join(ROOT, rel), encoding="utf-8") as fh:
             h.update(code_without_comments(fh.read()).encode())
     return h.hexdigest()[:16]
@@ -199,7 +201,7 @@ def recorded_traffic(workload: str, family: str):
     except (OSError, ValueError):
         return None
     ent = rec.get(workload, {}).get(family)
-    if not ent or ent.get("kernel_sources") != kernel_source_hash():
+    if not ent or family not in FAMILY_SOURCES or ent.get("kernel_sources") != kernel_source_hash(family):
         return None
     return ent.get("dram_bytes_per_step")
 

@@ -124,8 +124,18 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const TX *__restrict__ x,
 // rows ([team][part][h]; a thread only touches its own columns), so the
 // registers stay low enough for two blocks per SM; the teams are added in a
 // fixed order at the end.
+//
+//
+// Wide rows (VPT >= 4) with two column sums take two passes over the row
+// instead of holding it in registers: pass A computes the two row sums and
+// adds gy*xhat and gy into the column sums, pass B reads gy and x again (from
+// L1/L2: the row was just read) and writes dx.  The registers then drop far
+// enough for two blocks per SM, which the shared memory of two sums allows
+// (the LayerNorm-1 backward at hidden 10240: 108.7 -> 92.1 us).  With three
+// or four sums one block per SM fits either way, and the one-pass form is
+// faster there.
 template <typename T, typename TX, typename TR, bool D32, bool SUM_DX, bool SUM_RESID, int VPT>
-__global__ void __launch_bounds__(256, VPT <= 3 ? 2 : 1) ln_bwd_kernel(
+__global__ void __launch_bounds__(256, (VPT <= 3 || (!SUM_DX && !SUM_RESID)) ? 2 : 1) ln_bwd_kernel(
     const T *__restrict__ gy, const TX *__restrict__ x, const float *__restrict__ mu_in,
     const float *__restrict__ rstd_in, const T *__restrict__ gamma, const TR *__restrict__ resid,
     T *__restrict__ dx, float *__restrict__ dx32, float *__restrict__ part, int rows, int h,
@@ -137,10 +147,12 @@ __global__ void __launch_bounds__(256, VPT <= 3 ? 2 : 1) ln_bwd_kernel(
   const int RPB = blockDim.x / tpr;
   const int team = threadIdx.x / TPR, tl = threadIdx.x % TPR;
   float *acc = sm + (size_t)team * nparts * h;
-  float gm[VPT][8];
+  constexpr bool kTwoPass = VPT >= 4 && nparts == 2;
+  float gm[VPT][8];                          // gamma in registers (one-pass form only)
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
-    unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(gamma) + tl + i * TPR), gm[i]);
+    if constexpr (!kTwoPass)
+      unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(gamma) + tl + i * TPR), gm[i]);
 #pragma unroll
     for (int k = 0; k < nparts; ++k) {
       float4 *a4 = reinterpret_cast<float4 *>(acc + k * h + (tl + i * TPR) * 8);
@@ -168,6 +180,65 @@ __global__ void __launch_bounds__(256, VPT <= 3 ? 2 : 1) ln_bwd_kernel(
     const uint4 *gr = reinterpret_cast<const uint4 *>(gy + (long long)r * h);
     const TX *xr = x + (long long)r * h;
     const float mu = mu_in[r], rstd = rstd_in[r];
+    if constexpr (kTwoPass) {
+      const uint4 *g4 = reinterpret_cast<const uint4 *>(gamma);
+      float s1 = 0.f, s2 = 0.f;
+      // pass A: the row sums, and gy*xhat, gy into the column sums
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        float gv[8], xv[8], gmv[8], xh[8], gx[8];
+        unpack8<T>(gr[tl + i * TPR], gv);
+        load_vec8<TX, T>(xr, tl + i * TPR, xv);
+        unpack8<T>(__ldg(g4 + tl + i * TPR), gmv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          xh[e] = (xv[e] - mu) * rstd;
+          const float ghe = gv[e] * gmv[e];
+          s1 += ghe;
+          s2 += ghe * xh[e];
+          gx[e] = gv[e] * xh[e];
+        }
+        if (active) {
+          add8(0, i, gx);
+          add8(1, i, gv);
+        }
+      }
+      const float m1 = team_sum(s1, red, TPR) / (float)h;
+      const float m2 = team_sum(s2, red, TPR) / (float)h;
+      if (active) {
+        // pass B: dx from gy and x read again
+        const TR *rr = resid + (long long)r * h;
+        uint4 *dr = reinterpret_cast<uint4 *>(dx + (long long)r * h);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+          float gv[8], xv[8], gmv[8], rv[8], o[8];
+          unpack8<T>(gr[tl + i * TPR], gv);
+          load_vec8<TX, T>(xr, tl + i * TPR, xv);
+          unpack8<T>(__ldg(g4 + tl + i * TPR), gmv);
+          load_vec8<TR, T>(rr, tl + i * TPR, rv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float xh = (xv[e] - mu) * rstd;
+            o[e] = rv[e] + rstd * (gv[e] * gmv[e] - m1 - xh * m2);
+          }
+          const uint4 q = pack8<T>(o);
+          dr[tl + i * TPR] = q;
+          if constexpr (D32) store_vec8_f32(dx32 + (long long)r * h, tl + i * TPR, o);
+          if constexpr (SUM_DX) {
+            float oq[8];
+            if constexpr (D32) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) oq[e] = o[e];
+            } else {
+              unpack8<T>(q, oq);           // sum what was stored
+            }
+            add8(2, i, oq);
+          }
+          if constexpr (SUM_RESID) add8(SUM_DX ? 3 : 2, i, rv);
+        }
+      }
+      continue;
+    }
     float xh[VPT][8], gh[VPT][8], g[VPT][8];
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
