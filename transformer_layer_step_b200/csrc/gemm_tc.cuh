@@ -40,6 +40,15 @@ constexpr int kBM = 128;          // tile rows (UMMA M)
 constexpr int kBK = 64;           // tile depth per pipeline stage
 constexpr int kGemmThreads = 384;
 constexpr int kEpiWarps = 8;
+// registers per thread: the launch allocation (one CTA per SM at 384 threads
+// gets 168 each) and the split by role after setup.  The TMA / MMA warpgroup
+// gives registers up and the two epilogue warpgroups take them; the split
+// must add up to the launch allocation exactly, or the increase never
+// completes, so the host checks the compiled count before the first launch.
+constexpr int kGemmRegs = 168;
+constexpr int kRoleRegs = 56;
+constexpr int kEpiRegs = 224;
+static_assert(128 * kRoleRegs + 256 * kEpiRegs == kGemmThreads * kGemmRegs, "register split");
 
 enum : int { kActNone = 0, kActGelu = 1, kActDGelu = 2 };
 
@@ -399,6 +408,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // registers by role: the TMA / MMA warps (warpgroup 0) need few, the
+  // epilogue warps (warpgroups 1, 2) hold four accumulator chunks in flight
+  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRoleRegs) : "memory");
+  else asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kEpiRegs) : "memory");
 
   if (warp < 4) {
     const int pp = warp >> 1;                 // pipeline of this warp
@@ -487,7 +500,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     const bool wide = p.out_f32 || p.split > 1;     // fp32: one chunk per box
     const bool two = !wide && p.write_o2;     // a second output: both boxes per chunk pair
     // no bias, residual, activation or second K half: nothing to load per chunk
-    const bool grouped = !p.bias && !p.resid && p.act == kActNone && !p.pipe_k;
+    const bool grouped = !CS && !p.bias && !p.resid && p.act == kActNone && !p.pipe_k;
     const uint32_t my_boxes = staging_s + (uint32_t)((warp - 4) * 2 * kStageBoxBytes);
     int box_i = 0;                           // boxes issued by this warp (selects the buffer)
     bool bad = false;                        // an fp32 output value was inf or NaN
@@ -567,17 +580,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         }
       };
       if (grouped) {
-        // chunks in pairs, both tensor-memory loads in flight before one
-        // wait: the load latency, which bounds this epilogue, is paid once
-        // per 32 columns (measured on the 10240 x 10240 x 2048 weight-
-        // gradient product: 372 -> 353 us)
-        for (int c = c0; c < c1; c += 2) {
-          const bool has_b = c + 1 < c1;
-          ld(c, ra);
-          if (has_b) ld(c + 1, rb);
+        // the grouped path's chunk: the accumulator values go to the box as
+        // they are (fp32) or rounded to 16 bits, with no epilogue arithmetic
+        auto process_plain = [&](int c, const uint32_t (&r)[16]) {
+          const int slot = wide ? 0 : ((c - c0) & 1);
+          const bool first = slot == 0, last = wide || slot == 1 || c + 1 == c1;
+          const uint32_t buf = my_boxes + (uint32_t)((box_i & 1) * kStageBoxBytes);
+          if (first) {
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
+          if (wide) {
+            if (p.nonfinite && p.split == 1 && er.row_ok) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) bad |= not_finite(__uint_as_float(r[i]));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              st_shared_v4(box_piece(buf, lane, j), make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]));
+          } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float f[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * h + i]);
+              st_shared_v4(box_piece(buf, lane, 2 * slot + h), pack8<T>(f));
+            }
+          }
+          if (last) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              const int x = ti.n0 + (c - slot) * 16;
+              if (p.out_evict_first) tma_store_4d_hint(&p.map_o, buf, x, row0, oz, ow, l2_policy_evict_first());
+              else tma_store_4d(&p.map_o, buf, x, row0, oz, ow);
+              bulk_commit();
+            }
+            ++box_i;
+          }
+        };
+        // four chunks' tensor-memory loads in flight before one wait: the
+        // load latency, which bounds this epilogue, is paid once per 64 columns
+        for (int c = c0; c < c1; c += 4) {
+          uint32_t rg[4][16];
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            if (c + g < c1) ld(c + g, rg[g]);
           tmem_wait_ld();
-          process(c, ra, ia);
-          if (has_b) process(c + 1, rb, ia);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            if (c + g < c1) process_plain(c + g, rg[g]);
         }
         continue;
       }

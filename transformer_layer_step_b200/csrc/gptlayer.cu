@@ -335,6 +335,11 @@ int launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) 
   const int cs = p.colsum ? 1 : 0;
   auto kern = cs ? gemm_tc_kernel<T, true> : gemm_tc_kernel<T, false>;
   if (!attr_set[dev][cs]) {
+    // the kernel splits its registers by role (setmaxnreg), a split that
+    // adds up only when every thread was launched with kGemmRegs
+    cudaFuncAttributes fa{};
+    GPTL_CK(cudaFuncGetAttributes(&fa, kern));
+    if (fa.numRegs != kGemmRegs || fa.maxThreadsPerBlock < kGemmThreads) return GPTL_E_CUDA;
     GPTL_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
     attr_set[dev][cs] = true;
   }
