@@ -25,11 +25,6 @@
  *     the host with the device, except gptl_read_device_error().
  *   - Return value: 0 on success, a negative GPTL_E_* code otherwise.  Input
  *     validation happens before any launch: on error nothing is enqueued.
- *   - Host threads may call entry points concurrently (one thread per
- *     device, say): the library's host-side caches are per device and
- *     atomic or locked.  Calls that share buffers or a workspace are ordered
- *     by the caller, as for any CUDA work.  The profiling window
- *     (gptlayer_profile.h) belongs to one thread.
  *   - Kernels never trap.  A device-side failure (a bounded wait that timed
  *     out, an internal consistency check) sets a library-wide device error
  *     word, read with gptl_read_device_error().

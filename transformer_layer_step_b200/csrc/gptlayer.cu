@@ -11,7 +11,6 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include <atomic>
 #include <mutex>
 
 #include "bw_kernels.cuh"
@@ -49,14 +48,13 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // profiling window is open (gptl_profile_begin .. gptl_profile_end) an event
 // is also recorded on the launch stream at the start of each entry point and
 // after each launch, so that consecutive events bracket one kernel.  The
-// tag names the step of the layer the launch belongs to.  The launch count
-// and the window's open flag are atomic because entry points may run on
-// several host threads; the window itself belongs to one thread.
+// tag names the step of the layer the launch belongs to.
 struct ProfRec {
   int kind, tag;
   cudaEvent_t a, b;
 };
 struct Profiler {
+  bool on = false;
   cudaEvent_t *pool = nullptr;
   int pool_n = 0, pool_next = 0;
   ProfRec *recs = nullptr;
@@ -65,9 +63,8 @@ struct Profiler {
   cudaEvent_t prev = nullptr;
 };
 Profiler g_prof;
-std::atomic<bool> g_prof_on{false};
-thread_local int g_tag = GPTL_TAG_NONE;
-std::atomic<unsigned long long> g_launches{0};
+int g_tag = GPTL_TAG_NONE;
+unsigned long long g_launches = 0;
 // While a checked backward runs on this host thread (gpt_layer_bwd_checked),
 // the device word that the kernels writing gradients set on an inf or NaN:
 // the fp32-output GEMMs, their split-K sums and the column-sum reductions.
@@ -91,13 +88,13 @@ cudaEvent_t prof_event(cudaStream_t st) {
 
 // Marks the start of an entry point's launches on `st`.
 void prof_start(cudaStream_t st) {
-  if (g_prof_on.load(std::memory_order_relaxed)) g_prof.prev = prof_event(st);
+  if (g_prof.on) g_prof.prev = prof_event(st);
 }
 
 // Called after every successful launch on `st`.
 void prof_launched(cudaStream_t st, int kind) {
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  ++g_launches;
+  if (!g_prof.on) return;
   cudaEvent_t e = (g_prof.prev && g_prof.n < g_prof.cap) ? prof_event(st) : nullptr;
   if (!e) {
     ++g_prof.dropped;
@@ -114,24 +111,26 @@ struct TagScope {
   ~TagScope() { g_tag = saved; }
 };
 
-// per device: 0 = not looked up yet, -1 = not compute capability 10.x,
-// otherwise its SM count (atomic: entry points may run on several threads)
-std::atomic<int> g_dev_sms[kMaxDevices];
+struct DeviceInfo {
+  int checked = 0, ok = 0, sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
 
 int device_check(int *sms_out = nullptr) {
   int dev = 0;
   GPTL_CK(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return GPTL_E_ARCH;
-  int v = g_dev_sms[dev].load(std::memory_order_relaxed);
-  if (v == 0) {
+  DeviceInfo &d = g_dev[dev];
+  if (!d.checked) {
     int major = 0, sms = 0;
     GPTL_CK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
     GPTL_CK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-    v = (major == 10 && sms > 0) ? sms : -1;
-    g_dev_sms[dev].store(v, std::memory_order_relaxed);
+    d.ok = (major == 10);
+    d.sms = sms;
+    d.checked = 1;
   }
-  if (v < 0) return GPTL_E_ARCH;
-  if (sms_out) *sms_out = v;
+  if (!d.ok) return GPTL_E_ARCH;
+  if (sms_out) *sms_out = d.sms;
   return GPTL_OK;
 }
 
@@ -142,20 +141,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static std::atomic<EncodeTiledFn> fn{nullptr};   // the same value from every thread
-  EncodeTiledFn f = fn.load(std::memory_order_relaxed);
-  if (!f) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess) {
-      (void)cudaGetLastError();
+        q != cudaDriverEntryPointSuccess)
       return nullptr;
-    }
-    f = reinterpret_cast<EncodeTiledFn>(p);
-    fn.store(f, std::memory_order_relaxed);
+    fn = reinterpret_cast<EncodeTiledFn>(p);
   }
-  return f;
+  return fn;
 }
 
 int mn_chunk_width(long long rows_tile) {
@@ -334,20 +329,19 @@ GemmTiling choose_tiling(const gptl_gemm_desc &d, int sms, bool can_split) {
 template <typename T>
 int launch_gemm_t(const GemmParams &p, int grid, int smem, cudaStream_t stream) {
   // opt-ins per device, for the instantiations without and with column sums
-  static std::atomic<bool> attr_set[kMaxDevices][2];
+  static bool attr_set[kMaxDevices][2] = {};
   int dev = 0;
   GPTL_CK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return GPTL_E_ARCH;
   const int cs = p.colsum ? 1 : 0;
   auto kern = cs ? gemm_tc_kernel<T, true> : gemm_tc_kernel<T, false>;
-  if (!attr_set[dev][cs].load(std::memory_order_relaxed)) {
+  if (!attr_set[dev][cs]) {
     // the kernel splits its registers by role (setmaxnreg), a split that
     // adds up only when every thread was launched with kGemmRegs
     cudaFuncAttributes fa{};
     GPTL_CK(cudaFuncGetAttributes(&fa, kern));
     if (fa.numRegs != kGemmRegs || fa.maxThreadsPerBlock < kGemmThreads) return GPTL_E_CUDA;
     GPTL_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-    attr_set[dev][cs].store(true, std::memory_order_relaxed);
+    attr_set[dev][cs] = true;
   }
   kern<<<grid, kGemmThreads, smem, stream>>>(p);
   GPTL_CK(cudaGetLastError());
@@ -554,14 +548,13 @@ int run_attn_fwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
   const int grid = (int)(p.items < sms ? p.items : sms);
   // the shared-memory opt-in is recorded per device and per dtype (both
   // instantiations have the same function-pointer type)
-  static std::atomic<bool> attr_set[kMaxDevices][2];
+  static bool attr_set[kMaxDevices][2] = {};
   int dev = 0;
   GPTL_CK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return GPTL_E_ARCH;
   auto launch = [&](auto kern) -> int {
-    if (!attr_set[dev][dt].load(std::memory_order_relaxed)) {
+    if (!attr_set[dev][dt]) {
       GPTL_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-      attr_set[dev][dt].store(true, std::memory_order_relaxed);
+      attr_set[dev][dt] = true;
     }
     kern<<<grid, kAttnThreads, smem, st>>>(p);
     GPTL_CK(cudaGetLastError());
@@ -643,15 +636,14 @@ int run_attn_bwd(int b, int s, int hs, int as, int t, int d, gptl_dtype dt, cons
   if (smem_kv < 120 * 1024) smem_kv = 120 * 1024;
   if (smem_dq > kSmemLimit || smem_kv > kSmemLimit) return GPTL_E_SHAPE;
   const int grid = (int)(p.items < sms ? p.items : sms);
-  static std::atomic<bool> attr_set[kMaxDevices][2];
+  static bool attr_set[kMaxDevices][2] = {};
   int dev = 0;
   GPTL_CK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return GPTL_E_ARCH;
   auto launch = [&](auto kq, auto kkv) -> int {
-    if (!attr_set[dev][dt].load(std::memory_order_relaxed)) {
+    if (!attr_set[dev][dt]) {
       GPTL_CK(cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
       GPTL_CK(cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
-      attr_set[dev][dt].store(true, std::memory_order_relaxed);
+      attr_set[dev][dt] = true;
     }
     kq<<<grid, kAttnBwdThreads, smem_dq, st>>>(p);
     GPTL_CK(cudaGetLastError());
@@ -1820,11 +1812,11 @@ int gptl_colsum_noalloc(int rows, int n, int groups, long long ld, long long gst
 }
 
 // ------------------------------------------------------------- profiling
-unsigned long long gptl_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+unsigned long long gptl_launch_count(void) { return g_launches; }
 
 int gptl_profile_begin(int capacity) {
   if (capacity <= 0) return GPTL_E_ARG;
-  if (g_prof_on.load()) return GPTL_E_ARG;
+  if (g_prof.on) return GPTL_E_ARG;
   g_prof = Profiler();
   const int pool_n = 2 * capacity + 64;
   g_prof.pool = static_cast<cudaEvent_t *>(calloc((size_t)pool_n, sizeof(cudaEvent_t)));
@@ -1847,13 +1839,12 @@ int gptl_profile_begin(int capacity) {
   }
   g_prof.pool_n = pool_n;
   g_prof.cap = capacity;
-  g_prof_on.store(true);
+  g_prof.on = true;
   return GPTL_OK;
 }
 
 int gptl_profile_end(gptl_launch_record *out, int capacity, int *n_out, long long *dropped) {
-  if (!g_prof_on.load()) return GPTL_E_ARG;
-  g_prof_on.store(false);
+  if (!g_prof.on) return GPTL_E_ARG;
   int rc = GPTL_OK;
   if (cudaDeviceSynchronize() != cudaSuccess) {
     (void)cudaGetLastError();
