@@ -89,3 +89,34 @@ def test_optimizer_bytes_per_parameter_and_copies(name):
     # with the copies the backward has no weight transposes to do; without,
     # it reads and writes every matrix entry once
     assert nb["B0 weights^T"] == 4 * mats
+
+
+def test_roofline_arithmetic_on_recorded_launches():
+    """The per-kernel summary and the roofline figures from a made-up launch
+    record of two steps at the hidden-10240 shapes: achieved = algorithmic
+    work / summed launch time, frac = achieved / peak (the sustained GEMM
+    rate for the tensor-core families), shares over the step's total."""
+    c = synth.CONFIGS["large-h10240"]
+    sh = G.make_shape(c.batch, c.seq, c.hidden, c.heads, c.ffn, c.tp, c.dtype)
+    _, n = G.param_layout(sh)
+    peaks = {"hbm_gbs": 5000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1000.0}
+    flops = bench.step_flops(c)
+    K = 2
+    one_step = [("gemm", "F2 qkv", 1.0), ("gemm", "F10 ffn2", 3.0),
+                ("attn_fwd", "F3-F5 attn", 2.0), ("adam", "O2 adam", 4.0)]
+    rows, kinds, ms_step = bench.summarize_kernels(one_step * K, K, c, n, peaks, flops)
+    assert ms_step == pytest.approx(10.0)
+    assert kinds["gemm"]["ms_per_step"] == pytest.approx(4.0)
+    assert kinds["gemm"]["launches_per_step"] == 2
+    assert kinds["adam"]["share"] == pytest.approx(0.4)
+    adam = next(r for r in rows if r["step"] == "O2 adam")
+    want_gbs = 30 * n / 4.0e-3 / 1e9
+    assert adam["GB/s"] == pytest.approx(want_gbs, rel=1e-3)
+    assert adam["frac_hbm"] == pytest.approx(want_gbs / 5000.0, abs=1e-3)
+    roof = bench.kernel_rooflines(kinds, rows, c, n, flops, peaks, "test")
+    want_tf = flops["linear"] / 4.0e-3 / 1e12
+    assert roof["gemm"]["achieved"] == pytest.approx(want_tf, rel=1e-3)
+    assert roof["gemm"]["frac"] == pytest.approx(want_tf / 1000.0, rel=1e-3)
+    assert roof["attn_fwd"]["achieved"] == pytest.approx(flops["attn_fwd"] / 2.0e-3 / 1e12, rel=1e-3)
+    assert roof["adam"]["bytes"] == 30 * n
+    assert roof["adam"]["achieved"] == pytest.approx(want_gbs, rel=1e-3)
